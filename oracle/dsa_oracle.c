@@ -1,0 +1,353 @@
+/*
+ * DSA CPU oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, literal double-precision restatement of the three steps of
+ * DeepSeek Sparse Attention (DSA): lightning-indexer scores, per-query top-k
+ * selection, and MLA attention in its absorbed MQA form over the selected
+ * tokens.  It shares no code with the CUDA library; only tests/, the smoke
+ * check and the CPU-baseline leg of the benchmark may load it.
+ *
+ * Sources (page title, section):
+ *  - "DeepSeek-V3.2" (transformers model doc), section "DeepSeek Sparse
+ *    Attention (DSA)", item 1 "Lightning indexer": an index score between each
+ *    query and every preceding key, computed by a low-head-count module; item
+ *    2 "Fine-grained token selection": keep the top-index_topk tokens, main MLA
+ *    attention over those tokens only via an additive mask.
+ *  - "DeepSeek-V3.2 / Exp" (visual-learn explainer), "Different questions
+ *    select different tokens": cached entries are MLA's compressed vectors.
+ *  - "DeepSeek-V3.2 - Experimental Exp Version" (altools), "Technical
+ *    Principles": a small number of index heads; MLA with MQA so that key
+ *    entries are shared by all query heads.
+ *  - "DeepSeek-V3.2-Exp" (token-ids page), released config excerpt
+ *    (index_n_heads 64, index_head_dim 128, index_topk 2048, kv_lora_rank 512,
+ *    qk_rope_head_dim 64) and "Position IDs" (causal mask: -inf strictly above
+ *    the diagonal, so a query sees its own position).
+ *
+ * Readings where the pages are silent (all listed in the design notes):
+ *  - indexer score I[t,s] = sum_j w[t,j] * max(0, q_I[t,j,:] . k_I[s,:]),
+ *    defined for 0 <= s <= pos(t) (inclusive, matching the causal mask);
+ *  - top-k order: higher score first, then lower sequence-local index; rows
+ *    with fewer than k candidates keep all of them, padded with -1;
+ *  - absorbed MQA attention: logits z_s = scale * q[t,h,:Dqk] . c[s,:Dqk],
+ *    values are the first Dv columns of the same latent row c[s,:].
+ *
+ * Every function works on one query row at a time in double precision, with
+ * no blocking, fusion or reordering beyond the definition.  OpenMP splits the
+ * independent query rows across host cores.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* element kinds of an input array */
+enum { ORACLE_BF16 = 0, ORACLE_E4M3 = 1, ORACLE_F64 = 2 };
+
+/* bf16: the upper 16 bits of an IEEE-754 binary32 value (exact in double). */
+double oracle_bf16_to_double(uint16_t bits) {
+  uint32_t u = ((uint32_t)bits) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* OCP FP8 E4M3 ("fn" variant): 1 sign bit, 4 exponent bits with bias 7,
+ * 3 mantissa bits; exponent field 0 holds subnormals m * 2^-9; the pattern
+ * S.1111.111 is NaN (there are no infinities); everything else is
+ * (1 + m/8) * 2^(e-7). */
+double oracle_e4m3_to_double(uint8_t byte) {
+  int sign = (byte >> 7) & 1;
+  int e = (byte >> 3) & 15;
+  int m = byte & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m, -9);
+  else
+    v = ldexp(1.0 + m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+static double load_elem(int kind, const void* base, int64_t i, const float* row_scale, int64_t row) {
+  switch (kind) {
+    case ORACLE_BF16: return oracle_bf16_to_double(((const uint16_t*)base)[i]);
+    case ORACLE_E4M3: return oracle_e4m3_to_double(((const uint8_t*)base)[i]) * (double)row_scale[row];
+    default: return ((const double*)base)[i];
+  }
+}
+
+/* Which sequence holds global query row t, and its absolute position. */
+static int locate_row(int B, const int32_t* cu_q, const int32_t* cu_k, int64_t t, int* b_out,
+                      int64_t* pos_out, int64_t* kv_len_out) {
+  for (int b = 0; b < B; ++b) {
+    if (t >= cu_q[b] && t < cu_q[b + 1]) {
+      int64_t q_len = cu_q[b + 1] - cu_q[b];
+      int64_t kv_len = cu_k[b + 1] - cu_k[b];
+      *b_out = b;
+      *pos_out = kv_len - q_len + (t - cu_q[b]);
+      *kv_len_out = kv_len;
+      return 0;
+    }
+  }
+  return -1;
+}
+
+static int check_varlen(int B, const int32_t* cu_q, const int32_t* cu_k) {
+  if (B < 1 || cu_q[0] != 0 || cu_k[0] != 0) return -1;
+  for (int b = 0; b < B; ++b) {
+    int64_t q_len = cu_q[b + 1] - cu_q[b];
+    int64_t kv_len = cu_k[b + 1] - cu_k[b];
+    if (q_len < 0 || kv_len < q_len) return -1;
+  }
+  return 0;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/*
+ * Step 1, lightning indexer.  For each requested query row t (global index
+ * rows[r], or r itself when rows is NULL) and each key s of its sequence:
+ *   scores[r, s] = sum_j w[t,j] * max(0, sum_d q_idx[t,j,d] * k_idx[s,d])  for s <= pos(t)
+ *   scores[r, s] = -inf                                                     for s >  pos(t)
+ * q_idx: [T, H_I, d_I]; w: [T, H_I] (double); k_idx: [sum kv, d_I] with, for
+ * E4M3, one float32 scale per key row.
+ */
+int oracle_indexer_scores(int B, const int32_t* cu_q, const int32_t* cu_k, int H_I, int d_I,
+                          int q_kind, const void* q_idx, const double* w, int k_kind,
+                          const void* k_idx, const float* k_scale, int64_t n_rows,
+                          const int32_t* rows, double* scores, int64_t ld) {
+  if (check_varlen(B, cu_q, cu_k)) return -1;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t t = rows ? rows[r] : r;
+    int b;
+    int64_t pos, kv_len;
+    if (locate_row(B, cu_q, cu_k, t, &b, &pos, &kv_len) || kv_len > ld) {
+      bad = 1;
+      continue;
+    }
+    double* out = scores + r * ld;
+    for (int64_t s = 0; s < kv_len; ++s) {
+      if (s > pos) {
+        out[s] = -INFINITY;
+        continue;
+      }
+      int64_t key_row = cu_k[b] + s;
+      double total = 0.0;
+      for (int j = 0; j < H_I; ++j) {
+        double dot = 0.0;
+        for (int d = 0; d < d_I; ++d) {
+          double qv = load_elem(q_kind, q_idx, (t * H_I + j) * (int64_t)d_I + d, NULL, 0);
+          double kv = load_elem(k_kind, k_idx, key_row * d_I + d, k_scale, key_row);
+          dot += qv * kv;
+        }
+        double relu = dot > 0.0 ? dot : 0.0;
+        total += w[t * H_I + j] * relu;
+      }
+      out[s] = total;
+    }
+  }
+  return bad ? -1 : 0;
+}
+
+typedef struct {
+  double score;
+  int32_t index;
+} candidate;
+
+/* Total order of the selection: higher score first, then lower index. */
+static int candidate_cmp(const void* a, const void* b) {
+  const candidate* x = (const candidate*)a;
+  const candidate* y = (const candidate*)b;
+  if (x->score > y->score) return -1;
+  if (x->score < y->score) return 1;
+  return (x->index > y->index) - (x->index < y->index);
+}
+
+/*
+ * Step 2, fine-grained token selection.  For each requested row: sort the
+ * candidates s = 0..pos(t) by (score desc, index asc) and keep the first
+ * min(topk, pos(t)+1); idx[r, :] holds them in that order, then -1 padding.
+ * scores rows follow the layout written by oracle_indexer_scores.
+ */
+int oracle_topk(int B, const int32_t* cu_q, const int32_t* cu_k, int64_t n_rows, const int32_t* rows,
+                const double* scores, int64_t ld, int topk, int32_t* idx) {
+  if (check_varlen(B, cu_q, cu_k) || topk < 1) return -1;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t t = rows ? rows[r] : r;
+    int b;
+    int64_t pos, kv_len;
+    if (locate_row(B, cu_q, cu_k, t, &b, &pos, &kv_len) || kv_len > ld) {
+      bad = 1;
+      continue;
+    }
+    int64_t n = pos + 1;
+    candidate* c = (candidate*)malloc(sizeof(candidate) * (size_t)n);
+    if (!c) {
+      bad = 1;
+      continue;
+    }
+    for (int64_t s = 0; s < n; ++s) {
+      c[s].score = scores[r * ld + s];
+      c[s].index = (int32_t)s;
+    }
+    qsort(c, (size_t)n, sizeof(candidate), candidate_cmp);
+    int64_t keep = n < topk ? n : topk;
+    for (int64_t i = 0; i < topk; ++i) idx[r * topk + i] = i < keep ? c[i].index : -1;
+    free(c);
+  }
+  return bad ? -1 : 0;
+}
+
+/* An entry of idx takes part in attention for query position pos iff it is a
+ * key of the sequence at or before pos; -1 (padding) and anything else is
+ * ignored. */
+static int selected_entry_valid(int32_t s, int64_t pos, int64_t kv_len) {
+  return s >= 0 && s <= pos && s < kv_len;
+}
+
+/*
+ * Step 3, MLA attention in absorbed MQA form over the selected tokens.
+ * For each requested row t and head h, over the valid entries s of idx[r,:]:
+ *   z_s = scale * sum_{d < Dqk} q[t,h,d] * c[s,d]
+ *   out[r,h,:] = sum_s softmax(z)_s * c[s, :Dv],   lse[r,h] = log sum_s exp(z_s)
+ * The softmax is evaluated as exp(z_s - max z) / sum exp(z - max z).  With no
+ * valid entry, out = 0 and lse = -inf.
+ * q: [T, H, Dqk]; latent: [sum kv, Dqk]; out: [n_rows, H, Dv]; lse: [n_rows, H].
+ */
+int oracle_sparse_mla(int B, const int32_t* cu_q, const int32_t* cu_k, int H, int d_qk, int d_v,
+                      int q_kind, const void* q, int c_kind, const void* latent, int64_t n_rows,
+                      const int32_t* rows, const int32_t* idx, int topk, double scale, double* out,
+                      double* lse) {
+  if (check_varlen(B, cu_q, cu_k) || d_v > d_qk || topk < 1) return -1;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t t = rows ? rows[r] : r;
+    int b;
+    int64_t pos, kv_len;
+    if (locate_row(B, cu_q, cu_k, t, &b, &pos, &kv_len)) {
+      bad = 1;
+      continue;
+    }
+    double* z = (double*)malloc(sizeof(double) * (size_t)topk);
+    if (!z) {
+      bad = 1;
+      continue;
+    }
+    const int32_t* sel = idx + r * topk;
+    for (int h = 0; h < H; ++h) {
+      double zmax = -INFINITY;
+      for (int i = 0; i < topk; ++i) {
+        z[i] = -INFINITY;
+        if (!selected_entry_valid(sel[i], pos, kv_len)) continue;
+        int64_t row = cu_k[b] + sel[i];
+        double dot = 0.0;
+        for (int d = 0; d < d_qk; ++d)
+          dot += load_elem(q_kind, q, (t * H + h) * (int64_t)d_qk + d, NULL, 0) *
+                 load_elem(c_kind, latent, row * d_qk + d, NULL, 0);
+        z[i] = scale * dot;
+        if (z[i] > zmax) zmax = z[i];
+      }
+      double* o = out + (r * H + h) * (int64_t)d_v;
+      for (int d = 0; d < d_v; ++d) o[d] = 0.0;
+      if (zmax == -INFINITY) {
+        lse[r * H + h] = -INFINITY;
+        continue;
+      }
+      double denom = 0.0;
+      for (int i = 0; i < topk; ++i)
+        if (z[i] != -INFINITY) denom += exp(z[i] - zmax);
+      for (int i = 0; i < topk; ++i) {
+        if (z[i] == -INFINITY) continue;
+        double p = exp(z[i] - zmax) / denom;
+        int64_t row = cu_k[b] + sel[i];
+        for (int d = 0; d < d_v; ++d) o[d] += p * load_elem(c_kind, latent, row * d_qk + d, NULL, 0);
+      }
+      lse[r * H + h] = zmax + log(denom);
+    }
+    free(z);
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * The additive-mask formulation named on the transformers page: dense MLA
+ * attention over every key of the sequence, with mask 0 on the selected
+ * positions and -inf elsewhere (the causal mask is -inf strictly above the
+ * diagonal).  Mathematically identical to oracle_sparse_mla; kept as a
+ * separate literal restatement so that each pins the other.
+ */
+int oracle_dense_mla_masked(int B, const int32_t* cu_q, const int32_t* cu_k, int H, int d_qk,
+                            int d_v, int q_kind, const void* q, int c_kind, const void* latent,
+                            int64_t n_rows, const int32_t* rows, const int32_t* idx, int topk,
+                            double scale, double* out, double* lse) {
+  if (check_varlen(B, cu_q, cu_k) || d_v > d_qk || topk < 1) return -1;
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t t = rows ? rows[r] : r;
+    int b;
+    int64_t pos, kv_len;
+    if (locate_row(B, cu_q, cu_k, t, &b, &pos, &kv_len)) {
+      bad = 1;
+      continue;
+    }
+    double* mask = (double*)malloc(sizeof(double) * (size_t)kv_len);
+    double* z = (double*)malloc(sizeof(double) * (size_t)kv_len);
+    if (!mask || !z) {
+      free(mask);
+      free(z);
+      bad = 1;
+      continue;
+    }
+    for (int64_t s = 0; s < kv_len; ++s) mask[s] = -INFINITY;
+    for (int i = 0; i < topk; ++i) {
+      int32_t s = idx[r * topk + i];
+      if (s >= 0 && s < kv_len) mask[s] = 0.0;
+    }
+    for (int64_t s = pos + 1; s < kv_len; ++s) mask[s] = -INFINITY; /* causal */
+    for (int h = 0; h < H; ++h) {
+      double zmax = -INFINITY;
+      for (int64_t s = 0; s < kv_len; ++s) {
+        int64_t row = cu_k[b] + s;
+        double dot = 0.0;
+        for (int d = 0; d < d_qk; ++d)
+          dot += load_elem(q_kind, q, (t * H + h) * (int64_t)d_qk + d, NULL, 0) *
+                 load_elem(c_kind, latent, row * d_qk + d, NULL, 0);
+        z[s] = scale * dot + mask[s];
+        if (z[s] > zmax) zmax = z[s];
+      }
+      double* o = out + (r * H + h) * (int64_t)d_v;
+      for (int d = 0; d < d_v; ++d) o[d] = 0.0;
+      if (zmax == -INFINITY) {
+        lse[r * H + h] = -INFINITY;
+        continue;
+      }
+      double denom = 0.0;
+      for (int64_t s = 0; s < kv_len; ++s) denom += exp(z[s] - zmax);
+      for (int64_t s = 0; s < kv_len; ++s) {
+        double p = exp(z[s] - zmax) / denom;
+        if (p == 0.0) continue;
+        int64_t row = cu_k[b] + s;
+        for (int d = 0; d < d_v; ++d) o[d] += p * load_elem(c_kind, latent, row * d_qk + d, NULL, 0);
+      }
+      lse[r * H + h] = zmax + log(denom);
+    }
+    free(mask);
+    free(z);
+  }
+  return bad ? -1 : 0;
+}

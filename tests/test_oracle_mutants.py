@@ -1,0 +1,81 @@
+"""Plant one plausible mistake at a time in a copy of the oracle's C source and
+check that the pins in test_oracle_pins.py reject every such copy.  Runs on the
+CPU only; the real oracle is never modified."""
+import os
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "dsa_oracle.c")
+
+# (name, original text, mutated text); each original must occur exactly once
+MUTANTS = [
+    ("relu dropped", "double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot;"),
+    ("causal mask excludes the diagonal", "      if (s > pos) {\n        out[s] = -INFINITY;",
+     "      if (s >= pos) {\n        out[s] = -INFINITY;"),
+    ("sequence offset of key rows dropped", "int64_t key_row = cu_k[b] + s;", "int64_t key_row = s;"),
+    ("head weight of the wrong query", "total += w[t * H_I + j] * relu;", "total += w[j] * relu;"),
+    ("e4m3 exponent bias off by one", "v = ldexp(1.0 + m / 8.0, e - 7);", "v = ldexp(1.0 + m / 8.0, e - 8);"),
+    ("e4m3 subnormal scale", "v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    ("e4m3 scale not applied", "* (double)row_scale[row];", ";"),
+    ("bf16 bits misplaced", "uint32_t u = ((uint32_t)bits) << 16;", "uint32_t u = ((uint32_t)bits) << 15;"),
+    ("tie-break reversed", "return (x->index > y->index) - (x->index < y->index);",
+     "return (x->index < y->index) - (x->index > y->index);"),
+    ("ascending instead of descending", "if (x->score > y->score) return -1;\n  if (x->score < y->score) return 1;",
+     "if (x->score > y->score) return 1;\n  if (x->score < y->score) return -1;"),
+    ("diagonal candidate dropped", "int64_t n = pos + 1;\n    candidate*", "int64_t n = pos;\n    candidate*"),
+    ("softmax scale dropped", "z[i] = scale * dot;", "z[i] = dot;"),
+    ("values from the tail of the latent row",
+     "for (int d = 0; d < d_v; ++d) o[d] += p * load_elem(c_kind, latent, row * d_qk + d, NULL, 0);\n      }\n      lse[r * H + h] = zmax + log(denom);\n    }\n    free(z);",
+     "for (int d = 0; d < d_v; ++d) o[d] += p * load_elem(c_kind, latent, row * d_qk + (d_qk - d_v) + d, NULL, 0);\n      }\n      lse[r * H + h] = zmax + log(denom);\n    }\n    free(z);"),
+    ("lse without the max", "      lse[r * H + h] = zmax + log(denom);\n    }\n    free(z);",
+     "      lse[r * H + h] = log(denom);\n    }\n    free(z);"),
+    ("causal check of selected entries off by one", "return s >= 0 && s <= pos && s < kv_len;",
+     "return s >= 0 && s <= pos + 1 && s < kv_len;"),
+    ("query head stride wrong", "dot += load_elem(q_kind, q, (t * H + h) * (int64_t)d_qk + d, NULL, 0) *\n                 load_elem(c_kind, latent, row * d_qk + d, NULL, 0);\n        z[i]",
+     "dot += load_elem(q_kind, q, (t * H) * (int64_t)d_qk + d, NULL, 0) *\n                 load_elem(c_kind, latent, row * d_qk + d, NULL, 0);\n        z[i]"),
+]
+
+PIN_TESTS = [
+    ("test_e4m3_decode_exhaustive", {}),
+    ("test_bf16_decode_random_patterns", {}),
+    ("test_scores_match_einsum", {"kfp8": False}),
+    ("test_scores_match_einsum", {"kfp8": True}),
+    ("test_scores_exact_on_integer_inputs", {}),
+    ("test_hadamard_rotation_leaves_scores_unchanged", {}),
+    ("test_topk_matches_lexsort_with_ties", {"levels": 3}),
+    ("test_topk_invariants", {}),
+    ("test_sparse_equals_dense_causal_when_topk_covers_everything", {}),
+    ("test_sparse_equals_additive_mask_formulation", {}),
+    ("test_attention_closed_forms", {}),
+    ("test_attention_ignores_order_padding_and_invalid_entries", {}),
+]
+
+
+def _caught(lib_mod):
+    for name, kw in PIN_TESTS:
+        try:
+            getattr(pins, name)(lib_mod, **kw)
+        except Exception:
+            return name
+    return None
+
+
+def test_unmutated_copy_passes_every_pin(tmp_path):
+    so = oracle.compile_source(SRC, str(tmp_path / "copy.so"))
+    with oracle.use_library(so):
+        assert _caught(oracle) is None
+
+
+@pytest.mark.parametrize("name,orig,mut", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_reject_mutant(tmp_path, name, orig, mut):
+    src = open(SRC).read()
+    assert src.count(orig) == 1, f"mutation site not unique: {name}"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(orig, mut))
+    so = oracle.compile_source(str(path), str(tmp_path / "mutant.so"))
+    with oracle.use_library(so):
+        caught_by = _caught(oracle)
+    assert caught_by is not None, f"no pin rejects the mutant '{name}'"
