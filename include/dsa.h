@@ -1,0 +1,182 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * Three steps, each one call, plus a fused forward:
+ *   dsa_indexer_scores   lightning-indexer scores of every query against every
+ *                        causally preceding index key
+ *   dsa_topk             per-query top-k token selection over those scores
+ *   dsa_sparse_mla_attn  MLA attention (absorbed MQA form) over the selected rows
+ *   dsa_forward          the three in sequence, chunked over query rows
+ *
+ * Conventions shared by every entry point
+ *  - Every tensor pointer is DEVICE memory owned by the caller; the library
+ *    never allocates, frees or keeps a pointer after the call returns.
+ *  - Calls are asynchronous on `stream`.  Argument errors are detected on the
+ *    host and returned before anything is launched; nothing is written then.
+ *  - Sequences are packed ("varlen"): sequence b owns query rows
+ *    [cu_q[b], cu_q[b+1]) and key/cache rows [cu_k[b], cu_k[b+1]).  The new
+ *    queries are the last q_len_b tokens of the sequence, so local query i sits
+ *    at absolute position pos = kv_len_b - q_len_b + i and may attend to keys
+ *    0..pos (its own position included: the causal mask is -inf strictly above
+ *    the diagonal -- "DeepSeek-V3.2-Exp" token-ids page, "Position IDs").
+ *    Key indices in scores and idx are sequence-local (0 = first key of the
+ *    sequence).  The caller appends the new tokens to the index-key cache and to
+ *    the latent cache before the call ("DeepSeek-V3.2", transformers doc: the
+ *    indexer keeps its own per-token key cache beside the main cache and it is
+ *    updated before scoring).
+ *  - A query range [q_begin, q_end) of global query rows selects the rows a
+ *    call processes.  Tensors indexed by query row (q_idx, w, q, out, lse) are
+ *    addressed by GLOBAL row; the scores and idx buffers of the stage calls are
+ *    CHUNK-relative: their row r belongs to global row q_begin + r.
+ *  - Supported shapes: the released layer (index heads 64, index dim 128,
+ *    attention heads 128, q/k dim 576 = 512 latent + 64 RoPE, v dim 512) and a
+ *    tiny test shape (4, 32 | 4, 80, 64).  Others return DSA_ERR_UNSUPPORTED.
+ *  - Device-side waits are bounded.  If one gives up, the kernel records a code
+ *    in a library-global device word, skips its remaining work and returns;
+ *    dsa_device_error() reads and clears it.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,   /* null pointer, bad length, misaligned buffer, ... */
+  DSA_ERR_UNSUPPORTED = 2,   /* shape outside the supported set */
+  DSA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  DSA_ERR_DEVICE_TIMEOUT = 4,/* a bounded device-side wait gave up (see dsa_device_error) */
+  DSA_ERR_WORKSPACE = 5      /* workspace missing or smaller than dsa_forward_workspace_size */
+} dsa_status;
+
+typedef enum {
+  DSA_KIDX_BF16 = 0,        /* index keys stored as bf16 [sum kv, idx_dim] */
+  DSA_KIDX_FP8_E4M3 = 1     /* index keys stored as e4m3 bytes [sum kv, idx_dim] plus one fp32
+                               scale per key: k = e4m3(byte) * k_scale[key] */
+} dsa_kidx_dtype;
+
+/* Packed sequence layout.  The device and host copies must hold the same
+ * values: cu_q[0] = cu_k[0] = 0, non-decreasing, q_len_b <= kv_len_b. */
+typedef struct {
+  int32_t batch;              /* B >= 1 */
+  const int32_t* cu_q;        /* device, [B+1]: query-row offsets */
+  const int32_t* cu_k;        /* device, [B+1]: key/cache-row offsets */
+  const int32_t* cu_q_host;   /* host,   [B+1]: same values as cu_q */
+  const int32_t* cu_k_host;   /* host,   [B+1]: same values as cu_k */
+} dsa_varlen;
+
+/*
+ * Step 1: lightning-indexer scores.
+ * Source: "DeepSeek-V3.2" (transformers model doc), section "DeepSeek Sparse
+ * Attention (DSA)", item 1 -- a light, low-head-count module scores each query
+ * against every preceding key; the released config has index_n_heads 64 and
+ * index_head_dim 128 ("DeepSeek-V3.2-Exp" token-ids page).  Score:
+ *     I[t,s] = sum_j w[t,j] * max(0, q_idx[t,j,:] . k[s,:]),   0 <= s <= pos(t)
+ * q_idx     bf16 [T, n_idx_heads, idx_dim], row-major, global rows
+ * w         fp32 [T, n_idx_heads]
+ * k_idx     bf16 or e4m3 bytes [sum kv, idx_dim] (see dsa_kidx_dtype);
+ *           k_scale fp32 [sum kv] for e4m3, NULL for bf16
+ * scores    fp32 [q_end - q_begin, ld_scores], chunk-relative rows.  Row r
+ *           receives columns 0..pos(q_begin+r); columns past the diagonal in
+ *           the same 128-key tile are set to -inf; later columns are not
+ *           written.  ld_scores >= the longest kv_len among the rows.
+ * Accumulation is fp32 (bf16 x bf16 products are exact); for e4m3 keys the
+ * per-key scale multiplies the head-reduced score (scale > 0 commutes with ReLU).
+ * Alignment: all tensors 16-byte aligned; ld_scores a multiple of 4.
+ */
+dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_idx,
+                              const float* k_scale, dsa_kidx_dtype k_dtype, dsa_varlen v,
+                              int32_t n_idx_heads, int32_t idx_dim, int64_t q_begin,
+                              int64_t q_end, float* scores, int64_t ld_scores,
+                              cudaStream_t stream);
+
+/*
+ * Step 2: fine-grained token selection.
+ * Source: "DeepSeek-V3.2" (transformers model doc), section "DeepSeek Sparse
+ * Attention (DSA)", item 2 -- each query keeps the top index_topk (2048 by
+ * default) tokens.  Ties are broken toward the lower key index; -0.0 ties +0.0.
+ * scores    fp32 [q_end - q_begin, ld_scores] chunk-relative, as written by
+ *           dsa_indexer_scores (only columns 0..pos(t) are read)
+ * idx       int32 [q_end - q_begin, topk] chunk-relative.  Row r holds the
+ *           min(topk, pos+1) selected sequence-local key indices -- first those
+ *           with a score above the k-th largest, in increasing index order, then
+ *           those equal to it, in increasing index order -- followed by -1.
+ *           The SET is the definition; the order is fixed only so that
+ *           repeated runs are bit-identical.
+ * topk in [1, 2048].  Scores must not be NaN.
+ */
+dsa_status dsa_topk(const float* scores, int64_t ld_scores, dsa_varlen v, int64_t q_begin,
+                    int64_t q_end, int32_t topk, int32_t* idx, cudaStream_t stream);
+
+/*
+ * Step 3: MLA attention in absorbed MQA form over the selected rows.
+ * Sources: "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse
+ * Attention (DSA)", item 2 -- main MLA attention is computed only over the
+ * selected tokens; "DeepSeek-V3.2 - Experimental Exp Version" (altools),
+ * "Technical Principles" -- MLA with MQA, key entries shared by all query
+ * heads; "DeepSeek-V3.2 / Exp" (visual-learn explainer) -- the cached entries
+ * are MLA's compressed vectors.  For query row t, head h, selected row s:
+ *     z_s = scale * q[t,h,:d_qk] . latent[s,:d_qk]
+ *     out[t,h,:] = sum_s softmax(z)_s * latent[s, :d_v],   lse[t,h] = log sum_s exp(z_s)
+ * q         bf16 [T, n_heads, d_qk] global rows (RoPE part already applied)
+ * latent    bf16 [sum kv, d_qk]: per token the 512-d latent then the 64-d RoPE key
+ * idx       int32 [q_end - q_begin, topk] chunk-relative, sequence-local rows.
+ *           Entries outside 0..pos(t) (including the -1 padding) are ignored.
+ * out       bf16 [T, n_heads, d_v] global rows; lse fp32 [T, n_heads] (nullable).
+ *           A row with no valid entry gets out = 0 and lse = -inf.
+ * QK and PV run on the tensor cores (bf16 in, fp32 accumulate); the softmax
+ * probabilities are rounded to bf16 for PV.  topk must be a multiple of 64.
+ */
+dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t* idx,
+                               dsa_varlen v, int64_t q_begin, int64_t q_end, int32_t topk,
+                               int32_t n_heads, int32_t d_qk, int32_t d_v, float scale,
+                               void* out, float* lse, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace dsa_forward needs for this layout when it runs at
+ * most q_chunk query rows per pass (q_chunk <= 0: all rows in one pass).  The
+ * workspace holds one pass's fp32 scores and int32 selections.  Returns 0 for
+ * invalid arguments.
+ */
+size_t dsa_forward_workspace_size(dsa_varlen v, int32_t topk, int64_t q_chunk);
+
+/*
+ * The whole hot path for every query row: dsa_indexer_scores -> dsa_topk ->
+ * dsa_sparse_mla_attn, in passes of at most q_chunk rows so that the score
+ * buffer stays bounded; all launches go to `stream` in order.  Arguments as
+ * for the three steps.  idx_out (nullable) receives the selections of every
+ * row, [T, topk] int32, global rows.  workspace: device, at least
+ * dsa_forward_workspace_size(v, topk, q_chunk) bytes, 256-byte aligned.
+ * Prefill, chunked prefill and decode are the same call: they differ only in
+ * the lengths held by v.
+ */
+dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
+                       const float* k_scale, dsa_kidx_dtype k_dtype, const void* q,
+                       const void* latent, dsa_varlen v, int32_t n_idx_heads,
+                       int32_t idx_dim, int32_t topk, int32_t n_heads, int32_t d_qk,
+                       int32_t d_v, float scale, int64_t q_chunk, void* out, float* lse,
+                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/* Reads and clears the device error word of the current device (synchronises
+ * `stream` first).  *code = 0 when no device-side wait gave up. */
+dsa_status dsa_device_error(int32_t* code, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char* dsa_status_string(dsa_status status);
+
+/* Library version, "major.minor.patch". */
+const char* dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,184 @@
+"""B200 (sm_100a) DeepSeek Sparse Attention hot path -- Python binding.
+
+A thin ctypes layer over ``libdsa.so`` whose functions carry the names of the
+C ABI in ``include/dsa.h``: ``dsa_indexer_scores``, ``dsa_topk``,
+``dsa_sparse_mla_attn``, ``dsa_forward_workspace_size``, ``dsa_forward``,
+``dsa_device_error``, ``dsa_status_string``.  It only marshals arguments:
+every step of the computation runs in the library's CUDA kernels.  Tensors are
+torch tensors in device memory (PyTorch provides memory and streams); the
+packed sequence layout is described by :class:`Varlen`.
+
+There is no fallback: if ``libdsa.so`` is missing or cannot be loaded, the
+import of this package fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa.so")
+
+DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA, DSA_ERR_DEVICE_TIMEOUT, DSA_ERR_WORKSPACE = range(6)
+DSA_KIDX_BF16, DSA_KIDX_FP8_E4M3 = 0, 1
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {dsa_status_string(status)} (status {status})")
+        self.status = status
+
+
+class dsa_varlen(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("cu_q", ctypes.c_void_p),
+        ("cu_k", ctypes.c_void_p),
+        ("cu_q_host", ctypes.POINTER(ctypes.c_int32)),
+        ("cu_k_host", ctypes.POINTER(ctypes.c_int32)),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m sparse_attention_long_07_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    lib.dsa_indexer_scores.argtypes = [vp, vp, vp, vp, ctypes.c_int, dsa_varlen, i32, i32, i64, i64, vp, i64, vp]
+    lib.dsa_topk.argtypes = [vp, i64, dsa_varlen, i64, i64, i32, vp, vp]
+    lib.dsa_sparse_mla_attn.argtypes = [vp, vp, vp, dsa_varlen, i64, i64, i32, i32, i32, i32, f32, vp, vp, vp]
+    lib.dsa_forward_workspace_size.argtypes = [dsa_varlen, i32, i64]
+    lib.dsa_forward_workspace_size.restype = ctypes.c_size_t
+    lib.dsa_forward.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp, dsa_varlen, i32, i32, i32, i32, i32, i32,
+                                f32, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.dsa_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
+    lib.dsa_status_string.argtypes = [ctypes.c_int]
+    lib.dsa_status_string.restype = ctypes.c_char_p
+    lib.dsa_version.restype = ctypes.c_char_p
+    for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward", "dsa_device_error"):
+        getattr(lib, fn).restype = ctypes.c_int
+    return lib
+
+
+_lib = _load()
+
+EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward_workspace_size",
+            "dsa_forward", "dsa_device_error", "dsa_status_string", "dsa_version")
+
+
+def library():
+    """The loaded ctypes library (for symbol checks)."""
+    return _lib
+
+
+class Varlen:
+    """Packed sequence layout: cumulative query and key/cache row offsets.
+
+    Keeps both the device copies the kernels read and the host copies the
+    library validates and plans launches with.
+    """
+
+    def __init__(self, cu_q, cu_k, device=None):
+        cu_q = torch.as_tensor(cu_q, dtype=torch.int32).cpu().contiguous()
+        cu_k = torch.as_tensor(cu_k, dtype=torch.int32).cpu().contiguous()
+        self.cu_q_host, self.cu_k_host = cu_q, cu_k
+        if device is None:
+            self.cu_q, self.cu_k = cu_q, cu_k
+        else:
+            self.cu_q, self.cu_k = cu_q.to(device), cu_k.to(device)
+        self.batch = cu_q.numel() - 1
+        self.T = int(cu_q[-1])
+        self.S = int(cu_k[-1])
+        kv = (cu_k[1:] - cu_k[:-1])
+        self.max_kv = int(kv.max()) if kv.numel() else 0
+
+    def c(self) -> dsa_varlen:
+        return dsa_varlen(self.batch, self.cu_q.data_ptr(), self.cu_k.data_ptr(),
+                          ctypes.cast(self.cu_q_host.data_ptr(), ctypes.POINTER(ctypes.c_int32)),
+                          ctypes.cast(self.cu_k_host.data_ptr(), ctypes.POINTER(ctypes.c_int32)))
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(status: int, what: str):
+    if status != DSA_OK:
+        raise DSAError(status, what)
+
+
+def _kdtype(k_idx):
+    return DSA_KIDX_FP8_E4M3 if k_idx.dtype in (torch.float8_e4m3fn, torch.uint8) else DSA_KIDX_BF16
+
+
+def dsa_status_string(status: int) -> str:
+    return _lib.dsa_status_string(int(status)).decode()
+
+
+def dsa_version() -> str:
+    return _lib.dsa_version().decode()
+
+
+def dsa_indexer_scores(q_idx, w, k_idx, k_scale, v: Varlen, q_begin, q_end, scores, stream=None):
+    """Lightning-indexer scores for global query rows [q_begin, q_end) into
+    ``scores`` [q_end - q_begin, ld] fp32 (chunk-relative rows)."""
+    T, H_I, d_I = q_idx.shape
+    _check(_lib.dsa_indexer_scores(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _kdtype(k_idx), v.c(),
+                                   H_I, d_I, q_begin, q_end, _ptr(scores), scores.stride(0), _stream(stream)),
+           "dsa_indexer_scores")
+    return scores
+
+
+def dsa_topk(scores, v: Varlen, q_begin, q_end, topk, idx, stream=None):
+    """Top-k selection of chunk-relative score rows into ``idx`` [rows, topk] int32."""
+    _check(_lib.dsa_topk(_ptr(scores), scores.stride(0), v.c(), q_begin, q_end, topk, _ptr(idx),
+                         _stream(stream)), "dsa_topk")
+    return idx
+
+
+def dsa_sparse_mla_attn(q, latent, idx, v: Varlen, q_begin, q_end, scale, out, lse=None, d_v=None,
+                        stream=None):
+    """MLA attention (absorbed MQA) over the selected rows; writes out/lse for
+    global rows [q_begin, q_end)."""
+    T, H, d_qk = q.shape
+    d_v = out.shape[-1] if d_v is None else d_v
+    _check(_lib.dsa_sparse_mla_attn(_ptr(q), _ptr(latent), _ptr(idx), v.c(), q_begin, q_end, idx.shape[1], H,
+                                    d_qk, d_v, float(scale), _ptr(out), _ptr(lse), _stream(stream)),
+           "dsa_sparse_mla_attn")
+    return out, lse
+
+
+def dsa_forward_workspace_size(v: Varlen, topk: int, q_chunk: int = 0) -> int:
+    return int(_lib.dsa_forward_workspace_size(v.c(), topk, q_chunk))
+
+
+def dsa_forward(q_idx, w, k_idx, k_scale, q, latent, v: Varlen, topk, scale, out, lse, workspace,
+                idx_out=None, q_chunk: int = 0, stream=None):
+    """Indexer -> top-k -> sparse MLA for every query row (see include/dsa.h)."""
+    T, H_I, d_I = q_idx.shape
+    _, H, d_qk = q.shape
+    d_v = out.shape[-1]
+    _check(_lib.dsa_forward(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _kdtype(k_idx), _ptr(q),
+                            _ptr(latent), v.c(), H_I, d_I, topk, H, d_qk, d_v, float(scale), q_chunk,
+                            _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(workspace),
+                            0 if workspace is None else workspace.numel() * workspace.element_size(),
+                            _stream(stream)), "dsa_forward")
+    return out, lse
+
+
+def dsa_device_error(stream=None) -> int:
+    """Read and clear the library's device error word (0 = no device wait gave up)."""
+    code = ctypes.c_int32(0)
+    st = _lib.dsa_device_error(ctypes.byref(code), _stream(stream))
+    if st not in (DSA_OK, DSA_ERR_DEVICE_TIMEOUT):
+        raise DSAError(st, "dsa_device_error")
+    return int(code.value)

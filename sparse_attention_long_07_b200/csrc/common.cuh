@@ -1,0 +1,43 @@
+// common.cuh -- small device helpers shared by the DSA kernels.
+#pragma once
+
+#include <stdint.h>
+
+namespace dsa {
+
+// Where global query row t sits: its sequence, absolute position and the
+// sequence's key range.  Sequence b owns query rows [cu_q[b], cu_q[b+1]) and
+// key rows [cu_k[b], cu_k[b+1]); its q_len new queries are its last tokens.
+struct RowInfo {
+  int b;
+  int pos;       // absolute position of the query = last key index it may see
+  int kv_len;
+  int k_base;    // first global key row of the sequence
+};
+
+__device__ __forceinline__ RowInfo locate_row(const int32_t* __restrict__ cu_q,
+                                              const int32_t* __restrict__ cu_k, int B, int64_t t) {
+  // largest b with cu_q[b] <= t (then cu_q[b+1] > t, empty sequences skipped)
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (cu_q[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  RowInfo r;
+  r.b = lo;
+  int q0 = cu_q[lo], q1 = cu_q[lo + 1];
+  r.k_base = cu_k[lo];
+  r.kv_len = cu_k[lo + 1] - r.k_base;
+  r.pos = r.kv_len - (q1 - q0) + static_cast<int>(t - q0);
+  return r;
+}
+
+// Order-preserving map of a non-NaN float to uint32 (larger float -> larger
+// key); -0.0 is first folded onto +0.0 so that the two tie.
+__device__ __forceinline__ uint32_t order_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+}  // namespace dsa

@@ -1,0 +1,421 @@
+// dsa.cu -- C ABI of the DSA hot path (declarations and contracts in include/dsa.h).
+//
+// Host side: argument validation (all of it before the first CUDA call, so an
+// invalid call touches no device state), TMA descriptor encoding, launch
+// configuration, and the chunked forward.  Device side: the kernels in
+// indexer.cuh, topk.cuh and sparse_mla.cuh.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "dsa.h"
+#include "indexer.cuh"
+#include "sparse_mla.cuh"
+#include "topk.cuh"
+
+namespace {
+
+using dsa::IndexerCfg;
+using dsa::MlaCfg;
+
+// ----------------------------------------------------------------------------
+// Validation of the packed layout (host copies only)
+// ----------------------------------------------------------------------------
+struct Layout {
+  int B = 0;
+  int64_t T = 0;         // total query rows
+  int64_t S = 0;         // total key rows
+  int max_kv = 0;        // longest kv_len over sequences with a row in [q_begin, q_end)
+  int max_q_rows = 0;    // most rows of one sequence inside [q_begin, q_end)
+  int max_tiles = 0;     // most 128-key tiles one query row of the range needs
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dsa_status check_varlen(const dsa_varlen& v, int64_t q_begin, int64_t q_end, Layout* out) {
+  if (v.batch < 1 || !v.cu_q || !v.cu_k || !v.cu_q_host || !v.cu_k_host) return DSA_ERR_INVALID_ARG;
+  if (v.cu_q_host[0] != 0 || v.cu_k_host[0] != 0) return DSA_ERR_INVALID_ARG;
+  Layout L;
+  L.B = v.batch;
+  for (int b = 0; b < v.batch; ++b) {
+    const int64_t ql = static_cast<int64_t>(v.cu_q_host[b + 1]) - v.cu_q_host[b];
+    const int64_t kl = static_cast<int64_t>(v.cu_k_host[b + 1]) - v.cu_k_host[b];
+    if (ql < 0 || kl < ql) return DSA_ERR_INVALID_ARG;
+  }
+  L.T = v.cu_q_host[v.batch];
+  L.S = v.cu_k_host[v.batch];
+  if (q_begin < 0 || q_end < q_begin || q_end > L.T) return DSA_ERR_INVALID_ARG;
+  for (int b = 0; b < v.batch; ++b) {
+    const int64_t lo = std::max<int64_t>(v.cu_q_host[b], q_begin);
+    const int64_t hi = std::min<int64_t>(v.cu_q_host[b + 1], q_end);
+    if (lo >= hi) continue;
+    const int kl = v.cu_k_host[b + 1] - v.cu_k_host[b];
+    const int ql = v.cu_q_host[b + 1] - v.cu_q_host[b];
+    const int pos_last = kl - ql + static_cast<int>(hi - 1 - v.cu_q_host[b]);
+    L.max_kv = std::max(L.max_kv, kl);
+    L.max_q_rows = std::max(L.max_q_rows, static_cast<int>(hi - lo));
+    L.max_tiles = std::max(L.max_tiles, pos_last / 128 + 1);
+  }
+  *out = L;
+  return DSA_OK;
+}
+
+// Optional host-side fault injection for tests of the error paths:
+// DSA_INJECT_FAULT=cuda | timeout makes the next entry point report that
+// failure without launching anything.
+dsa_status injected_fault() {
+  const char* f = std::getenv("DSA_INJECT_FAULT");
+  if (!f) return DSA_OK;
+  if (!std::strcmp(f, "cuda")) return DSA_ERR_CUDA;
+  if (!std::strcmp(f, "timeout")) return DSA_ERR_DEVICE_TIMEOUT;
+  return DSA_OK;
+}
+
+// ----------------------------------------------------------------------------
+// TMA descriptors (cuTensorMapEncodeTiled through the runtime's entry point)
+// ----------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Row-major 2D tensor [rows, cols] with a row stride in bytes; box
+// {box_cols, box_rows}; out-of-bounds elements read as zero.
+bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t cols,
+              uint64_t rows, uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows,
+              CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+bool is_released_indexer(int h, int d) { return h == 64 && d == 128; }
+bool is_tiny_indexer(int h, int d) { return h == 4 && d == 32; }
+bool is_released_mla(int h, int dqk, int dv) { return h == 128 && dqk == 576 && dv == 512; }
+bool is_tiny_mla(int h, int dqk, int dv) { return h == 4 && dqk == 80 && dv == 64; }
+
+// ----------------------------------------------------------------------------
+// Launchers (arguments already validated)
+// ----------------------------------------------------------------------------
+template <class C>
+dsa_status launch_indexer(const void* q_idx, const float* w, const void* k_idx,
+                          const float* k_scale, const dsa_varlen& v, const Layout& L,
+                          int64_t q_begin, int64_t q_end, float* scores, int64_t ld,
+                          cudaStream_t stream) {
+  CUtensorMap tm_q, tm_k;
+  if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q_idx, C::D_I,
+                static_cast<uint64_t>(L.T) * C::H_I, C::D_I * 2, C::ATOM_ELEMS, C::N,
+                C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+    return DSA_ERR_CUDA;
+  if (C::KFP8) {
+    if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_idx, C::D_I, static_cast<uint64_t>(L.S),
+                  C::D_I, C::D_I, C::BK, CU_TENSOR_MAP_SWIZZLE_128B))
+      return DSA_ERR_CUDA;
+  } else {
+    if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k_idx, C::D_I,
+                  static_cast<uint64_t>(L.S), C::D_I * 2, C::ATOM_ELEMS, C::BK,
+                  C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+      return DSA_ERR_CUDA;
+  }
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] { attr_err = set_smem(dsa::indexer_scores_kernel<C>, C::SMEM_BYTES); });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+
+  dsa::IndexerParams p;
+  p.w = w;
+  p.k_scale = k_scale;
+  p.cu_q = v.cu_q;
+  p.cu_k = v.cu_k;
+  p.B = v.batch;
+  p.q_begin = q_begin;
+  p.q_end = q_end;
+  p.scores = scores;
+  p.ld = ld;
+  p.chunk_tiles = C::NQ == 1 ? 32 : 64;
+  const int qblocks = (L.max_q_rows + C::NQ - 1) / C::NQ;
+  const int chunks = (L.max_tiles + p.chunk_tiles - 1) / p.chunk_tiles;
+  if (qblocks == 0 || chunks == 0) return DSA_OK;
+  if (chunks > 65535 || v.batch > 65535) return DSA_ERR_UNSUPPORTED;
+  if (qblocks > 65535) return DSA_ERR_UNSUPPORTED;   // gridDim.y limit
+  dim3 grid(chunks, qblocks, v.batch);
+  dsa::indexer_scores_kernel<C><<<grid, C::NT, C::SMEM_BYTES, stream>>>(tm_q, tm_k, p);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+template <class C>
+dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, const dsa_varlen& v,
+                      const Layout& L, int64_t q_begin, int64_t q_end, int topk, float scale,
+                      void* out, float* lse, cudaStream_t stream) {
+  CUtensorMap tm_q, tm_lat;
+  if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, C::DQK, static_cast<uint64_t>(L.T) * C::H,
+                C::DQK * 2, C::ATOM, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  if (!make_map(&tm_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, latent, C::DQK, static_cast<uint64_t>(L.S),
+                C::DQK * 2, C::ATOM, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] { attr_err = set_smem(dsa::sparse_mla_kernel<C>, C::SMEM_BYTES); });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+
+  dsa::MlaParams p;
+  p.idx = idx;
+  p.cu_q = v.cu_q;
+  p.cu_k = v.cu_k;
+  p.B = v.batch;
+  p.q_begin = q_begin;
+  p.topk = topk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  const int64_t rows = q_end - q_begin;
+  if (rows == 0) return DSA_OK;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * C::SPLIT), 1, 1);
+  cfg.blockDim = dim3(C::NT, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C::SPLIT;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, dsa::sparse_mla_kernel<C>, tm_q, tm_lat, p);
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status check_indexer_args(const void* q_idx, const float* w, const void* k_idx,
+                              const float* k_scale, dsa_kidx_dtype kd, int h, int d,
+                              const float* scores, int64_t ld, const Layout& L) {
+  if (!q_idx || !w || !k_idx || !scores) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores))
+    return DSA_ERR_INVALID_ARG;
+  if (kd != DSA_KIDX_BF16 && kd != DSA_KIDX_FP8_E4M3) return DSA_ERR_INVALID_ARG;
+  if (kd == DSA_KIDX_FP8_E4M3 && !k_scale) return DSA_ERR_INVALID_ARG;
+  if (ld < L.max_kv || ld % 4 != 0) return DSA_ERR_INVALID_ARG;
+  if (is_released_indexer(h, d)) return DSA_OK;
+  if (is_tiny_indexer(h, d) && kd == DSA_KIDX_BF16) return DSA_OK;
+  return DSA_ERR_UNSUPPORTED;
+}
+
+dsa_status check_mla_args(const void* q, const void* latent, const int32_t* idx, int topk, int h,
+                          int dqk, int dv, float scale, const void* out, const float* lse) {
+  if (!q || !latent || !idx || !out) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(latent) || !aligned16(idx) || !aligned16(out) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return DSA_ERR_INVALID_ARG;
+  if (topk < 1 || topk > 2048) return DSA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return DSA_ERR_INVALID_ARG;
+  if (is_released_mla(h, dqk, dv) || is_tiny_mla(h, dqk, dv)) return DSA_OK;
+  return DSA_ERR_UNSUPPORTED;
+}
+
+dsa_status run_indexer(const void* q_idx, const float* w, const void* k_idx, const float* k_scale,
+                       dsa_kidx_dtype kd, const dsa_varlen& v, const Layout& L, int h, int d,
+                       int64_t q_begin, int64_t q_end, float* scores, int64_t ld,
+                       cudaStream_t stream) {
+  if (q_end == q_begin) return DSA_OK;
+  const bool decode_like = L.max_q_rows <= 2;
+  if (is_tiny_indexer(h, d))
+    return launch_indexer<IndexerCfg<4, 32, 4, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                        scores, ld, stream);
+  if (kd == DSA_KIDX_FP8_E4M3) {
+    if (decode_like)
+      return launch_indexer<IndexerCfg<64, 128, 1, true>>(q_idx, w, k_idx, k_scale, v, L, q_begin,
+                                                           q_end, scores, ld, stream);
+    return launch_indexer<IndexerCfg<64, 128, 4, true>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                         scores, ld, stream);
+  }
+  if (decode_like)
+    return launch_indexer<IndexerCfg<64, 128, 1, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin,
+                                                          q_end, scores, ld, stream);
+  return launch_indexer<IndexerCfg<64, 128, 4, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                        scores, ld, stream);
+}
+
+dsa_status run_topk(const float* scores, int64_t ld, const dsa_varlen& v, int64_t q_begin,
+                    int64_t q_end, int topk, int32_t* idx, cudaStream_t stream) {
+  const int64_t rows = q_end - q_begin;
+  if (rows == 0) return DSA_OK;
+  if (rows > 0x7FFFFFFF) return DSA_ERR_UNSUPPORTED;
+  dsa::topk_radix_kernel<512><<<static_cast<unsigned>(rows), 512, 0, stream>>>(
+      scores, ld, v.cu_q, v.cu_k, v.batch, q_begin, topk, idx);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status run_mla(const void* q, const void* latent, const int32_t* idx, const dsa_varlen& v,
+                   const Layout& L, int64_t q_begin, int64_t q_end, int topk, int h, int dqk, int dv,
+                   float scale, void* out, float* lse, cudaStream_t stream) {
+  if (is_tiny_mla(h, dqk, dv))
+    return launch_mla<MlaCfg<4, 80, 64, 1>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, out,
+                                            lse, stream);
+  return launch_mla<MlaCfg<128, 576, 512, 2>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, out,
+                                              lse, stream);
+}
+
+constexpr size_t kWsAlign = 256;
+size_t align_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+int64_t scores_ld(const Layout& L) { return std::max<int64_t>(4, (L.max_kv + 3) / 4 * 4); }
+
+}  // namespace
+
+extern "C" {
+
+dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_idx,
+                              const float* k_scale, dsa_kidx_dtype k_dtype, dsa_varlen v,
+                              int32_t n_idx_heads, int32_t idx_dim, int64_t q_begin,
+                              int64_t q_end, float* scores, int64_t ld_scores,
+                              cudaStream_t stream) {
+  Layout L;
+  dsa_status st = check_varlen(v, q_begin, q_end, &L);
+  if (st != DSA_OK) return st;
+  st = check_indexer_args(q_idx, w, k_idx, k_scale, k_dtype, n_idx_heads, idx_dim, scores, ld_scores, L);
+  if (st != DSA_OK) return st;
+  if ((st = injected_fault()) != DSA_OK) return st;
+  return run_indexer(q_idx, w, k_idx, k_scale, k_dtype, v, L, n_idx_heads, idx_dim, q_begin, q_end,
+                     scores, ld_scores, stream);
+}
+
+dsa_status dsa_topk(const float* scores, int64_t ld_scores, dsa_varlen v, int64_t q_begin,
+                    int64_t q_end, int32_t topk, int32_t* idx, cudaStream_t stream) {
+  Layout L;
+  dsa_status st = check_varlen(v, q_begin, q_end, &L);
+  if (st != DSA_OK) return st;
+  if (!scores || !idx || !aligned16(scores) || (reinterpret_cast<uintptr_t>(idx) & 3u))
+    return DSA_ERR_INVALID_ARG;
+  if (topk < 1 || topk > 2048 || ld_scores < L.max_kv || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+  if ((st = injected_fault()) != DSA_OK) return st;
+  return run_topk(scores, ld_scores, v, q_begin, q_end, topk, idx, stream);
+}
+
+dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t* idx,
+                               dsa_varlen v, int64_t q_begin, int64_t q_end, int32_t topk,
+                               int32_t n_heads, int32_t d_qk, int32_t d_v, float scale,
+                               void* out, float* lse, cudaStream_t stream) {
+  Layout L;
+  dsa_status st = check_varlen(v, q_begin, q_end, &L);
+  if (st != DSA_OK) return st;
+  st = check_mla_args(q, latent, idx, topk, n_heads, d_qk, d_v, scale, out, lse);
+  if (st != DSA_OK) return st;
+  if ((st = injected_fault()) != DSA_OK) return st;
+  return run_mla(q, latent, idx, v, L, q_begin, q_end, topk, n_heads, d_qk, d_v, scale, out, lse,
+                 stream);
+}
+
+size_t dsa_forward_workspace_size(dsa_varlen v, int32_t topk, int64_t q_chunk) {
+  Layout full;
+  if (v.batch < 1 || !v.cu_q_host || topk < 1 || topk > 2048) return 0;
+  if (check_varlen(v, 0, v.cu_q_host[v.batch], &full) != DSA_OK) return 0;
+  const int64_t rows = q_chunk > 0 ? std::min<int64_t>(q_chunk, full.T) : full.T;
+  const int64_t ld = scores_ld(full);
+  return align_up(static_cast<size_t>(std::max<int64_t>(rows, 1)) * ld * sizeof(float)) +
+         align_up(static_cast<size_t>(std::max<int64_t>(rows, 1)) * topk * sizeof(int32_t));
+}
+
+dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
+                       const float* k_scale, dsa_kidx_dtype k_dtype, const void* q,
+                       const void* latent, dsa_varlen v, int32_t n_idx_heads,
+                       int32_t idx_dim, int32_t topk, int32_t n_heads, int32_t d_qk,
+                       int32_t d_v, float scale, int64_t q_chunk, void* out, float* lse,
+                       int32_t* idx_out, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+  if (v.batch < 1 || !v.cu_q_host) return DSA_ERR_INVALID_ARG;
+  Layout full;
+  dsa_status st = check_varlen(v, 0, v.cu_q_host[v.batch], &full);
+  if (st != DSA_OK) return st;
+  if (!workspace) return DSA_ERR_WORKSPACE;
+  const int64_t ld = scores_ld(full);
+  st = check_indexer_args(q_idx, w, k_idx, k_scale, k_dtype, n_idx_heads, idx_dim,
+                          static_cast<const float*>(workspace), ld, full);
+  if (st != DSA_OK) return st;
+  st = check_mla_args(q, latent, idx_out ? idx_out : static_cast<const int32_t*>(workspace), topk,
+                      n_heads, d_qk, d_v, scale, out, lse);
+  if (st != DSA_OK) return st;
+  if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign) return DSA_ERR_INVALID_ARG;
+  const size_t need = dsa_forward_workspace_size(v, topk, q_chunk);
+  if (need == 0) return DSA_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return DSA_ERR_WORKSPACE;
+  if ((st = injected_fault()) != DSA_OK) return st;
+
+  const int64_t T = full.T;
+  const int64_t rows = q_chunk > 0 ? std::min<int64_t>(q_chunk, T) : T;
+  float* scores = static_cast<float*>(workspace);
+  int32_t* idx_ws = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
+                                               align_up(static_cast<size_t>(std::max<int64_t>(rows, 1)) * ld * sizeof(float)));
+  for (int64_t q0 = 0; q0 < T; q0 += rows) {
+    const int64_t q1 = std::min(T, q0 + rows);
+    Layout L;
+    if ((st = check_varlen(v, q0, q1, &L)) != DSA_OK) return st;
+    int32_t* idx = idx_out ? idx_out + q0 * topk : idx_ws;
+    if ((st = run_indexer(q_idx, w, k_idx, k_scale, k_dtype, v, L, n_idx_heads, idx_dim, q0, q1, scores,
+                          ld, stream)) != DSA_OK)
+      return st;
+    if ((st = run_topk(scores, ld, v, q0, q1, topk, idx, stream)) != DSA_OK) return st;
+    if ((st = run_mla(q, latent, idx, v, L, q0, q1, topk, n_heads, d_qk, d_v, scale, out, lse,
+                      stream)) != DSA_OK)
+      return st;
+  }
+  return DSA_OK;
+}
+
+dsa_status dsa_device_error(int32_t* code, cudaStream_t stream) {
+  if (!code) return DSA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return DSA_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, dsa::g_device_error, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(dsa::g_device_error, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  *code = v;
+  return v == 0 ? DSA_OK : DSA_ERR_DEVICE_TIMEOUT;
+}
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case DSA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char* dsa_version(void) { return "0.1.0"; }
+
+}  // extern "C"

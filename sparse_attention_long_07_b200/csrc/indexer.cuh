@@ -1,0 +1,342 @@
+// indexer.cuh -- lightning-indexer scores on the tcgen05 tensor cores.
+//
+// "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse Attention
+// (DSA)", item 1: a light module with few index heads scores each query
+// against every preceding key.  With index heads j, per-query head weights w
+// and a single-head index key per token:
+//     I[t,s] = sum_j w[t,j] * max(0, q_I[t,j,:] . k_I[s,:]),   s <= pos(t).
+//
+// GEMM view: A = a tile of 128 index keys (M = 128, one key per TMEM lane),
+// B = the index queries of NQ consecutive query tokens (N = NQ * H_I rows,
+// K = d_I), D = [128 keys x NQ*H_I logits] in fp32 tensor memory.  The
+// epilogue reads one key row per thread, so the ReLU, the head weights and the
+// sum over heads stay inside one thread and the [T x L x H_I] logits never
+// leave the SM; only the fp32 score per (query, key) is written.
+//
+// Roles: one TMA warp streams key tiles through a shared-memory ring; one
+// thread issues the MMAs into two TMEM accumulators (double buffer); one or two
+// epilogue warpgroups drain them.  For an e4m3 index-key cache, four more
+// warps widen each raw tile to bf16 in the UMMA layout (exact: every e4m3 value
+// is a bf16 value), and the per-key fp32 scale multiplies the head-reduced
+// score (a positive scale commutes with ReLU).
+#pragma once
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dsa {
+
+__host__ __device__ constexpr int pow2_at_least(int v, int lo) {
+  int p = lo;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+template <int H_I_, int D_I_, int NQ_, bool KFP8_>
+struct IndexerCfg {
+  static constexpr int H_I = H_I_, D_I = D_I_, NQ = NQ_;
+  static constexpr bool KFP8 = KFP8_;
+  static constexpr int BK = 128;                          // keys per tile (MMA M)
+  static constexpr int N = NQ * H_I;                      // MMA N
+  static constexpr int ROWB = D_I * 2;                    // bytes of one bf16 row
+  static constexpr int SWB = ROWB >= 128 ? 128 : ROWB;    // swizzle span (128 or 64 bytes)
+  static constexpr uint32_t SWZ = SWB == 128 ? 2u : 4u;   // descriptor swizzle code
+  static constexpr int NATOM = ROWB / SWB;                // swizzle-atom columns per row
+  static constexpr int ATOM_ELEMS = SWB / 2;
+  static constexpr int KSTEPS = D_I / 16;
+  static constexpr int STAGES = KFP8 ? 2 : 4;             // bf16 key-tile ring
+  static constexpr int RSTAGES = KFP8 ? 4 : 0;            // raw e4m3 ring
+  static constexpr int A_TILE = BK * ROWB;
+  static constexpr int B_TILE = N * ROWB;
+  static constexpr int RAW_TILE = BK * D_I;
+  static constexpr int EPI_WG = N >= 256 ? 2 : 1;         // epilogue warpgroups
+  static constexpr int QW = NQ / EPI_WG;                  // queries per epilogue warpgroup
+  static constexpr int COLS_PER_THREAD = QW * H_I;
+  static constexpr int LD_CHUNK = COLS_PER_THREAD >= 32 ? 32 : 16;
+  static constexpr int TMEM_COLS = pow2_at_least(2 * N, 32);
+  static constexpr int EPI_THREADS = 128 * EPI_WG;
+  static constexpr int PRODUCER_WARP = 4 * EPI_WG;
+  static constexpr int MMA_WARP = PRODUCER_WARP + 1;
+  static constexpr int CONVERT_WARP0 = MMA_WARP + 1;
+  static constexpr int NWARPS = MMA_WARP + 1 + (KFP8 ? 4 : 0);
+  static constexpr int NT = NWARPS * 32;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(128, N, false, false);
+  // shared memory layout (offsets from a 1024-byte aligned base)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + B_TILE;
+  static constexpr int OFF_RAW = OFF_K + STAGES * A_TILE;
+  static constexpr int OFF_W = OFF_RAW + RSTAGES * RAW_TILE;
+  static constexpr int OFF_BAR = OFF_W + NQ * H_I * 4;
+  static constexpr int NBAR = 2 + 2 * STAGES + 2 * RSTAGES + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
+  static_assert(B_TILE % 1024 == 0 && A_TILE % 1024 == 0, "atom alignment");
+  static_assert(COLS_PER_THREAD % LD_CHUNK == 0, "TMEM load chunking");
+  static_assert(!KFP8 || D_I == 128, "e4m3 keys: 128-byte rows");
+};
+
+struct IndexerParams {
+  const float* w;            // [T, H_I]
+  const float* k_scale;      // [sum kv] (e4m3 keys) or null
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int B;
+  int64_t q_begin, q_end;    // global query rows of this call
+  float* scores;             // [q_end - q_begin, ld]
+  int64_t ld;
+  int chunk_tiles;           // key tiles per CTA
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::NT, 1)
+    indexer_scores_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k, const IndexerParams p) {
+  // ---------------------------------------------------------------- work unit
+  const int b = blockIdx.z;
+  const int qb = gridDim.y - 1 - blockIdx.y;  // heaviest query blocks first
+  const int cq0 = p.cu_q[b], cq1 = p.cu_q[b + 1];
+  const int k_base = p.cu_k[b];
+  const int kv_len = p.cu_k[b + 1] - k_base;
+  const int64_t lo = cq0 > p.q_begin ? cq0 : p.q_begin;
+  const int64_t hi = cq1 < p.q_end ? cq1 : p.q_end;
+  const int64_t q0 = lo + static_cast<int64_t>(qb) * C::NQ;
+  if (q0 >= hi) return;
+  const int nq = static_cast<int>(hi - q0 < C::NQ ? hi - q0 : C::NQ);
+  const int pos0 = kv_len - (cq1 - cq0) + static_cast<int>(q0 - cq0);  // position of query q0
+  const int ntiles = (pos0 + nq - 1) / C::BK + 1;
+  const int t_begin = blockIdx.x * p.chunk_tiles;
+  const int t_end = min(ntiles, t_begin + p.chunk_tiles);
+  if (t_begin >= t_end || device_error_pending()) return;
+  const int n_iter = t_end - t_begin;
+
+  // ---------------------------------------------------------------- shared memory
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t s_q = sbase + C::OFF_Q;
+  const uint32_t s_k = sbase + C::OFF_K;
+  const uint32_t s_raw = sbase + C::OFF_RAW;
+  float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const uint32_t bar_q_full = bar0;
+  const uint32_t bar_drain = bar0 + 8;
+  auto bar_k_full = [&](int s) { return bar0 + 16 + 8 * s; };
+  auto bar_k_empty = [&](int s) { return bar0 + 16 + 8 * (C::STAGES + s); };
+  auto bar_raw_full = [&](int s) { return bar0 + 16 + 8 * (2 * C::STAGES + s); };
+  auto bar_raw_empty = [&](int s) { return bar0 + 16 + 8 * (2 * C::STAGES + C::RSTAGES + s); };
+  auto bar_acc_full = [&](int a) { return bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + a); };
+  auto bar_acc_empty = [&](int a) { return bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + 2 + a); };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full, 1);
+    mbar_init(bar_drain, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar_k_full(s), C::KFP8 ? 128 : 1);
+      mbar_init(bar_k_empty(s), 1);
+    }
+    for (int s = 0; s < C::RSTAGES; ++s) {
+      mbar_init(bar_raw_full(s), 1);
+      mbar_init(bar_raw_empty(s), 128);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_acc_full(a), 1);
+      mbar_init(bar_acc_empty(a), C::EPI_THREADS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == C::PRODUCER_WARP && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+  }
+  // head weights of this block's queries (rows past the block are zero)
+  for (int i = threadIdx.x; i < C::NQ * C::H_I; i += C::NT) {
+    const int qi = i / C::H_I;
+    w_s[i] = qi < nq ? p.w[(q0 + qi) * C::H_I + (i % C::H_I)] : 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int armed_q = 0;
+      mbar_arrive_expect_tx(bar_q_full, C::B_TILE);
+      for (int a = 0; a < C::NATOM; ++a)
+        tma_load_2d(s_q + a * C::N * C::SWB, &tm_q, bar_q_full, a * C::ATOM_ELEMS,
+                    static_cast<int32_t>(q0 * C::H_I));
+      armed_q = 1;
+      int it = 0;
+      for (; it < n_iter; ++it) {
+        const int y = k_base + (t_begin + it) * C::BK;
+        if constexpr (C::KFP8) {
+          const int r = it % C::RSTAGES;
+          if (!mbar_wait(bar_raw_empty(r), ((it / C::RSTAGES) & 1) ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(bar_raw_full(r), C::RAW_TILE);
+          tma_load_2d(s_raw + r * C::RAW_TILE, &tm_k, bar_raw_full(r), 0, y);
+        } else {
+          const int s = it % C::STAGES;
+          if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(bar_k_full(s), C::A_TILE);
+          for (int a = 0; a < C::NATOM; ++a)
+            tma_load_2d(s_k + s * C::A_TILE + a * C::BK * C::SWB, &tm_k, bar_k_full(s),
+                        a * C::ATOM_ELEMS, y);
+        }
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA's memory is released
+        long long t0 = clock64();
+        constexpr int ring = C::KFP8 ? C::RSTAGES : C::STAGES;
+        for (int j = (it > ring ? it - ring : 0); j < it; ++j) {
+          const uint32_t bar = C::KFP8 ? bar_raw_full(j % ring) : bar_k_full(j % ring);
+          while (!mbar_try_wait(bar, (j / ring) & 1) && clock64() - t0 < kWaitLimitCycles) {
+          }
+        }
+        if (armed_q)
+          while (!mbar_try_wait(bar_q_full, 0) && clock64() - t0 < kWaitLimitCycles) {
+          }
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      if (mbar_wait(bar_q_full, 0, abort_flag)) {
+        tc_fence_after();
+        for (int it = 0; it < n_iter; ++it) {
+          const int s = it % C::STAGES;
+          const int a = it & 1;
+          if (!mbar_wait(bar_k_full(s), (it / C::STAGES) & 1, abort_flag)) break;
+          if (!mbar_wait(bar_acc_empty(a), ((it >> 1) & 1) ^ 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t a_base = s_k + s * C::A_TILE;
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const int atom = (kk * 32) / C::SWB;
+            const int off = (kk * 32) % C::SWB;
+            const uint64_t ad = smem_desc(a_base + atom * C::BK * C::SWB + off, 16, 8 * C::SWB, C::SWZ);
+            const uint64_t bd = smem_desc(s_q + atom * C::N * C::SWB + off, 16, 8 * C::SWB, C::SWZ);
+            umma_ss(tmem + a * C::N, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_k_empty(s));
+          umma_commit(bar_acc_full(a));
+        }
+      }
+      // every MMA issued above has completed once this arrives
+      umma_commit(bar_drain);
+      long long t0 = clock64();
+      while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+      }
+    }
+  } else if (C::KFP8 && warp >= C::CONVERT_WARP0) {
+    // ------------------------------------------------------------ e4m3 -> bf16
+    if constexpr (C::KFP8) {
+    const int row = threadIdx.x - C::CONVERT_WARP0 * 32;  // key row of the tile
+    for (int it = 0; it < n_iter; ++it) {
+      const int r = it % C::RSTAGES;
+      const int s = it % C::STAGES;
+      if (!mbar_wait(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag)) break;
+      const uint8_t* raw_row = smem + C::OFF_RAW + r * C::RAW_TILE + row * 128;
+      uint4 chunk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)  // 128-byte swizzle: logical chunk j sits at j ^ (row & 7)
+        chunk[j] = *reinterpret_cast<const uint4*>(raw_row + ((j ^ (row & 7)) << 4));
+      mbar_arrive(bar_raw_empty(r));
+      if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag)) break;
+      uint8_t* dst_tile = smem + C::OFF_K + s * C::A_TILE;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t src[4] = {chunk[j].x, chunk[j].y, chunk[j].z, chunk[j].w};
+        uint32_t outw[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          // 4 e4m3 bytes -> 2 x f16x2 (exact) -> 4 floats -> 2 x bf16x2 (exact)
+          uint32_t h01, h23;
+          asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+              "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+              : "=r"(h01), "=r"(h23)
+              : "r"(src[e]));
+          const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+          const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+          uint32_t b01, b23;
+          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b01) : "f"(f01.y), "f"(f01.x));
+          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b23) : "f"(f23.y), "f"(f23.x));
+          outw[2 * e] = b01;
+          outw[2 * e + 1] = b23;
+        }
+        // 16 bf16 = logical chunks 2j, 2j+1 of the row; 64 elements per atom
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int lc = 2 * j + h;
+          uint8_t* dst = dst_tile + (lc >> 3) * (C::BK * 128) + row * 128 + (((lc & 7) ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(outw[4 * h], outw[4 * h + 1], outw[4 * h + 2], outw[4 * h + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar_k_full(s));
+    }
+    }
+  } else if (warp < C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ epilogue
+    const int g = warp >> 2;        // epilogue warpgroup
+    const int sub = warp & 3;       // TMEM sub-partition = lanes 32*sub ..
+    const int key_in_tile = sub * 32 + lane;
+    for (int it = 0; it < n_iter; ++it) {
+      const int a = it & 1;
+      if (!mbar_wait_warp(bar_acc_full(a), (it >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      float acc[C::QW];
+#pragma unroll
+      for (int q = 0; q < C::QW; ++q) acc[q] = 0.f;
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(sub * 32) << 16) + a * C::N + g * C::COLS_PER_THREAD;
+#pragma unroll
+      for (int c0 = 0; c0 < C::COLS_PER_THREAD; c0 += C::LD_CHUNK) {
+        uint32_t v[32];
+        if (C::LD_CHUNK == 32) tmem_ld32(t_row + c0, v); else tmem_ld16(t_row + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < C::LD_CHUNK; ++j) {
+          const int c = c0 + j;
+          const int q = c / C::H_I;
+          const float wv = w_s[(g * C::QW + q) * C::H_I + (c % C::H_I)];
+          acc[q] = fmaf(wv, fmaxf(__uint_as_float(v[j]), 0.f), acc[q]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_acc_empty(a));
+      const int s = (t_begin + it) * C::BK + key_in_tile;
+      if (s < kv_len) {
+        float kscale = 1.f;
+        if (C::KFP8) kscale = p.k_scale[k_base + s];
+#pragma unroll
+        for (int q = 0; q < C::QW; ++q) {
+          const int qi = g * C::QW + q;
+          if (qi < nq) {
+            const float val = s <= pos0 + qi ? acc[q] * kscale : -INFINITY;
+            p.scores[(q0 + qi - p.q_begin) * p.ld + s] = val;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace dsa

@@ -1,0 +1,417 @@
+// sparse_mla.cuh -- MLA attention in absorbed MQA form over the selected rows.
+//
+// "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse Attention
+// (DSA)", item 2: main MLA attention runs only over the top-k tokens of each
+// query.  "DeepSeek-V3.2 - Experimental Exp Version" (altools), "Technical
+// Principles": MLA with MQA, so one cached entry per token serves every query
+// head; the entry is the compressed latent (512) plus the RoPE key (64)
+// (released config: kv_lora_rank 512, qk_rope_head_dim 64, 128 heads).
+//
+// Per query t: S = q[t] (128 heads x 576) . C_sel^T (576 x k),
+// out = softmax(scale * S) . C_sel[:, :512], lse = log-sum-exp per head.
+//
+// sm_100a mapping.  The 128 heads are the MMA M dimension and the selected
+// rows stream through in tiles of BN = 32, gathered straight from the latent
+// cache by TMA tile::gather4 (four arbitrary rows per instruction).  The fp32
+// output accumulator O[128 x 512] alone fills all 512 columns of an SM's
+// tensor memory, so the released shape runs on a cluster of two CTAs (two
+// SMs): CTA r owns output columns [256 r, 256 r + 256).  QK is split along K
+// the same way -- CTA 0 multiplies latent columns [0, 256), CTA 1 columns
+// [256, 576) -- so each CTA gathers only its own 256 or 320 columns of every
+// selected row and no MMA is duplicated.  The two partial score tiles are
+// exchanged through distributed shared memory (each CTA stores its part into
+// the peer's buffer and signals the peer's mbarrier); both CTAs add them in
+// the same commutative way, so both hold bit-identical scores and take the
+// same softmax decisions.  The online softmax keeps a per-head running max
+// and only rescales O (in TMEM) when the max grows by more than 2^8, which
+// is exact arithmetic with the same final normalisation.
+//
+// Roles per CTA: warps 0-3 softmax + epilogue (one head row per thread),
+// warp 4 gather producer, warp 5 MMA issuer (and TMEM owner).
+#pragma once
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dsa {
+
+template <int H_, int DQK_, int DV_, int SPLIT_>
+struct MlaCfg {
+  static constexpr int H = H_, DQK = DQK_, DV = DV_, SPLIT = SPLIT_;
+  static constexpr int BN = 32;                           // selected rows per tile
+  static constexpr int ATOM = 64;                         // bf16 columns per 128-byte swizzle atom
+  static constexpr int DQK_PAD = (DQK + ATOM - 1) / ATOM * ATOM;
+  static constexpr int NATOM_ALL = DQK_PAD / ATOM;
+  static constexpr int DVS = DV / SPLIT;                  // output columns per CTA
+  static constexpr int NV = DVS / ATOM;                   // value atoms per CTA
+  static constexpr int SPLIT_ATOM = SPLIT == 1 ? NATOM_ALL : DV / (2 * ATOM);
+  static constexpr int NA0 = SPLIT_ATOM;                  // atoms gathered by rank 0
+  static constexpr int NA1 = NATOM_ALL - SPLIT_ATOM;      // atoms gathered by rank 1
+  static constexpr int NA_MAX = NA0 > NA1 ? NA0 : NA1;
+  static constexpr int NS = SPLIT == 1 ? 4 : 5;           // gather ring depth
+  static constexpr int Q_ATOM_BYTES = 128 * 128;          // 128 head rows x 128 bytes
+  static constexpr int C_ATOM_BYTES = BN * 128;
+  static constexpr int C_STAGE = NA_MAX * C_ATOM_BYTES;
+  static constexpr int P_BYTES = 128 * BN * 2;            // one P tile, 64-byte swizzle
+  static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_C = OFF_Q + NA_MAX * Q_ATOM_BYTES;
+  static constexpr int OFF_P = OFF_C + NS * C_STAGE;
+  static constexpr int OFF_X = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_MASK = OFF_X + X_BYTES;
+  static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
+  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int TMEM_S = DVS;                      // S buffers follow O
+  static constexpr int TMEM_COLS = DVS + 2 * BN <= 128 ? 128 : (DVS + 2 * BN <= 256 ? 256 : 512);
+  static constexpr int NT = 6 * 32;
+  static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, BN, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, DVS, false, true);
+  static constexpr float kRescaleThreshold = 8.0f;        // log2 units
+  static_assert(H <= 128, "heads = MMA M rows");
+  static_assert(DV % (SPLIT * ATOM) == 0 && DVS <= 256, "PV N");
+  static_assert(SPLIT == 1 || NV <= NA1, "rank 1 must gather its value columns");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(DVS + 2 * BN <= 512, "tensor memory");
+};
+
+struct MlaParams {
+  const int32_t* idx;        // [q_end - q_begin, topk]
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int B;
+  int64_t q_begin;
+  int topk;
+  float scale_log2;          // softmax scale * log2(e)
+  __nv_bfloat16* out;        // [T, H, DV]
+  float* lse;                // [T, H] or null
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::NT, 1)
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_lat, const MlaParams p) {
+  const uint32_t rank = C::SPLIT == 2 ? cluster_ctarank() : 0u;
+  const uint32_t peer = rank ^ 1u;
+  const int64_t r_local = blockIdx.x / C::SPLIT;          // chunk-relative query row
+  const int64_t t = p.q_begin + r_local;
+  const RowInfo ri = locate_row(p.cu_q, p.cu_k, p.B, t);
+  const int32_t* __restrict__ idx_row = p.idx + r_local * p.topk;
+  const int a0 = rank == 0 ? 0 : C::SPLIT_ATOM;           // first gathered atom (global)
+  const int na = rank == 0 ? C::NA0 : C::NA1;             // atoms gathered by this CTA
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t s_q = sbase + C::OFF_Q;
+  const uint32_t s_c = sbase + C::OFF_C;
+  const uint32_t s_p = sbase + C::OFF_P;
+  float* xbuf = reinterpret_cast<float*>(smem + C::OFF_X);
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const uint32_t bar_q_full = bar0;
+  auto bar_c_full = [&](int s) { return bar0 + 8 * (1 + s); };
+  auto bar_c_empty = [&](int s) { return bar0 + 8 * (1 + C::NS + s); };
+  auto bar_s_full = [&](int a) { return bar0 + 8 * (1 + 2 * C::NS + a); };
+  auto bar_s_free = [&](int a) { return bar0 + 8 * (3 + 2 * C::NS + a); };
+  auto bar_p_full = [&](int a) { return bar0 + 8 * (5 + 2 * C::NS + a); };
+  auto bar_pv_done = [&](int a) { return bar0 + 8 * (7 + 2 * C::NS + a); };
+  const uint32_t bar_x_full = bar0 + 8 * (9 + 2 * C::NS);
+  const uint32_t bar_x_empty = bar0 + 8 * (10 + 2 * C::NS);
+  const uint32_t bar_drain = bar0 + 8 * (11 + 2 * C::NS);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  int* ntiles_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
+  uint32_t* pending_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 12);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar_c_full(s), 1);
+      mbar_init(bar_c_empty(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_s_full(a), 1);
+      mbar_init(bar_s_free(a), 128);
+      mbar_init(bar_p_full(a), 128);
+      mbar_init(bar_pv_done(a), 1);
+    }
+    mbar_init(bar_x_full, 128);
+    mbar_init(bar_x_empty, 128);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    *ntiles_s = 0;
+    // an error recorded earlier by any CTA of this library: skip the work
+    *pending_s = device_error_pending() ? 1u : 0u;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == C::PRODUCER_WARP && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_lat);
+  }
+  __syncthreads();
+  // Tiles up to the last one holding a valid entry (trailing -1 padding is skipped).
+  {
+    int last = -1;
+    for (int e = threadIdx.x; e < p.topk; e += C::NT) {
+      const int s = idx_row[e];
+      if (s >= 0 && s <= ri.pos) last = e;
+    }
+    for (int off = 16; off > 0; off >>= 1) last = max(last, __shfl_xor_sync(0xFFFFFFFFu, last, off));
+    if (lane == 0 && last >= 0) atomicMax(ntiles_s, last / C::BN + 1);
+  }
+  tc_fence_before();
+  if (C::SPLIT == 2) cluster_sync(); else __syncthreads();   // peer barriers initialised
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  // Both CTAs of a cluster take the same skip decision (own flag OR the peer's),
+  // so neither leaves the other waiting at a cluster barrier.
+  bool skip = *pending_s != 0u;
+  if (C::SPLIT == 2) skip = skip || ld_cluster_u32(mapa_shared(smem_u32(pending_s), peer)) != 0u;
+  const int n_tiles = skip ? 0 : *ntiles_s;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ gather producer
+    int it = 0;
+    if (n_tiles > 0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar_q_full, na * C::Q_ATOM_BYTES);
+        for (int a = 0; a < na; ++a)
+          tma_load_2d(s_q + a * C::Q_ATOM_BYTES, &tm_q, bar_q_full, (a0 + a) * C::ATOM,
+                      static_cast<int32_t>(t * C::H));
+      }
+      for (; it < n_tiles; ++it) {
+        const int s = it % C::NS;
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(bar_c_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag);
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        const int e = it * C::BN + lane;
+        const int sel = e < p.topk ? idx_row[e] : -1;
+        const bool valid = sel >= 0 && sel <= ri.pos;
+        const int grow = ri.k_base + (valid ? sel : 0);
+        const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid);
+        int y[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) y[j] = __shfl_sync(0xFFFFFFFFu, grow, (4 * lane + j) & 31);
+        if (lane == 0) {
+          mask_s[s] = vmask;
+          mbar_arrive_expect_tx(bar_c_full(s), na * C::C_ATOM_BYTES);
+        }
+        __syncwarp();
+        if (lane < C::BN / 4) {
+          const uint32_t dst = s_c + s * C::C_STAGE + lane * 4 * 128;
+          for (int a = 0; a < na; ++a)
+            tma_gather4(dst + a * C::C_ATOM_BYTES, &tm_lat, bar_c_full(s), (a0 + a) * C::ATOM, y[0],
+                        y[1], y[2], y[3]);
+        }
+      }
+      if (lane == 0 && *abort_flag) {
+        long long t0 = clock64();
+        for (int j = (it > C::NS ? it - C::NS : 0); j < it; ++j)
+          while (!mbar_try_wait(bar_c_full(j % C::NS), (j / C::NS) & 1) &&
+                 clock64() - t0 < kWaitLimitCycles) {
+          }
+        while (!mbar_try_wait(bar_q_full, 0) && clock64() - t0 < kWaitLimitCycles) {
+        }
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      auto issue_pv = [&](int j) -> bool {
+        const int pb = j & 1;
+        if (!mbar_wait(bar_p_full(pb), (j >> 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t v_base = s_c + (j % C::NS) * C::C_STAGE;
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          const uint64_t ad = smem_desc(s_p + pb * C::P_BYTES + kk * 32, 16, 512, 4);
+          const uint64_t bd = smem_desc(v_base + kk * 16 * 128, C::C_ATOM_BYTES, 1024, 2);
+          umma_ss(tmem, ad, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_c_empty(j % C::NS));
+        umma_commit(bar_pv_done(pb));
+        return true;
+      };
+      bool ok = mbar_wait(bar_q_full, 0, abort_flag);
+      tc_fence_after();
+      const int ksteps = na * (C::ATOM / 16);
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        const int s = it % C::NS;
+        const int sb = it & 1;
+        if (!mbar_wait(bar_c_full(s), (it / C::NS) & 1, abort_flag)) break;
+        if (!mbar_wait(bar_s_free(sb), ((it >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t c_base = s_c + s * C::C_STAGE;
+        for (int kk = 0; kk < ksteps; ++kk) {
+          const int atom = kk >> 2;
+          const int off = (kk & 3) * 32;
+          const uint64_t ad = smem_desc(s_q + atom * C::Q_ATOM_BYTES + off, 16, 1024, 2);
+          const uint64_t bd = smem_desc(c_base + atom * C::C_ATOM_BYTES + off, 16, 1024, 2);
+          umma_ss(tmem + C::TMEM_S + sb * C::BN, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_s_full(sb));
+        if (it > 0 && !issue_pv(it - 1)) { ok = false; break; }
+      }
+      if (ok && !*abort_flag) issue_pv(n_tiles - 1);
+    }
+    if (lane == 0) {
+      umma_commit(bar_drain);
+      long long t0 = clock64();
+      while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int h = warp * 32 + lane;                       // head row = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t x_peer = C::SPLIT == 2 ? mapa_shared(smem_u32(xbuf), peer) : 0u;
+    const uint32_t bar_x_full_peer = C::SPLIT == 2 ? mapa_shared(bar_x_full, peer) : 0u;
+    const uint32_t bar_x_empty_peer = C::SPLIT == 2 ? mapa_shared(bar_x_empty, peer) : 0u;
+    float m_used = -INFINITY;    // running max (log2 units) the exponentials are taken against
+    float l_run = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_tiles; ++it) {
+      const int sb = it & 1;
+      if (!mbar_wait_warp(bar_s_full(sb), (it >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t raw[32];
+      tmem_ld32(tmem + lane_base + C::TMEM_S + sb * C::BN, raw);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar_s_free(sb));
+      float sv[C::BN];
+#pragma unroll
+      for (int j = 0; j < C::BN; ++j) sv[j] = __uint_as_float(raw[j]);
+      if (C::SPLIT == 2) {
+        // push my partial scores into the peer's buffer, row h, 16-byte chunks rotated by h
+        if (!mbar_wait_warp<true>(bar_x_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+        for (int c = 0; c < C::BN / 4; ++c) {
+          const int slot = (c + h) & (C::BN / 4 - 1);
+          st_cluster_v4(x_peer + (h * C::BN + slot * 4) * 4, sv[4 * c], sv[4 * c + 1], sv[4 * c + 2],
+                        sv[4 * c + 3]);
+        }
+        mbar_arrive_remote(bar_x_full_peer);
+        if (!mbar_wait_warp<true>(bar_x_full, it & 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+        for (int c = 0; c < C::BN / 4; ++c) {
+          const int slot = (c + h) & (C::BN / 4 - 1);
+          const float4 v = *reinterpret_cast<const float4*>(xbuf + h * C::BN + slot * 4);
+          sv[4 * c] += v.x;
+          sv[4 * c + 1] += v.y;
+          sv[4 * c + 2] += v.z;
+          sv[4 * c + 3] += v.w;
+        }
+        mbar_arrive_remote(bar_x_empty_peer);
+      }
+      // validity of the tile's entries (written by the producer before it armed c_full)
+      if (!mbar_wait_warp(bar_c_full(it % C::NS), (it / C::NS) & 1, abort_flag)) { ok = false; break; }
+      const uint32_t vmask = mask_s[it % C::NS];
+      float mt = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < C::BN; ++j) {
+        sv[j] = ((vmask >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, sv[j]);
+      }
+      float corr = 1.f;
+      if (mt > m_used + C::kRescaleThreshold) {
+        corr = exp2f(m_used - mt);   // 0 on the first tile with a valid entry
+        m_used = mt;
+      }
+      // P tile of this iteration reuses the buffer of tile it-2: PV(it-2) must be done
+      if (it >= 2 && !mbar_wait_warp(bar_pv_done(sb), ((it - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+      uint32_t pk[C::BN / 2];
+      float psum = 0.f;
+#pragma unroll
+      for (int j = 0; j < C::BN; j += 2) {
+        const float e0 = sv[j] == -INFINITY ? 0.f : exp2f(sv[j] - m_used);
+        const float e1 = sv[j + 1] == -INFINITY ? 0.f : exp2f(sv[j + 1] - m_used);
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
+        const float2 back = __bfloat1622float2(b2);
+        psum += back.x + back.y;
+        pk[j / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      l_run = l_run * corr + psum;
+      if (corr != 1.f && it > 0) {
+        // O must hold every earlier PV before it is rescaled in place
+        if (!mbar_wait_warp(bar_pv_done((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < C::DVS; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(tmem + lane_base + c0, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
+          tmem_st16(tmem + lane_base + c0, o);
+        }
+        tmem_wait_st();
+      }
+      // P row h, K-major with the 64-byte swizzle: 16-byte chunk c sits at c ^ ((h & 7) >> 1)
+      uint8_t* prow = smem + C::OFF_P + sb * C::P_BYTES + (h >> 3) * 512 + (h & 7) * 64;
+#pragma unroll
+      for (int c = 0; c < C::BN / 8; ++c)
+        *reinterpret_cast<uint4*>(prow + ((c ^ ((h & 7) >> 1)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_p_full(sb));
+    }
+    // ------------------------------------------------------------ epilogue
+    const int t_out = static_cast<int>(t);
+    if (ok && n_tiles > 0) {
+      const int j = n_tiles - 1;
+      ok = mbar_wait_warp(bar_pv_done(j & 1), (j >> 1) & 1, abort_flag);
+      tc_fence_after();
+    }
+    if (ok && !skip && h < C::H) {
+      __nv_bfloat16* orow = p.out + (static_cast<int64_t>(t_out) * C::H + h) * C::DV + rank * C::DVS;
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < C::DVS; c0 += 16) {
+        uint32_t o[16];
+        if (n_tiles > 0) {
+          tmem_ld16(tmem + lane_base + c0, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) o[jj] = 0u;
+        }
+        uint32_t pk[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[2 * jj]) * inv_l,
+                                                         __uint_as_float(o[2 * jj + 1]) * inv_l);
+          pk[jj] = *reinterpret_cast<const uint32_t*>(&b2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+      if (rank == 0 && p.lse != nullptr)
+        p.lse[static_cast<int64_t>(t_out) * C::H + h] =
+            l_run > 0.f ? (m_used + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (C::SPLIT == 2) cluster_sync();   // no remote access into this CTA after this point
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace dsa

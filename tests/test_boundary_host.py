@@ -1,0 +1,151 @@
+"""Host-side tests of the C-ABI library: it loads, exports every entry point
+declared in include/dsa.h, and rejects invalid arguments on the host before
+any CUDA call (so these run without a GPU).  Device pointers here are fake,
+aligned addresses: validation never dereferences them."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    from sparse_attention_long_07_b200 import build
+    build.build()
+    import sparse_attention_long_07_b200 as m
+    return m
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward",
+                 "dsa_forward_workspace_size", "dsa_status_string"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(dsa):
+    lib = dsa.library()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    assert dsa.dsa_version().count(".") == 2
+
+
+def test_status_strings(dsa):
+    for s in range(6):
+        assert dsa.dsa_status_string(s) not in ("", "unknown status")
+    assert dsa.dsa_status_string(99) == "unknown status"
+
+
+FAKE = 1 << 20  # an aligned, never-dereferenced "device" address
+
+
+def fake(n=1):
+    return [FAKE * (i + 1) for i in range(n)]
+
+
+def varlen(cu_q, cu_k):
+    from sparse_attention_long_07_b200 import dsa_varlen
+    qh = (ctypes.c_int32 * len(cu_q))(*cu_q)
+    kh = (ctypes.c_int32 * len(cu_k))(*cu_k)
+    v = dsa_varlen(len(cu_q) - 1, FAKE, FAKE, ctypes.cast(qh, ctypes.POINTER(ctypes.c_int32)),
+                   ctypes.cast(kh, ctypes.POINTER(ctypes.c_int32)))
+    v._keep = (qh, kh)
+    return v
+
+
+def scores_call(dsa, v, q_begin=0, q_end=None, ld=None, h=64, d=128, kd=0, ptrs=None, kscale=FAKE):
+    lib = dsa.library()
+    q_end = v.cu_q_host[v.batch] if q_end is None else q_end
+    ld = 1024 if ld is None else ld
+    p = ptrs or fake(4)
+    return lib.dsa_indexer_scores(p[0], p[1], p[2], kscale, kd, v, h, d, q_begin, q_end, p[3], ld, None)
+
+
+def test_indexer_argument_validation(dsa):
+    INV, UNS = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED
+    ok = varlen([0, 3, 5], [0, 10, 300])
+    assert scores_call(dsa, varlen([0, 3, 5], [0, 2, 300])) == INV            # q_len > kv_len
+    assert scores_call(dsa, varlen([1, 3], [0, 10])) == INV                   # cu_q[0] != 0
+    assert scores_call(dsa, varlen([0, 5, 3], [0, 10, 20])) == INV            # decreasing
+    assert scores_call(dsa, ok, q_begin=-1) == INV
+    assert scores_call(dsa, ok, q_begin=4, q_end=3) == INV
+    assert scores_call(dsa, ok, q_end=6) == INV                               # past T
+    assert scores_call(dsa, ok, ld=288) == INV                                # ld < longest kv (290)
+    assert scores_call(dsa, ok, ld=302) == INV                                # ld % 4
+    assert scores_call(dsa, ok, ptrs=[FAKE + 4, FAKE, FAKE, FAKE]) == INV     # misaligned q_idx
+    assert scores_call(dsa, ok, ptrs=[0, FAKE, FAKE, FAKE]) == INV            # null
+    assert scores_call(dsa, ok, kd=1, kscale=None) == INV                     # e4m3 without scales
+    assert scores_call(dsa, ok, kd=7) == INV
+    assert scores_call(dsa, ok, h=32) == UNS
+    assert scores_call(dsa, ok, h=4, d=32, kd=1) == UNS                       # tiny shape is bf16 only
+
+
+def test_topk_and_attention_validation(dsa):
+    lib = dsa.library()
+    INV, UNS = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED
+    v = varlen([0, 4], [0, 100])
+    assert lib.dsa_topk(FAKE, 100, v, 0, 4, 0, FAKE, None) == INV
+    assert lib.dsa_topk(FAKE, 100, v, 0, 4, 2049, FAKE, None) == INV
+    assert lib.dsa_topk(FAKE, 96, v, 0, 4, 16, FAKE, None) == INV
+    assert lib.dsa_topk(0, 100, v, 0, 4, 16, FAKE, None) == INV
+    args = dict(topk=64, h=128, dqk=576, dv=512, scale=0.07)
+
+    def mla(**kw):
+        a = dict(args)
+        a.update(kw)
+        return lib.dsa_sparse_mla_attn(FAKE, FAKE, FAKE, v, 0, 4, a["topk"], a["h"], a["dqk"], a["dv"],
+                                       ctypes.c_float(a["scale"]), FAKE, FAKE, None)
+    assert mla(topk=0) == INV
+    assert mla(scale=0.0) == INV
+    assert mla(scale=float("nan")) == INV
+    assert mla(h=64) == UNS
+    assert mla(dqk=512) == UNS
+
+
+def test_forward_workspace_contract(dsa):
+    lib = dsa.library()
+    v = varlen([0, 3, 5], [0, 10, 301])
+    ld = 292                       # longest kv_len 291, rounded up to a multiple of 4
+    need = lib.dsa_forward_workspace_size(v, 16, 0)
+    al = lambda x: (x + 255) // 256 * 256
+    assert need == al(5 * ld * 4) + al(5 * 16 * 4)
+    assert lib.dsa_forward_workspace_size(v, 16, 2) == al(2 * ld * 4) + al(2 * 16 * 4)
+    assert lib.dsa_forward_workspace_size(v, 0, 0) == 0
+    assert lib.dsa_forward_workspace_size(varlen([0, 3], [0, 2]), 16, 0) == 0
+
+    def fwd(ws, ws_bytes, topk=16, h_i=64, d_i=128):
+        return lib.dsa_forward(FAKE, FAKE, FAKE, None, 0, FAKE, FAKE, v, h_i, d_i, topk, 128, 576, 512,
+                               ctypes.c_float(0.07), 0, FAKE, FAKE, None, ws, ws_bytes, None)
+    assert fwd(None, 0) == dsa.DSA_ERR_WORKSPACE
+    assert fwd(FAKE, need - 1) == dsa.DSA_ERR_WORKSPACE
+    assert fwd(FAKE + 16, need) == dsa.DSA_ERR_INVALID_ARG              # not 256-byte aligned
+    assert fwd(FAKE, need, h_i=8) == dsa.DSA_ERR_UNSUPPORTED
+
+
+def test_injected_faults_are_reported_without_launching(dsa, monkeypatch):
+    lib = dsa.library()
+    v = varlen([0, 3], [0, 10])
+    monkeypatch.setenv("DSA_INJECT_FAULT", "cuda")
+    assert scores_call(dsa, v) == dsa.DSA_ERR_CUDA
+    assert lib.dsa_topk(FAKE, 16, v, 0, 3, 4, FAKE, None) == dsa.DSA_ERR_CUDA
+    monkeypatch.setenv("DSA_INJECT_FAULT", "timeout")
+    assert scores_call(dsa, v) == dsa.DSA_ERR_DEVICE_TIMEOUT
+
+
+def test_binding_raises_on_bad_status(dsa):
+    v = dsa.Varlen([0, 2], [0, 1])     # q_len > kv_len
+    q_idx = torch.zeros(2, 64, 128, dtype=torch.bfloat16)
+    with pytest.raises(dsa.DSAError) as e:
+        dsa.dsa_indexer_scores(q_idx, torch.zeros(2, 64), torch.zeros(1, 128, dtype=torch.bfloat16), None, v, 0,
+                               2, torch.zeros(2, 4), stream=0)
+    assert e.value.status == dsa.DSA_ERR_INVALID_ARG

@@ -1,0 +1,300 @@
+"""GPU parity: every step of the CUDA path, called through the C ABI, against
+the CPU oracle on the same seeded inputs.  Tolerances live in tests/parity.py.
+
+Small cases run the oracle on every row (several tiles and ragged tails);
+the full-size workloads run in the launch configuration the benchmark times
+and compare a seeded sample of rows that the oracle computes one by one."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import dsa_inputs as di
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+RELEASED = dict(H_I=64, d_I=128, topk=2048, H=128, d_qk=576, d_v=512, scale=1.0 / math.sqrt(192.0))
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import sparse_attention_long_07_b200 as m
+    return m
+
+
+def released(name, q_lens, kv_lens, seed, **kw):
+    return di.Spec(name, tuple(q_lens), tuple(kv_lens), seed=seed, **{**RELEASED, **kw})
+
+
+def gpu_scores(dsa, d, v, q_begin, q_end, ld):
+    sc = torch.full((q_end - q_begin, ld), float("nan"), dtype=torch.float32, device="cuda")
+    dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, q_begin, q_end, sc)
+    torch.cuda.synchronize()
+    return sc
+
+
+def ld_for(spec):
+    return (max(spec.kv_lens) + 3) // 4 * 4
+
+
+# ------------------------------------------------------------------ top-k
+
+TOPK_CASES = [
+    # q_lens, kv_lens, k, levels (None = continuous normal scores)
+    ((1,) * 8, (1, 31, 32, 33, 2047, 2048, 2049, 5000), 2048, 3),
+    ((1,) * 4, (3000, 20000, 65, 131072), 2048, None),
+    ((6, 1), (70, 40), 32, 1),
+    ((3,), (9000,), 2048, 0),           # every score equal: the lowest indices win
+]
+
+
+@pytest.mark.parametrize("case", TOPK_CASES, ids=[f"case{i}" for i in range(len(TOPK_CASES))])
+def test_topk_bit_exact_against_oracle(dsa, oracle_lib, case):
+    q_lens, kv_lens, k, levels = case
+    cu_q, cu_k = di.cu_seqlens(q_lens), di.cu_seqlens(kv_lens)
+    T = sum(q_lens)
+    ld = (max(kv_lens) + 3) // 4 * 4
+    g = np.random.default_rng(len(q_lens) * 7 + k)
+    if levels is None:
+        sc = g.standard_normal((T, ld)).astype(np.float32)
+    else:
+        sc = g.integers(-levels, levels + 1, size=(T, ld)).astype(np.float32)
+    sc[g.random(sc.shape) < 0.02] = -0.0
+    pos = P.row_positions(cu_q, cu_k)
+    for r, p_ in enumerate(pos):
+        sc[r, p_ + 1:] = 1e30                        # never read: beyond the diagonal
+    v = dsa.Varlen(cu_q, cu_k, "cuda")
+    sc_gpu = torch.from_numpy(sc).cuda()
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(sc_gpu, v, 0, T, k, idx)
+    idx2 = torch.empty_like(idx)
+    dsa.dsa_topk(sc_gpu, v, 0, T, k, idx2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2), "top-k must be deterministic"
+    o_rows = sc.astype(np.float64)
+    for r, p_ in enumerate(pos):
+        o_rows[r, p_ + 1:] = -np.inf
+    ref = oracle_lib.topk(cu_q, cu_k, o_rows, k)
+    got = idx.cpu().numpy()
+    P.assert_index_sets(got, ref, o_rows, pos, exact=True)
+    # documented order: keys above the threshold, then the tied ones, each in index order
+    for r, p_ in enumerate(pos):
+        n = min(k, p_ + 1)
+        row = got[r, :n]
+        keys = o_rows[r, row]
+        thr = keys.min()
+        above, tied = row[keys > thr], row[keys == thr]
+        assert np.array_equal(row, np.concatenate([above, tied]))
+        assert np.all(np.diff(above) > 0) and np.all(np.diff(tied) > 0)
+        assert np.all(got[r, n:] == -1)
+
+
+def test_topk_on_a_chunk_of_rows(dsa, oracle_lib):
+    q_lens, kv_lens, k = (5, 9), (300, 2600), 64
+    cu_q, cu_k = di.cu_seqlens(q_lens), di.cu_seqlens(kv_lens)
+    ld = 2600
+    g = np.random.default_rng(1)
+    sc = g.standard_normal((14, ld)).astype(np.float32)
+    v = dsa.Varlen(cu_q, cu_k, "cuda")
+    q0, q1 = 3, 11
+    idx = torch.empty((q1 - q0, k), dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(torch.from_numpy(sc[q0:q1]).cuda(), v, q0, q1, k, idx)
+    pos = P.row_positions(cu_q, cu_k)[q0:q1]
+    o = sc[q0:q1].astype(np.float64)
+    ref = oracle_lib.topk(cu_q, cu_k, o, k, rows=list(range(q0, q1)))
+    P.assert_index_sets(idx.cpu().numpy(), ref, o, pos, exact=True)
+
+
+# ------------------------------------------------------------------ indexer
+
+def test_indexer_tiny_integer_scores_are_exact(dsa, oracle_lib):
+    spec = di.config("tiny")
+    d = di.make_inputs(spec)
+    dd = P.to_device(d)
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], "cuda")
+    got = gpu_scores(dsa, dd, v, 0, spec.T, 256).cpu().numpy()
+    ref = oracle_lib.indexer_scores(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"])
+    pos = P.row_positions(d["cu_q"], d["cu_k"])
+    P.assert_scores_close(got, ref, pos, exact=True)
+    for r, p_ in enumerate(pos):           # -inf after the diagonal inside its 128-key tile
+        end = min((p_ // 128 + 1) * 128, 256)
+        assert np.all(np.isneginf(got[r, p_ + 1:end]))
+
+
+@pytest.mark.parametrize("kfp8,q_lens,kv_lens", [
+    (False, (5, 130, 1, 7), (5, 700, 333, 2000)),
+    (False, (64,), (64,)),
+    (True, (1, 1, 1, 1, 2), (1, 129, 1000, 4097, 300)),
+    (True, (37, 3), (600, 128)),
+], ids=["bf16-ragged", "bf16-square", "e4m3-decode", "e4m3-prefill"])
+def test_indexer_released_shape(dsa, oracle_lib, kfp8, q_lens, kv_lens):
+    spec = released("idx", q_lens, kv_lens, seed=5, kfp8=kfp8)
+    d = di.make_inputs(spec)
+    dd = P.to_device(d)
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], "cuda")
+    ld = ld_for(spec)
+    got = gpu_scores(dsa, dd, v, 0, spec.T, ld).cpu().numpy()
+    ref = oracle_lib.indexer_scores(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"], d["k_scale"], ld=ld)
+    pos = P.row_positions(d["cu_q"], d["cu_k"])
+    P.assert_scores_close(got, ref, pos)
+    # a sub-range of rows (chunk-relative output) gives the same values
+    q0, q1 = spec.T // 3, spec.T
+    part = gpu_scores(dsa, dd, v, q0, q1, ld).cpu().numpy()
+    for r in range(q1 - q0):
+        p_ = pos[q0 + r]
+        assert np.array_equal(part[r, : p_ + 1], got[q0 + r, : p_ + 1])
+
+
+# ------------------------------------------------------------------ sparse MLA
+
+def _attention_case(dsa, oracle_lib, spec, idx=None):
+    d = di.make_inputs(spec)
+    dd = P.to_device(d)
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], "cuda")
+    if idx is None:
+        sc = oracle_lib.indexer_scores(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"], d["k_scale"])
+        idx = oracle_lib.topk(d["cu_q"], d["cu_k"], sc, spec.topk)
+    out = torch.full((spec.T, spec.H, spec.d_v), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((spec.T, spec.H), float("nan"), dtype=torch.float32, device="cuda")
+    dsa.dsa_sparse_mla_attn(dd["q"], dd["latent"], torch.from_numpy(np.ascontiguousarray(idx)).cuda(), v, 0,
+                            spec.T, spec.softmax_scale, out, lse)
+    torch.cuda.synchronize()
+    o_out, o_lse = oracle_lib.sparse_mla(d["cu_q"], d["cu_k"], d["q"], d["latent"], idx, spec.softmax_scale,
+                                         spec.d_v)
+    return out.float().cpu().numpy(), lse.cpu().numpy(), o_out, o_lse
+
+
+def test_sparse_mla_tiny(dsa, oracle_lib):
+    g_out, g_lse, o_out, o_lse = _attention_case(dsa, oracle_lib, di.config("tiny"))
+    P.assert_attention_close(g_out, g_lse, o_out, o_lse, "tiny")
+
+
+def test_sparse_mla_released_shape(dsa, oracle_lib):
+    spec = released("mla", (3, 2, 1), (3000, 70, 2500), seed=6)
+    g_out, g_lse, o_out, o_lse = _attention_case(dsa, oracle_lib, spec)
+    P.assert_attention_close(g_out, g_lse, o_out, o_lse, "released")
+
+
+def test_sparse_mla_ignores_invalid_entries_and_empty_rows(dsa, oracle_lib):
+    spec = released("mla-edge", (4,), (300,), seed=7, topk=128)
+    g = np.random.default_rng(2)
+    idx = np.full((4, 128), -1, np.int32)
+    idx[0, :50] = g.permutation(297)[:50]
+    idx[0, 50:55] = [298, 299, 5000, -7, 297]      # 298, 299 beyond pos 297; 5000 beyond the cache
+    idx[1, 60:70] = np.arange(10)                  # valid entries only in the second tile
+    idx[3, :] = g.permutation(300)[:128]
+    # row 2 keeps no valid entry
+    g_out, g_lse, o_out, o_lse = _attention_case(dsa, oracle_lib, spec, idx=idx)
+    P.assert_attention_close(g_out, g_lse, o_out, o_lse, "edges")
+    assert np.all(g_out[2] == 0) and np.all(np.isneginf(g_lse[2]))
+
+
+# ------------------------------------------------------------------ fused forward
+
+def _forward(dsa, dd, spec, v, q_chunk=0):
+    ws = torch.empty(dsa.dsa_forward_workspace_size(v, spec.topk, q_chunk), dtype=torch.uint8, device="cuda")
+    out = torch.full((spec.T, spec.H, spec.d_v), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((spec.T, spec.H), float("nan"), dtype=torch.float32, device="cuda")
+    idx = torch.full((spec.T, spec.topk), -2, dtype=torch.int32, device="cuda")
+    dsa.dsa_forward(dd["q_idx"], dd["w"], dd["k_idx"], dd["k_scale"], dd["q"], dd["latent"], v, spec.topk,
+                    spec.softmax_scale, out, lse, ws, idx_out=idx, q_chunk=q_chunk)
+    torch.cuda.synchronize()
+    return out, lse, idx
+
+
+def test_forward_tiny_end_to_end_bit_exact_sets(dsa, oracle_lib):
+    spec = di.config("tiny")
+    d = di.make_inputs(spec)
+    dd = P.to_device(d)
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], "cuda")
+    out, lse, idx = _forward(dsa, dd, spec, v)
+    sc, o_idx, o_out, o_lse = oracle_lib.forward(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"], None,
+                                                 d["q"], d["latent"], spec.topk, spec.softmax_scale, spec.d_v)
+    pos = P.row_positions(d["cu_q"], d["cu_k"])
+    P.assert_index_sets(idx.cpu().numpy(), o_idx, sc, pos, exact=True)
+    P.assert_attention_close(out.float().cpu().numpy(), lse.cpu().numpy(), o_out, o_lse, "tiny e2e")
+    assert dsa.dsa_device_error() == 0
+
+
+def test_forward_chunking_does_not_change_results(dsa):
+    spec = released("chunk", (70, 9), (400, 3000), seed=8)
+    d = di.make_inputs(spec)
+    dd = P.to_device(d)
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], "cuda")
+    a = _forward(dsa, dd, spec, v, q_chunk=0)
+    b = _forward(dsa, dd, spec, v, q_chunk=17)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def _check_sampled(dsa, oracle_lib, spec, dd, cu_q, cu_k, out, lse, idx, rows):
+    """Oracle on sampled rows of a (possibly huge) GPU-resident workload."""
+    cu_q_l, cu_k_l = list(map(int, cu_q)), list(map(int, cu_k))
+    by_seq = {}
+    for t in rows:
+        b = max(i for i in range(len(cu_q_l) - 1) if cu_q_l[i] <= t < cu_q_l[i + 1])
+        by_seq.setdefault(b, []).append(t)
+    for b, ts in by_seq.items():
+        q0, q1, k0, k1 = cu_q_l[b], cu_q_l[b + 1], cu_k_l[b], cu_k_l[b + 1]
+        scq, sck = [0, q1 - q0], [0, k1 - k0]
+        sub = {n: dd[n][q0:q1].cpu() for n in ("q_idx", "w", "q")}
+        sub["k_idx"] = dd["k_idx"][k0:k1].cpu()
+        sub["k_scale"] = None if dd["k_scale"] is None else dd["k_scale"][k0:k1].cpu()
+        sub["latent"] = dd["latent"][k0:k1].cpu()
+        local = [t - q0 for t in ts]
+        sc = oracle_lib.indexer_scores(scq, sck, sub["q_idx"], sub["w"], sub["k_idx"], sub["k_scale"], rows=local)
+        o_idx = oracle_lib.topk(scq, sck, sc, spec.topk, rows=local)
+        pos = [(k1 - k0) - (q1 - q0) + i for i in local]
+        g_idx = idx[ts].cpu().numpy()
+        P.assert_index_sets(g_idx, o_idx, sc, pos)
+        g_out = out[ts].float().cpu().numpy()
+        g_lse = lse[ts].cpu().numpy()
+        # attention on the GPU's own selection isolates the attention kernel ...
+        a_out, a_lse = oracle_lib.sparse_mla(scq, sck, sub["q"], sub["latent"], g_idx, spec.softmax_scale,
+                                             spec.d_v, rows=local)
+        P.assert_attention_close(g_out, g_lse, a_out, a_lse, f"seq {b} (gpu idx)")
+        # ... and on the oracle's selection it is the end-to-end check
+        e_out, e_lse = oracle_lib.sparse_mla(scq, sck, sub["q"], sub["latent"], o_idx, spec.softmax_scale,
+                                             spec.d_v, rows=local)
+        P.assert_attention_close(g_out, g_lse, e_out, e_lse, f"seq {b} (oracle idx)")
+
+
+def _full_size(dsa, oracle_lib, name, n_per_seq, q_chunk=0, max_seqs=None):
+    spec = di.config(name)
+    dd = di.make_inputs(spec, device="cuda")
+    v = dsa.Varlen(dd["cu_q"], dd["cu_k"], "cuda")
+    out, lse, idx = _forward(dsa, dd, spec, v, q_chunk=q_chunk)
+    assert dsa.dsa_device_error() == 0
+    rows = P.sample_rows(dd["cu_q"], n_per_seq, seed=spec.seed)
+    if max_seqs is not None:
+        g = np.random.default_rng(spec.seed)
+        keep = set(int(b) for b in g.choice(spec.B, size=max_seqs, replace=False))
+        cu_q_l = list(map(int, dd["cu_q"]))
+        rows = [t for t in rows if any(cu_q_l[b] <= t < cu_q_l[b + 1] for b in keep)]
+    _check_sampled(dsa, oracle_lib, spec, dd, dd["cu_q"], dd["cu_k"], out, lse, idx, rows)
+    del dd, out, lse, idx
+    torch.cuda.empty_cache()
+
+
+def test_full_prefill4k(dsa, oracle_lib):
+    _full_size(dsa, oracle_lib, "prefill4k", n_per_seq=24)
+
+
+def test_full_decode128k(dsa, oracle_lib):
+    _full_size(dsa, oracle_lib, "decode128k", n_per_seq=1, max_seqs=8)
+
+
+def test_full_ragged128k(dsa, oracle_lib):
+    _full_size(dsa, oracle_lib, "ragged128k", n_per_seq=3)
+
+
+def test_full_prefill32k(dsa, oracle_lib):
+    _full_size(dsa, oracle_lib, "prefill32k", n_per_seq=8, q_chunk=8192)
+
+
+def test_full_prefill64k(dsa, oracle_lib):
+    _full_size(dsa, oracle_lib, "prefill64k", n_per_seq=8, q_chunk=8192)
