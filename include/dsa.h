@@ -105,9 +105,10 @@ dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_i
  * scores    fp32 [q_end - q_begin, ld_scores] chunk-relative, as written by
  *           dsa_indexer_scores (only columns 0..pos(t) are read)
  * idx       int32 [q_end - q_begin, topk] chunk-relative.  Row r holds the
- *           min(topk, pos+1) selected sequence-local key indices -- first those
- *           with a score above the k-th largest, in increasing index order, then
- *           those equal to it, in increasing index order -- followed by -1.
+ *           min(topk, pos+1) selected sequence-local key indices followed by
+ *           -1.  With pos+1 <= topk that is 0..pos; otherwise first the keys
+ *           scoring above the k-th largest score, in increasing index order,
+ *           then those equal to it, in increasing index order.
  *           The SET is the definition; the order is fixed only so that
  *           repeated runs are bit-identical.
  * topk in [1, 2048].  Scores must not be NaN.

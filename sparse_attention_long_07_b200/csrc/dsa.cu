@@ -180,11 +180,13 @@ dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, con
                       const Layout& L, int64_t q_begin, int64_t q_end, int topk, float scale,
                       void* out, float* lse, cudaStream_t stream) {
   CUtensorMap tm_q, tm_lat;
+  const CUtensorMapSwizzle swz = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : (C::SWB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
   if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, C::DQK, static_cast<uint64_t>(L.T) * C::H,
-                C::DQK * 2, C::ATOM, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+                C::DQK * 2, C::ATOM, 128, swz))
     return DSA_ERR_CUDA;
   if (!make_map(&tm_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, latent, C::DQK, static_cast<uint64_t>(L.S),
-                C::DQK * 2, C::ATOM, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+                C::DQK * 2, C::ATOM, 1, swz))
     return DSA_ERR_CUDA;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -282,10 +284,10 @@ dsa_status run_mla(const void* q, const void* latent, const int32_t* idx, const 
                    const Layout& L, int64_t q_begin, int64_t q_end, int topk, int h, int dqk, int dv,
                    float scale, void* out, float* lse, cudaStream_t stream) {
   if (is_tiny_mla(h, dqk, dv))
-    return launch_mla<MlaCfg<4, 80, 64, 1>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, out,
-                                            lse, stream);
-  return launch_mla<MlaCfg<128, 576, 512, 2>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, out,
-                                              lse, stream);
+    return launch_mla<MlaCfg<4, 80, 64, 1, 32>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, out,
+                                                lse, stream);
+  return launch_mla<MlaCfg<128, 576, 512, 2, 128>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, out,
+                                                   lse, stream);
 }
 
 constexpr size_t kWsAlign = 256;

@@ -183,12 +183,12 @@ __global__ void __launch_bounds__(C::NT, 1)
         const int y = k_base + (t_begin + it) * C::BK;
         if constexpr (C::KFP8) {
           const int r = it % C::RSTAGES;
-          if (!mbar_wait(bar_raw_empty(r), ((it / C::RSTAGES) & 1) ^ 1, abort_flag)) break;
+          if (!mbar_wait(bar_raw_empty(r), ((it / C::RSTAGES) & 1) ^ 1, abort_flag, 11)) break;
           mbar_arrive_expect_tx(bar_raw_full(r), C::RAW_TILE);
           tma_load_2d(s_raw + r * C::RAW_TILE, &tm_k, bar_raw_full(r), 0, y);
         } else {
           const int s = it % C::STAGES;
-          if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag)) break;
+          if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, 12)) break;
           mbar_arrive_expect_tx(bar_k_full(s), C::A_TILE);
           for (int a = 0; a < C::NATOM; ++a)
             tma_load_2d(s_k + s * C::A_TILE + a * C::BK * C::SWB, &tm_k, bar_k_full(s),
@@ -212,13 +212,13 @@ __global__ void __launch_bounds__(C::NT, 1)
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      if (mbar_wait(bar_q_full, 0, abort_flag)) {
+      if (mbar_wait(bar_q_full, 0, abort_flag, 13)) {
         tc_fence_after();
         for (int it = 0; it < n_iter; ++it) {
           const int s = it % C::STAGES;
           const int a = it & 1;
-          if (!mbar_wait(bar_k_full(s), (it / C::STAGES) & 1, abort_flag)) break;
-          if (!mbar_wait(bar_acc_empty(a), ((it >> 1) & 1) ^ 1, abort_flag)) break;
+          if (!mbar_wait(bar_k_full(s), (it / C::STAGES) & 1, abort_flag, 14)) break;
+          if (!mbar_wait(bar_acc_empty(a), ((it >> 1) & 1) ^ 1, abort_flag, 15)) break;
           tc_fence_after();
           const uint32_t a_base = s_k + s * C::A_TILE;
 #pragma unroll
@@ -246,14 +246,14 @@ __global__ void __launch_bounds__(C::NT, 1)
     for (int it = 0; it < n_iter; ++it) {
       const int r = it % C::RSTAGES;
       const int s = it % C::STAGES;
-      if (!mbar_wait(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag)) break;
+      if (!mbar_wait(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag, 16)) break;
       const uint8_t* raw_row = smem + C::OFF_RAW + r * C::RAW_TILE + row * 128;
       uint4 chunk[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)  // 128-byte swizzle: logical chunk j sits at j ^ (row & 7)
         chunk[j] = *reinterpret_cast<const uint4*>(raw_row + ((j ^ (row & 7)) << 4));
       mbar_arrive(bar_raw_empty(r));
-      if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag)) break;
+      if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, 17)) break;
       uint8_t* dst_tile = smem + C::OFF_K + s * C::A_TILE;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     const int key_in_tile = sub * 32 + lane;
     for (int it = 0; it < n_iter; ++it) {
       const int a = it & 1;
-      if (!mbar_wait_warp(bar_acc_full(a), (it >> 1) & 1, abort_flag)) break;
+      if (!mbar_wait_warp(bar_acc_full(a), (it >> 1) & 1, abort_flag, 18)) break;
       tc_fence_after();
       float acc[C::QW];
 #pragma unroll

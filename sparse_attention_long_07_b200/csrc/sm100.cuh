@@ -16,7 +16,7 @@ namespace dsa {
 __device__ int g_device_error;
 
 enum DeviceErrorCode : int {
-  kErrWaitTimeout = 1,      // an mbarrier wait exceeded its limit
+  kErrWaitTimeout = 1,      // an mbarrier wait exceeded its limit; bits 8.. hold the wait site
 };
 
 // ~2 s at the 1.9 GHz boost clock: far above any legitimate wait in these kernels.
@@ -106,7 +106,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // wait itself exceeds kWaitLimitCycles, in which case it records the error and
 // raises the flag.  Every role polls the same flag, so a CTA always drains.
 template <bool kClusterScope = false>
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int site = 0) {
   long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
     bool ok = kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
@@ -117,7 +118,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       if (t0 == 0) {
         t0 = now;
       } else if (now - t0 > kWaitLimitCycles) {
-        record_device_error(kErrWaitTimeout);
+        record_device_error(kErrWaitTimeout | (site << 8));
         *abort_flag = 1;
         return false;
       }
@@ -128,8 +129,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // Warp-uniform form: every lane waits, and the warp agrees on the outcome, so
 // that .sync.aligned instructions after it are reached by the whole warp.
 template <bool kClusterScope = false>
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = mbar_wait<kClusterScope>(bar, parity, abort_flag);
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               int site = 0) {
+  const bool ok = mbar_wait<kClusterScope>(bar, parity, abort_flag, site);
   return __all_sync(0xFFFFFFFFu, ok) != 0;
 }
 

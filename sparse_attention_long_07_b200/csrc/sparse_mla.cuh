@@ -12,7 +12,9 @@
 //
 // sm_100a mapping.  The 128 heads are the MMA M dimension and the selected
 // rows stream through in tiles of BN = 32, gathered straight from the latent
-// cache by TMA tile::gather4 (four arbitrary rows per instruction).  The fp32
+// cache by TMA tile::gather4 (four arbitrary rows per instruction) into
+// swizzled K-major atoms (128-byte atoms for the released shape; narrower atoms
+// for narrow test shapes, so that every TMA box lies inside the row).  The fp32
 // output accumulator O[128 x 512] alone fills all 512 columns of an SM's
 // tensor memory, so the released shape runs on a cluster of two CTAs (two
 // SMs): CTA r owns output columns [256 r, 256 r + 256).  QK is split along K
@@ -35,22 +37,24 @@
 
 namespace dsa {
 
-template <int H_, int DQK_, int DV_, int SPLIT_>
+template <int H_, int DQK_, int DV_, int SPLIT_, int SWB_>
 struct MlaCfg {
   static constexpr int H = H_, DQK = DQK_, DV = DV_, SPLIT = SPLIT_;
+  static constexpr int SWB = SWB_;                        // swizzle-atom row bytes (128, 64 or 32)
+  static constexpr uint32_t SWZ = SWB == 128 ? 2u : (SWB == 64 ? 4u : 6u);
   static constexpr int BN = 32;                           // selected rows per tile
-  static constexpr int ATOM = 64;                         // bf16 columns per 128-byte swizzle atom
-  static constexpr int DQK_PAD = (DQK + ATOM - 1) / ATOM * ATOM;
-  static constexpr int NATOM_ALL = DQK_PAD / ATOM;
+  static constexpr int ATOM = SWB / 2;                    // bf16 columns per swizzle atom
+  static constexpr int KPA = SWB / 32;                    // 16-wide k-steps per atom
+  static constexpr int NATOM_ALL = DQK / ATOM;
   static constexpr int DVS = DV / SPLIT;                  // output columns per CTA
   static constexpr int NV = DVS / ATOM;                   // value atoms per CTA
-  static constexpr int SPLIT_ATOM = SPLIT == 1 ? NATOM_ALL : DV / (2 * ATOM);
+  static constexpr int SPLIT_ATOM = SPLIT == 1 ? NATOM_ALL : DVS / ATOM;
   static constexpr int NA0 = SPLIT_ATOM;                  // atoms gathered by rank 0
   static constexpr int NA1 = NATOM_ALL - SPLIT_ATOM;      // atoms gathered by rank 1
   static constexpr int NA_MAX = NA0 > NA1 ? NA0 : NA1;
   static constexpr int NS = SPLIT == 1 ? 4 : 5;           // gather ring depth
-  static constexpr int Q_ATOM_BYTES = 128 * 128;          // 128 head rows x 128 bytes
-  static constexpr int C_ATOM_BYTES = BN * 128;
+  static constexpr int Q_ATOM_BYTES = 128 * SWB;          // 128 head rows
+  static constexpr int C_ATOM_BYTES = BN * SWB;
   static constexpr int C_STAGE = NA_MAX * C_ATOM_BYTES;
   static constexpr int P_BYTES = 128 * BN * 2;            // one P tile, 64-byte swizzle
   static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;
@@ -71,7 +75,8 @@ struct MlaCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, DVS, false, true);
   static constexpr float kRescaleThreshold = 8.0f;        // log2 units
   static_assert(H <= 128, "heads = MMA M rows");
-  static_assert(DV % (SPLIT * ATOM) == 0 && DVS <= 256, "PV N");
+  static_assert(DQK % ATOM == 0, "every TMA box stays inside the row: no partial atoms");
+  static_assert(DVS % ATOM == 0 && DVS <= 256 && DVS % 16 == 0, "PV N");
   static_assert(SPLIT == 1 || NV <= NA1, "rank 1 must gather its value columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(DVS + 2 * BN <= 512, "tensor memory");
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       for (; it < n_tiles; ++it) {
         const int s = it % C::NS;
         int ok = 1;
-        if (lane == 0) ok = mbar_wait(bar_c_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag);
+        if (lane == 0) ok = mbar_wait(bar_c_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, 21);
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) break;
         const int e = it * C::BN + lane;
@@ -209,7 +214,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
         __syncwarp();
         if (lane < C::BN / 4) {
-          const uint32_t dst = s_c + s * C::C_STAGE + lane * 4 * 128;
+          const uint32_t dst = s_c + s * C::C_STAGE + lane * 4 * C::SWB;
           for (int a = 0; a < na; ++a)
             tma_gather4(dst + a * C::C_ATOM_BYTES, &tm_lat, bar_c_full(s), (a0 + a) * C::ATOM, y[0],
                         y[1], y[2], y[3]);
@@ -230,34 +235,34 @@ __global__ void __launch_bounds__(C::NT, 1)
     if (lane == 0 && n_tiles > 0) {
       auto issue_pv = [&](int j) -> bool {
         const int pb = j & 1;
-        if (!mbar_wait(bar_p_full(pb), (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar_p_full(pb), (j >> 1) & 1, abort_flag, 22)) return false;
         tc_fence_after();
         const uint32_t v_base = s_c + (j % C::NS) * C::C_STAGE;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           const uint64_t ad = smem_desc(s_p + pb * C::P_BYTES + kk * 32, 16, 512, 4);
-          const uint64_t bd = smem_desc(v_base + kk * 16 * 128, C::C_ATOM_BYTES, 1024, 2);
+          const uint64_t bd = smem_desc(v_base + kk * 16 * C::SWB, C::C_ATOM_BYTES, 8 * C::SWB, C::SWZ);
           umma_ss(tmem, ad, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar_c_empty(j % C::NS));
         umma_commit(bar_pv_done(pb));
         return true;
       };
-      bool ok = mbar_wait(bar_q_full, 0, abort_flag);
+      bool ok = mbar_wait(bar_q_full, 0, abort_flag, 23);
       tc_fence_after();
-      const int ksteps = na * (C::ATOM / 16);
+      const int ksteps = na * C::KPA;
       for (int it = 0; ok && it < n_tiles; ++it) {
         const int s = it % C::NS;
         const int sb = it & 1;
-        if (!mbar_wait(bar_c_full(s), (it / C::NS) & 1, abort_flag)) break;
-        if (!mbar_wait(bar_s_free(sb), ((it >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(bar_c_full(s), (it / C::NS) & 1, abort_flag, 24)) break;
+        if (!mbar_wait(bar_s_free(sb), ((it >> 1) & 1) ^ 1, abort_flag, 25)) break;
         tc_fence_after();
         const uint32_t c_base = s_c + s * C::C_STAGE;
         for (int kk = 0; kk < ksteps; ++kk) {
-          const int atom = kk >> 2;
-          const int off = (kk & 3) * 32;
-          const uint64_t ad = smem_desc(s_q + atom * C::Q_ATOM_BYTES + off, 16, 1024, 2);
-          const uint64_t bd = smem_desc(c_base + atom * C::C_ATOM_BYTES + off, 16, 1024, 2);
+          const int atom = kk / C::KPA;
+          const int off = (kk % C::KPA) * 32;
+          const uint64_t ad = smem_desc(s_q + atom * C::Q_ATOM_BYTES + off, 16, 8 * C::SWB, C::SWZ);
+          const uint64_t bd = smem_desc(c_base + atom * C::C_ATOM_BYTES + off, 16, 8 * C::SWB, C::SWZ);
           umma_ss(tmem + C::TMEM_S + sb * C::BN, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_s_full(sb));
@@ -283,7 +288,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     bool ok = true;
     for (int it = 0; it < n_tiles; ++it) {
       const int sb = it & 1;
-      if (!mbar_wait_warp(bar_s_full(sb), (it >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(bar_s_full(sb), (it >> 1) & 1, abort_flag, 26)) { ok = false; break; }
       tc_fence_after();
       uint32_t raw[32];
       tmem_ld32(tmem + lane_base + C::TMEM_S + sb * C::BN, raw);
@@ -295,7 +300,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       for (int j = 0; j < C::BN; ++j) sv[j] = __uint_as_float(raw[j]);
       if (C::SPLIT == 2) {
         // push my partial scores into the peer's buffer, row h, 16-byte chunks rotated by h
-        if (!mbar_wait_warp<true>(bar_x_empty, (it & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp<true>(bar_x_empty, (it & 1) ^ 1, abort_flag, 27)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < C::BN / 4; ++c) {
           const int slot = (c + h) & (C::BN / 4 - 1);
@@ -303,7 +308,7 @@ __global__ void __launch_bounds__(C::NT, 1)
                         sv[4 * c + 3]);
         }
         mbar_arrive_remote(bar_x_full_peer);
-        if (!mbar_wait_warp<true>(bar_x_full, it & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp<true>(bar_x_full, it & 1, abort_flag, 28)) { ok = false; break; }
 #pragma unroll
         for (int c = 0; c < C::BN / 4; ++c) {
           const int slot = (c + h) & (C::BN / 4 - 1);
@@ -316,7 +321,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         mbar_arrive_remote(bar_x_empty_peer);
       }
       // validity of the tile's entries (written by the producer before it armed c_full)
-      if (!mbar_wait_warp(bar_c_full(it % C::NS), (it / C::NS) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(bar_c_full(it % C::NS), (it / C::NS) & 1, abort_flag, 29)) { ok = false; break; }
       const uint32_t vmask = mask_s[it % C::NS];
       float mt = -INFINITY;
 #pragma unroll
@@ -330,7 +335,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         m_used = mt;
       }
       // P tile of this iteration reuses the buffer of tile it-2: PV(it-2) must be done
-      if (it >= 2 && !mbar_wait_warp(bar_pv_done(sb), ((it - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (it >= 2 && !mbar_wait_warp(bar_pv_done(sb), ((it - 2) >> 1) & 1, abort_flag, 30)) { ok = false; break; }
       uint32_t pk[C::BN / 2];
       float psum = 0.f;
 #pragma unroll
@@ -343,9 +348,12 @@ __global__ void __launch_bounds__(C::NT, 1)
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&b2);
       }
       l_run = l_run * corr + psum;
-      if (corr != 1.f && it > 0) {
+      // The rescale decision is per head row, but the TMEM accesses below are
+      // warp-collective (.sync.aligned): the warp rescales if any lane needs
+      // it, and lanes that do not multiply by 1.
+      if (__any_sync(0xFFFFFFFFu, corr != 1.f && it > 0)) {
         // O must hold every earlier PV before it is rescaled in place
-        if (!mbar_wait_warp(bar_pv_done((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(bar_pv_done((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, 31)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
         for (int c0 = 0; c0 < C::DVS; c0 += 16) {
@@ -372,11 +380,13 @@ __global__ void __launch_bounds__(C::NT, 1)
     const int t_out = static_cast<int>(t);
     if (ok && n_tiles > 0) {
       const int j = n_tiles - 1;
-      ok = mbar_wait_warp(bar_pv_done(j & 1), (j >> 1) & 1, abort_flag);
+      ok = mbar_wait_warp(bar_pv_done(j & 1), (j >> 1) & 1, abort_flag, 32);
       tc_fence_after();
     }
-    if (ok && !skip && h < C::H) {
-      __nv_bfloat16* orow = p.out + (static_cast<int64_t>(t_out) * C::H + h) * C::DV + rank * C::DVS;
+    // every lane takes part in the warp-collective TMEM loads; only rows h < H are stored
+    if (ok && !skip) {
+      const bool store = h < C::H;
+      __nv_bfloat16* orow = p.out + (static_cast<int64_t>(t_out) * C::H + (store ? h : 0)) * C::DV + rank * C::DVS;
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
       for (int c0 = 0; c0 < C::DVS; c0 += 16) {
@@ -395,11 +405,13 @@ __global__ void __launch_bounds__(C::NT, 1)
                                                          __uint_as_float(o[2 * jj + 1]) * inv_l);
           pk[jj] = *reinterpret_cast<const uint32_t*>(&b2);
         }
-        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        if (store) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
       }
-      if (rank == 0 && p.lse != nullptr)
+      if (store && rank == 0 && p.lse != nullptr)
         p.lse[static_cast<int64_t>(t_out) * C::H + h] =
             l_run > 0.f ? (m_used + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }

@@ -85,6 +85,9 @@ def test_topk_bit_exact_against_oracle(dsa, oracle_lib, case):
     for r, p_ in enumerate(pos):
         n = min(k, p_ + 1)
         row = got[r, :n]
+        if p_ + 1 <= k:                      # every candidate kept, in index order
+            assert np.array_equal(row, np.arange(n)) and np.all(got[r, n:] == -1)
+            continue
         keys = o_rows[r, row]
         thr = keys.min()
         above, tied = row[keys > thr], row[keys == thr]
@@ -163,6 +166,8 @@ def _attention_case(dsa, oracle_lib, spec, idx=None):
     dsa.dsa_sparse_mla_attn(dd["q"], dd["latent"], torch.from_numpy(np.ascontiguousarray(idx)).cuda(), v, 0,
                             spec.T, spec.softmax_scale, out, lse)
     torch.cuda.synchronize()
+    code = dsa.dsa_device_error()
+    assert code == 0, f"device error word {code:#x} (a bounded wait gave up at site {code >> 8})"
     o_out, o_lse = oracle_lib.sparse_mla(d["cu_q"], d["cu_k"], d["q"], d["latent"], idx, spec.softmax_scale,
                                          spec.d_v)
     return out.float().cpu().numpy(), lse.cpu().numpy(), o_out, o_lse
@@ -203,6 +208,8 @@ def _forward(dsa, dd, spec, v, q_chunk=0):
     dsa.dsa_forward(dd["q_idx"], dd["w"], dd["k_idx"], dd["k_scale"], dd["q"], dd["latent"], v, spec.topk,
                     spec.softmax_scale, out, lse, ws, idx_out=idx, q_chunk=q_chunk)
     torch.cuda.synchronize()
+    code = dsa.dsa_device_error()
+    assert code == 0, f"device error word {code:#x} (a bounded wait gave up at site {code >> 8})"
     return out, lse, idx
 
 
