@@ -106,11 +106,9 @@ dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_i
  *           dsa_indexer_scores (only columns 0..pos(t) are read)
  * idx       int32 [q_end - q_begin, topk] chunk-relative.  Row r holds the
  *           min(topk, pos+1) selected sequence-local key indices followed by
- *           -1.  With pos+1 <= topk that is 0..pos; otherwise first the keys
- *           scoring above the k-th largest score, in increasing index order,
- *           then those equal to it, in increasing index order.
- *           The SET is the definition; the order is fixed only so that
- *           repeated runs are bit-identical.
+ *           -1.  With pos+1 <= topk that is 0..pos.  The SET is the
+ *           definition; the order within a row is unspecified but
+ *           deterministic, so repeated runs are bit-identical.
  * topk in [1, 2048].  Scores must not be NaN.
  */
 dsa_status dsa_topk(const float* scores, int64_t ld_scores, dsa_varlen v, int64_t q_begin,
@@ -169,6 +167,15 @@ dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
 /* Reads and clears the device error word of the current device (synchronises
  * `stream` first).  *code = 0 when no device-side wait gave up. */
 dsa_status dsa_device_error(int32_t* code, cudaStream_t stream);
+
+/* Diagnostics for profiling builds (compiled with -DDSA_PROFILE_WAITS): for
+ * each bounded-wait site (index = the site code recorded on a timeout), the
+ * device cycles lane 0 of the waiting warps spent in completed waits and how
+ * many such waits there were.  Synchronises the device; copies min(n, 64)
+ * entries into the host arrays; reset != 0 clears the counters.  Regular
+ * builds return DSA_ERR_UNSUPPORTED and touch nothing.  No counterpart on the
+ * pages: it exists to attribute kernel time to pipeline stages. */
+dsa_status dsa_debug_wait_profile(uint64_t* cycles, uint64_t* counts, int32_t n, int32_t reset);
 
 /* Static description of a status code. */
 const char* dsa_status_string(dsa_status status);

@@ -44,8 +44,12 @@ class dsa_varlen(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m sparse_attention_long_07_b200.build`")
+            f"{LIB_PATH} is missing: build it with `python sparse_attention_long_07_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
+    for name in EXPORTED:
+        if not hasattr(lib, name):
+            raise ImportError(f"{LIB_PATH} predates the binding (no symbol {name}): rebuild it with "
+                              "`python sparse_attention_long_07_b200/build.py --force`")
     vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
     lib.dsa_indexer_scores.argtypes = [vp, vp, vp, vp, ctypes.c_int, dsa_varlen, i32, i32, i64, i64, vp, i64, vp]
     lib.dsa_topk.argtypes = [vp, i64, dsa_varlen, i64, i64, i32, vp, vp]
@@ -58,15 +62,18 @@ def _load():
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_version.restype = ctypes.c_char_p
+    lib.dsa_debug_wait_profile.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
+                                           ctypes.c_int32, ctypes.c_int32]
+    lib.dsa_debug_wait_profile.restype = ctypes.c_int
     for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward", "dsa_device_error"):
         getattr(lib, fn).restype = ctypes.c_int
     return lib
 
 
-_lib = _load()
-
 EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward_workspace_size",
-            "dsa_forward", "dsa_device_error", "dsa_status_string", "dsa_version")
+            "dsa_forward", "dsa_device_error", "dsa_status_string", "dsa_version", "dsa_debug_wait_profile")
+
+_lib = _load()
 
 
 def library():
@@ -182,3 +189,15 @@ def dsa_device_error(stream=None) -> int:
     if st not in (DSA_OK, DSA_ERR_DEVICE_TIMEOUT):
         raise DSAError(st, "dsa_device_error")
     return int(code.value)
+
+
+def dsa_debug_wait_profile(reset: bool = True):
+    """Per wait site (cycles, completed waits) from a profiling build, or None."""
+    n = 64
+    cyc = (ctypes.c_uint64 * n)()
+    cnt = (ctypes.c_uint64 * n)()
+    st = _lib.dsa_debug_wait_profile(cyc, cnt, n, 1 if reset else 0)
+    if st == DSA_ERR_UNSUPPORTED:
+        return None
+    _check(st, "dsa_debug_wait_profile")
+    return {i: (int(cyc[i]), int(cnt[i])) for i in range(n) if cnt[i]}

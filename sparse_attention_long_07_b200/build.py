@@ -1,6 +1,9 @@
 """Build libdsa.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m sparse_attention_long_07_b200.build [--force]
+    python sparse_attention_long_07_b200/build.py [--force] [--profile-waits]
+
+Run it by path (or load it with load_builder()): importing the package itself
+loads the library, which is what this script produces.
 """
 from __future__ import annotations
 
@@ -32,11 +35,14 @@ def stale() -> bool:
     return any(os.path.getmtime(p) > t for p in DEPS if os.path.exists(p))
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, profile_waits: bool = False) -> str:
+    """Compile libdsa.so.  profile_waits=True adds the per-wait-site cycle
+    counters read by dsa_debug_wait_profile (a diagnostic build, not for timing)."""
     if not force and not stale():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *FLAGS, "-I", INCLUDE, "-I", CSRC, *SOURCES, "-o", tmp, "-ldl", "-lrt", "-lpthread"]
+    extra = ["-DDSA_PROFILE_WAITS"] if profile_waits else []
+    cmd = [NVCC, *FLAGS, *extra, "-I", INCLUDE, "-I", CSRC, *SOURCES, "-o", tmp, "-ldl", "-lrt", "-lpthread"]
     res = subprocess.run(cmd, capture_output=True, text=True)
     log = os.path.join(HERE, "build.log")
     with open(log, "w") as f:
@@ -51,4 +57,5 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv or "--profile-waits" in sys.argv, verbose=True,
+                profile_waits="--profile-waits" in sys.argv))

@@ -175,6 +175,63 @@ dsa_status launch_indexer(const void* q_idx, const float* w, const void* k_idx,
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
+int num_sms() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n = 0;
+  });
+  return n;
+}
+
+// Decode-like calls: one persistent CTA per SM over the flat (sequence, key tile) list.
+template <class C>
+dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const void* k_idx,
+                                     const float* k_scale, const dsa_varlen& v, const Layout& L,
+                                     int64_t q_begin, int64_t q_end, float* scores, int64_t ld,
+                                     cudaStream_t stream) {
+  int64_t units = 0;
+  for (int b = 0; b < v.batch; ++b) {
+    const int64_t lo = std::max<int64_t>(v.cu_q_host[b], q_begin);
+    const int64_t hi = std::min<int64_t>(v.cu_q_host[b + 1], q_end);
+    if (lo >= hi) continue;
+    const int kv = v.cu_k_host[b + 1] - v.cu_k_host[b];
+    const int ql = v.cu_q_host[b + 1] - v.cu_q_host[b];
+    units += (kv - ql + static_cast<int>(lo - v.cu_q_host[b])) / C::BK + 1;
+  }
+  const int sms = num_sms();
+  if (units == 0) return DSA_OK;
+  if (sms <= 0) return DSA_ERR_CUDA;
+  CUtensorMap tm_q, tm_k;
+  if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q_idx, C::D_I, static_cast<uint64_t>(L.T) * C::H_I,
+                C::D_I * 2, C::ATOM_ELEMS, C::N, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_idx, C::D_I, static_cast<uint64_t>(L.S), C::D_I, C::D_I,
+                C::BK, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] { attr_err = set_smem(dsa::indexer_persistent_kernel<C>, C::SMEM_BYTES); });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  dsa::IndexerParams p;
+  p.w = w;
+  p.k_scale = k_scale;
+  p.cu_q = v.cu_q;
+  p.cu_k = v.cu_k;
+  p.B = v.batch;
+  p.q_begin = q_begin;
+  p.q_end = q_end;
+  p.scores = scores;
+  p.ld = ld;
+  p.chunk_tiles = 0;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, sms));
+  dsa::indexer_persistent_kernel<C><<<grid, C::NT, C::SMEM_BYTES, stream>>>(tm_q, tm_k, p);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
 template <class C>
 dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, const dsa_varlen& v,
                       const Layout& L, int64_t q_begin, int64_t q_end, int topk, float scale,
@@ -257,6 +314,10 @@ dsa_status run_indexer(const void* q_idx, const float* w, const void* k_idx, con
     return launch_indexer<IndexerCfg<4, 32, 4, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
                                                         scores, ld, stream);
   if (kd == DSA_KIDX_FP8_E4M3) {
+    using Persist = IndexerCfg<64, 128, 1, true, true>;
+    if (L.max_q_rows <= 1 && v.batch <= Persist::MAX_SEQ)
+      return launch_indexer_persistent<Persist>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end, scores, ld,
+                                                stream);
     if (decode_like)
       return launch_indexer<IndexerCfg<64, 128, 1, true>>(q_idx, w, k_idx, k_scale, v, L, q_begin,
                                                            q_end, scores, ld, stream);
@@ -270,12 +331,17 @@ dsa_status run_indexer(const void* q_idx, const float* w, const void* k_idx, con
                                                         scores, ld, stream);
 }
 
-dsa_status run_topk(const float* scores, int64_t ld, const dsa_varlen& v, int64_t q_begin,
-                    int64_t q_end, int topk, int32_t* idx, cudaStream_t stream) {
+dsa_status run_topk(const float* scores, int64_t ld, const dsa_varlen& v, const Layout& L,
+                    int64_t q_begin, int64_t q_end, int topk, int32_t* idx, cudaStream_t stream) {
   const int64_t rows = q_end - q_begin;
   if (rows == 0) return DSA_OK;
   if (rows > 0x7FFFFFFF) return DSA_ERR_UNSUPPORTED;
-  dsa::topk_radix_kernel<512><<<static_cast<unsigned>(rows), 512, 0, stream>>>(
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] { attr_err = set_smem(dsa::topk_kernel, dsa::TopkCfg::SMEM_BYTES); });
+  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  if (L.max_kv > dsa::TopkCfg::MAX_N) return DSA_ERR_UNSUPPORTED;   // 16-bit pass-1 counters
+  dsa::topk_kernel<<<static_cast<unsigned>(rows), dsa::TopkCfg::NT, dsa::TopkCfg::SMEM_BYTES, stream>>>(
       scores, ld, v.cu_q, v.cu_k, v.batch, q_begin, topk, idx);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
@@ -323,7 +389,7 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, dsa_varlen v, int64_
     return DSA_ERR_INVALID_ARG;
   if (topk < 1 || topk > 2048 || ld_scores < L.max_kv || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
   if ((st = injected_fault()) != DSA_OK) return st;
-  return run_topk(scores, ld_scores, v, q_begin, q_end, topk, idx, stream);
+  return run_topk(scores, ld_scores, v, L, q_begin, q_end, topk, idx, stream);
 }
 
 dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t* idx,
@@ -388,7 +454,7 @@ dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
     if ((st = run_indexer(q_idx, w, k_idx, k_scale, k_dtype, v, L, n_idx_heads, idx_dim, q0, q1, scores,
                           ld, stream)) != DSA_OK)
       return st;
-    if ((st = run_topk(scores, ld, v, q0, q1, topk, idx, stream)) != DSA_OK) return st;
+    if ((st = run_topk(scores, ld, v, L, q0, q1, topk, idx, stream)) != DSA_OK) return st;
     if ((st = run_mla(q, latent, idx, v, L, q0, q1, topk, n_heads, d_qk, d_v, scale, out, lse,
                       stream)) != DSA_OK)
       return st;
@@ -404,6 +470,30 @@ dsa_status dsa_device_error(int32_t* code, cudaStream_t stream) {
   if (cudaMemcpyToSymbol(dsa::g_device_error, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
   *code = v;
   return v == 0 ? DSA_OK : DSA_ERR_DEVICE_TIMEOUT;
+}
+
+dsa_status dsa_debug_wait_profile(uint64_t* cycles, uint64_t* counts, int32_t n, int32_t reset) {
+#ifdef DSA_PROFILE_WAITS
+  if (!cycles || !counts || n < 1) return DSA_ERR_INVALID_ARG;
+  const int m = n < dsa::kWaitSites ? n : dsa::kWaitSites;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(cycles, dsa::g_wait_cycles, m * sizeof(uint64_t)) != cudaSuccess ||
+      cudaMemcpyFromSymbol(counts, dsa::g_wait_count, m * sizeof(uint64_t)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (reset) {
+    static const unsigned long long zeros[dsa::kWaitSites] = {};
+    if (cudaMemcpyToSymbol(dsa::g_wait_cycles, zeros, sizeof(zeros)) != cudaSuccess ||
+        cudaMemcpyToSymbol(dsa::g_wait_count, zeros, sizeof(zeros)) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+  return DSA_OK;
+#else
+  (void)cycles;
+  (void)counts;
+  (void)n;
+  (void)reset;
+  return DSA_ERR_UNSUPPORTED;
+#endif
 }
 
 const char* dsa_status_string(dsa_status s) {

@@ -32,10 +32,12 @@ __host__ __device__ constexpr int pow2_at_least(int v, int lo) {
   return p;
 }
 
-template <int H_I_, int D_I_, int NQ_, bool KFP8_>
+template <int H_I_, int D_I_, int NQ_, bool KFP8_, bool PERSIST_ = false>
 struct IndexerCfg {
   static constexpr int H_I = H_I_, D_I = D_I_, NQ = NQ_;
   static constexpr bool KFP8 = KFP8_;
+  static constexpr bool PERSIST = PERSIST_;                 // one CTA per SM over a flat unit list
+  static constexpr int MAX_SEQ = 2048;                    // persistent: sequences per call
   static constexpr int BK = 128;                          // keys per tile (MMA M)
   static constexpr int N = NQ * H_I;                      // MMA N
   static constexpr int ROWB = D_I * 2;                    // bytes of one bf16 row
@@ -45,7 +47,7 @@ struct IndexerCfg {
   static constexpr int ATOM_ELEMS = SWB / 2;
   static constexpr int KSTEPS = D_I / 16;
   static constexpr int STAGES = KFP8 ? 2 : 4;             // bf16 key-tile ring
-  static constexpr int RSTAGES = KFP8 ? 4 : 0;            // raw e4m3 ring
+  static constexpr int RSTAGES = KFP8 ? (PERSIST ? 6 : 4) : 0;   // raw e4m3 ring
   static constexpr int A_TILE = BK * ROWB;
   static constexpr int B_TILE = N * ROWB;
   static constexpr int RAW_TILE = BK * D_I;
@@ -67,14 +69,54 @@ struct IndexerCfg {
   static constexpr int OFF_RAW = OFF_K + STAGES * A_TILE;
   static constexpr int OFF_W = OFF_RAW + RSTAGES * RAW_TILE;
   static constexpr int OFF_BAR = OFF_W + NQ * H_I * 4;
-  static constexpr int NBAR = 2 + 2 * STAGES + 2 * RSTAGES + 4;
+  static constexpr int NBAR = 2 + 2 * STAGES + 2 * RSTAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
+  static constexpr int OFF_UPRE = OFF_MISC + 16;          // persistent: unit prefix per sequence
+  static constexpr int SMEM_BYTES = OFF_UPRE + (PERSIST ? (MAX_SEQ + 1) * 4 : 0) + 1024;  // + alignment slack
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
   static_assert(B_TILE % 1024 == 0 && A_TILE % 1024 == 0, "atom alignment");
   static_assert(COLS_PER_THREAD % LD_CHUNK == 0, "TMEM load chunking");
   static_assert(!KFP8 || D_I == 128, "e4m3 keys: 128-byte rows");
+  static_assert(!PERSIST || NQ == 1, "persistent schedule: one query per sequence block");
 };
+
+// One key row of a raw e4m3 tile (128 bytes, 128-byte TMA swizzle) -> the
+// same row of the bf16 UMMA tile (two 128-byte swizzle atoms).  Exact: every
+// e4m3 value is a bf16 value (e4m3 -> f16x2 -> f32 -> bf16x2, all exact).
+template <int BK>
+__device__ __forceinline__ void e4m3_row_to_bf16(const uint8_t* raw_row, uint8_t* dst_tile, int row) {
+  uint4 chunk[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)  // 128-byte swizzle: logical chunk j sits at j ^ (row & 7)
+    chunk[j] = *reinterpret_cast<const uint4*>(raw_row + ((j ^ (row & 7)) << 4));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t src[4] = {chunk[j].x, chunk[j].y, chunk[j].z, chunk[j].w};
+    uint32_t outw[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t h01, h23;
+      asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+          "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+          : "=r"(h01), "=r"(h23)
+          : "r"(src[e]));
+      const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+      const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+      uint32_t b01, b23;
+      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b01) : "f"(f01.y), "f"(f01.x));
+      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b23) : "f"(f23.y), "f"(f23.x));
+      outw[2 * e] = b01;
+      outw[2 * e + 1] = b23;
+    }
+    // 16 bf16 = logical chunks 2j, 2j+1 of the row; 64 elements per atom
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int lc = 2 * j + h;
+      uint8_t* dst = dst_tile + (lc >> 3) * (BK * 128) + row * 128 + (((lc & 7) ^ (row & 7)) << 4);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(outw[4 * h], outw[4 * h + 1], outw[4 * h + 2], outw[4 * h + 3]);
+    }
+  }
+}
 
 struct IndexerParams {
   const float* w;            // [T, H_I]
@@ -248,41 +290,10 @@ __global__ void __launch_bounds__(C::NT, 1)
       const int s = it % C::STAGES;
       if (!mbar_wait(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag, 16)) break;
       const uint8_t* raw_row = smem + C::OFF_RAW + r * C::RAW_TILE + row * 128;
-      uint4 chunk[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j)  // 128-byte swizzle: logical chunk j sits at j ^ (row & 7)
-        chunk[j] = *reinterpret_cast<const uint4*>(raw_row + ((j ^ (row & 7)) << 4));
-      mbar_arrive(bar_raw_empty(r));
+      // the raw stage is read into registers inside the conversion; release it after
       if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, 17)) break;
-      uint8_t* dst_tile = smem + C::OFF_K + s * C::A_TILE;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t src[4] = {chunk[j].x, chunk[j].y, chunk[j].z, chunk[j].w};
-        uint32_t outw[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          // 4 e4m3 bytes -> 2 x f16x2 (exact) -> 4 floats -> 2 x bf16x2 (exact)
-          uint32_t h01, h23;
-          asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-              "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
-              : "=r"(h01), "=r"(h23)
-              : "r"(src[e]));
-          const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-          const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-          uint32_t b01, b23;
-          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b01) : "f"(f01.y), "f"(f01.x));
-          asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b23) : "f"(f23.y), "f"(f23.x));
-          outw[2 * e] = b01;
-          outw[2 * e + 1] = b23;
-        }
-        // 16 bf16 = logical chunks 2j, 2j+1 of the row; 64 elements per atom
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int lc = 2 * j + h;
-          uint8_t* dst = dst_tile + (lc >> 3) * (C::BK * 128) + row * 128 + (((lc & 7) ^ (row & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(outw[4 * h], outw[4 * h + 1], outw[4 * h + 2], outw[4 * h + 3]);
-        }
-      }
+      e4m3_row_to_bf16<C::BK>(raw_row, smem + C::OFF_K + s * C::A_TILE, row);
+      mbar_arrive(bar_raw_empty(r));
       fence_proxy_async_smem();
       mbar_arrive(bar_k_full(s));
     }
@@ -327,6 +338,262 @@ __global__ void __launch_bounds__(C::NT, 1)
             p.scores[(q0 + qi - p.q_begin) * p.ld + s] = val;
           }
         }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Persistent schedule for decode-like calls (at most one query row per
+// sequence in the call).  The work units are the (sequence, 128-key tile)
+// pairs of the call, flattened in sequence order; CTA c of G (G = number of
+// SMs) takes units [c U / G, (c+1) U / G), so every SM streams the same
+// number of key tiles.  Consecutive units of one sequence share its query tile,
+// which is reloaded only when the sequence changes.
+template <class C>
+__global__ void __launch_bounds__(C::NT, 1)
+    indexer_persistent_kernel(const __grid_constant__ CUtensorMap tm_q,
+                              const __grid_constant__ CUtensorMap tm_k, const IndexerParams p) {
+  static_assert(C::PERSIST && C::KFP8 && C::NQ == 1, "persistent path: e4m3 keys, one query per block");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int* upre = reinterpret_cast<int*>(smem + C::OFF_UPRE);      // upre[b] = first unit of sequence b
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (device_error_pending()) return;
+
+  // ---------------------------------------------------------------- unit list
+  for (int b = threadIdx.x; b < p.B; b += C::NT) {
+    const int cq0 = p.cu_q[b], cq1 = p.cu_q[b + 1];
+    const int64_t lo = cq0 > p.q_begin ? cq0 : p.q_begin;
+    const int64_t hi = cq1 < p.q_end ? cq1 : p.q_end;
+    int cnt = 0;
+    if (lo < hi) {
+      const int kv = p.cu_k[b + 1] - p.cu_k[b];
+      const int pos = kv - (cq1 - cq0) + static_cast<int>(lo - cq0);
+      cnt = pos / C::BK + 1;
+    }
+    upre[b + 1] = cnt;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    upre[0] = 0;
+    for (int b = 0; b < p.B; ++b) upre[b + 1] += upre[b];
+  }
+  __syncthreads();
+  const int64_t U = upre[p.B];
+  const int u0 = static_cast<int>(U * blockIdx.x / gridDim.x);
+  const int u1 = static_cast<int>(U * (blockIdx.x + 1) / gridDim.x);
+  if (u0 >= u1) return;
+  const int n_iter = u1 - u0;
+  int b_first = 0;
+  {
+    int lo = 0, hi = p.B - 1;     // largest b with upre[b] <= u0
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (upre[mid] <= u0) lo = mid; else hi = mid - 1;
+    }
+    b_first = lo;
+  }
+  // per-sequence facts of unit u (walks b forward as u increases)
+  struct Seq {
+    int b, q0, pos, k_base, kv_len;
+  };
+  auto seq_of = [&](int b) {
+    Seq q;
+    q.b = b;
+    const int cq0 = p.cu_q[b], cq1 = p.cu_q[b + 1];
+    q.q0 = static_cast<int>(cq0 > p.q_begin ? cq0 : p.q_begin);
+    q.k_base = p.cu_k[b];
+    q.kv_len = p.cu_k[b + 1] - q.k_base;
+    q.pos = q.kv_len - (cq1 - cq0) + (q.q0 - cq0);
+    return q;
+  };
+
+  // ---------------------------------------------------------------- shared memory
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t s_q = sbase + C::OFF_Q;
+  const uint32_t s_raw = sbase + C::OFF_RAW;
+  const uint32_t s_k = sbase + C::OFF_K;
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  const uint32_t bar_q_full = bar0;
+  const uint32_t bar_drain = bar0 + 8;
+  auto bar_k_full = [&](int s) { return bar0 + 16 + 8 * s; };
+  auto bar_k_empty = [&](int s) { return bar0 + 16 + 8 * (C::STAGES + s); };
+  auto bar_raw_full = [&](int s) { return bar0 + 16 + 8 * (2 * C::STAGES + s); };
+  auto bar_raw_empty = [&](int s) { return bar0 + 16 + 8 * (2 * C::STAGES + C::RSTAGES + s); };
+  auto bar_acc_full = [&](int a) { return bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + a); };
+  auto bar_acc_empty = [&](int a) { return bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + 2 + a); };
+  const uint32_t bar_q_empty = bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full, 1);
+    mbar_init(bar_q_empty, 1);
+    mbar_init(bar_drain, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar_k_full(s), 128);
+      mbar_init(bar_k_empty(s), 1);
+    }
+    for (int s = 0; s < C::RSTAGES; ++s) {
+      mbar_init(bar_raw_full(s), 1);
+      mbar_init(bar_raw_empty(s), 128);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_acc_full(a), 1);
+      mbar_init(bar_acc_empty(a), C::EPI_THREADS);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == C::PRODUCER_WARP && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int b = b_first, seg = -1, armed_q = 0, it = 0;
+      Seq q{};
+      for (; it < n_iter; ++it) {
+        const int u = u0 + it;
+        while (u >= upre[b + 1]) ++b;
+        if (b != q.b || seg < 0) {
+          ++seg;
+          if (seg > 0 && !mbar_wait(bar_q_empty, (seg - 1) & 1, abort_flag, 50)) break;
+          q = seq_of(b);
+          mbar_arrive_expect_tx(bar_q_full, C::B_TILE);
+          for (int at = 0; at < C::NATOM; ++at)
+            tma_load_2d(s_q + at * C::N * C::SWB, &tm_q, bar_q_full, at * C::ATOM_ELEMS, q.q0 * C::H_I);
+          armed_q = seg + 1;
+        }
+        const int tile = u - upre[b];
+        const int r = it % C::RSTAGES;
+        if (!mbar_wait(bar_raw_empty(r), ((it / C::RSTAGES) & 1) ^ 1, abort_flag, 51)) break;
+        mbar_arrive_expect_tx(bar_raw_full(r), C::RAW_TILE);
+        tma_load_2d(s_raw + r * C::RAW_TILE, &tm_k, bar_raw_full(r), 0, q.k_base + tile * C::BK);
+      }
+      if (*abort_flag) {
+        long long t0 = clock64();
+        for (int j = (it > C::RSTAGES ? it - C::RSTAGES : 0); j < it; ++j)
+          while (!mbar_try_wait(bar_raw_full(j % C::RSTAGES), (j / C::RSTAGES) & 1) &&
+                 clock64() - t0 < kWaitLimitCycles) {
+          }
+        if (armed_q)
+          while (!mbar_try_wait(bar_q_full, (armed_q - 1) & 1) && clock64() - t0 < kWaitLimitCycles) {
+          }
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int b = b_first, seg = -1, cur = -1;
+      for (int it = 0; it < n_iter; ++it) {
+        const int u = u0 + it;
+        while (u >= upre[b + 1]) ++b;
+        if (b != cur) {
+          ++seg;
+          cur = b;
+          if (!mbar_wait(bar_q_full, seg & 1, abort_flag, 52)) break;
+          tc_fence_after();
+        }
+        const int s = it % C::STAGES;
+        const int a = it & 1;
+        if (!mbar_wait(bar_k_full(s), (it / C::STAGES) & 1, abort_flag, 53)) break;
+        if (!mbar_wait(bar_acc_empty(a), ((it >> 1) & 1) ^ 1, abort_flag, 54)) break;
+        tc_fence_after();
+        const uint32_t a_base = s_k + s * C::A_TILE;
+#pragma unroll
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          const int atom = (kk * 32) / C::SWB;
+          const int off = (kk * 32) % C::SWB;
+          const uint64_t ad = smem_desc(a_base + atom * C::BK * C::SWB + off, 16, 8 * C::SWB, C::SWZ);
+          const uint64_t bd = smem_desc(s_q + atom * C::N * C::SWB + off, 16, 8 * C::SWB, C::SWZ);
+          umma_ss(tmem + a * C::N, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_k_empty(s));
+        umma_commit(bar_acc_full(a));
+        if (u + 1 == u1 || u + 1 >= upre[b + 1]) umma_commit(bar_q_empty);   // last tile of the sequence
+      }
+      umma_commit(bar_drain);
+      long long t0 = clock64();
+      while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < kWaitLimitCycles) {
+      }
+    }
+  } else if (warp >= C::CONVERT_WARP0) {
+    // ------------------------------------------------------------ e4m3 -> bf16
+    const int row = threadIdx.x - C::CONVERT_WARP0 * 32;
+    for (int it = 0; it < n_iter; ++it) {
+      const int r = it % C::RSTAGES;
+      const int s = it % C::STAGES;
+      if (!mbar_wait(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag, 55)) break;
+      if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, 56)) break;
+      e4m3_row_to_bf16<C::BK>(smem + C::OFF_RAW + r * C::RAW_TILE + row * 128, smem + C::OFF_K + s * C::A_TILE,
+                              row);
+      mbar_arrive(bar_raw_empty(r));
+      fence_proxy_async_smem();
+      mbar_arrive(bar_k_full(s));
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (one warpgroup)
+    const int sub = warp & 3;
+    const int key_in_tile = sub * 32 + lane;
+    int b = b_first, cur = -1;
+    Seq q{};
+    float wreg[C::H_I];
+    for (int it = 0; it < n_iter; ++it) {
+      const int u = u0 + it;
+      while (u >= upre[b + 1]) ++b;
+      if (b != cur) {
+        cur = b;
+        q = seq_of(b);
+        const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(q.q0) * C::H_I);
+#pragma unroll
+        for (int j = 0; j < C::H_I / 4; ++j) {
+          const float4 v = w4[j];
+          wreg[4 * j] = v.x;
+          wreg[4 * j + 1] = v.y;
+          wreg[4 * j + 2] = v.z;
+          wreg[4 * j + 3] = v.w;
+        }
+      }
+      const int a = it & 1;
+      if (!mbar_wait_warp(bar_acc_full(a), (it >> 1) & 1, abort_flag, 57)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(sub * 32) << 16) + a * C::N;
+      uint32_t v0[32], v1[32];
+      tmem_ld32(t_row, v0);
+      tmem_ld32(t_row + 32, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar_acc_empty(a));
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        acc0 = fmaf(wreg[j], fmaxf(__uint_as_float(v0[j]), 0.f), acc0);
+        acc1 = fmaf(wreg[32 + j], fmaxf(__uint_as_float(v1[j]), 0.f), acc1);
+      }
+      const int tile = u - upre[b];
+      const int s_key = tile * C::BK + key_in_tile;
+      if (s_key < q.kv_len) {
+        const float val = s_key <= q.pos ? (acc0 + acc1) * p.k_scale[q.k_base + s_key] : -INFINITY;
+        p.scores[(static_cast<int64_t>(q.q0) - p.q_begin) * p.ld + s_key] = val;
       }
     }
   }

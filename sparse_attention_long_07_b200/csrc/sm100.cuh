@@ -19,6 +19,13 @@ enum DeviceErrorCode : int {
   kErrWaitTimeout = 1,      // an mbarrier wait exceeded its limit; bits 8.. hold the wait site
 };
 
+#ifdef DSA_PROFILE_WAITS
+// Profiling builds only: cycles spent and waits completed per wait site.
+constexpr int kWaitSites = 64;
+__device__ unsigned long long g_wait_cycles[kWaitSites];
+__device__ unsigned long long g_wait_count[kWaitSites];
+#endif
+
 // ~2 s at the 1.9 GHz boost clock: far above any legitimate wait in these kernels.
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
@@ -109,9 +116,20 @@ template <bool kClusterScope = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           int site = 0) {
   long long t0 = 0;
+#ifdef DSA_PROFILE_WAITS
+  const long long t_enter = clock64();
+#endif
   for (uint32_t it = 0;; ++it) {
     bool ok = kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
-    if (ok) return true;
+    if (ok) {
+#ifdef DSA_PROFILE_WAITS
+      if ((threadIdx.x & 31) == 0 && site > 0 && site < kWaitSites) {
+        atomicAdd(&g_wait_cycles[site], static_cast<unsigned long long>(clock64() - t_enter));
+        atomicAdd(&g_wait_count[site], 1ull);
+      }
+#endif
+      return true;
+    }
     if ((it & 63u) == 63u) {
       if (*abort_flag) return false;
       long long now = clock64();
@@ -180,6 +198,15 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Contiguous bulk copy global -> this CTA's shared memory (both addresses and
+// the size multiples of 16 bytes), completing transaction bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // tcgen05: tensor memory, MMA, commit, loads/stores
 // ----------------------------------------------------------------------------
@@ -236,6 +263,18 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T (A: 128 lanes x K, two 16-bit elements per
+// 32-bit column), issued by one thread.
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -307,6 +346,17 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float a, fl
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a),
                "f"(b), "f"(c), "f"(d)
                : "memory");
+}
+
+// Asynchronous store into another CTA's shared memory that completes 16
+// transaction bytes on that CTA's mbarrier (no fence needed on this side).
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, float b, float c, float d,
+                                            uint32_t cluster_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+          cluster_addr),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
+      : "memory");
 }
 
 __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {

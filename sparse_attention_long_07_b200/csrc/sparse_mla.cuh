@@ -56,19 +56,20 @@ struct MlaCfg {
   static constexpr int Q_ATOM_BYTES = 128 * SWB;          // 128 head rows
   static constexpr int C_ATOM_BYTES = BN * SWB;
   static constexpr int C_STAGE = NA_MAX * C_ATOM_BYTES;
-  static constexpr int P_BYTES = 128 * BN * 2;            // one P tile, 64-byte swizzle
-  static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;
+  static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;   // one partial-score buffer
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_C = OFF_Q + NA_MAX * Q_ATOM_BYTES;
-  static constexpr int OFF_P = OFF_C + NS * C_STAGE;
-  static constexpr int OFF_X = OFF_P + 2 * P_BYTES;
-  static constexpr int OFF_MASK = OFF_X + X_BYTES;
+  static constexpr int OFF_X = OFF_C + NS * C_STAGE;      // two partial-score buffers
+  static constexpr int OFF_MASK = OFF_X + 2 * X_BYTES;
   static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
-  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 2 + 2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr int TMEM_S = DVS;                      // S buffers follow O
-  static constexpr int TMEM_COLS = DVS + 2 * BN <= 128 ? 128 : (DVS + 2 * BN <= 256 ? 256 : 512);
+  // tensor memory columns: O [0, DVS), S[2] (fp32, BN each), P[2] (bf16 pairs, BN/2 each)
+  static constexpr int TMEM_S = DVS;
+  static constexpr int TMEM_P = DVS + 2 * BN;
+  static constexpr int TMEM_USED = TMEM_P + BN;
+  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static constexpr int NT = 6 * 32;
   static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, BN, false, false);
@@ -79,7 +80,7 @@ struct MlaCfg {
   static_assert(DVS % ATOM == 0 && DVS <= 256 && DVS % 16 == 0, "PV N");
   static_assert(SPLIT == 1 || NV <= NA1, "rank 1 must gather its value columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
-  static_assert(DVS + 2 * BN <= 512, "tensor memory");
+  static_assert(TMEM_USED <= 512, "tensor memory");
 };
 
 struct MlaParams {
@@ -112,7 +113,6 @@ __global__ void __launch_bounds__(C::NT, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t s_q = sbase + C::OFF_Q;
   const uint32_t s_c = sbase + C::OFF_C;
-  const uint32_t s_p = sbase + C::OFF_P;
   float* xbuf = reinterpret_cast<float*>(smem + C::OFF_X);
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
   const uint32_t bar0 = sbase + C::OFF_BAR;
@@ -123,9 +123,9 @@ __global__ void __launch_bounds__(C::NT, 1)
   auto bar_s_free = [&](int a) { return bar0 + 8 * (3 + 2 * C::NS + a); };
   auto bar_p_full = [&](int a) { return bar0 + 8 * (5 + 2 * C::NS + a); };
   auto bar_pv_done = [&](int a) { return bar0 + 8 * (7 + 2 * C::NS + a); };
-  const uint32_t bar_x_full = bar0 + 8 * (9 + 2 * C::NS);
-  const uint32_t bar_x_empty = bar0 + 8 * (10 + 2 * C::NS);
-  const uint32_t bar_drain = bar0 + 8 * (11 + 2 * C::NS);
+  auto bar_x_full = [&](int b) { return bar0 + 8 * (9 + 2 * C::NS + b); };
+  auto bar_x_empty = [&](int b) { return bar0 + 8 * (11 + 2 * C::NS + b); };
+  const uint32_t bar_drain = bar0 + 8 * (13 + 2 * C::NS);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* ntiles_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -146,8 +146,10 @@ __global__ void __launch_bounds__(C::NT, 1)
       mbar_init(bar_p_full(a), 128);
       mbar_init(bar_pv_done(a), 1);
     }
-    mbar_init(bar_x_full, 128);
-    mbar_init(bar_x_empty, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_x_full(b), 1);    // armed locally; filled by the peer's st.async bytes
+      mbar_init(bar_x_empty(b), 4);   // one release-arrive per softmax warp of the peer
+    }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     *ntiles_s = 0;
@@ -240,9 +242,10 @@ __global__ void __launch_bounds__(C::NT, 1)
         const uint32_t v_base = s_c + (j % C::NS) * C::C_STAGE;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          const uint64_t ad = smem_desc(s_p + pb * C::P_BYTES + kk * 32, 16, 512, 4);
+          // A = P from tensor memory: 16 k-elements = 8 columns per step
+          const uint32_t a_tmem = tmem + C::TMEM_P + pb * (C::BN / 2) + kk * 8;
           const uint64_t bd = smem_desc(v_base + kk * 16 * C::SWB, C::C_ATOM_BYTES, 8 * C::SWB, C::SWZ);
-          umma_ss(tmem, ad, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem, a_tmem, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar_c_empty(j % C::NS));
         umma_commit(bar_pv_done(pb));
@@ -281,8 +284,8 @@ __global__ void __launch_bounds__(C::NT, 1)
     const int h = warp * 32 + lane;                       // head row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t x_peer = C::SPLIT == 2 ? mapa_shared(smem_u32(xbuf), peer) : 0u;
-    const uint32_t bar_x_full_peer = C::SPLIT == 2 ? mapa_shared(bar_x_full, peer) : 0u;
-    const uint32_t bar_x_empty_peer = C::SPLIT == 2 ? mapa_shared(bar_x_empty, peer) : 0u;
+    const uint32_t bar_x_full_peer0 = C::SPLIT == 2 ? mapa_shared(bar_x_full(0), peer) : 0u;
+    const uint32_t bar_x_empty_peer0 = C::SPLIT == 2 ? mapa_shared(bar_x_empty(0), peer) : 0u;
     float m_used = -INFINITY;    // running max (log2 units) the exponentials are taken against
     float l_run = 0.f;
     bool ok = true;
@@ -299,26 +302,35 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
       for (int j = 0; j < C::BN; ++j) sv[j] = __uint_as_float(raw[j]);
       if (C::SPLIT == 2) {
-        // push my partial scores into the peer's buffer, row h, 16-byte chunks rotated by h
-        if (!mbar_wait_warp<true>(bar_x_empty, (it & 1) ^ 1, abort_flag, 27)) { ok = false; break; }
+        // Exchange the partial scores with the peer CTA (buffer xb of each side).
+        // Receive side: arm this tile's phase with the bytes the peer will send.
+        const int xb = it & 1;
+        const uint32_t xph = (it >> 1) & 1;
+        if (h == 0) mbar_arrive_expect_tx(bar_x_full(xb), C::X_BYTES);
+        // Send side: the peer must have released its buffer xb (tile it-2).
+        if (!mbar_wait_warp<true>(bar_x_empty(xb), xph ^ 1, abort_flag, 27)) { ok = false; break; }
+        const uint32_t dst_row = x_peer + xb * C::X_BYTES + h * C::BN * 4;
 #pragma unroll
         for (int c = 0; c < C::BN / 4; ++c) {
-          const int slot = (c + h) & (C::BN / 4 - 1);
-          st_cluster_v4(x_peer + (h * C::BN + slot * 4) * 4, sv[4 * c], sv[4 * c + 1], sv[4 * c + 2],
-                        sv[4 * c + 3]);
+          const int slot = (c + h) & (C::BN / 4 - 1);   // rotate 16-byte chunks: no bank conflicts
+          st_async_v4(dst_row + slot * 16, sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3],
+                      bar_x_full_peer0 + 8 * xb);
         }
-        mbar_arrive_remote(bar_x_full_peer);
-        if (!mbar_wait_warp<true>(bar_x_full, it & 1, abort_flag, 28)) { ok = false; break; }
+        if (!mbar_wait_warp<true>(bar_x_full(xb), xph, abort_flag, 28)) { ok = false; break; }
+        const float* xrow = xbuf + xb * (C::X_BYTES / 4) + h * C::BN;
 #pragma unroll
         for (int c = 0; c < C::BN / 4; ++c) {
           const int slot = (c + h) & (C::BN / 4 - 1);
-          const float4 v = *reinterpret_cast<const float4*>(xbuf + h * C::BN + slot * 4);
+          const float4 v = *reinterpret_cast<const float4*>(xrow + slot * 4);
           sv[4 * c] += v.x;
           sv[4 * c + 1] += v.y;
           sv[4 * c + 2] += v.z;
           sv[4 * c + 3] += v.w;
         }
-        mbar_arrive_remote(bar_x_empty_peer);
+        // this warp's 32 rows of buffer xb are read: hand them back to the peer
+        // (one release-arrive per warp; no CTA-wide barrier inside the loop)
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(bar_x_empty_peer0 + 8 * xb);
       }
       // validity of the tile's entries (written by the producer before it armed c_full)
       if (!mbar_wait_warp(bar_c_full(it % C::NS), (it / C::NS) & 1, abort_flag, 29)) { ok = false; break; }
@@ -366,13 +378,9 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
         tmem_wait_st();
       }
-      // P row h, K-major with the 64-byte swizzle: 16-byte chunk c sits at c ^ ((h & 7) >> 1)
-      uint8_t* prow = smem + C::OFF_P + sb * C::P_BYTES + (h >> 3) * 512 + (h & 7) * 64;
-#pragma unroll
-      for (int c = 0; c < C::BN / 8; ++c)
-        *reinterpret_cast<uint4*>(prow + ((c ^ ((h & 7) >> 1)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
+      // P row h (bf16 pairs) into tensor memory; the PV MMA reads it from there
+      tmem_st16(tmem + lane_base + C::TMEM_P + sb * (C::BN / 2), pk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p_full(sb));
     }

@@ -1,36 +1,69 @@
-// topk.cuh -- per-query top-k token selection (radix select).
+// topk.cuh -- per-query top-k token selection.
 //
 // "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse Attention (DSA)",
 // item 2: every query keeps the index_topk highest-scoring earlier tokens.
+// Order: higher score first, ties to the lower index; -0.0 ties +0.0.
 //
-// One CTA per query row.  Scores are mapped to order-preserving 32-bit keys
-// and the k-th largest key is found digit by digit (4 passes of 8 bits, a
-// 256-bin shared-memory histogram per pass, restricted to keys that match the
-// digits found so far).  A last pass over the row, in index order, emits every
-// key above that threshold and the lowest-index keys equal to it; ranks come
-// from warp ballots and a block scan, so the output is deterministic:
-// [keys > thr in index order][first keys == thr in index order][-1 ...].
-// Rows are read from global memory (L2-resident right after the indexer
-// wrote them) with 16-byte loads.
+// One CTA per query row.  The row (fp32 scores, usually still in L2 after the
+// indexer wrote it) streams through a 3-stage shared-memory ring of 32 KB bulk
+// async copies issued by one thread, so each SM keeps ~96 KB in flight.
+// Scores become order-preserving 32-bit keys.
+//   pass 1  histogram of the top 11 key bits (2048 bins; every warp counts into
+//           its own copy, so the hot bins of a score distribution never see
+//           atomics from two warps)  ->  the bin B that holds the k-th largest
+//           key, and the count above it;
+//   pass 2  every key in a bin above B is emitted; the keys of bin B are
+//           compacted into shared memory (in index order);
+//   refine  radix select on the remaining 21 bits among those candidates, then
+//           emit the candidates above the threshold and the lowest-index ones
+//           equal to it.
+// If bin B holds more candidates than fit in shared memory (massive ties), the
+// refinement runs over the row in global memory instead, with the same result.
+// Ranks come from ballots and warp/CTA prefix sums in index order, so the
+// output order is deterministic.
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace dsa {
 
-template <int NT>
-__global__ void __launch_bounds__(NT) topk_radix_kernel(const float* __restrict__ scores,
-                                                        int64_t ld, const int32_t* __restrict__ cu_q,
-                                                        const int32_t* __restrict__ cu_k, int B,
-                                                        int64_t q_begin, int topk,
-                                                        int32_t* __restrict__ idx) {
-  constexpr int NW = NT / 32;
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_digit, s_above;
-  __shared__ uint32_t warp_cnt[NW];
+struct TopkCfg {
+  static constexpr int NT = 512, NW = NT / 32;
+  static constexpr int CHUNK = 8192;                  // scores per streamed stage (32 KB)
+  static constexpr int PER_WARP = CHUNK / NW;         // 512: 4 float4 per lane
+  static constexpr int STAGES = 3;
+  static constexpr int BITS1 = 11, BINS1 = 1 << BITS1, SHIFT1 = 32 - BITS1;
+  static constexpr int CAP = 6144;                    // bin-B candidates kept in shared memory
+  static constexpr int MAX_N = (65535 / PER_WARP) * CHUNK;   // 16-bit per-warp pass-1 counters
+  static constexpr int OFF_RING = 0;
+  static constexpr int OFF_WHIST = OFF_RING + STAGES * CHUNK * 4;   // per-warp pass-1 histograms
+  static constexpr int OFF_HIST = OFF_WHIST + NW * (BINS1 / 2) * 4; // two 16-bit counters per word
+  static constexpr int OFF_CKEY = OFF_HIST + BINS1 * 4;
+  static constexpr int OFF_CIDX = OFF_CKEY + CAP * 4;
+  static constexpr int OFF_WTOT = OFF_CIDX + CAP * 4;
+  static constexpr int OFF_BAR = OFF_WTOT + 2 * NW * 4;
+  static constexpr int OFF_MISC = OFF_BAR + STAGES * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 128;   // + alignment slack
+};
 
-  const int tid = threadIdx.x;
-  const int lane = tid & 31, warp = tid >> 5;
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t lane, uint32_t* total) {
+  uint32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= static_cast<uint32_t>(off)) incl += u;
+  }
+  *total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  return incl - v;
+}
+
+__global__ void __launch_bounds__(TopkCfg::NT, 1)
+    topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ cu_q,
+                const int32_t* __restrict__ cu_k, int B, int64_t q_begin, int topk,
+                int32_t* __restrict__ idx) {
+  using C = TopkCfg;
+  const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t r = blockIdx.x;
   const RowInfo ri = locate_row(cu_q, cu_k, B, q_begin + r);
   const int n = ri.pos + 1;
@@ -38,113 +71,305 @@ __global__ void __launch_bounds__(NT) topk_radix_kernel(const float* __restrict_
   int32_t* __restrict__ out = idx + r * topk;
 
   if (n <= topk) {  // every candidate is selected
-    for (int i = tid; i < topk; i += NT) out[i] = i < n ? i : -1;
+    for (int i = tid; i < topk; i += C::NT) out[i] = i < n ? i : -1;
     return;
   }
+  if (device_error_pending()) return;
 
-  const int n4 = n >> 2;  // rows start 16-byte aligned (ld % 4 == 0)
-  const float4* __restrict__ row4 = reinterpret_cast<const float4*>(row);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  float* ring = reinterpret_cast<float*>(smem + C::OFF_RING);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
+  uint32_t* ckey = reinterpret_cast<uint32_t*>(smem + C::OFF_CKEY);
+  int32_t* cidx = reinterpret_cast<int32_t*>(smem + C::OFF_CIDX);
+  uint32_t* wtot = reinterpret_cast<uint32_t*>(smem + C::OFF_WTOT);
+  const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 16);
 
-  uint32_t prefix = 0;
-  int remaining = topk;
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int i = tid; i < 256; i += NT) hist[i] = 0u;
-    __syncthreads();
-    auto count = [&](uint32_t key, bool valid) {
-      const bool m = valid && ((key & hi_mask) == prefix);
-      const uint32_t bin = (key >> shift) & 255u;
-      const uint32_t active = __ballot_sync(0xFFFFFFFFu, m);
-      if (m) {
-        const uint32_t peers = __match_any_sync(active, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
-      }
-    };
-    for (int base = 0; base < n4; base += NT) {
-      const int i4 = base + tid;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      const bool ok = i4 < n4;
-      if (ok) v = row4[i4];
-      count(order_key(v.x), ok);
-      count(order_key(v.y), ok);
-      count(order_key(v.z), ok);
-      count(order_key(v.w), ok);
-    }
-    {  // ragged tail (fewer than 4 elements)
-      const int i = 4 * n4 + tid;
-      const bool ok = tid < 32 && i < n;
-      if (warp == 0) count(ok ? order_key(row[i]) : 0u, ok);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l owns bins 255-8l .. 248-8l (descending); scan counts from the top
-      uint32_t c[8], sum = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        c[j] = hist[255 - 8 * lane - j];
-        sum += c[j];
-      }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      const uint32_t excl = incl - sum;
-      const uint32_t need = static_cast<uint32_t>(remaining);
-      if (excl < need && need <= incl) {
-        uint32_t acc = excl;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (acc + c[j] >= need) {
-            s_digit = 255u - 8u * lane - j;
-            s_above = acc;
-            break;
-          }
-          acc += c[j];
-        }
-      }
-    }
-    __syncthreads();
-    prefix |= s_digit << shift;
-    remaining -= static_cast<int>(s_above);
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(bar0 + 8 * s, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
   }
+  uint32_t* whist = reinterpret_cast<uint32_t*>(smem + C::OFF_WHIST) + warp * (C::BINS1 / 2);
+  for (int i = tid; i < C::NW * (C::BINS1 / 2); i += C::NT) reinterpret_cast<uint32_t*>(smem + C::OFF_WHIST)[i] = 0u;
+  __syncthreads();
 
-  // keys > prefix: exactly topk - remaining of them; keys == prefix: take the
-  // first `remaining` in index order.
-  const uint32_t thr = prefix;
-  const int need_eq = remaining;
-  const int n_gt = topk - remaining;
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  int gt_base = 0, eq_base = 0;
-#pragma unroll 1
-  for (int base = 0; base < n; base += NT) {
-    const int i = base + tid;
-    const uint32_t key = i < n ? order_key(row[i]) : 0u;
-    const bool gt = i < n && key > thr;
-    const bool eq = i < n && key == thr;
-    const uint32_t bg = __ballot_sync(0xFFFFFFFFu, gt);
-    const uint32_t be = __ballot_sync(0xFFFFFFFFu, eq);
-    if (lane == 0) warp_cnt[warp] = (static_cast<uint32_t>(__popc(bg)) << 16) | __popc(be);
+  // ------------------------------------------------------------------ streaming
+  const int nchunks = (n + C::CHUNK - 1) / C::CHUNK;
+  int g = 0;           // chunks streamed before the current pass (barrier phases)
+  int issued = 0;      // global chunk counter of copies issued (thread 0)
+  auto issue = [&](int c, int gg) {
+    const int s = gg % C::STAGES;
+    const int cnt = min(C::CHUNK, n - c * C::CHUNK);
+    const uint32_t bytes = static_cast<uint32_t>((cnt + 3) & ~3) * 4u;  // rows hold ld >= n rounded up to 4
+    mbar_arrive_expect_tx(bar0 + 8 * s, bytes);
+    bulk_load(smem_u32(ring + s * C::CHUNK), row + static_cast<int64_t>(c) * C::CHUNK, bytes, bar0 + 8 * s);
+    issued = gg + 1;
+  };
+  auto stream = [&](auto&& body) -> bool {
+    if (tid == 0)
+      for (int j = 0; j < min(C::STAGES, nchunks); ++j) issue(j, g + j);
+    bool ok = true;
+    int c = 0;
+    for (; c < nchunks; ++c) {
+      const int gg = g + c, s = gg % C::STAGES;
+      const bool got = mbar_wait(bar0 + 8 * s, (gg / C::STAGES) & 1, abort_flag, 40);
+      if (__syncthreads_or(!got)) { ok = false; break; }
+      // every thread is done with chunk c-1: refill its stage
+      if (tid == 0 && c >= 1 && c - 1 + C::STAGES < nchunks) issue(c - 1 + C::STAGES, gg - 1 + C::STAGES);
+      body(c, ring + s * C::CHUNK);
+    }
+    if (!ok && tid == 0) {  // let copies in flight land before the CTA leaves
+      long long t0 = clock64();
+      for (int gg = g + c; gg < issued; ++gg)
+        while (!mbar_try_wait(bar0 + 8 * (gg % C::STAGES), (gg / C::STAGES) & 1) &&
+               clock64() - t0 < kWaitLimitCycles) {
+        }
+    }
     __syncthreads();
-    uint32_t off = 0, tot = 0;
+    g += nchunks;
+    return ok;
+  };
+
+  // warp-aggregated histogram increment
+  auto hist_add = [&](uint32_t* h, uint32_t bin, bool valid) {
+    const uint32_t active = __ballot_sync(0xFFFFFFFFu, valid);
+    if (valid) {
+      const uint32_t peers = __match_any_sync(active, bin);
+      if (lane == static_cast<uint32_t>(__ffs(peers) - 1)) atomicAdd(&h[bin], static_cast<uint32_t>(__popc(peers)));
+    }
+  };
+
+  // pass-1 increment into this warp's private histogram (two 16-bit counters per word)
+  auto whist_add = [&](uint32_t bin, bool valid) {
+    const uint32_t active = __ballot_sync(0xFFFFFFFFu, valid);
+    if (valid) {
+      const uint32_t peers = __match_any_sync(active, bin);
+      if (lane == static_cast<uint32_t>(__ffs(peers) - 1))
+        atomicAdd(&whist[bin >> 1], static_cast<uint32_t>(__popc(peers)) << (16 * (bin & 1)));
+    }
+  };
+
+  // Classify the chunk's elements (gt / eq flags) and emit them with ranks in
+  // index order: element order inside a chunk is (warp, rr, lane, e).
+  // emit_gt(rank, index, key), emit_eq(rank, index, key); bases advance by the chunk totals.
+  uint32_t gt_base = 0, eq_base = 0;
+  auto scan_chunk = [&](int c, const float* buf, auto&& classify, auto&& emit_gt, auto&& emit_eq) {
+    uint32_t keys[16], flags = 0, rank_base[4];
+    uint32_t wacc = 0;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const uint32_t v = warp_cnt[w];
-      off += w < warp ? v : 0u;
-      tot += v;
+    for (int rr = 0; rr < 4; ++rr) {
+      const int off = static_cast<int>(warp) * C::PER_WARP + (static_cast<int>(lane) + 32 * rr) * 4;
+      const float4 v = *reinterpret_cast<const float4*>(buf + off);
+      const float vals[4] = {v.x, v.y, v.z, v.w};
+      uint32_t cg = 0, ce = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int gi = c * C::CHUNK + off + e;
+        const uint32_t key = order_key(vals[e]);
+        keys[rr * 4 + e] = key;
+        bool gt = false, eq = false;
+        if (gi < n) classify(key, gt, eq);
+        flags |= (gt ? 1u : 0u) << (2 * (rr * 4 + e));
+        flags |= (eq ? 2u : 0u) << (2 * (rr * 4 + e));
+        cg += gt;
+        ce += eq;
+      }
+      uint32_t tot;
+      const uint32_t pre = warp_excl_scan(cg | (ce << 16), lane, &tot);
+      rank_base[rr] = wacc + pre;
+      wacc += tot;
     }
-    if (gt) out[gt_base + static_cast<int>(off >> 16) + __popc(bg & lt_mask)] = i;
-    if (eq) {
-      const int rk = eq_base + static_cast<int>(off & 0xFFFFu) + __popc(be & lt_mask);
-      if (rk < need_eq) out[n_gt + rk] = i;
-    }
-    gt_base += static_cast<int>(tot >> 16);
-    eq_base += static_cast<int>(tot & 0xFFFFu);
+    if (lane == 31) wtot[(c & 1) * C::NW + warp] = wacc;
     __syncthreads();
-    if (gt_base >= n_gt && eq_base >= need_eq) break;
+    uint32_t wpre = 0, ctot = 0;
+#pragma unroll
+    for (int w = 0; w < C::NW; ++w) {
+      const uint32_t v = wtot[(c & 1) * C::NW + w];
+      wpre += static_cast<uint32_t>(w) < warp ? v : 0u;
+      ctot += v;
+    }
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      uint32_t rg = gt_base + (wpre & 0xFFFFu) + (rank_base[rr] & 0xFFFFu);
+      uint32_t re = eq_base + (wpre >> 16) + (rank_base[rr] >> 16);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t f = (flags >> (2 * (rr * 4 + e))) & 3u;
+        const int gi = c * C::CHUNK + static_cast<int>(warp) * C::PER_WARP + (static_cast<int>(lane) + 32 * rr) * 4 + e;
+        if (f & 1u) emit_gt(rg++, gi, keys[rr * 4 + e]);
+        if (f & 2u) emit_eq(re++, gi, keys[rr * 4 + e]);
+      }
+    }
+    gt_base += ctot & 0xFFFFu;
+    eq_base += ctot >> 16;
+  };
+
+  // ------------------------------------------------------------------ pass 1
+  bool ok = stream([&](int c, const float* buf) {
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr) {
+      const int off = static_cast<int>(warp) * C::PER_WARP + (static_cast<int>(lane) + 32 * rr) * 4;
+      const float4 v = *reinterpret_cast<const float4*>(buf + off);
+      const int gi = c * C::CHUNK + off;
+      whist_add(order_key(v.x) >> C::SHIFT1, gi < n);
+      whist_add(order_key(v.y) >> C::SHIFT1, gi + 1 < n);
+      whist_add(order_key(v.z) >> C::SHIFT1, gi + 2 < n);
+      whist_add(order_key(v.w) >> C::SHIFT1, gi + 3 < n);
+    }
+  });
+  if (!ok) return;
+  // merge the per-warp counts
+  for (int bin = tid; bin < C::BINS1; bin += C::NT) {
+    uint32_t sum = 0;
+#pragma unroll
+    for (int w = 0; w < C::NW; ++w)
+      sum += (reinterpret_cast<const uint32_t*>(smem + C::OFF_WHIST)[w * (C::BINS1 / 2) + (bin >> 1)] >>
+              (16 * (bin & 1))) & 0xFFFFu;
+    hist[bin] = sum;
+  }
+  __syncthreads();
+
+  // k-th largest lies in bin B: lane l scans bins 2047-64l .. 1984-64l (descending)
+  auto find_digit = [&](const uint32_t* h, int nbins, uint32_t need, uint32_t* digit, uint32_t* above) {
+    const int per = nbins / 32;
+    uint32_t sum = 0;
+    for (int j = 0; j < per; ++j) sum += h[nbins - 1 - per * static_cast<int>(lane) - j];
+    uint32_t tot;
+    const uint32_t excl = warp_excl_scan(sum, lane, &tot);
+    if (excl < need && need <= excl + sum) {
+      uint32_t acc = excl;
+      for (int j = 0; j < per; ++j) {
+        const uint32_t cnt = h[nbins - 1 - per * static_cast<int>(lane) - j];
+        if (acc + cnt >= need) {
+          *digit = static_cast<uint32_t>(nbins - 1 - per * static_cast<int>(lane) - j);
+          *above = acc;
+          break;
+        }
+        acc += cnt;
+      }
+    }
+  };
+  if (warp == 0) find_digit(hist, C::BINS1, static_cast<uint32_t>(topk), &misc[0], &misc[1]);
+  __syncthreads();
+  const uint32_t bin_b = misc[0];
+  const uint32_t above = misc[1];
+  const uint32_t need = static_cast<uint32_t>(topk) - above;
+
+  // ------------------------------------------------------------------ pass 2
+  ok = stream([&](int c, const float* buf) {
+    scan_chunk(
+        c, buf,
+        [&](uint32_t key, bool& gt, bool& eq) {
+          const uint32_t b = key >> C::SHIFT1;
+          gt = b > bin_b;
+          eq = b == bin_b;
+        },
+        [&](uint32_t rank, int gi, uint32_t) { out[rank] = gi; },
+        [&](uint32_t rank, int gi, uint32_t key) {
+          if (rank < static_cast<uint32_t>(C::CAP)) {
+            ckey[rank] = key;
+            cidx[rank] = gi;
+          }
+        });
+  });
+  if (!ok) return;
+  const uint32_t n_eq = eq_base;          // keys in bin B (all of them, even past CAP)
+
+  // ------------------------------------------------------------------ refine inside bin B
+  // 21 remaining key bits as digits of 8, 8 and 5 bits.
+  uint32_t prefix = bin_b << C::SHIFT1;
+  uint32_t remaining = need;
+  const bool in_smem = n_eq <= static_cast<uint32_t>(C::CAP);
+  const int shifts[3] = {13, 5, 0};
+  const int widths[3] = {8, 8, 5};
+  for (int d = 0; d < 3; ++d) {
+    const int shift = shifts[d], bits = widths[d];
+    const uint32_t dmask = (1u << bits) - 1u;
+    const int hi = shift + bits;                  // bits at or above `hi` are fixed by prefix
+    for (int i = tid; i < 256; i += C::NT) hist[i] = 0u;
+    __syncthreads();
+    auto count_key = [&](uint32_t key, bool valid) {
+      const bool m = valid && ((key >> hi) == (prefix >> hi));
+      hist_add(hist, (key >> shift) & dmask, m);
+    };
+    if (in_smem) {
+      for (uint32_t base = 0; base < n_eq; base += C::NT) {
+        const uint32_t i = base + tid;
+        count_key(i < n_eq ? ckey[i] : 0u, i < n_eq);
+      }
+    } else {
+      ok = stream([&](int c, const float* buf) {
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int off = static_cast<int>(warp) * C::PER_WARP + (static_cast<int>(lane) + 32 * rr) * 4;
+          const float4 v = *reinterpret_cast<const float4*>(buf + off);
+          const int gi = c * C::CHUNK + off;
+          count_key(order_key(v.x), gi < n);
+          count_key(order_key(v.y), gi + 1 < n);
+          count_key(order_key(v.z), gi + 2 < n);
+          count_key(order_key(v.w), gi + 3 < n);
+        }
+      });
+      if (!ok) return;
+    }
+    __syncthreads();
+    if (warp == 0) find_digit(hist, 1 << bits, remaining, &misc[2], &misc[3]);
+    __syncthreads();
+    prefix |= misc[2] << shift;
+    remaining -= misc[3];
+    __syncthreads();
+  }
+  const uint32_t thr = prefix;            // the k-th largest key
+  const uint32_t need_eq = remaining;     // how many keys equal to it are taken
+  const uint32_t n_gt = need - need_eq;   // keys of bin B above it
+  int32_t* out_b = out + above;
+
+  // ------------------------------------------------------------------ emit bin B's selection
+  gt_base = 0;
+  eq_base = 0;
+  if (in_smem) {
+    for (uint32_t base = 0; base < n_eq; base += C::NT) {
+      const uint32_t i = base + tid;
+      const uint32_t key = i < n_eq ? ckey[i] : 0u;
+      const bool gt = i < n_eq && key > thr;
+      const bool eq = i < n_eq && key == thr;
+      const uint32_t lt = (1u << lane) - 1u;
+      const uint32_t bg = __ballot_sync(0xFFFFFFFFu, gt), be = __ballot_sync(0xFFFFFFFFu, eq);
+      if (lane == 0) wtot[warp] = (static_cast<uint32_t>(__popc(bg))) | (static_cast<uint32_t>(__popc(be)) << 16);
+      __syncthreads();
+      uint32_t wpre = 0, ctot = 0;
+#pragma unroll
+      for (int w = 0; w < C::NW; ++w) {
+        const uint32_t v = wtot[w];
+        wpre += static_cast<uint32_t>(w) < warp ? v : 0u;
+        ctot += v;
+      }
+      if (gt) out_b[gt_base + (wpre & 0xFFFFu) + __popc(bg & lt)] = cidx[i];
+      if (eq) {
+        const uint32_t rk = eq_base + (wpre >> 16) + __popc(be & lt);
+        if (rk < need_eq) out_b[n_gt + rk] = cidx[i];
+      }
+      gt_base += ctot & 0xFFFFu;
+      eq_base += ctot >> 16;
+      __syncthreads();
+    }
+  } else {
+    stream([&](int c, const float* buf) {
+      scan_chunk(
+          c, buf,
+          [&](uint32_t key, bool& gt, bool& eq) {
+            const bool inb = (key >> C::SHIFT1) == bin_b;
+            gt = inb && key > thr;
+            eq = inb && key == thr;
+          },
+          [&](uint32_t rank, int gi, uint32_t) { out_b[rank] = gi; },
+          [&](uint32_t rank, int gi, uint32_t) {
+            if (rank < need_eq) out_b[n_gt + rank] = gi;
+          });
+    });
   }
 }
 

@@ -1,0 +1,83 @@
+"""Run one stage of the DSA hot path in a loop, for profilers (ncu).
+
+    python -m sparse_attention_long_07_b200.profile_stage --workload decode128k \
+        --seqs 16 --stage indexer --iters 3
+
+--seqs keeps the first N sequences of the named workload (same values as the
+full workload), so a capture can stay at a few GB of device memory while its
+inputs remain larger than the L2 cache.  Prints the kernel's mean duration
+(CUDA events, not under a profiler) and the sizes it ran on.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import dsa_inputs as di  # noqa: E402
+import sparse_attention_long_07_b200 as dsa  # noqa: E402
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="decode128k", choices=list(di.CONFIG_NAMES))
+    ap.add_argument("--seqs", type=int, default=0, help="first N sequences only (0 = all)")
+    ap.add_argument("--stage", default="indexer", choices=["indexer", "topk", "attention", "forward"])
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--wait-profile", action="store_true",
+                    help="print per-wait-site cycles (library built with --profile-waits)")
+    args = ap.parse_args()
+    spec = di.config(args.workload)
+    seqs = list(range(spec.B)) if args.seqs <= 0 else list(range(min(args.seqs, spec.B)))
+    dev = torch.device("cuda", 0)
+    d = di.make_inputs(spec, device=dev, seqs=seqs)
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], dev)
+    T, k = v.T, spec.topk
+    ld = (v.max_kv + 3) // 4 * 4
+    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    out = torch.empty((T, spec.H, spec.d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, spec.H), dtype=torch.float32, device=dev)
+    ws = torch.empty(dsa.dsa_forward_workspace_size(v, k), dtype=torch.uint8, device=dev)
+    # inputs of the later stages
+    dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores)
+    dsa.dsa_topk(scores, v, 0, T, k, idx)
+    torch.cuda.synchronize()
+
+    def run():
+        if args.stage == "indexer":
+            dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores)
+        elif args.stage == "topk":
+            dsa.dsa_topk(scores, v, 0, T, k, idx)
+        elif args.stage == "attention":
+            dsa.dsa_sparse_mla_attn(d["q"], d["latent"], idx, v, 0, T, spec.softmax_scale, out, lse)
+        else:
+            dsa.dsa_forward(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], d["q"], d["latent"], v, k,
+                            spec.softmax_scale, out, lse, ws)
+
+    if args.wait_profile:
+        dsa.dsa_debug_wait_profile(reset=True)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.iters):
+        run()
+    b.record()
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_error() == 0
+    if args.wait_profile:
+        prof = dsa.dsa_debug_wait_profile(reset=True) or {}
+        print(json.dumps({"wait_sites": {str(k): {"cycles_per_wait": round(c / max(n, 1), 1), "waits": n,
+                                                  "cycles_total": c} for k, (c, n) in sorted(prof.items())}}))
+    print(json.dumps({"workload": spec.name, "seqs": len(seqs), "stage": args.stage, "query_rows": T,
+                      "keys": v.S, "mean_ms": a.elapsed_time(b) / args.iters,
+                      "device_bytes_allocated": torch.cuda.memory_allocated()}))
+
+
+if __name__ == "__main__":
+    main()

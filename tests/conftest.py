@@ -18,3 +18,13 @@ def oracle_lib():
     import oracle
     oracle.build()
     return oracle
+
+
+def build_library():
+    """Compile libdsa.so if stale (the builder is loaded by path, not through the package)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "dsa_build", os.path.join(ROOT, "sparse_attention_long_07_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()

@@ -14,8 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def dsa():
-    from sparse_attention_long_07_b200 import build
-    build.build()
+    from tests.conftest import build_library
+    build_library()
     import sparse_attention_long_07_b200 as m
     return m
 
