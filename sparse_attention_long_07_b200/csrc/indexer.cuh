@@ -46,13 +46,15 @@ struct IndexerCfg {
   static constexpr int NATOM = ROWB / SWB;                // swizzle-atom columns per row
   static constexpr int ATOM_ELEMS = SWB / 2;
   static constexpr int KSTEPS = D_I / 16;
-  static constexpr int STAGES = KFP8 ? 2 : 4;             // bf16 key-tile ring
+  static constexpr int STAGES = KFP8 ? (PERSIST ? 3 : 2) : 4;   // bf16 key-tile ring
   static constexpr int RSTAGES = KFP8 ? (PERSIST ? 6 : 4) : 0;   // raw e4m3 ring
   static constexpr int A_TILE = BK * ROWB;
   static constexpr int B_TILE = N * ROWB;
   static constexpr int RAW_TILE = BK * D_I;
-  static constexpr int EPI_WG = N >= 256 ? 2 : 1;         // epilogue warpgroups
-  static constexpr int QW = NQ / EPI_WG;                  // queries per epilogue warpgroup
+  // epilogue warpgroups: two split the queries of a wide tile, or (persistent
+  // schedule) take alternate tiles, each owning one TMEM accumulator
+  static constexpr int EPI_WG = (PERSIST || N >= 256) ? 2 : 1;
+  static constexpr int QW = PERSIST ? NQ : NQ / EPI_WG;   // queries per epilogue warpgroup
   static constexpr int COLS_PER_THREAD = QW * H_I;
   static constexpr int LD_CHUNK = COLS_PER_THREAD >= 32 ? 32 : 16;
   static constexpr int TMEM_COLS = pow2_at_least(2 * N, 32);
@@ -448,7 +450,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar_acc_full(a), 1);
-      mbar_init(bar_acc_empty(a), C::EPI_THREADS);
+      mbar_init(bar_acc_empty(a), 128);   // drained by warpgroup a
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -551,13 +553,26 @@ __global__ void __launch_bounds__(C::NT, 1)
       mbar_arrive(bar_k_full(s));
     }
   } else {
-    // ------------------------------------------------------------ epilogue (one warpgroup)
+    // ------------------------------------------------------------ epilogue
+    // Warpgroup g drains accumulator g, i.e. tiles it = g, g+2, ...; the key
+    // scales of its next tile are loaded one iteration ahead.
+    const int g = warp >> 2;
     const int sub = warp & 3;
     const int key_in_tile = sub * 32 + lane;
-    int b = b_first, cur = -1;
+    int b = b_first, cur = -1, bp = b_first;
     Seq q{};
     float wreg[C::H_I];
-    for (int it = 0; it < n_iter; ++it) {
+    auto fetch_scale = [&](int itx) -> float {
+      if (itx >= n_iter) return 0.f;
+      const int u = u0 + itx;
+      while (u >= upre[bp + 1]) ++bp;
+      const int kb = p.cu_k[bp];
+      const int s_key = (u - upre[bp]) * C::BK + key_in_tile;
+      return s_key < p.cu_k[bp + 1] - kb ? p.k_scale[kb + s_key] : 0.f;
+    };
+    float ks = fetch_scale(g);
+    for (int it = g; it < n_iter; it += 2) {
+      const float ks_next = fetch_scale(it + 2);
       const int u = u0 + it;
       while (u >= upre[b + 1]) ++b;
       if (b != cur) {
@@ -573,28 +588,29 @@ __global__ void __launch_bounds__(C::NT, 1)
           wreg[4 * j + 3] = v.w;
         }
       }
-      const int a = it & 1;
-      if (!mbar_wait_warp(bar_acc_full(a), (it >> 1) & 1, abort_flag, 57)) break;
+      if (!mbar_wait_warp(bar_acc_full(g), (it >> 1) & 1, abort_flag, 57)) break;
       tc_fence_after();
-      const uint32_t t_row = tmem + (static_cast<uint32_t>(sub * 32) << 16) + a * C::N;
-      uint32_t v0[32], v1[32];
-      tmem_ld32(t_row, v0);
-      tmem_ld32(t_row + 32, v1);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar_acc_empty(a));
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(sub * 32) << 16) + g * C::N;
       float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        acc0 = fmaf(wreg[j], fmaxf(__uint_as_float(v0[j]), 0.f), acc0);
-        acc1 = fmaf(wreg[32 + j], fmaxf(__uint_as_float(v1[j]), 0.f), acc1);
+      for (int half = 0; half < C::H_I / 32; ++half) {
+        uint32_t v[32];
+        tmem_ld32(t_row + 32 * half, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          acc0 = fmaf(wreg[32 * half + j], fmaxf(__uint_as_float(v[j]), 0.f), acc0);
+          acc1 = fmaf(wreg[32 * half + j + 1], fmaxf(__uint_as_float(v[j + 1]), 0.f), acc1);
+        }
       }
-      const int tile = u - upre[b];
-      const int s_key = tile * C::BK + key_in_tile;
+      tc_fence_before();
+      mbar_arrive(bar_acc_empty(g));
+      const int s_key = (u - upre[b]) * C::BK + key_in_tile;
       if (s_key < q.kv_len) {
-        const float val = s_key <= q.pos ? (acc0 + acc1) * p.k_scale[q.k_base + s_key] : -INFINITY;
+        const float val = s_key <= q.pos ? (acc0 + acc1) * ks : -INFINITY;
         p.scores[(static_cast<int64_t>(q.q0) - p.q_begin) * p.ld + s_key] = val;
       }
+      ks = ks_next;
     }
   }
 

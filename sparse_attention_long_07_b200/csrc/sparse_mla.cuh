@@ -62,12 +62,13 @@ struct MlaCfg {
   static constexpr int OFF_X = OFF_C + NS * C_STAGE;      // two partial-score buffers
   static constexpr int OFF_MASK = OFF_X + 2 * X_BYTES;
   static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
-  static constexpr int NBAR = 1 + 2 * NS + 2 + 2 + 2 + 2 + 4 + 1;
+  static constexpr int NSB = 3;                            // S buffers: QK runs up to 3 tiles ahead
+  static constexpr int NBAR = 1 + 2 * NS + 2 * NSB + 2 + 2 + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  // tensor memory columns: O [0, DVS), S[2] (fp32, BN each), P[2] (bf16 pairs, BN/2 each)
+  // tensor memory columns: O [0, DVS), S[3] (fp32, BN each), P[2] (bf16 pairs, BN/2 each)
   static constexpr int TMEM_S = DVS;
-  static constexpr int TMEM_P = DVS + 2 * BN;
+  static constexpr int TMEM_P = DVS + NSB * BN;
   static constexpr int TMEM_USED = TMEM_P + BN;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static constexpr int NT = 6 * 32;
@@ -119,13 +120,14 @@ __global__ void __launch_bounds__(C::NT, 1)
   const uint32_t bar_q_full = bar0;
   auto bar_c_full = [&](int s) { return bar0 + 8 * (1 + s); };
   auto bar_c_empty = [&](int s) { return bar0 + 8 * (1 + C::NS + s); };
-  auto bar_s_full = [&](int a) { return bar0 + 8 * (1 + 2 * C::NS + a); };
-  auto bar_s_free = [&](int a) { return bar0 + 8 * (3 + 2 * C::NS + a); };
-  auto bar_p_full = [&](int a) { return bar0 + 8 * (5 + 2 * C::NS + a); };
-  auto bar_pv_done = [&](int a) { return bar0 + 8 * (7 + 2 * C::NS + a); };
-  auto bar_x_full = [&](int b) { return bar0 + 8 * (9 + 2 * C::NS + b); };
-  auto bar_x_empty = [&](int b) { return bar0 + 8 * (11 + 2 * C::NS + b); };
-  const uint32_t bar_drain = bar0 + 8 * (13 + 2 * C::NS);
+  constexpr int SB0 = 1 + 2 * C::NS;                     // first S barrier
+  auto bar_s_full = [&](int a) { return bar0 + 8 * (SB0 + a); };
+  auto bar_s_free = [&](int a) { return bar0 + 8 * (SB0 + C::NSB + a); };
+  auto bar_p_full = [&](int a) { return bar0 + 8 * (SB0 + 2 * C::NSB + a); };
+  auto bar_pv_done = [&](int a) { return bar0 + 8 * (SB0 + 2 * C::NSB + 2 + a); };
+  auto bar_x_full = [&](int b) { return bar0 + 8 * (SB0 + 2 * C::NSB + 4 + b); };
+  auto bar_x_empty = [&](int b) { return bar0 + 8 * (SB0 + 2 * C::NSB + 6 + b); };
+  const uint32_t bar_drain = bar0 + 8 * (SB0 + 2 * C::NSB + 8);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* ntiles_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -140,9 +142,11 @@ __global__ void __launch_bounds__(C::NT, 1)
       mbar_init(bar_c_full(s), 1);
       mbar_init(bar_c_empty(s), 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < C::NSB; ++a) {
       mbar_init(bar_s_full(a), 1);
       mbar_init(bar_s_free(a), 128);
+    }
+    for (int a = 0; a < 2; ++a) {
       mbar_init(bar_p_full(a), 128);
       mbar_init(bar_pv_done(a), 1);
     }
@@ -251,14 +255,13 @@ __global__ void __launch_bounds__(C::NT, 1)
         umma_commit(bar_pv_done(pb));
         return true;
       };
-      bool ok = mbar_wait(bar_q_full, 0, abort_flag, 23);
-      tc_fence_after();
       const int ksteps = na * C::KPA;
-      for (int it = 0; ok && it < n_tiles; ++it) {
-        const int s = it % C::NS;
-        const int sb = it & 1;
-        if (!mbar_wait(bar_c_full(s), (it / C::NS) & 1, abort_flag, 24)) break;
-        if (!mbar_wait(bar_s_free(sb), ((it >> 1) & 1) ^ 1, abort_flag, 25)) break;
+      // QK(j) -> S[j % 3]; issued up to three tiles ahead of the PV that trails it
+      auto issue_qk = [&](int j) -> bool {
+        const int s = j % C::NS;
+        const int sb = j % C::NSB;
+        if (!mbar_wait(bar_c_full(s), (j / C::NS) & 1, abort_flag, 24)) return false;
+        if (!mbar_wait(bar_s_free(sb), ((j / C::NSB) & 1) ^ 1, abort_flag, 25)) return false;
         tc_fence_after();
         const uint32_t c_base = s_c + s * C::C_STAGE;
         for (int kk = 0; kk < ksteps; ++kk) {
@@ -269,9 +272,15 @@ __global__ void __launch_bounds__(C::NT, 1)
           umma_ss(tmem + C::TMEM_S + sb * C::BN, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_s_full(sb));
-        if (it > 0 && !issue_pv(it - 1)) { ok = false; break; }
+        return true;
+      };
+      bool ok = mbar_wait(bar_q_full, 0, abort_flag, 23);
+      tc_fence_after();
+      for (int j = 0; ok && j < C::NSB && j < n_tiles; ++j) ok = issue_qk(j);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (!issue_pv(j)) break;
+        if (j + C::NSB < n_tiles && !issue_qk(j + C::NSB)) break;
       }
-      if (ok && !*abort_flag) issue_pv(n_tiles - 1);
     }
     if (lane == 0) {
       umma_commit(bar_drain);
@@ -289,34 +298,44 @@ __global__ void __launch_bounds__(C::NT, 1)
     float m_used = -INFINITY;    // running max (log2 units) the exponentials are taken against
     float l_run = 0.f;
     bool ok = true;
-    for (int it = 0; it < n_tiles; ++it) {
-      const int sb = it & 1;
-      if (!mbar_wait_warp(bar_s_full(sb), (it >> 1) & 1, abort_flag, 26)) { ok = false; break; }
+    // Load tile j's partial scores S[j % 3] and (2-CTA split) start sending them
+    // to the peer.  Tile it+1 is started before tile it is finished, so the
+    // exchange of a tile has a whole softmax iteration to complete.
+    auto load_and_push = [&](int j, float* dst) -> bool {
+      const int sb = j % C::NSB;
+      if (!mbar_wait_warp(bar_s_full(sb), (j / C::NSB) & 1, abort_flag, 26)) return false;
       tc_fence_after();
       uint32_t raw[32];
       tmem_ld32(tmem + lane_base + C::TMEM_S + sb * C::BN, raw);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar_s_free(sb));
-      float sv[C::BN];
 #pragma unroll
-      for (int j = 0; j < C::BN; ++j) sv[j] = __uint_as_float(raw[j]);
+      for (int c = 0; c < C::BN; ++c) dst[c] = __uint_as_float(raw[c]);
       if (C::SPLIT == 2) {
-        // Exchange the partial scores with the peer CTA (buffer xb of each side).
-        // Receive side: arm this tile's phase with the bytes the peer will send.
-        const int xb = it & 1;
-        const uint32_t xph = (it >> 1) & 1;
+        const int xb = j & 1;
+        // receive side: arm tile j's phase with the bytes the peer will send
         if (h == 0) mbar_arrive_expect_tx(bar_x_full(xb), C::X_BYTES);
-        // Send side: the peer must have released its buffer xb (tile it-2).
-        if (!mbar_wait_warp<true>(bar_x_empty(xb), xph ^ 1, abort_flag, 27)) { ok = false; break; }
+        // send side: the peer must have released its buffer xb (tile j-2)
+        if (!mbar_wait_warp<true>(bar_x_empty(xb), ((j >> 1) & 1) ^ 1, abort_flag, 27)) return false;
         const uint32_t dst_row = x_peer + xb * C::X_BYTES + h * C::BN * 4;
 #pragma unroll
         for (int c = 0; c < C::BN / 4; ++c) {
           const int slot = (c + h) & (C::BN / 4 - 1);   // rotate 16-byte chunks: no bank conflicts
-          st_async_v4(dst_row + slot * 16, sv[4 * c], sv[4 * c + 1], sv[4 * c + 2], sv[4 * c + 3],
+          st_async_v4(dst_row + slot * 16, dst[4 * c], dst[4 * c + 1], dst[4 * c + 2], dst[4 * c + 3],
                       bar_x_full_peer0 + 8 * xb);
         }
-        if (!mbar_wait_warp<true>(bar_x_full(xb), xph, abort_flag, 28)) { ok = false; break; }
+      }
+      return true;
+    };
+    float sv[C::BN], s_next[C::BN];
+    if (n_tiles > 0 && !load_and_push(0, sv)) ok = false;
+    for (int it = 0; ok && it < n_tiles; ++it) {
+      const int sb = it & 1;
+      if (it + 1 < n_tiles && !load_and_push(it + 1, s_next)) { ok = false; break; }
+      if (C::SPLIT == 2) {
+        const int xb = it & 1;
+        if (!mbar_wait_warp<true>(bar_x_full(xb), (it >> 1) & 1, abort_flag, 28)) { ok = false; break; }
         const float* xrow = xbuf + xb * (C::X_BYTES / 4) + h * C::BN;
 #pragma unroll
         for (int c = 0; c < C::BN / 4; ++c) {
@@ -383,6 +402,8 @@ __global__ void __launch_bounds__(C::NT, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p_full(sb));
+#pragma unroll
+      for (int c = 0; c < C::BN; ++c) sv[c] = s_next[c];
     }
     // ------------------------------------------------------------ epilogue
     const int t_out = static_cast<int>(t);

@@ -36,8 +36,13 @@ struct TopkCfg {
   static constexpr int BITS1 = 11, BINS1 = 1 << BITS1, SHIFT1 = 32 - BITS1;
   static constexpr int CAP = 6144;                    // bin-B candidates kept in shared memory
   static constexpr int MAX_N = (65535 / PER_WARP) * CHUNK;   // 16-bit per-warp pass-1 counters
+  static constexpr int PMAX_CAP = 8192;               // fast path: part maxima kept
+  static constexpr int BITMAP_BITS = 262144;          // fast path: longest row (one bit per key)
   static constexpr int OFF_RING = 0;
+  // union: per-warp pass-1 histograms (exact path) | part maxima + selection bitmap (fast path)
   static constexpr int OFF_WHIST = OFF_RING + STAGES * CHUNK * 4;   // per-warp pass-1 histograms
+  static constexpr int OFF_PMAX = OFF_WHIST;
+  static constexpr int OFF_BITMAP = OFF_WHIST + PMAX_CAP * 4;
   static constexpr int OFF_HIST = OFF_WHIST + NW * (BINS1 / 2) * 4; // two 16-bit counters per word
   static constexpr int OFF_CKEY = OFF_HIST + BINS1 * 4;
   static constexpr int OFF_CIDX = OFF_CKEY + CAP * 4;
@@ -45,6 +50,7 @@ struct TopkCfg {
   static constexpr int OFF_BAR = OFF_WTOT + 2 * NW * 4;
   static constexpr int OFF_MISC = OFF_BAR + STAGES * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 128;   // + alignment slack
+  static_assert(PMAX_CAP * 4 + BITMAP_BITS / 8 <= NW * (BINS1 / 2) * 4, "fast-path union fits");
 };
 
 __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t lane, uint32_t* total) {
@@ -93,7 +99,6 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     fence_mbar_init();
   }
   uint32_t* whist = reinterpret_cast<uint32_t*>(smem + C::OFF_WHIST) + warp * (C::BINS1 / 2);
-  for (int i = tid; i < C::NW * (C::BINS1 / 2); i += C::NT) reinterpret_cast<uint32_t*>(smem + C::OFF_WHIST)[i] = 0u;
   __syncthreads();
 
   // ------------------------------------------------------------------ streaming
@@ -207,6 +212,225 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     eq_base += ctot >> 16;
   };
 
+  // digit of the `need`-th largest entry: lane l scans bins nbins-1-per*l .. (descending)
+  auto find_digit_fn = [&](const uint32_t* h, int nbins, uint32_t need, uint32_t* digit, uint32_t* above) {
+    const int per = nbins / 32;
+    uint32_t sum = 0;
+    for (int j = 0; j < per; ++j) sum += h[nbins - 1 - per * static_cast<int>(lane) - j];
+    uint32_t tot;
+    const uint32_t excl = warp_excl_scan(sum, lane, &tot);
+    if (excl < need && need <= excl + sum) {
+      uint32_t acc = excl;
+      for (int j = 0; j < per; ++j) {
+        const uint32_t cnt = h[nbins - 1 - per * static_cast<int>(lane) - j];
+        if (acc + cnt >= need) {
+          *digit = static_cast<uint32_t>(nbins - 1 - per * static_cast<int>(lane) - j);
+          *above = acc;
+          break;
+        }
+        acc += cnt;
+      }
+    }
+  };
+  // ================================================================== fast path
+  // Split the row into parts of PS scores (part = PS consecutive scores of one
+  // thread's 16 per chunk, or one thread's scores over G chunks).  At least k
+  // scores are >= the k-th largest part maximum, so the lowest key b of the
+  // 11-bit bin holding that part maximum is a safe lower bound on the k-th
+  // largest score.  One pass keeps the scores >= b (typically ~1.2-2 k of
+  // them), the exact selection runs among those in shared memory, and the
+  // selected indices are written in increasing order through a bitmap.
+  // Rows where this cannot apply or the candidates overflow fall through to
+  // the exact path below.
+  {
+    int PS = 16;
+    while (PS > 1 && n / PS < 2 * topk) PS >>= 1;
+    const int parts_per_thread = 16 / PS;
+    const int G = max(1, (nchunks * C::NT * parts_per_thread + C::PMAX_CAP - 1) / C::PMAX_CAP);
+    const int P = ((nchunks + G - 1) / G) * C::NT * parts_per_thread;
+    const bool eligible = n <= C::BITMAP_BITS && n > topk && P <= C::PMAX_CAP && (G == 1 || PS == 16);
+    if (eligible) {
+      uint32_t* pmax = reinterpret_cast<uint32_t*>(smem + C::OFF_PMAX);
+      uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + C::OFF_BITMAP);
+      for (int i = tid; i < P; i += C::NT) pmax[i] = 0u;
+      for (int i = tid; i < C::BINS1; i += C::NT) hist[i] = 0u;
+      __syncthreads();
+      // ---- part maxima
+      uint32_t run = 0u;     // G > 1: running max of this thread's part over a chunk group
+      bool ok = stream([&](int c, const float* buf) {
+        uint32_t l0[16];      // keys of this thread's 16 scores, then pairwise maxima
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int off = static_cast<int>(warp) * C::PER_WARP + (static_cast<int>(lane) + 32 * rr) * 4;
+          const float4 v = *reinterpret_cast<const float4*>(buf + off);
+          const float vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            l0[rr * 4 + e] = c * C::CHUNK + off + e < n ? order_key(vals[e]) : 0u;
+        }
+        uint32_t l1[8], l2[4], l3[2];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) l1[j] = max(l0[2 * j], l0[2 * j + 1]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) l2[j] = max(l1[2 * j], l1[2 * j + 1]);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) l3[j] = max(l2[2 * j], l2[2 * j + 1]);
+        const uint32_t l4 = max(l3[0], l3[1]);
+        const int pbase = (c * C::NT + static_cast<int>(tid)) * parts_per_thread;
+        switch (PS) {
+          case 1:
+#pragma unroll
+            for (int q = 0; q < 16; ++q) pmax[pbase + q] = l0[q];
+            break;
+          case 2:
+#pragma unroll
+            for (int q = 0; q < 8; ++q) pmax[pbase + q] = l1[q];
+            break;
+          case 4:
+#pragma unroll
+            for (int q = 0; q < 4; ++q) pmax[pbase + q] = l2[q];
+            break;
+          case 8:
+            pmax[pbase] = l3[0];
+            pmax[pbase + 1] = l3[1];
+            break;
+          default:
+            if (G == 1) {
+              pmax[pbase] = l4;
+            } else {
+              run = max(run, l4);
+              if ((c + 1) % G == 0 || c + 1 == nchunks) {
+                pmax[(c / G) * C::NT + static_cast<int>(tid)] = run;
+                run = 0u;
+              }
+            }
+        }
+      });
+      if (!ok) return;
+      // ---- lower bound b from the k-th largest part maximum
+      for (int i = tid; i < P; i += C::NT) {
+        const uint32_t key = pmax[i];
+        hist_add(hist, key >> C::SHIFT1, true);
+      }
+      __syncthreads();
+      if (warp == 0) find_digit_fn(hist, C::BINS1, static_cast<uint32_t>(topk), &misc[0], &misc[1]);
+      if (tid == 0) misc[4] = 0u;   // candidate count
+      __syncthreads();
+      const uint32_t b_lo = misc[0] << C::SHIFT1;
+      // ---- keep every score >= b_lo
+      uint32_t* cand_n = &misc[4];
+      ok = stream([&](int c, const float* buf) {
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const int off = static_cast<int>(warp) * C::PER_WARP + (static_cast<int>(lane) + 32 * rr) * 4;
+          const float4 v = *reinterpret_cast<const float4*>(buf + off);
+          const float vals[4] = {v.x, v.y, v.z, v.w};
+          uint32_t keys[4], cnt = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            keys[e] = order_key(vals[e]);
+            cnt += (c * C::CHUNK + off + e < n && keys[e] >= b_lo) ? 1u : 0u;
+          }
+          uint32_t tot;
+          const uint32_t pre = warp_excl_scan(cnt, lane, &tot);
+          uint32_t base = 0;
+          if (lane == 0 && tot) base = atomicAdd(cand_n, tot);
+          base = __shfl_sync(0xFFFFFFFFu, base, 0) + pre;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (c * C::CHUNK + off + e < n && keys[e] >= b_lo) {
+              if (base < static_cast<uint32_t>(C::CAP)) {
+                ckey[base] = keys[e];
+                cidx[base] = c * C::CHUNK + off + e;
+              }
+              ++base;
+            }
+          }
+        }
+      });
+      if (!ok) return;
+      const uint32_t nc = *cand_n;
+      if (nc <= static_cast<uint32_t>(C::CAP)) {
+        // ---- exact k-th largest key among the candidates (digits 11, 11, 10 bits)
+        auto select = [&](auto&& key_of, auto&& use, uint32_t kth, uint32_t* out_thr, uint32_t* out_rem) {
+          uint32_t prefix = 0, remaining = kth;
+          const int shifts[3] = {21, 10, 0};
+          const int widths[3] = {11, 11, 10};
+          for (int d = 0; d < 3; ++d) {
+            const int shift = shifts[d], bits = widths[d];
+            const int hi = shift + bits;
+            for (int i = tid; i < (1 << bits); i += C::NT) hist[i] = 0u;
+            __syncthreads();
+            for (uint32_t base = 0; base < nc; base += C::NT) {
+              const uint32_t i = base + tid;
+              const bool in = i < nc && use(i);
+              const uint32_t key = in ? key_of(i) : 0u;
+              const bool m = in && (hi >= 32 || (key >> hi) == (prefix >> hi));
+              hist_add(hist, (key >> shift) & ((1u << bits) - 1u), m);
+            }
+            __syncthreads();
+            if (warp == 0) find_digit_fn(hist, 1 << bits, remaining, &misc[2], &misc[3]);
+            __syncthreads();
+            prefix |= misc[2] << shift;
+            remaining -= misc[3];
+            __syncthreads();
+          }
+          *out_thr = prefix;
+          *out_rem = remaining;
+        };
+        uint32_t thr, need_eq;
+        select([&](uint32_t i) { return ckey[i]; }, [&](uint32_t) { return true; },
+               static_cast<uint32_t>(topk), &thr, &need_eq);
+        // ties at the threshold: the need_eq lowest indices (largest ~index)
+        if (tid == 0) misc[5] = 0u;
+        __syncthreads();
+        for (uint32_t i = tid; i < nc; i += C::NT)
+          if (ckey[i] == thr) atomicAdd(&misc[5], 1u);
+        __syncthreads();
+        uint32_t inv_idx_thr = 0u;   // select every tie
+        if (misc[5] > need_eq) {
+          uint32_t rem2;
+          select([&](uint32_t i) { return ~static_cast<uint32_t>(cidx[i]); },
+                 [&](uint32_t i) { return ckey[i] == thr; }, need_eq, &inv_idx_thr, &rem2);
+        }
+        // ---- selection -> bitmap -> indices in increasing order
+        const int nwords = (n + 31) / 32;
+        for (int i = tid; i < nwords; i += C::NT) bitmap[i] = 0u;
+        __syncthreads();
+        for (uint32_t i = tid; i < nc; i += C::NT) {
+          const uint32_t key = ckey[i];
+          const int id = cidx[i];
+          if (key > thr || (key == thr && ~static_cast<uint32_t>(id) >= inv_idx_thr))
+            atomicOr(&bitmap[id >> 5], 1u << (id & 31));
+        }
+        __syncthreads();
+        const int per = (nwords + C::NT - 1) / C::NT;
+        const int w0 = min(nwords, static_cast<int>(tid) * per), w1 = min(nwords, w0 + per);
+        uint32_t cnt = 0;
+        for (int wdx = w0; wdx < w1; ++wdx) cnt += __popc(bitmap[wdx]);
+        uint32_t wt;
+        const uint32_t pre = warp_excl_scan(cnt, lane, &wt);
+        if (lane == 31) wtot[warp] = pre + cnt;
+        __syncthreads();
+        uint32_t pos_out = pre;
+        for (int w = 0; w < static_cast<int>(warp); ++w) pos_out += wtot[w];
+        for (int wdx = w0; wdx < w1; ++wdx) {
+          uint32_t bits = bitmap[wdx];
+          while (bits) {
+            const int bpos = __ffs(bits) - 1;
+            bits &= bits - 1;
+            out[pos_out++] = wdx * 32 + bpos;
+          }
+        }
+        return;
+      }
+      __syncthreads();   // candidates overflowed: the exact path below
+    }
+  }
+  for (int i = tid; i < C::NW * (C::BINS1 / 2); i += C::NT) reinterpret_cast<uint32_t*>(smem + C::OFF_WHIST)[i] = 0u;
+  for (int i = tid; i < C::BINS1; i += C::NT) hist[i] = 0u;
+  __syncthreads();
+
   // ------------------------------------------------------------------ pass 1
   bool ok = stream([&](int c, const float* buf) {
 #pragma unroll
@@ -232,27 +456,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
   }
   __syncthreads();
 
-  // k-th largest lies in bin B: lane l scans bins 2047-64l .. 1984-64l (descending)
-  auto find_digit = [&](const uint32_t* h, int nbins, uint32_t need, uint32_t* digit, uint32_t* above) {
-    const int per = nbins / 32;
-    uint32_t sum = 0;
-    for (int j = 0; j < per; ++j) sum += h[nbins - 1 - per * static_cast<int>(lane) - j];
-    uint32_t tot;
-    const uint32_t excl = warp_excl_scan(sum, lane, &tot);
-    if (excl < need && need <= excl + sum) {
-      uint32_t acc = excl;
-      for (int j = 0; j < per; ++j) {
-        const uint32_t cnt = h[nbins - 1 - per * static_cast<int>(lane) - j];
-        if (acc + cnt >= need) {
-          *digit = static_cast<uint32_t>(nbins - 1 - per * static_cast<int>(lane) - j);
-          *above = acc;
-          break;
-        }
-        acc += cnt;
-      }
-    }
-  };
-  if (warp == 0) find_digit(hist, C::BINS1, static_cast<uint32_t>(topk), &misc[0], &misc[1]);
+  if (warp == 0) find_digit_fn(hist, C::BINS1, static_cast<uint32_t>(topk), &misc[0], &misc[1]);
   __syncthreads();
   const uint32_t bin_b = misc[0];
   const uint32_t above = misc[1];
@@ -316,7 +520,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
       if (!ok) return;
     }
     __syncthreads();
-    if (warp == 0) find_digit(hist, 1 << bits, remaining, &misc[2], &misc[3]);
+    if (warp == 0) find_digit_fn(hist, 1 << bits, remaining, &misc[2], &misc[3]);
     __syncthreads();
     prefix |= misc[2] << shift;
     remaining -= misc[3];

@@ -51,6 +51,8 @@ TOPK_CASES = [
     ((1,) * 4, (3000, 20000, 65, 131072), 2048, None),
     ((6, 1), (70, 40), 32, 1),
     ((3,), (9000,), 2048, 0),           # every score equal: the lowest indices win
+    ((1, 1), (200000, 300000), 2048, None),   # grouped part maxima; a row past the bitmap
+    ((2,), (100000,), 64, 40),          # small k on a long row, ties
 ]
 
 
