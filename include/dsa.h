@@ -164,6 +164,40 @@ dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
                        int32_t* idx_out, void* workspace, size_t workspace_bytes,
                        cudaStream_t stream);
 
+/*
+ * dsa_forward without a caller-provided workspace, for callers that cannot
+ * allocate device memory: code whose device memory belongs to a host
+ * framework or a preallocated pool that forbids cudaMalloc once serving has
+ * started, or a latency-critical loop that cannot afford the device-wide
+ * synchronisation cudaMalloc/cudaFree imply.  The pages describe no such
+ * entry point; it exists only for those callers.
+ *
+ * Scratch (the fp32 scores and int32 selections of one pass) lives in one
+ * file-scope device array of DSA_STATIC_SCRATCH_BYTES, which every GPU that
+ * loads the library keeps until the process exits.  Inputs and outputs are
+ * still the caller's, exactly as for dsa_forward; the query rows are processed
+ * in the largest passes whose scratch fits the array.  Returns
+ * DSA_ERR_WORKSPACE (nothing launched) when even one query row's scores and
+ * selections do not fit, i.e. when the longest kv_len reaches ~8M keys.
+ * Calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls on a device share the array and it
+ * keeps the last call's contents; nothing in it needs to start at zero (every
+ * score and selection is written before it is read).  Calls whose kernels
+ * overlap on the GPU (other streams, other host threads) race on the array:
+ * serialise them.
+ */
+#define DSA_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+dsa_status dsa_forward_static_scratch(const void* q_idx, const float* w, const void* k_idx,
+                                      const float* k_scale, dsa_kidx_dtype k_dtype,
+                                      const void* q, const void* latent, dsa_varlen v,
+                                      int32_t n_idx_heads, int32_t idx_dim, int32_t topk,
+                                      int32_t n_heads, int32_t d_qk, int32_t d_v, float scale,
+                                      void* out, float* lse, int32_t* idx_out,
+                                      cudaStream_t stream);
+
 /* Reads and clears the device error word of the current device (synchronises
  * `stream` first).  *code = 0 when no device-side wait gave up. */
 dsa_status dsa_device_error(int32_t* code, cudaStream_t stream);

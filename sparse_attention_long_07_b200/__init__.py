@@ -65,13 +65,20 @@ def _load():
     lib.dsa_debug_wait_profile.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
                                            ctypes.c_int32, ctypes.c_int32]
     lib.dsa_debug_wait_profile.restype = ctypes.c_int
+    lib.dsa_forward_static_scratch.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp, dsa_varlen, i32, i32, i32,
+                                               i32, i32, i32, f32, vp, vp, vp, vp]
+    lib.dsa_forward_static_scratch.restype = ctypes.c_int
     for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward", "dsa_device_error"):
         getattr(lib, fn).restype = ctypes.c_int
     return lib
 
 
 EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward_workspace_size",
-            "dsa_forward", "dsa_device_error", "dsa_status_string", "dsa_version", "dsa_debug_wait_profile")
+            "dsa_forward", "dsa_device_error", "dsa_status_string", "dsa_version", "dsa_debug_wait_profile",
+            "dsa_forward_static_scratch")
+
+# bytes of the library's static scratch array (DSA_STATIC_SCRATCH_BYTES in include/dsa.h)
+DSA_STATIC_SCRATCH_BYTES = 32 << 20
 
 _lib = _load()
 
@@ -179,6 +186,21 @@ def dsa_forward(q_idx, w, k_idx, k_scale, q, latent, v: Varlen, topk, scale, out
                             _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(workspace),
                             0 if workspace is None else workspace.numel() * workspace.element_size(),
                             _stream(stream)), "dsa_forward")
+    return out, lse
+
+
+def dsa_forward_static_scratch(q_idx, w, k_idx, k_scale, q, latent, v: Varlen, topk, scale, out, lse,
+                               idx_out=None, stream=None):
+    """dsa_forward for callers that cannot allocate device memory: the scratch
+    is the library's own static device array (see include/dsa.h for who needs
+    this, the size limit, and why overlapping calls must be serialised)."""
+    T, H_I, d_I = q_idx.shape
+    _, H, d_qk = q.shape
+    d_v = out.shape[-1]
+    _check(_lib.dsa_forward_static_scratch(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _kdtype(k_idx),
+                                           _ptr(q), _ptr(latent), v.c(), H_I, d_I, topk, H, d_qk, d_v,
+                                           float(scale), _ptr(out), _ptr(lse), _ptr(idx_out), _stream(stream)),
+           "dsa_forward_static_scratch")
     return out, lse
 
 

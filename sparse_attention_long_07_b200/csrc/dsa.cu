@@ -462,6 +462,50 @@ dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
   return DSA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Forward for callers that cannot allocate: the workspace is a file-scope
+// device array instead of caller memory (contract in include/dsa.h).
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_dsa_static_scratch[DSA_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::once_flag g_scratch_once[kMaxDevices];
+void* g_scratch_ptr[kMaxDevices];
+cudaError_t g_scratch_err[kMaxDevices];
+}  // namespace
+
+dsa_status dsa_forward_static_scratch(const void* q_idx, const float* w, const void* k_idx,
+                                      const float* k_scale, dsa_kidx_dtype k_dtype,
+                                      const void* q, const void* latent, dsa_varlen v,
+                                      int32_t n_idx_heads, int32_t idx_dim, int32_t topk,
+                                      int32_t n_heads, int32_t d_qk, int32_t d_v, float scale,
+                                      void* out, float* lse, int32_t* idx_out,
+                                      cudaStream_t stream) {
+  if (v.batch < 1 || !v.cu_q_host) return DSA_ERR_INVALID_ARG;
+  // largest pass (query rows) whose scores + selections fit the array
+  const size_t per_pass_one = dsa_forward_workspace_size(v, topk, 1);
+  if (per_pass_one == 0) return DSA_ERR_INVALID_ARG;
+  if (per_pass_one > DSA_STATIC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE;
+  const int64_t T = v.cu_q_host[v.batch];
+  int64_t lo = 1, hi = T > 1 ? T : 1;     // dsa_forward_workspace_size is monotone in the pass size
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo + 1) / 2;
+    if (dsa_forward_workspace_size(v, topk, mid) <= DSA_STATIC_SCRATCH_BYTES) lo = mid; else hi = mid - 1;
+  }
+  const int64_t q_chunk = lo;
+  // the array's device address, looked up once per device with that device current
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::call_once(g_scratch_once[dev], [dev] {
+    g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_ptr[dev], g_dsa_static_scratch);
+  });
+  if (g_scratch_err[dev] != cudaSuccess || g_scratch_ptr[dev] == nullptr) return DSA_ERR_CUDA;
+  return dsa_forward(q_idx, w, k_idx, k_scale, k_dtype, q, latent, v, n_idx_heads, idx_dim, topk, n_heads,
+                     d_qk, d_v, scale, q_chunk, out, lse, idx_out, g_scratch_ptr[dev], DSA_STATIC_SCRATCH_BYTES,
+                     stream);
+}
+
 dsa_status dsa_device_error(int32_t* code, cudaStream_t stream) {
   if (!code) return DSA_ERR_INVALID_ARG;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return DSA_ERR_CUDA;
