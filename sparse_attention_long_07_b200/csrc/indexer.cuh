@@ -62,7 +62,8 @@ struct IndexerCfg {
   static constexpr int PRODUCER_WARP = 4 * EPI_WG;
   static constexpr int MMA_WARP = PRODUCER_WARP + 1;
   static constexpr int CONVERT_WARP0 = MMA_WARP + 1;
-  static constexpr int NWARPS = MMA_WARP + 1 + (KFP8 ? 4 : 0);
+  static constexpr int CONV_TEAMS = PERSIST ? 2 : 1;      // e4m3 converter teams (alternate tiles)
+  static constexpr int NWARPS = MMA_WARP + 1 + (KFP8 ? 4 * CONV_TEAMS : 0);
   static constexpr int NT = NWARPS * 32;
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, N, false, false);
   // shared memory layout (offsets from a 1024-byte aligned base)
@@ -74,12 +75,17 @@ struct IndexerCfg {
   static constexpr int NBAR = 2 + 2 * STAGES + 2 * RSTAGES + 4 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_UPRE = OFF_MISC + 16;          // persistent: unit prefix per sequence
-  static constexpr int SMEM_BYTES = OFF_UPRE + (PERSIST ? (MAX_SEQ + 1) * 4 : 0) + 1024;  // + alignment slack
+  // persistent: per-warp head weights, read as float4 (16-byte aligned)
+  static constexpr int OFF_WEPI = (OFF_UPRE + (PERSIST ? (MAX_SEQ + 1) * 4 : 0) + 15) / 16 * 16;
+  static constexpr int SMEM_BYTES = OFF_WEPI + (PERSIST ? 4 * EPI_WG * H_I * 4 : 0) + 1024;  // + alignment slack
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
   static_assert(B_TILE % 1024 == 0 && A_TILE % 1024 == 0, "atom alignment");
   static_assert(COLS_PER_THREAD % LD_CHUNK == 0, "TMEM load chunking");
   static_assert(!KFP8 || D_I == 128, "e4m3 keys: 128-byte rows");
   static_assert(!PERSIST || NQ == 1, "persistent schedule: one query per sequence block");
+  static_assert(OFF_K % 1024 == 0 && OFF_RAW % 1024 == 0, "swizzled tiles on 1024-byte boundaries");
+  static_assert(OFF_WEPI % 16 == 0 && OFF_W % 16 == 0, "16-byte vector accesses");
+  static_assert(OFF_BAR % 8 == 0 && OFF_UPRE % 4 == 0, "barrier / prefix alignment");
 };
 
 // One key row of a raw e4m3 tile (128 bytes, 128-byte TMA swizzle) -> the
@@ -255,6 +261,8 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
+    const uint64_t a_desc0 = smem_desc(s_k, 16, 8 * C::SWB, C::SWZ);
+    const uint64_t b_desc0 = smem_desc(s_q, 16, 8 * C::SWB, C::SWZ);
     if (lane == 0) {
       if (mbar_wait(bar_q_full, 0, abort_flag, 13)) {
         tc_fence_after();
@@ -264,13 +272,13 @@ __global__ void __launch_bounds__(C::NT, 1)
           if (!mbar_wait(bar_k_full(s), (it / C::STAGES) & 1, abort_flag, 14)) break;
           if (!mbar_wait(bar_acc_empty(a), ((it >> 1) & 1) ^ 1, abort_flag, 15)) break;
           tc_fence_after();
-          const uint32_t a_base = s_k + s * C::A_TILE;
+          const uint64_t a_stage = a_desc0 + static_cast<uint64_t>((s * C::A_TILE) >> 4);
 #pragma unroll
           for (int kk = 0; kk < C::KSTEPS; ++kk) {
             const int atom = (kk * 32) / C::SWB;
             const int off = (kk * 32) % C::SWB;
-            const uint64_t ad = smem_desc(a_base + atom * C::BK * C::SWB + off, 16, 8 * C::SWB, C::SWZ);
-            const uint64_t bd = smem_desc(s_q + atom * C::N * C::SWB + off, 16, 8 * C::SWB, C::SWZ);
+            const uint64_t ad = a_stage + static_cast<uint64_t>((atom * C::BK * C::SWB + off) >> 4);
+            const uint64_t bd = b_desc0 + static_cast<uint64_t>((atom * C::N * C::SWB + off) >> 4);
             umma_ss(tmem + a * C::N, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar_k_empty(s));
@@ -383,6 +391,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
     upre[b + 1] = cnt;
   }
+  DSA_PROF_BEGIN();
   __syncthreads();
   if (threadIdx.x == 0) {
     upre[0] = 0;
@@ -467,6 +476,7 @@ __global__ void __launch_bounds__(C::NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const long long t_role = clock64();
 
   if (warp == C::PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producer
@@ -502,8 +512,11 @@ __global__ void __launch_bounds__(C::NT, 1)
           }
       }
     }
+    if (lane == 0) DSA_PROF_SPAN(61, t_role);
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
+    const uint64_t a_desc0 = smem_desc(s_k, 16, 8 * C::SWB, C::SWZ);
+    const uint64_t b_desc0 = smem_desc(s_q, 16, 8 * C::SWB, C::SWZ);
     if (lane == 0) {
       int b = b_first, seg = -1, cur = -1;
       for (int it = 0; it < n_iter; ++it) {
@@ -520,19 +533,22 @@ __global__ void __launch_bounds__(C::NT, 1)
         if (!mbar_wait(bar_k_full(s), (it / C::STAGES) & 1, abort_flag, 53)) break;
         if (!mbar_wait(bar_acc_empty(a), ((it >> 1) & 1) ^ 1, abort_flag, 54)) break;
         tc_fence_after();
-        const uint32_t a_base = s_k + s * C::A_TILE;
+        // descriptors: the start-address field (16-byte units, low bits) advances
+        // by the stage and k-step offsets; it never carries (addresses < 256 KB)
+        const uint64_t a_stage = a_desc0 + static_cast<uint64_t>((s * C::A_TILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const int atom = (kk * 32) / C::SWB;
           const int off = (kk * 32) % C::SWB;
-          const uint64_t ad = smem_desc(a_base + atom * C::BK * C::SWB + off, 16, 8 * C::SWB, C::SWZ);
-          const uint64_t bd = smem_desc(s_q + atom * C::N * C::SWB + off, 16, 8 * C::SWB, C::SWZ);
+          const uint64_t ad = a_stage + static_cast<uint64_t>((atom * C::BK * C::SWB + off) >> 4);
+          const uint64_t bd = b_desc0 + static_cast<uint64_t>((atom * C::N * C::SWB + off) >> 4);
           umma_ss(tmem + a * C::N, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_k_empty(s));
         umma_commit(bar_acc_full(a));
         if (u + 1 == u1 || u + 1 >= upre[b + 1]) umma_commit(bar_q_empty);   // last tile of the sequence
       }
+      DSA_PROF_SPAN(62, t_role);
       umma_commit(bar_drain);
       long long t0 = clock64();
       while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < kWaitLimitCycles) {
@@ -540,8 +556,9 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
   } else if (warp >= C::CONVERT_WARP0) {
     // ------------------------------------------------------------ e4m3 -> bf16
-    const int row = threadIdx.x - C::CONVERT_WARP0 * 32;
-    for (int it = 0; it < n_iter; ++it) {
+    const int team = (warp - C::CONVERT_WARP0) / 4;
+    const int row = threadIdx.x - (C::CONVERT_WARP0 + 4 * team) * 32;
+    for (int it = team; it < n_iter; it += C::CONV_TEAMS) {
       const int r = it % C::RSTAGES;
       const int s = it % C::STAGES;
       if (!mbar_wait(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag, 55)) break;
@@ -552,6 +569,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       fence_proxy_async_smem();
       mbar_arrive(bar_k_full(s));
     }
+    if (lane == 0) DSA_PROF_SPAN(63, t_role);
   } else {
     // ------------------------------------------------------------ epilogue
     // Warpgroup g drains accumulator g, i.e. tiles it = g, g+2, ...; the key
@@ -561,7 +579,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     const int key_in_tile = sub * 32 + lane;
     int b = b_first, cur = -1, bp = b_first;
     Seq q{};
-    float wreg[C::H_I];
+    float* wsm = reinterpret_cast<float*>(smem + C::OFF_WEPI) + warp * C::H_I;   // this warp's copy
     auto fetch_scale = [&](int itx) -> float {
       if (itx >= n_iter) return 0.f;
       const int u = u0 + itx;
@@ -578,15 +596,10 @@ __global__ void __launch_bounds__(C::NT, 1)
       if (b != cur) {
         cur = b;
         q = seq_of(b);
+        __syncwarp();
         const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(q.q0) * C::H_I);
-#pragma unroll
-        for (int j = 0; j < C::H_I / 4; ++j) {
-          const float4 v = w4[j];
-          wreg[4 * j] = v.x;
-          wreg[4 * j + 1] = v.y;
-          wreg[4 * j + 2] = v.z;
-          wreg[4 * j + 3] = v.w;
-        }
+        if (lane < C::H_I / 4) reinterpret_cast<float4*>(wsm)[lane] = w4[lane];
+        __syncwarp();
       }
       if (!mbar_wait_warp(bar_acc_full(g), (it >> 1) & 1, abort_flag, 57)) break;
       tc_fence_after();
@@ -598,9 +611,12 @@ __global__ void __launch_bounds__(C::NT, 1)
         tmem_ld32(t_row + 32 * half, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          acc0 = fmaf(wreg[32 * half + j], fmaxf(__uint_as_float(v[j]), 0.f), acc0);
-          acc1 = fmaf(wreg[32 * half + j + 1], fmaxf(__uint_as_float(v[j + 1]), 0.f), acc1);
+        for (int j = 0; j < 32; j += 4) {
+          const float4 wv = reinterpret_cast<const float4*>(wsm)[(32 * half + j) / 4];
+          acc0 = fmaf(wv.x, fmaxf(__uint_as_float(v[j]), 0.f), acc0);
+          acc1 = fmaf(wv.y, fmaxf(__uint_as_float(v[j + 1]), 0.f), acc1);
+          acc0 = fmaf(wv.z, fmaxf(__uint_as_float(v[j + 2]), 0.f), acc0);
+          acc1 = fmaf(wv.w, fmaxf(__uint_as_float(v[j + 3]), 0.f), acc1);
         }
       }
       tc_fence_before();
@@ -612,6 +628,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
       ks = ks_next;
     }
+    if (lane == 0) DSA_PROF_SPAN(60, t_role);
   }
 
   tc_fence_before();
@@ -620,6 +637,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  DSA_PROF_END();
 }
 
 }  // namespace dsa

@@ -20,10 +20,44 @@ enum DeviceErrorCode : int {
 };
 
 #ifdef DSA_PROFILE_WAITS
-// Profiling builds only: cycles spent and waits completed per wait site.
+// Profiling builds only: cycles spent and waits completed per wait site (and
+// per role span), accumulated per CTA in shared memory and added to these
+// device counters once per CTA.
 constexpr int kWaitSites = 64;
 __device__ unsigned long long g_wait_cycles[kWaitSites];
 __device__ unsigned long long g_wait_count[kWaitSites];
+__device__ __forceinline__ unsigned long long* prof_acc() {
+  __shared__ unsigned long long acc[2 * kWaitSites];
+  return acc;
+}
+__device__ __forceinline__ void prof_add(int site, long long cycles) {
+  if (site > 0 && site < kWaitSites) {
+    atomicAdd(&prof_acc()[site], static_cast<unsigned long long>(cycles));
+    atomicAdd(&prof_acc()[kWaitSites + site], 1ull);
+  }
+}
+#define DSA_PROF_BEGIN()                                                                   \
+  for (int i_ = threadIdx.x; i_ < 2 * ::dsa::kWaitSites; i_ += blockDim.x) ::dsa::prof_acc()[i_] = 0ull
+#define DSA_PROF_END()                                                                     \
+  do {                                                                                    \
+    __syncthreads();                                                                      \
+    for (int i_ = threadIdx.x; i_ < ::dsa::kWaitSites; i_ += blockDim.x)                   \
+      if (::dsa::prof_acc()[::dsa::kWaitSites + i_]) {                                     \
+        atomicAdd(&::dsa::g_wait_cycles[i_], ::dsa::prof_acc()[i_]);                        \
+        atomicAdd(&::dsa::g_wait_count[i_], ::dsa::prof_acc()[::dsa::kWaitSites + i_]);     \
+      }                                                                                   \
+  } while (0)
+#define DSA_PROF_SPAN(site, t0) ::dsa::prof_add((site), clock64() - (t0))
+#else
+#define DSA_PROF_BEGIN() \
+  do {                   \
+  } while (0)
+#define DSA_PROF_END() \
+  do {                 \
+  } while (0)
+#define DSA_PROF_SPAN(site, t0) \
+  do {                          \
+  } while (0)
 #endif
 
 // ~2 s at the 1.9 GHz boost clock: far above any legitimate wait in these kernels.
@@ -123,10 +157,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     bool ok = kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
     if (ok) {
 #ifdef DSA_PROFILE_WAITS
-      if ((threadIdx.x & 31) == 0 && site > 0 && site < kWaitSites) {
-        atomicAdd(&g_wait_cycles[site], static_cast<unsigned long long>(clock64() - t_enter));
-        atomicAdd(&g_wait_count[site], 1ull);
-      }
+      if ((threadIdx.x & 31) == 0) prof_add(site, clock64() - t_enter);
 #endif
       return true;
     }

@@ -82,6 +82,8 @@ struct MlaCfg {
   static_assert(SPLIT == 1 || NV <= NA1, "rank 1 must gather its value columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(TMEM_USED <= 512, "tensor memory");
+  static_assert(OFF_C % 1024 == 0 && C_STAGE % 1024 == 0 && C_ATOM_BYTES % 1024 == 0, "swizzle atoms");
+  static_assert(OFF_X % 16 == 0 && OFF_BAR % 8 == 0, "vector / barrier alignment");
 };
 
 struct MlaParams {
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_lat);
   }
+  DSA_PROF_BEGIN();
   __syncthreads();
   // Tiles up to the last one holding a valid entry (trailing -1 padding is skipped).
   {
@@ -190,6 +193,7 @@ __global__ void __launch_bounds__(C::NT, 1)
   if (C::SPLIT == 2) skip = skip || ld_cluster_u32(mapa_shared(smem_u32(pending_s), peer)) != 0u;
   const int n_tiles = skip ? 0 : *ntiles_s;
 
+  const long long t_role = clock64();
   if (warp == C::PRODUCER_WARP) {
     // ------------------------------------------------------------ gather producer
     int it = 0;
@@ -236,6 +240,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
       }
     }
+    if (lane == 0) DSA_PROF_SPAN(61, t_role);
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_tiles > 0) {
@@ -283,6 +288,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
     }
     if (lane == 0) {
+      DSA_PROF_SPAN(62, t_role);
       umma_commit(bar_drain);
       long long t0 = clock64();
       while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < kWaitLimitCycles) {
@@ -405,6 +411,7 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
       for (int c = 0; c < C::BN; ++c) sv[c] = s_next[c];
     }
+    if (lane == 0) DSA_PROF_SPAN(63, t_role);
     // ------------------------------------------------------------ epilogue
     const int t_out = static_cast<int>(t);
     if (ok && n_tiles > 0) {
@@ -446,9 +453,11 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
   }
 
+  if (lane == 0 && warp < 4) DSA_PROF_SPAN(60, t_role);
   tc_fence_before();
   __syncthreads();
   if (C::SPLIT == 2) cluster_sync();   // no remote access into this CTA after this point
+  DSA_PROF_END();
   if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);

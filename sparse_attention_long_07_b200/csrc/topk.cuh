@@ -51,6 +51,8 @@ struct TopkCfg {
   static constexpr int OFF_MISC = OFF_BAR + STAGES * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 128;   // + alignment slack
   static_assert(PMAX_CAP * 4 + BITMAP_BITS / 8 <= NW * (BINS1 / 2) * 4, "fast-path union fits");
+  static_assert(OFF_RING % 128 == 0 && (CHUNK * 4) % 128 == 0, "bulk-copy destinations");
+  static_assert(OFF_BAR % 8 == 0 && OFF_MISC % 8 == 0, "barrier alignment");
 };
 
 __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t lane, uint32_t* total) {
@@ -98,6 +100,13 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  DSA_PROF_BEGIN();
+  long long t_phase = clock64();
+  // profiling builds: cycles of each phase (thread 0), sites 41..47
+  auto phase = [&](int site) {
+    if (tid == 0) DSA_PROF_SPAN(site, t_phase);
+    t_phase = clock64();
+  };
   uint32_t* whist = reinterpret_cast<uint32_t*>(smem + C::OFF_WHIST) + warp * (C::BINS1 / 2);
   __syncthreads();
 
@@ -212,26 +221,40 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     eq_base += ctot >> 16;
   };
 
-  // digit of the `need`-th largest entry: lane l scans bins nbins-1-per*l .. (descending)
+  // Digit of the `need`-th largest entry of a histogram h[nbins] (nbins <= 4 NT):
+  // thread t owns the bins nbins-1-4t .. nbins-4-4t (descending), a CTA-wide
+  // exclusive scan gives the count above each thread's bins, and the thread
+  // whose range crosses `need` writes the digit and the count above it.
+  // Called by every thread of the CTA (it contains __syncthreads).
   auto find_digit_fn = [&](const uint32_t* h, int nbins, uint32_t need, uint32_t* digit, uint32_t* above) {
-    const int per = nbins / 32;
-    uint32_t sum = 0;
-    for (int j = 0; j < per; ++j) sum += h[nbins - 1 - per * static_cast<int>(lane) - j];
-    uint32_t tot;
-    const uint32_t excl = warp_excl_scan(sum, lane, &tot);
-    if (excl < need && need <= excl + sum) {
+    const int top = nbins - 1 - 4 * static_cast<int>(tid);
+    uint32_t c4[4], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      c4[j] = top - j >= 0 ? h[top - j] : 0u;
+      sum += c4[j];
+    }
+    uint32_t wt;
+    const uint32_t pre = warp_excl_scan(sum, lane, &wt);
+    if (lane == 31) wtot[warp] = pre + sum;
+    __syncthreads();
+    uint32_t excl = pre;
+    for (int w = 0; w < static_cast<int>(warp); ++w) excl += wtot[w];
+    if (top >= 0 && excl < need && need <= excl + sum) {
       uint32_t acc = excl;
-      for (int j = 0; j < per; ++j) {
-        const uint32_t cnt = h[nbins - 1 - per * static_cast<int>(lane) - j];
-        if (acc + cnt >= need) {
-          *digit = static_cast<uint32_t>(nbins - 1 - per * static_cast<int>(lane) - j);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (acc + c4[j] >= need) {
+          *digit = static_cast<uint32_t>(top - j);
           *above = acc;
           break;
         }
-        acc += cnt;
+        acc += c4[j];
       }
     }
+    __syncthreads();
   };
+
   // ================================================================== fast path
   // Split the row into parts of PS scores (part = PS consecutive scores of one
   // thread's 16 per chunk, or one thread's scores over G chunks).  At least k
@@ -306,81 +329,89 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
             }
         }
       });
-      if (!ok) return;
-      // ---- lower bound b from the k-th largest part maximum
-      for (int i = tid; i < P; i += C::NT) {
-        const uint32_t key = pmax[i];
-        hist_add(hist, key >> C::SHIFT1, true);
-      }
-      __syncthreads();
-      if (warp == 0) find_digit_fn(hist, C::BINS1, static_cast<uint32_t>(topk), &misc[0], &misc[1]);
+      phase(41);
+      if (!ok) { DSA_PROF_END(); return; }
+    // exact kth-largest key among entries i < count with use(i) (digits of 11, 11, 10 bits)
+    auto select = [&](uint32_t count, auto&& key_of, auto&& use, uint32_t kth, uint32_t* out_thr,
+                      uint32_t* out_rem) {
+        uint32_t prefix = 0, remaining = kth;
+        const int shifts[3] = {21, 10, 0};
+        const int widths[3] = {11, 11, 10};
+        for (int d = 0; d < 3; ++d) {
+          const int shift = shifts[d], bits = widths[d];
+          const int hi = shift + bits;
+          for (int i = tid; i < (1 << bits); i += C::NT) hist[i] = 0u;
+          __syncthreads();
+          for (uint32_t base = 0; base < count; base += C::NT) {
+            const uint32_t i = base + tid;
+            const bool in = i < count && use(i);
+            const uint32_t key = in ? key_of(i) : 0u;
+            const bool m = in && (hi >= 32 || (key >> hi) == (prefix >> hi));
+            hist_add(hist, (key >> shift) & ((1u << bits) - 1u), m);
+          }
+          __syncthreads();
+          find_digit_fn(hist, 1 << bits, remaining, &misc[2], &misc[3]);
+          __syncthreads();
+          prefix |= misc[2] << shift;
+          remaining -= misc[3];
+          __syncthreads();
+        }
+        *out_thr = prefix;
+        *out_rem = remaining;
+      };
+      // ---- lower bound b = the k-th largest part maximum (exact)
+      uint32_t b_lo, unused_rem;
+      select(static_cast<uint32_t>(P), [&](uint32_t i) { return pmax[i]; }, [&](uint32_t) { return true; },
+             static_cast<uint32_t>(topk), &b_lo, &unused_rem);
       if (tid == 0) misc[4] = 0u;   // candidate count
       __syncthreads();
-      const uint32_t b_lo = misc[0] << C::SHIFT1;
+      phase(42);
       // ---- keep every score >= b_lo
       uint32_t* cand_n = &misc[4];
       ok = stream([&](int c, const float* buf) {
+        // one ballot per element slot, one atomic per warp and chunk
+        uint32_t keys[16], bal[16];
+        uint32_t wsum = 0;
+        const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
         for (int rr = 0; rr < 4; ++rr) {
           const int off = static_cast<int>(warp) * C::PER_WARP + (static_cast<int>(lane) + 32 * rr) * 4;
           const float4 v = *reinterpret_cast<const float4*>(buf + off);
           const float vals[4] = {v.x, v.y, v.z, v.w};
-          uint32_t keys[4], cnt = 0;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            keys[e] = order_key(vals[e]);
-            cnt += (c * C::CHUNK + off + e < n && keys[e] >= b_lo) ? 1u : 0u;
+            keys[rr * 4 + e] = order_key(vals[e]);
+            const bool keep = c * C::CHUNK + off + e < n && keys[rr * 4 + e] >= b_lo;
+            bal[rr * 4 + e] = __ballot_sync(0xFFFFFFFFu, keep);
+            wsum += __popc(bal[rr * 4 + e]);
           }
-          uint32_t tot;
-          const uint32_t pre = warp_excl_scan(cnt, lane, &tot);
+        }
+        if (wsum) {
           uint32_t base = 0;
-          if (lane == 0 && tot) base = atomicAdd(cand_n, tot);
-          base = __shfl_sync(0xFFFFFFFFu, base, 0) + pre;
+          if (lane == 0) base = atomicAdd(cand_n, wsum);
+          base = __shfl_sync(0xFFFFFFFFu, base, 0);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (c * C::CHUNK + off + e < n && keys[e] >= b_lo) {
-              if (base < static_cast<uint32_t>(C::CAP)) {
-                ckey[base] = keys[e];
-                cidx[base] = c * C::CHUNK + off + e;
+          for (int j = 0; j < 16; ++j) {
+            if ((bal[j] >> lane) & 1u) {
+              const uint32_t at = base + __popc(bal[j] & lt);
+              if (at < static_cast<uint32_t>(C::CAP)) {
+                ckey[at] = keys[j];
+                cidx[at] = c * C::CHUNK + static_cast<int>(warp) * C::PER_WARP +
+                           (static_cast<int>(lane) + 32 * (j >> 2)) * 4 + (j & 3);
               }
-              ++base;
             }
+            base += __popc(bal[j]);
           }
         }
       });
-      if (!ok) return;
+      phase(43);
+      if (!ok) { DSA_PROF_END(); return; }
       const uint32_t nc = *cand_n;
       if (nc <= static_cast<uint32_t>(C::CAP)) {
-        // ---- exact k-th largest key among the candidates (digits 11, 11, 10 bits)
-        auto select = [&](auto&& key_of, auto&& use, uint32_t kth, uint32_t* out_thr, uint32_t* out_rem) {
-          uint32_t prefix = 0, remaining = kth;
-          const int shifts[3] = {21, 10, 0};
-          const int widths[3] = {11, 11, 10};
-          for (int d = 0; d < 3; ++d) {
-            const int shift = shifts[d], bits = widths[d];
-            const int hi = shift + bits;
-            for (int i = tid; i < (1 << bits); i += C::NT) hist[i] = 0u;
-            __syncthreads();
-            for (uint32_t base = 0; base < nc; base += C::NT) {
-              const uint32_t i = base + tid;
-              const bool in = i < nc && use(i);
-              const uint32_t key = in ? key_of(i) : 0u;
-              const bool m = in && (hi >= 32 || (key >> hi) == (prefix >> hi));
-              hist_add(hist, (key >> shift) & ((1u << bits) - 1u), m);
-            }
-            __syncthreads();
-            if (warp == 0) find_digit_fn(hist, 1 << bits, remaining, &misc[2], &misc[3]);
-            __syncthreads();
-            prefix |= misc[2] << shift;
-            remaining -= misc[3];
-            __syncthreads();
-          }
-          *out_thr = prefix;
-          *out_rem = remaining;
-        };
         uint32_t thr, need_eq;
-        select([&](uint32_t i) { return ckey[i]; }, [&](uint32_t) { return true; },
+        select(nc, [&](uint32_t i) { return ckey[i]; }, [&](uint32_t) { return true; },
                static_cast<uint32_t>(topk), &thr, &need_eq);
+        phase(44);
         // ties at the threshold: the need_eq lowest indices (largest ~index)
         if (tid == 0) misc[5] = 0u;
         __syncthreads();
@@ -390,7 +421,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
         uint32_t inv_idx_thr = 0u;   // select every tie
         if (misc[5] > need_eq) {
           uint32_t rem2;
-          select([&](uint32_t i) { return ~static_cast<uint32_t>(cidx[i]); },
+          select(nc, [&](uint32_t i) { return ~static_cast<uint32_t>(cidx[i]); },
                  [&](uint32_t i) { return ckey[i] == thr; }, need_eq, &inv_idx_thr, &rem2);
         }
         // ---- selection -> bitmap -> indices in increasing order
@@ -422,9 +453,12 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
             out[pos_out++] = wdx * 32 + bpos;
           }
         }
+        phase(45);
+        DSA_PROF_END();
         return;
       }
       __syncthreads();   // candidates overflowed: the exact path below
+      phase(46);
     }
   }
   for (int i = tid; i < C::NW * (C::BINS1 / 2); i += C::NT) reinterpret_cast<uint32_t*>(smem + C::OFF_WHIST)[i] = 0u;
@@ -444,7 +478,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
       whist_add(order_key(v.w) >> C::SHIFT1, gi + 3 < n);
     }
   });
-  if (!ok) return;
+  if (!ok) { DSA_PROF_END(); return; }
   // merge the per-warp counts
   for (int bin = tid; bin < C::BINS1; bin += C::NT) {
     uint32_t sum = 0;
@@ -456,7 +490,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
   }
   __syncthreads();
 
-  if (warp == 0) find_digit_fn(hist, C::BINS1, static_cast<uint32_t>(topk), &misc[0], &misc[1]);
+  find_digit_fn(hist, C::BINS1, static_cast<uint32_t>(topk), &misc[0], &misc[1]);
   __syncthreads();
   const uint32_t bin_b = misc[0];
   const uint32_t above = misc[1];
@@ -479,7 +513,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
           }
         });
   });
-  if (!ok) return;
+  if (!ok) { DSA_PROF_END(); return; }
   const uint32_t n_eq = eq_base;          // keys in bin B (all of them, even past CAP)
 
   // ------------------------------------------------------------------ refine inside bin B
@@ -517,10 +551,10 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
           count_key(order_key(v.w), gi + 3 < n);
         }
       });
-      if (!ok) return;
+      if (!ok) { DSA_PROF_END(); return; }
     }
     __syncthreads();
-    if (warp == 0) find_digit_fn(hist, 1 << bits, remaining, &misc[2], &misc[3]);
+    find_digit_fn(hist, 1 << bits, remaining, &misc[2], &misc[3]);
     __syncthreads();
     prefix |= misc[2] << shift;
     remaining -= misc[3];
@@ -575,6 +609,8 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
           });
     });
   }
+  phase(47);
+  DSA_PROF_END();
 }
 
 }  // namespace dsa
