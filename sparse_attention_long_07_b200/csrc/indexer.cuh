@@ -46,8 +46,12 @@ struct IndexerCfg {
   static constexpr int NATOM = ROWB / SWB;                // swizzle-atom columns per row
   static constexpr int ATOM_ELEMS = SWB / 2;
   static constexpr int KSTEPS = D_I / 16;
-  static constexpr int STAGES = KFP8 ? (PERSIST ? 3 : 2) : 4;   // bf16 key-tile ring
-  static constexpr int RSTAGES = KFP8 ? (PERSIST ? 6 : 4) : 0;   // raw e4m3 ring
+  // Persistent schedule: the widened bf16 key tile is written to tensor memory
+  // and read from there as the A operand (TS-form MMA), so shared memory holds
+  // only the raw e4m3 ring; otherwise the bf16 tile ring is in shared memory.
+  static constexpr bool K_IN_TMEM = PERSIST;
+  static constexpr int STAGES = K_IN_TMEM ? 4 : (KFP8 ? 2 : 4);  // bf16 key-tile ring
+  static constexpr int RSTAGES = KFP8 ? (PERSIST ? 11 : 4) : 0;  // raw e4m3 ring
   static constexpr int A_TILE = BK * ROWB;
   static constexpr int B_TILE = N * ROWB;
   static constexpr int RAW_TILE = BK * D_I;
@@ -57,7 +61,12 @@ struct IndexerCfg {
   static constexpr int QW = PERSIST ? NQ : NQ / EPI_WG;   // queries per epilogue warpgroup
   static constexpr int COLS_PER_THREAD = QW * H_I;
   static constexpr int LD_CHUNK = COLS_PER_THREAD >= 32 ? 32 : 16;
-  static constexpr int TMEM_COLS = pow2_at_least(2 * N, 32);
+  // fp32 accumulators: the persistent schedule keeps four in flight so that
+  // the MMAs of the next tiles never wait for the epilogue of the last one
+  static constexpr int NACC = PERSIST ? 4 : 2;
+  static constexpr int ACC_COLS = NACC * N;
+  static constexpr int A_COLS = D_I / 2;                  // one bf16 key tile in tensor memory
+  static constexpr int TMEM_COLS = pow2_at_least(ACC_COLS + (K_IN_TMEM ? STAGES * A_COLS : 0), 32);
   static constexpr int EPI_THREADS = 128 * EPI_WG;
   static constexpr int PRODUCER_WARP = 4 * EPI_WG;
   static constexpr int MMA_WARP = PRODUCER_WARP + 1;
@@ -69,10 +78,10 @@ struct IndexerCfg {
   // shared memory layout (offsets from a 1024-byte aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + B_TILE;
-  static constexpr int OFF_RAW = OFF_K + STAGES * A_TILE;
+  static constexpr int OFF_RAW = OFF_K + (K_IN_TMEM ? 0 : STAGES * A_TILE);
   static constexpr int OFF_W = OFF_RAW + RSTAGES * RAW_TILE;
   static constexpr int OFF_BAR = OFF_W + NQ * H_I * 4;
-  static constexpr int NBAR = 2 + 2 * STAGES + 2 * RSTAGES + 4 + 1;
+  static constexpr int NBAR = 2 + 2 * STAGES + 2 * RSTAGES + 2 * NACC + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_UPRE = OFF_MISC + 16;          // persistent: unit prefix per sequence
   // persistent: per-warp head weights, read as float4 (16-byte aligned)
@@ -82,6 +91,10 @@ struct IndexerCfg {
   static_assert(B_TILE % 1024 == 0 && A_TILE % 1024 == 0, "atom alignment");
   static_assert(COLS_PER_THREAD % LD_CHUNK == 0, "TMEM load chunking");
   static_assert(!KFP8 || D_I == 128, "e4m3 keys: 128-byte rows");
+  static_assert(TMEM_COLS <= 512, "tensor memory columns");
+  static_assert(!K_IN_TMEM || (KFP8 && STAGES % CONV_TEAMS == 0), "converter teams own alternate stages");
+  static_assert(NACC % EPI_WG == 0, "each accumulator is drained by one epilogue warpgroup");
+  static_assert(!K_IN_TMEM || STAGES == NACC, "key stage and accumulator of a tile share one barrier");
   static_assert(!PERSIST || NQ == 1, "persistent schedule: one query per sequence block");
   static_assert(OFF_K % 1024 == 0 && OFF_RAW % 1024 == 0, "swizzled tiles on 1024-byte boundaries");
   static_assert(OFF_WEPI % 16 == 0 && OFF_W % 16 == 0, "16-byte vector accesses");
@@ -124,6 +137,26 @@ __device__ __forceinline__ void e4m3_row_to_bf16(const uint8_t* raw_row, uint8_t
       *reinterpret_cast<uint4*>(dst) = make_uint4(outw[4 * h], outw[4 * h + 1], outw[4 * h + 2], outw[4 * h + 3]);
     }
   }
+}
+
+// Four e4m3 bytes -> four bf16 values (two bf16x2 words, lower element in the
+// low half), with integer and bf16 arithmetic only.  PRMT puts each byte in
+// the low byte of a 16-bit half and fills the high byte with copies of its
+// sign bit; shifting left by 4 and masking leaves the sign in bit 15 and the
+// byte's 4 exponent and 3 mantissa bits in bits 10..4.  Read as bf16 that is
+// 2^(e-127)(1 + m/8), or 2^-126 (m/8) when e = 0, and one multiplication by
+// 2^120 (exact; bf16 arithmetic keeps subnormal operands) gives the e4m3 value
+// 2^(e-7)(1 + m/8), or 2^-6 (m/8).  The two NaN codes (0x7F, 0xFF) are not
+// special-cased: key caches hold finite values.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t src, uint32_t& lo, uint32_t& hi) {
+  uint32_t a, b;
+  // selector nibbles, low byte first: byte 0, sign of byte 0, byte 1, sign of byte 1
+  asm("prmt.b32 %0, %1, 0, 0x9180;" : "=r"(a) : "r"(src));
+  asm("prmt.b32 %0, %1, 0, 0xB3A2;" : "=r"(b) : "r"(src));   // the same for bytes 2 and 3
+  a = (a << 4) & 0x87F087F0u;
+  b = (b << 4) & 0x87F087F0u;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0x7B807B80u));   // 0x7B80 = bf16 2^120
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0x7B807B80u));
 }
 
 struct IndexerParams {
@@ -431,17 +464,15 @@ __global__ void __launch_bounds__(C::NT, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t s_q = sbase + C::OFF_Q;
   const uint32_t s_raw = sbase + C::OFF_RAW;
-  const uint32_t s_k = sbase + C::OFF_K;
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const uint32_t bar_q_full = bar0;
   const uint32_t bar_drain = bar0 + 8;
   auto bar_k_full = [&](int s) { return bar0 + 16 + 8 * s; };
-  auto bar_k_empty = [&](int s) { return bar0 + 16 + 8 * (C::STAGES + s); };
   auto bar_raw_full = [&](int s) { return bar0 + 16 + 8 * (2 * C::STAGES + s); };
   auto bar_raw_empty = [&](int s) { return bar0 + 16 + 8 * (2 * C::STAGES + C::RSTAGES + s); };
   auto bar_acc_full = [&](int a) { return bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + a); };
-  auto bar_acc_empty = [&](int a) { return bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + 2 + a); };
-  const uint32_t bar_q_empty = bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + 4);
+  auto bar_acc_empty = [&](int a) { return bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + C::NACC + a); };
+  const uint32_t bar_q_empty = bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + 2 * C::NACC);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -449,17 +480,14 @@ __global__ void __launch_bounds__(C::NT, 1)
     mbar_init(bar_q_full, 1);
     mbar_init(bar_q_empty, 1);
     mbar_init(bar_drain, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(bar_k_full(s), 128);
-      mbar_init(bar_k_empty(s), 1);
-    }
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(bar_k_full(s), 128);
     for (int s = 0; s < C::RSTAGES; ++s) {
       mbar_init(bar_raw_full(s), 1);
       mbar_init(bar_raw_empty(s), 128);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < C::NACC; ++a) {
       mbar_init(bar_acc_full(a), 1);
-      mbar_init(bar_acc_empty(a), 128);   // drained by warpgroup a
+      mbar_init(bar_acc_empty(a), 128);   // drained by warpgroup a % EPI_WG
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -515,7 +543,6 @@ __global__ void __launch_bounds__(C::NT, 1)
     if (lane == 0) DSA_PROF_SPAN(61, t_role);
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    const uint64_t a_desc0 = smem_desc(s_k, 16, 8 * C::SWB, C::SWZ);
     const uint64_t b_desc0 = smem_desc(s_q, 16, 8 * C::SWB, C::SWZ);
     if (lane == 0) {
       int b = b_first, seg = -1, cur = -1;
@@ -529,23 +556,22 @@ __global__ void __launch_bounds__(C::NT, 1)
           tc_fence_after();
         }
         const int s = it % C::STAGES;
-        const int a = it & 1;
+        const int a = it % C::NACC;
         if (!mbar_wait(bar_k_full(s), (it / C::STAGES) & 1, abort_flag, 53)) break;
-        if (!mbar_wait(bar_acc_empty(a), ((it >> 1) & 1) ^ 1, abort_flag, 54)) break;
+        if (!mbar_wait(bar_acc_empty(a), ((it / C::NACC) & 1) ^ 1, abort_flag, 54)) break;
         tc_fence_after();
-        // descriptors: the start-address field (16-byte units, low bits) advances
-        // by the stage and k-step offsets; it never carries (addresses < 256 KB)
-        const uint64_t a_stage = a_desc0 + static_cast<uint64_t>((s * C::A_TILE) >> 4);
+        // A: the key tile in tensor memory, 8 columns (16 bf16) per k-step.
+        // B: the query descriptor's start-address field (16-byte units, low
+        // bits) advances by the k-step offset; it never carries.
+        const uint32_t a_tile = tmem + C::ACC_COLS + s * C::A_COLS;
 #pragma unroll
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const int atom = (kk * 32) / C::SWB;
           const int off = (kk * 32) % C::SWB;
-          const uint64_t ad = a_stage + static_cast<uint64_t>((atom * C::BK * C::SWB + off) >> 4);
           const uint64_t bd = b_desc0 + static_cast<uint64_t>((atom * C::N * C::SWB + off) >> 4);
-          umma_ss(tmem + a * C::N, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+          umma_ts(tmem + a * C::N, a_tile + kk * 8, bd, C::IDESC, kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar_k_empty(s));
-        umma_commit(bar_acc_full(a));
+        umma_commit(bar_acc_full(a));   // also frees key stage s (== a): one commit per tile
         if (u + 1 == u1 || u + 1 >= upre[b + 1]) umma_commit(bar_q_empty);   // last tile of the sequence
       }
       DSA_PROF_SPAN(62, t_role);
@@ -556,24 +582,47 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
   } else if (warp >= C::CONVERT_WARP0) {
     // ------------------------------------------------------------ e4m3 -> bf16
+    // Each thread widens one key row into its own TMEM lane: a warp reaches
+    // lanes 32 (warp % 4) .. +31, so the row is fixed by the warp's position.
     const int team = (warp - C::CONVERT_WARP0) / 4;
-    const int row = threadIdx.x - (C::CONVERT_WARP0 + 4 * team) * 32;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + C::ACC_COLS;
     for (int it = team; it < n_iter; it += C::CONV_TEAMS) {
       const int r = it % C::RSTAGES;
       const int s = it % C::STAGES;
       if (!mbar_wait(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag, 55)) break;
-      if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, 56)) break;
-      e4m3_row_to_bf16<C::BK>(smem + C::OFF_RAW + r * C::RAW_TILE + row * 128, smem + C::OFF_K + s * C::A_TILE,
-                              row);
+      const uint8_t* raw_row = smem + C::OFF_RAW + r * C::RAW_TILE + row * 128;
+      uint4 chunk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)  // 128-byte swizzle: logical chunk j sits at j ^ (row & 7)
+        chunk[j] = *reinterpret_cast<const uint4*>(raw_row + ((j ^ (row & 7)) << 4));
       mbar_arrive(bar_raw_empty(r));
-      fence_proxy_async_smem();
+      // stage s is free once the MMAs of tile it - STAGES completed: the phase
+      // before the one the epilogue of tile it waits for on the same barrier
+      if (!mbar_wait(bar_acc_full(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, 56)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {   // 64 elements (32 columns) per store
+        uint32_t cols[32];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 c = chunk[4 * h + j];
+          e4m3x4_to_bf16x4(c.x, cols[8 * j + 0], cols[8 * j + 1]);
+          e4m3x4_to_bf16x4(c.y, cols[8 * j + 2], cols[8 * j + 3]);
+          e4m3x4_to_bf16x4(c.z, cols[8 * j + 4], cols[8 * j + 5]);
+          e4m3x4_to_bf16x4(c.w, cols[8 * j + 6], cols[8 * j + 7]);
+        }
+        tmem_st32(t_lane + s * C::A_COLS + 32 * h, cols);
+      }
+      tmem_wait_st();
+      tc_fence_before();
       mbar_arrive(bar_k_full(s));
     }
     if (lane == 0) DSA_PROF_SPAN(63, t_role);
   } else {
     // ------------------------------------------------------------ epilogue
-    // Warpgroup g drains accumulator g, i.e. tiles it = g, g+2, ...; the key
-    // scales of its next tile are loaded one iteration ahead.
+    // Warpgroup g drains tiles it = g, g + EPI_WG, ... (accumulator it % NACC);
+    // the key scales of its next tile are loaded one iteration ahead.
     const int g = warp >> 2;
     const int sub = warp & 3;
     const int key_in_tile = sub * 32 + lane;
@@ -589,8 +638,9 @@ __global__ void __launch_bounds__(C::NT, 1)
       return s_key < p.cu_k[bp + 1] - kb ? p.k_scale[kb + s_key] : 0.f;
     };
     float ks = fetch_scale(g);
-    for (int it = g; it < n_iter; it += 2) {
-      const float ks_next = fetch_scale(it + 2);
+    for (int it = g; it < n_iter; it += C::EPI_WG) {
+      const float ks_next = fetch_scale(it + C::EPI_WG);
+      const int a = it % C::NACC;
       const int u = u0 + it;
       while (u >= upre[b + 1]) ++b;
       if (b != cur) {
@@ -601,9 +651,9 @@ __global__ void __launch_bounds__(C::NT, 1)
         if (lane < C::H_I / 4) reinterpret_cast<float4*>(wsm)[lane] = w4[lane];
         __syncwarp();
       }
-      if (!mbar_wait_warp(bar_acc_full(g), (it >> 1) & 1, abort_flag, 57)) break;
+      if (!mbar_wait_warp(bar_acc_full(a), (it / C::NACC) & 1, abort_flag, 57)) break;
       tc_fence_after();
-      const uint32_t t_row = tmem + (static_cast<uint32_t>(sub * 32) << 16) + g * C::N;
+      const uint32_t t_row = tmem + (static_cast<uint32_t>(sub * 32) << 16) + a * C::N;
       float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
       for (int half = 0; half < C::H_I / 32; ++half) {
@@ -620,7 +670,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_acc_empty(g));
+      mbar_arrive(bar_acc_empty(a));
       const int s_key = (u - upre[b]) * C::BK + key_in_tile;
       if (s_key < q.kv_len) {
         const float val = s_key <= q.pos ? (acc0 + acc1) * ks : -INFINITY;

@@ -151,6 +151,47 @@ def test_indexer_released_shape(dsa, oracle_lib, kfp8, q_lens, kv_lens):
         assert np.array_equal(part[r, : p_ + 1], got[q0 + r, : p_ + 1])
 
 
+def _all_e4m3_codes_case(q_lens, kv_lens):
+    """Index keys whose bytes run through every finite e4m3 code (key s, dim d
+    holds code (s + 7 d) mod 256, the two NaN codes replaced by zeros), scale
+    1; query row t is a one-hot vector at dim d_t with sign +1 or -1 in index
+    head 0, and only head 0 has weight.  Score[t, s] = ReLU(sign_t *
+    decode(code)), one product per score, so the widened keys are checked
+    code by code and must match the oracle exactly."""
+    B = len(q_lens)
+    cu_q = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(kv_lens)]).astype(np.int32)
+    T, S = int(cu_q[-1]), int(cu_k[-1])
+    codes = np.zeros((S, 128), dtype=np.uint8)
+    for b in range(B):
+        s = np.arange(kv_lens[b])[:, None]
+        codes[cu_k[b]:cu_k[b + 1]] = (s + 7 * np.arange(128)[None, :]) % 256
+    codes[codes == 0x7F] = 0x00
+    codes[codes == 0xFF] = 0x80
+    q = torch.zeros((T, 64, 128), dtype=torch.float32)
+    for t in range(T):
+        q[t, 0, (5 * t) % 128] = 1.0 if t % 2 == 0 else -1.0
+    w = torch.zeros((T, 64), dtype=torch.float32)
+    w[:, 0] = 1.0
+    return {"cu_q": cu_q, "cu_k": cu_k, "q_idx": q.to(torch.bfloat16), "w": w,
+            "k_idx": torch.from_numpy(codes).view(torch.float8_e4m3fn), "k_scale": torch.ones(S, dtype=torch.float32)}
+
+
+@pytest.mark.parametrize("q_lens,kv_lens", [
+    ((1,) * 128, tuple(256 + b for b in range(128))),   # persistent decode schedule
+    ((5, 5, 5, 3), (300, 260, 400, 257)),                # query-block schedule
+], ids=["decode", "prefill"])
+def test_indexer_widens_every_e4m3_code_exactly(dsa, oracle_lib, q_lens, kv_lens):
+    d = _all_e4m3_codes_case(q_lens, kv_lens)
+    dd = P.to_device(d)
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], "cuda")
+    ld = (max(kv_lens) + 3) // 4 * 4
+    got = gpu_scores(dsa, dd, v, 0, sum(q_lens), ld).cpu().numpy()
+    ref = oracle_lib.indexer_scores(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"], d["k_scale"], ld=ld)
+    pos = P.row_positions(d["cu_q"], d["cu_k"])
+    P.assert_scores_close(got, ref, pos, exact=True)
+
+
 # ------------------------------------------------------------------ sparse MLA
 
 def _attention_case(dsa, oracle_lib, spec, idx=None):
