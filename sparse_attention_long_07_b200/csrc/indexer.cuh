@@ -70,14 +70,18 @@ struct IndexerCfg {
   static constexpr int EPI_THREADS = 128 * EPI_WG;
   static constexpr int PRODUCER_WARP = 4 * EPI_WG;
   static constexpr int MMA_WARP = PRODUCER_WARP + 1;
-  static constexpr int CONVERT_WARP0 = MMA_WARP + 1;
+  // persistent schedule: two MMA-issuing threads (one per warp) take alternate
+  // tiles, so one's barrier waits and commits overlap the other's MMAs
+  static constexpr int MMA_THREADS = PERSIST ? 2 : 1;
+  static constexpr int CONVERT_WARP0 = MMA_WARP + MMA_THREADS;
   static constexpr int CONV_TEAMS = PERSIST ? 2 : 1;      // e4m3 converter teams (alternate tiles)
-  static constexpr int NWARPS = MMA_WARP + 1 + (KFP8 ? 4 * CONV_TEAMS : 0);
+  static constexpr int NWARPS = MMA_WARP + MMA_THREADS + (KFP8 ? 4 * CONV_TEAMS : 0);
   static constexpr int NT = NWARPS * 32;
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, N, false, false);
   // shared memory layout (offsets from a 1024-byte aligned base)
+  static constexpr int QBUF = PERSIST ? 2 : 1;            // query tiles (double buffer when persistent)
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + B_TILE;
+  static constexpr int OFF_K = OFF_Q + QBUF * B_TILE;
   static constexpr int OFF_RAW = OFF_K + (K_IN_TMEM ? 0 : STAGES * A_TILE);
   static constexpr int OFF_W = OFF_RAW + RSTAGES * RAW_TILE;
   static constexpr int OFF_BAR = OFF_W + NQ * H_I * 4;
@@ -94,6 +98,8 @@ struct IndexerCfg {
   static_assert(TMEM_COLS <= 512, "tensor memory columns");
   static_assert(!K_IN_TMEM || (KFP8 && STAGES % CONV_TEAMS == 0), "converter teams own alternate stages");
   static_assert(NACC % EPI_WG == 0, "each accumulator is drained by one epilogue warpgroup");
+  static_assert(!PERSIST || 7 + STAGES + 2 * RSTAGES + NACC <= NBAR, "persistent barrier layout");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(!K_IN_TMEM || STAGES == NACC, "key stage and accumulator of a tile share one barrier");
   static_assert(!PERSIST || NQ == 1, "persistent schedule: one query per sequence block");
   static_assert(OFF_K % 1024 == 0 && OFF_RAW % 1024 == 0, "swizzled tiles on 1024-byte boundaries");
@@ -465,32 +471,37 @@ __global__ void __launch_bounds__(C::NT, 1)
   const uint32_t s_q = sbase + C::OFF_Q;
   const uint32_t s_raw = sbase + C::OFF_RAW;
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  const uint32_t bar_q_full = bar0;
-  const uint32_t bar_drain = bar0 + 8;
-  auto bar_k_full = [&](int s) { return bar0 + 16 + 8 * s; };
-  auto bar_raw_full = [&](int s) { return bar0 + 16 + 8 * (2 * C::STAGES + s); };
-  auto bar_raw_empty = [&](int s) { return bar0 + 16 + 8 * (2 * C::STAGES + C::RSTAGES + s); };
-  auto bar_acc_full = [&](int a) { return bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + a); };
-  auto bar_acc_empty = [&](int a) { return bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + C::NACC + a); };
-  const uint32_t bar_q_empty = bar0 + 16 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + 2 * C::NACC);
+  const uint32_t bar_drain = bar0;
+  // query tile of segment g (the g-th sequence of this CTA) in buffer g & 1:
+  // q_full(buf) from the TMA, q_empty(t, buf) from MMA thread t, once per
+  // segment, after its last MMA that reads the tile
+  auto bar_q_full = [&](int buf) { return bar0 + 8 + 8 * buf; };
+  auto bar_q_empty = [&](int t, int buf) { return bar0 + 24 + 8 * (2 * t + buf); };
+  // ready(s): tile it (s = it % STAGES) is widened in TMEM and its accumulator
+  // (the same index) has been drained: 128 converter + 128 epilogue arrivals
+  auto bar_ready = [&](int s) { return bar0 + 56 + 8 * s; };
+  auto bar_raw_full = [&](int s) { return bar0 + 56 + 8 * (C::STAGES + s); };
+  auto bar_raw_empty = [&](int s) { return bar0 + 56 + 8 * (C::STAGES + C::RSTAGES + s); };
+  auto bar_acc_full = [&](int a) { return bar0 + 56 + 8 * (C::STAGES + 2 * C::RSTAGES + a); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q_full, 1);
-    mbar_init(bar_q_empty, 1);
-    mbar_init(bar_drain, 1);
-    for (int s = 0; s < C::STAGES; ++s) mbar_init(bar_k_full(s), 128);
+    mbar_init(bar_drain, C::MMA_THREADS);
+    for (int buf = 0; buf < 2; ++buf) {
+      mbar_init(bar_q_full(buf), 1);
+      for (int t = 0; t < C::MMA_THREADS; ++t) mbar_init(bar_q_empty(t, buf), 1);
+    }
+    for (int s = 0; s < C::STAGES; ++s) mbar_init(bar_ready(s), 256);
     for (int s = 0; s < C::RSTAGES; ++s) {
       mbar_init(bar_raw_full(s), 1);
       mbar_init(bar_raw_empty(s), 128);
     }
-    for (int a = 0; a < C::NACC; ++a) {
-      mbar_init(bar_acc_full(a), 1);
-      mbar_init(bar_acc_empty(a), 128);   // drained by warpgroup a % EPI_WG
-    }
+    for (int a = 0; a < C::NACC; ++a) mbar_init(bar_acc_full(a), 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // every accumulator starts drained: the epilogue's share of the first phase
+    for (int s = 0; s < C::STAGES; ++s) mbar_arrive_count(bar_ready(s), 128);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -509,19 +520,26 @@ __global__ void __launch_bounds__(C::NT, 1)
   if (warp == C::PRODUCER_WARP) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int b = b_first, seg = -1, armed_q = 0, it = 0;
+      int b = b_first, seg = -1, loaded_q = 0, it = 0;
       Seq q{};
       for (; it < n_iter; ++it) {
         const int u = u0 + it;
         while (u >= upre[b + 1]) ++b;
         if (b != q.b || seg < 0) {
           ++seg;
-          if (seg > 0 && !mbar_wait(bar_q_empty, (seg - 1) & 1, abort_flag, 50)) break;
+          const int buf = seg & 1;
+          if (seg >= 2) {   // both MMA threads are done with segment seg - 2
+            bool free_ = true;
+            for (int t = 0; t < C::MMA_THREADS && free_; ++t)
+              free_ = mbar_wait(bar_q_empty(t, buf), ((seg - 2) >> 1) & 1, abort_flag, 50);
+            if (!free_) break;
+          }
           q = seq_of(b);
-          mbar_arrive_expect_tx(bar_q_full, C::B_TILE);
+          mbar_arrive_expect_tx(bar_q_full(buf), C::B_TILE);
           for (int at = 0; at < C::NATOM; ++at)
-            tma_load_2d(s_q + at * C::N * C::SWB, &tm_q, bar_q_full, at * C::ATOM_ELEMS, q.q0 * C::H_I);
-          armed_q = seg + 1;
+            tma_load_2d(s_q + buf * C::B_TILE + at * C::N * C::SWB, &tm_q, bar_q_full(buf), at * C::ATOM_ELEMS,
+                        q.q0 * C::H_I);
+          loaded_q = seg + 1;
         }
         const int tile = u - upre[b];
         const int r = it % C::RSTAGES;
@@ -535,30 +553,52 @@ __global__ void __launch_bounds__(C::NT, 1)
           while (!mbar_try_wait(bar_raw_full(j % C::RSTAGES), (j / C::RSTAGES) & 1) &&
                  clock64() - t0 < kWaitLimitCycles) {
           }
-        if (armed_q)
-          while (!mbar_try_wait(bar_q_full, (armed_q - 1) & 1) && clock64() - t0 < kWaitLimitCycles) {
+        for (int g = (loaded_q > 2 ? loaded_q - 2 : 0); g < loaded_q; ++g)
+          while (!mbar_try_wait(bar_q_full(g & 1), (g >> 1) & 1) && clock64() - t0 < kWaitLimitCycles) {
           }
       }
     }
     if (lane == 0) DSA_PROF_SPAN(61, t_role);
-  } else if (warp == C::MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= C::MMA_WARP && warp < C::CONVERT_WARP0) {
+    // ------------------------------------------------------------ MMA issuers
+    // Thread t (lane 0 of warp MMA_WARP + t) issues tiles it = t, t + 2, ...
+    // It walks the CTA's segments in order and, for every segment, waits for
+    // its query tile and commits q_empty(t, .) once, also for a segment in
+    // which it has no tile, so that the producer can count on both threads.
+    const int mt = warp - C::MMA_WARP;
     const uint64_t b_desc0 = smem_desc(s_q, 16, 8 * C::SWB, C::SWZ);
     if (lane == 0) {
-      int b = b_first, seg = -1, cur = -1;
-      for (int it = 0; it < n_iter; ++it) {
+      int b = b_first, seg = 0, seq_end = upre[b_first + 1];
+      bool have_q = false, ok = true;
+      uint64_t b_desc = b_desc0;
+      auto next_segment = [&]() {
+        ++seg;
+        do {
+          ++b;
+        } while (upre[b + 1] == upre[b]);   // sequences without units in the call
+        seq_end = upre[b + 1];
+      };
+      auto release_segment = [&]() -> bool {   // done with segment seg
+        if (!have_q && !mbar_wait(bar_q_full(seg & 1), (seg >> 1) & 1, abort_flag, 52)) return false;
+        umma_commit(bar_q_empty(mt, seg & 1));
+        have_q = false;
+        return true;
+      };
+      for (int it = mt; it < n_iter; it += C::MMA_THREADS) {
         const int u = u0 + it;
-        while (u >= upre[b + 1]) ++b;
-        if (b != cur) {
-          ++seg;
-          cur = b;
-          if (!mbar_wait(bar_q_full, seg & 1, abort_flag, 52)) break;
-          tc_fence_after();
+        while (ok && u >= seq_end) {
+          ok = release_segment();
+          next_segment();
+        }
+        if (!ok) break;
+        if (!have_q) {
+          if (!mbar_wait(bar_q_full(seg & 1), (seg >> 1) & 1, abort_flag, 52)) { ok = false; break; }
+          have_q = true;
+          b_desc = b_desc0 + static_cast<uint64_t>(((seg & 1) * C::B_TILE) >> 4);
         }
         const int s = it % C::STAGES;
-        const int a = it % C::NACC;
-        if (!mbar_wait(bar_k_full(s), (it / C::STAGES) & 1, abort_flag, 53)) break;
-        if (!mbar_wait(bar_acc_empty(a), ((it / C::NACC) & 1) ^ 1, abort_flag, 54)) break;
+        const int a = s;
+        if (!mbar_wait(bar_ready(s), (it / C::STAGES) & 1, abort_flag, 53)) { ok = false; break; }
         tc_fence_after();
         // A: the key tile in tensor memory, 8 columns (16 bf16) per k-step.
         // B: the query descriptor's start-address field (16-byte units, low
@@ -568,11 +608,16 @@ __global__ void __launch_bounds__(C::NT, 1)
         for (int kk = 0; kk < C::KSTEPS; ++kk) {
           const int atom = (kk * 32) / C::SWB;
           const int off = (kk * 32) % C::SWB;
-          const uint64_t bd = b_desc0 + static_cast<uint64_t>((atom * C::N * C::SWB + off) >> 4);
+          const uint64_t bd = b_desc + static_cast<uint64_t>((atom * C::N * C::SWB + off) >> 4);
           umma_ts(tmem + a * C::N, a_tile + kk * 8, bd, C::IDESC, kk > 0 ? 1u : 0u);
         }
-        umma_commit(bar_acc_full(a));   // also frees key stage s (== a): one commit per tile
-        if (u + 1 == u1 || u + 1 >= upre[b + 1]) umma_commit(bar_q_empty);   // last tile of the sequence
+        umma_commit(bar_acc_full(a));   // also frees key stage s (== a)
+      }
+      // release the current segment and every later one of the CTA
+      while (ok && !*abort_flag) {
+        ok = release_segment();
+        if (seq_end >= u1) break;
+        next_segment();
       }
       DSA_PROF_SPAN(62, t_role);
       umma_commit(bar_drain);
@@ -616,7 +661,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_k_full(s));
+      mbar_arrive(bar_ready(s));
     }
     if (lane == 0) DSA_PROF_SPAN(63, t_role);
   } else {
@@ -670,7 +715,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_acc_empty(a));
+      mbar_arrive(bar_ready(a));   // accumulator a is free for tile it + NACC
       const int s_key = (u - upre[b]) * C::BK + key_in_tile;
       if (s_key < q.kv_len) {
         const float val = s_key <= q.pos ? (acc0 + acc1) * ks : -INFINITY;
