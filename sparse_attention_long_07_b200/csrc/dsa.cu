@@ -236,12 +236,9 @@ template <class C>
 dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, const dsa_varlen& v,
                       const Layout& L, int64_t q_begin, int64_t q_end, int topk, float scale,
                       void* out, float* lse, cudaStream_t stream) {
-  CUtensorMap tm_q, tm_lat;
+  CUtensorMap tm_lat;
   const CUtensorMapSwizzle swz = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : (C::SWB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
-  if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, C::DQK, static_cast<uint64_t>(L.T) * C::H,
-                C::DQK * 2, C::ATOM, 128, swz))
-    return DSA_ERR_CUDA;
   if (!make_map(&tm_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, latent, C::DQK, static_cast<uint64_t>(L.S),
                 C::DQK * 2, C::ATOM, 1, swz))
     return DSA_ERR_CUDA;
@@ -251,6 +248,7 @@ dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, con
   if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
 
   dsa::MlaParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
   p.idx = idx;
   p.cu_q = v.cu_q;
   p.cu_k = v.cu_k;
@@ -274,7 +272,7 @@ dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, con
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, dsa::sparse_mla_kernel<C>, tm_q, tm_lat, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, dsa::sparse_mla_kernel<C>, tm_lat, p);
   return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

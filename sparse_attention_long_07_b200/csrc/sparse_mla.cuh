@@ -21,15 +21,19 @@
 // the same way -- CTA 0 multiplies latent columns [0, 256), CTA 1 columns
 // [256, 576) -- so each CTA gathers only its own 256 or 320 columns of every
 // selected row and no MMA is duplicated.  The two partial score tiles are
-// exchanged through distributed shared memory (each CTA stores its part into
-// the peer's buffer and signals the peer's mbarrier); both CTAs add them in
-// the same commutative way, so both hold bit-identical scores and take the
-// same softmax decisions.  The online softmax keeps a per-head running max
+// exchanged through distributed shared memory (each CTA stages its part in its
+// own shared memory and one bulk copy moves it into the peer's buffer,
+// completing on the peer's mbarrier); both CTAs add them in the same
+// commutative way, so both hold bit-identical scores and take the same
+// softmax decisions.  Tensor memory holds O, three score buffers (a tile's P,
+// in bf16, overwrites its scores once they are in registers) and this CTA's
+// slice of the query, the A operand of every QK MMA, so shared memory is left
+// to an eight-deep ring of gathered rows and the score exchange.  The online softmax keeps a per-head running max
 // and only rescales O (in TMEM) when the max grows by more than 2^8, which
 // is exact arithmetic with the same final normalisation.
 //
-// Roles per CTA: warps 0-3 softmax + epilogue (one head row per thread),
-// warp 4 gather producer, warp 5 MMA issuer (and TMEM owner).
+// Roles per CTA: warps 0-3 query load, softmax and epilogue (one head row per
+// thread), warp 4 gather producer, warp 5 MMA issuer (and TMEM owner).
 #pragma once
 
 #include "common.cuh"
@@ -52,24 +56,27 @@ struct MlaCfg {
   static constexpr int NA0 = SPLIT_ATOM;                  // atoms gathered by rank 0
   static constexpr int NA1 = NATOM_ALL - SPLIT_ATOM;      // atoms gathered by rank 1
   static constexpr int NA_MAX = NA0 > NA1 ? NA0 : NA1;
-  static constexpr int NS = SPLIT == 1 ? 4 : 5;           // gather ring depth
-  static constexpr int Q_ATOM_BYTES = 128 * SWB;          // 128 head rows
+  static constexpr int NS = SPLIT == 1 ? 4 : 8;           // gather ring depth
   static constexpr int C_ATOM_BYTES = BN * SWB;
   static constexpr int C_STAGE = NA_MAX * C_ATOM_BYTES;
-  static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;   // one partial-score buffer
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_C = OFF_Q + NA_MAX * Q_ATOM_BYTES;
-  static constexpr int OFF_X = OFF_C + NS * C_STAGE;      // two partial-score buffers
-  static constexpr int OFF_MASK = OFF_X + 2 * X_BYTES;
+  static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;   // one partial-score tile
+  static constexpr int OFF_C = 0;
+  static constexpr int OFF_X = OFF_C + NS * C_STAGE;      // two received partial-score tiles
+  static constexpr int OFF_XS = OFF_X + 2 * X_BYTES;      // two staged outgoing tiles
+  static constexpr int OFF_MASK = OFF_XS + 2 * X_BYTES;
   static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
-  static constexpr int NSB = 3;                            // S buffers: QK runs up to 3 tiles ahead
-  static constexpr int NBAR = 1 + 2 * NS + 2 * NSB + 2 + 2 + 4 + 1;
+  static constexpr int NSB = 3;                            // S buffers (each later holds its P)
+  static constexpr int LOOKAHEAD = 2;                      // QK tiles issued ahead of PV
+  static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + 9;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  // tensor memory columns: O [0, DVS), S[3] (fp32, BN each), P[2] (bf16 pairs, BN/2 each)
+  // tensor memory columns: O [0, DVS); S[NSB] (fp32, BN each; P of the same
+  // tile, bf16 pairs, overwrites the first BN/2 columns once S is read); the
+  // query slice this CTA multiplies, bf16 pairs (the A operand of QK)
   static constexpr int TMEM_S = DVS;
-  static constexpr int TMEM_P = DVS + NSB * BN;
-  static constexpr int TMEM_USED = TMEM_P + BN;
+  static constexpr int TMEM_Q = DVS + NSB * BN;
+  static constexpr int QCOLS = NA_MAX * ATOM / 2;
+  static constexpr int TMEM_USED = TMEM_Q + QCOLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   static constexpr int NT = 6 * 32;
   static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
@@ -81,12 +88,15 @@ struct MlaCfg {
   static_assert(DVS % ATOM == 0 && DVS <= 256 && DVS % 16 == 0, "PV N");
   static_assert(SPLIT == 1 || NV <= NA1, "rank 1 must gather its value columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(LOOKAHEAD < NSB && LOOKAHEAD + 2 <= NS, "S buffers and gather stages in flight");
+  static_assert(QCOLS % 8 == 0, "query columns are stored eight at a time");
   static_assert(TMEM_USED <= 512, "tensor memory");
   static_assert(OFF_C % 1024 == 0 && C_STAGE % 1024 == 0 && C_ATOM_BYTES % 1024 == 0, "swizzle atoms");
-  static_assert(OFF_X % 16 == 0 && OFF_BAR % 8 == 0, "vector / barrier alignment");
+  static_assert(OFF_X % 16 == 0 && OFF_XS % 16 == 0 && OFF_BAR % 8 == 0, "vector / bulk-copy / barrier alignment");
 };
 
 struct MlaParams {
+  const __nv_bfloat16* q;    // [T, H, DQK]
   const int32_t* idx;        // [q_end - q_begin, topk]
   const int32_t* cu_q;
   const int32_t* cu_k;
@@ -100,8 +110,7 @@ struct MlaParams {
 
 template <class C>
 __global__ void __launch_bounds__(C::NT, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q,
-                      const __grid_constant__ CUtensorMap tm_lat, const MlaParams p) {
+    sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_lat, const MlaParams p) {
   const uint32_t rank = C::SPLIT == 2 ? cluster_ctarank() : 0u;
   const uint32_t peer = rank ^ 1u;
   const int64_t r_local = blockIdx.x / C::SPLIT;          // chunk-relative query row
@@ -114,22 +123,27 @@ __global__ void __launch_bounds__(C::NT, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t s_q = sbase + C::OFF_Q;
   const uint32_t s_c = sbase + C::OFF_C;
   float* xbuf = reinterpret_cast<float*>(smem + C::OFF_X);
+  float* xs = reinterpret_cast<float*>(smem + C::OFF_XS);
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
   const uint32_t bar0 = sbase + C::OFF_BAR;
-  const uint32_t bar_q_full = bar0;
+  const uint32_t bar_q_ready = bar0;                     // query slice stored in TMEM (128 arrivals)
   auto bar_c_full = [&](int s) { return bar0 + 8 * (1 + s); };
   auto bar_c_empty = [&](int s) { return bar0 + 8 * (1 + C::NS + s); };
   constexpr int SB0 = 1 + 2 * C::NS;                     // first S barrier
   auto bar_s_full = [&](int a) { return bar0 + 8 * (SB0 + a); };
-  auto bar_s_free = [&](int a) { return bar0 + 8 * (SB0 + C::NSB + a); };
+  auto bar_pv_done = [&](int a) { return bar0 + 8 * (SB0 + C::NSB + a); };   // PV of the P in S buffer a
+  // p_full(a): P of tile j (a = j % NSB) stored; one per S buffer, so the
+  // softmax can never complete a phase twice ahead of the MMA thread's wait
   auto bar_p_full = [&](int a) { return bar0 + 8 * (SB0 + 2 * C::NSB + a); };
-  auto bar_pv_done = [&](int a) { return bar0 + 8 * (SB0 + 2 * C::NSB + 2 + a); };
-  auto bar_x_full = [&](int b) { return bar0 + 8 * (SB0 + 2 * C::NSB + 4 + b); };
-  auto bar_x_empty = [&](int b) { return bar0 + 8 * (SB0 + 2 * C::NSB + 6 + b); };
-  const uint32_t bar_drain = bar0 + 8 * (SB0 + 2 * C::NSB + 8);
+  constexpr int XB0 = SB0 + 3 * C::NSB;
+  auto bar_x_full = [&](int b) { return bar0 + 8 * (XB0 + b); };
+  auto bar_x_empty = [&](int b) { return bar0 + 8 * (XB0 + 2 + b); };
+  const uint32_t bar_drain = bar0 + 8 * (XB0 + 4);
+  // outgoing staging buffer b: every row written (128 arrivals) / read by its copy (thread 0)
+  auto bar_xs_full = [&](int b) { return bar0 + 8 * (XB0 + 5 + b); };
+  auto bar_xs_free = [&](int b) { return bar0 + 8 * (XB0 + 7 + b); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* ntiles_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -139,24 +153,25 @@ __global__ void __launch_bounds__(C::NT, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q_full, 1);
+    mbar_init(bar_q_ready, 128);
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar_c_full(s), 1);
       mbar_init(bar_c_empty(s), 1);
     }
     for (int a = 0; a < C::NSB; ++a) {
       mbar_init(bar_s_full(a), 1);
-      mbar_init(bar_s_free(a), 128);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(bar_p_full(a), 128);
       mbar_init(bar_pv_done(a), 1);
+      mbar_init(bar_p_full(a), 128);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_x_full(b), 1);    // armed locally; filled by the peer's st.async bytes
+      mbar_init(bar_x_full(b), 1);    // armed locally; filled by the peer's bulk copy
       mbar_init(bar_x_empty(b), 4);   // one release-arrive per softmax warp of the peer
     }
     mbar_init(bar_drain, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_xs_full(b), 128);
+      mbar_init(bar_xs_free(b), 1);
+    }
     *abort_flag = 0;
     *ntiles_s = 0;
     // an error recorded earlier by any CTA of this library: skip the work
@@ -167,10 +182,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == C::PRODUCER_WARP && lane == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_lat);
-  }
+  if (warp == C::PRODUCER_WARP && lane == 0) tma_prefetch_desc(&tm_lat);
   DSA_PROF_BEGIN();
   __syncthreads();
   // Tiles up to the last one holding a valid entry (trailing -1 padding is skipped).
@@ -198,12 +210,6 @@ __global__ void __launch_bounds__(C::NT, 1)
     // ------------------------------------------------------------ gather producer
     int it = 0;
     if (n_tiles > 0) {
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar_q_full, na * C::Q_ATOM_BYTES);
-        for (int a = 0; a < na; ++a)
-          tma_load_2d(s_q + a * C::Q_ATOM_BYTES, &tm_q, bar_q_full, (a0 + a) * C::ATOM,
-                      static_cast<int32_t>(t * C::H));
-      }
       for (; it < n_tiles; ++it) {
         const int s = it % C::NS;
         int ok = 1;
@@ -236,8 +242,6 @@ __global__ void __launch_bounds__(C::NT, 1)
           while (!mbar_try_wait(bar_c_full(j % C::NS), (j / C::NS) & 1) &&
                  clock64() - t0 < kWaitLimitCycles) {
           }
-        while (!mbar_try_wait(bar_q_full, 0) && clock64() - t0 < kWaitLimitCycles) {
-        }
       }
     }
     if (lane == 0) DSA_PROF_SPAN(61, t_role);
@@ -245,46 +249,51 @@ __global__ void __launch_bounds__(C::NT, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_tiles > 0) {
       auto issue_pv = [&](int j) -> bool {
-        const int pb = j & 1;
-        if (!mbar_wait(bar_p_full(pb), (j >> 1) & 1, abort_flag, 22)) return false;
+        const int sb = j % C::NSB;
+        if (!mbar_wait(bar_p_full(sb), (j / C::NSB) & 1, abort_flag, 22)) return false;
         tc_fence_after();
         const uint32_t v_base = s_c + (j % C::NS) * C::C_STAGE;
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          // A = P from tensor memory: 16 k-elements = 8 columns per step
-          const uint32_t a_tmem = tmem + C::TMEM_P + pb * (C::BN / 2) + kk * 8;
+          // A = P (bf16 pairs in S buffer sb): 16 k-elements = 8 columns per step
+          const uint32_t a_tmem = tmem + C::TMEM_S + sb * C::BN + kk * 8;
           const uint64_t bd = smem_desc(v_base + kk * 16 * C::SWB, C::C_ATOM_BYTES, 8 * C::SWB, C::SWZ);
           umma_ts(tmem, a_tmem, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(bar_c_empty(j % C::NS));
-        umma_commit(bar_pv_done(pb));
+        umma_commit(bar_pv_done(sb));
         return true;
       };
       const int ksteps = na * C::KPA;
-      // QK(j) -> S[j % 3]; issued up to three tiles ahead of the PV that trails it
+      // QK(j) -> S[j % NSB]; issued LOOKAHEAD tiles ahead of the PV that trails it
       auto issue_qk = [&](int j) -> bool {
         const int s = j % C::NS;
         const int sb = j % C::NSB;
         if (!mbar_wait(bar_c_full(s), (j / C::NS) & 1, abort_flag, 24)) return false;
-        if (!mbar_wait(bar_s_free(sb), ((j / C::NSB) & 1) ^ 1, abort_flag, 25)) return false;
+        // S buffer sb last held P(j - NSB): its PV must have read it
+        if (!mbar_wait(bar_pv_done(sb), ((j / C::NSB) & 1) ^ 1, abort_flag, 25)) return false;
         tc_fence_after();
         const uint32_t c_base = s_c + s * C::C_STAGE;
         for (int kk = 0; kk < ksteps; ++kk) {
+          // A = the query slice in tensor memory (8 columns per 16-wide k-step)
           const int atom = kk / C::KPA;
           const int off = (kk % C::KPA) * 32;
-          const uint64_t ad = smem_desc(s_q + atom * C::Q_ATOM_BYTES + off, 16, 8 * C::SWB, C::SWZ);
           const uint64_t bd = smem_desc(c_base + atom * C::C_ATOM_BYTES + off, 16, 8 * C::SWB, C::SWZ);
-          umma_ss(tmem + C::TMEM_S + sb * C::BN, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          umma_ts(tmem + C::TMEM_S + sb * C::BN, tmem + C::TMEM_Q + kk * 8, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_s_full(sb));
         return true;
       };
-      bool ok = mbar_wait(bar_q_full, 0, abort_flag, 23);
+      // QK runs LOOKAHEAD tiles ahead of PV, and QK(j + LOOKAHEAD) is issued
+      // before PV(j): it needs only S buffer (j + LOOKAHEAD) % NSB, which the
+      // softmax frees when it starts on tile j - 1, so the tensor core works on
+      // the next scores while the softmax finishes tile j.
+      bool ok = mbar_wait(bar_q_ready, 0, abort_flag, 23);
       tc_fence_after();
-      for (int j = 0; ok && j < C::NSB && j < n_tiles; ++j) ok = issue_qk(j);
+      for (int j = 0; ok && j < C::LOOKAHEAD && j < n_tiles; ++j) ok = issue_qk(j);
       for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + C::LOOKAHEAD < n_tiles && !issue_qk(j + C::LOOKAHEAD)) break;
         if (!issue_pv(j)) break;
-        if (j + C::NSB < n_tiles && !issue_qk(j + C::NSB)) break;
       }
     }
     if (lane == 0) {
@@ -304,6 +313,26 @@ __global__ void __launch_bounds__(C::NT, 1)
     float m_used = -INFINITY;    // running max (log2 units) the exponentials are taken against
     float l_run = 0.f;
     bool ok = true;
+    // Query slice of head row h (the gathered columns) into TMEM lane h: the A
+    // operand of every QK MMA.  Rows h >= H hold zeros.
+    if (n_tiles > 0) {
+      const bool row_ok = h < C::H;
+      const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * C::H + (row_ok ? h : 0)) * C::DQK +
+                                                         a0 * C::ATOM);
+#pragma unroll 1
+      for (int c0 = 0; c0 < na * C::ATOM / 2; c0 += 8) {   // 8 columns = 16 bf16 = two 16-byte loads
+        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+        if (row_ok) {
+          v0 = __ldg(qrow + c0 / 4);
+          v1 = __ldg(qrow + c0 / 4 + 1);
+        }
+        const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        tmem_st8(tmem + lane_base + C::TMEM_Q + c0, w8);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_q_ready);
+    }
     // Load tile j's partial scores S[j % 3] and (2-CTA split) start sending them
     // to the peer.  Tile it+1 is started before tile it is finished, so the
     // exchange of a tile has a whole softmax iteration to complete.
@@ -314,30 +343,50 @@ __global__ void __launch_bounds__(C::NT, 1)
       uint32_t raw[32];
       tmem_ld32(tmem + lane_base + C::TMEM_S + sb * C::BN, raw);
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar_s_free(sb));
 #pragma unroll
       for (int c = 0; c < C::BN; ++c) dst[c] = __uint_as_float(raw[c]);
       if (C::SPLIT == 2) {
+        // The tile goes to the peer in one bulk copy: every thread stages its
+        // row in this CTA's buffer xb, then thread 0 copies the 128 rows.
         const int xb = j & 1;
         // receive side: arm tile j's phase with the bytes the peer will send
         if (h == 0) mbar_arrive_expect_tx(bar_x_full(xb), C::X_BYTES);
-        // send side: the peer must have released its buffer xb (tile j-2)
-        if (!mbar_wait_warp<true>(bar_x_empty(xb), ((j >> 1) & 1) ^ 1, abort_flag, 27)) return false;
-        const uint32_t dst_row = x_peer + xb * C::X_BYTES + h * C::BN * 4;
+        // staging buffer xb is free once the copy of tile j-2 has read it
+        if (!mbar_wait_warp(bar_xs_free(xb), ((j >> 1) & 1) ^ 1, abort_flag, 33)) return false;
+        float* row = xs + xb * (C::X_BYTES / 4) + h * C::BN;
 #pragma unroll
         for (int c = 0; c < C::BN / 4; ++c) {
           const int slot = (c + h) & (C::BN / 4 - 1);   // rotate 16-byte chunks: no bank conflicts
-          st_async_v4(dst_row + slot * 16, dst[4 * c], dst[4 * c + 1], dst[4 * c + 2], dst[4 * c + 3],
-                      bar_x_full_peer0 + 8 * xb);
+          *reinterpret_cast<float4*>(row + slot * 4) = make_float4(dst[4 * c], dst[4 * c + 1], dst[4 * c + 2],
+                                                                   dst[4 * c + 3]);
         }
+        fence_proxy_async_smem();
+        mbar_arrive(bar_xs_full(xb));
+        int go = 1;
+        if (h == 0) {
+          // all rows staged, and the peer has released its receive buffer xb (tile j-2)
+          go = mbar_wait(bar_xs_full(xb), (j >> 1) & 1, abort_flag, 34) &&
+               mbar_wait<true>(bar_x_empty(xb), ((j >> 1) & 1) ^ 1, abort_flag, 27);
+          if (go) {
+            bulk_copy_to_peer(x_peer + xb * C::X_BYTES, smem_u32(xs) + xb * C::X_BYTES, C::X_BYTES,
+                              bar_x_full_peer0 + 8 * xb);
+            bulk_commit_group();
+            // the copy of tile j-1 has read staging buffer xb ^ 1: tile j+1 may refill it
+            if (j >= 1) {
+              bulk_wait_group_read<1>();
+              mbar_arrive(bar_xs_free(xb ^ 1));
+            }
+          }
+        }
+        // warp 0 leaves together if thread 0 gave up; other warps see the abort flag
+        if (__shfl_sync(0xFFFFFFFFu, go, 0) == 0) return false;
       }
       return true;
     };
     float sv[C::BN], s_next[C::BN];
     if (n_tiles > 0 && !load_and_push(0, sv)) ok = false;
     for (int it = 0; ok && it < n_tiles; ++it) {
-      const int sb = it & 1;
+      const int sb = it % C::NSB;   // S buffer of this tile; its P goes there too
       if (it + 1 < n_tiles && !load_and_push(it + 1, s_next)) { ok = false; break; }
       if (C::SPLIT == 2) {
         const int xb = it & 1;
@@ -360,37 +409,39 @@ __global__ void __launch_bounds__(C::NT, 1)
       // validity of the tile's entries (written by the producer before it armed c_full)
       if (!mbar_wait_warp(bar_c_full(it % C::NS), (it / C::NS) & 1, abort_flag, 29)) { ok = false; break; }
       const uint32_t vmask = mask_s[it % C::NS];
-      float mt = -INFINITY;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int j = 0; j < C::BN; ++j) {
         sv[j] = ((vmask >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, sv[j]);
+        mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
       }
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       float corr = 1.f;
       if (mt > m_used + C::kRescaleThreshold) {
         corr = exp2f(m_used - mt);   // 0 on the first tile with a valid entry
         m_used = mt;
       }
-      // P tile of this iteration reuses the buffer of tile it-2: PV(it-2) must be done
-      if (it >= 2 && !mbar_wait_warp(bar_pv_done(sb), ((it - 2) >> 1) & 1, abort_flag, 30)) { ok = false; break; }
       uint32_t pk[C::BN / 2];
-      float psum = 0.f;
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < C::BN; j += 2) {
-        const float e0 = sv[j] == -INFINITY ? 0.f : exp2f(sv[j] - m_used);
-        const float e1 = sv[j + 1] == -INFINITY ? 0.f : exp2f(sv[j + 1] - m_used);
+        const float e0 = sv[j] == -INFINITY ? 0.f : ex2_approx(sv[j] - m_used);
+        const float e1 = sv[j + 1] == -INFINITY ? 0.f : ex2_approx(sv[j + 1] - m_used);
         const __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
         const float2 back = __bfloat1622float2(b2);
-        psum += back.x + back.y;
+        ps[(j >> 1) & 3] += back.x + back.y;
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&b2);
       }
-      l_run = l_run * corr + psum;
+      l_run = l_run * corr + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       // The rescale decision is per head row, but the TMEM accesses below are
       // warp-collective (.sync.aligned): the warp rescales if any lane needs
       // it, and lanes that do not multiply by 1.
       if (__any_sync(0xFFFFFFFFu, corr != 1.f && it > 0)) {
         // O must hold every earlier PV before it is rescaled in place
-        if (!mbar_wait_warp(bar_pv_done((it - 1) & 1), ((it - 1) >> 1) & 1, abort_flag, 31)) { ok = false; break; }
+        if (!mbar_wait_warp(bar_pv_done((it - 1) % C::NSB), ((it - 1) / C::NSB) & 1, abort_flag, 31)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
 #pragma unroll 1
         for (int c0 = 0; c0 < C::DVS; c0 += 16) {
@@ -403,20 +454,22 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
         tmem_wait_st();
       }
-      // P row h (bf16 pairs) into tensor memory; the PV MMA reads it from there
-      tmem_st16(tmem + lane_base + C::TMEM_P + sb * (C::BN / 2), pk);
+      // P row h (bf16 pairs) over the scores of this tile (already in registers);
+      // the PV MMA reads it from there
+      tmem_st16(tmem + lane_base + C::TMEM_S + sb * C::BN, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p_full(sb));
 #pragma unroll
       for (int c = 0; c < C::BN; ++c) sv[c] = s_next[c];
     }
+    if (C::SPLIT == 2 && h == 0) bulk_wait_group<0>();   // outgoing copies have completed
     if (lane == 0) DSA_PROF_SPAN(63, t_role);
     // ------------------------------------------------------------ epilogue
     const int t_out = static_cast<int>(t);
     if (ok && n_tiles > 0) {
       const int j = n_tiles - 1;
-      ok = mbar_wait_warp(bar_pv_done(j & 1), (j >> 1) & 1, abort_flag, 32);
+      ok = mbar_wait_warp(bar_pv_done(j % C::NSB), (j / C::NSB) & 1, abort_flag, 32);
       tc_fence_after();
     }
     // every lane takes part in the warp-collective TMEM loads; only rows h < H are stored
