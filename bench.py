@@ -271,8 +271,9 @@ def gpu_arm(args, rank, world):
         achieved = w["flops"] / launches / (per_launch_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
-    roof["kernel"] = {"indexer": "indexer_scores_kernel", "topk": "topk_radix_kernel",
-                      "attention": "sparse_mla_kernel"}[dom]
+    persistent = idx_fp8 and all(q == 1 for q in spec.q_lens) and spec.B <= 2048
+    roof["kernel"] = {"indexer": "indexer_persistent_kernel" if persistent else "indexer_scores_kernel",
+                      "topk": "topk_kernel", "attention": "sparse_mla_kernel"}[dom]
     roof["traffic"] = load_traffic(dom, spec.name, w["bytes"] / launches)
     roof["peak_source"] = f"{peaks_src} ({'MEASURED_PEAKS.json' if peaks_src == 'measured' else 'recipe fallback'})"
     # whole-step roofline: sum over stages of max(bytes / HBM, flops / TC)
