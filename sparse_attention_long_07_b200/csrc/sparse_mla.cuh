@@ -56,18 +56,23 @@ struct MlaCfg {
   static constexpr int NA0 = SPLIT_ATOM;                  // atoms gathered by rank 0
   static constexpr int NA1 = NATOM_ALL - SPLIT_ATOM;      // atoms gathered by rank 1
   static constexpr int NA_MAX = NA0 > NA1 ? NA0 : NA1;
-  static constexpr int NS = SPLIT == 1 ? 4 : 8;           // gather ring depth
+  static constexpr int NS = SPLIT == 1 ? 4 : 6;           // gather ring depth
   static constexpr int C_ATOM_BYTES = BN * SWB;
   static constexpr int C_STAGE = NA_MAX * C_ATOM_BYTES;
   static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;   // one partial-score tile
   static constexpr int OFF_C = 0;
-  static constexpr int OFF_X = OFF_C + NS * C_STAGE;      // two received partial-score tiles
-  static constexpr int OFF_XS = OFF_X + 2 * X_BYTES;      // two staged outgoing tiles
+  // Received partial-score tiles: tile j lands in buffer j % XR.  With four
+  // buffers a CTA never has to be told that the peer is done with one: the
+  // peer sent tile j - 2 (which this CTA waited for before it sends tile j)
+  // only after it had consumed tile j - 4, the buffer's previous content.
+  static constexpr int XR = 4;
+  static constexpr int OFF_X = OFF_C + NS * C_STAGE;
+  static constexpr int OFF_XS = OFF_X + XR * X_BYTES;     // two staged outgoing tiles
   static constexpr int OFF_MASK = OFF_XS + 2 * X_BYTES;
   static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
   static constexpr int NSB = 3;                            // S buffers (each later holds its P)
   static constexpr int LOOKAHEAD = 2;                      // QK tiles issued ahead of PV
-  static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + 9;
+  static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + XR + 5;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // tensor memory columns: O [0, DVS); S[NSB] (fp32, BN each; P of the same
@@ -138,12 +143,11 @@ __global__ void __launch_bounds__(C::NT, 1)
   // softmax can never complete a phase twice ahead of the MMA thread's wait
   auto bar_p_full = [&](int a) { return bar0 + 8 * (SB0 + 2 * C::NSB + a); };
   constexpr int XB0 = SB0 + 3 * C::NSB;
-  auto bar_x_full = [&](int b) { return bar0 + 8 * (XB0 + b); };
-  auto bar_x_empty = [&](int b) { return bar0 + 8 * (XB0 + 2 + b); };
-  const uint32_t bar_drain = bar0 + 8 * (XB0 + 4);
+  auto bar_x_full = [&](int b) { return bar0 + 8 * (XB0 + b); };          // b < XR
+  const uint32_t bar_drain = bar0 + 8 * (XB0 + C::XR);
   // outgoing staging buffer b: every row written (128 arrivals) / read by its copy (thread 0)
-  auto bar_xs_full = [&](int b) { return bar0 + 8 * (XB0 + 5 + b); };
-  auto bar_xs_free = [&](int b) { return bar0 + 8 * (XB0 + 7 + b); };
+  auto bar_xs_full = [&](int b) { return bar0 + 8 * (XB0 + C::XR + 1 + b); };
+  auto bar_xs_free = [&](int b) { return bar0 + 8 * (XB0 + C::XR + 3 + b); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* ntiles_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -163,10 +167,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       mbar_init(bar_pv_done(a), 1);
       mbar_init(bar_p_full(a), 128);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_x_full(b), 1);    // armed locally; filled by the peer's bulk copy
-      mbar_init(bar_x_empty(b), 4);   // one release-arrive per softmax warp of the peer
-    }
+    for (int b = 0; b < C::XR; ++b) mbar_init(bar_x_full(b), 1);   // armed locally; filled by the peer's copy
     mbar_init(bar_drain, 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_xs_full(b), 128);
@@ -309,7 +310,6 @@ __global__ void __launch_bounds__(C::NT, 1)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t x_peer = C::SPLIT == 2 ? mapa_shared(smem_u32(xbuf), peer) : 0u;
     const uint32_t bar_x_full_peer0 = C::SPLIT == 2 ? mapa_shared(bar_x_full(0), peer) : 0u;
-    const uint32_t bar_x_empty_peer0 = C::SPLIT == 2 ? mapa_shared(bar_x_empty(0), peer) : 0u;
     float m_used = -INFINITY;    // running max (log2 units) the exponentials are taken against
     float l_run = 0.f;
     bool ok = true;
@@ -348,9 +348,10 @@ __global__ void __launch_bounds__(C::NT, 1)
       if (C::SPLIT == 2) {
         // The tile goes to the peer in one bulk copy: every thread stages its
         // row in this CTA's buffer xb, then thread 0 copies the 128 rows.
-        const int xb = j & 1;
+        const int xb = j & 1;        // staging buffer
+        const int xr = j % C::XR;    // receive buffer of tile j, on both CTAs
         // receive side: arm tile j's phase with the bytes the peer will send
-        if (h == 0) mbar_arrive_expect_tx(bar_x_full(xb), C::X_BYTES);
+        if (h == 0) mbar_arrive_expect_tx(bar_x_full(xr), C::X_BYTES);
         // staging buffer xb is free once the copy of tile j-2 has read it
         if (!mbar_wait_warp(bar_xs_free(xb), ((j >> 1) & 1) ^ 1, abort_flag, 33)) return false;
         float* row = xs + xb * (C::X_BYTES / 4) + h * C::BN;
@@ -364,12 +365,11 @@ __global__ void __launch_bounds__(C::NT, 1)
         mbar_arrive(bar_xs_full(xb));
         int go = 1;
         if (h == 0) {
-          // all rows staged, and the peer has released its receive buffer xb (tile j-2)
-          go = mbar_wait(bar_xs_full(xb), (j >> 1) & 1, abort_flag, 34) &&
-               mbar_wait<true>(bar_x_empty(xb), ((j >> 1) & 1) ^ 1, abort_flag, 27);
+          // all rows staged (the peer's buffer xr is free: see XR)
+          go = mbar_wait(bar_xs_full(xb), (j >> 1) & 1, abort_flag, 34);
           if (go) {
-            bulk_copy_to_peer(x_peer + xb * C::X_BYTES, smem_u32(xs) + xb * C::X_BYTES, C::X_BYTES,
-                              bar_x_full_peer0 + 8 * xb);
+            bulk_copy_to_peer(x_peer + xr * C::X_BYTES, smem_u32(xs) + xb * C::X_BYTES, C::X_BYTES,
+                              bar_x_full_peer0 + 8 * xr);
             bulk_commit_group();
             // the copy of tile j-1 has read staging buffer xb ^ 1: tile j+1 may refill it
             if (j >= 1) {
@@ -389,9 +389,10 @@ __global__ void __launch_bounds__(C::NT, 1)
       const int sb = it % C::NSB;   // S buffer of this tile; its P goes there too
       if (it + 1 < n_tiles && !load_and_push(it + 1, s_next)) { ok = false; break; }
       if (C::SPLIT == 2) {
-        const int xb = it & 1;
-        if (!mbar_wait_warp<true>(bar_x_full(xb), (it >> 1) & 1, abort_flag, 28)) { ok = false; break; }
-        const float* xrow = xbuf + xb * (C::X_BYTES / 4) + h * C::BN;
+        // the copy completes on this CTA's own barrier: CTA-scope acquire, as for a TMA load
+        const int xr = it % C::XR;
+        if (!mbar_wait_warp(bar_x_full(xr), (it / C::XR) & 1, abort_flag, 28)) { ok = false; break; }
+        const float* xrow = xbuf + xr * (C::X_BYTES / 4) + h * C::BN;
 #pragma unroll
         for (int c = 0; c < C::BN / 4; ++c) {
           const int slot = (c + h) & (C::BN / 4 - 1);
@@ -401,10 +402,6 @@ __global__ void __launch_bounds__(C::NT, 1)
           sv[4 * c + 2] += v.z;
           sv[4 * c + 3] += v.w;
         }
-        // this warp's 32 rows of buffer xb are read: hand them back to the peer
-        // (one release-arrive per warp; no CTA-wide barrier inside the loop)
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(bar_x_empty_peer0 + 8 * xb);
       }
       // validity of the tile's entries (written by the producer before it armed c_full)
       if (!mbar_wait_warp(bar_c_full(it % C::NS), (it / C::NS) & 1, abort_flag, 29)) { ok = false; break; }
