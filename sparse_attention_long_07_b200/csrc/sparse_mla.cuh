@@ -56,7 +56,7 @@ struct MlaCfg {
   static constexpr int NA0 = SPLIT_ATOM;                  // atoms gathered by rank 0
   static constexpr int NA1 = NATOM_ALL - SPLIT_ATOM;      // atoms gathered by rank 1
   static constexpr int NA_MAX = NA0 > NA1 ? NA0 : NA1;
-  static constexpr int NS = SPLIT == 1 ? 4 : 6;           // gather ring depth
+  static constexpr int NS = SPLIT == 1 ? 4 : 7;           // gather ring depth
   static constexpr int C_ATOM_BYTES = BN * SWB;
   static constexpr int C_STAGE = NA_MAX * C_ATOM_BYTES;
   static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;   // one partial-score tile
@@ -67,8 +67,8 @@ struct MlaCfg {
   // only after it had consumed tile j - 4, the buffer's previous content.
   static constexpr int XR = 4;
   static constexpr int OFF_X = OFF_C + NS * C_STAGE;
-  static constexpr int OFF_XS = OFF_X + XR * X_BYTES;     // two staged outgoing tiles
-  static constexpr int OFF_MASK = OFF_XS + 2 * X_BYTES;
+  static constexpr int OFF_XS = OFF_X + XR * X_BYTES;     // the staged outgoing tile
+  static constexpr int OFF_MASK = OFF_XS + X_BYTES;
   static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
   static constexpr int NSB = 3;                            // S buffers (each later holds its P)
   static constexpr int LOOKAHEAD = 2;                      // QK tiles issued ahead of PV
@@ -145,9 +145,9 @@ __global__ void __launch_bounds__(C::NT, 1)
   constexpr int XB0 = SB0 + 3 * C::NSB;
   auto bar_x_full = [&](int b) { return bar0 + 8 * (XB0 + b); };          // b < XR
   const uint32_t bar_drain = bar0 + 8 * (XB0 + C::XR);
-  // outgoing staging buffer b: every row written (128 arrivals) / read by its copy (thread 0)
-  auto bar_xs_full = [&](int b) { return bar0 + 8 * (XB0 + C::XR + 1 + b); };
-  auto bar_xs_free = [&](int b) { return bar0 + 8 * (XB0 + C::XR + 3 + b); };
+  // outgoing staging buffer: every row written (128 arrivals) / read by the previous copy (thread 0)
+  const uint32_t bar_xs_full = bar0 + 8 * (XB0 + C::XR + 1);
+  const uint32_t bar_xs_free = bar0 + 8 * (XB0 + C::XR + 2);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* ntiles_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -169,10 +169,8 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
     for (int b = 0; b < C::XR; ++b) mbar_init(bar_x_full(b), 1);   // armed locally; filled by the peer's copy
     mbar_init(bar_drain, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_xs_full(b), 128);
-      mbar_init(bar_xs_free(b), 1);
-    }
+    mbar_init(bar_xs_full, 128);
+    mbar_init(bar_xs_free, 1);
     *abort_flag = 0;
     *ntiles_s = 0;
     // an error recorded earlier by any CTA of this library: skip the work
@@ -347,14 +345,19 @@ __global__ void __launch_bounds__(C::NT, 1)
       for (int c = 0; c < C::BN; ++c) dst[c] = __uint_as_float(raw[c]);
       if (C::SPLIT == 2) {
         // The tile goes to the peer in one bulk copy: every thread stages its
-        // row in this CTA's buffer xb, then thread 0 copies the 128 rows.
-        const int xb = j & 1;        // staging buffer
+        // row in this CTA's staging buffer, then thread 0 copies the 128 rows.
         const int xr = j % C::XR;    // receive buffer of tile j, on both CTAs
-        // receive side: arm tile j's phase with the bytes the peer will send
-        if (h == 0) mbar_arrive_expect_tx(bar_x_full(xr), C::X_BYTES);
-        // staging buffer xb is free once the copy of tile j-2 has read it
-        if (!mbar_wait_warp(bar_xs_free(xb), ((j >> 1) & 1) ^ 1, abort_flag, 33)) return false;
-        float* row = xs + xb * (C::X_BYTES / 4) + h * C::BN;
+        if (h == 0) {
+          // receive side: arm tile j's phase with the bytes the peer will send
+          mbar_arrive_expect_tx(bar_x_full(xr), C::X_BYTES);
+          // the copy of tile j-1 (an iteration ago) has read the staging buffer
+          if (j >= 1) {
+            bulk_wait_group_read<0>();
+            mbar_arrive(bar_xs_free);
+          }
+        }
+        if (j >= 1 && !mbar_wait_warp(bar_xs_free, (j - 1) & 1, abort_flag, 33)) return false;
+        float* row = xs + h * C::BN;
 #pragma unroll
         for (int c = 0; c < C::BN / 4; ++c) {
           const int slot = (c + h) & (C::BN / 4 - 1);   // rotate 16-byte chunks: no bank conflicts
@@ -362,20 +365,14 @@ __global__ void __launch_bounds__(C::NT, 1)
                                                                    dst[4 * c + 3]);
         }
         fence_proxy_async_smem();
-        mbar_arrive(bar_xs_full(xb));
+        mbar_arrive(bar_xs_full);
         int go = 1;
         if (h == 0) {
           // all rows staged (the peer's buffer xr is free: see XR)
-          go = mbar_wait(bar_xs_full(xb), (j >> 1) & 1, abort_flag, 34);
+          go = mbar_wait(bar_xs_full, j & 1, abort_flag, 34);
           if (go) {
-            bulk_copy_to_peer(x_peer + xr * C::X_BYTES, smem_u32(xs) + xb * C::X_BYTES, C::X_BYTES,
-                              bar_x_full_peer0 + 8 * xr);
+            bulk_copy_to_peer(x_peer + xr * C::X_BYTES, smem_u32(xs), C::X_BYTES, bar_x_full_peer0 + 8 * xr);
             bulk_commit_group();
-            // the copy of tile j-1 has read staging buffer xb ^ 1: tile j+1 may refill it
-            if (j >= 1) {
-              bulk_wait_group_read<1>();
-              mbar_arrive(bar_xs_free(xb ^ 1));
-            }
           }
         }
         // warp 0 leaves together if thread 0 gave up; other warps see the abort flag
