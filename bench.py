@@ -71,11 +71,27 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The slowest rank's time (NCCL group: a device tensor; gloo, as in the CPU
+    tests of this path: a host tensor)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_spec(spec, rank, world):
+    """Weak scaling: every rank serves its own batch of the same shape (its own seed)."""
+    if world == 1:
+        return spec
+    import dataclasses
+    return dataclasses.replace(spec, seed=spec.seed + 1000 * rank)
+
+
+def aggregate_throughput(tokens_per_rank, ms_per_step, world):
+    """Whole-job query tokens/s: all ranks' tokens over the max-over-ranks step time."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
 
 
 # --------------------------------------------------------------------------- algorithmic work
@@ -186,10 +202,7 @@ def pick_chunk(spec):
 def gpu_arm(args, rank, world):
     import sparse_attention_long_07_b200 as dsa
 
-    spec = di.config(args.workload)
-    if world > 1:                        # each rank serves its own batch of sequences
-        import dataclasses
-        spec = dataclasses.replace(spec, seed=spec.seed + 1000 * rank)
+    spec = rank_spec(di.config(args.workload), rank, world)   # each rank serves its own batch
     idx_fp8 = spec.kfp8
     dev = torch.device("cuda", torch.cuda.current_device())
     d = di.make_inputs(spec, device=dev)
@@ -249,7 +262,7 @@ def gpu_arm(args, rank, world):
         stage_ms["attention"] += e[2].elapsed_time(e[3])
     stage_ms = {n: t / args.steps for n, t in stage_ms.items()}   # per step
     ms_per_step = elapsed_ms / args.steps
-    value = world * T / (ms_per_step / 1e3)
+    value = aggregate_throughput(T, ms_per_step, world)
 
     # ---------------------------------------------------------------- e2e (public API, host buffers)
     e2e = e2e_measure(dsa, spec, d, v, q_chunk, args, world)
