@@ -13,12 +13,14 @@
 // sum over heads stay inside one thread and the [T x L x H_I] logits never
 // leave the SM; only the fp32 score per (query, key) is written.
 //
-// Roles: one TMA warp streams key tiles through a shared-memory ring; one
-// thread issues the MMAs into two TMEM accumulators (double buffer); one or two
-// epilogue warpgroups drain them.  For an e4m3 index-key cache, four more
-// warps widen each raw tile to bf16 in the UMMA layout (exact: every e4m3 value
-// is a bf16 value), and the per-key fp32 scale multiplies the head-reduced
-// score (a positive scale commutes with ReLU).
+// Roles (query-block grid): one TMA warp streams key tiles through a
+// shared-memory ring; one thread issues the MMAs into two TMEM accumulators;
+// one or two epilogue warpgroups drain them.  For an e4m3 index-key cache, four
+// more warps widen each raw tile to bf16 in the shared-memory UMMA layout
+// (exact: every e4m3 value is a bf16 value), and the per-key fp32 scale
+// multiplies the head-reduced score (a positive scale commutes with ReLU).
+// The persistent decode schedule (below) widens keys into tensor memory
+// instead, and issues MMAs from two threads.
 #pragma once
 
 #include "common.cuh"
