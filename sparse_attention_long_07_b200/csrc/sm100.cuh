@@ -115,13 +115,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-// Arrive on an mbarrier of another CTA of the cluster (address from mapa),
-// releasing this thread's earlier writes at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
-               : "memory");
-}
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -427,24 +420,6 @@ __device__ __forceinline__ void bulk_wait_group() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float a, float b, float c,
-                                              float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a),
-               "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
-// Asynchronous store into another CTA's shared memory that completes 16
-// transaction bytes on that CTA's mbarrier (no fence needed on this side).
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, float b, float c, float d,
-                                            uint32_t cluster_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-          cluster_addr),
-      "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
-      : "memory");
-}
-
 __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
   uint32_t v;
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
@@ -457,8 +432,5 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // Named barrier over `nthreads` threads (multiple of 32) of this CTA.
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 }  // namespace dsa
