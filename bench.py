@@ -433,7 +433,37 @@ def cpu_rows_target(cores):
     return max(2, min(16, cores))
 
 
+REFERENCE_BUDGET_S = 150.0     # oracle work of one whole --impl reference run, all steps
+
+
+def _truncated_rows(spec, d_cpu, seqs, m):
+    """One query row per sequence over the first min(kv_len, m) keys of its
+    cache (the row's query placed at the last of those positions)."""
+    cu_k = [int(x) for x in d_cpu["cu_k"]]
+    cu_q = [int(x) for x in d_cpu["cu_q"]]
+    out = {n: [] for n in ("q_idx", "w", "q", "k_idx", "k_scale", "latent")}
+    lens = []
+    for i, b in enumerate(seqs):
+        n = min(spec.kv_lens[b], m)
+        lens.append(n)
+        for name in ("q_idx", "w", "q"):
+            out[name].append(d_cpu[name][cu_q[i + 1] - 1:cu_q[i + 1]])
+        for name in ("k_idx", "latent") + (("k_scale",) if spec.kfp8 else ()):
+            out[name].append(d_cpu[name][cu_k[i]:cu_k[i] + n])
+    d = {name: (torch.cat(v) if v else None) for name, v in out.items()}
+    d["cu_q"] = di.cu_seqlens([1] * len(seqs))
+    d["cu_k"] = di.cu_seqlens(lens)
+    return d, lens
+
+
 def reference_arm(args, rank, world):
+    """The oracle as it stands, on the host cores.  Decode: every step runs one
+    query row per core (the first sequences of the batch, in parallel).  With
+    few steps the rows keep their whole caches; with many, each row's cache is
+    cut to its first m keys, m sized so that all steps together cost about
+    REFERENCE_BUDGET_S of oracle time, and the step is credited with the
+    fraction of a whole-cache step it represents, from a per-row time model
+    T(n) = a + b n + c min(k, n) fitted on three cut lengths (untimed)."""
     if rank != 0:
         return None
     spec = di.config(args.workload)
@@ -441,16 +471,68 @@ def reference_arm(args, rank, world):
     oracle.build()
     cores = oracle.num_threads()
     rows = cpu_rows_target(cores)
-    for _ in range(args.warmup):
-        pass                                      # the oracle has no warm-up state
-    times = []
-    vals = []
-    sample = None
-    for _ in range(max(1, args.steps)):
-        v, dt, sample, used = run_oracle(spec, rows)
-        vals.append(v)
-        times.append(dt)
-    value = len(times) * 1.0 / sum(1.0 / v for v in vals)      # harmonic mean of per-step throughput
+    steps = max(1, args.steps)
+    decode = all(q == 1 for q in spec.q_lens)
+    times, tokens = [], 0.0
+    if decode:
+        seqs = oracle_sample(spec, rows)
+        d_cpu = di.make_inputs(spec, seqs=seqs)     # generated once for all steps
+        full = [spec.kv_lens[b] for b in seqs]
+
+        def run(m):
+            d, lens = _truncated_rows(spec, d_cpu, seqs, m)
+            t0 = time.perf_counter()
+            oracle.forward(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"], d["k_scale"], d["q"],
+                           d["latent"], spec.topk, spec.softmax_scale, spec.d_v)
+            return time.perf_counter() - t0, lens
+
+        # Calibration (untimed): the step time of this sample as a function of the
+        # cache length n, T(n) = a + b n + c min(k, n) (overhead, per-key work of
+        # the indexer and top-k, per-selected-row work of the attention), fitted
+        # exactly through three cut lengths.
+        k = spec.topk
+        pts = [max(64, k // 4), k, 4 * k]
+        ts = [run(n)[0] for n in pts]
+        n1, n2, n3 = pts
+        bc = (ts[1] - ts[0]) / (n2 - n1)                     # b + c (n <= k)
+        b_ = max((ts[2] - ts[1]) / (n3 - n2), 1e-12)          # n > k: only b grows
+        c_ = max(bc - b_, 0.0)
+        a_ = max(ts[0] - bc * n1, 0.0)
+
+        def t_row(n):
+            return a_ + b_ * n + c_ * min(k, n)
+
+        per_step = REFERENCE_BUDGET_S / steps
+        m = 64
+        while m < max(full) and t_row(2 * m) <= per_step:
+            m *= 2
+        if t_row(max(full)) <= per_step:
+            m = max(full)
+
+        # A whole-cache step yields one token per row in the time of its longest
+        # row (the rows run in parallel); a cut step is credited in proportion.
+        t_full = max(t_row(f) for f in full)
+
+        def frac_tokens(lens):
+            return len(lens) * max(t_row(n) for n in lens) / t_full
+
+        for _ in range(steps):
+            dt, lens = run(m)
+            times.append(dt)
+            tokens += frac_tokens(lens)
+        whole = m >= max(full)
+        sample = (f"{len(seqs)} of {spec.B} decode sequences, one query row each, "
+                  + ("whole caches" if whole else
+                     f"caches cut to their first {m} keys; a step counts {len(seqs)} x T(cut)/T(whole) tokens, "
+                     f"T(n) = a + b n + c min(k, n) per row fitted on cuts of {pts} keys "
+                     f"(a={a_:.3g} s, b={b_:.3g} s/key, c={c_:.3g} s/row), T(whole) of the longest row"))
+        used = min(cores, len(seqs))
+    else:
+        for _ in range(steps):
+            v, dt, sample, used = run_oracle(spec, rows)
+            times.append(dt)
+            tokens += v * dt
+    value = tokens / sum(times)
     ms = 1e3 * sum(times) / len(times)
     cb = {"value": value, "unit": "query tokens/s", "cores": used, "kind": "oracle", "sample": sample}
     return {
