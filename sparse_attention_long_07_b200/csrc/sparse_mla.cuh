@@ -28,9 +28,10 @@
 // softmax decisions.  Tensor memory holds O, three score buffers (a tile's P,
 // in bf16, overwrites its scores once they are in registers) and this CTA's
 // slice of the query, the A operand of every QK MMA, so shared memory is left
-// to a seven-deep ring of gathered rows and the score exchange.  The online softmax keeps a per-head running max
-// and only rescales O (in TMEM) when the max grows by more than 2^8, which
-// is exact arithmetic with the same final normalisation.
+// to a seven-deep ring of gathered rows and the score exchange.  The online
+// softmax keeps a per-head running max and only rescales O (in TMEM) when the
+// max grows by more than 2^8, which is exact arithmetic with the same final
+// normalisation.
 //
 // Roles per CTA: warps 0-3 query load, softmax and epilogue (one head row per
 // thread), warp 4 gather producer, warp 5 MMA issuer (and TMEM owner).
