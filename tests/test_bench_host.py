@@ -50,3 +50,40 @@ def test_cut_cache_sample_keeps_each_rows_query_and_its_first_keys():
         assert torch.equal(cut["q_idx"][i], d["q_idx"][b])          # one query row per sequence
         a = int(cut["cu_k"][i])
         assert torch.equal(cut["latent"][a:a + lens[i]], d["latent"][cu_k[b]:cu_k[b] + lens[i]])
+
+
+def test_bench_line_carries_every_contract_key(monkeypatch, capsys):
+    """The JSON line main() prints, with the GPU arm and the oracle timing
+    replaced by fixed results (no device here)."""
+    fake_roof = {"bound": "tensor", "achieved": 250.0, "peak": 1364.1, "unit": "TFLOP/s", "frac": 0.18,
+                 "kernel": "sparse_mla_kernel", "traffic": 169466112, "peak_source": "measured"}
+    spec = di.config("decode128k")
+
+    def fake_gpu_arm(args, rank, world):
+        return {"value": 1.0e5, "ms_per_step": 0.64, "stage_ms": {"indexer": 0.2, "topk": 0.1, "attention": 0.3},
+                "roofline": fake_roof, "step_roofline_frac": 0.3,
+                "e2e": {"value": 5.0e4, "unit": "query tokens/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 2},
+                "gpu_launches": 3 * args.steps, "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
+                "config": bench.describe(spec, spec.kfp8), "q_chunk": 0, "inputs": None}
+
+    monkeypatch.setattr(bench, "gpu_arm", fake_gpu_arm)
+    monkeypatch.setattr(bench, "run_oracle", lambda spec, rows, d_full=None: (1.5, 10.0, "sample", 8))
+    monkeypatch.setattr(bench, "dist_setup", lambda n: (0, 1, 0))
+    monkeypatch.setattr("sys.argv", ["bench.py", "--steps", "5", "--warmup", "3"])
+    bench.main()
+    import json
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks",
+                "cpu_baseline"):
+        assert key in line, key
+    assert line["steps"] == 5 and line["warmup"] == 3 and line["n_gpus"] == 1
+    assert line["higher_is_better"] is True and line["scaling"] == "weak"
+    assert line["config"]["workload"] == "decode128k"
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in line["roofline"], key
+    for key in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
+        assert key in line["e2e"], key
+    for key in ("value", "unit", "cores", "kind", "sample"):
+        assert key in line["cpu_baseline"], key
+    assert line["cpu_baseline"]["kind"] == "oracle"
