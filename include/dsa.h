@@ -109,7 +109,8 @@ dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_i
  *           -1.  With pos+1 <= topk that is 0..pos.  The SET is the
  *           definition; the order within a row is unspecified but
  *           deterministic, so repeated runs are bit-identical.
- * topk in [1, 2048].  Scores must not be NaN.
+ * topk in [1, 2048].  Scores must not be NaN.  Rows longer than 1,040,384
+ * keys return DSA_ERR_UNSUPPORTED (nothing launched).
  */
 dsa_status dsa_topk(const float* scores, int64_t ld_scores, dsa_varlen v, int64_t q_begin,
                     int64_t q_end, int32_t topk, int32_t* idx, cudaStream_t stream);
@@ -131,7 +132,9 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, dsa_varlen v, int64_
  * out       bf16 [T, n_heads, d_v] global rows; lse fp32 [T, n_heads] (nullable).
  *           A row with no valid entry gets out = 0 and lse = -inf.
  * QK and PV run on the tensor cores (bf16 in, fp32 accumulate); the softmax
- * probabilities are rounded to bf16 for PV.  topk must be a multiple of 64.
+ * probabilities are rounded to bf16 for PV.  topk in [1, 2048]; any value in
+ * that range (the rows are processed in tiles of 32 and the tail of the last
+ * tile is skipped).
  */
 dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t* idx,
                                dsa_varlen v, int64_t q_begin, int64_t q_end, int32_t topk,
@@ -154,7 +157,8 @@ size_t dsa_forward_workspace_size(dsa_varlen v, int32_t topk, int64_t q_chunk);
  * row, [T, topk] int32, global rows.  workspace: device, at least
  * dsa_forward_workspace_size(v, topk, q_chunk) bytes, 256-byte aligned.
  * Prefill, chunked prefill and decode are the same call: they differ only in
- * the lengths held by v.
+ * the lengths held by v.  Every pass's argument and launch-limit checks run
+ * before the first launch, so an error status means nothing was launched.
  */
 dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
                        const float* k_scale, dsa_kidx_dtype k_dtype, const void* q,
@@ -176,14 +180,20 @@ dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
  * file-scope device array of DSA_STATIC_SCRATCH_BYTES, which every GPU that
  * loads the library keeps until the process exits.  Inputs and outputs are
  * still the caller's, exactly as for dsa_forward; the query rows are processed
- * in the largest passes whose scratch fits the array.  Returns
- * DSA_ERR_WORKSPACE (nothing launched) when even one query row's scores and
- * selections do not fit, i.e. when the longest kv_len reaches ~8M keys.
- * Calls no cudaMalloc, cudaFree or other allocating routine.
+ * in the largest passes whose scratch fits the array.  The array holds one
+ * query row of any layout the top-k supports (rows up to 1,040,384 keys;
+ * longer rows return DSA_ERR_UNSUPPORTED as for dsa_forward); were a row's
+ * scores and selections ever larger than the array, the call would return
+ * DSA_ERR_WORKSPACE.  Either way nothing is launched.  Calls no cudaMalloc,
+ * cudaFree or other allocating routine.
  *
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  All calls on a device share the array and it
+ * Device memory for the array: the CUDA runtime loads this library's device
+ * code on a device lazily, at the first call into the library there (of any
+ * entry point), and that load allocates the array and may synchronise the
+ * device.  The first call of this entry point on a device also looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current).
+ * So make one warm-up call per device before serving starts and before any
+ * stream capture.  All calls on a device share the array and it
  * keeps the last call's contents; nothing in it needs to start at zero (every
  * score and selection is written before it is read).  Calls whose kernels
  * overlap on the GPU (other streams, other host threads) race on the array:
@@ -210,6 +220,17 @@ dsa_status dsa_device_error(int32_t* code, cudaStream_t stream);
  * builds return DSA_ERR_UNSUPPORTED and touch nothing.  No counterpart on the
  * pages: it exists to attribute kernel time to pipeline stages. */
 dsa_status dsa_debug_wait_profile(uint64_t* cycles, uint64_t* counts, int32_t n, int32_t reset);
+
+/* Diagnostics: exercises the bounded-wait timeout path on the GPU without
+ * faulting or hanging it.  Launches one CTA (one warp) on `stream` whose only
+ * work is one bounded wait on an mbarrier that nothing ever arrives on; after
+ * limit_cycles device cycles (1 .. 2e9; about 1 ms per 2e6 cycles at the
+ * boost clock) the wait gives up the way every wait of the DSA kernels does:
+ * it records 1 | (99 << 8) (timeout, wait site 99) in the device error word
+ * and the kernel returns.  Read and clear the word with dsa_device_error()
+ * before the next real call: kernels that start while it is set skip their
+ * work.  No counterpart on the pages: it exists to test failure detection. */
+dsa_status dsa_debug_wait_selftest(int64_t limit_cycles, cudaStream_t stream);
 
 /* Static description of a status code. */
 const char* dsa_status_string(dsa_status status);

@@ -68,6 +68,8 @@ def _load():
     lib.dsa_forward_static_scratch.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp, dsa_varlen, i32, i32, i32,
                                                i32, i32, i32, f32, vp, vp, vp, vp]
     lib.dsa_forward_static_scratch.restype = ctypes.c_int
+    lib.dsa_debug_wait_selftest.argtypes = [i64, vp]
+    lib.dsa_debug_wait_selftest.restype = ctypes.c_int
     for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward", "dsa_device_error"):
         getattr(lib, fn).restype = ctypes.c_int
     return lib
@@ -75,7 +77,7 @@ def _load():
 
 EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward_workspace_size",
             "dsa_forward", "dsa_device_error", "dsa_status_string", "dsa_version", "dsa_debug_wait_profile",
-            "dsa_forward_static_scratch")
+            "dsa_forward_static_scratch", "dsa_debug_wait_selftest")
 
 # bytes of the library's static scratch array (DSA_STATIC_SCRATCH_BYTES in include/dsa.h)
 DSA_STATIC_SCRATCH_BYTES = 32 << 20
@@ -211,6 +213,12 @@ def dsa_device_error(stream=None) -> int:
     if st not in (DSA_OK, DSA_ERR_DEVICE_TIMEOUT):
         raise DSAError(st, "dsa_device_error")
     return int(code.value)
+
+
+def dsa_debug_wait_selftest(limit_cycles: int, stream=None):
+    """Launch the one-wait self-test kernel whose wait gives up after
+    ``limit_cycles`` device cycles (read the result with dsa_device_error)."""
+    _check(_lib.dsa_debug_wait_selftest(int(limit_cycles), _stream(stream)), "dsa_debug_wait_selftest")
 
 
 def dsa_debug_wait_profile(reset: bool = True):

@@ -116,9 +116,40 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <class K>
-cudaError_t set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+// Per-device state.  Kernel attributes (the dynamic shared-memory limit) and
+// the SM count belong to a device, so they are kept per device ordinal and set
+// up the first time a kernel runs on that device.
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+// Raise Kernel's dynamic shared-memory limit to `bytes` on the current device
+// (once per device).
+template <auto Kernel>
+cudaError_t ensure_smem(int bytes) {
+  static std::once_flag once[kMaxDevices];
+  static cudaError_t err[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev, bytes] {
+    err[dev] = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+  return err[dev];
+}
+
+int num_sms() {
+  static std::once_flag once[kMaxDevices];
+  static int n[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return 0;
+  std::call_once(once[dev], [dev] {
+    if (cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n[dev] = 0;
+  });
+  return n[dev];
 }
 
 bool is_released_indexer(int h, int d) { return h == 64 && d == 128; }
@@ -149,10 +180,7 @@ dsa_status launch_indexer(const void* q_idx, const float* w, const void* k_idx,
                   C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
       return DSA_ERR_CUDA;
   }
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] { attr_err = set_smem(dsa::indexer_scores_kernel<C>, C::SMEM_BYTES); });
-  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  if (ensure_smem<dsa::indexer_scores_kernel<C>>(C::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
 
   dsa::IndexerParams p;
   p.w = w;
@@ -168,23 +196,10 @@ dsa_status launch_indexer(const void* q_idx, const float* w, const void* k_idx,
   const int qblocks = (L.max_q_rows + C::NQ - 1) / C::NQ;
   const int chunks = (L.max_tiles + p.chunk_tiles - 1) / p.chunk_tiles;
   if (qblocks == 0 || chunks == 0) return DSA_OK;
-  if (chunks > 65535 || v.batch > 65535) return DSA_ERR_UNSUPPORTED;
-  if (qblocks > 65535) return DSA_ERR_UNSUPPORTED;   // gridDim.y limit
+  if (qblocks > 65535 || v.batch > 65535) return DSA_ERR_UNSUPPORTED;   // checked by indexer_limits first
   dim3 grid(chunks, qblocks, v.batch);
   dsa::indexer_scores_kernel<C><<<grid, C::NT, C::SMEM_BYTES, stream>>>(tm_q, tm_k, p);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
-}
-
-int num_sms() {
-  static int n = 0;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      n = 0;
-  });
-  return n;
 }
 
 // Decode-like calls: one persistent CTA per SM over the flat (sequence, key tile) list.
@@ -212,10 +227,7 @@ dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const vo
   if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_idx, C::D_I, static_cast<uint64_t>(L.S), C::D_I, C::D_I,
                 C::BK, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] { attr_err = set_smem(dsa::indexer_persistent_kernel<C>, C::SMEM_BYTES); });
-  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  if (ensure_smem<dsa::indexer_persistent_kernel<C>>(C::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
   dsa::IndexerParams p;
   p.w = w;
   p.k_scale = k_scale;
@@ -242,10 +254,7 @@ dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, con
   if (!make_map(&tm_lat, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, latent, C::DQK, static_cast<uint64_t>(L.S),
                 C::DQK * 2, C::ATOM, 1, swz))
     return DSA_ERR_CUDA;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] { attr_err = set_smem(dsa::sparse_mla_kernel<C>, C::SMEM_BYTES); });
-  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
+  if (ensure_smem<dsa::sparse_mla_kernel<C>>(C::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
 
   dsa::MlaParams p;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -279,8 +288,9 @@ dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, con
 dsa_status check_indexer_args(const void* q_idx, const float* w, const void* k_idx,
                               const float* k_scale, dsa_kidx_dtype kd, int h, int d,
                               const float* scores, int64_t ld, const Layout& L) {
-  if (!q_idx || !w || !k_idx || !scores) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || !aligned16(scores))
+  // scores == nullptr: the score buffer is validated by the caller (dsa_forward's workspace)
+  if (!q_idx || !w || !k_idx) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || (scores && !aligned16(scores)))
     return DSA_ERR_INVALID_ARG;
   if (kd != DSA_KIDX_BF16 && kd != DSA_KIDX_FP8_E4M3) return DSA_ERR_INVALID_ARG;
   if (kd == DSA_KIDX_FP8_E4M3 && !k_scale) return DSA_ERR_INVALID_ARG;
@@ -292,8 +302,9 @@ dsa_status check_indexer_args(const void* q_idx, const float* w, const void* k_i
 
 dsa_status check_mla_args(const void* q, const void* latent, const int32_t* idx, int topk, int h,
                           int dqk, int dv, float scale, const void* out, const float* lse) {
-  if (!q || !latent || !idx || !out) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(latent) || !aligned16(idx) || !aligned16(out) ||
+  // idx == nullptr: the selections are validated by the caller (dsa_forward)
+  if (!q || !latent || !out) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(latent) || (idx && !aligned16(idx)) || !aligned16(out) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return DSA_ERR_INVALID_ARG;
   if (topk < 1 || topk > 2048) return DSA_ERR_INVALID_ARG;
@@ -302,43 +313,76 @@ dsa_status check_mla_args(const void* q, const void* latent, const int32_t* idx,
   return DSA_ERR_UNSUPPORTED;
 }
 
+// Which indexer kernel a pass uses.  Decode-like passes (at most one query row
+// per sequence) over an e4m3 cache take the persistent kernel; otherwise the
+// query-block grid kernel with 1 or 4 queries per CTA.
+enum class IndexerKind { kTiny, kPersistent, kGridFp8x1, kGridFp8x4, kGridBf16x1, kGridBf16x4 };
+
+IndexerKind choose_indexer(dsa_kidx_dtype kd, int h, int d, const dsa_varlen& v, const Layout& L) {
+  if (is_tiny_indexer(h, d)) return IndexerKind::kTiny;
+  const bool decode_like = L.max_q_rows <= 2;
+  if (kd == DSA_KIDX_FP8_E4M3) {
+    if (L.max_q_rows <= 1 && v.batch <= IndexerCfg<64, 128, 1, true, true>::MAX_SEQ) return IndexerKind::kPersistent;
+    return decode_like ? IndexerKind::kGridFp8x1 : IndexerKind::kGridFp8x4;
+  }
+  return decode_like ? IndexerKind::kGridBf16x1 : IndexerKind::kGridBf16x4;
+}
+
+// Launch limits of one indexer pass, checked before anything is launched.
+dsa_status indexer_limits(dsa_kidx_dtype kd, int h, int d, const dsa_varlen& v, const Layout& L) {
+  if (L.max_q_rows == 0) return DSA_OK;
+  const IndexerKind k = choose_indexer(kd, h, d, v, L);
+  if (k == IndexerKind::kPersistent) return DSA_OK;
+  const int nq = (k == IndexerKind::kGridFp8x1 || k == IndexerKind::kGridBf16x1) ? 1 : 4;
+  const int64_t qblocks = (L.max_q_rows + nq - 1) / nq;
+  if (qblocks > 65535 || v.batch > 65535) return DSA_ERR_UNSUPPORTED;   // gridDim.y / gridDim.z
+  return DSA_OK;
+}
+
 dsa_status run_indexer(const void* q_idx, const float* w, const void* k_idx, const float* k_scale,
                        dsa_kidx_dtype kd, const dsa_varlen& v, const Layout& L, int h, int d,
                        int64_t q_begin, int64_t q_end, float* scores, int64_t ld,
                        cudaStream_t stream) {
   if (q_end == q_begin) return DSA_OK;
-  const bool decode_like = L.max_q_rows <= 2;
-  if (is_tiny_indexer(h, d))
-    return launch_indexer<IndexerCfg<4, 32, 4, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
-                                                        scores, ld, stream);
-  if (kd == DSA_KIDX_FP8_E4M3) {
-    using Persist = IndexerCfg<64, 128, 1, true, true>;
-    if (L.max_q_rows <= 1 && v.batch <= Persist::MAX_SEQ)
-      return launch_indexer_persistent<Persist>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end, scores, ld,
-                                                stream);
-    if (decode_like)
-      return launch_indexer<IndexerCfg<64, 128, 1, true>>(q_idx, w, k_idx, k_scale, v, L, q_begin,
-                                                           q_end, scores, ld, stream);
-    return launch_indexer<IndexerCfg<64, 128, 4, true>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
-                                                         scores, ld, stream);
+  switch (choose_indexer(kd, h, d, v, L)) {
+    case IndexerKind::kTiny:
+      return launch_indexer<IndexerCfg<4, 32, 4, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                          scores, ld, stream);
+    case IndexerKind::kPersistent:
+      return launch_indexer_persistent<IndexerCfg<64, 128, 1, true, true>>(q_idx, w, k_idx, k_scale, v, L,
+                                                                           q_begin, q_end, scores, ld, stream);
+    case IndexerKind::kGridFp8x1:
+      return launch_indexer<IndexerCfg<64, 128, 1, true>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                           scores, ld, stream);
+    case IndexerKind::kGridFp8x4:
+      return launch_indexer<IndexerCfg<64, 128, 4, true>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                           scores, ld, stream);
+    case IndexerKind::kGridBf16x1:
+      return launch_indexer<IndexerCfg<64, 128, 1, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                            scores, ld, stream);
+    case IndexerKind::kGridBf16x4:
+      return launch_indexer<IndexerCfg<64, 128, 4, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                            scores, ld, stream);
   }
-  if (decode_like)
-    return launch_indexer<IndexerCfg<64, 128, 1, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin,
-                                                          q_end, scores, ld, stream);
-  return launch_indexer<IndexerCfg<64, 128, 4, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
-                                                        scores, ld, stream);
+  return DSA_ERR_UNSUPPORTED;
 }
+
+// Launch limits of one top-k pass: one CTA per row; rows up to MAX_N keys.
+dsa_status topk_limits(const Layout& L, int64_t rows) {
+  if (rows > 0x7FFFFFFF) return DSA_ERR_UNSUPPORTED;
+  if (L.max_kv > dsa::TopkCfg::MAX_N) return DSA_ERR_UNSUPPORTED;   // 16-bit pass-1 counters
+  return DSA_OK;
+}
+
+// Launch limits of one attention pass: one cluster of SPLIT CTAs per row.
+dsa_status mla_limits(int64_t rows) { return rows * 2 > 0x7FFFFFFF ? DSA_ERR_UNSUPPORTED : DSA_OK; }
 
 dsa_status run_topk(const float* scores, int64_t ld, const dsa_varlen& v, const Layout& L,
                     int64_t q_begin, int64_t q_end, int topk, int32_t* idx, cudaStream_t stream) {
   const int64_t rows = q_end - q_begin;
   if (rows == 0) return DSA_OK;
-  if (rows > 0x7FFFFFFF) return DSA_ERR_UNSUPPORTED;
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] { attr_err = set_smem(dsa::topk_kernel, dsa::TopkCfg::SMEM_BYTES); });
-  if (attr_err != cudaSuccess) return DSA_ERR_CUDA;
-  if (L.max_kv > dsa::TopkCfg::MAX_N) return DSA_ERR_UNSUPPORTED;   // 16-bit pass-1 counters
+  if (topk_limits(L, rows) != DSA_OK) return DSA_ERR_UNSUPPORTED;
+  if (ensure_smem<dsa::topk_kernel>(dsa::TopkCfg::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
   dsa::topk_kernel<<<static_cast<unsigned>(rows), dsa::TopkCfg::NT, dsa::TopkCfg::SMEM_BYTES, stream>>>(
       scores, ld, v.cu_q, v.cu_k, v.batch, q_begin, topk, idx);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
@@ -371,8 +415,10 @@ dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_i
   Layout L;
   dsa_status st = check_varlen(v, q_begin, q_end, &L);
   if (st != DSA_OK) return st;
+  if (!scores) return DSA_ERR_INVALID_ARG;
   st = check_indexer_args(q_idx, w, k_idx, k_scale, k_dtype, n_idx_heads, idx_dim, scores, ld_scores, L);
   if (st != DSA_OK) return st;
+  if ((st = indexer_limits(k_dtype, n_idx_heads, idx_dim, v, L)) != DSA_OK) return st;
   if ((st = injected_fault()) != DSA_OK) return st;
   return run_indexer(q_idx, w, k_idx, k_scale, k_dtype, v, L, n_idx_heads, idx_dim, q_begin, q_end,
                      scores, ld_scores, stream);
@@ -386,6 +432,7 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, dsa_varlen v, int64_
   if (!scores || !idx || !aligned16(scores) || (reinterpret_cast<uintptr_t>(idx) & 3u))
     return DSA_ERR_INVALID_ARG;
   if (topk < 1 || topk > 2048 || ld_scores < L.max_kv || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+  if ((st = topk_limits(L, q_end - q_begin)) != DSA_OK) return st;
   if ((st = injected_fault()) != DSA_OK) return st;
   return run_topk(scores, ld_scores, v, L, q_begin, q_end, topk, idx, stream);
 }
@@ -397,8 +444,10 @@ dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t*
   Layout L;
   dsa_status st = check_varlen(v, q_begin, q_end, &L);
   if (st != DSA_OK) return st;
+  if (!idx) return DSA_ERR_INVALID_ARG;
   st = check_mla_args(q, latent, idx, topk, n_heads, d_qk, d_v, scale, out, lse);
   if (st != DSA_OK) return st;
+  if ((st = mla_limits(q_end - q_begin)) != DSA_OK) return st;
   if ((st = injected_fault()) != DSA_OK) return st;
   return run_mla(q, latent, idx, v, L, q_begin, q_end, topk, n_heads, d_qk, d_v, scale, out, lse,
                  stream);
@@ -414,6 +463,46 @@ size_t dsa_forward_workspace_size(dsa_varlen v, int32_t topk, int64_t q_chunk) {
          align_up(static_cast<size_t>(std::max<int64_t>(rows, 1)) * topk * sizeof(int32_t));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Every check of a dsa_forward call that does not involve the workspace:
+// arguments, supported shapes and each pass's launch limits.  Host arithmetic
+// only (no CUDA call).
+dsa_status forward_checks(const void* q_idx, const float* w, const void* k_idx, const float* k_scale,
+                          dsa_kidx_dtype k_dtype, const void* q, const void* latent, const dsa_varlen& v,
+                          int32_t n_idx_heads, int32_t idx_dim, int32_t topk, int32_t n_heads, int32_t d_qk,
+                          int32_t d_v, float scale, int64_t q_chunk, const void* out, const float* lse,
+                          const int32_t* idx_out) {
+  if (v.batch < 1 || !v.cu_q_host) return DSA_ERR_INVALID_ARG;
+  Layout full;
+  dsa_status st = check_varlen(v, 0, v.cu_q_host[v.batch], &full);
+  if (st != DSA_OK) return st;
+  const int64_t ld = scores_ld(full);
+  // the score buffer is the (256-byte aligned) workspace: checked by the caller
+  st = check_indexer_args(q_idx, w, k_idx, k_scale, k_dtype, n_idx_heads, idx_dim, nullptr, ld, full);
+  if (st != DSA_OK) return st;
+  if (idx_out && (reinterpret_cast<uintptr_t>(idx_out) & 15u)) return DSA_ERR_INVALID_ARG;
+  st = check_mla_args(q, latent, nullptr, topk, n_heads, d_qk, d_v, scale, out, lse);
+  if (st != DSA_OK) return st;
+  const int64_t T = full.T;
+  const int64_t rows = q_chunk > 0 ? std::min<int64_t>(q_chunk, T) : T;
+  for (int64_t q0 = 0; q0 < T; q0 += rows) {
+    const int64_t q1 = std::min(T, q0 + rows);
+    Layout L;
+    if ((st = check_varlen(v, q0, q1, &L)) != DSA_OK) return st;
+    if ((st = indexer_limits(k_dtype, n_idx_heads, idx_dim, v, L)) != DSA_OK) return st;
+    if ((st = topk_limits(L, q1 - q0)) != DSA_OK) return st;
+    if ((st = mla_limits(q1 - q0)) != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
                        const float* k_scale, dsa_kidx_dtype k_dtype, const void* q,
                        const void* latent, dsa_varlen v, int32_t n_idx_heads,
@@ -421,24 +510,19 @@ dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
                        int32_t d_v, float scale, int64_t q_chunk, void* out, float* lse,
                        int32_t* idx_out, void* workspace, size_t workspace_bytes,
                        cudaStream_t stream) {
-  if (v.batch < 1 || !v.cu_q_host) return DSA_ERR_INVALID_ARG;
-  Layout full;
-  dsa_status st = check_varlen(v, 0, v.cu_q_host[v.batch], &full);
+  dsa_status st = forward_checks(q_idx, w, k_idx, k_scale, k_dtype, q, latent, v, n_idx_heads, idx_dim, topk,
+                                 n_heads, d_qk, d_v, scale, q_chunk, out, lse, idx_out);
   if (st != DSA_OK) return st;
   if (!workspace) return DSA_ERR_WORKSPACE;
-  const int64_t ld = scores_ld(full);
-  st = check_indexer_args(q_idx, w, k_idx, k_scale, k_dtype, n_idx_heads, idx_dim,
-                          static_cast<const float*>(workspace), ld, full);
-  if (st != DSA_OK) return st;
-  st = check_mla_args(q, latent, idx_out ? idx_out : static_cast<const int32_t*>(workspace), topk,
-                      n_heads, d_qk, d_v, scale, out, lse);
-  if (st != DSA_OK) return st;
   if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign) return DSA_ERR_INVALID_ARG;
   const size_t need = dsa_forward_workspace_size(v, topk, q_chunk);
   if (need == 0) return DSA_ERR_INVALID_ARG;
   if (workspace_bytes < need) return DSA_ERR_WORKSPACE;
   if ((st = injected_fault()) != DSA_OK) return st;
 
+  Layout full;
+  check_varlen(v, 0, v.cu_q_host[v.batch], &full);
+  const int64_t ld = scores_ld(full);
   const int64_t T = full.T;
   const int64_t rows = q_chunk > 0 ? std::min<int64_t>(q_chunk, T) : T;
   float* scores = static_cast<float*>(workspace);
@@ -467,7 +551,6 @@ dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
 static __device__ __align__(256) uint8_t g_dsa_static_scratch[DSA_STATIC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
 std::once_flag g_scratch_once[kMaxDevices];
 void* g_scratch_ptr[kMaxDevices];
 cudaError_t g_scratch_err[kMaxDevices];
@@ -492,6 +575,9 @@ dsa_status dsa_forward_static_scratch(const void* q_idx, const float* w, const v
     if (dsa_forward_workspace_size(v, topk, mid) <= DSA_STATIC_SCRATCH_BYTES) lo = mid; else hi = mid - 1;
   }
   const int64_t q_chunk = lo;
+  dsa_status st = forward_checks(q_idx, w, k_idx, k_scale, k_dtype, q, latent, v, n_idx_heads, idx_dim, topk,
+                                 n_heads, d_qk, d_v, scale, q_chunk, out, lse, idx_out);
+  if (st != DSA_OK) return st;
   // the array's device address, looked up once per device with that device current
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
@@ -512,6 +598,36 @@ dsa_status dsa_device_error(int32_t* code, cudaStream_t stream) {
   if (cudaMemcpyToSymbol(dsa::g_device_error, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
   *code = v;
   return v == 0 ? DSA_OK : DSA_ERR_DEVICE_TIMEOUT;
+}
+
+}  // extern "C"
+
+namespace dsa {
+// One bounded wait on an mbarrier that nothing arrives on: it gives up after
+// limit_cycles, records the timeout (site kSelftestSite) in the device error
+// word and returns, exactly as the waits of the DSA kernels do.  No copy or
+// MMA is in flight, so the CTA can leave at once.
+constexpr int kSelftestSite = 99;
+__global__ void wait_selftest_kernel(long long limit_cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, kSelftestSite, limit_cycles);
+}
+}  // namespace dsa
+
+extern "C" {
+
+dsa_status dsa_debug_wait_selftest(int64_t limit_cycles, cudaStream_t stream) {
+  if (limit_cycles < 1 || limit_cycles > 2000000000LL) return DSA_ERR_INVALID_ARG;
+  if (injected_fault() != DSA_OK) return injected_fault();
+  dsa::wait_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<long long>(limit_cycles));
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status dsa_debug_wait_profile(uint64_t* cycles, uint64_t* counts, int32_t n, int32_t reset) {

@@ -146,7 +146,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // raises the flag.  Every role polls the same flag, so a CTA always drains.
 template <bool kClusterScope = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int site = 0) {
+                                          int site = 0, long long limit_cycles = kWaitLimitCycles) {
   long long t0 = 0;
 #ifdef DSA_PROFILE_WAITS
   const long long t_enter = clock64();
@@ -164,7 +164,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       long long now = clock64();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > kWaitLimitCycles) {
+      } else if (now - t0 > limit_cycles) {
         record_device_error(kErrWaitTimeout | (site << 8));
         *abort_flag = 1;
         return false;

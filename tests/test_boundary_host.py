@@ -1,7 +1,11 @@
 """Host-side tests of the C-ABI library: it loads, exports every entry point
 declared in include/dsa.h, and rejects invalid arguments on the host before
-any CUDA call (so these run without a GPU).  Device pointers here are fake,
-aligned addresses: validation never dereferences them."""
+any CUDA call (so these run without a GPU).  The validation tests pass
+invented, aligned "device" addresses that validation never dereferences; they
+run only where no GPU is present, so that a regression in the order of the
+checks can never launch a kernel on addresses that are not mapped.  Without a
+GPU, a call that got as far as a CUDA call would return DSA_ERR_CUDA instead of
+the expected status, so these tests also prove that nothing was launched."""
 import ctypes
 import os
 import re
@@ -48,6 +52,9 @@ def test_status_strings(dsa):
 
 FAKE = 1 << 20  # an aligned, never-dereferenced "device" address
 
+host_only = pytest.mark.skipif(torch.cuda.is_available(),
+                               reason="passes invented device addresses: runs only where no GPU is present")
+
 
 def fake(n=1):
     return [FAKE * (i + 1) for i in range(n)]
@@ -71,6 +78,7 @@ def scores_call(dsa, v, q_begin=0, q_end=None, ld=None, h=64, d=128, kd=0, ptrs=
     return lib.dsa_indexer_scores(p[0], p[1], p[2], kscale, kd, v, h, d, q_begin, q_end, p[3], ld, None)
 
 
+@host_only
 def test_indexer_argument_validation(dsa):
     INV, UNS = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED
     ok = varlen([0, 3, 5], [0, 10, 300])
@@ -90,6 +98,7 @@ def test_indexer_argument_validation(dsa):
     assert scores_call(dsa, ok, h=4, d=32, kd=1) == UNS                       # tiny shape is bf16 only
 
 
+@host_only
 def test_topk_and_attention_validation(dsa):
     lib = dsa.library()
     INV, UNS = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED
@@ -112,6 +121,7 @@ def test_topk_and_attention_validation(dsa):
     assert mla(dqk=512) == UNS
 
 
+@host_only
 def test_forward_workspace_contract(dsa):
     lib = dsa.library()
     v = varlen([0, 3, 5], [0, 10, 301])
@@ -132,6 +142,7 @@ def test_forward_workspace_contract(dsa):
     assert fwd(FAKE, need, h_i=8) == dsa.DSA_ERR_UNSUPPORTED
 
 
+@host_only
 def test_injected_faults_are_reported_without_launching(dsa, monkeypatch):
     lib = dsa.library()
     v = varlen([0, 3], [0, 10])
@@ -149,3 +160,32 @@ def test_binding_raises_on_bad_status(dsa):
         dsa.dsa_indexer_scores(q_idx, torch.zeros(2, 64), torch.zeros(1, 128, dtype=torch.bfloat16), None, v, 0,
                                2, torch.zeros(2, 4), stream=0)
     assert e.value.status == dsa.DSA_ERR_INVALID_ARG
+
+
+@host_only
+def test_layouts_beyond_the_launch_limits_are_rejected_before_any_launch(dsa):
+    """Rows longer than the top-k supports: every entry point returns
+    DSA_ERR_UNSUPPORTED before launching anything (the indexer of the first
+    pass included), and the static-scratch forward returns DSA_ERR_WORKSPACE
+    for a row whose scores alone exceed its array."""
+    lib = dsa.library()
+    f = ctypes.c_float(0.07)
+    long_row = varlen([0, 1], [0, 2_000_000])           # past the top-k row limit
+    assert lib.dsa_topk(FAKE, 2_000_000, long_row, 0, 1, 2048, FAKE, None) == dsa.DSA_ERR_UNSUPPORTED
+    need = lib.dsa_forward_workspace_size(long_row, 2048, 0)
+    assert need > 0
+    assert lib.dsa_forward(FAKE, FAKE, FAKE, None, 0, FAKE, FAKE, long_row, 64, 128, 2048, 128, 576, 512, f, 0,
+                           FAKE, FAKE, None, FAKE, need, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_forward_static_scratch(FAKE, FAKE, FAKE, None, 0, FAKE, FAKE, long_row, 64, 128, 2048, 128,
+                                          576, 512, f, FAKE, FAKE, None, None) == dsa.DSA_ERR_UNSUPPORTED
+    kv = (dsa.DSA_STATIC_SCRATCH_BYTES // 4) + 1000     # one row of scores alone exceeds the array
+    huge = varlen([0, 1], [0, kv])
+    assert lib.dsa_forward_static_scratch(FAKE, FAKE, FAKE, None, 0, FAKE, FAKE, huge, 64, 128, 2048, 128, 576,
+                                          512, f, FAKE, FAKE, None, None) == dsa.DSA_ERR_WORKSPACE
+
+
+@host_only
+def test_self_test_arguments(dsa):
+    lib = dsa.library()
+    assert lib.dsa_debug_wait_selftest(0, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_debug_wait_selftest(3_000_000_000, None) == dsa.DSA_ERR_INVALID_ARG

@@ -8,8 +8,6 @@ Each case calls it twice in a row (the array keeps the previous call's
 contents) and compares both results with dsa_forward given a caller
 workspace, within the parity tolerances of the other GPU tests.  The file is
 named so that pytest collects it last."""
-import ctypes
-
 import numpy as np
 import pytest
 import torch
@@ -75,16 +73,3 @@ def test_static_scratch_matches_workspace_forward_on_two_calls(dsa, name):
             assert np.all(idx[r][len(a):] == -1)
         P.assert_attention_close(out, lse, ref_out.astype(np.float64), ref_lse.astype(np.float64),
                                  f"{name} call {call}")
-
-
-def test_static_scratch_rejects_layouts_beyond_its_size(dsa):
-    lib = dsa.library()
-    kv = (dsa.DSA_STATIC_SCRATCH_BYTES // 4) + 1000      # one row of scores alone exceeds the array
-    cu_q = (ctypes.c_int32 * 2)(0, 1)
-    cu_k = (ctypes.c_int32 * 2)(0, kv)
-    fake = 1 << 20                                        # never dereferenced: rejected on the host
-    v = dsa.dsa_varlen(1, fake, fake, ctypes.cast(cu_q, ctypes.POINTER(ctypes.c_int32)),
-                       ctypes.cast(cu_k, ctypes.POINTER(ctypes.c_int32)))
-    st = lib.dsa_forward_static_scratch(fake, fake, fake, None, 0, fake, fake, v, 64, 128, 2048, 128, 576, 512,
-                                        ctypes.c_float(0.07), fake, fake, None, None)
-    assert st == dsa.DSA_ERR_WORKSPACE
