@@ -51,6 +51,18 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
+SUSTAINED_AFTER_S = 2.0   # timed regions longer than this run into the power cap
+
+
+def tc_peak_for(peaks, region_s):
+    """bf16 tensor peak (TF/s) that applies to kernels timed in a region of
+    region_s seconds: the burst figure for short regions, the sustained one
+    for long ones."""
+    if region_s >= SUSTAINED_AFTER_S and "bf16_tflops_sustained" in peaks:
+        return peaks["bf16_tflops_sustained"], "sustained"
+    return peaks["bf16_tflops"], "burst"
+
+
 def dist_setup(n_gpus):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -266,23 +278,28 @@ def gpu_arm(args, rank, world):
 
     # ---------------------------------------------------------------- e2e (public API, host buffers)
     e2e = e2e_measure(dsa, spec, d, v, q_chunk, args, world)
+    peaks, peaks_src = load_peaks()
+    # the indexer on a long causal prefill (its dense tensor-core regime), 1 GPU only
+    idx_prefill = None
+    if world == 1 and not args.no_indexer_prefill and args.workload == "decode128k":
+        idx_prefill = indexer_prefill_measure(dsa, args, peaks)
 
     # ---------------------------------------------------------------- roofline of the dominant kernel
-    peaks, peaks_src = load_peaks()
     work = work_model(spec, idx_fp8)
     dom = max(stage_ms, key=stage_ms.get)
     launches = len(chunks)
     per_launch_ms = stage_ms[dom] / launches
     w = work[dom]
     hbm_t = w["bytes"] / (peaks["hbm_gbs"] * 1e9)
-    tc_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tc_peak, tc_kind = tc_peak_for(peaks, elapsed_ms / 1e3)
     tc_t = w["flops"] / (tc_peak * 1e12)
     if hbm_t >= tc_t:
         achieved = w["bytes"] / launches / (per_launch_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     else:
         achieved = w["flops"] / launches / (per_launch_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                "peak_kind": f"bf16 {tc_kind}"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     persistent = idx_fp8 and all(q == 1 for q in spec.q_lens) and spec.B <= 2048
     roof["kernel"] = {"indexer": "indexer_persistent_kernel" if persistent else "indexer_scores_kernel",
@@ -296,7 +313,7 @@ def gpu_arm(args, rank, world):
         "value": value, "ms_per_step": ms_per_step, "stage_ms": {n: round(t, 4) for n, t in stage_ms.items()},
         "roofline": roof, "step_roofline_frac": round(t_roof * 1e3 / ms_per_step, 4), "e2e": e2e,
         "gpu_launches": 3 * launches * args.steps, "clocks": clocks, "config": describe(spec, idx_fp8),
-        "q_chunk": q_chunk, "inputs": d,
+        "q_chunk": q_chunk, "inputs": d, "indexer_prefill": idx_prefill,
     }
 
 
@@ -314,60 +331,139 @@ def load_traffic(stage, workload, alg_bytes_per_launch):
         return None
 
 
+INDEXER_PREFILL_WORKLOAD = "prefill32k"
+
+
+def indexer_prefill_measure(dsa, args, peaks):
+    """The indexer stage alone on the 32K-token causal prefill (the O(L^2)
+    dense contraction of the method), timed with CUDA events over a few
+    launches: flops = causal (query, key) pairs x 2 x H_I x d_I."""
+    spec = di.config(INDEXER_PREFILL_WORKLOAD)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    d = di.make_inputs(spec, device=dev, tensors=("q_idx", "w", "k_idx"))
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], dev)
+    ld = (max(spec.kv_lens) + 3) // 4 * 4
+    scores = torch.empty((spec.T, ld), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def launch():
+        dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, spec.T, scores, stream)
+
+    for _ in range(3):
+        launch()
+    torch.cuda.synchronize()
+    n = 5
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        a.record(stream)
+        for _ in range(n):
+            launch()
+        b.record(stream)
+        torch.cuda.synchronize()
+    assert dsa.dsa_device_error() == 0
+    ms = a.elapsed_time(b) / n
+    flops = work_model(spec, False)["indexer"]["flops"]
+    tflops = flops / (ms / 1e3) / 1e12
+    del d, scores
+    torch.cuda.empty_cache()
+    return {"workload": spec.name, "launches": n, "ms_per_launch": round(ms, 4), "tflops": round(tflops, 1),
+            "flops_per_launch": flops, "kernel": "indexer_scores_kernel (4 queries per CTA)",
+            "frac_of_burst_peak": round(tflops / peaks["bf16_tflops"], 4),
+            "frac_of_sustained_peak": round(tflops / peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]), 4),
+            "clocks": clk.summary()}
+
+
+class _E2ELane:
+    """One batch in flight for the end-to-end measurement: its own stream,
+    device inputs, pinned host copies of the step's inputs, outputs and
+    workspace."""
+
+    def __init__(self, dsa, spec, d, v, q_chunk, decode):
+        dev = d["q"].device
+        self.spec, self.d, self.v, self.q_chunk, self.decode = spec, d, v, q_chunk, decode
+        self.stream = torch.cuda.Stream(device=dev)
+        cu_k = [int(x) for x in d["cu_k"]]
+        # decode: the step's new inputs are the query tensors and the new
+        # token's cache rows (the caches are resident device state); prefill:
+        # every input tensor is the step's input
+        self.names = ["q_idx", "w", "q"] + ([] if decode else ["k_idx", "latent"] + (["k_scale"] if spec.kfp8 else []))
+        self.host = {n: d[n].cpu().pin_memory() for n in self.names}
+        self.k_bytes = d["k_idx"].view(torch.uint8) if spec.kfp8 else d["k_idx"]
+        if decode:
+            self.new_rows = torch.tensor([c - 1 for c in cu_k[1:]], dtype=torch.long, device=dev)
+            self.host["k_rows"] = self.k_bytes[self.new_rows].cpu().pin_memory()
+            self.host["lat_rows"] = d["latent"][self.new_rows].cpu().pin_memory()
+            if spec.kfp8:
+                self.host["ks_rows"] = d["k_scale"][self.new_rows].cpu().pin_memory()
+            self.rows_dev = {n: torch.empty(self.host[n].shape, dtype=self.host[n].dtype, device=dev)
+                             for n in ("k_rows", "lat_rows", "ks_rows") if n in self.host}
+        self.out = torch.empty((spec.T, spec.H, spec.d_v), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((spec.T, spec.H), dtype=torch.float32, device=dev)
+        self.out_h = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        self.lse_h = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
+        self.ws = torch.empty(dsa.dsa_forward_workspace_size(v, spec.topk, q_chunk), dtype=torch.uint8, device=dev)
+        self.h2d = sum(t.numel() * t.element_size() for t in self.host.values())
+        self.d2h = self.out_h.numel() * self.out_h.element_size() + self.lse_h.numel() * self.lse_h.element_size()
+
+    def step(self, dsa):
+        d, spec = self.d, self.spec
+        with torch.cuda.stream(self.stream):
+            for n in self.names:
+                d[n].copy_(self.host[n], non_blocking=True)
+            if self.decode:
+                for n, rd in self.rows_dev.items():
+                    rd.copy_(self.host[n], non_blocking=True)
+                self.k_bytes.index_copy_(0, self.new_rows, self.rows_dev["k_rows"])
+                d["latent"].index_copy_(0, self.new_rows, self.rows_dev["lat_rows"])
+                if spec.kfp8:
+                    d["k_scale"].index_copy_(0, self.new_rows, self.rows_dev["ks_rows"])
+            dsa.dsa_forward(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], d["q"], d["latent"], self.v, spec.topk,
+                            spec.softmax_scale, self.out, self.lse, self.ws, q_chunk=self.q_chunk, stream=self.stream)
+            self.out_h.copy_(self.out, non_blocking=True)
+            self.lse_h.copy_(self.lse, non_blocking=True)
+
+
+E2E_MIN_CALLS = 100
+
+
 def e2e_measure(dsa, spec, d, v, q_chunk, args, world):
-    """dsa_forward through the public API with the step's inputs in pinned host
-    memory.  Decode: the step's new inputs are the query tensors and the new
-    token's cache rows (the caches themselves are resident device state);
-    prefill: every input tensor is the step's input."""
+    """dsa_forward through the public API, each step's inputs copied from
+    pinned host memory and its outputs copied back.  Two batches are kept in
+    flight, as a server would: lane 0 serves the benchmark's batch and lane 1
+    another batch of the same shape (other seed), each on its own stream with
+    its own buffers, and the steps alternate between them, so that one lane's
+    host transfers overlap the other lane's kernels.  Every step still copies
+    its whole input in and its whole output out."""
+    import dataclasses
     dev = d["q"].device
     decode = all(q == 1 for q in spec.q_lens)
-    cu_k = [int(x) for x in d["cu_k"]]
-    new_rows = torch.tensor([c - 1 for c in cu_k[1:]], dtype=torch.long, device=dev) if decode else None
-    names = ["q_idx", "w", "q"] + ([] if decode else ["k_idx", "latent"] + (["k_scale"] if spec.kfp8 else []))
-    host = {n: d[n].cpu().pin_memory() for n in names}
-    k_bytes = d["k_idx"].view(torch.uint8) if spec.kfp8 else d["k_idx"]
-    if decode:
-        host["k_rows"] = k_bytes[new_rows].cpu().pin_memory()
-        host["lat_rows"] = d["latent"][new_rows].cpu().pin_memory()
-        host["ks_rows"] = d["k_scale"][new_rows].cpu().pin_memory() if spec.kfp8 else None
-    dev_in = {n: d[n] for n in names}
-    out = torch.empty((spec.T, spec.H, spec.d_v), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((spec.T, spec.H), dtype=torch.float32, device=dev)
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    ws = torch.empty(dsa.dsa_forward_workspace_size(v, spec.topk, q_chunk), dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
-    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
-
-    def one():
-        for n in names:
-            dev_in[n].copy_(host[n], non_blocking=True)
-        if decode:
-            k_bytes.index_copy_(0, new_rows, host["k_rows"].to(dev, non_blocking=True))
-            d["latent"].index_copy_(0, new_rows, host["lat_rows"].to(dev, non_blocking=True))
-            if spec.kfp8:
-                d["k_scale"].index_copy_(0, new_rows, host["ks_rows"].to(dev, non_blocking=True))
-        dsa.dsa_forward(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], d["q"], d["latent"], v, spec.topk,
-                        spec.softmax_scale, out, lse, ws, q_chunk=q_chunk, stream=stream)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
-
-    for _ in range(max(3, args.warmup // 4)):
-        one()
+    spec2 = dataclasses.replace(spec, seed=spec.seed + 500)
+    d2 = di.make_inputs(spec2, device=dev)
+    v2 = type(v)(d2["cu_q"], d2["cu_k"], dev)
+    lanes = [_E2ELane(dsa, spec, d, v, q_chunk, decode), _E2ELane(dsa, spec2, d2, v2, q_chunk, decode)]
+    for i in range(4):
+        lanes[i % 2].step(dsa)
     torch.cuda.synchronize()
-    n = max(3, args.steps // 4)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(E2E_MIN_CALLS, min(args.steps, 1000))
+    start = torch.cuda.Event(enable_timing=True)
+    ends = [torch.cuda.Event(enable_timing=True) for _ in lanes]
     barrier(world)
     torch.cuda.synchronize()
-    a.record(stream)
-    for _ in range(n):
-        one()
-    b.record(stream)
+    start.record(lanes[0].stream)
+    lanes[1].stream.wait_event(start)
+    for i in range(n):
+        lanes[i % 2].step(dsa)
+    for e, ln in zip(ends, lanes):
+        e.record(ln.stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(a.elapsed_time(b), world) / n
+    ms = max_over_ranks(max(start.elapsed_time(e) for e in ends), world) / n
+    assert dsa.dsa_device_error() == 0
+    h2d, d2h = lanes[0].h2d, lanes[0].d2h
+    del lanes, d2
+    torch.cuda.empty_cache()
     return {"value": world * spec.T / (ms / 1e3), "unit": "query tokens/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4), "steps": n}
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4), "steps": n, "api": "dsa_forward",
+            "batches_in_flight": 2}
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -433,115 +529,62 @@ def cpu_rows_target(cores):
     return max(2, min(16, cores))
 
 
-REFERENCE_BUDGET_S = 150.0     # oracle work of one whole --impl reference run, all steps
-
-
-def _truncated_rows(spec, d_cpu, seqs, m):
-    """One query row per sequence over the first min(kv_len, m) keys of its
-    cache (the row's query placed at the last of those positions)."""
-    cu_k = [int(x) for x in d_cpu["cu_k"]]
-    cu_q = [int(x) for x in d_cpu["cu_q"]]
-    out = {n: [] for n in ("q_idx", "w", "q", "k_idx", "k_scale", "latent")}
-    lens = []
-    for i, b in enumerate(seqs):
-        n = min(spec.kv_lens[b], m)
-        lens.append(n)
-        for name in ("q_idx", "w", "q"):
-            out[name].append(d_cpu[name][cu_q[i + 1] - 1:cu_q[i + 1]])
-        for name in ("k_idx", "latent") + (("k_scale",) if spec.kfp8 else ()):
-            out[name].append(d_cpu[name][cu_k[i]:cu_k[i] + n])
-    d = {name: (torch.cat(v) if v else None) for name, v in out.items()}
-    d["cu_q"] = di.cu_seqlens([1] * len(seqs))
-    d["cu_k"] = di.cu_seqlens(lens)
-    return d, lens
+REFERENCE_BUDGET_S = 240.0    # oracle time of one whole --impl reference run
 
 
 def reference_arm(args, rank, world):
-    """The oracle as it stands, on the host cores.  Decode: every step runs one
-    query row per core (the first sequences of the batch, in parallel).  With
-    few steps the rows keep their whole caches; with many, each row's cache is
-    cut to its first m keys, m sized so that all steps together cost about
-    REFERENCE_BUDGET_S of oracle time, and the step is credited with the
-    fraction of a whole-cache step it represents, from a per-row time model
-    T(n) = a + b n + c min(k, n) fitted on three cut lengths (untimed)."""
+    """The oracle as it stands, on the host cores.  Every step runs it on the
+    same bounded sample of the workload, whole caches: for decode one query
+    row per host core (the first sequences of the batch, in parallel); for
+    prefill the last rows of the longest sequence.  Steps stop once
+    REFERENCE_BUDGET_S of oracle time has been spent (at least one step); the
+    sample string says how many ran.  value = query rows timed / oracle time."""
     if rank != 0:
         return None
     spec = di.config(args.workload)
     import oracle
     oracle.build()
     cores = oracle.num_threads()
-    rows = cpu_rows_target(cores)
+    rows_target = cpu_rows_target(cores)
     steps = max(1, args.steps)
     decode = all(q == 1 for q in spec.q_lens)
-    times, tokens = [], 0.0
     if decode:
-        seqs = oracle_sample(spec, rows)
-        d_cpu = di.make_inputs(spec, seqs=seqs)     # generated once for all steps
-        full = [spec.kv_lens[b] for b in seqs]
-
-        def run(m):
-            d, lens = _truncated_rows(spec, d_cpu, seqs, m)
-            t0 = time.perf_counter()
-            oracle.forward(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"], d["k_scale"], d["q"],
-                           d["latent"], spec.topk, spec.softmax_scale, spec.d_v)
-            return time.perf_counter() - t0, lens
-
-        # Calibration (untimed): the step time of this sample as a function of the
-        # cache length n, T(n) = a + b n + c min(k, n) (overhead, per-key work of
-        # the indexer and top-k, per-selected-row work of the attention), fitted
-        # exactly through three cut lengths.
-        k = spec.topk
-        pts = [max(64, k // 4), k, 4 * k]
-        ts = [run(n)[0] for n in pts]
-        n1, n2, n3 = pts
-        bc = (ts[1] - ts[0]) / (n2 - n1)                     # b + c (n <= k)
-        b_ = max((ts[2] - ts[1]) / (n3 - n2), 1e-12)          # n > k: only b grows
-        c_ = max(bc - b_, 0.0)
-        a_ = max(ts[0] - bc * n1, 0.0)
-
-        def t_row(n):
-            return a_ + b_ * n + c_ * min(k, n)
-
-        per_step = REFERENCE_BUDGET_S / steps
-        m = 64
-        while m < max(full) and t_row(2 * m) <= per_step:
-            m *= 2
-        if t_row(max(full)) <= per_step:
-            m = max(full)
-
-        # A whole-cache step yields one token per row in the time of its longest
-        # row (the rows run in parallel); a cut step is credited in proportion.
-        t_full = max(t_row(f) for f in full)
-
-        def frac_tokens(lens):
-            return len(lens) * max(t_row(n) for n in lens) / t_full
-
-        for _ in range(steps):
-            dt, lens = run(m)
-            times.append(dt)
-            tokens += frac_tokens(lens)
-        whole = m >= max(full)
-        sample = (f"{len(seqs)} of {spec.B} decode sequences, one query row each, "
-                  + ("whole caches" if whole else
-                     f"caches cut to their first {m} keys; a step counts {len(seqs)} x T(cut)/T(whole) tokens, "
-                     f"T(n) = a + b n + c min(k, n) per row fitted on cuts of {pts} keys "
-                     f"(a={a_:.3g} s, b={b_:.3g} s/key, c={c_:.3g} s/row), T(whole) of the longest row"))
-        used = min(cores, len(seqs))
+        seqs = oracle_sample(spec, rows_target)
+        d = di.make_inputs(spec, seqs=seqs)         # generated once for all steps (untimed)
+        rows = None
+        sample = f"{len(seqs)} of {spec.B} decode sequences (whole caches), one query row each"
+        n_rows = len(seqs)
     else:
-        for _ in range(steps):
-            v, dt, sample, used = run_oracle(spec, rows)
-            times.append(dt)
-            tokens += v * dt
-    value = tokens / sum(times)
+        b = max(range(spec.B), key=lambda i: spec.kv_lens[i])
+        d = di.make_inputs(spec, seqs=[b])
+        ql = spec.q_lens[b]
+        rows = list(range(max(0, ql - rows_target), ql))
+        sample = f"last {len(rows)} query rows of sequence {b} (kv_len {spec.kv_lens[b]})"
+        n_rows = len(rows)
+    times = []
+    for _ in range(steps):
+        t0 = time.perf_counter()
+        oracle.forward(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"], d["k_scale"], d["q"], d["latent"],
+                       spec.topk, spec.softmax_scale, spec.d_v, rows=rows)
+        times.append(time.perf_counter() - t0)
+        if sum(times) >= REFERENCE_BUDGET_S:
+            break
+    value = n_rows * len(times) / sum(times)
     ms = 1e3 * sum(times) / len(times)
+    used = min(cores, n_rows)
+    sample += f"; {len(times)} of {steps} steps timed (budget {REFERENCE_BUDGET_S:.0f} s)"
     cb = {"value": value, "unit": "query tokens/s", "cores": used, "kind": "oracle", "sample": sample}
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "query tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": describe(spec, spec.kfp8), "cpu_baseline": cb,
+        "config": {**describe(spec, spec.kfp8), "parallelism": parallelism(world)}, "cpu_baseline": cb,
         "e2e": {"value": value, "unit": "query tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+def parallelism(world):
+    return f"replicas x{world} (sequences sharded, no exchange)"
 
 
 METRIC = "DSA query tokens/s (indexer+top-k+sparse MLA) at 128K ctx; % of roofline"
@@ -555,6 +598,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="decode128k", choices=list(di.CONFIG_NAMES))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-indexer-prefill", action="store_true",
+                    help="skip the secondary indexer measurement on the 32K prefill")
     args = ap.parse_args()
     if args.impl == "reference":
         args.steps = 1 if args.steps is None else args.steps
@@ -578,10 +623,12 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based generator; shapes of the released layer)",
-            "config": {**r["config"], "parallelism": f"replicas x{world} (sequences sharded, no exchange)"},
+            "config": {**r["config"], "parallelism": parallelism(world)},
             "roofline": r["roofline"], "step_roofline_frac": r["step_roofline_frac"],
             "stage_ms": r["stage_ms"], "e2e": r["e2e"], "gpu_launches": r["gpu_launches"], "clocks": r["clocks"],
         }
+        if r.get("indexer_prefill"):
+            line["indexer_prefill"] = r["indexer_prefill"]
         if world == 1 and not args.no_cpu_baseline:
             spec = di.config(args.workload)
             import oracle

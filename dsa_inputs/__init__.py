@@ -205,11 +205,16 @@ def _dup_map(spec: Spec, b: int, kv_len: int):
     return tgt[keep], src[keep]
 
 
-def make_inputs(spec: Spec, device="cpu", seqs=None):
+ALL_TENSORS = ("q_idx", "w", "q", "latent", "k_idx")
+
+
+def make_inputs(spec: Spec, device="cpu", seqs=None, tensors=ALL_TENSORS):
     """Generate the workload's tensors on `device`.
 
     seqs: optional list of sequence indices; only those sequences are built
     (their values are identical to the same rows of the full workload).
+    tensors: which of q_idx, w, q, latent, k_idx (with k_scale) to build; the
+    others are None (a tensor's values do not depend on which others are built).
 
     Returns a dict with cu_q/cu_k (int32, CPU), q_idx [T,H_I,d_I] bf16,
     w [T,H_I] fp32, k_idx [sum kv,d_I] (bf16, or float8_e4m3fn with
@@ -228,15 +233,22 @@ def make_inputs(spec: Spec, device="cpu", seqs=None):
     d = dict(spec=spec, cu_q=cu_q, cu_k=cu_k, seqs=list(seqs))
     bf = torch.bfloat16
     kind = spec.dist
-    d["q_idx"] = torch.empty((T, spec.H_I, spec.d_I), dtype=bf, device=device)
-    _fill_rows(d["q_idx"], spec.seed, T_QIDX, qrows, spec.H_I * spec.d_I, kind)
-    d["w"] = torch.empty((T, spec.H_I), dtype=torch.float32, device=device)
-    _fill_rows(d["w"], spec.seed, T_W, qrows, spec.H_I, kind, std=1.0 / 8.0)
-    d["q"] = torch.empty((T, spec.H, spec.d_qk), dtype=bf, device=device)
-    _fill_rows(d["q"], spec.seed, T_Q, qrows, spec.H * spec.d_qk, kind)
-    d["latent"] = torch.empty((S, spec.d_qk), dtype=bf, device=device)
-    _fill_rows(d["latent"], spec.seed, T_LAT, krows, spec.d_qk, kind)
-    if spec.kfp8:
+    d.update(q_idx=None, w=None, q=None, latent=None, k_idx=None, k_scale=None)
+    if "q_idx" in tensors:
+        d["q_idx"] = torch.empty((T, spec.H_I, spec.d_I), dtype=bf, device=device)
+        _fill_rows(d["q_idx"], spec.seed, T_QIDX, qrows, spec.H_I * spec.d_I, kind)
+    if "w" in tensors:
+        d["w"] = torch.empty((T, spec.H_I), dtype=torch.float32, device=device)
+        _fill_rows(d["w"], spec.seed, T_W, qrows, spec.H_I, kind, std=1.0 / 8.0)
+    if "q" in tensors:
+        d["q"] = torch.empty((T, spec.H, spec.d_qk), dtype=bf, device=device)
+        _fill_rows(d["q"], spec.seed, T_Q, qrows, spec.H * spec.d_qk, kind)
+    if "latent" in tensors:
+        d["latent"] = torch.empty((S, spec.d_qk), dtype=bf, device=device)
+        _fill_rows(d["latent"], spec.seed, T_LAT, krows, spec.d_qk, kind)
+    if "k_idx" not in tensors:
+        pass
+    elif spec.kfp8:
         kf = torch.empty((S, spec.d_I), dtype=torch.float64, device=device)
         _fill_rows(kf, spec.seed, T_KIDX, krows, spec.d_I, kind)
         # Quantised index-key cache: one fp32 scale per key = amax / 448 (the
@@ -259,6 +271,8 @@ def make_inputs(spec: Spec, device="cpu", seqs=None):
         tgt, src = (m[0] + int(cu_k[i])).to(device), (m[1] + int(cu_k[i])).to(device)
         for name in ("k_idx", "latent") + (("k_scale",) if spec.kfp8 else ()):
             t = d[name]
+            if t is None:
+                continue
             vals = t[src].clone()          # read every source before any write
             t[tgt] = vals
     return d

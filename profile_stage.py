@@ -1,6 +1,6 @@
 """Run one stage of the DSA hot path in a loop, for profilers (ncu).
 
-    python -m sparse_attention_long_07_b200.profile_stage --workload decode128k \
+    python profile_stage.py --workload decode128k \
         --seqs 16 --stage indexer --iters 3
 
 --seqs keeps the first N sequences of the named workload (same values as the
@@ -17,7 +17,7 @@ import sys
 
 import torch
 
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import dsa_inputs as di  # noqa: E402

@@ -28,3 +28,21 @@ def build_library():
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
     return mod.build()
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Largest error-to-limit fractions seen by the parity checks of this session."""
+    try:
+        from tests import parity
+    except ImportError:
+        return
+    if not parity.MARGINS:
+        return
+    worst = {}
+    for what, ratio in parity.MARGINS:
+        key = what.split(" (")[0]
+        if ratio >= worst.get(key, (-1.0, ""))[0]:
+            worst[key] = (ratio, what)
+    terminalreporter.write_sep("-", "parity margins (worst error / limit; 1.0 = at the limit)")
+    for key, (ratio, what) in sorted(worst.items()):
+        terminalreporter.write_line(f"{key:18s} {ratio:.4f}   [{what}]")

@@ -36,20 +36,24 @@ def test_work_model_prefill_counts_causal_pairs():
     assert w["attention"]["flops"] == sel * 2 * spec.H * (spec.d_qk + spec.d_v)
 
 
-def test_cut_cache_sample_keeps_each_rows_query_and_its_first_keys():
-    spec = di.Spec("cut", (1, 1, 1), (40, 7, 100), H_I=4, d_I=32, topk=32, H=4, d_qk=80, d_v=64,
-                   scale=1.0 / math.sqrt(80.0), seed=3)
-    d = di.make_inputs(spec)
-    seqs = [0, 1, 2]
-    cut, lens = bench._truncated_rows(spec, d, seqs, 16)
-    assert lens == [16, 7, 16]
-    assert [int(x) for x in cut["cu_k"]] == [0, 16, 23, 39]
-    assert [int(x) for x in cut["cu_q"]] == [0, 1, 2, 3]
-    cu_k = [int(x) for x in d["cu_k"]]
-    for i, b in enumerate(seqs):
-        assert torch.equal(cut["q_idx"][i], d["q_idx"][b])          # one query row per sequence
-        a = int(cut["cu_k"][i])
-        assert torch.equal(cut["latent"][a:a + lens[i]], d["latent"][cu_k[b]:cu_k[b] + lens[i]])
+def test_reference_arm_times_whole_rows_and_names_its_workload(oracle_lib):
+    """The reference arm on the tiny workload: an exact timing of whole rows,
+    with the GPU line's config keys (parallelism included)."""
+    import argparse
+    args = argparse.Namespace(workload="tiny", steps=2, warmup=0)
+    line = bench.reference_arm(args, 0, 1)
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["config"] == {**bench.describe(di.config("tiny"), False), "parallelism": bench.parallelism(1)}
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and "2 of 2 steps timed" in cb["sample"]
+    assert line["e2e"]["value"] == line["value"]
+    assert bench.reference_arm(args, 1, 2) is None           # only rank 0 runs it
+
+
+def test_tensor_peak_follows_the_length_of_the_timed_region():
+    peaks = {"hbm_gbs": 6538.3, "bf16_tflops": 1674.7, "bf16_tflops_sustained": 1364.1}
+    assert bench.tc_peak_for(peaks, 0.007) == (1674.7, "burst")
+    assert bench.tc_peak_for(peaks, 30.0) == (1364.1, "sustained")
 
 
 def test_bench_line_carries_every_contract_key(monkeypatch, capsys):

@@ -318,8 +318,10 @@ def _full_size(dsa, oracle_lib, name, n_per_seq, q_chunk=0, max_seqs=None):
     assert dsa.dsa_device_error() == 0
     rows = P.sample_rows(dd["cu_q"], n_per_seq, seed=spec.seed)
     if max_seqs is not None:
+        # a seeded sample of sequences, always with the longest and the shortest cache
         g = np.random.default_rng(spec.seed)
         keep = set(int(b) for b in g.choice(spec.B, size=max_seqs, replace=False))
+        keep |= {int(np.argmax(spec.kv_lens)), int(np.argmin(spec.kv_lens))}
         cu_q_l = list(map(int, dd["cu_q"]))
         rows = [t for t in rows if any(cu_q_l[b] <= t < cu_q_l[b + 1] for b in keep)]
     _check_sampled(dsa, oracle_lib, spec, dd, dd["cu_q"], dd["cu_k"], out, lse, idx, rows)
