@@ -72,6 +72,21 @@ def _load():
             lib.oracle_topk.argtypes = [
                 ctypes.c_int, _I32P, _I32P, ctypes.c_int64, _I32P, _F64P, ctypes.c_int64,
                 ctypes.c_int, _I32P]
+            lib.oracle_hadamard.restype = ctypes.c_int
+            lib.oracle_hadamard.argtypes = [ctypes.c_int64, ctypes.c_int, _F64P, _F64P]
+            lib.oracle_double_to_e4m3.restype = ctypes.c_uint8
+            lib.oracle_double_to_e4m3.argtypes = [ctypes.c_double]
+            lib.oracle_quant_e4m3_pow2.restype = ctypes.c_int
+            lib.oracle_quant_e4m3_pow2.argtypes = [ctypes.c_int64, ctypes.c_int, _F64P, vp, _F32P]
+            lib.oracle_indexer_scores_fp8.restype = ctypes.c_int
+            lib.oracle_indexer_scores_fp8.argtypes = [
+                ctypes.c_int, _I32P, _I32P, ctypes.c_int, ctypes.c_int, vp, _F32P, _F64P, vp, _F32P,
+                ctypes.c_int64, _I32P, _F64P, ctypes.c_int64]
+            lib.oracle_rope.restype = ctypes.c_int
+            lib.oracle_rope.argtypes = [ctypes.c_int64, ctypes.c_int, _F64P, _I32P, _F64P, ctypes.c_int64, _F64P]
+            lib.oracle_up_proj.restype = ctypes.c_int
+            lib.oracle_up_proj.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _F64P,
+                                           ctypes.c_int, vp, _F64P]
             for name in ("oracle_sparse_mla", "oracle_dense_mla_masked"):
                 fn = getattr(lib, name)
                 fn.restype = ctypes.c_int
@@ -224,6 +239,100 @@ def forward(cu_q, cu_k, q_idx, w, k_idx, k_scale, q, latent, k, scale, d_v, rows
     ix = topk(cu_q, cu_k, sc, k, rows=rows)
     out, lse = sparse_mla(cu_q, cu_k, q, latent, ix, scale, d_v, rows=rows)
     return sc, ix, out, lse
+
+
+def _f64(x):
+    a, kind = _np(x)
+    if kind == BF16:
+        import torch
+        a = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def hadamard(x):
+    """Orthonormal Sylvester-Hadamard rotation of the last axis (a power of two)."""
+    xa = _f64(x)
+    d = xa.shape[-1]
+    y = np.empty_like(xa)
+    if _load().oracle_hadamard(xa.size // d, d, _ptr(xa, _F64P), _ptr(y, _F64P)) != 0:
+        raise ValueError("oracle_hadamard: the length must be a power of two")
+    return y
+
+
+def double_to_e4m3(v: float) -> int:
+    """The e4m3 byte nearest to v (ties to even, saturating at +-448)."""
+    return int(_load().oracle_double_to_e4m3(float(v)))
+
+
+def quant_e4m3_pow2(x):
+    """Per-vector (last axis) e4m3 quantization with power-of-two scales:
+    (bytes uint8 [..., d], scale float32 [...])."""
+    xa = _f64(x)
+    d = xa.shape[-1]
+    n = xa.size // d
+    q = np.empty(xa.shape, dtype=np.uint8)
+    sc = np.empty(xa.shape[:-1], dtype=np.float32)
+    if _load().oracle_quant_e4m3_pow2(n, d, _ptr(xa, _F64P), q.ctypes.data_as(ctypes.c_void_p),
+                                      _ptr(sc, _F32P)) != 0:
+        raise ValueError("oracle_quant_e4m3_pow2 rejected its arguments")
+    return q, sc
+
+
+def indexer_scores_fp8(cu_q, cu_k, q_bytes, q_scale, w, k_bytes, k_scale, rows=None, ld=None):
+    """Indexer scores with e4m3 index queries [T, H_I, d_I] (scales [T, H_I])
+    and e4m3 index keys [sum kv, d_I] (scales [sum kv]): [n_rows, ld] float64."""
+    lib = _load()
+    cu_q, cu_k = _i32(cu_q), _i32(cu_k)
+    B = cu_q.size - 1
+    T = int(cu_q[-1])
+    qa, _ = _np(q_bytes)
+    ka, _ = _np(k_bytes)
+    T_, H_I, d_I = qa.shape
+    assert T_ == T
+    qs = np.ascontiguousarray(np.asarray(_np(q_scale)[0], dtype=np.float32)).reshape(T, H_I)
+    ks = np.ascontiguousarray(np.asarray(_np(k_scale)[0], dtype=np.float32))
+    wa = np.ascontiguousarray(np.asarray(_np(w)[0], dtype=np.float64)).reshape(T, H_I)
+    kv_lens = np.diff(cu_k)
+    if ld is None:
+        ld = int(kv_lens.max()) if kv_lens.size else 1
+    r, n = _rows(rows, T)
+    out = np.full((n, ld), -np.inf, dtype=np.float64)
+    rc = lib.oracle_indexer_scores_fp8(
+        B, _ptr(cu_q, _I32P), _ptr(cu_k, _I32P), H_I, d_I, qa.ctypes.data_as(ctypes.c_void_p), _ptr(qs, _F32P),
+        _ptr(wa, _F64P), ka.ctypes.data_as(ctypes.c_void_p), _ptr(ks, _F32P), n,
+        None if r is None else _ptr(r, _I32P), _ptr(out, _F64P), ld)
+    if rc != 0:
+        raise ValueError("oracle_indexer_scores_fp8 rejected its arguments")
+    return out
+
+
+def rope(x, pos, freqs):
+    """Rotary embedding of the last axis (consecutive pairs as complex numbers)
+    by the table freqs [max_pos, d/2, 2] = (cos, sin) at each vector's position."""
+    xa = _f64(x)
+    d = xa.shape[-1]
+    n = xa.size // d
+    pa = _i32(np.broadcast_to(np.asarray(pos), xa.shape[:-1]).reshape(-1))
+    fa = np.ascontiguousarray(np.asarray(freqs, dtype=np.float64))
+    y = np.empty_like(xa)
+    if _load().oracle_rope(n, d, _ptr(xa, _F64P), _ptr(pa, _I32P), _ptr(fa, _F64P), fa.shape[0],
+                           _ptr(y, _F64P)) != 0:
+        raise ValueError("oracle_rope rejected its arguments")
+    return y
+
+
+def up_proj(o, w_uv):
+    """Per-head up-projection y[r, h, :] = o[r, h, :] @ w_uv[h] ([n, H, d_c] x [H, d_c, d_v])."""
+    oa = _f64(o)
+    wa, wk = _np(w_uv)
+    n, H, d_c = oa.shape
+    H_, d_c_, d_v = wa.shape
+    assert (H_, d_c_) == (H, d_c)
+    y = np.empty((n, H, d_v), dtype=np.float64)
+    if _load().oracle_up_proj(n, H, d_c, d_v, _ptr(oa, _F64P), wk, wa.ctypes.data_as(ctypes.c_void_p),
+                              _ptr(y, _F64P)) != 0:
+        raise ValueError("oracle_up_proj rejected its arguments")
+    return y
 
 
 class use_library:

@@ -121,10 +121,10 @@ int oracle_num_threads(void) {
  * q_idx: [T, H_I, d_I]; w: [T, H_I] (double); k_idx: [sum kv, d_I] with, for
  * E4M3, one float32 scale per key row.
  */
-int oracle_indexer_scores(int B, const int32_t* cu_q, const int32_t* cu_k, int H_I, int d_I,
-                          int q_kind, const void* q_idx, const double* w, int k_kind,
-                          const void* k_idx, const float* k_scale, int64_t n_rows,
-                          const int32_t* rows, double* scores, int64_t ld) {
+static int indexer_scores(int B, const int32_t* cu_q, const int32_t* cu_k, int H_I, int d_I, int q_kind,
+                          const void* q_idx, const float* q_scale, const double* w, int k_kind,
+                          const void* k_idx, const float* k_scale, int64_t n_rows, const int32_t* rows,
+                          double* scores, int64_t ld) {
   if (check_varlen(B, cu_q, cu_k)) return -1;
   int bad = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
@@ -147,7 +147,7 @@ int oracle_indexer_scores(int B, const int32_t* cu_q, const int32_t* cu_k, int H
       for (int j = 0; j < H_I; ++j) {
         double dot = 0.0;
         for (int d = 0; d < d_I; ++d) {
-          double qv = load_elem(q_kind, q_idx, (t * H_I + j) * (int64_t)d_I + d, NULL, 0);
+          double qv = load_elem(q_kind, q_idx, (t * H_I + j) * (int64_t)d_I + d, q_scale, t * H_I + j);
           double kv = load_elem(k_kind, k_idx, key_row * d_I + d, k_scale, key_row);
           dot += qv * kv;
         }
@@ -158,6 +158,16 @@ int oracle_indexer_scores(int B, const int32_t* cu_q, const int32_t* cu_k, int H
     }
   }
   return bad ? -1 : 0;
+}
+
+/* bf16 / float64 index queries (q_kind); keys as described above. */
+int oracle_indexer_scores(int B, const int32_t* cu_q, const int32_t* cu_k, int H_I, int d_I,
+                          int q_kind, const void* q_idx, const double* w, int k_kind,
+                          const void* k_idx, const float* k_scale, int64_t n_rows,
+                          const int32_t* rows, double* scores, int64_t ld) {
+  if (q_kind == ORACLE_E4M3) return -1;   /* e4m3 queries need their scales: oracle_indexer_scores_fp8 */
+  return indexer_scores(B, cu_q, cu_k, H_I, d_I, q_kind, q_idx, NULL, w, k_kind, k_idx, k_scale, n_rows, rows,
+                        scores, ld);
 }
 
 typedef struct {
@@ -350,4 +360,141 @@ int oracle_dense_mla_masked(int B, const int32_t* cu_q, const int32_t* cu_k, int
     free(z);
   }
   return bad ? -1 : 0;
+}
+
+/* ===========================================================================
+ * The FP8 indexer ("DeepSeek-V3.2", transformers model doc, section "DeepSeek
+ * Sparse Attention (DSA)", item 1: the reference indexer runs in FP8 with a
+ * Hadamard (rotate_activation) transform; "DeepSeek-V3.2-Exp" token-ids page,
+ * released config: scale_fmt "ue8m0").  Readings where the pages are silent:
+ *  - the rotation is the orthonormal Sylvester-Hadamard matrix of order d
+ *    (d a power of two): y = H x / sqrt(d) with H[i][j] = (-1)^popcount(i & j);
+ *  - quantization is per vector of d values (one index-head query, or one
+ *    index key): a power-of-two scale s = 2^ceil(log2(amax / 448)) (an ue8m0
+ *    exponent; s = 1 for a zero vector), values e4m3(x / s) rounded to
+ *    nearest, ties to even;
+ *  - the FP8 score is the indexer score of the dequantized values,
+ *    sum_j w[t,j] * max(0, (s_q[t,j] qq[t,j,:]) . (s_k[s] kq[s,:])).
+ * =========================================================================*/
+
+/* y[v,:] = H x[v,:] / sqrt(d) for n_vec vectors of length d (d a power of two). */
+int oracle_hadamard(int64_t n_vec, int d, const double* x, double* y) {
+  if (d < 1 || (d & (d - 1))) return -1;
+  const double norm = 1.0 / sqrt((double)d);
+#pragma omp parallel for schedule(static)
+  for (int64_t v = 0; v < n_vec; ++v) {
+    for (int i = 0; i < d; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < d; ++j) {
+        const int sign = __builtin_popcount((unsigned)(i & j)) & 1;
+        acc += sign ? -x[v * d + j] : x[v * d + j];
+      }
+      y[v * d + i] = acc * norm;
+    }
+  }
+  return 0;
+}
+
+/* The e4m3 byte nearest to v (ties to the even mantissa), saturating at
+ * +-448 (the largest finite magnitude); v must not be NaN.  Candidates are
+ * the 127 finite non-negative codes, compared by distance in double. */
+uint8_t oracle_double_to_e4m3(double v) {
+  const int neg = signbit(v) ? 1 : 0;
+  const double a = fabs(v);
+  int best = 0;
+  double best_err = INFINITY;
+  for (int code = 0; code < 127; ++code) {   /* 0x00 .. 0x7E: every finite non-negative value */
+    const double c = oracle_e4m3_to_double((uint8_t)code);
+    const double err = fabs(c - a);
+    /* on a tie the even mantissa (code & 1 == 0) wins */
+    if (err < best_err || (err == best_err && (code & 1) == 0)) {
+      best = code;
+      best_err = err;
+    }
+  }
+  return (uint8_t)(best | (neg << 7));
+}
+
+/* Per-vector e4m3 quantization with a power-of-two scale (see above). */
+int oracle_quant_e4m3_pow2(int64_t n_vec, int d, const double* x, uint8_t* q, float* scale) {
+  if (d < 1) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t v = 0; v < n_vec; ++v) {
+    double amax = 0.0;
+    for (int i = 0; i < d; ++i) amax = fmax(amax, fabs(x[v * d + i]));
+    const double s = amax > 0.0 ? ldexp(1.0, (int)ceil(log2(amax / 448.0))) : 1.0;
+    scale[v] = (float)s;
+    for (int i = 0; i < d; ++i) q[v * d + i] = oracle_double_to_e4m3(x[v * d + i] / s);
+  }
+  return 0;
+}
+
+/* Indexer scores with e4m3 index queries (one float32 scale per query head
+ * vector, q_scale[t * H_I + j]) and e4m3 index keys (one float32 scale per
+ * key).  Same definition and layout as oracle_indexer_scores. */
+int oracle_indexer_scores_fp8(int B, const int32_t* cu_q, const int32_t* cu_k, int H_I, int d_I,
+                              const uint8_t* q_idx, const float* q_scale, const double* w,
+                              const uint8_t* k_idx, const float* k_scale, int64_t n_rows,
+                              const int32_t* rows, double* scores, int64_t ld) {
+  return indexer_scores(B, cu_q, cu_k, H_I, d_I, ORACLE_E4M3, q_idx, q_scale, w, ORACLE_E4M3, k_idx, k_scale,
+                        n_rows, rows, scores, ld);
+}
+
+/* ===========================================================================
+ * Rotary position embedding of the RoPE part of queries and keys
+ * ("DeepSeek-V3.2-Exp" token-ids page, "Position IDs": a per-position table
+ * freqs_cis, sliced by position and handed to every layer; released config:
+ * qk_rope_head_dim 64).  Reading: every consecutive pair (x[2i], x[2i+1]) is
+ * a complex number multiplied by the table entry of its position and pair,
+ * freqs[pos][i] = (cos, sin); the table itself is an input.
+ * y[v, 2i]   = x[v, 2i] cos - x[v, 2i+1] sin
+ * y[v, 2i+1] = x[v, 2i] sin + x[v, 2i+1] cos,   (cos, sin) = freqs[pos[v]][i]
+ * x, y: [n_vec, d]; pos: [n_vec]; freqs: [max_pos, d/2, 2].
+ * =========================================================================*/
+int oracle_rope(int64_t n_vec, int d, const double* x, const int32_t* pos, const double* freqs,
+                int64_t max_pos, double* y) {
+  if (d < 2 || (d & 1)) return -1;
+  int bad = 0;
+#pragma omp parallel for schedule(static) reduction(| : bad)
+  for (int64_t v = 0; v < n_vec; ++v) {
+    if (pos[v] < 0 || pos[v] >= max_pos) {
+      bad = 1;
+      continue;
+    }
+    for (int i = 0; i < d / 2; ++i) {
+      const double c = freqs[((int64_t)pos[v] * (d / 2) + i) * 2 + 0];
+      const double s = freqs[((int64_t)pos[v] * (d / 2) + i) * 2 + 1];
+      const double re = x[v * d + 2 * i], im = x[v * d + 2 * i + 1];
+      y[v * d + 2 * i] = re * c - im * s;
+      y[v * d + 2 * i + 1] = re * s + im * c;
+    }
+  }
+  return bad ? -1 : 0;
+}
+
+/* ===========================================================================
+ * Up-projection of the absorbed attention output out of latent space
+ * ("DeepSeek-V3.2-Exp" token-ids page, released config: kv_lora_rank 512,
+ * v_head_dim 128, n_heads 128; "DeepSeek-V3.2" transformers doc: MLA with the
+ * cached entries shared by all heads, so each head's output is formed in the
+ * shared latent space).  Reading: per head h a matrix W_UV[h] of
+ * [d_c = kv_lora_rank, d_v = v_head_dim],
+ *   y[r, h, e] = sum_c o[r, h, c] * W_UV[h, c, e].
+ * o: [n_rows, H, d_c] (double); w: [H, d_c, d_v] (bf16 or double); y: [n_rows, H, d_v].
+ * =========================================================================*/
+int oracle_up_proj(int64_t n_rows, int H, int d_c, int d_v, const double* o, int w_kind, const void* w,
+                   double* y) {
+  if (H < 1 || d_c < 1 || d_v < 1) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    for (int h = 0; h < H; ++h) {
+      for (int e = 0; e < d_v; ++e) {
+        double acc = 0.0;
+        for (int c = 0; c < d_c; ++c)
+          acc += o[(r * H + h) * (int64_t)d_c + c] * load_elem(w_kind, w, ((int64_t)h * d_c + c) * d_v + e, NULL, 0);
+        y[(r * H + h) * (int64_t)d_v + e] = acc;
+      }
+    }
+  }
+  return 0;
 }

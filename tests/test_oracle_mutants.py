@@ -36,7 +36,25 @@ MUTANTS = [
      "return s >= 0 && s <= pos + 1 && s < kv_len;"),
     ("query head stride wrong", "dot += load_elem(q_kind, q, (t * H + h) * (int64_t)d_qk + d, NULL, 0) *\n                 load_elem(c_kind, latent, row * d_qk + d, NULL, 0);\n        z[i]",
      "dot += load_elem(q_kind, q, (t * H) * (int64_t)d_qk + d, NULL, 0) *\n                 load_elem(c_kind, latent, row * d_qk + d, NULL, 0);\n        z[i]"),
+    # FP8 indexer: rotation, encoding, scales
+    ("Hadamard signs dropped", "acc += sign ? -x[v * d + j] : x[v * d + j];", "acc += x[v * d + j];"),
+    ("Hadamard not normalised", "y[v * d + i] = acc * norm;", "y[v * d + i] = acc;"),
+    ("e4m3 ties to odd", "(err == best_err && (code & 1) == 0)", "(err == best_err && (code & 1) == 1)"),
+    ("e4m3 sign dropped", "return (uint8_t)(best | (neg << 7));", "return (uint8_t)best;"),
+    ("power-of-two scale rounded down", "ldexp(1.0, (int)ceil(log2(amax / 448.0)))",
+     "ldexp(1.0, (int)floor(log2(amax / 448.0)))"),
+    ("query scale of the wrong head", "(t * H_I + j) * (int64_t)d_I + d, q_scale, t * H_I + j);",
+     "(t * H_I + j) * (int64_t)d_I + d, q_scale, t * H_I);"),
+    # rotary embedding
+    ("rotation sign", "y[v * d + 2 * i] = re * c - im * s;", "y[v * d + 2 * i] = re * c + im * s;"),
+    ("pair halves swapped", "const double re = x[v * d + 2 * i], im = x[v * d + 2 * i + 1];",
+     "const double re = x[v * d + 2 * i + 1], im = x[v * d + 2 * i];"),
+    # up-projection
+    ("up-projection matrix transposed", "load_elem(w_kind, w, ((int64_t)h * d_c + c) * d_v + e, NULL, 0);",
+     "load_elem(w_kind, w, ((int64_t)h * d_v + e) * d_c + c, NULL, 0);"),
 ]
+
+from tests import test_oracle_pins_ext as pins_ext
 
 PIN_TESTS = [
     ("test_e4m3_decode_exhaustive", {}),
@@ -53,13 +71,25 @@ PIN_TESTS = [
     ("test_attention_ignores_order_padding_and_invalid_entries", {}),
 ]
 
+PIN_TESTS_EXT = [
+    ("test_hadamard_is_the_normalised_sylvester_matrix", {"d": 32}),
+    ("test_e4m3_encoding_round_trips_every_finite_code", {}),
+    ("test_e4m3_encoding_matches_torch_round_to_nearest_even", {}),
+    ("test_quantization_scale_is_the_smallest_power_of_two_that_fits", {}),
+    ("test_fp8_scores_match_einsum_of_the_dequantized_values", {}),
+    ("test_rope_is_complex_multiplication_by_the_table", {}),
+    ("test_rope_closed_forms", {}),
+    ("test_up_projection_matches_einsum_and_selects_with_a_unit_matrix", {}),
+]
+
 
 def _caught(lib_mod):
-    for name, kw in PIN_TESTS:
-        try:
-            getattr(pins, name)(lib_mod, **kw)
-        except Exception:
-            return name
+    for module, tests in ((pins, PIN_TESTS), (pins_ext, PIN_TESTS_EXT)):
+        for name, kw in tests:
+            try:
+                getattr(module, name)(lib_mod, **kw)
+            except Exception:
+                return name
     return None
 
 
