@@ -108,23 +108,34 @@ def aggregate_throughput(tokens_per_rank, ms_per_step, world):
 
 # --------------------------------------------------------------------------- algorithmic work
 
+PART = 8   # keys per part maximum
+
+
 def work_model(spec, idx_fp8):
-    """Algorithmic bytes / flops per step, per stage (compulsory traffic only)."""
+    """Algorithmic bytes / flops per step, per stage (compulsory traffic only).
+
+    The indexer writes every causal score and one part maximum per 8 keys.
+    The top-k must read a row's part maxima and at least the k parts that
+    hold the selection (8 scores each; the whole row when it is shorter), and
+    write k indices per query."""
     H_I, d_I, k, H, dqk, dv = spec.H_I, spec.d_I, spec.topk, spec.H, spec.d_qk, spec.d_v
     pairs = 0          # causal (query, key) pairs
     rows_sel = 0       # selected rows over all queries
-    score_cells = 0
+    parts = 0          # part maxima over all queries
+    topk_read = 0      # scores the top-k must read
     for ql, kl in zip(spec.q_lens, spec.kv_lens):
         for i in range(ql):
-            pos = kl - ql + i
-            pairs += pos + 1
-            rows_sel += min(k, pos + 1)
+            n = kl - ql + i + 1
+            pairs += n
+            rows_sel += min(k, n)
+            parts += (n + PART - 1) // PART
+            topk_read += min(n, PART * k)
     score_cells = pairs
     key_bytes = (d_I + 4) if idx_fp8 else 2 * d_I
     kv_total = sum(spec.kv_lens)
     T = spec.T
-    idx_bytes = kv_total * key_bytes + T * (H_I * d_I * 2 + H_I * 4) + score_cells * 4
-    topk_bytes = score_cells * 4 + T * k * 4
+    idx_bytes = kv_total * key_bytes + T * (H_I * d_I * 2 + H_I * 4) + score_cells * 4 + parts * 4
+    topk_bytes = parts * 4 + topk_read * 4 + T * k * 4
     att_bytes = rows_sel * dqk * 2 + T * (H * dqk * 2 + H * dv * 2 + H * 4) + T * k * 4
     return {
         "indexer": {"bytes": idx_bytes, "flops": pairs * 2 * H_I * d_I},
@@ -224,6 +235,7 @@ def gpu_arm(args, rank, world):
     rows = T if q_chunk == 0 else q_chunk
     ld = (max(spec.kv_lens) + 3) // 4 * 4
     scores = torch.empty((rows, ld), dtype=torch.float32, device=dev)
+    part_max = torch.empty((rows, dsa.part_max_ld(ld)), dtype=torch.float32, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     out = torch.empty((T, spec.H, spec.d_v), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((T, spec.H), dtype=torch.float32, device=dev)
@@ -232,8 +244,9 @@ def gpu_arm(args, rank, world):
 
     def step():
         for q0, q1 in chunks:
-            dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, q0, q1, scores, stream)
-            dsa.dsa_topk(scores, v, q0, q1, k, idx[q0:q1], stream)
+            dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, q0, q1, scores, stream,
+                                   part_max=part_max)
+            dsa.dsa_topk(scores, v, q0, q1, k, idx[q0:q1], stream, part_max=part_max)
             dsa.dsa_sparse_mla_attn(d["q"], d["latent"], idx[q0:q1], v, q0, q1, spec.softmax_scale, out, lse,
                                     stream=stream)
 
@@ -255,9 +268,10 @@ def gpu_arm(args, rank, world):
                 e = evs[i]
                 i += 1
                 e[0].record(stream)
-                dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, q0, q1, scores, stream)
+                dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, q0, q1, scores, stream,
+                                       part_max=part_max)
                 e[1].record(stream)
-                dsa.dsa_topk(scores, v, q0, q1, k, idx[q0:q1], stream)
+                dsa.dsa_topk(scores, v, q0, q1, k, idx[q0:q1], stream, part_max=part_max)
                 e[2].record(stream)
                 dsa.dsa_sparse_mla_attn(d["q"], d["latent"], idx[q0:q1], v, q0, q1, spec.softmax_scale, out, lse,
                                         stream=stream)
@@ -352,7 +366,7 @@ def indexer_prefill_measure(dsa, args, peaks):
     for _ in range(3):
         launch()
     torch.cuda.synchronize()
-    n = 5
+    n = 30
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(torch.cuda.current_device()) as clk:
         a.record(stream)

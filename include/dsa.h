@@ -79,7 +79,16 @@ typedef struct {
  * against every preceding key; the released config has index_n_heads 64 and
  * index_head_dim 128 ("DeepSeek-V3.2-Exp" token-ids page).  Score:
  *     I[t,s] = sum_j w[t,j] * max(0, q_idx[t,j,:] . k[s,:]),   0 <= s <= pos(t)
- * q_idx     bf16 [T, n_idx_heads, idx_dim], row-major, global rows
+ * q_idx     bf16 [T, n_idx_heads, idx_dim], row-major, global rows; or, for
+ *           the FP8 indexer (q_scale not NULL), e4m3 bytes of the same shape
+ *           from dsa_hadamard_quantize_fp8
+ * q_scale   NULL (bf16 queries), or fp32 [T, n_idx_heads]: the scale of each
+ *           query head vector from dsa_hadamard_quantize_fp8.  The keys must
+ *           then be e4m3 prepared the same way (k_dtype DSA_KIDX_FP8_E4M3);
+ *           the MMAs take both e4m3 operands as they are and the score is
+ *           sum_j w[t,j] q_scale[t,j] 2^-7 max(0, qq[t,j,:] . kq[s,:]) k_scale[s]
+ *           (2^-7 undoes the factor 128 of the unnormalised rotation).
+ *           Released shape only.
  * w         fp32 [T, n_idx_heads]
  * k_idx     bf16 or e4m3 bytes [sum kv, idx_dim] (see dsa_kidx_dtype);
  *           k_scale fp32 [sum kv] for e4m3, NULL for bf16
@@ -87,15 +96,22 @@ typedef struct {
  *           receives columns 0..pos(q_begin+r); columns past the diagonal in
  *           the same 128-key tile are set to -inf; later columns are not
  *           written.  ld_scores >= the longest kv_len among the rows.
+ * part_max  fp32 [q_end - q_begin, ld_part_max] or NULL: the first step of
+ *           the top-k, done in the same epilogue.  Element (r, p) is the
+ *           largest score of keys 8p .. 8p+7 of row r that are <= pos (keys
+ *           past pos count as -inf); written for every part whose first key
+ *           is inside the sequence.  ld_part_max >= ceil(longest kv_len / 8),
+ *           a multiple of 4.  dsa_topk given these maxima reads only the
+ *           parts of the row that can hold a selected key.
  * Accumulation is fp32 (bf16 x bf16 products are exact); for e4m3 keys the
  * per-key scale multiplies the head-reduced score (scale > 0 commutes with ReLU).
  * Alignment: all tensors 16-byte aligned; ld_scores a multiple of 4.
  */
-dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_idx,
+dsa_status dsa_indexer_scores(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                               const float* k_scale, dsa_kidx_dtype k_dtype, dsa_varlen v,
                               int32_t n_idx_heads, int32_t idx_dim, int64_t q_begin,
-                              int64_t q_end, float* scores, int64_t ld_scores,
-                              cudaStream_t stream);
+                              int64_t q_end, float* scores, int64_t ld_scores, float* part_max,
+                              int64_t ld_part_max, cudaStream_t stream);
 
 /*
  * Step 2: fine-grained token selection.
@@ -104,6 +120,13 @@ dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_i
  * default) tokens.  Ties are broken toward the lower key index; -0.0 ties +0.0.
  * scores    fp32 [q_end - q_begin, ld_scores] chunk-relative, as written by
  *           dsa_indexer_scores (only columns 0..pos(t) are read)
+ * part_max  NULL, or the part maxima dsa_indexer_scores wrote beside these
+ *           scores (same rows, layout as described there).  With them, a row
+ *           with at least topk parts and at most 262,144 keys is selected
+ *           from the maxima and the parts whose maximum reaches the topk-th
+ *           largest maximum; the result is the same set.  Maxima that do not
+ *           belong to the scores give a wrong selection (never an access
+ *           outside the row).
  * idx       int32 [q_end - q_begin, topk] chunk-relative.  Row r holds the
  *           min(topk, pos+1) selected sequence-local key indices followed by
  *           -1.  With pos+1 <= topk that is 0..pos.  The SET is the
@@ -112,8 +135,9 @@ dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_i
  * topk in [1, 2048].  Scores must not be NaN.  Rows longer than 1,040,384
  * keys return DSA_ERR_UNSUPPORTED (nothing launched).
  */
-dsa_status dsa_topk(const float* scores, int64_t ld_scores, dsa_varlen v, int64_t q_begin,
-                    int64_t q_end, int32_t topk, int32_t* idx, cudaStream_t stream);
+dsa_status dsa_topk(const float* scores, int64_t ld_scores, const float* part_max, int64_t ld_part_max,
+                    dsa_varlen v, int64_t q_begin, int64_t q_end, int32_t topk, int32_t* idx,
+                    cudaStream_t stream);
 
 /*
  * Step 3: MLA attention in absorbed MQA form over the selected rows.
@@ -142,10 +166,29 @@ dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t*
                                void* out, float* lse, cudaStream_t stream);
 
 /*
+ * Inputs of the FP8 indexer.
+ * Source: "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse
+ * Attention (DSA)", item 1 -- the reference indexer runs in FP8 with a
+ * Hadamard (rotate_activation) transform; "DeepSeek-V3.2-Exp" token-ids page,
+ * released config: scale_fmt ue8m0 (power-of-two scales).
+ * Each of the n vectors of 128 values is rotated by the Sylvester-Hadamard
+ * matrix H (entries +-1, H[i][j] = (-1)^popcount(i & j), not normalised) and
+ * quantized: scale[v] = 2^e with e the smallest integer such that
+ * max|Hx| <= 448 * 2^e (scale 1 for a zero vector), q[v, i] = the e4m3 byte
+ * nearest to (Hx)_i / scale[v] (ties to even).  Index queries ([T * 64]
+ * vectors) and index keys ([sum kv] vectors) prepared this way are the FP8
+ * indexer's operands (dsa_indexer_scores with q_scale); since
+ * (Hq).(Hk) = 128 (q.k), that score divides the factor 128 back out.
+ * x  bf16 [n, 128];  q  e4m3 bytes [n, 128];  scale  fp32 [n].
+ * x and q 16-byte aligned.
+ */
+dsa_status dsa_hadamard_quantize_fp8(const void* x, int64_t n, void* q, float* scale, cudaStream_t stream);
+
+/*
  * Bytes of device workspace dsa_forward needs for this layout when it runs at
  * most q_chunk query rows per pass (q_chunk <= 0: all rows in one pass).  The
- * workspace holds one pass's fp32 scores and int32 selections.  Returns 0 for
- * invalid arguments.
+ * workspace holds one pass's fp32 scores, their part maxima (one per 8 keys)
+ * and the int32 selections.  Returns 0 for invalid arguments.
  */
 size_t dsa_forward_workspace_size(dsa_varlen v, int32_t topk, int64_t q_chunk);
 
@@ -153,14 +196,15 @@ size_t dsa_forward_workspace_size(dsa_varlen v, int32_t topk, int64_t q_chunk);
  * The whole hot path for every query row: dsa_indexer_scores -> dsa_topk ->
  * dsa_sparse_mla_attn, in passes of at most q_chunk rows so that the score
  * buffer stays bounded; all launches go to `stream` in order.  Arguments as
- * for the three steps.  idx_out (nullable) receives the selections of every
- * row, [T, topk] int32, global rows.  workspace: device, at least
+ * for the three steps (q_scale not NULL: the FP8 indexer).  idx_out
+ * (nullable) receives the selections of every row, [T, topk] int32, global
+ * rows.  workspace: device, at least
  * dsa_forward_workspace_size(v, topk, q_chunk) bytes, 256-byte aligned.
  * Prefill, chunked prefill and decode are the same call: they differ only in
  * the lengths held by v.  Every pass's argument and launch-limit checks run
  * before the first launch, so an error status means nothing was launched.
  */
-dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
+dsa_status dsa_forward(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                        const float* k_scale, dsa_kidx_dtype k_dtype, const void* q,
                        const void* latent, dsa_varlen v, int32_t n_idx_heads,
                        int32_t idx_dim, int32_t topk, int32_t n_heads, int32_t d_qk,
@@ -200,7 +244,7 @@ dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
  * serialise them.
  */
 #define DSA_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
-dsa_status dsa_forward_static_scratch(const void* q_idx, const float* w, const void* k_idx,
+dsa_status dsa_forward_static_scratch(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                                       const float* k_scale, dsa_kidx_dtype k_dtype,
                                       const void* q, const void* latent, dsa_varlen v,
                                       int32_t n_idx_heads, int32_t idx_dim, int32_t topk,

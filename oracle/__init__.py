@@ -73,7 +73,7 @@ def _load():
                 ctypes.c_int, _I32P, _I32P, ctypes.c_int64, _I32P, _F64P, ctypes.c_int64,
                 ctypes.c_int, _I32P]
             lib.oracle_hadamard.restype = ctypes.c_int
-            lib.oracle_hadamard.argtypes = [ctypes.c_int64, ctypes.c_int, _F64P, _F64P]
+            lib.oracle_hadamard.argtypes = [ctypes.c_int64, ctypes.c_int, _F64P, _F64P, ctypes.c_int]
             lib.oracle_double_to_e4m3.restype = ctypes.c_uint8
             lib.oracle_double_to_e4m3.argtypes = [ctypes.c_double]
             lib.oracle_quant_e4m3_pow2.restype = ctypes.c_int
@@ -249,12 +249,13 @@ def _f64(x):
     return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
 
 
-def hadamard(x):
-    """Orthonormal Sylvester-Hadamard rotation of the last axis (a power of two)."""
+def hadamard(x, normalize=True):
+    """Sylvester-Hadamard rotation of the last axis (a power of two):
+    orthonormal (H / sqrt(d)) by default, the +-1 matrix H itself otherwise."""
     xa = _f64(x)
     d = xa.shape[-1]
     y = np.empty_like(xa)
-    if _load().oracle_hadamard(xa.size // d, d, _ptr(xa, _F64P), _ptr(y, _F64P)) != 0:
+    if _load().oracle_hadamard(xa.size // d, d, _ptr(xa, _F64P), _ptr(y, _F64P), 1 if normalize else 0) != 0:
         raise ValueError("oracle_hadamard: the length must be a power of two")
     return y
 

@@ -367,8 +367,10 @@ int oracle_dense_mla_masked(int B, const int32_t* cu_q, const int32_t* cu_k, int
  * Sparse Attention (DSA)", item 1: the reference indexer runs in FP8 with a
  * Hadamard (rotate_activation) transform; "DeepSeek-V3.2-Exp" token-ids page,
  * released config: scale_fmt "ue8m0").  Readings where the pages are silent:
- *  - the rotation is the orthonormal Sylvester-Hadamard matrix of order d
- *    (d a power of two): y = H x / sqrt(d) with H[i][j] = (-1)^popcount(i & j);
+ *  - the rotation is the Sylvester-Hadamard matrix of order d (d a power of
+ *    two), H[i][j] = (-1)^popcount(i & j), orthonormal as H / sqrt(d); the
+ *    FP8 path rotates both operands by H itself, so (Hq).(Hk) = d (q.k) and
+ *    the score divides the factor d out (exact: d is a power of two);
  *  - quantization is per vector of d values (one index-head query, or one
  *    index key): a power-of-two scale s = 2^ceil(log2(amax / 448)) (an ue8m0
  *    exponent; s = 1 for a zero vector), values e4m3(x / s) rounded to
@@ -377,10 +379,11 @@ int oracle_dense_mla_masked(int B, const int32_t* cu_q, const int32_t* cu_k, int
  *    sum_j w[t,j] * max(0, (s_q[t,j] qq[t,j,:]) . (s_k[s] kq[s,:])).
  * =========================================================================*/
 
-/* y[v,:] = H x[v,:] / sqrt(d) for n_vec vectors of length d (d a power of two). */
-int oracle_hadamard(int64_t n_vec, int d, const double* x, double* y) {
+/* y[v,:] = H x[v,:] / sqrt(d) (normalize != 0) or H x[v,:] (normalize == 0)
+ * for n_vec vectors of length d (d a power of two). */
+int oracle_hadamard(int64_t n_vec, int d, const double* x, double* y, int normalize) {
   if (d < 1 || (d & (d - 1))) return -1;
-  const double norm = 1.0 / sqrt((double)d);
+  const double norm = normalize ? 1.0 / sqrt((double)d) : 1.0;
 #pragma omp parallel for schedule(static)
   for (int64_t v = 0; v < n_vec; ++v) {
     for (int i = 0; i < d; ++i) {

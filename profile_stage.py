@@ -41,20 +41,21 @@ def main():
     T, k = v.T, spec.topk
     ld = (v.max_kv + 3) // 4 * 4
     scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    part_max = torch.empty((T, dsa.part_max_ld(ld)), dtype=torch.float32, device=dev)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     out = torch.empty((T, spec.H, spec.d_v), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((T, spec.H), dtype=torch.float32, device=dev)
     ws = torch.empty(dsa.dsa_forward_workspace_size(v, k), dtype=torch.uint8, device=dev)
     # inputs of the later stages
-    dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores)
-    dsa.dsa_topk(scores, v, 0, T, k, idx)
+    dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores, part_max=part_max)
+    dsa.dsa_topk(scores, v, 0, T, k, idx, part_max=part_max)
     torch.cuda.synchronize()
 
     def run():
         if args.stage == "indexer":
-            dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores)
+            dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores, part_max=part_max)
         elif args.stage == "topk":
-            dsa.dsa_topk(scores, v, 0, T, k, idx)
+            dsa.dsa_topk(scores, v, 0, T, k, idx, part_max=part_max)
         elif args.stage == "attention":
             dsa.dsa_sparse_mla_attn(d["q"], d["latent"], idx, v, 0, T, spec.softmax_scale, out, lse)
         else:

@@ -51,12 +51,13 @@ def _load():
             raise ImportError(f"{LIB_PATH} predates the binding (no symbol {name}): rebuild it with "
                               "`python sparse_attention_long_07_b200/build.py --force`")
     vp, i32, i64, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
-    lib.dsa_indexer_scores.argtypes = [vp, vp, vp, vp, ctypes.c_int, dsa_varlen, i32, i32, i64, i64, vp, i64, vp]
-    lib.dsa_topk.argtypes = [vp, i64, dsa_varlen, i64, i64, i32, vp, vp]
+    lib.dsa_indexer_scores.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, dsa_varlen, i32, i32, i64, i64, vp, i64,
+                                       vp, i64, vp]
+    lib.dsa_topk.argtypes = [vp, i64, vp, i64, dsa_varlen, i64, i64, i32, vp, vp]
     lib.dsa_sparse_mla_attn.argtypes = [vp, vp, vp, dsa_varlen, i64, i64, i32, i32, i32, i32, f32, vp, vp, vp]
     lib.dsa_forward_workspace_size.argtypes = [dsa_varlen, i32, i64]
     lib.dsa_forward_workspace_size.restype = ctypes.c_size_t
-    lib.dsa_forward.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp, dsa_varlen, i32, i32, i32, i32, i32, i32,
+    lib.dsa_forward.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, dsa_varlen, i32, i32, i32, i32, i32, i32,
                                 f32, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.dsa_device_error.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     lib.dsa_status_string.argtypes = [ctypes.c_int]
@@ -65,9 +66,11 @@ def _load():
     lib.dsa_debug_wait_profile.argtypes = [ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
                                            ctypes.c_int32, ctypes.c_int32]
     lib.dsa_debug_wait_profile.restype = ctypes.c_int
-    lib.dsa_forward_static_scratch.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, vp, dsa_varlen, i32, i32, i32,
+    lib.dsa_forward_static_scratch.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, dsa_varlen, i32, i32, i32,
                                                i32, i32, i32, f32, vp, vp, vp, vp]
     lib.dsa_forward_static_scratch.restype = ctypes.c_int
+    lib.dsa_hadamard_quantize_fp8.argtypes = [vp, i64, vp, vp, vp]
+    lib.dsa_hadamard_quantize_fp8.restype = ctypes.c_int
     lib.dsa_debug_wait_selftest.argtypes = [i64, vp]
     lib.dsa_debug_wait_selftest.restype = ctypes.c_int
     for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward", "dsa_device_error"):
@@ -77,7 +80,7 @@ def _load():
 
 EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward_workspace_size",
             "dsa_forward", "dsa_device_error", "dsa_status_string", "dsa_version", "dsa_debug_wait_profile",
-            "dsa_forward_static_scratch", "dsa_debug_wait_selftest")
+            "dsa_forward_static_scratch", "dsa_debug_wait_selftest", "dsa_hadamard_quantize_fp8")
 
 # bytes of the library's static scratch array (DSA_STATIC_SCRATCH_BYTES in include/dsa.h)
 DSA_STATIC_SCRATCH_BYTES = 32 << 20
@@ -144,19 +147,35 @@ def dsa_version() -> str:
     return _lib.dsa_version().decode()
 
 
-def dsa_indexer_scores(q_idx, w, k_idx, k_scale, v: Varlen, q_begin, q_end, scores, stream=None):
+PART = 8  # keys per part maximum
+
+
+def part_max_ld(ld_scores: int) -> int:
+    """Row stride of the part maxima for score rows of stride ld_scores."""
+    return max(4, ((ld_scores + PART - 1) // PART + 3) // 4 * 4)
+
+
+def dsa_indexer_scores(q_idx, w, k_idx, k_scale, v: Varlen, q_begin, q_end, scores, stream=None, part_max=None,
+                       q_scale=None):
     """Lightning-indexer scores for global query rows [q_begin, q_end) into
-    ``scores`` [q_end - q_begin, ld] fp32 (chunk-relative rows)."""
+    ``scores`` [q_end - q_begin, ld] fp32 (chunk-relative rows), and, when
+    ``part_max`` is given, the maximum of every 8 consecutive keys of each row.
+    With ``q_scale`` the FP8 indexer: q_idx and k_idx are e4m3 from
+    dsa_hadamard_quantize_fp8, q_scale / k_scale their scales."""
     T, H_I, d_I = q_idx.shape
-    _check(_lib.dsa_indexer_scores(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _kdtype(k_idx), v.c(),
-                                   H_I, d_I, q_begin, q_end, _ptr(scores), scores.stride(0), _stream(stream)),
+    _check(_lib.dsa_indexer_scores(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(k_idx), _ptr(k_scale), _kdtype(k_idx),
+                                   v.c(),
+                                   H_I, d_I, q_begin, q_end, _ptr(scores), scores.stride(0), _ptr(part_max),
+                                   0 if part_max is None else part_max.stride(0), _stream(stream)),
            "dsa_indexer_scores")
     return scores
 
 
-def dsa_topk(scores, v: Varlen, q_begin, q_end, topk, idx, stream=None):
-    """Top-k selection of chunk-relative score rows into ``idx`` [rows, topk] int32."""
-    _check(_lib.dsa_topk(_ptr(scores), scores.stride(0), v.c(), q_begin, q_end, topk, _ptr(idx),
+def dsa_topk(scores, v: Varlen, q_begin, q_end, topk, idx, stream=None, part_max=None):
+    """Top-k selection of chunk-relative score rows into ``idx`` [rows, topk]
+    int32 (with the indexer's part maxima when ``part_max`` is given)."""
+    _check(_lib.dsa_topk(_ptr(scores), scores.stride(0), _ptr(part_max),
+                         0 if part_max is None else part_max.stride(0), v.c(), q_begin, q_end, topk, _ptr(idx),
                          _stream(stream)), "dsa_topk")
     return idx
 
@@ -173,17 +192,30 @@ def dsa_sparse_mla_attn(q, latent, idx, v: Varlen, q_begin, q_end, scale, out, l
     return out, lse
 
 
+def dsa_hadamard_quantize_fp8(x, q=None, scale=None, stream=None):
+    """Hadamard rotation and e4m3 quantization of the 128-value vectors of x
+    (bf16 [..., 128]); returns (q e4m3 [..., 128], scale fp32 [...])."""
+    n = x.numel() // 128
+    if q is None:
+        q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    if scale is None:
+        scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check(_lib.dsa_hadamard_quantize_fp8(_ptr(x), n, _ptr(q), _ptr(scale), _stream(stream)),
+           "dsa_hadamard_quantize_fp8")
+    return q, scale
+
+
 def dsa_forward_workspace_size(v: Varlen, topk: int, q_chunk: int = 0) -> int:
     return int(_lib.dsa_forward_workspace_size(v.c(), topk, q_chunk))
 
 
 def dsa_forward(q_idx, w, k_idx, k_scale, q, latent, v: Varlen, topk, scale, out, lse, workspace,
-                idx_out=None, q_chunk: int = 0, stream=None):
+                idx_out=None, q_chunk: int = 0, stream=None, q_scale=None):
     """Indexer -> top-k -> sparse MLA for every query row (see include/dsa.h)."""
     T, H_I, d_I = q_idx.shape
     _, H, d_qk = q.shape
     d_v = out.shape[-1]
-    _check(_lib.dsa_forward(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _kdtype(k_idx), _ptr(q),
+    _check(_lib.dsa_forward(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(k_idx), _ptr(k_scale), _kdtype(k_idx), _ptr(q),
                             _ptr(latent), v.c(), H_I, d_I, topk, H, d_qk, d_v, float(scale), q_chunk,
                             _ptr(out), _ptr(lse), _ptr(idx_out), _ptr(workspace),
                             0 if workspace is None else workspace.numel() * workspace.element_size(),
@@ -192,14 +224,15 @@ def dsa_forward(q_idx, w, k_idx, k_scale, q, latent, v: Varlen, topk, scale, out
 
 
 def dsa_forward_static_scratch(q_idx, w, k_idx, k_scale, q, latent, v: Varlen, topk, scale, out, lse,
-                               idx_out=None, stream=None):
+                               idx_out=None, stream=None, q_scale=None):
     """dsa_forward for callers that cannot allocate device memory: the scratch
     is the library's own static device array (see include/dsa.h for who needs
     this, the size limit, and why overlapping calls must be serialised)."""
     T, H_I, d_I = q_idx.shape
     _, H, d_qk = q.shape
     d_v = out.shape[-1]
-    _check(_lib.dsa_forward_static_scratch(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_scale), _kdtype(k_idx),
+    _check(_lib.dsa_forward_static_scratch(_ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(k_idx), _ptr(k_scale),
+                                           _kdtype(k_idx),
                                            _ptr(q), _ptr(latent), v.c(), H_I, d_I, topk, H, d_qk, d_v,
                                            float(scale), _ptr(out), _ptr(lse), _ptr(idx_out), _stream(stream)),
            "dsa_forward_static_scratch")

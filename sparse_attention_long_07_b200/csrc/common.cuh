@@ -5,6 +5,11 @@
 
 namespace dsa {
 
+// Keys per part of the part maxima that the indexer's epilogue emits beside
+// the scores and the top-k reads: the maximum score of keys 8p .. 8p+7 of a
+// row (eight consecutive keys are eight consecutive lanes of one epilogue warp).
+constexpr int PART = 8;
+
 // Where global query row t sits: its sequence, absolute position and the
 // sequence's key range.  Sequence b owns query rows [cu_q[b], cu_q[b+1]) and
 // key rows [cu_k[b], cu_k[b+1]); its q_len new queries are its last tokens.

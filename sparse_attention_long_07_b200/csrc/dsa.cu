@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "dsa.h"
+#include "fp8.cuh"
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
@@ -161,13 +162,13 @@ bool is_tiny_mla(int h, int dqk, int dv) { return h == 4 && dqk == 80 && dv == 6
 // Launchers (arguments already validated)
 // ----------------------------------------------------------------------------
 template <class C>
-dsa_status launch_indexer(const void* q_idx, const float* w, const void* k_idx,
+dsa_status launch_indexer(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                           const float* k_scale, const dsa_varlen& v, const Layout& L,
                           int64_t q_begin, int64_t q_end, float* scores, int64_t ld,
-                          cudaStream_t stream) {
+                          float* part_max, int64_t ld_pm, cudaStream_t stream) {
   CUtensorMap tm_q, tm_k;
-  if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q_idx, C::D_I,
-                static_cast<uint64_t>(L.T) * C::H_I, C::D_I * 2, C::ATOM_ELEMS, C::N,
+  if (!make_map(&tm_q, C::QFP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q_idx, C::D_I,
+                static_cast<uint64_t>(L.T) * C::H_I, C::D_I * C::ELEM, C::ATOM_ELEMS, C::N,
                 C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return DSA_ERR_CUDA;
   if (C::KFP8) {
@@ -184,6 +185,7 @@ dsa_status launch_indexer(const void* q_idx, const float* w, const void* k_idx,
 
   dsa::IndexerParams p;
   p.w = w;
+  p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.cu_q = v.cu_q;
   p.cu_k = v.cu_k;
@@ -192,6 +194,8 @@ dsa_status launch_indexer(const void* q_idx, const float* w, const void* k_idx,
   p.q_end = q_end;
   p.scores = scores;
   p.ld = ld;
+  p.part_max = part_max;
+  p.ld_pm = ld_pm;
   p.chunk_tiles = C::NQ == 1 ? 32 : 64;
   const int qblocks = (L.max_q_rows + C::NQ - 1) / C::NQ;
   const int chunks = (L.max_tiles + p.chunk_tiles - 1) / p.chunk_tiles;
@@ -207,7 +211,7 @@ template <class C>
 dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const void* k_idx,
                                      const float* k_scale, const dsa_varlen& v, const Layout& L,
                                      int64_t q_begin, int64_t q_end, float* scores, int64_t ld,
-                                     cudaStream_t stream) {
+                                     float* part_max, int64_t ld_pm, cudaStream_t stream) {
   int64_t units = 0;
   for (int b = 0; b < v.batch; ++b) {
     const int64_t lo = std::max<int64_t>(v.cu_q_host[b], q_begin);
@@ -230,6 +234,7 @@ dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const vo
   if (ensure_smem<dsa::indexer_persistent_kernel<C>>(C::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
   dsa::IndexerParams p;
   p.w = w;
+  p.q_scale = nullptr;
   p.k_scale = k_scale;
   p.cu_q = v.cu_q;
   p.cu_k = v.cu_k;
@@ -238,6 +243,8 @@ dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const vo
   p.q_end = q_end;
   p.scores = scores;
   p.ld = ld;
+  p.part_max = part_max;
+  p.ld_pm = ld_pm;
   p.chunk_tiles = 0;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, sms));
   dsa::indexer_persistent_kernel<C><<<grid, C::NT, C::SMEM_BYTES, stream>>>(tm_q, tm_k, p);
@@ -285,9 +292,15 @@ dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, con
   return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
-dsa_status check_indexer_args(const void* q_idx, const float* w, const void* k_idx,
+dsa_status check_indexer_args(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                               const float* k_scale, dsa_kidx_dtype kd, int h, int d,
                               const float* scores, int64_t ld, const Layout& L) {
+  // FP8 indexer (q_scale given): e4m3 queries and keys, released shape only
+  if (q_scale) {
+    if (reinterpret_cast<uintptr_t>(q_scale) & 3u) return DSA_ERR_INVALID_ARG;
+    if (kd != DSA_KIDX_FP8_E4M3) return DSA_ERR_INVALID_ARG;
+    if (!is_released_indexer(h, d)) return DSA_ERR_UNSUPPORTED;
+  }
   // scores == nullptr: the score buffer is validated by the caller (dsa_forward's workspace)
   if (!q_idx || !w || !k_idx) return DSA_ERR_INVALID_ARG;
   if (!aligned16(q_idx) || !aligned16(w) || !aligned16(k_idx) || (scores && !aligned16(scores)))
@@ -316,11 +329,12 @@ dsa_status check_mla_args(const void* q, const void* latent, const int32_t* idx,
 // Which indexer kernel a pass uses.  Decode-like passes (at most one query row
 // per sequence) over an e4m3 cache take the persistent kernel; otherwise the
 // query-block grid kernel with 1 or 4 queries per CTA.
-enum class IndexerKind { kTiny, kPersistent, kGridFp8x1, kGridFp8x4, kGridBf16x1, kGridBf16x4 };
+enum class IndexerKind { kTiny, kPersistent, kGridFp8x1, kGridFp8x4, kGridBf16x1, kGridBf16x4, kFp8Fp8x1, kFp8Fp8x4 };
 
-IndexerKind choose_indexer(dsa_kidx_dtype kd, int h, int d, const dsa_varlen& v, const Layout& L) {
+IndexerKind choose_indexer(bool q_fp8, dsa_kidx_dtype kd, int h, int d, const dsa_varlen& v, const Layout& L) {
   if (is_tiny_indexer(h, d)) return IndexerKind::kTiny;
   const bool decode_like = L.max_q_rows <= 2;
+  if (q_fp8) return decode_like ? IndexerKind::kFp8Fp8x1 : IndexerKind::kFp8Fp8x4;
   if (kd == DSA_KIDX_FP8_E4M3) {
     if (L.max_q_rows <= 1 && v.batch <= IndexerCfg<64, 128, 1, true, true>::MAX_SEQ) return IndexerKind::kPersistent;
     return decode_like ? IndexerKind::kGridFp8x1 : IndexerKind::kGridFp8x4;
@@ -329,40 +343,48 @@ IndexerKind choose_indexer(dsa_kidx_dtype kd, int h, int d, const dsa_varlen& v,
 }
 
 // Launch limits of one indexer pass, checked before anything is launched.
-dsa_status indexer_limits(dsa_kidx_dtype kd, int h, int d, const dsa_varlen& v, const Layout& L) {
+dsa_status indexer_limits(bool q_fp8, dsa_kidx_dtype kd, int h, int d, const dsa_varlen& v, const Layout& L) {
   if (L.max_q_rows == 0) return DSA_OK;
-  const IndexerKind k = choose_indexer(kd, h, d, v, L);
+  const IndexerKind k = choose_indexer(q_fp8, kd, h, d, v, L);
   if (k == IndexerKind::kPersistent) return DSA_OK;
-  const int nq = (k == IndexerKind::kGridFp8x1 || k == IndexerKind::kGridBf16x1) ? 1 : 4;
+  const int nq = (k == IndexerKind::kGridFp8x1 || k == IndexerKind::kGridBf16x1 || k == IndexerKind::kFp8Fp8x1) ? 1 : 4;
   const int64_t qblocks = (L.max_q_rows + nq - 1) / nq;
   if (qblocks > 65535 || v.batch > 65535) return DSA_ERR_UNSUPPORTED;   // gridDim.y / gridDim.z
   return DSA_OK;
 }
 
-dsa_status run_indexer(const void* q_idx, const float* w, const void* k_idx, const float* k_scale,
-                       dsa_kidx_dtype kd, const dsa_varlen& v, const Layout& L, int h, int d,
-                       int64_t q_begin, int64_t q_end, float* scores, int64_t ld,
-                       cudaStream_t stream) {
+dsa_status run_indexer(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
+                       const float* k_scale, dsa_kidx_dtype kd, const dsa_varlen& v, const Layout& L, int h, int d,
+                       int64_t q_begin, int64_t q_end, float* scores, int64_t ld, float* part_max,
+                       int64_t ld_pm, cudaStream_t stream) {
   if (q_end == q_begin) return DSA_OK;
-  switch (choose_indexer(kd, h, d, v, L)) {
+  switch (choose_indexer(q_scale != nullptr, kd, h, d, v, L)) {
+    case IndexerKind::kFp8Fp8x1:
+      return launch_indexer<IndexerCfg<64, 128, 1, true, false, true>>(q_idx, q_scale, w, k_idx, k_scale, v, L,
+                                                                        q_begin, q_end, scores, ld, part_max, ld_pm,
+                                                                        stream);
+    case IndexerKind::kFp8Fp8x4:
+      return launch_indexer<IndexerCfg<64, 128, 4, true, false, true>>(q_idx, q_scale, w, k_idx, k_scale, v, L,
+                                                                        q_begin, q_end, scores, ld, part_max, ld_pm,
+                                                                        stream);
     case IndexerKind::kTiny:
-      return launch_indexer<IndexerCfg<4, 32, 4, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
-                                                          scores, ld, stream);
+      return launch_indexer<IndexerCfg<4, 32, 4, false>>(q_idx, nullptr, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                          scores, ld, part_max, ld_pm, stream);
     case IndexerKind::kPersistent:
       return launch_indexer_persistent<IndexerCfg<64, 128, 1, true, true>>(q_idx, w, k_idx, k_scale, v, L,
-                                                                           q_begin, q_end, scores, ld, stream);
+                                                                           q_begin, q_end, scores, ld, part_max, ld_pm, stream);
     case IndexerKind::kGridFp8x1:
-      return launch_indexer<IndexerCfg<64, 128, 1, true>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
-                                                           scores, ld, stream);
+      return launch_indexer<IndexerCfg<64, 128, 1, true>>(q_idx, nullptr, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                           scores, ld, part_max, ld_pm, stream);
     case IndexerKind::kGridFp8x4:
-      return launch_indexer<IndexerCfg<64, 128, 4, true>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
-                                                           scores, ld, stream);
+      return launch_indexer<IndexerCfg<64, 128, 4, true>>(q_idx, nullptr, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                           scores, ld, part_max, ld_pm, stream);
     case IndexerKind::kGridBf16x1:
-      return launch_indexer<IndexerCfg<64, 128, 1, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
-                                                            scores, ld, stream);
+      return launch_indexer<IndexerCfg<64, 128, 1, false>>(q_idx, nullptr, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                            scores, ld, part_max, ld_pm, stream);
     case IndexerKind::kGridBf16x4:
-      return launch_indexer<IndexerCfg<64, 128, 4, false>>(q_idx, w, k_idx, k_scale, v, L, q_begin, q_end,
-                                                            scores, ld, stream);
+      return launch_indexer<IndexerCfg<64, 128, 4, false>>(q_idx, nullptr, w, k_idx, k_scale, v, L, q_begin, q_end,
+                                                            scores, ld, part_max, ld_pm, stream);
   }
   return DSA_ERR_UNSUPPORTED;
 }
@@ -377,14 +399,14 @@ dsa_status topk_limits(const Layout& L, int64_t rows) {
 // Launch limits of one attention pass: one cluster of SPLIT CTAs per row.
 dsa_status mla_limits(int64_t rows) { return rows * 2 > 0x7FFFFFFF ? DSA_ERR_UNSUPPORTED : DSA_OK; }
 
-dsa_status run_topk(const float* scores, int64_t ld, const dsa_varlen& v, const Layout& L,
-                    int64_t q_begin, int64_t q_end, int topk, int32_t* idx, cudaStream_t stream) {
+dsa_status run_topk(const float* scores, int64_t ld, const float* part_max, int64_t ld_pm, const dsa_varlen& v,
+                    const Layout& L, int64_t q_begin, int64_t q_end, int topk, int32_t* idx, cudaStream_t stream) {
   const int64_t rows = q_end - q_begin;
   if (rows == 0) return DSA_OK;
   if (topk_limits(L, rows) != DSA_OK) return DSA_ERR_UNSUPPORTED;
   if (ensure_smem<dsa::topk_kernel>(dsa::TopkCfg::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
   dsa::topk_kernel<<<static_cast<unsigned>(rows), dsa::TopkCfg::NT, dsa::TopkCfg::SMEM_BYTES, stream>>>(
-      scores, ld, v.cu_q, v.cu_k, v.batch, q_begin, topk, idx);
+      scores, ld, part_max, ld_pm, v.cu_q, v.cu_k, v.batch, q_begin, topk, idx);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -403,38 +425,52 @@ size_t align_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
 
 int64_t scores_ld(const Layout& L) { return std::max<int64_t>(4, (L.max_kv + 3) / 4 * 4); }
 
+// Row stride of the part maxima: one per PART keys, rounded up to 4 (16-byte rows).
+int64_t part_max_ld(int64_t ld_scores) { return std::max<int64_t>(4, ((ld_scores + dsa::PART - 1) / dsa::PART + 3) / 4 * 4); }
+
+// part_max (nullable) must cover every part of the longest row, 16-byte rows.
+dsa_status check_part_max(const float* part_max, int64_t ld_pm, const Layout& L) {
+  if (!part_max) return DSA_OK;
+  if (!aligned16(part_max) || ld_pm % 4 != 0 || ld_pm < (L.max_kv + dsa::PART - 1) / dsa::PART)
+    return DSA_ERR_INVALID_ARG;
+  return DSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
 
-dsa_status dsa_indexer_scores(const void* q_idx, const float* w, const void* k_idx,
+dsa_status dsa_indexer_scores(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                               const float* k_scale, dsa_kidx_dtype k_dtype, dsa_varlen v,
                               int32_t n_idx_heads, int32_t idx_dim, int64_t q_begin,
-                              int64_t q_end, float* scores, int64_t ld_scores,
-                              cudaStream_t stream) {
+                              int64_t q_end, float* scores, int64_t ld_scores, float* part_max,
+                              int64_t ld_part_max, cudaStream_t stream) {
   Layout L;
   dsa_status st = check_varlen(v, q_begin, q_end, &L);
   if (st != DSA_OK) return st;
   if (!scores) return DSA_ERR_INVALID_ARG;
-  st = check_indexer_args(q_idx, w, k_idx, k_scale, k_dtype, n_idx_heads, idx_dim, scores, ld_scores, L);
+  st = check_indexer_args(q_idx, q_scale, w, k_idx, k_scale, k_dtype, n_idx_heads, idx_dim, scores, ld_scores, L);
   if (st != DSA_OK) return st;
-  if ((st = indexer_limits(k_dtype, n_idx_heads, idx_dim, v, L)) != DSA_OK) return st;
+  if ((st = check_part_max(part_max, ld_part_max, L)) != DSA_OK) return st;
+  if ((st = indexer_limits(q_scale != nullptr, k_dtype, n_idx_heads, idx_dim, v, L)) != DSA_OK) return st;
   if ((st = injected_fault()) != DSA_OK) return st;
-  return run_indexer(q_idx, w, k_idx, k_scale, k_dtype, v, L, n_idx_heads, idx_dim, q_begin, q_end,
-                     scores, ld_scores, stream);
+  return run_indexer(q_idx, q_scale, w, k_idx, k_scale, k_dtype, v, L, n_idx_heads, idx_dim, q_begin, q_end,
+                     scores, ld_scores, part_max, ld_part_max, stream);
 }
 
-dsa_status dsa_topk(const float* scores, int64_t ld_scores, dsa_varlen v, int64_t q_begin,
-                    int64_t q_end, int32_t topk, int32_t* idx, cudaStream_t stream) {
+dsa_status dsa_topk(const float* scores, int64_t ld_scores, const float* part_max, int64_t ld_part_max,
+                    dsa_varlen v, int64_t q_begin, int64_t q_end, int32_t topk, int32_t* idx,
+                    cudaStream_t stream) {
   Layout L;
   dsa_status st = check_varlen(v, q_begin, q_end, &L);
   if (st != DSA_OK) return st;
   if (!scores || !idx || !aligned16(scores) || (reinterpret_cast<uintptr_t>(idx) & 3u))
     return DSA_ERR_INVALID_ARG;
   if (topk < 1 || topk > 2048 || ld_scores < L.max_kv || ld_scores % 4 != 0) return DSA_ERR_INVALID_ARG;
+  if ((st = check_part_max(part_max, ld_part_max, L)) != DSA_OK) return st;
   if ((st = topk_limits(L, q_end - q_begin)) != DSA_OK) return st;
   if ((st = injected_fault()) != DSA_OK) return st;
-  return run_topk(scores, ld_scores, v, L, q_begin, q_end, topk, idx, stream);
+  return run_topk(scores, ld_scores, part_max, ld_part_max, v, L, q_begin, q_end, topk, idx, stream);
 }
 
 dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t* idx,
@@ -457,10 +493,11 @@ size_t dsa_forward_workspace_size(dsa_varlen v, int32_t topk, int64_t q_chunk) {
   Layout full;
   if (v.batch < 1 || !v.cu_q_host || topk < 1 || topk > 2048) return 0;
   if (check_varlen(v, 0, v.cu_q_host[v.batch], &full) != DSA_OK) return 0;
-  const int64_t rows = q_chunk > 0 ? std::min<int64_t>(q_chunk, full.T) : full.T;
+  const int64_t rows = std::max<int64_t>(1, q_chunk > 0 ? std::min<int64_t>(q_chunk, full.T) : full.T);
   const int64_t ld = scores_ld(full);
-  return align_up(static_cast<size_t>(std::max<int64_t>(rows, 1)) * ld * sizeof(float)) +
-         align_up(static_cast<size_t>(std::max<int64_t>(rows, 1)) * topk * sizeof(int32_t));
+  return align_up(static_cast<size_t>(rows) * ld * sizeof(float)) +
+         align_up(static_cast<size_t>(rows) * part_max_ld(ld) * sizeof(float)) +
+         align_up(static_cast<size_t>(rows) * topk * sizeof(int32_t));
 }
 
 }  // extern "C"
@@ -470,7 +507,8 @@ namespace {
 // Every check of a dsa_forward call that does not involve the workspace:
 // arguments, supported shapes and each pass's launch limits.  Host arithmetic
 // only (no CUDA call).
-dsa_status forward_checks(const void* q_idx, const float* w, const void* k_idx, const float* k_scale,
+dsa_status forward_checks(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
+                          const float* k_scale,
                           dsa_kidx_dtype k_dtype, const void* q, const void* latent, const dsa_varlen& v,
                           int32_t n_idx_heads, int32_t idx_dim, int32_t topk, int32_t n_heads, int32_t d_qk,
                           int32_t d_v, float scale, int64_t q_chunk, const void* out, const float* lse,
@@ -481,7 +519,7 @@ dsa_status forward_checks(const void* q_idx, const float* w, const void* k_idx, 
   if (st != DSA_OK) return st;
   const int64_t ld = scores_ld(full);
   // the score buffer is the (256-byte aligned) workspace: checked by the caller
-  st = check_indexer_args(q_idx, w, k_idx, k_scale, k_dtype, n_idx_heads, idx_dim, nullptr, ld, full);
+  st = check_indexer_args(q_idx, q_scale, w, k_idx, k_scale, k_dtype, n_idx_heads, idx_dim, nullptr, ld, full);
   if (st != DSA_OK) return st;
   if (idx_out && (reinterpret_cast<uintptr_t>(idx_out) & 15u)) return DSA_ERR_INVALID_ARG;
   st = check_mla_args(q, latent, nullptr, topk, n_heads, d_qk, d_v, scale, out, lse);
@@ -492,7 +530,7 @@ dsa_status forward_checks(const void* q_idx, const float* w, const void* k_idx, 
     const int64_t q1 = std::min(T, q0 + rows);
     Layout L;
     if ((st = check_varlen(v, q0, q1, &L)) != DSA_OK) return st;
-    if ((st = indexer_limits(k_dtype, n_idx_heads, idx_dim, v, L)) != DSA_OK) return st;
+    if ((st = indexer_limits(q_scale != nullptr, k_dtype, n_idx_heads, idx_dim, v, L)) != DSA_OK) return st;
     if ((st = topk_limits(L, q1 - q0)) != DSA_OK) return st;
     if ((st = mla_limits(q1 - q0)) != DSA_OK) return st;
   }
@@ -503,15 +541,15 @@ dsa_status forward_checks(const void* q_idx, const float* w, const void* k_idx, 
 
 extern "C" {
 
-dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
+dsa_status dsa_forward(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                        const float* k_scale, dsa_kidx_dtype k_dtype, const void* q,
                        const void* latent, dsa_varlen v, int32_t n_idx_heads,
                        int32_t idx_dim, int32_t topk, int32_t n_heads, int32_t d_qk,
                        int32_t d_v, float scale, int64_t q_chunk, void* out, float* lse,
                        int32_t* idx_out, void* workspace, size_t workspace_bytes,
                        cudaStream_t stream) {
-  dsa_status st = forward_checks(q_idx, w, k_idx, k_scale, k_dtype, q, latent, v, n_idx_heads, idx_dim, topk,
-                                 n_heads, d_qk, d_v, scale, q_chunk, out, lse, idx_out);
+  dsa_status st = forward_checks(q_idx, q_scale, w, k_idx, k_scale, k_dtype, q, latent, v, n_idx_heads, idx_dim,
+                                 topk, n_heads, d_qk, d_v, scale, q_chunk, out, lse, idx_out);
   if (st != DSA_OK) return st;
   if (!workspace) return DSA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign) return DSA_ERR_INVALID_ARG;
@@ -525,18 +563,22 @@ dsa_status dsa_forward(const void* q_idx, const float* w, const void* k_idx,
   const int64_t ld = scores_ld(full);
   const int64_t T = full.T;
   const int64_t rows = q_chunk > 0 ? std::min<int64_t>(q_chunk, T) : T;
+  // workspace: one pass's scores | part maxima | selections
+  const int64_t ld_pm = part_max_ld(ld);
+  const size_t rows_ws = static_cast<size_t>(std::max<int64_t>(rows, 1));
   float* scores = static_cast<float*>(workspace);
-  int32_t* idx_ws = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(workspace) +
-                                               align_up(static_cast<size_t>(std::max<int64_t>(rows, 1)) * ld * sizeof(float)));
+  float* part_max = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align_up(rows_ws * ld * sizeof(float)));
+  int32_t* idx_ws = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(part_max) +
+                                               align_up(rows_ws * ld_pm * sizeof(float)));
   for (int64_t q0 = 0; q0 < T; q0 += rows) {
     const int64_t q1 = std::min(T, q0 + rows);
     Layout L;
     if ((st = check_varlen(v, q0, q1, &L)) != DSA_OK) return st;
     int32_t* idx = idx_out ? idx_out + q0 * topk : idx_ws;
-    if ((st = run_indexer(q_idx, w, k_idx, k_scale, k_dtype, v, L, n_idx_heads, idx_dim, q0, q1, scores,
-                          ld, stream)) != DSA_OK)
+    if ((st = run_indexer(q_idx, q_scale, w, k_idx, k_scale, k_dtype, v, L, n_idx_heads, idx_dim, q0, q1, scores,
+                          ld, part_max, ld_pm, stream)) != DSA_OK)
       return st;
-    if ((st = run_topk(scores, ld, v, L, q0, q1, topk, idx, stream)) != DSA_OK) return st;
+    if ((st = run_topk(scores, ld, part_max, ld_pm, v, L, q0, q1, topk, idx, stream)) != DSA_OK) return st;
     if ((st = run_mla(q, latent, idx, v, L, q0, q1, topk, n_heads, d_qk, d_v, scale, out, lse,
                       stream)) != DSA_OK)
       return st;
@@ -556,7 +598,7 @@ void* g_scratch_ptr[kMaxDevices];
 cudaError_t g_scratch_err[kMaxDevices];
 }  // namespace
 
-dsa_status dsa_forward_static_scratch(const void* q_idx, const float* w, const void* k_idx,
+dsa_status dsa_forward_static_scratch(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                                       const float* k_scale, dsa_kidx_dtype k_dtype,
                                       const void* q, const void* latent, dsa_varlen v,
                                       int32_t n_idx_heads, int32_t idx_dim, int32_t topk,
@@ -575,8 +617,8 @@ dsa_status dsa_forward_static_scratch(const void* q_idx, const float* w, const v
     if (dsa_forward_workspace_size(v, topk, mid) <= DSA_STATIC_SCRATCH_BYTES) lo = mid; else hi = mid - 1;
   }
   const int64_t q_chunk = lo;
-  dsa_status st = forward_checks(q_idx, w, k_idx, k_scale, k_dtype, q, latent, v, n_idx_heads, idx_dim, topk,
-                                 n_heads, d_qk, d_v, scale, q_chunk, out, lse, idx_out);
+  dsa_status st = forward_checks(q_idx, q_scale, w, k_idx, k_scale, k_dtype, q, latent, v, n_idx_heads, idx_dim,
+                                 topk, n_heads, d_qk, d_v, scale, q_chunk, out, lse, idx_out);
   if (st != DSA_OK) return st;
   // the array's device address, looked up once per device with that device current
   int dev = 0;
@@ -585,7 +627,7 @@ dsa_status dsa_forward_static_scratch(const void* q_idx, const float* w, const v
     g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_ptr[dev], g_dsa_static_scratch);
   });
   if (g_scratch_err[dev] != cudaSuccess || g_scratch_ptr[dev] == nullptr) return DSA_ERR_CUDA;
-  return dsa_forward(q_idx, w, k_idx, k_scale, k_dtype, q, latent, v, n_idx_heads, idx_dim, topk, n_heads,
+  return dsa_forward(q_idx, q_scale, w, k_idx, k_scale, k_dtype, q, latent, v, n_idx_heads, idx_dim, topk, n_heads,
                      d_qk, d_v, scale, q_chunk, out, lse, idx_out, g_scratch_ptr[dev], DSA_STATIC_SCRATCH_BYTES,
                      stream);
 }
@@ -598,6 +640,19 @@ dsa_status dsa_device_error(int32_t* code, cudaStream_t stream) {
   if (cudaMemcpyToSymbol(dsa::g_device_error, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
   *code = v;
   return v == 0 ? DSA_OK : DSA_ERR_DEVICE_TIMEOUT;
+}
+
+dsa_status dsa_hadamard_quantize_fp8(const void* x, int64_t n, void* q, float* scale, cudaStream_t stream) {
+  if (n < 0) return DSA_ERR_INVALID_ARG;
+  if (n == 0) return DSA_OK;
+  if (!x || !q || !scale || !aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(scale) & 3u))
+    return DSA_ERR_INVALID_ARG;
+  if ((n + 7) / 8 > 0x7FFFFFFF) return DSA_ERR_UNSUPPORTED;
+  dsa_status st;
+  if ((st = injected_fault()) != DSA_OK) return st;
+  dsa::hadamard_quantize_kernel<<<static_cast<unsigned>((n + 7) / 8), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), n, static_cast<uint8_t*>(q), scale);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // extern "C"

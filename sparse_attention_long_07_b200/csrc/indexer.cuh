@@ -24,6 +24,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "fp8.cuh"
 #include "sm100.cuh"
 
 namespace dsa {
@@ -34,26 +35,32 @@ __host__ __device__ constexpr int pow2_at_least(int v, int lo) {
   return p;
 }
 
-template <int H_I_, int D_I_, int NQ_, bool KFP8_, bool PERSIST_ = false>
+template <int H_I_, int D_I_, int NQ_, bool KFP8_, bool PERSIST_ = false, bool QFP8_ = false>
 struct IndexerCfg {
   static constexpr int H_I = H_I_, D_I = D_I_, NQ = NQ_;
   static constexpr bool KFP8 = KFP8_;
+  // FP8 indexer: e4m3 queries and keys (Hadamard-rotated, power-of-two scales)
+  // multiplied as they are by kind::f8f6f4 MMAs; otherwise bf16 MMAs, with
+  // e4m3 keys widened to bf16 first (CONVERT)
+  static constexpr bool QFP8 = QFP8_;
+  static constexpr bool CONVERT = KFP8 && !QFP8;
   static constexpr bool PERSIST = PERSIST_;                 // one CTA per SM over a flat unit list
   static constexpr int MAX_SEQ = 2048;                    // persistent: sequences per call
   static constexpr int BK = 128;                          // keys per tile (MMA M)
   static constexpr int N = NQ * H_I;                      // MMA N
-  static constexpr int ROWB = D_I * 2;                    // bytes of one bf16 row
+  static constexpr int ELEM = QFP8 ? 1 : 2;               // bytes per MMA operand element
+  static constexpr int ROWB = D_I * ELEM;                 // bytes of one operand row
   static constexpr int SWB = ROWB >= 128 ? 128 : ROWB;    // swizzle span (128 or 64 bytes)
   static constexpr uint32_t SWZ = SWB == 128 ? 2u : 4u;   // descriptor swizzle code
   static constexpr int NATOM = ROWB / SWB;                // swizzle-atom columns per row
-  static constexpr int ATOM_ELEMS = SWB / 2;
-  static constexpr int KSTEPS = D_I / 16;
+  static constexpr int ATOM_ELEMS = SWB / ELEM;
+  static constexpr int KSTEPS = ROWB / 32;                // 32 bytes of K per MMA (16 bf16 or 32 e4m3)
   // Persistent schedule: the widened bf16 key tile is written to tensor memory
   // and read from there as the A operand (TS-form MMA), so shared memory holds
   // only the raw e4m3 ring; otherwise the bf16 tile ring is in shared memory.
   static constexpr bool K_IN_TMEM = PERSIST;
-  static constexpr int STAGES = K_IN_TMEM ? 4 : (KFP8 ? 2 : 4);  // bf16 key-tile ring
-  static constexpr int RSTAGES = KFP8 ? (PERSIST ? 11 : 4) : 0;  // raw e4m3 ring
+  static constexpr int STAGES = K_IN_TMEM ? 4 : (CONVERT ? 2 : 4);  // key-tile ring (MMA operand)
+  static constexpr int RSTAGES = CONVERT ? (PERSIST ? 11 : 4) : 0;  // raw e4m3 ring (to widen)
   static constexpr int A_TILE = BK * ROWB;
   static constexpr int B_TILE = N * ROWB;
   static constexpr int RAW_TILE = BK * D_I;
@@ -77,9 +84,9 @@ struct IndexerCfg {
   static constexpr int MMA_THREADS = PERSIST ? 2 : 1;
   static constexpr int CONVERT_WARP0 = MMA_WARP + MMA_THREADS;
   static constexpr int CONV_TEAMS = PERSIST ? 2 : 1;      // e4m3 converter teams (alternate tiles)
-  static constexpr int NWARPS = MMA_WARP + MMA_THREADS + (KFP8 ? 4 * CONV_TEAMS : 0);
+  static constexpr int NWARPS = MMA_WARP + MMA_THREADS + (CONVERT ? 4 * CONV_TEAMS : 0);
   static constexpr int NT = NWARPS * 32;
-  static constexpr uint32_t IDESC = idesc_bf16_f32(128, N, false, false);
+  static constexpr uint32_t IDESC = QFP8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N, false, false);
   // shared memory layout (offsets from a 1024-byte aligned base)
   static constexpr int QBUF = PERSIST ? 2 : 1;            // query tiles (double buffer when persistent)
   static constexpr int OFF_Q = 0;
@@ -97,6 +104,7 @@ struct IndexerCfg {
   static_assert(B_TILE % 1024 == 0 && A_TILE % 1024 == 0, "atom alignment");
   static_assert(COLS_PER_THREAD % LD_CHUNK == 0, "TMEM load chunking");
   static_assert(!KFP8 || D_I == 128, "e4m3 keys: 128-byte rows");
+  static_assert(!QFP8 || (KFP8 && !PERSIST && D_I == 128), "FP8 indexer: e4m3 keys, query-block grid, 128-byte rows");
   static_assert(TMEM_COLS <= 512, "tensor memory columns");
   static_assert(!K_IN_TMEM || (KFP8 && STAGES % CONV_TEAMS == 0), "converter teams own alternate stages");
   static_assert(NACC % EPI_WG == 0, "each accumulator is drained by one epilogue warpgroup");
@@ -169,6 +177,7 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t src, uint32_t& lo, uin
 
 struct IndexerParams {
   const float* w;            // [T, H_I]
+  const float* q_scale;      // [T, H_I] (FP8 indexer) or null
   const float* k_scale;      // [sum kv] (e4m3 keys) or null
   const int32_t* cu_q;
   const int32_t* cu_k;
@@ -176,8 +185,19 @@ struct IndexerParams {
   int64_t q_begin, q_end;    // global query rows of this call
   float* scores;             // [q_end - q_begin, ld]
   int64_t ld;
+  float* part_max;           // [q_end - q_begin, ld_pm] or null: max over each part of PART keys
+  int64_t ld_pm;
   int chunk_tiles;           // key tiles per CTA
 };
+
+// Max over the PART consecutive lanes of `v` (lanes 8i .. 8i+7); every lane
+// of the warp takes part.  Lane 8i gets the maximum of its part.
+__device__ __forceinline__ float part_max8(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, 1));
+  v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, 2));
+  v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, 4));
+  return v;
+}
 
 template <class C>
 __global__ void __launch_bounds__(C::NT, 1)
@@ -228,7 +248,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     mbar_init(bar_q_full, 1);
     mbar_init(bar_drain, 1);
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(bar_k_full(s), C::KFP8 ? 128 : 1);
+      mbar_init(bar_k_full(s), C::CONVERT ? 128 : 1);
       mbar_init(bar_k_empty(s), 1);
     }
     for (int s = 0; s < C::RSTAGES; ++s) {
@@ -250,10 +270,17 @@ __global__ void __launch_bounds__(C::NT, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
   }
-  // head weights of this block's queries (rows past the block are zero)
+  // head weights of this block's queries (rows past the block are zero); the
+  // FP8 indexer folds in each query head's scale and the 2^-7 of the rotation
   for (int i = threadIdx.x; i < C::NQ * C::H_I; i += C::NT) {
     const int qi = i / C::H_I;
-    w_s[i] = qi < nq ? p.w[(q0 + qi) * C::H_I + (i % C::H_I)] : 0.f;
+    float wv = 0.f;
+    if (qi < nq) {
+      const int64_t g = (q0 + qi) * C::H_I + (i % C::H_I);
+      wv = p.w[g];
+      if (C::QFP8) wv *= ldexpf(p.q_scale[g], -FP8_HADAMARD_LOG2);
+    }
+    w_s[i] = wv;
   }
   tc_fence_before();
   __syncthreads();
@@ -272,7 +299,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       int it = 0;
       for (; it < n_iter; ++it) {
         const int y = k_base + (t_begin + it) * C::BK;
-        if constexpr (C::KFP8) {
+        if constexpr (C::CONVERT) {
           const int r = it % C::RSTAGES;
           if (!mbar_wait(bar_raw_empty(r), ((it / C::RSTAGES) & 1) ^ 1, abort_flag, 11)) break;
           mbar_arrive_expect_tx(bar_raw_full(r), C::RAW_TILE);
@@ -289,9 +316,9 @@ __global__ void __launch_bounds__(C::NT, 1)
       if (*abort_flag) {
         // let copies already in flight land before the CTA's memory is released
         long long t0 = clock64();
-        constexpr int ring = C::KFP8 ? C::RSTAGES : C::STAGES;
+        constexpr int ring = C::CONVERT ? C::RSTAGES : C::STAGES;
         for (int j = (it > ring ? it - ring : 0); j < it; ++j) {
-          const uint32_t bar = C::KFP8 ? bar_raw_full(j % ring) : bar_k_full(j % ring);
+          const uint32_t bar = C::CONVERT ? bar_raw_full(j % ring) : bar_k_full(j % ring);
           while (!mbar_try_wait(bar, (j / ring) & 1) && clock64() - t0 < kWaitLimitCycles) {
           }
         }
@@ -320,7 +347,8 @@ __global__ void __launch_bounds__(C::NT, 1)
             const int off = (kk * 32) % C::SWB;
             const uint64_t ad = a_stage + static_cast<uint64_t>((atom * C::BK * C::SWB + off) >> 4);
             const uint64_t bd = b_desc0 + static_cast<uint64_t>((atom * C::N * C::SWB + off) >> 4);
-            umma_ss(tmem + a * C::N, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+            if constexpr (C::QFP8) umma_ss_e4m3(tmem + a * C::N, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
+            else umma_ss(tmem + a * C::N, ad, bd, C::IDESC, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar_k_empty(s));
           umma_commit(bar_acc_full(a));
@@ -332,9 +360,9 @@ __global__ void __launch_bounds__(C::NT, 1)
       while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < kWaitLimitCycles) {
       }
     }
-  } else if (C::KFP8 && warp >= C::CONVERT_WARP0) {
+  } else if (C::CONVERT && warp >= C::CONVERT_WARP0) {
     // ------------------------------------------------------------ e4m3 -> bf16
-    if constexpr (C::KFP8) {
+    if constexpr (C::CONVERT) {
     const int row = threadIdx.x - C::CONVERT_WARP0 * 32;  // key row of the tile
     for (int it = 0; it < n_iter; ++it) {
       const int r = it % C::RSTAGES;
@@ -378,15 +406,20 @@ __global__ void __launch_bounds__(C::NT, 1)
       tc_fence_before();
       mbar_arrive(bar_acc_empty(a));
       const int s = (t_begin + it) * C::BK + key_in_tile;
-      if (s < kv_len) {
-        float kscale = 1.f;
-        if (C::KFP8) kscale = p.k_scale[k_base + s];
+      const bool in_seq = s < kv_len;
+      float kscale = 1.f;
+      if (C::KFP8 && in_seq) kscale = p.k_scale[k_base + s];
 #pragma unroll
-        for (int q = 0; q < C::QW; ++q) {
-          const int qi = g * C::QW + q;
-          if (qi < nq) {
-            const float val = s <= pos0 + qi ? acc[q] * kscale : -INFINITY;
-            p.scores[(q0 + qi - p.q_begin) * p.ld + s] = val;
+      for (int q = 0; q < C::QW; ++q) {
+        const int qi = g * C::QW + q;          // the same for the whole warp
+        if (qi < nq) {
+          // keys past the query's position (and past the cache) score -inf
+          const float val = s <= pos0 + qi ? acc[q] * kscale : -INFINITY;
+          const int64_t row = q0 + qi - p.q_begin;
+          if (in_seq) p.scores[row * p.ld + s] = val;
+          if (p.part_max != nullptr) {
+            const float m = part_max8(val);
+            if ((lane & (PART - 1)) == 0 && in_seq) p.part_max[row * p.ld_pm + s / PART] = m;
           }
         }
       }
@@ -637,16 +670,16 @@ __global__ void __launch_bounds__(C::NT, 1)
     for (int it = team; it < n_iter; it += C::CONV_TEAMS) {
       const int r = it % C::RSTAGES;
       const int s = it % C::STAGES;
-      if (!mbar_wait(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag, 55)) break;
+      if (!mbar_wait_warp(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag, 55)) break;
       const uint8_t* raw_row = smem + C::OFF_RAW + r * C::RAW_TILE + row * 128;
       uint4 chunk[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)  // 128-byte swizzle: logical chunk j sits at j ^ (row & 7)
         chunk[j] = *reinterpret_cast<const uint4*>(raw_row + ((j ^ (row & 7)) << 4));
-      mbar_arrive(bar_raw_empty(r));
+      mbar_arrive_warp(bar_raw_empty(r));
       // stage s is free once the MMAs of tile it - STAGES completed: the phase
       // before the one the epilogue of tile it waits for on the same barrier
-      if (!mbar_wait(bar_acc_full(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, 56)) break;
+      if (!mbar_wait_warp(bar_acc_full(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, 56)) break;
       tc_fence_after();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {   // 64 elements (32 columns) per store
@@ -663,7 +696,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_ready(s));
+      mbar_arrive_warp(bar_ready(s));
     }
     if (lane == 0) DSA_PROF_SPAN(63, t_role);
   } else {
@@ -717,11 +750,15 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar_ready(a));   // accumulator a is free for tile it + NACC
+      mbar_arrive_warp(bar_ready(a));   // accumulator a is free for tile it + NACC
       const int s_key = (u - upre[b]) * C::BK + key_in_tile;
-      if (s_key < q.kv_len) {
-        const float val = s_key <= q.pos ? (acc0 + acc1) * ks : -INFINITY;
-        p.scores[(static_cast<int64_t>(q.q0) - p.q_begin) * p.ld + s_key] = val;
+      // keys past the query's position (and past the cache) score -inf
+      const float val = s_key <= q.pos ? (acc0 + acc1) * ks : -INFINITY;
+      const int64_t row = static_cast<int64_t>(q.q0) - p.q_begin;
+      if (s_key < q.kv_len) p.scores[row * p.ld + s_key] = val;
+      if (p.part_max != nullptr) {
+        const float m = part_max8(val);
+        if ((lane & (PART - 1)) == 0 && s_key < q.kv_len) p.part_max[row * p.ld_pm + s_key / PART] = m;
       }
       ks = ks_next;
     }

@@ -19,8 +19,15 @@
 // tensor memory, so the released shape runs on a cluster of two CTAs (two
 // SMs): CTA r owns output columns [256 r, 256 r + 256).  QK is split along K
 // the same way -- CTA 0 multiplies latent columns [0, 256), CTA 1 columns
-// [256, 576) -- so each CTA gathers only its own 256 or 320 columns of every
-// selected row and no MMA is duplicated.  The two partial score tiles are
+// [256, 576) -- so each CTA needs only its own 256 or 320 columns of every
+// selected row and no MMA is duplicated.  Fetching, though, goes by whole
+// rows: the cost of a random-row gather is set mostly by the number of rows
+// an SM requests, not by their bytes, so each CTA fetches the complete
+// 1152-byte rows of half of every tile (8 warps issuing TMA gathers, one
+// atom each) -- its own columns straight into its atom blocks, the peer's
+// columns into a staging block that a forwarder thread then copies into the
+// peer's atom blocks through distributed shared memory (flow-controlled by
+// per-stage barriers in both CTAs).  The two partial score tiles are
 // exchanged through distributed shared memory (each CTA stages its part in its
 // own shared memory and one bulk copy moves it into the peer's buffer,
 // completing on the peer's mbarrier); both CTAs add them in the same
@@ -28,13 +35,15 @@
 // softmax decisions.  Tensor memory holds O, three score buffers (a tile's P,
 // in bf16, overwrites its scores once they are in registers) and this CTA's
 // slice of the query, the A operand of every QK MMA, so shared memory is left
-// to a seven-deep ring of gathered rows and the score exchange.  The online
+// to a five-deep ring of gathered rows (and their staging) and the score
+// exchange.  The online
 // softmax keeps a per-head running max and only rescales O (in TMEM) when the
 // max grows by more than 2^8, which is exact arithmetic with the same final
 // normalisation.
 //
 // Roles per CTA: warps 0-3 query load, softmax and epilogue (one head row per
-// thread), warp 4 gather producer, warp 5 MMA issuer (and TMEM owner).
+// thread), warp 4 MMA issuer (and TMEM owner); with two CTAs warp 5 forwards
+// the staging to the peer and warps 6-13 gather; with one CTA warp 5 gathers.
 #pragma once
 
 #include "common.cuh"
@@ -57,9 +66,18 @@ struct MlaCfg {
   static constexpr int NA0 = SPLIT_ATOM;                  // atoms gathered by rank 0
   static constexpr int NA1 = NATOM_ALL - SPLIT_ATOM;      // atoms gathered by rank 1
   static constexpr int NA_MAX = NA0 > NA1 ? NA0 : NA1;
-  static constexpr int NS = SPLIT == 1 ? 4 : 7;           // gather ring depth
+  static constexpr int NS = SPLIT == 1 ? 4 : 5;           // gather ring depth
   static constexpr int C_ATOM_BYTES = BN * SWB;
-  static constexpr int C_STAGE = NA_MAX * C_ATOM_BYTES;
+  // 2-CTA split: each CTA fetches whole rows for HALF of a tile's rows; its
+  // own atoms land in its atom blocks (rows HALF*rank ..), the peer's atoms in
+  // a staging block that is then copied into the peer's atom blocks.
+  static constexpr int HALF = BN / 2;
+  static constexpr int HALF_ATOM_BYTES = HALF * SWB;
+  static constexpr int STG_MAX = SPLIT == 2 ? (NA0 > NA1 ? NA0 : NA1) : 0;   // staging blocks (the peer's atoms)
+  static constexpr int C_STAGE = SPLIT == 2 ? (NA0 * C_ATOM_BYTES + NA1 * HALF_ATOM_BYTES > NA1 * C_ATOM_BYTES + NA0 * HALF_ATOM_BYTES
+                                                   ? NA0 * C_ATOM_BYTES + NA1 * HALF_ATOM_BYTES
+                                                   : NA1 * C_ATOM_BYTES + NA0 * HALF_ATOM_BYTES)
+                                              : NA_MAX * C_ATOM_BYTES;
   static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;   // one partial-score tile
   static constexpr int OFF_C = 0;
   // Received partial-score tiles: tile j lands in buffer j % XR.  With four
@@ -73,7 +91,10 @@ struct MlaCfg {
   static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
   static constexpr int NSB = 3;                            // S buffers (each later holds its P)
   static constexpr int LOOKAHEAD = 2;                      // QK tiles issued ahead of PV
-  static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + XR + 5;
+  // q_ready, c_full/c_empty per stage, 3 per S buffer, x_full per receive
+  // buffer, drain, xs_full, xs_free; the 2-CTA split adds stg_full (staging
+  // landed) and partner_free (the peer's stage is free) per stage
+  static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + XR + 5 + (SPLIT == 2 ? 2 * NS : 0);
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // tensor memory columns: O [0, DVS); S[NSB] (fp32, BN each; P of the same
@@ -84,8 +105,14 @@ struct MlaCfg {
   static constexpr int QCOLS = NA_MAX * ATOM / 2;
   static constexpr int TMEM_USED = TMEM_Q + QCOLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
-  static constexpr int NT = 6 * 32;
-  static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
+  // roles: warps 0-3 softmax and epilogue, MMA_WARP the MMA issuer (and TMEM
+  // owner); the 2-CTA split has a forwarder warp and NPROD gather warps
+  // (more warps issuing TMA gathers raise the row rate of one SM)
+  static constexpr int MMA_WARP = 4;
+  static constexpr int FWD_WARP = 5;
+  static constexpr int NPROD = SPLIT == 2 ? 8 : 1;
+  static constexpr int PROD_WARP0 = SPLIT == 2 ? 6 : 5;
+  static constexpr int NT = (PROD_WARP0 + NPROD) * 32;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, DVS, false, true);
   static constexpr float kRescaleThreshold = 8.0f;        // log2 units
@@ -98,6 +125,8 @@ struct MlaCfg {
   static_assert(QCOLS % 8 == 0, "query columns are stored eight at a time");
   static_assert(TMEM_USED <= 512, "tensor memory");
   static_assert(OFF_C % 1024 == 0 && C_STAGE % 1024 == 0 && C_ATOM_BYTES % 1024 == 0, "swizzle atoms");
+  static_assert(SPLIT == 1 || (HALF_ATOM_BYTES % 1024 == 0 && HALF % 4 == 0 && NATOM_ALL <= 2 * NPROD),
+                "half-tile blocks keep the swizzle phase; every atom has a gather warp");
   static_assert(OFF_X % 16 == 0 && OFF_XS % 16 == 0 && OFF_BAR % 8 == 0, "vector / bulk-copy / barrier alignment");
 };
 
@@ -123,8 +152,10 @@ __global__ void __launch_bounds__(C::NT, 1)
   const int64_t t = p.q_begin + r_local;
   const RowInfo ri = locate_row(p.cu_q, p.cu_k, p.B, t);
   const int32_t* __restrict__ idx_row = p.idx + r_local * p.topk;
-  const int a0 = rank == 0 ? 0 : C::SPLIT_ATOM;           // first gathered atom (global)
-  const int na = rank == 0 ? C::NA0 : C::NA1;             // atoms gathered by this CTA
+  const int a0 = rank == 0 ? 0 : C::SPLIT_ATOM;           // first atom of this CTA's columns (global)
+  const int na = rank == 0 ? C::NA0 : C::NA1;             // atoms of this CTA's columns
+  const int p0 = rank == 0 ? C::SPLIT_ATOM : 0;           // the peer's columns
+  const int np = rank == 0 ? C::NA1 : C::NA0;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -149,6 +180,14 @@ __global__ void __launch_bounds__(C::NT, 1)
   // outgoing staging buffer: every row written (128 arrivals) / read by the previous copy (thread 0)
   const uint32_t bar_xs_full = bar0 + 8 * (XB0 + C::XR + 1);
   const uint32_t bar_xs_free = bar0 + 8 * (XB0 + C::XR + 2);
+  // 2-CTA split: this CTA's staging of stage s landed (the peer's atoms of
+  // its own rows) / the peer's stage s is free for this CTA's rows
+  constexpr int FB0 = XB0 + C::XR + 3;
+  auto bar_stg_full = [&](int s) { return bar0 + 8 * (FB0 + s); };
+  auto bar_partner_free = [&](int s) { return bar0 + 8 * (FB0 + C::NS + s); };
+  // stage s: this CTA's atom blocks (BN rows each), then the staging blocks (HALF rows each)
+  auto own_block = [&](int s, int l) { return s_c + s * C::C_STAGE + l * C::C_ATOM_BYTES; };
+  auto stg_block = [&](int s, int m) { return s_c + s * C::C_STAGE + na * C::C_ATOM_BYTES + m * C::HALF_ATOM_BYTES; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* ntiles_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -160,8 +199,17 @@ __global__ void __launch_bounds__(C::NT, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar_q_ready, 128);
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(bar_c_full(s), 1);
-      mbar_init(bar_c_empty(s), 1);
+      if (C::SPLIT == 2) {
+        // c_full: every gather warp (its bytes) + the peer's forwarded rows;
+        // c_empty: the MMAs that read the stage + the forwarder (staging read)
+        mbar_init(bar_c_full(s), C::NPROD + 1);
+        mbar_init(bar_c_empty(s), 2);
+        mbar_init(bar_stg_full(s), C::NPROD);
+        mbar_init(bar_partner_free(s), 1);
+      } else {
+        mbar_init(bar_c_full(s), 1);
+        mbar_init(bar_c_empty(s), 1);
+      }
     }
     for (int a = 0; a < C::NSB; ++a) {
       mbar_init(bar_s_full(a), 1);
@@ -182,7 +230,7 @@ __global__ void __launch_bounds__(C::NT, 1)
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == C::PRODUCER_WARP && lane == 0) tma_prefetch_desc(&tm_lat);
+  if (warp >= C::PROD_WARP0 && lane == 0) tma_prefetch_desc(&tm_lat);
   DSA_PROF_BEGIN();
   __syncthreads();
   // Tiles up to the last one holding a valid entry (trailing -1 padding is skipped).
@@ -206,8 +254,8 @@ __global__ void __launch_bounds__(C::NT, 1)
   const int n_tiles = skip ? 0 : *ntiles_s;
 
   const long long t_role = clock64();
-  if (warp == C::PRODUCER_WARP) {
-    // ------------------------------------------------------------ gather producer
+  if (C::SPLIT == 1 && warp >= C::PROD_WARP0) {
+    // ------------------------------------------------------------ gather producer (one CTA)
     int it = 0;
     if (n_tiles > 0) {
       for (; it < n_tiles; ++it) {
@@ -245,6 +293,99 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
     }
     if (lane == 0) DSA_PROF_SPAN(61, t_role);
+  } else if (C::SPLIT == 2 && warp >= C::PROD_WARP0) {
+    // ------------------------------------------------------------ gather warps (2-CTA split)
+    // This CTA fetches the whole rows HALF*rank .. HALF*rank + HALF-1 of every
+    // tile: its own atoms into its atom blocks, the peer's atoms into staging.
+    // Gather warp w takes the atoms g = w, w + NPROD, ... of the 9; lanes
+    // 0..HALF/4-1 each issue one gather4 (four rows) per atom.
+    const int w = warp - C::PROD_WARP0;
+    int n_own = 0, n_stg = 0;
+    for (int g = w; g < C::NATOM_ALL; g += C::NPROD) {
+      if (g >= a0 && g < a0 + na) ++n_own; else ++n_stg;
+    }
+    int it = 0;
+    if (n_tiles > 0) {
+      for (; it < n_tiles; ++it) {
+        const int s = it % C::NS;
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(bar_c_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, 21);
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) break;
+        // this CTA's rows of the tile (lanes 0..HALF-1)
+        const int e = it * C::BN + C::HALF * static_cast<int>(rank) + (lane & (C::HALF - 1));
+        const int sel = e < p.topk ? idx_row[e] : -1;
+        const bool valid = sel >= 0 && sel <= ri.pos;
+        const int grow = ri.k_base + (valid ? sel : 0);
+        int y[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) y[j] = __shfl_sync(0xFFFFFFFFu, grow, (4 * lane + j) & (C::HALF - 1));
+        if (w == 0) {
+          // validity of all BN rows of the tile (both halves), read after c_full
+          const int e2 = it * C::BN + lane;
+          const int sel2 = e2 < p.topk ? idx_row[e2] : -1;
+          const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, sel2 >= 0 && sel2 <= ri.pos);
+          if (lane == 0) mask_s[s] = vmask;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_c_full(s), n_own * C::HALF_ATOM_BYTES);
+          mbar_arrive_expect_tx(bar_stg_full(s), n_stg * C::HALF_ATOM_BYTES);
+        }
+        __syncwarp();
+        if (lane < C::HALF / 4) {
+          for (int g = w; g < C::NATOM_ALL; g += C::NPROD) {
+            if (g >= a0 && g < a0 + na)
+              tma_gather4(own_block(s, g - a0) + rank * C::HALF_ATOM_BYTES + lane * 4 * C::SWB, &tm_lat,
+                          bar_c_full(s), g * C::ATOM, y[0], y[1], y[2], y[3]);
+            else
+              tma_gather4(stg_block(s, g - p0) + lane * 4 * C::SWB, &tm_lat, bar_stg_full(s), g * C::ATOM, y[0],
+                          y[1], y[2], y[3]);
+          }
+        }
+      }
+      if (lane == 0 && *abort_flag) {
+        // let this warp's copies in flight land before the CTA leaves (c_full
+        // also waits for the peer's rows, which may never come after an
+        // error: the wait is bounded)
+        long long t0 = clock64();
+        for (int j = (it > C::NS ? it - C::NS : 0); j < it; ++j) {
+          while (!mbar_try_wait(bar_stg_full(j % C::NS), (j / C::NS) & 1) && clock64() - t0 < kWaitLimitCycles) {
+          }
+          while (!mbar_try_wait(bar_c_full(j % C::NS), (j / C::NS) & 1) && clock64() - t0 < kWaitLimitCycles) {
+          }
+        }
+      }
+    }
+    if (lane == 0 && w == 0) DSA_PROF_SPAN(61, t_role);
+  } else if (C::SPLIT == 2 && warp == C::FWD_WARP) {
+    // ------------------------------------------------------------ forwarder (2-CTA split)
+    // Per tile: (1) once this CTA's stage s no longer holds tile it - NS, tell
+    // the peer it may copy its rows of tile it there; (2) wait for this CTA's
+    // staging of tile it and (3) for the peer's go-ahead; (4) copy the
+    // staging into the peer's atom blocks (rows HALF*rank ..), completing on
+    // the peer's c_full; (5) once the copies have read the staging, count as
+    // the staging's share of this stage's c_empty.
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t peer_stage0 = mapa_shared(s_c, peer);
+      int it = 0;
+      for (; it < n_tiles; ++it) {
+        const int s = it % C::NS;
+        if (it >= C::NS && !mbar_wait(bar_c_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, 35)) break;
+        mbar_arrive_remote(mapa_shared(bar_partner_free(s), peer));
+        if (!mbar_wait(bar_stg_full(s), (it / C::NS) & 1, abort_flag, 36)) break;
+        if (!mbar_wait<true>(bar_partner_free(s), (it / C::NS) & 1, abort_flag, 37)) break;
+        const uint32_t peer_full = mapa_shared(bar_c_full(s), peer);
+        mbar_arrive_expect_tx_remote(peer_full, np * C::HALF_ATOM_BYTES);
+        for (int m = 0; m < np; ++m)
+          bulk_copy_to_peer(peer_stage0 + s * C::C_STAGE + m * C::C_ATOM_BYTES + rank * C::HALF_ATOM_BYTES,
+                            stg_block(s, m), C::HALF_ATOM_BYTES, peer_full);
+        bulk_commit_group();
+        bulk_wait_group_read<0>();
+        mbar_arrive(bar_c_empty(s));
+      }
+      bulk_wait_group<0>();   // the copies have landed in the peer before this CTA can leave
+      DSA_PROF_SPAN(59, t_role);
+    }
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_tiles > 0) {
@@ -330,7 +471,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_q_ready);
+      mbar_arrive_warp(bar_q_ready);
     }
     // Load tile j's partial scores S[j % 3] and (2-CTA split) start sending them
     // to the peer.  Tile it+1 is started before tile it is finished, so the
@@ -366,7 +507,7 @@ __global__ void __launch_bounds__(C::NT, 1)
                                                                    dst[4 * c + 3]);
         }
         fence_proxy_async_smem();
-        mbar_arrive(bar_xs_full);
+        mbar_arrive_warp(bar_xs_full);
         int go = 1;
         if (h == 0) {
           // all rows staged (the peer's buffer xr is free: see XR)
@@ -454,7 +595,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       tmem_st16(tmem + lane_base + C::TMEM_S + sb * C::BN, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p_full(sb));
+      mbar_arrive_warp(bar_p_full(sb));
 #pragma unroll
       for (int c = 0; c < C::BN; ++c) sv[c] = s_next[c];
     }

@@ -38,6 +38,8 @@ struct TopkCfg {
   static constexpr int MAX_N = (65535 / PER_WARP) * CHUNK;   // 16-bit per-warp pass-1 counters
   static constexpr int PMAX_CAP = 8192;               // fast path: part maxima kept
   static constexpr int BITMAP_BITS = 262144;          // fast path: longest row (one bit per key)
+  static constexpr int PM_CAP = STAGES * CHUNK;       // part-maxima path: groups kept (in the ring)
+  static constexpr int PLIST_CAP = 16384;             // part-maxima path: groups that can hold a selection
   static constexpr int OFF_RING = 0;
   // union: per-warp pass-1 histograms (exact path) | part maxima + selection bitmap (fast path)
   static constexpr int OFF_WHIST = OFF_RING + STAGES * CHUNK * 4;   // per-warp pass-1 histograms
@@ -47,10 +49,12 @@ struct TopkCfg {
   static constexpr int OFF_CKEY = OFF_HIST + BINS1 * 4;
   static constexpr int OFF_CIDX = OFF_CKEY + CAP * 4;
   static constexpr int OFF_WTOT = OFF_CIDX + CAP * 4;
-  static constexpr int OFF_BAR = OFF_WTOT + 2 * NW * 4;
+  static constexpr int OFF_CNT = OFF_WTOT + 2 * NW * 4;   // select: per-warp digit counts + totals
+  static constexpr int OFF_BAR = OFF_CNT + (128 + NW) * 4;
   static constexpr int OFF_MISC = OFF_BAR + STAGES * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 128;   // + alignment slack
   static_assert(PMAX_CAP * 4 + BITMAP_BITS / 8 <= NW * (BINS1 / 2) * 4, "fast-path union fits");
+  static_assert(PLIST_CAP * 4 <= NW * (BINS1 / 2) * 4, "group list fits the histogram union");
   static_assert(OFF_RING % 128 == 0 && (CHUNK * 4) % 128 == 0, "bulk-copy destinations");
   static_assert(OFF_BAR % 8 == 0 && OFF_MISC % 8 == 0, "barrier alignment");
 };
@@ -67,9 +71,9 @@ __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t lane, ui
 }
 
 __global__ void __launch_bounds__(TopkCfg::NT, 1)
-    topk_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ cu_q,
-                const int32_t* __restrict__ cu_k, int B, int64_t q_begin, int topk,
-                int32_t* __restrict__ idx) {
+    topk_kernel(const float* __restrict__ scores, int64_t ld, const float* __restrict__ part_max, int64_t ld_pm,
+                const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_k, int B, int64_t q_begin,
+                int topk, int32_t* __restrict__ idx) {
   using C = TopkCfg;
   const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t r = blockIdx.x;
@@ -91,6 +95,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
   uint32_t* ckey = reinterpret_cast<uint32_t*>(smem + C::OFF_CKEY);
   int32_t* cidx = reinterpret_cast<int32_t*>(smem + C::OFF_CIDX);
   uint32_t* wtot = reinterpret_cast<uint32_t*>(smem + C::OFF_WTOT);
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + C::OFF_CNT);
   const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 16);
@@ -255,6 +260,318 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     __syncthreads();
   };
 
+  // Radix-4 selection.  select(count, key_of, use, kth, &thr, &rem, steps):
+  // the kth largest key among the entries i < count with use(i) (at least kth
+  // of them), found 2 bits at a time from the top: each step counts, for the
+  // 3 candidate values of the next digit, the entries at or above them
+  // (compares in registers, warp sums by redux, one shared slot per warp and
+  // value), and keeps the largest digit with at least kth entries at or above
+  // it.  No atomics, so concentrated key distributions cost nothing extra.
+  // Up to SEL_REG entries per thread are read once into registers.  With
+  // steps < 16 only the top 2*steps bits are resolved and the lower bits are
+  // 0: thr is then a lower bound of the kth largest key with at least kth
+  // entries >= thr.  *rem = kth - (entries > thr) (meaningful for steps = 16).
+  // Called by every thread.
+  uint32_t* slots = cnt;   // [16 warps][4]; slots + 64: the 3 totals
+  auto select = [&](uint32_t count, auto&& key_of, auto&& use, uint32_t kth, uint32_t* out_thr,
+                    uint32_t* out_rem, int steps = 16) {
+    constexpr int SEL_REG = 12;
+    const bool in_regs = count <= static_cast<uint32_t>(SEL_REG * C::NT);
+    uint32_t kr[SEL_REG];   // this thread's keys (entries tid, tid + NT, ...); unused ones are 0 with use = false
+    uint32_t ur = 0;        // bit e: entry e is used
+#pragma unroll
+    for (int e = 0; e < SEL_REG; ++e) {
+      const uint32_t i = tid + static_cast<uint32_t>(e) * C::NT;
+      kr[e] = 0u;
+      if (in_regs && i < count && use(i)) {
+        kr[e] = key_of(i);
+        ur |= 1u << e;
+      }
+    }
+    uint32_t prefix = 0;
+    for (int st = 0; st < steps; ++st) {
+      const int shift = 30 - 2 * st;
+      const uint32_t t1 = prefix | (1u << shift), t2 = prefix | (2u << shift), t3 = prefix | (3u << shift);
+      uint32_t c1 = 0, c2 = 0, c3 = 0;
+      if (in_regs) {
+#pragma unroll
+        for (int e = 0; e < SEL_REG; ++e) {
+          const uint32_t k = kr[e];
+          const uint32_t u = (ur >> e) & 1u;
+          c1 += u & (k >= t1 ? 1u : 0u);
+          c2 += u & (k >= t2 ? 1u : 0u);
+          c3 += u & (k >= t3 ? 1u : 0u);
+        }
+      } else {
+        for (uint32_t i = tid; i < count; i += C::NT) {
+          if (!use(i)) continue;
+          const uint32_t k = key_of(i);
+          c1 += k >= t1 ? 1u : 0u;
+          c2 += k >= t2 ? 1u : 0u;
+          c3 += k >= t3 ? 1u : 0u;
+        }
+      }
+      c1 = __reduce_add_sync(0xFFFFFFFFu, c1);
+      c2 = __reduce_add_sync(0xFFFFFFFFu, c2);
+      c3 = __reduce_add_sync(0xFFFFFFFFu, c3);
+      uint32_t* sl = slots + (st & 1) * 64;   // alternate slot sets: one barrier per step
+      if (lane == 0) {
+        sl[warp * 4 + 0] = c1;
+        sl[warp * 4 + 1] = c2;
+        sl[warp * 4 + 2] = c3;
+      }
+      __syncthreads();
+      uint32_t s1 = 0, s2 = 0, s3 = 0;
+#pragma unroll
+      for (int w = 0; w < C::NW; ++w) {
+        s1 += sl[w * 4 + 0];
+        s2 += sl[w * 4 + 1];
+        s3 += sl[w * 4 + 2];
+      }
+      const uint32_t digit = (s1 >= kth ? 1u : 0u) + (s2 >= kth ? 1u : 0u) + (s3 >= kth ? 1u : 0u);
+      prefix |= digit << shift;
+    }
+    uint32_t gt = 0;
+    if (steps == 16) {
+      if (in_regs) {
+#pragma unroll
+        for (int e = 0; e < SEL_REG; ++e) gt += ((ur >> e) & 1u) & (kr[e] > prefix ? 1u : 0u);
+      } else {
+        for (uint32_t i = tid; i < count; i += C::NT) gt += (use(i) && key_of(i) > prefix) ? 1u : 0u;
+      }
+    }
+    gt = __reduce_add_sync(0xFFFFFFFFu, gt);
+    uint32_t* sl = slots + 128;
+    if (lane == 0) sl[warp] = gt;
+    __syncthreads();
+    uint32_t total = 0;
+#pragma unroll
+    for (int w = 0; w < C::NW; ++w) total += sl[w];
+    __syncthreads();
+    *out_thr = prefix;
+    *out_rem = kth - total;
+  };
+  // Block-wide exclusive prefix of one count per thread (in thread order) and the total.
+  auto block_scan = [&](uint32_t v, uint32_t* total) -> uint32_t {
+    uint32_t wt;
+    const uint32_t pre = warp_excl_scan(v, lane, &wt);
+    if (lane == 31) wtot[warp] = pre + v;
+    __syncthreads();
+    uint32_t base = pre, tot = 0;
+#pragma unroll
+    for (int w = 0; w < C::NW; ++w) {
+      const uint32_t x = wtot[w];
+      base += w < static_cast<int>(warp) ? x : 0u;
+      tot += x;
+    }
+    __syncthreads();
+    *total = tot;
+    return base;
+  };
+  // Exact selection among candidates ckey/cidx[0, nc) that hold every key
+  // >= some bound b with at least topk keys >= b: the topk largest keys, ties
+  // to the lowest index, written in increasing index order through a bitmap
+  // of the row (n <= BITMAP_BITS).  Called by every thread.
+  auto finish_candidates = [&](uint32_t nc) {
+    uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + C::OFF_BITMAP);
+    uint32_t thr, need_eq;
+    select(nc, [&](uint32_t i) { return ckey[i]; }, [&](uint32_t) { return true; },
+           static_cast<uint32_t>(topk), &thr, &need_eq);
+    // ties at the threshold: the need_eq lowest indices (largest ~index)
+    uint32_t ties_mine = 0, n_ties;
+    for (uint32_t i = tid; i < nc; i += C::NT) ties_mine += ckey[i] == thr ? 1u : 0u;
+    block_scan(ties_mine, &n_ties);
+    uint32_t inv_idx_thr = 0u;   // select every tie
+    if (n_ties > need_eq) {
+      uint32_t rem2;
+      select(nc, [&](uint32_t i) { return ~static_cast<uint32_t>(cidx[i]); },
+             [&](uint32_t i) { return ckey[i] == thr; }, need_eq, &inv_idx_thr, &rem2);
+    }
+    // ---- selection -> bitmap -> indices in increasing order
+    const int nwords = (n + 31) / 32;
+    for (int i = tid; i < nwords; i += C::NT) bitmap[i] = 0u;
+    __syncthreads();
+    for (uint32_t i = tid; i < nc; i += C::NT) {
+      const uint32_t key = ckey[i];
+      const int id = cidx[i];
+      if (key > thr || (key == thr && ~static_cast<uint32_t>(id) >= inv_idx_thr))
+        atomicOr(&bitmap[id >> 5], 1u << (id & 31));
+    }
+    __syncthreads();
+    const int per = (nwords + C::NT - 1) / C::NT;
+    const int w0 = min(nwords, static_cast<int>(tid) * per), w1 = min(nwords, w0 + per);
+    uint32_t cnt = 0;
+    for (int wdx = w0; wdx < w1; ++wdx) cnt += __popc(bitmap[wdx]);
+    uint32_t wt;
+    const uint32_t pre = warp_excl_scan(cnt, lane, &wt);
+    if (lane == 31) wtot[warp] = pre + cnt;
+    __syncthreads();
+    uint32_t pos_out = pre;
+    for (int w = 0; w < static_cast<int>(warp); ++w) pos_out += wtot[w];
+    for (int wdx = w0; wdx < w1; ++wdx) {
+      uint32_t bits = bitmap[wdx];
+      while (bits) {
+        const int bpos = __ffs(bits) - 1;
+        bits &= bits - 1;
+        out[pos_out++] = wdx * 32 + bpos;
+      }
+    }
+  };
+
+  // ================================================================== part-maxima path
+  // The indexer's epilogue wrote, beside the scores, the maximum of every
+  // part of PART consecutive keys (-inf past the query's position).  Parts are
+  // grouped G2 at a time (G2 a power of two: about 2 k to 4 k groups, at most
+  // PM_CAP).  At least k scores are >= the k-th largest part maximum b (each
+  // of the k parts above it holds one), so every selected score is >= b and
+  // only the parts whose maximum is >= b (about k of them) can hold one:
+  // those parts are read from the row, their scores >= b become the
+  // candidates, and the exact selection runs among them.  The row itself is
+  // read only where it matters.  Rows with fewer than 1.25 k groups, rows past
+  // the bitmap, or candidate overflows (massive ties) take the paths below.
+  if (part_max != nullptr && n <= C::BITMAP_BITS) {
+    const int P = (n + PART - 1) / PART;
+    // Groups of G2 parts: about 2 k to 4 k groups keep the selection cheap
+    // (its cost grows with the groups) while the candidates stay near k.
+    int G2 = 1;
+    while ((P + 2 * G2 - 1) / (2 * G2) >= 2 * topk || (P + G2 - 1) / G2 > C::PM_CAP) G2 <<= 1;
+    const int Pg = (P + G2 - 1) / G2;
+    // With few groups per selected key the bound b is low and the candidates
+    // would overflow; 1.25 k groups keep them at ~2.5 k for continuous scores.
+    if (4 * static_cast<int64_t>(Pg) >= 5 * static_cast<int64_t>(topk)) {
+      uint32_t* pk = reinterpret_cast<uint32_t*>(smem + C::OFF_RING);    // group maxima as keys
+      int32_t* plist = reinterpret_cast<int32_t*>(smem + C::OFF_WHIST);  // groups that can hold a selection
+      const float4* __restrict__ pm4 = reinterpret_cast<const float4*>(part_max + r * ld_pm);
+      // Group maxima from 16-byte loads of 4 part maxima (rows of ld_pm, a
+      // multiple of 4 that covers P, so a load that starts below P stays in
+      // the row); parts past P count as the smallest key.
+      const int nf4 = (P + 3) / 4;
+      auto keys4 = [&](int f, uint32_t* k) {
+        const float4 v = pm4[f];
+        const float vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) k[e] = 4 * f + e < P ? order_key(vals[e]) : 0u;
+      };
+      if (G2 >= 4) {
+        const int f4g = G2 / 4;
+#pragma unroll 4
+        for (int i = tid; i < Pg; i += C::NT) {
+          uint32_t m = 0u;
+          for (int j = 0; j < f4g; ++j) {
+            const int f = i * f4g + j;
+            if (f < nf4) {
+              uint32_t k[4];
+              keys4(f, k);
+              m = max(m, max(max(k[0], k[1]), max(k[2], k[3])));
+            }
+          }
+          pk[i] = m;
+        }
+      } else {
+#pragma unroll 4
+        for (int f = tid; f < nf4; f += C::NT) {
+          uint32_t k[4];
+          keys4(f, k);
+          if (G2 == 1) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (4 * f + e < Pg) pk[4 * f + e] = k[e];
+          } else {
+            if (2 * f < Pg) pk[2 * f] = max(k[0], k[1]);
+            if (2 * f + 1 < Pg) pk[2 * f + 1] = max(k[2], k[3]);
+          }
+        }
+      }
+      __syncthreads();
+      phase(48);
+      // A lower bound of the k-th largest group maximum (its top 16 bits):
+      // at least k groups, hence k scores, are >= b.
+      uint32_t b, unused_rem;
+      select(static_cast<uint32_t>(Pg), [&](uint32_t i) { return pk[i]; }, [&](uint32_t) { return true; },
+             static_cast<uint32_t>(topk), &b, &unused_rem, 8);
+      phase(50);
+      // the groups whose maximum is >= b, in order (contiguous ranges per thread, one block scan)
+      const int per = (Pg + C::NT - 1) / C::NT;
+      const int g_lo = min(Pg, static_cast<int>(tid) * per), g_hi = min(Pg, g_lo + per);
+      uint32_t mine = 0;
+      for (int i = g_lo; i < g_hi; ++i) mine += pk[i] >= b ? 1u : 0u;
+      uint32_t ng;
+      uint32_t at = block_scan(mine, &ng);
+      for (int i = g_lo; i < g_hi; ++i)
+        if (pk[i] >= b) {
+          if (at < static_cast<uint32_t>(C::PLIST_CAP)) plist[at] = i;
+          ++at;
+        }
+      __syncthreads();
+      if (ng <= static_cast<uint32_t>(C::PLIST_CAP)) {
+        // Candidates: the scores >= b of those groups, counted in a first
+        // pass and written in a second at offsets from a block scan (no
+        // atomics).  16-byte loads; a load starts below n, and n <= ld with ld
+        // a multiple of 4, so it stays inside the row.
+        const int f4_per_group = G2 * PART / 4;
+        const uint32_t items = ng * static_cast<uint32_t>(f4_per_group);
+        // Items (16-byte loads) in batches of IB per thread, every load of a
+        // batch issued before any is used, so that the L2 latency overlaps.
+        constexpr int IB = 8;
+        auto batch = [&](uint32_t base, uint32_t* k, int* k0) {
+          float4 v[IB];
+#pragma unroll
+          for (int u = 0; u < IB; ++u) {
+            const uint32_t it = base + static_cast<uint32_t>(u) * C::NT;
+            k0[u] = n;
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (it < items) {
+              k0[u] = plist[it / f4_per_group] * G2 * PART + static_cast<int>(it % f4_per_group) * 4;
+              if (k0[u] < n) v[u] = *reinterpret_cast<const float4*>(row + k0[u]);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < IB; ++u) {
+            k[4 * u + 0] = order_key(v[u].x);
+            k[4 * u + 1] = order_key(v[u].y);
+            k[4 * u + 2] = order_key(v[u].z);
+            k[4 * u + 3] = order_key(v[u].w);
+          }
+        };
+        uint32_t count = 0;
+        for (uint32_t base = tid; base < items; base += IB * C::NT) {
+          uint32_t k[4 * IB];
+          int k0[IB];
+          batch(base, k, k0);
+#pragma unroll
+          for (int u = 0; u < IB; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) count += (k0[u] + e < n && k[4 * u + e] >= b) ? 1u : 0u;
+        }
+        uint32_t nc;
+        uint32_t w_at = block_scan(count, &nc);
+        if (nc <= static_cast<uint32_t>(C::CAP)) {
+          for (uint32_t base = tid; base < items; base += IB * C::NT) {
+            uint32_t k[4 * IB];
+            int k0[IB];
+            batch(base, k, k0);
+#pragma unroll
+            for (int u = 0; u < IB; ++u)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                if (k0[u] + e < n && k[4 * u + e] >= b) {
+                  ckey[w_at] = k[4 * u + e];
+                  cidx[w_at] = k0[u] + e;
+                  ++w_at;
+                }
+          }
+          __syncthreads();
+          phase(49);
+          finish_candidates(nc);
+          phase(45);
+          DSA_PROF_END();
+          return;
+        }
+      }
+      __syncthreads();   // overflow: the paths below
+    }
+  }
+
   // ================================================================== fast path
   // Split the row into parts of PS scores (part = PS consecutive scores of one
   // thread's 16 per chunk, or one thread's scores over G chunks).  At least k
@@ -274,7 +591,6 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     const bool eligible = n <= C::BITMAP_BITS && n > topk && P <= C::PMAX_CAP && (G == 1 || PS == 16);
     if (eligible) {
       uint32_t* pmax = reinterpret_cast<uint32_t*>(smem + C::OFF_PMAX);
-      uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + C::OFF_BITMAP);
       for (int i = tid; i < P; i += C::NT) pmax[i] = 0u;
       for (int i = tid; i < C::BINS1; i += C::NT) hist[i] = 0u;
       __syncthreads();
@@ -331,38 +647,10 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
       });
       phase(41);
       if (!ok) { DSA_PROF_END(); return; }
-    // exact kth-largest key among entries i < count with use(i) (digits of 11, 11, 10 bits)
-    auto select = [&](uint32_t count, auto&& key_of, auto&& use, uint32_t kth, uint32_t* out_thr,
-                      uint32_t* out_rem) {
-        uint32_t prefix = 0, remaining = kth;
-        const int shifts[3] = {21, 10, 0};
-        const int widths[3] = {11, 11, 10};
-        for (int d = 0; d < 3; ++d) {
-          const int shift = shifts[d], bits = widths[d];
-          const int hi = shift + bits;
-          for (int i = tid; i < (1 << bits); i += C::NT) hist[i] = 0u;
-          __syncthreads();
-          for (uint32_t base = 0; base < count; base += C::NT) {
-            const uint32_t i = base + tid;
-            const bool in = i < count && use(i);
-            const uint32_t key = in ? key_of(i) : 0u;
-            const bool m = in && (hi >= 32 || (key >> hi) == (prefix >> hi));
-            hist_add(hist, (key >> shift) & ((1u << bits) - 1u), m);
-          }
-          __syncthreads();
-          find_digit_fn(hist, 1 << bits, remaining, &misc[2], &misc[3]);
-          __syncthreads();
-          prefix |= misc[2] << shift;
-          remaining -= misc[3];
-          __syncthreads();
-        }
-        *out_thr = prefix;
-        *out_rem = remaining;
-      };
-      // ---- lower bound b = the k-th largest part maximum (exact)
+      // ---- lower bound b of the k-th largest part maximum (its top 16 bits)
       uint32_t b_lo, unused_rem;
       select(static_cast<uint32_t>(P), [&](uint32_t i) { return pmax[i]; }, [&](uint32_t) { return true; },
-             static_cast<uint32_t>(topk), &b_lo, &unused_rem);
+             static_cast<uint32_t>(topk), &b_lo, &unused_rem, 8);
       if (tid == 0) misc[4] = 0u;   // candidate count
       __syncthreads();
       phase(42);
@@ -408,51 +696,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
       if (!ok) { DSA_PROF_END(); return; }
       const uint32_t nc = *cand_n;
       if (nc <= static_cast<uint32_t>(C::CAP)) {
-        uint32_t thr, need_eq;
-        select(nc, [&](uint32_t i) { return ckey[i]; }, [&](uint32_t) { return true; },
-               static_cast<uint32_t>(topk), &thr, &need_eq);
-        phase(44);
-        // ties at the threshold: the need_eq lowest indices (largest ~index)
-        if (tid == 0) misc[5] = 0u;
-        __syncthreads();
-        for (uint32_t i = tid; i < nc; i += C::NT)
-          if (ckey[i] == thr) atomicAdd(&misc[5], 1u);
-        __syncthreads();
-        uint32_t inv_idx_thr = 0u;   // select every tie
-        if (misc[5] > need_eq) {
-          uint32_t rem2;
-          select(nc, [&](uint32_t i) { return ~static_cast<uint32_t>(cidx[i]); },
-                 [&](uint32_t i) { return ckey[i] == thr; }, need_eq, &inv_idx_thr, &rem2);
-        }
-        // ---- selection -> bitmap -> indices in increasing order
-        const int nwords = (n + 31) / 32;
-        for (int i = tid; i < nwords; i += C::NT) bitmap[i] = 0u;
-        __syncthreads();
-        for (uint32_t i = tid; i < nc; i += C::NT) {
-          const uint32_t key = ckey[i];
-          const int id = cidx[i];
-          if (key > thr || (key == thr && ~static_cast<uint32_t>(id) >= inv_idx_thr))
-            atomicOr(&bitmap[id >> 5], 1u << (id & 31));
-        }
-        __syncthreads();
-        const int per = (nwords + C::NT - 1) / C::NT;
-        const int w0 = min(nwords, static_cast<int>(tid) * per), w1 = min(nwords, w0 + per);
-        uint32_t cnt = 0;
-        for (int wdx = w0; wdx < w1; ++wdx) cnt += __popc(bitmap[wdx]);
-        uint32_t wt;
-        const uint32_t pre = warp_excl_scan(cnt, lane, &wt);
-        if (lane == 31) wtot[warp] = pre + cnt;
-        __syncthreads();
-        uint32_t pos_out = pre;
-        for (int w = 0; w < static_cast<int>(warp); ++w) pos_out += wtot[w];
-        for (int wdx = w0; wdx < w1; ++wdx) {
-          uint32_t bits = bitmap[wdx];
-          while (bits) {
-            const int bpos = __ffs(bits) - 1;
-            bits &= bits - 1;
-            out[pos_out++] = wdx * 32 + bpos;
-          }
-        }
+        finish_candidates(nc);
         phase(45);
         DSA_PROF_END();
         return;

@@ -17,14 +17,18 @@ def test_work_model_counts_the_definitions():
     # one query per sequence at position kv_len - 1: it scores every key of its cache
     assert w["indexer"]["flops"] == kv * 2 * spec.H_I * spec.d_I
     # e4m3 key (128 B) + fp32 scale per key, the query block and weights, one fp32 score per pair
-    assert w["indexer"]["bytes"] == kv * (spec.d_I + 4) + spec.T * (spec.H_I * spec.d_I * 2 + spec.H_I * 4) + kv * 4
+    # and one fp32 part maximum per 8 keys
+    parts = sum((n + 7) // 8 for n in spec.kv_lens)
+    assert w["indexer"]["bytes"] == (kv * (spec.d_I + 4) + spec.T * (spec.H_I * spec.d_I * 2 + spec.H_I * 4)
+                                     + kv * 4 + parts * 4)
     # every decode row here is longer than k: k selected rows per query
     assert all(n > spec.topk for n in spec.kv_lens)
     rows = spec.T * spec.topk
     assert w["attention"]["flops"] == rows * 2 * spec.H * (spec.d_qk + spec.d_v)
     assert w["attention"]["bytes"] == (rows * spec.d_qk * 2 + spec.T * (spec.H * spec.d_qk * 2 + spec.H * spec.d_v * 2
                                        + spec.H * 4) + spec.T * spec.topk * 4)
-    assert w["topk"]["bytes"] == kv * 4 + spec.T * spec.topk * 4
+    # top-k: the part maxima, the k parts of 8 scores that hold the selection, k indices out
+    assert w["topk"]["bytes"] == parts * 4 + spec.T * 8 * spec.topk * 4 + spec.T * spec.topk * 4
 
 
 def test_work_model_prefill_counts_causal_pairs():

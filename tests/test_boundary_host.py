@@ -70,12 +70,14 @@ def varlen(cu_q, cu_k):
     return v
 
 
-def scores_call(dsa, v, q_begin=0, q_end=None, ld=None, h=64, d=128, kd=0, ptrs=None, kscale=FAKE):
+def scores_call(dsa, v, q_begin=0, q_end=None, ld=None, h=64, d=128, kd=0, ptrs=None, kscale=FAKE, pm=None,
+                ld_pm=0, qscale=None):
     lib = dsa.library()
     q_end = v.cu_q_host[v.batch] if q_end is None else q_end
     ld = 1024 if ld is None else ld
     p = ptrs or fake(4)
-    return lib.dsa_indexer_scores(p[0], p[1], p[2], kscale, kd, v, h, d, q_begin, q_end, p[3], ld, None)
+    return lib.dsa_indexer_scores(p[0], qscale, p[1], p[2], kscale, kd, v, h, d, q_begin, q_end, p[3], ld, pm, ld_pm,
+                                  None)
 
 
 @host_only
@@ -96,6 +98,12 @@ def test_indexer_argument_validation(dsa):
     assert scores_call(dsa, ok, kd=7) == INV
     assert scores_call(dsa, ok, h=32) == UNS
     assert scores_call(dsa, ok, h=4, d=32, kd=1) == UNS                       # tiny shape is bf16 only
+    assert scores_call(dsa, ok, pm=FAKE, ld_pm=36) == INV                     # part maxima: ld < ceil(290 / 8)
+    assert scores_call(dsa, ok, pm=FAKE, ld_pm=38) == INV                     # ld % 4
+    assert scores_call(dsa, ok, pm=FAKE + 8, ld_pm=40) == INV                 # misaligned
+    assert scores_call(dsa, ok, qscale=FAKE, kd=0) == INV                      # FP8 queries need e4m3 keys
+    assert scores_call(dsa, ok, qscale=FAKE + 2, kd=1) == INV                  # misaligned scales
+    assert scores_call(dsa, ok, qscale=FAKE, kd=1, h=4, d=32) == UNS          # FP8 indexer: released shape only
 
 
 @host_only
@@ -103,10 +111,10 @@ def test_topk_and_attention_validation(dsa):
     lib = dsa.library()
     INV, UNS = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED
     v = varlen([0, 4], [0, 100])
-    assert lib.dsa_topk(FAKE, 100, v, 0, 4, 0, FAKE, None) == INV
-    assert lib.dsa_topk(FAKE, 100, v, 0, 4, 2049, FAKE, None) == INV
-    assert lib.dsa_topk(FAKE, 96, v, 0, 4, 16, FAKE, None) == INV
-    assert lib.dsa_topk(0, 100, v, 0, 4, 16, FAKE, None) == INV
+    assert lib.dsa_topk(FAKE, 100, None, 0, v, 0, 4, 0, FAKE, None) == INV
+    assert lib.dsa_topk(FAKE, 100, None, 0, v, 0, 4, 2049, FAKE, None) == INV
+    assert lib.dsa_topk(FAKE, 96, None, 0, v, 0, 4, 16, FAKE, None) == INV
+    assert lib.dsa_topk(0, 100, None, 0, v, 0, 4, 16, FAKE, None) == INV
     args = dict(topk=64, h=128, dqk=576, dv=512, scale=0.07)
 
     def mla(**kw):
@@ -128,13 +136,15 @@ def test_forward_workspace_contract(dsa):
     ld = 292                       # longest kv_len 291, rounded up to a multiple of 4
     need = lib.dsa_forward_workspace_size(v, 16, 0)
     al = lambda x: (x + 255) // 256 * 256
-    assert need == al(5 * ld * 4) + al(5 * 16 * 4)
-    assert lib.dsa_forward_workspace_size(v, 16, 2) == al(2 * ld * 4) + al(2 * 16 * 4)
+    ld_pm = (ld // 8 + 1 + 3) // 4 * 4         # one part maximum per 8 keys, rows of a multiple of 4
+    assert ld_pm == dsa.part_max_ld(ld) == 40
+    assert need == al(5 * ld * 4) + al(5 * ld_pm * 4) + al(5 * 16 * 4)
+    assert lib.dsa_forward_workspace_size(v, 16, 2) == al(2 * ld * 4) + al(2 * ld_pm * 4) + al(2 * 16 * 4)
     assert lib.dsa_forward_workspace_size(v, 0, 0) == 0
     assert lib.dsa_forward_workspace_size(varlen([0, 3], [0, 2]), 16, 0) == 0
 
     def fwd(ws, ws_bytes, topk=16, h_i=64, d_i=128):
-        return lib.dsa_forward(FAKE, FAKE, FAKE, None, 0, FAKE, FAKE, v, h_i, d_i, topk, 128, 576, 512,
+        return lib.dsa_forward(FAKE, None, FAKE, FAKE, None, 0, FAKE, FAKE, v, h_i, d_i, topk, 128, 576, 512,
                                ctypes.c_float(0.07), 0, FAKE, FAKE, None, ws, ws_bytes, None)
     assert fwd(None, 0) == dsa.DSA_ERR_WORKSPACE
     assert fwd(FAKE, need - 1) == dsa.DSA_ERR_WORKSPACE
@@ -148,7 +158,7 @@ def test_injected_faults_are_reported_without_launching(dsa, monkeypatch):
     v = varlen([0, 3], [0, 10])
     monkeypatch.setenv("DSA_INJECT_FAULT", "cuda")
     assert scores_call(dsa, v) == dsa.DSA_ERR_CUDA
-    assert lib.dsa_topk(FAKE, 16, v, 0, 3, 4, FAKE, None) == dsa.DSA_ERR_CUDA
+    assert lib.dsa_topk(FAKE, 16, None, 0, v, 0, 3, 4, FAKE, None) == dsa.DSA_ERR_CUDA
     monkeypatch.setenv("DSA_INJECT_FAULT", "timeout")
     assert scores_call(dsa, v) == dsa.DSA_ERR_DEVICE_TIMEOUT
 
@@ -171,16 +181,16 @@ def test_layouts_beyond_the_launch_limits_are_rejected_before_any_launch(dsa):
     lib = dsa.library()
     f = ctypes.c_float(0.07)
     long_row = varlen([0, 1], [0, 2_000_000])           # past the top-k row limit
-    assert lib.dsa_topk(FAKE, 2_000_000, long_row, 0, 1, 2048, FAKE, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_topk(FAKE, 2_000_000, None, 0, long_row, 0, 1, 2048, FAKE, None) == dsa.DSA_ERR_UNSUPPORTED
     need = lib.dsa_forward_workspace_size(long_row, 2048, 0)
     assert need > 0
-    assert lib.dsa_forward(FAKE, FAKE, FAKE, None, 0, FAKE, FAKE, long_row, 64, 128, 2048, 128, 576, 512, f, 0,
+    assert lib.dsa_forward(FAKE, None, FAKE, FAKE, None, 0, FAKE, FAKE, long_row, 64, 128, 2048, 128, 576, 512, f, 0,
                            FAKE, FAKE, None, FAKE, need, None) == dsa.DSA_ERR_UNSUPPORTED
-    assert lib.dsa_forward_static_scratch(FAKE, FAKE, FAKE, None, 0, FAKE, FAKE, long_row, 64, 128, 2048, 128,
+    assert lib.dsa_forward_static_scratch(FAKE, None, FAKE, FAKE, None, 0, FAKE, FAKE, long_row, 64, 128, 2048, 128,
                                           576, 512, f, FAKE, FAKE, None, None) == dsa.DSA_ERR_UNSUPPORTED
     kv = (dsa.DSA_STATIC_SCRATCH_BYTES // 4) + 1000     # one row of scores alone exceeds the array
     huge = varlen([0, 1], [0, kv])
-    assert lib.dsa_forward_static_scratch(FAKE, FAKE, FAKE, None, 0, FAKE, FAKE, huge, 64, 128, 2048, 128, 576,
+    assert lib.dsa_forward_static_scratch(FAKE, None, FAKE, FAKE, None, 0, FAKE, FAKE, huge, 64, 128, 2048, 128, 576,
                                           512, f, FAKE, FAKE, None, None) == dsa.DSA_ERR_WORKSPACE
 
 
@@ -189,3 +199,12 @@ def test_self_test_arguments(dsa):
     lib = dsa.library()
     assert lib.dsa_debug_wait_selftest(0, None) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_debug_wait_selftest(3_000_000_000, None) == dsa.DSA_ERR_INVALID_ARG
+
+
+@host_only
+def test_fp8_quantize_arguments(dsa):
+    lib = dsa.library()
+    assert lib.dsa_hadamard_quantize_fp8(FAKE, -1, FAKE, FAKE, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_hadamard_quantize_fp8(FAKE, 0, FAKE, FAKE, None) == dsa.DSA_OK          # nothing to do
+    assert lib.dsa_hadamard_quantize_fp8(FAKE + 8, 4, FAKE, FAKE, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_hadamard_quantize_fp8(FAKE, 4, FAKE, FAKE + 2, None) == dsa.DSA_ERR_INVALID_ARG

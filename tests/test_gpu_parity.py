@@ -53,11 +53,27 @@ TOPK_CASES = [
     ((3,), (9000,), 2048, 0),           # every score equal: the lowest indices win
     ((1, 1), (200000, 300000), 2048, None),   # grouped part maxima; a row past the bitmap
     ((2,), (100000,), 64, 40),          # small k on a long row, ties
+    ((1, 1), (40000, 16390), 2048, 0),  # all equal on rows with >= k parts: candidate overflow
+    ((1, 1, 1), (20472, 20480, 20489), 2048, None),   # just below and at 1.25 k parts; a ragged last part
+    ((1,), (262144,), 2048, 2),         # the longest row of the bitmap, heavy ties; parts grouped by 2
 ]
 
 
+def host_part_max(sc, pos, ld_pm):
+    """Part maxima as the indexer writes them: max over keys 8p .. 8p+7 that are <= pos."""
+    pm = np.full((sc.shape[0], ld_pm), np.nan, dtype=np.float32)
+    for r, p_ in enumerate(pos):
+        n = p_ + 1
+        P = (n + 7) // 8
+        row = np.full(P * 8, -np.inf, dtype=np.float32)
+        row[:n] = sc[r, :n]
+        pm[r, :P] = row.reshape(P, 8).max(axis=1)
+    return pm
+
+
+@pytest.mark.parametrize("use_pm", [False, True], ids=["scores", "part-max"])
 @pytest.mark.parametrize("case", TOPK_CASES, ids=[f"case{i}" for i in range(len(TOPK_CASES))])
-def test_topk_bit_exact_against_oracle(dsa, oracle_lib, case):
+def test_topk_bit_exact_against_oracle(dsa, oracle_lib, case, use_pm):
     q_lens, kv_lens, k, levels = case
     cu_q, cu_k = di.cu_seqlens(q_lens), di.cu_seqlens(kv_lens)
     T = sum(q_lens)
@@ -73,10 +89,13 @@ def test_topk_bit_exact_against_oracle(dsa, oracle_lib, case):
         sc[r, p_ + 1:] = 1e30                        # never read: beyond the diagonal
     v = dsa.Varlen(cu_q, cu_k, "cuda")
     sc_gpu = torch.from_numpy(sc).cuda()
+    pm = None
+    if use_pm:
+        pm = torch.from_numpy(host_part_max(sc, pos, dsa.part_max_ld(ld))).cuda()
     idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
-    dsa.dsa_topk(sc_gpu, v, 0, T, k, idx)
+    dsa.dsa_topk(sc_gpu, v, 0, T, k, idx, part_max=pm)
     idx2 = torch.empty_like(idx)
-    dsa.dsa_topk(sc_gpu, v, 0, T, k, idx2)
+    dsa.dsa_topk(sc_gpu, v, 0, T, k, idx2, part_max=pm)
     torch.cuda.synchronize()
     assert dsa.dsa_device_error() == 0
     assert torch.equal(idx, idx2), "top-k must be deterministic"
@@ -143,6 +162,19 @@ def test_indexer_released_shape(dsa, oracle_lib, kfp8, q_lens, kv_lens):
     ref = oracle_lib.indexer_scores(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"], d["k_scale"], ld=ld)
     pos = P.row_positions(d["cu_q"], d["cu_k"])
     P.assert_scores_close(got, ref, pos)
+    # the part maxima written beside the scores: exact maxima of the GPU's own scores
+    pm = torch.full((spec.T, dsa.part_max_ld(ld)), float("nan"), dtype=torch.float32, device="cuda")
+    again = torch.full((spec.T, ld), float("nan"), dtype=torch.float32, device="cuda")
+    dsa.dsa_indexer_scores(dd["q_idx"], dd["w"], dd["k_idx"], dd["k_scale"], v, 0, spec.T, again, part_max=pm)
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_error() == 0
+    again = again.cpu().numpy()
+    want = host_part_max(again, pos, pm.shape[1])
+    got_pm = pm.cpu().numpy()
+    for r, p_ in enumerate(pos):
+        assert np.array_equal(again[r, : p_ + 1], got[r, : p_ + 1]), "scores must not depend on part_max"
+        n_parts = (p_ + 1 + 7) // 8
+        assert np.array_equal(got_pm[r, :n_parts], want[r, :n_parts]), f"row {r}: part maxima"
     # a sub-range of rows (chunk-relative output) gives the same values
     q0, q1 = spec.T // 3, spec.T
     part = gpu_scores(dsa, dd, v, q0, q1, ld).cpu().numpy()

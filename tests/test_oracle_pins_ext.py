@@ -33,6 +33,11 @@ def test_hadamard_is_the_normalised_sylvester_matrix(oracle_lib, d):
     np.testing.assert_allclose(oracle_lib.hadamard(oracle_lib.hadamard(x)), x, rtol=0, atol=1e-12)
     # the unit vectors map to the matrix columns
     np.testing.assert_allclose(oracle_lib.hadamard(np.eye(d)), sylvester(d).T / np.sqrt(d), atol=1e-15)
+    # unnormalised: the +-1 matrix itself, exactly, and (Hq).(Hk) = d (q.k)
+    assert np.array_equal(oracle_lib.hadamard(np.eye(d), normalize=False), sylvester(d).T)
+    q, k = x[0], x[1]
+    hq, hk = oracle_lib.hadamard(q[None], normalize=False)[0], oracle_lib.hadamard(k[None], normalize=False)[0]
+    assert abs(hq @ hk - d * (q @ k)) <= 1e-11 * d * (np.abs(q) @ np.abs(k))
 
 
 def test_hadamard_rejects_lengths_that_are_not_powers_of_two(oracle_lib):
