@@ -87,6 +87,11 @@ def _load():
             lib.oracle_up_proj.restype = ctypes.c_int
             lib.oracle_up_proj.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _F64P,
                                            ctypes.c_int, vp, _F64P]
+            lib.oracle_paged_rows.restype = ctypes.c_int
+            lib.oracle_paged_rows.argtypes = [ctypes.c_int, _I32P, _I32P, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
+            lib.oracle_quant_e4m3_amax.restype = ctypes.c_int
+            lib.oracle_quant_e4m3_amax.argtypes = [ctypes.c_int64, ctypes.c_int, _F64P, vp, _F32P]
             for name in ("oracle_sparse_mla", "oracle_dense_mla_masked"):
                 fn = getattr(lib, name)
                 fn.restype = ctypes.c_int
@@ -334,6 +339,78 @@ def up_proj(o, w_uv):
                               _ptr(y, _F64P)) != 0:
         raise ValueError("oracle_up_proj rejected its arguments")
     return y
+
+
+def paged_rows(cu_k, block_table=None, page_size=0, n_pages=0):
+    """Cache row of every entry, in packed order: rows[cu_k[b] + s] for entry s
+    of sequence b (int64; -1 where the block table has no valid page).
+    block_table: None (packed caches) or int32 [B, pages_per_seq]."""
+    ck = _i32(cu_k)
+    B = ck.shape[0] - 1
+    rows = np.empty(int(ck[-1]), dtype=np.int64)
+    bt = None if block_table is None else _i32(block_table)
+    pps = 0 if bt is None else bt.shape[1]
+    if _load().oracle_paged_rows(B, _ptr(ck, _I32P), None if bt is None else _ptr(bt, _I32P), page_size, pps,
+                                 n_pages, rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))) != 0:
+        raise ValueError("oracle_paged_rows rejected its arguments")
+    return rows
+
+
+def quant_e4m3_amax(x):
+    """Per-vector (last axis) e4m3 quantization with scale amax / 448 in
+    float32: (bytes uint8 [..., d], scale float32 [...])."""
+    xa = _f64(x)
+    d = xa.shape[-1]
+    n = xa.size // d
+    q = np.empty(xa.shape, dtype=np.uint8)
+    sc = np.empty(xa.shape[:-1], dtype=np.float32)
+    if _load().oracle_quant_e4m3_amax(n, d, _ptr(xa, _F64P), q.ctypes.data_as(ctypes.c_void_p),
+                                      _ptr(sc, _F32P)) != 0:
+        raise ValueError("oracle_quant_e4m3_amax rejected its arguments")
+    return q, sc
+
+
+KQ_BF16, KQ_E4M3_AMAX, KQ_E4M3_HADAMARD = 0, 1, 2
+
+
+def cache_append(cu_q, cu_k, latent_new=None, kidx_new=None, k_quant=KQ_BF16, rope_freqs=None, d_v=None,
+                 block_table=None, page_size=0, n_pages=0):
+    """What appending a step's new tokens writes into the caches.
+
+    The new tokens are the step's query rows: row t is entry pos(t) of its
+    sequence (the lengths in cu_k already count it).  Returns a dict with
+    rows (int64 [T], the cache row of each new token, -1 if unmapped),
+    latent (float64 [T, d_qk]: the latent row, its columns from d_v on
+    rotated by rope_freqs at pos(t) when a table is given), and the index-key
+    row: k (float64 [T, d_I] values, k_quant KQ_BF16) or k (uint8 bytes) with
+    k_scale (float32 [T]) for the two e4m3 forms (amax / 448 scale, or the
+    Hadamard rotation with a power-of-two scale)."""
+    cq, ck = _i32(cu_q), _i32(cu_k)
+    T = int(cq[-1])
+    pos = np.empty(T, dtype=np.int64)
+    packed = np.empty(T, dtype=np.int64)
+    for b in range(cq.shape[0] - 1):
+        q_len, kv_len = int(cq[b + 1] - cq[b]), int(ck[b + 1] - ck[b])
+        for i in range(q_len):
+            pos[cq[b] + i] = kv_len - q_len + i
+            packed[cq[b] + i] = ck[b] + kv_len - q_len + i
+    out = dict(rows=paged_rows(ck, block_table, page_size, n_pages)[packed], pos=pos)
+    if latent_new is not None:
+        lat = _f64(latent_new).copy()
+        if rope_freqs is not None:
+            lat[:, d_v:] = rope(lat[:, d_v:], pos.astype(np.int32), rope_freqs)
+        out["latent"] = lat
+    if kidx_new is not None:
+        k = _f64(kidx_new)
+        if k_quant == KQ_BF16:
+            out["k"], out["k_scale"] = k.copy(), None
+        elif k_quant == KQ_E4M3_AMAX:
+            out["k"], out["k_scale"] = quant_e4m3_amax(k)
+        elif k_quant == KQ_E4M3_HADAMARD:
+            out["k"], out["k_scale"] = quant_e4m3_pow2(hadamard(k, normalize=False))
+        else:
+            raise ValueError("k_quant")
+    return out
 
 
 class use_library:

@@ -501,3 +501,56 @@ int oracle_up_proj(int64_t n_rows, int H, int d_c, int d_v, const double* o, int
   }
   return 0;
 }
+
+/* ===========================================================================
+ * Cache rows of a paged layout ("DeepSeek-V3.2" transformers doc, DSA: the
+ * indexer keeps its own per-token key cache beside the main cache, in a
+ * growing (DynamicIndexedLayer) or a preallocated (StaticIndexedLayer) cache
+ * layer).  Reading: a preallocated pool of n_pages pages of page_size rows
+ * each, shared by the index-key cache and the latent cache; entry s of
+ * sequence b sits in page block_table[b * pages_per_seq + s / page_size], at
+ * row s % page_size of that page.  With no block table the caches are packed:
+ * entry s of sequence b is row cu_k[b] + s.
+ * rows[cu_k[b] + s] receives the cache row of entry s of sequence b, or -1
+ * when its page entry is missing (s / page_size >= pages_per_seq) or outside
+ * [0, n_pages).
+ * =========================================================================*/
+int oracle_paged_rows(int B, const int32_t* cu_k, const int32_t* block_table, int page_size, int pages_per_seq,
+                      int64_t n_pages, int64_t* rows) {
+  if (B < 1 || cu_k[0] != 0) return -1;
+  if (block_table && (page_size < 1 || pages_per_seq < 1 || n_pages < 1)) return -1;
+  for (int b = 0; b < B; ++b) {
+    if (cu_k[b + 1] < cu_k[b]) return -1;
+    for (int64_t s = 0; s < cu_k[b + 1] - cu_k[b]; ++s) {
+      int64_t r = cu_k[b] + s;
+      if (block_table) {
+        const int64_t j = s / page_size;
+        const int64_t page = j < pages_per_seq ? block_table[(int64_t)b * pages_per_seq + j] : -1;
+        r = (page >= 0 && page < n_pages) ? page * page_size + s % page_size : -1;
+      }
+      rows[cu_k[b] + s] = r;
+    }
+  }
+  return 0;
+}
+
+/* e4m3 with one float32 scale per vector, scale = amax / 448 rounded to
+ * float32 (448: the largest finite e4m3 magnitude; scale 1 for a zero
+ * vector); byte i = the e4m3 value nearest (ties to even) to x_i / scale, the
+ * quotient taken in float32 (x_i and scale are float32 values; the double
+ * quotient of two float32 values rounded to float32 is the float32 quotient). */
+int oracle_quant_e4m3_amax(int64_t n_vec, int d, const double* x, uint8_t* q, float* scale) {
+  if (d < 1) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t v = 0; v < n_vec; ++v) {
+    double amax = 0.0;
+    for (int i = 0; i < d; ++i) amax = fmax(amax, fabs(x[v * d + i]));
+    const float s = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+    scale[v] = s;
+    for (int i = 0; i < d; ++i) {
+      const float qf = (float)((double)(float)x[v * d + i] / (double)s);
+      q[v * d + i] = oracle_double_to_e4m3((double)qf);
+    }
+  }
+  return 0;
+}

@@ -50,10 +50,17 @@ MUTANTS = [
     ("pair halves swapped", "const double re = x[v * d + 2 * i], im = x[v * d + 2 * i + 1];",
      "const double re = x[v * d + 2 * i + 1], im = x[v * d + 2 * i];"),
     # up-projection
+    # paged layout and append quantization
+    ("row inside the page taken from the wrong end", "r = (page >= 0 && page < n_pages) ? page * page_size + s % page_size : -1;",
+     "r = (page >= 0 && page < n_pages) ? page * page_size + (page_size - 1 - s % page_size) : -1;"),
+    ("page table row stride dropped", "block_table[(int64_t)b * pages_per_seq + j]", "block_table[j]"),
+    ("pages beyond the pool accepted", "r = (page >= 0 && page < n_pages) ?", "r = (page >= 0) ?"),
+    ("amax scale of the wrong format maximum", "(float)(amax / 448.0)", "(float)(amax / 240.0)"),
     ("up-projection matrix transposed", "load_elem(w_kind, w, ((int64_t)h * d_c + c) * d_v + e, NULL, 0);",
      "load_elem(w_kind, w, ((int64_t)h * d_v + e) * d_c + c, NULL, 0);"),
 ]
 
+from tests import test_oracle_pins_cache as pins_cache
 from tests import test_oracle_pins_ext as pins_ext
 
 PIN_TESTS = [
@@ -82,9 +89,19 @@ PIN_TESTS_EXT = [
     ("test_up_projection_matches_einsum_and_selects_with_a_unit_matrix", {}),
 ]
 
+PIN_TESTS_CACHE = [
+    ("test_paged_rows_worked_example", {}),
+    ("test_packed_layout_is_the_identity", {}),
+    ("test_paged_rows_agree_with_a_pool_filled_page_by_page", {}),
+    ("test_paged_rows_mark_missing_pages", {}),
+    ("test_amax_quantization_matches_float32_division_and_torch_cast", {}),
+    ("test_append_decode_rows_are_the_last_rows_and_rope_closed_forms", {}),
+    ("test_append_prefill_rows_and_paging", {}),
+]
+
 
 def _caught(lib_mod):
-    for module, tests in ((pins, PIN_TESTS), (pins_ext, PIN_TESTS_EXT)):
+    for module, tests in ((pins, PIN_TESTS), (pins_ext, PIN_TESTS_EXT), (pins_cache, PIN_TESTS_CACHE)):
         for name, kw in tests:
             try:
                 getattr(module, name)(lib_mod, **kw)
