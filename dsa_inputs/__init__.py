@@ -88,7 +88,7 @@ def normal(h: torch.Tensor) -> torch.Tensor:
 
 
 # tensor ids of the streams
-T_QIDX, T_W, T_KIDX, T_Q, T_LAT, T_LEN, T_DUP, T_DUPSRC = range(1, 9)
+T_QIDX, T_W, T_KIDX, T_Q, T_LAT, T_LEN, T_DUP, T_DUPSRC, T_WUV, T_O = range(1, 11)
 
 _CHUNK = 1 << 25  # elements per generation chunk (bounded temporaries)
 
@@ -281,3 +281,18 @@ def make_inputs(spec: Spec, device="cpu", seqs=None, tensors=ALL_TENSORS):
 def with_lengths(spec: Spec, q_lens, kv_lens, **kw) -> Spec:
     """A copy of `spec` with other sequence lengths (and optional overrides)."""
     return replace(spec, q_lens=tuple(q_lens), kv_lens=tuple(kv_lens), **kw)
+
+
+def make_w_uv(seed: int, H: int = 128, d_c: int = 512, d_v: int = 128, device="cpu"):
+    """Per-head value up-projection weights W_UV [H, d_c, d_v] bf16, normal
+    with standard deviation 1/sqrt(d_c) (random init: no trained weights)."""
+    w = torch.empty((H, d_c, d_v), dtype=torch.bfloat16, device=device)
+    _fill(w, seed, T_WUV, 0, "normal", std=1.0 / math.sqrt(d_c))
+    return w
+
+
+def make_latent_out(seed: int, n: int, H: int = 128, d_c: int = 512, device="cpu"):
+    """An attention output in latent space, o [n, H, d_c] bf16 (standard normal)."""
+    o = torch.empty((n, H, d_c), dtype=torch.bfloat16, device=device)
+    _fill(o, seed, T_O, 0, "normal")
+    return o

@@ -62,14 +62,36 @@ typedef enum {
                                scale per key: k = e4m3(byte) * k_scale[key] */
 } dsa_kidx_dtype;
 
-/* Packed sequence layout.  The device and host copies must hold the same
- * values: cu_q[0] = cu_k[0] = 0, non-decreasing, q_len_b <= kv_len_b. */
+/* Sequence layout.  The device and host copies must hold the same values:
+ * cu_q[0] = cu_k[0] = 0, non-decreasing, q_len_b <= kv_len_b.  kv_len_b =
+ * cu_k[b+1] - cu_k[b] is the number of cache entries of sequence b (its new
+ * tokens included).
+ *
+ * Caches ("DeepSeek-V3.2", transformers doc, DSA: the indexer's per-token key
+ * cache is kept beside the main cache, in a growing or a preallocated cache
+ * layer).  The index-key cache (with its scales) and the latent cache share
+ * one row layout:
+ *  - packed (block_table NULL; the page fields are then ignored): entry s of
+ *    sequence b is cache row cu_k[b] + s, and the caches hold cu_k[B] rows;
+ *  - paged: a pool of n_pages pages of page_size rows; entry s of sequence b
+ *    is row s % page_size of page block_table[b * pages_per_seq + s / page_size].
+ *    page_size is a power of two >= 64, pages_per_seq * page_size >= every kv_len,
+ *    n_pages * page_size <= 2^31 - 1, block_table 4-byte aligned (else
+ *    DSA_ERR_INVALID_ARG).  The table lives on the device and is not read by
+ *    the host: a page entry outside [0, n_pages) reads as zeros in the
+ *    indexer, makes the attention skip that entry and records device error
+ *    code 2 (see dsa_device_error); it never causes an access outside the
+ *    caches. */
 typedef struct {
   int32_t batch;              /* B >= 1 */
   const int32_t* cu_q;        /* device, [B+1]: query-row offsets */
-  const int32_t* cu_k;        /* device, [B+1]: key/cache-row offsets */
+  const int32_t* cu_k;        /* device, [B+1]: cache-entry offsets */
   const int32_t* cu_q_host;   /* host,   [B+1]: same values as cu_q */
   const int32_t* cu_k_host;   /* host,   [B+1]: same values as cu_k */
+  const int32_t* block_table; /* device, [B, pages_per_seq] page ids, or NULL (packed caches) */
+  int32_t page_size;          /* rows per page (paged): a power of two >= 64 */
+  int32_t pages_per_seq;      /* row stride of block_table (paged) */
+  int64_t n_pages;            /* pages in the pool (paged) */
 } dsa_varlen;
 
 /*
@@ -149,8 +171,19 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, const float* part_ma
  * are MLA's compressed vectors.  For query row t, head h, selected row s:
  *     z_s = scale * q[t,h,:d_qk] . latent[s,:d_qk]
  *     out[t,h,:] = sum_s softmax(z)_s * latent[s, :d_v],   lse[t,h] = log sum_s exp(z_s)
- * q         bf16 [T, n_heads, d_qk] global rows (RoPE part already applied)
+ * q         bf16 [T, n_heads, d_qk] global rows: per head the d_v-wide absorbed
+ *           query then the (d_qk - d_v)-wide RoPE part
  * latent    bf16 [sum kv, d_qk]: per token the 512-d latent then the 64-d RoPE key
+ *           (already rotated at its own position)
+ * rope_cs   NULL: q's RoPE part is used as given (already rotated).  Otherwise
+ *           fp32 [rope_max_pos, (d_qk - d_v) / 2, 2], 8-byte aligned: the
+ *           (cos, sin) of each position and rotation pair ("DeepSeek-V3.2-Exp"
+ *           token-ids page, released config: qk_rope_head_dim 64).  The
+ *           kernel rotates the RoPE part of every query row at its position
+ *           pos(t) while loading it: element pair (2i, 2i+1) of that part,
+ *           read as the complex number x_2i + i x_2i+1, is multiplied by
+ *           cos + i sin of entry [pos(t)][i] (fp32, rounded back to bf16).
+ *           rope_max_pos must be at least the longest kv length of the range.
  * idx       int32 [q_end - q_begin, topk] chunk-relative, sequence-local rows.
  *           Entries outside 0..pos(t) (including the -1 padding) are ignored.
  * out       bf16 [T, n_heads, d_v] global rows; lse fp32 [T, n_heads] (nullable).
@@ -163,6 +196,7 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, const float* part_ma
 dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t* idx,
                                dsa_varlen v, int64_t q_begin, int64_t q_end, int32_t topk,
                                int32_t n_heads, int32_t d_qk, int32_t d_v, float scale,
+                               const float* rope_cs, int64_t rope_max_pos,
                                void* out, float* lse, cudaStream_t stream);
 
 /*
@@ -183,6 +217,61 @@ dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t*
  * x and q 16-byte aligned.
  */
 dsa_status dsa_hadamard_quantize_fp8(const void* x, int64_t n, void* q, float* scale, cudaStream_t stream);
+
+/* How dsa_cache_append stores an index key. */
+typedef enum {
+  DSA_KQ_BF16 = 0,           /* bf16 copy (a DSA_KIDX_BF16 cache) */
+  DSA_KQ_E4M3_AMAX = 1,      /* e4m3, scale = amax / 448 in fp32 (1 for a zero key), byte = nearest e4m3
+                                (ties to even) to the fp32 quotient x / scale (a DSA_KIDX_FP8_E4M3 cache) */
+  DSA_KQ_E4M3_HADAMARD = 2   /* the Hadamard rotation and power-of-two scale of dsa_hadamard_quantize_fp8:
+                                the keys of the FP8 indexer (dsa_indexer_scores with q_scale) */
+} dsa_kidx_quant;
+
+/*
+ * Appends a step's new tokens to the caches (the update before scoring).
+ * Source: "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse
+ * Attention (DSA)": the indexer keeps its own per-token key cache beside the
+ * main cache and updates it every step (update_indexer), in a growing or a
+ * preallocated cache layer; "DeepSeek-V3.2-Exp" token-ids page, released
+ * config: kv_lora_rank 512, qk_rope_head_dim 64, index_head_dim 128.
+ * The new tokens are the step's query rows: global row t is entry pos(t) of
+ * its sequence (v's kv lengths already count the new tokens), stored at that
+ * entry's cache row (packed or paged, see dsa_varlen).
+ * latent_new   bf16 [T, d_qk] or NULL: the new latent rows; latent_cache bf16
+ *              [cache rows, d_qk] (NULL with latent_new NULL).  (d_qk, d_v) is
+ *              (576, 512) or (80, 64).
+ * rope_cs      NULL (latents stored as given), or fp32 [rope_max_pos,
+ *              (d_qk - d_v) / 2, 2] (cos, sin), 8-byte aligned: columns from
+ *              d_v on are rotated at pos(t) as dsa_sparse_mla_attn rotates
+ *              queries (fp32, rounded to bf16).  rope_max_pos >= longest kv.
+ * kidx_new     bf16 [T, idx_dim] or NULL: the new index keys; k_cache [cache
+ *              rows, idx_dim] bf16 (DSA_KQ_BF16, idx_dim 128 or 32) or e4m3
+ *              bytes (the two e4m3 forms, idx_dim 128) with k_scale fp32
+ *              [cache rows].
+ * Buffers 16-byte aligned (k_scale 4).  Entries whose page is missing are not
+ * written and record device error code 2.  Other cache rows are untouched.
+ */
+dsa_status dsa_cache_append(const void* latent_new, const void* kidx_new, dsa_varlen v, int32_t d_qk, int32_t d_v,
+                            int32_t idx_dim, const float* rope_cs, int64_t rope_max_pos, dsa_kidx_quant k_quant,
+                            void* latent_cache, void* k_cache, float* k_scale, cudaStream_t stream);
+
+/*
+ * Per-head value up-projection of the attention output (the end of step 3).
+ * Source: "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse
+ * Attention (DSA)": MLA, whose cached entries (the compressed latents) are
+ * shared by all heads, so the absorbed attention of dsa_sparse_mla_attn leaves
+ * each head's output in the 512-wide latent space; "DeepSeek-V3.2-Exp"
+ * token-ids page, released config: kv_lora_rank 512, v_head_dim 128,
+ * n_heads 128.  Each head h has its own W_UV[h] of [d_c, d_v]:
+ *     y[r, h, e] = sum_c o[r, h, c] * W_UV[h, c, e]
+ * o     bf16 [n_rows, n_heads, d_c] (the out of dsa_sparse_mla_attn)
+ * w_uv  bf16 [n_heads, d_c, d_v], row-major; y  bf16 [n_rows, n_heads, d_v]
+ * All three 16-byte aligned.  Released shape only (128, 512, 128), else
+ * DSA_ERR_UNSUPPORTED; n_rows <= 8,388,480.  Tensor cores, bf16 in, fp32
+ * accumulate, y rounded to bf16 (nearest even).  n_rows = 0 is a no-op.
+ */
+dsa_status dsa_mla_up_proj(const void* o, const void* w_uv, int64_t n_rows, int32_t n_heads, int32_t d_c,
+                           int32_t d_v, void* y, cudaStream_t stream);
 
 /*
  * Bytes of device workspace dsa_forward needs for this layout when it runs at
@@ -253,7 +342,10 @@ dsa_status dsa_forward_static_scratch(const void* q_idx, const float* q_scale, c
                                       cudaStream_t stream);
 
 /* Reads and clears the device error word of the current device (synchronises
- * `stream` first).  *code = 0 when no device-side wait gave up. */
+ * `stream` first).  *code = 0 when nothing was recorded.  Otherwise the low 8
+ * bits give the kind and bits 8.. the site: kind 1, a bounded device-side
+ * wait gave up (the kernel skipped its remaining work); kind 2, a paged cache
+ * entry that was needed had no valid page (that entry was skipped). */
 dsa_status dsa_device_error(int32_t* code, cudaStream_t stream);
 
 /* Diagnostics for profiling builds (compiled with -DDSA_PROFILE_WAITS): for

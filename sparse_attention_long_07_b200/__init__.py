@@ -38,6 +38,10 @@ class dsa_varlen(ctypes.Structure):
         ("cu_k", ctypes.c_void_p),
         ("cu_q_host", ctypes.POINTER(ctypes.c_int32)),
         ("cu_k_host", ctypes.POINTER(ctypes.c_int32)),
+        ("block_table", ctypes.c_void_p),
+        ("page_size", ctypes.c_int32),
+        ("pages_per_seq", ctypes.c_int32),
+        ("n_pages", ctypes.c_int64),
     ]
 
 
@@ -54,7 +58,8 @@ def _load():
     lib.dsa_indexer_scores.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, dsa_varlen, i32, i32, i64, i64, vp, i64,
                                        vp, i64, vp]
     lib.dsa_topk.argtypes = [vp, i64, vp, i64, dsa_varlen, i64, i64, i32, vp, vp]
-    lib.dsa_sparse_mla_attn.argtypes = [vp, vp, vp, dsa_varlen, i64, i64, i32, i32, i32, i32, f32, vp, vp, vp]
+    lib.dsa_sparse_mla_attn.argtypes = [vp, vp, vp, dsa_varlen, i64, i64, i32, i32, i32, i32, f32, vp, i64, vp, vp,
+                                        vp]
     lib.dsa_forward_workspace_size.argtypes = [dsa_varlen, i32, i64]
     lib.dsa_forward_workspace_size.restype = ctypes.c_size_t
     lib.dsa_forward.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, dsa_varlen, i32, i32, i32, i32, i32, i32,
@@ -71,6 +76,10 @@ def _load():
     lib.dsa_forward_static_scratch.restype = ctypes.c_int
     lib.dsa_hadamard_quantize_fp8.argtypes = [vp, i64, vp, vp, vp]
     lib.dsa_hadamard_quantize_fp8.restype = ctypes.c_int
+    lib.dsa_mla_up_proj.argtypes = [vp, vp, i64, i32, i32, i32, vp, vp]
+    lib.dsa_cache_append.argtypes = [vp, vp, dsa_varlen, i32, i32, i32, vp, i64, ctypes.c_int, vp, vp, vp, vp]
+    lib.dsa_cache_append.restype = ctypes.c_int
+    lib.dsa_mla_up_proj.restype = ctypes.c_int
     lib.dsa_debug_wait_selftest.argtypes = [i64, vp]
     lib.dsa_debug_wait_selftest.restype = ctypes.c_int
     for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward", "dsa_device_error"):
@@ -80,7 +89,8 @@ def _load():
 
 EXPORTED = ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_forward_workspace_size",
             "dsa_forward", "dsa_device_error", "dsa_status_string", "dsa_version", "dsa_debug_wait_profile",
-            "dsa_forward_static_scratch", "dsa_debug_wait_selftest", "dsa_hadamard_quantize_fp8")
+            "dsa_forward_static_scratch", "dsa_debug_wait_selftest", "dsa_hadamard_quantize_fp8",
+            "dsa_mla_up_proj", "dsa_cache_append")
 
 # bytes of the library's static scratch array (DSA_STATIC_SCRATCH_BYTES in include/dsa.h)
 DSA_STATIC_SCRATCH_BYTES = 32 << 20
@@ -94,13 +104,17 @@ def library():
 
 
 class Varlen:
-    """Packed sequence layout: cumulative query and key/cache row offsets.
+    """Sequence layout: cumulative query-row and cache-entry offsets, and
+    (optionally) the page table of paged caches.
 
     Keeps both the device copies the kernels read and the host copies the
-    library validates and plans launches with.
+    library validates and plans launches with.  block_table: int32 [B,
+    pages_per_seq] device tensor of page ids (None: packed caches, entry s of
+    sequence b at row cu_k[b] + s); page_size a power of two >= 64; n_pages
+    the pages of the pool the caches hold.
     """
 
-    def __init__(self, cu_q, cu_k, device=None):
+    def __init__(self, cu_q, cu_k, device=None, block_table=None, page_size=0, n_pages=0):
         cu_q = torch.as_tensor(cu_q, dtype=torch.int32).cpu().contiguous()
         cu_k = torch.as_tensor(cu_k, dtype=torch.int32).cpu().contiguous()
         self.cu_q_host, self.cu_k_host = cu_q, cu_k
@@ -113,11 +127,15 @@ class Varlen:
         self.S = int(cu_k[-1])
         kv = (cu_k[1:] - cu_k[:-1])
         self.max_kv = int(kv.max()) if kv.numel() else 0
+        self.block_table = None if block_table is None else block_table.contiguous()
+        self.page_size, self.n_pages = int(page_size), int(n_pages)
+        self.pages_per_seq = 0 if block_table is None else int(self.block_table.shape[1])
 
     def c(self) -> dsa_varlen:
         return dsa_varlen(self.batch, self.cu_q.data_ptr(), self.cu_k.data_ptr(),
                           ctypes.cast(self.cu_q_host.data_ptr(), ctypes.POINTER(ctypes.c_int32)),
-                          ctypes.cast(self.cu_k_host.data_ptr(), ctypes.POINTER(ctypes.c_int32)))
+                          ctypes.cast(self.cu_k_host.data_ptr(), ctypes.POINTER(ctypes.c_int32)),
+                          _ptr(self.block_table), self.page_size, self.pages_per_seq, self.n_pages)
 
 
 def _ptr(t):
@@ -181,13 +199,17 @@ def dsa_topk(scores, v: Varlen, q_begin, q_end, topk, idx, stream=None, part_max
 
 
 def dsa_sparse_mla_attn(q, latent, idx, v: Varlen, q_begin, q_end, scale, out, lse=None, d_v=None,
-                        stream=None):
+                        stream=None, rope=None):
     """MLA attention (absorbed MQA) over the selected rows; writes out/lse for
-    global rows [q_begin, q_end)."""
+    global rows [q_begin, q_end).  rope (optional): fp32 [max_pos, (d_qk -
+    d_v) / 2, 2] (cos, sin) table; the kernel then rotates q's RoPE part at
+    each row's position."""
     T, H, d_qk = q.shape
     d_v = out.shape[-1] if d_v is None else d_v
+    max_pos = 0 if rope is None else rope.shape[0]
     _check(_lib.dsa_sparse_mla_attn(_ptr(q), _ptr(latent), _ptr(idx), v.c(), q_begin, q_end, idx.shape[1], H,
-                                    d_qk, d_v, float(scale), _ptr(out), _ptr(lse), _stream(stream)),
+                                    d_qk, d_v, float(scale), _ptr(rope), max_pos, _ptr(out), _ptr(lse),
+                                    _stream(stream)),
            "dsa_sparse_mla_attn")
     return out, lse
 
@@ -203,6 +225,35 @@ def dsa_hadamard_quantize_fp8(x, q=None, scale=None, stream=None):
     _check(_lib.dsa_hadamard_quantize_fp8(_ptr(x), n, _ptr(q), _ptr(scale), _stream(stream)),
            "dsa_hadamard_quantize_fp8")
     return q, scale
+
+
+DSA_KQ_BF16, DSA_KQ_E4M3_AMAX, DSA_KQ_E4M3_HADAMARD = 0, 1, 2
+
+
+def dsa_cache_append(v: Varlen, latent_new=None, latent_cache=None, kidx_new=None, k_cache=None, k_scale=None,
+                     k_quant=DSA_KQ_BF16, rope=None, d_v=None, stream=None):
+    """Write the step's new tokens (its query rows, at positions pos(t)) into
+    the latent cache (optionally rotating its RoPE columns with the (cos, sin)
+    table `rope`) and the index-key cache (bf16 copy or one of the e4m3 forms)."""
+    d_qk = 0 if latent_new is None else latent_new.shape[-1]
+    if d_v is None:
+        d_v = {576: 512, 80: 64}.get(d_qk, 0)
+    idx_dim = 0 if kidx_new is None else kidx_new.shape[-1]
+    max_pos = 0 if rope is None else rope.shape[0]
+    _check(_lib.dsa_cache_append(_ptr(latent_new), _ptr(kidx_new), v.c(), d_qk, d_v, idx_dim, _ptr(rope), max_pos,
+                                 int(k_quant), _ptr(latent_cache), _ptr(k_cache), _ptr(k_scale), _stream(stream)),
+           "dsa_cache_append")
+
+
+def dsa_mla_up_proj(o, w_uv, y=None, stream=None):
+    """Per-head up-projection y[r, h, :] = o[r, h, :] @ w_uv[h] (o bf16
+    [n, H, d_c], w_uv bf16 [H, d_c, d_v]); returns y bf16 [n, H, d_v]."""
+    n, H, d_c = o.shape
+    d_v = w_uv.shape[-1]
+    if y is None:
+        y = torch.empty((n, H, d_v), dtype=torch.bfloat16, device=o.device)
+    _check(_lib.dsa_mla_up_proj(_ptr(o), _ptr(w_uv), n, H, d_c, d_v, _ptr(y), _stream(stream)), "dsa_mla_up_proj")
+    return y
 
 
 def dsa_forward_workspace_size(v: Varlen, topk: int, q_chunk: int = 0) -> int:

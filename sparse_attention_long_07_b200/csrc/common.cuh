@@ -10,6 +10,32 @@ namespace dsa {
 // row (eight consecutive keys are eight consecutive lanes of one epilogue warp).
 constexpr int PART = 8;
 
+// Where the caches keep entry s of sequence b.  Packed caches (no block
+// table): row k_base + s, k_base = cu_k[b].  Paged caches: a pool of n_pages
+// pages of page_size rows shared by the index-key and latent caches; entry s
+// sits at row s % page_size of page block_table[b * pages_per_seq +
+// s / page_size] ("DeepSeek-V3.2" transformers doc, DSA: the indexer's key
+// cache lives beside the main cache, growing or preallocated).  page_size is
+// a power of two of at least 64, so a 64-row span starting at a multiple of
+// 64 never crosses a page.
+struct PageMap {
+  const int32_t* block_table;   // [B, pages_per_seq] or null (packed)
+  int page_shift;               // log2(page_size)
+  int pages_per_seq;
+  int n_pages;
+
+  __device__ __forceinline__ bool paged() const { return block_table != nullptr; }
+  // Cache row of entry s (s >= 0) of sequence b, or -1 if its page is missing.
+  __device__ __forceinline__ int row(int b, int k_base, int s) const {
+    if (block_table == nullptr) return k_base + s;
+    const int j = s >> page_shift;
+    const int page = j < pages_per_seq ? __ldg(block_table + static_cast<int64_t>(b) * pages_per_seq + j) : -1;
+    return (static_cast<unsigned>(page) < static_cast<unsigned>(n_pages))
+               ? (page << page_shift) + (s & ((1 << page_shift) - 1))
+               : -1;
+  }
+};
+
 // Where global query row t sits: its sequence, absolute position and the
 // sequence's key range.  Sequence b owns query rows [cu_q[b], cu_q[b+1]) and
 // key rows [cu_k[b], cu_k[b+1]); its q_len new queries are its last tokens.

@@ -17,10 +17,12 @@
 #include <mutex>
 
 #include "dsa.h"
+#include "cache.cuh"
 #include "fp8.cuh"
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
+#include "up_proj.cuh"
 
 namespace {
 
@@ -28,18 +30,28 @@ using dsa::IndexerCfg;
 using dsa::MlaCfg;
 
 // ----------------------------------------------------------------------------
-// Validation of the packed layout (host copies only)
+// Validation of the sequence and cache layout (host copies only)
 // ----------------------------------------------------------------------------
 struct Layout {
   int B = 0;
   int64_t T = 0;         // total query rows
-  int64_t S = 0;         // total key rows
+  int64_t S = 0;         // cache rows (packed: cu_k[B]; paged: n_pages * page_size)
   int max_kv = 0;        // longest kv_len over sequences with a row in [q_begin, q_end)
   int max_q_rows = 0;    // most rows of one sequence inside [q_begin, q_end)
   int max_tiles = 0;     // most 128-key tiles one query row of the range needs
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dsa::PageMap page_map(const dsa_varlen& v) {
+  dsa::PageMap m;
+  m.block_table = v.block_table;
+  m.page_shift = 0;
+  while (v.block_table && (1 << m.page_shift) < v.page_size) ++m.page_shift;
+  m.pages_per_seq = v.block_table ? v.pages_per_seq : 0;
+  m.n_pages = v.block_table ? static_cast<int>(v.n_pages) : 0;
+  return m;
+}
 
 dsa_status check_varlen(const dsa_varlen& v, int64_t q_begin, int64_t q_end, Layout* out) {
   if (v.batch < 1 || !v.cu_q || !v.cu_k || !v.cu_q_host || !v.cu_k_host) return DSA_ERR_INVALID_ARG;
@@ -53,6 +65,16 @@ dsa_status check_varlen(const dsa_varlen& v, int64_t q_begin, int64_t q_end, Lay
   }
   L.T = v.cu_q_host[v.batch];
   L.S = v.cu_k_host[v.batch];
+  if (v.block_table) {
+    if ((reinterpret_cast<uintptr_t>(v.block_table) & 3u) || v.page_size < 64 || (v.page_size & (v.page_size - 1)) ||
+        v.pages_per_seq < 1 || v.n_pages < 1 || v.n_pages > 0x7FFFFFFF / v.page_size)
+      return DSA_ERR_INVALID_ARG;
+    for (int b = 0; b < v.batch; ++b) {
+      const int64_t kl = static_cast<int64_t>(v.cu_k_host[b + 1]) - v.cu_k_host[b];
+      if (kl > static_cast<int64_t>(v.pages_per_seq) * v.page_size) return DSA_ERR_INVALID_ARG;
+    }
+    L.S = v.n_pages * v.page_size;
+  }
   if (q_begin < 0 || q_end < q_begin || q_end > L.T) return DSA_ERR_INVALID_ARG;
   for (int b = 0; b < v.batch; ++b) {
     const int64_t lo = std::max<int64_t>(v.cu_q_host[b], q_begin);
@@ -117,6 +139,19 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D tiled map: dims (d0, d1, d2) innermost first, byte strides of dims 1 and 2.
+bool make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, const uint64_t dims[3],
+                 const uint64_t strides[2], const uint32_t box[3], CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t st[2] = {strides[0], strides[1]};
+  const cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(map, dt, 3, const_cast<void*>(base), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Per-device state.  Kernel attributes (the dynamic shared-memory limit) and
 // the SM count belong to a device, so they are kept per device ordinal and set
 // up the first time a kernel runs on that device.
@@ -171,13 +206,14 @@ dsa_status launch_indexer(const void* q_idx, const float* q_scale, const float* 
                 static_cast<uint64_t>(L.T) * C::H_I, C::D_I * C::ELEM, C::ATOM_ELEMS, C::N,
                 C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return DSA_ERR_CUDA;
+  const uint32_t box_rows = v.block_table ? 64u : static_cast<uint32_t>(C::BK);   // paged: 64-row boxes
   if (C::KFP8) {
     if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_idx, C::D_I, static_cast<uint64_t>(L.S),
-                  C::D_I, C::D_I, C::BK, CU_TENSOR_MAP_SWIZZLE_128B))
+                  C::D_I, C::D_I, box_rows, CU_TENSOR_MAP_SWIZZLE_128B))
       return DSA_ERR_CUDA;
   } else {
     if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k_idx, C::D_I,
-                  static_cast<uint64_t>(L.S), C::D_I * 2, C::ATOM_ELEMS, C::BK,
+                  static_cast<uint64_t>(L.S), C::D_I * 2, C::ATOM_ELEMS, box_rows,
                   C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
       return DSA_ERR_CUDA;
   }
@@ -187,6 +223,7 @@ dsa_status launch_indexer(const void* q_idx, const float* q_scale, const float* 
   p.w = w;
   p.q_scale = q_scale;
   p.k_scale = k_scale;
+  p.pages = page_map(v);
   p.cu_q = v.cu_q;
   p.cu_k = v.cu_k;
   p.B = v.batch;
@@ -229,13 +266,14 @@ dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const vo
                 C::D_I * 2, C::ATOM_ELEMS, C::N, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_idx, C::D_I, static_cast<uint64_t>(L.S), C::D_I, C::D_I,
-                C::BK, CU_TENSOR_MAP_SWIZZLE_128B))
+                v.block_table ? 64u : static_cast<uint32_t>(C::BK), CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   if (ensure_smem<dsa::indexer_persistent_kernel<C>>(C::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
   dsa::IndexerParams p;
   p.w = w;
   p.q_scale = nullptr;
   p.k_scale = k_scale;
+  p.pages = page_map(v);
   p.cu_q = v.cu_q;
   p.cu_k = v.cu_k;
   p.B = v.batch;
@@ -254,7 +292,7 @@ dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const vo
 template <class C>
 dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, const dsa_varlen& v,
                       const Layout& L, int64_t q_begin, int64_t q_end, int topk, float scale,
-                      void* out, float* lse, cudaStream_t stream) {
+                      const float* rope, void* out, float* lse, cudaStream_t stream) {
   CUtensorMap tm_lat;
   const CUtensorMapSwizzle swz = C::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                  : (C::SWB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
@@ -268,10 +306,12 @@ dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, con
   p.idx = idx;
   p.cu_q = v.cu_q;
   p.cu_k = v.cu_k;
+  p.pages = page_map(v);
   p.B = v.batch;
   p.q_begin = q_begin;
   p.topk = topk;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.rope = reinterpret_cast<const float2*>(rope);
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   const int64_t rows = q_end - q_begin;
@@ -412,11 +452,11 @@ dsa_status run_topk(const float* scores, int64_t ld, const float* part_max, int6
 
 dsa_status run_mla(const void* q, const void* latent, const int32_t* idx, const dsa_varlen& v,
                    const Layout& L, int64_t q_begin, int64_t q_end, int topk, int h, int dqk, int dv,
-                   float scale, void* out, float* lse, cudaStream_t stream) {
+                   float scale, const float* rope, void* out, float* lse, cudaStream_t stream) {
   if (is_tiny_mla(h, dqk, dv))
-    return launch_mla<MlaCfg<4, 80, 64, 1, 32>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, out,
+    return launch_mla<MlaCfg<4, 80, 64, 1, 32>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, rope, out,
                                                 lse, stream);
-  return launch_mla<MlaCfg<128, 576, 512, 2, 128>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, out,
+  return launch_mla<MlaCfg<128, 576, 512, 2, 128>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, rope, out,
                                                    lse, stream);
 }
 
@@ -476,6 +516,7 @@ dsa_status dsa_topk(const float* scores, int64_t ld_scores, const float* part_ma
 dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t* idx,
                                dsa_varlen v, int64_t q_begin, int64_t q_end, int32_t topk,
                                int32_t n_heads, int32_t d_qk, int32_t d_v, float scale,
+                               const float* rope_cs, int64_t rope_max_pos,
                                void* out, float* lse, cudaStream_t stream) {
   Layout L;
   dsa_status st = check_varlen(v, q_begin, q_end, &L);
@@ -483,9 +524,12 @@ dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t*
   if (!idx) return DSA_ERR_INVALID_ARG;
   st = check_mla_args(q, latent, idx, topk, n_heads, d_qk, d_v, scale, out, lse);
   if (st != DSA_OK) return st;
+  // every row's position is below its sequence's kv length
+  if (rope_cs && ((reinterpret_cast<uintptr_t>(rope_cs) & 7u) || rope_max_pos < L.max_kv))
+    return DSA_ERR_INVALID_ARG;
   if ((st = mla_limits(q_end - q_begin)) != DSA_OK) return st;
   if ((st = injected_fault()) != DSA_OK) return st;
-  return run_mla(q, latent, idx, v, L, q_begin, q_end, topk, n_heads, d_qk, d_v, scale, out, lse,
+  return run_mla(q, latent, idx, v, L, q_begin, q_end, topk, n_heads, d_qk, d_v, scale, rope_cs, out, lse,
                  stream);
 }
 
@@ -579,7 +623,7 @@ dsa_status dsa_forward(const void* q_idx, const float* q_scale, const float* w, 
                           ld, part_max, ld_pm, stream)) != DSA_OK)
       return st;
     if ((st = run_topk(scores, ld, part_max, ld_pm, v, L, q0, q1, topk, idx, stream)) != DSA_OK) return st;
-    if ((st = run_mla(q, latent, idx, v, L, q0, q1, topk, n_heads, d_qk, d_v, scale, out, lse,
+    if ((st = run_mla(q, latent, idx, v, L, q0, q1, topk, n_heads, d_qk, d_v, scale, nullptr, out, lse,
                       stream)) != DSA_OK)
       return st;
   }
@@ -652,6 +696,85 @@ dsa_status dsa_hadamard_quantize_fp8(const void* x, int64_t n, void* q, float* s
   if ((st = injected_fault()) != DSA_OK) return st;
   dsa::hadamard_quantize_kernel<<<static_cast<unsigned>((n + 7) / 8), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(x), n, static_cast<uint8_t*>(q), scale);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status dsa_cache_append(const void* latent_new, const void* kidx_new, dsa_varlen v, int32_t d_qk, int32_t d_v,
+                            int32_t idx_dim, const float* rope_cs, int64_t rope_max_pos, dsa_kidx_quant k_quant,
+                            void* latent_cache, void* k_cache, float* k_scale, cudaStream_t stream) {
+  if (v.batch < 1 || !v.cu_q_host) return DSA_ERR_INVALID_ARG;
+  Layout L;
+  dsa_status st = check_varlen(v, 0, v.cu_q_host[v.batch], &L);
+  if (st != DSA_OK) return st;
+  if ((latent_new == nullptr) != (latent_cache == nullptr) || (kidx_new == nullptr) != (k_cache == nullptr))
+    return DSA_ERR_INVALID_ARG;
+  if ((latent_new && (!aligned16(latent_new) || !aligned16(latent_cache))) ||
+      (kidx_new && (!aligned16(kidx_new) || !aligned16(k_cache))))
+    return DSA_ERR_INVALID_ARG;
+  if (latent_new && !is_released_mla(128, d_qk, d_v) && !is_tiny_mla(4, d_qk, d_v)) return DSA_ERR_UNSUPPORTED;
+  if (rope_cs && (!latent_new || (reinterpret_cast<uintptr_t>(rope_cs) & 7u) || rope_max_pos < L.max_kv))
+    return DSA_ERR_INVALID_ARG;
+  if (kidx_new) {
+    if (k_quant != DSA_KQ_BF16 && k_quant != DSA_KQ_E4M3_AMAX && k_quant != DSA_KQ_E4M3_HADAMARD)
+      return DSA_ERR_INVALID_ARG;
+    if (k_quant == DSA_KQ_BF16) {
+      if (!is_released_indexer(64, idx_dim) && !is_tiny_indexer(4, idx_dim)) return DSA_ERR_UNSUPPORTED;
+    } else {
+      if (!k_scale || (reinterpret_cast<uintptr_t>(k_scale) & 3u)) return DSA_ERR_INVALID_ARG;
+      if (idx_dim != dsa::FP8_DIM) return DSA_ERR_UNSUPPORTED;
+    }
+  }
+  if ((L.T + 7) / 8 > 0x7FFFFFFF) return DSA_ERR_UNSUPPORTED;
+  if (L.T == 0 || (!latent_new && !kidx_new)) return DSA_OK;
+  if ((st = injected_fault()) != DSA_OK) return st;
+  dsa::AppendParams p;
+  p.latent_new = static_cast<const __nv_bfloat16*>(latent_new);
+  p.kidx_new = static_cast<const __nv_bfloat16*>(kidx_new);
+  p.cu_q = v.cu_q;
+  p.cu_k = v.cu_k;
+  p.B = v.batch;
+  p.T = L.T;
+  p.pages = page_map(v);
+  p.rope = reinterpret_cast<const float2*>(rope_cs);
+  p.dqk = d_qk;
+  p.dv = d_v;
+  p.di = idx_dim;
+  p.k_quant = static_cast<int>(k_quant);
+  p.latent_cache = static_cast<__nv_bfloat16*>(latent_cache);
+  p.k_cache = k_cache;
+  p.k_scale = k_scale;
+  dsa::cache_append_kernel<<<static_cast<unsigned>((L.T + 7) / 8), 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status dsa_mla_up_proj(const void* o, const void* w_uv, int64_t n_rows, int32_t n_heads, int32_t d_c,
+                           int32_t d_v, void* y, cudaStream_t stream) {
+  using C = dsa::UpProjCfg;
+  if (n_rows < 0) return DSA_ERR_INVALID_ARG;
+  if (!o || !w_uv || !y || !aligned16(o) || !aligned16(w_uv) || !aligned16(y)) return DSA_ERR_INVALID_ARG;
+  if (n_heads != C::H || d_c != C::DC || d_v != C::DV) return DSA_ERR_UNSUPPORTED;
+  if ((n_rows + C::BM - 1) / C::BM > 65535) return DSA_ERR_UNSUPPORTED;
+  if (n_rows == 0) return DSA_OK;
+  dsa_status st;
+  if ((st = injected_fault()) != DSA_OK) return st;
+  CUtensorMap tm_o, tm_w;
+  {
+    const uint64_t dims[3] = {C::DC, C::H, static_cast<uint64_t>(n_rows)};
+    const uint64_t strides[2] = {C::DC * 2ull, static_cast<uint64_t>(C::H) * C::DC * 2ull};
+    const uint32_t box[3] = {C::BKC, 1, C::BM};
+    if (!make_map_3d(&tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, o, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return DSA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {C::DV, C::DC, C::H};
+    const uint64_t strides[2] = {C::DV * 2ull, static_cast<uint64_t>(C::DC) * C::DV * 2ull};
+    const uint32_t box[3] = {64, C::BKC, 1};
+    if (!make_map_3d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w_uv, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return DSA_ERR_CUDA;
+  }
+  if (ensure_smem<dsa::up_proj_kernel>(C::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
+  const dim3 grid(C::H, static_cast<unsigned>((n_rows + C::BM - 1) / C::BM));
+  dsa::up_proj_kernel<<<grid, C::NT, C::SMEM_BYTES, stream>>>(tm_o, tm_w, static_cast<__nv_bfloat16*>(y), n_rows);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

@@ -63,7 +63,8 @@ struct IndexerCfg {
   static constexpr int RSTAGES = CONVERT ? (PERSIST ? 11 : 4) : 0;  // raw e4m3 ring (to widen)
   static constexpr int A_TILE = BK * ROWB;
   static constexpr int B_TILE = N * ROWB;
-  static constexpr int RAW_TILE = BK * D_I;
+  static constexpr int RAW_ROWB = D_I;                    // bytes of one e4m3 key row
+  static constexpr int RAW_TILE = BK * RAW_ROWB;
   // epilogue warpgroups: two split the queries of a wide tile, or (persistent
   // schedule) take alternate tiles, each owning one TMEM accumulator
   static constexpr int EPI_WG = (PERSIST || N >= 256) ? 2 : 1;
@@ -178,7 +179,8 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t src, uint32_t& lo, uin
 struct IndexerParams {
   const float* w;            // [T, H_I]
   const float* q_scale;      // [T, H_I] (FP8 indexer) or null
-  const float* k_scale;      // [sum kv] (e4m3 keys) or null
+  const float* k_scale;      // [cache rows] (e4m3 keys) or null
+  PageMap pages;             // where the caches keep each entry
   const int32_t* cu_q;
   const int32_t* cu_k;
   int B;
@@ -298,19 +300,31 @@ __global__ void __launch_bounds__(C::NT, 1)
       armed_q = 1;
       int it = 0;
       for (; it < n_iter; ++it) {
-        const int y = k_base + (t_begin + it) * C::BK;
+        // Key tile: one box of BK rows (packed), or BK / 64 boxes of 64 rows,
+        // each inside one page (paged; a missing page loads as zeros from a
+        // row coordinate outside the cache).
+        const int s0 = (t_begin + it) * C::BK;
+        int y[C::BK / 64];
+#pragma unroll
+        for (int h = 0; h < C::BK / 64; ++h) {
+          const int r = p.pages.row(b, k_base, s0 + 64 * h);
+          y[h] = r >= 0 ? r : -64;
+        }
+        const int nbox = p.pages.paged() ? C::BK / 64 : 1;
         if constexpr (C::CONVERT) {
           const int r = it % C::RSTAGES;
           if (!mbar_wait(bar_raw_empty(r), ((it / C::RSTAGES) & 1) ^ 1, abort_flag, 11)) break;
           mbar_arrive_expect_tx(bar_raw_full(r), C::RAW_TILE);
-          tma_load_2d(s_raw + r * C::RAW_TILE, &tm_k, bar_raw_full(r), 0, y);
+          for (int h = 0; h < nbox; ++h)
+            tma_load_2d(s_raw + r * C::RAW_TILE + h * 64 * C::RAW_ROWB, &tm_k, bar_raw_full(r), 0, y[h]);
         } else {
           const int s = it % C::STAGES;
           if (!mbar_wait(bar_k_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, 12)) break;
           mbar_arrive_expect_tx(bar_k_full(s), C::A_TILE);
           for (int a = 0; a < C::NATOM; ++a)
-            tma_load_2d(s_k + s * C::A_TILE + a * C::BK * C::SWB, &tm_k, bar_k_full(s),
-                        a * C::ATOM_ELEMS, y);
+            for (int h = 0; h < nbox; ++h)
+              tma_load_2d(s_k + s * C::A_TILE + a * C::BK * C::SWB + h * 64 * C::SWB, &tm_k, bar_k_full(s),
+                          a * C::ATOM_ELEMS, y[h]);
         }
       }
       if (*abort_flag) {
@@ -408,7 +422,14 @@ __global__ void __launch_bounds__(C::NT, 1)
       const int s = (t_begin + it) * C::BK + key_in_tile;
       const bool in_seq = s < kv_len;
       float kscale = 1.f;
-      if (C::KFP8 && in_seq) kscale = p.k_scale[k_base + s];
+      if (C::KFP8 && in_seq) {
+        if (!p.pages.paged()) {
+          kscale = p.k_scale[k_base + s];
+        } else {
+          const int r = p.pages.row(b, k_base, s);
+          kscale = r >= 0 ? p.k_scale[r] : 0.f;
+        }
+      }
 #pragma unroll
       for (int q = 0; q < C::QW; ++q) {
         const int qi = g * C::QW + q;          // the same for the whole warp
@@ -580,7 +601,14 @@ __global__ void __launch_bounds__(C::NT, 1)
         const int r = it % C::RSTAGES;
         if (!mbar_wait(bar_raw_empty(r), ((it / C::RSTAGES) & 1) ^ 1, abort_flag, 51)) break;
         mbar_arrive_expect_tx(bar_raw_full(r), C::RAW_TILE);
-        tma_load_2d(s_raw + r * C::RAW_TILE, &tm_k, bar_raw_full(r), 0, q.k_base + tile * C::BK);
+        if (!p.pages.paged()) {
+          tma_load_2d(s_raw + r * C::RAW_TILE, &tm_k, bar_raw_full(r), 0, q.k_base + tile * C::BK);
+        } else {
+          for (int h = 0; h < C::BK / 64; ++h) {   // 64-row boxes, each inside one page
+            const int y = p.pages.row(q.b, q.k_base, tile * C::BK + 64 * h);
+            tma_load_2d(s_raw + r * C::RAW_TILE + h * 64 * C::RAW_ROWB, &tm_k, bar_raw_full(r), 0, y >= 0 ? y : -64);
+          }
+        }
       }
       if (*abort_flag) {
         long long t0 = clock64();
@@ -715,7 +743,9 @@ __global__ void __launch_bounds__(C::NT, 1)
       while (u >= upre[bp + 1]) ++bp;
       const int kb = p.cu_k[bp];
       const int s_key = (u - upre[bp]) * C::BK + key_in_tile;
-      return s_key < p.cu_k[bp + 1] - kb ? p.k_scale[kb + s_key] : 0.f;
+      if (s_key >= p.cu_k[bp + 1] - kb) return 0.f;
+      const int r = p.pages.row(bp, kb, s_key);
+      return r >= 0 ? p.k_scale[r] : 0.f;
     };
     float ks = fetch_scale(g);
     for (int it = g; it < n_iter; it += C::EPI_WG) {

@@ -17,6 +17,7 @@ __device__ int g_device_error;
 
 enum DeviceErrorCode : int {
   kErrWaitTimeout = 1,      // an mbarrier wait exceeded its limit; bits 8.. hold the wait site
+  kErrMissingPage = 2,      // a paged cache entry that was needed had no valid page; bits 8.. hold the site
 };
 
 #ifdef DSA_PROFILE_WAITS
@@ -235,6 +236,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+// 3D tiled load of box (x, y, z), x innermost.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 

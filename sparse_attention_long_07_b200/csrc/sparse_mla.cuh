@@ -20,14 +20,10 @@
 // SMs): CTA r owns output columns [256 r, 256 r + 256).  QK is split along K
 // the same way -- CTA 0 multiplies latent columns [0, 256), CTA 1 columns
 // [256, 576) -- so each CTA needs only its own 256 or 320 columns of every
-// selected row and no MMA is duplicated.  Fetching, though, goes by whole
-// rows: the cost of a random-row gather is set mostly by the number of rows
-// an SM requests, not by their bytes, so each CTA fetches the complete
-// 1152-byte rows of half of every tile (8 warps issuing TMA gathers, one
-// atom each) -- its own columns straight into its atom blocks, the peer's
-// columns into a staging block that a forwarder thread then copies into the
-// peer's atom blocks through distributed shared memory (flow-controlled by
-// per-stage barriers in both CTAs).  The two partial score tiles are
+// selected row and no MMA is duplicated.  Random-row gathers are bound by
+// the rate at which an SM can have rows requested and in flight, so eight
+// warps issue them (warp w the four rows 4w .. 4w+3 of a tile, one gather4
+// per atom) into a seven-deep ring.  The two partial score tiles are
 // exchanged through distributed shared memory (each CTA stages its part in its
 // own shared memory and one bulk copy moves it into the peer's buffer,
 // completing on the peer's mbarrier); both CTAs add them in the same
@@ -35,15 +31,14 @@
 // softmax decisions.  Tensor memory holds O, three score buffers (a tile's P,
 // in bf16, overwrites its scores once they are in registers) and this CTA's
 // slice of the query, the A operand of every QK MMA, so shared memory is left
-// to a five-deep ring of gathered rows (and their staging) and the score
-// exchange.  The online
+// to the ring of gathered rows and the score exchange.  The online
 // softmax keeps a per-head running max and only rescales O (in TMEM) when the
 // max grows by more than 2^8, which is exact arithmetic with the same final
 // normalisation.
 //
-// Roles per CTA: warps 0-3 query load, softmax and epilogue (one head row per
-// thread), warp 4 MMA issuer (and TMEM owner); with two CTAs warp 5 forwards
-// the staging to the peer and warps 6-13 gather; with one CTA warp 5 gathers.
+// Roles per CTA: warps 0-7 query load, softmax and epilogue (a head row and
+// half of a tile's columns per thread), warp 8 MMA issuer (and TMEM owner),
+// warps 9.. gather (eight with two CTAs, one with one CTA).
 #pragma once
 
 #include "common.cuh"
@@ -66,18 +61,9 @@ struct MlaCfg {
   static constexpr int NA0 = SPLIT_ATOM;                  // atoms gathered by rank 0
   static constexpr int NA1 = NATOM_ALL - SPLIT_ATOM;      // atoms gathered by rank 1
   static constexpr int NA_MAX = NA0 > NA1 ? NA0 : NA1;
-  static constexpr int NS = SPLIT == 1 ? 4 : 5;           // gather ring depth
+  static constexpr int NS = SPLIT == 1 ? 4 : 6;           // gather ring depth
   static constexpr int C_ATOM_BYTES = BN * SWB;
-  // 2-CTA split: each CTA fetches whole rows for HALF of a tile's rows; its
-  // own atoms land in its atom blocks (rows HALF*rank ..), the peer's atoms in
-  // a staging block that is then copied into the peer's atom blocks.
-  static constexpr int HALF = BN / 2;
-  static constexpr int HALF_ATOM_BYTES = HALF * SWB;
-  static constexpr int STG_MAX = SPLIT == 2 ? (NA0 > NA1 ? NA0 : NA1) : 0;   // staging blocks (the peer's atoms)
-  static constexpr int C_STAGE = SPLIT == 2 ? (NA0 * C_ATOM_BYTES + NA1 * HALF_ATOM_BYTES > NA1 * C_ATOM_BYTES + NA0 * HALF_ATOM_BYTES
-                                                   ? NA0 * C_ATOM_BYTES + NA1 * HALF_ATOM_BYTES
-                                                   : NA1 * C_ATOM_BYTES + NA0 * HALF_ATOM_BYTES)
-                                              : NA_MAX * C_ATOM_BYTES;
+  static constexpr int C_STAGE = NA_MAX * C_ATOM_BYTES;
   static constexpr int X_BYTES = SPLIT == 2 ? 128 * BN * 4 : 0;   // one partial-score tile
   static constexpr int OFF_C = 0;
   // Received partial-score tiles: tile j lands in buffer j % XR.  With four
@@ -86,15 +72,23 @@ struct MlaCfg {
   // only after it had consumed tile j - 4, the buffer's previous content.
   static constexpr int XR = 4;
   static constexpr int OFF_X = OFF_C + NS * C_STAGE;
-  static constexpr int OFF_XS = OFF_X + XR * X_BYTES;     // the staged outgoing tile
-  static constexpr int OFF_MASK = OFF_XS + X_BYTES;
+  static constexpr int XS = 2;                             // outgoing tiles staged (double buffer)
+  static constexpr int OFF_XS = OFF_X + XR * X_BYTES;
+  // softmax warps: two per TMEM lane quarter, each thread one head row and
+  // half of a tile's columns; the pair exchanges row maxima (by tile parity)
+  // and, at the end, row sums through shared memory
+  static constexpr int NSM = 8;
+  static constexpr int HB = BN / 2;                        // columns of a tile per softmax thread
+  static constexpr int OFF_MX = OFF_XS + XS * X_BYTES;     // [2 parities][2 halves][128] fp32
+  static constexpr int OFF_LS = OFF_MX + 2 * 2 * 128 * 4;  // [2 halves][128] fp32
+  static constexpr int OFF_MASK = OFF_LS + 2 * 128 * 4;
   static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
   static constexpr int NSB = 3;                            // S buffers (each later holds its P)
   static constexpr int LOOKAHEAD = 2;                      // QK tiles issued ahead of PV
   // q_ready, c_full/c_empty per stage, 3 per S buffer, x_full per receive
-  // buffer, drain, xs_full, xs_free; the 2-CTA split adds stg_full (staging
-  // landed) and partner_free (the peer's stage is free) per stage
-  static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + XR + 5 + (SPLIT == 2 ? 2 * NS : 0);
+  // buffer, drain, xs_full, xs_free per staging buffer, and per lane quarter
+  // the pair's max exchange (two tile parities) and row-sum exchange
+  static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + XR + 3 + XS + 4 * 3;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // tensor memory columns: O [0, DVS); S[NSB] (fp32, BN each; P of the same
@@ -106,12 +100,11 @@ struct MlaCfg {
   static constexpr int TMEM_USED = TMEM_Q + QCOLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   // roles: warps 0-3 softmax and epilogue, MMA_WARP the MMA issuer (and TMEM
-  // owner); the 2-CTA split has a forwarder warp and NPROD gather warps
-  // (more warps issuing TMA gathers raise the row rate of one SM)
-  static constexpr int MMA_WARP = 4;
-  static constexpr int FWD_WARP = 5;
-  static constexpr int NPROD = SPLIT == 2 ? 8 : 1;
-  static constexpr int PROD_WARP0 = SPLIT == 2 ? 6 : 5;
+  // owner), then NPROD gather warps: more warps issuing TMA gathers raise the
+  // rate at which one SM requests rows
+  static constexpr int MMA_WARP = NSM;
+  static constexpr int NPROD = SPLIT == 2 ? BN / 4 : 1;   // one per four-row group of a tile
+  static constexpr int PROD_WARP0 = NSM + 1;
   static constexpr int NT = (PROD_WARP0 + NPROD) * 32;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, DVS, false, true);
@@ -125,8 +118,9 @@ struct MlaCfg {
   static_assert(QCOLS % 8 == 0, "query columns are stored eight at a time");
   static_assert(TMEM_USED <= 512, "tensor memory");
   static_assert(OFF_C % 1024 == 0 && C_STAGE % 1024 == 0 && C_ATOM_BYTES % 1024 == 0, "swizzle atoms");
-  static_assert(SPLIT == 1 || (HALF_ATOM_BYTES % 1024 == 0 && HALF % 4 == 0 && NATOM_ALL <= 2 * NPROD),
-                "half-tile blocks keep the swizzle phase; every atom has a gather warp");
+  static_assert(SPLIT == 1 || NA_MAX <= 32, "one lane per atom");
+  static_assert(HB % 16 == 0 && (DVS / 2) % 16 == 0 && QCOLS % 8 == 0, "column halves of the softmax threads");
+  static_assert(OFF_XS % 16 == 0 && OFF_MX % 16 == 0, "bulk-copy / vector alignment");
   static_assert(OFF_X % 16 == 0 && OFF_XS % 16 == 0 && OFF_BAR % 8 == 0, "vector / bulk-copy / barrier alignment");
 };
 
@@ -135,13 +129,26 @@ struct MlaParams {
   const int32_t* idx;        // [q_end - q_begin, topk]
   const int32_t* cu_q;
   const int32_t* cu_k;
+  PageMap pages;             // where the latent cache keeps each entry
   int B;
   int64_t q_begin;
   int topk;
   float scale_log2;          // softmax scale * log2(e)
+  const float2* rope;        // null, or [max_pos, (DQK - DV) / 2] (cos, sin): RoPE on q's rope columns
   __nv_bfloat16* out;        // [T, H, DV]
   float* lse;                // [T, H] or null
 };
+
+// Cache row of selected entry sel of query row ri, or -1 when the entry is
+// skipped: outside 0 .. pos (the -1 padding included), or (paged caches) on
+// a missing page, which is also recorded in the device error word.  Skipped
+// entries are gathered from row 0 and masked.
+__device__ __forceinline__ int gather_row(const PageMap& pages, const RowInfo& ri, int sel) {
+  if (sel < 0 || sel > ri.pos) return -1;
+  const int r = pages.row(ri.b, ri.k_base, sel);
+  if (r < 0) record_device_error(kErrMissingPage | (23 << 8));
+  return r;
+}
 
 template <class C>
 __global__ void __launch_bounds__(C::NT, 1)
@@ -154,8 +161,6 @@ __global__ void __launch_bounds__(C::NT, 1)
   const int32_t* __restrict__ idx_row = p.idx + r_local * p.topk;
   const int a0 = rank == 0 ? 0 : C::SPLIT_ATOM;           // first atom of this CTA's columns (global)
   const int na = rank == 0 ? C::NA0 : C::NA1;             // atoms of this CTA's columns
-  const int p0 = rank == 0 ? C::SPLIT_ATOM : 0;           // the peer's columns
-  const int np = rank == 0 ? C::NA1 : C::NA0;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -163,6 +168,8 @@ __global__ void __launch_bounds__(C::NT, 1)
   const uint32_t s_c = sbase + C::OFF_C;
   float* xbuf = reinterpret_cast<float*>(smem + C::OFF_X);
   float* xs = reinterpret_cast<float*>(smem + C::OFF_XS);
+  float* mx_s = reinterpret_cast<float*>(smem + C::OFF_MX);
+  float* l_s = reinterpret_cast<float*>(smem + C::OFF_LS);
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const uint32_t bar_q_ready = bar0;                     // query slice stored in TMEM (128 arrivals)
@@ -177,17 +184,15 @@ __global__ void __launch_bounds__(C::NT, 1)
   constexpr int XB0 = SB0 + 3 * C::NSB;
   auto bar_x_full = [&](int b) { return bar0 + 8 * (XB0 + b); };          // b < XR
   const uint32_t bar_drain = bar0 + 8 * (XB0 + C::XR);
-  // outgoing staging buffer: every row written (128 arrivals) / read by the previous copy (thread 0)
+  // outgoing staging: every row written (one arrival per softmax thread) /
+  // staging buffer b read by its last copy (thread 0)
   const uint32_t bar_xs_full = bar0 + 8 * (XB0 + C::XR + 1);
-  const uint32_t bar_xs_free = bar0 + 8 * (XB0 + C::XR + 2);
-  // 2-CTA split: this CTA's staging of stage s landed (the peer's atoms of
-  // its own rows) / the peer's stage s is free for this CTA's rows
-  constexpr int FB0 = XB0 + C::XR + 3;
-  auto bar_stg_full = [&](int s) { return bar0 + 8 * (FB0 + s); };
-  auto bar_partner_free = [&](int s) { return bar0 + 8 * (FB0 + C::NS + s); };
-  // stage s: this CTA's atom blocks (BN rows each), then the staging blocks (HALF rows each)
-  auto own_block = [&](int s, int l) { return s_c + s * C::C_STAGE + l * C::C_ATOM_BYTES; };
-  auto stg_block = [&](int s, int m) { return s_c + s * C::C_STAGE + na * C::C_ATOM_BYTES + m * C::HALF_ATOM_BYTES; };
+  auto bar_xs_free = [&](int b) { return bar0 + 8 * (XB0 + C::XR + 2 + b); };
+  // the two softmax warps of lane quarter q meet here (64 arrivals): row
+  // maxima of tiles of parity par, and the row sums at the end
+  constexpr int PB0 = XB0 + C::XR + 2 + C::XS;
+  auto bar_pair_mx = [&](int q, int par) { return bar0 + 8 * (PB0 + 2 * q + par); };
+  auto bar_pair_l = [&](int q) { return bar0 + 8 * (PB0 + 8 + q); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* ntiles_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -197,29 +202,25 @@ __global__ void __launch_bounds__(C::NT, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q_ready, 128);
+    mbar_init(bar_q_ready, C::NSM * 32);
     for (int s = 0; s < C::NS; ++s) {
-      if (C::SPLIT == 2) {
-        // c_full: every gather warp (its bytes) + the peer's forwarded rows;
-        // c_empty: the MMAs that read the stage + the forwarder (staging read)
-        mbar_init(bar_c_full(s), C::NPROD + 1);
-        mbar_init(bar_c_empty(s), 2);
-        mbar_init(bar_stg_full(s), C::NPROD);
-        mbar_init(bar_partner_free(s), 1);
-      } else {
-        mbar_init(bar_c_full(s), 1);
-        mbar_init(bar_c_empty(s), 1);
-      }
+      mbar_init(bar_c_full(s), C::NPROD);   // every gather warp arrives with its bytes
+      mbar_init(bar_c_empty(s), 1);
     }
     for (int a = 0; a < C::NSB; ++a) {
       mbar_init(bar_s_full(a), 1);
       mbar_init(bar_pv_done(a), 1);
-      mbar_init(bar_p_full(a), 128);
+      mbar_init(bar_p_full(a), C::NSM * 32);
     }
     for (int b = 0; b < C::XR; ++b) mbar_init(bar_x_full(b), 1);   // armed locally; filled by the peer's copy
     mbar_init(bar_drain, 1);
-    mbar_init(bar_xs_full, 128);
-    mbar_init(bar_xs_free, 1);
+    mbar_init(bar_xs_full, C::NSM * 32);
+    for (int b = 0; b < C::XS; ++b) mbar_init(bar_xs_free(b), 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(bar_pair_mx(q, 0), 64);
+      mbar_init(bar_pair_mx(q, 1), 64);
+      mbar_init(bar_pair_l(q), 64);
+    }
     *abort_flag = 0;
     *ntiles_s = 0;
     // an error recorded earlier by any CTA of this library: skip the work
@@ -266,12 +267,12 @@ __global__ void __launch_bounds__(C::NT, 1)
         if (!ok) break;
         const int e = it * C::BN + lane;
         const int sel = e < p.topk ? idx_row[e] : -1;
-        const bool valid = sel >= 0 && sel <= ri.pos;
-        const int grow = ri.k_base + (valid ? sel : 0);
+        const int grow = gather_row(p.pages, ri, sel);
+        const bool valid = grow >= 0;
         const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid);
         int y[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) y[j] = __shfl_sync(0xFFFFFFFFu, grow, (4 * lane + j) & 31);
+        for (int j = 0; j < 4; ++j) y[j] = __shfl_sync(0xFFFFFFFFu, valid ? grow : 0, (4 * lane + j) & 31);
         if (lane == 0) {
           mask_s[s] = vmask;
           mbar_arrive_expect_tx(bar_c_full(s), na * C::C_ATOM_BYTES);
@@ -295,15 +296,9 @@ __global__ void __launch_bounds__(C::NT, 1)
     if (lane == 0) DSA_PROF_SPAN(61, t_role);
   } else if (C::SPLIT == 2 && warp >= C::PROD_WARP0) {
     // ------------------------------------------------------------ gather warps (2-CTA split)
-    // This CTA fetches the whole rows HALF*rank .. HALF*rank + HALF-1 of every
-    // tile: its own atoms into its atom blocks, the peer's atoms into staging.
-    // Gather warp w takes the atoms g = w, w + NPROD, ... of the 9; lanes
-    // 0..HALF/4-1 each issue one gather4 (four rows) per atom.
+    // Gather warp w fetches the four rows 4w .. 4w+3 of every tile, lane a
+    // the 64-column atom a of this CTA's columns (one gather4 each).
     const int w = warp - C::PROD_WARP0;
-    int n_own = 0, n_stg = 0;
-    for (int g = w; g < C::NATOM_ALL; g += C::NPROD) {
-      if (g >= a0 && g < a0 + na) ++n_own; else ++n_stg;
-    }
     int it = 0;
     if (n_tiles > 0) {
       for (; it < n_tiles; ++it) {
@@ -312,80 +307,32 @@ __global__ void __launch_bounds__(C::NT, 1)
         if (lane == 0) ok = mbar_wait(bar_c_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, 21);
         ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
         if (!ok) break;
-        // this CTA's rows of the tile (lanes 0..HALF-1)
-        const int e = it * C::BN + C::HALF * static_cast<int>(rank) + (lane & (C::HALF - 1));
+        const int e = it * C::BN + lane;
         const int sel = e < p.topk ? idx_row[e] : -1;
-        const bool valid = sel >= 0 && sel <= ri.pos;
-        const int grow = ri.k_base + (valid ? sel : 0);
+        const int grow = gather_row(p.pages, ri, sel);
+        const bool valid = grow >= 0;
         int y[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) y[j] = __shfl_sync(0xFFFFFFFFu, grow, (4 * lane + j) & (C::HALF - 1));
+        for (int j = 0; j < 4; ++j) y[j] = __shfl_sync(0xFFFFFFFFu, valid ? grow : 0, 4 * w + j);
         if (w == 0) {
-          // validity of all BN rows of the tile (both halves), read after c_full
-          const int e2 = it * C::BN + lane;
-          const int sel2 = e2 < p.topk ? idx_row[e2] : -1;
-          const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, sel2 >= 0 && sel2 <= ri.pos);
+          const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid);   // validity of the tile's rows
           if (lane == 0) mask_s[s] = vmask;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(bar_c_full(s), n_own * C::HALF_ATOM_BYTES);
-          mbar_arrive_expect_tx(bar_stg_full(s), n_stg * C::HALF_ATOM_BYTES);
-        }
+        if (lane == 0) mbar_arrive_expect_tx(bar_c_full(s), na * 4 * C::SWB);
         __syncwarp();
-        if (lane < C::HALF / 4) {
-          for (int g = w; g < C::NATOM_ALL; g += C::NPROD) {
-            if (g >= a0 && g < a0 + na)
-              tma_gather4(own_block(s, g - a0) + rank * C::HALF_ATOM_BYTES + lane * 4 * C::SWB, &tm_lat,
-                          bar_c_full(s), g * C::ATOM, y[0], y[1], y[2], y[3]);
-            else
-              tma_gather4(stg_block(s, g - p0) + lane * 4 * C::SWB, &tm_lat, bar_stg_full(s), g * C::ATOM, y[0],
-                          y[1], y[2], y[3]);
-          }
-        }
+        if (lane < na)
+          tma_gather4(s_c + s * C::C_STAGE + lane * C::C_ATOM_BYTES + w * 4 * C::SWB, &tm_lat, bar_c_full(s),
+                      (a0 + lane) * C::ATOM, y[0], y[1], y[2], y[3]);
       }
       if (lane == 0 && *abort_flag) {
-        // let this warp's copies in flight land before the CTA leaves (c_full
-        // also waits for the peer's rows, which may never come after an
-        // error: the wait is bounded)
+        // let this warp's copies in flight land before the CTA leaves
         long long t0 = clock64();
-        for (int j = (it > C::NS ? it - C::NS : 0); j < it; ++j) {
-          while (!mbar_try_wait(bar_stg_full(j % C::NS), (j / C::NS) & 1) && clock64() - t0 < kWaitLimitCycles) {
-          }
+        for (int j = (it > C::NS ? it - C::NS : 0); j < it; ++j)
           while (!mbar_try_wait(bar_c_full(j % C::NS), (j / C::NS) & 1) && clock64() - t0 < kWaitLimitCycles) {
           }
-        }
       }
     }
     if (lane == 0 && w == 0) DSA_PROF_SPAN(61, t_role);
-  } else if (C::SPLIT == 2 && warp == C::FWD_WARP) {
-    // ------------------------------------------------------------ forwarder (2-CTA split)
-    // Per tile: (1) once this CTA's stage s no longer holds tile it - NS, tell
-    // the peer it may copy its rows of tile it there; (2) wait for this CTA's
-    // staging of tile it and (3) for the peer's go-ahead; (4) copy the
-    // staging into the peer's atom blocks (rows HALF*rank ..), completing on
-    // the peer's c_full; (5) once the copies have read the staging, count as
-    // the staging's share of this stage's c_empty.
-    if (lane == 0 && n_tiles > 0) {
-      const uint32_t peer_stage0 = mapa_shared(s_c, peer);
-      int it = 0;
-      for (; it < n_tiles; ++it) {
-        const int s = it % C::NS;
-        if (it >= C::NS && !mbar_wait(bar_c_empty(s), ((it / C::NS) & 1) ^ 1, abort_flag, 35)) break;
-        mbar_arrive_remote(mapa_shared(bar_partner_free(s), peer));
-        if (!mbar_wait(bar_stg_full(s), (it / C::NS) & 1, abort_flag, 36)) break;
-        if (!mbar_wait<true>(bar_partner_free(s), (it / C::NS) & 1, abort_flag, 37)) break;
-        const uint32_t peer_full = mapa_shared(bar_c_full(s), peer);
-        mbar_arrive_expect_tx_remote(peer_full, np * C::HALF_ATOM_BYTES);
-        for (int m = 0; m < np; ++m)
-          bulk_copy_to_peer(peer_stage0 + s * C::C_STAGE + m * C::C_ATOM_BYTES + rank * C::HALF_ATOM_BYTES,
-                            stg_block(s, m), C::HALF_ATOM_BYTES, peer_full);
-        bulk_commit_group();
-        bulk_wait_group_read<0>();
-        mbar_arrive(bar_c_empty(s));
-      }
-      bulk_wait_group<0>();   // the copies have landed in the peer before this CTA can leave
-      DSA_PROF_SPAN(59, t_role);
-    }
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_tiles > 0) {
@@ -446,12 +393,17 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int h = warp * 32 + lane;                       // head row = TMEM lane
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    // Thread (head row h, column half c): warps q4 and q4 + 4 share the TMEM
+    // lanes 32 q4 .. 32 q4 + 31; warp q4 + 4c takes columns [c HB, c HB + HB)
+    // of every score tile, columns [c DVS/2, ...) of O, and the 8-column
+    // chunks c, c + 2, ... of the query slice.
+    const int q4 = warp & 3, c = warp >> 2;
+    const int h = q4 * 32 + lane;                          // head row = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t x_peer = C::SPLIT == 2 ? mapa_shared(smem_u32(xbuf), peer) : 0u;
     const uint32_t bar_x_full_peer0 = C::SPLIT == 2 ? mapa_shared(bar_x_full(0), peer) : 0u;
     float m_used = -INFINITY;    // running max (log2 units) the exponentials are taken against
-    float l_run = 0.f;
+    float l_run = 0.f;           // this thread's columns only; the pair adds at the end
     bool ok = true;
     // Query slice of head row h (the gathered columns) into TMEM lane h: the A
     // operand of every QK MMA.  Rows h >= H hold zeros.
@@ -460,60 +412,77 @@ __global__ void __launch_bounds__(C::NT, 1)
       const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * C::H + (row_ok ? h : 0)) * C::DQK +
                                                          a0 * C::ATOM);
 #pragma unroll 1
-      for (int c0 = 0; c0 < na * C::ATOM / 2; c0 += 8) {   // 8 columns = 16 bf16 = two 16-byte loads
+      for (int c0 = 8 * c; c0 < na * C::ATOM / 2; c0 += 16) {   // 8 columns = 16 bf16 = two 16-byte loads
         uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
         if (row_ok) {
           v0 = __ldg(qrow + c0 / 4);
           v1 = __ldg(qrow + c0 / 4 + 1);
         }
-        const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const int g0 = a0 * C::ATOM + 2 * c0;   // first query element of this chunk
+        if (p.rope != nullptr && g0 >= C::DV) {
+          // RoPE of the rope columns at this row's position: element pair
+          // (2i, 2i + 1) of the rope part times (cos, sin) of pair i.
+          const float2* cs = p.rope + static_cast<int64_t>(ri.pos) * ((C::DQK - C::DV) / 2) + (g0 - C::DV) / 2;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float re = __uint_as_float(w8[j] << 16), im = __uint_as_float(w8[j] & 0xFFFF0000u);
+            const float2 r = __ldg(cs + j);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(re, r.x, -im * r.y), fmaf(re, r.y, im * r.x));
+            w8[j] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+        }
         tmem_st8(tmem + lane_base + C::TMEM_Q + c0, w8);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(bar_q_ready);
     }
-    // Load tile j's partial scores S[j % 3] and (2-CTA split) start sending them
-    // to the peer.  Tile it+1 is started before tile it is finished, so the
-    // exchange of a tile has a whole softmax iteration to complete.
+    // Load this thread's half of tile j's partial scores S[j % 3] and (2-CTA
+    // split) start sending them to the peer.  Tile it+1 is started before
+    // tile it is finished, so the exchange of a tile has a whole softmax
+    // iteration to complete.  Staging row h holds 8 16-byte chunks, chunk k
+    // at slot (k + h) & 7 (no bank conflicts); this thread writes chunks 4c ..
     auto load_and_push = [&](int j, float* dst) -> bool {
       const int sb = j % C::NSB;
       if (!mbar_wait_warp(bar_s_full(sb), (j / C::NSB) & 1, abort_flag, 26)) return false;
       tc_fence_after();
-      uint32_t raw[32];
-      tmem_ld32(tmem + lane_base + C::TMEM_S + sb * C::BN, raw);
+      uint32_t raw[C::HB];
+      tmem_ld16(tmem + lane_base + C::TMEM_S + sb * C::BN + c * C::HB, raw);
       tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < C::BN; ++c) dst[c] = __uint_as_float(raw[c]);
+      for (int k = 0; k < C::HB; ++k) dst[k] = __uint_as_float(raw[k]);
       if (C::SPLIT == 2) {
         // The tile goes to the peer in one bulk copy: every thread stages its
-        // row in this CTA's staging buffer, then thread 0 copies the 128 rows.
+        // half row, then thread 0 copies the 128 rows.  Staging buffer j & 1
+        // was last read by the copy of tile j - 2.
         const int xr = j % C::XR;    // receive buffer of tile j, on both CTAs
-        if (h == 0) {
+        const int xb = j & 1;
+        if (threadIdx.x == 0) {
           // receive side: arm tile j's phase with the bytes the peer will send
           mbar_arrive_expect_tx(bar_x_full(xr), C::X_BYTES);
-          // the copy of tile j-1 (an iteration ago) has read the staging buffer
-          if (j >= 1) {
-            bulk_wait_group_read<0>();
-            mbar_arrive(bar_xs_free);
+          if (j >= 2) {
+            bulk_wait_group_read<1>();   // every copy but the last one (tile j - 1) has read its source
+            mbar_arrive(bar_xs_free(xb));
           }
         }
-        if (j >= 1 && !mbar_wait_warp(bar_xs_free, (j - 1) & 1, abort_flag, 33)) return false;
-        float* row = xs + h * C::BN;
+        if (j >= 2 && !mbar_wait_warp(bar_xs_free(xb), ((j >> 1) - 1) & 1, abort_flag, 33)) return false;
+        float* row = xs + xb * (C::X_BYTES / 4) + h * C::BN;
 #pragma unroll
-        for (int c = 0; c < C::BN / 4; ++c) {
-          const int slot = (c + h) & (C::BN / 4 - 1);   // rotate 16-byte chunks: no bank conflicts
-          *reinterpret_cast<float4*>(row + slot * 4) = make_float4(dst[4 * c], dst[4 * c + 1], dst[4 * c + 2],
-                                                                   dst[4 * c + 3]);
+        for (int k = 0; k < C::HB / 4; ++k) {
+          const int slot = (4 * c + k + h) & (C::BN / 4 - 1);
+          *reinterpret_cast<float4*>(row + slot * 4) = make_float4(dst[4 * k], dst[4 * k + 1], dst[4 * k + 2],
+                                                                   dst[4 * k + 3]);
         }
         fence_proxy_async_smem();
         mbar_arrive_warp(bar_xs_full);
         int go = 1;
-        if (h == 0) {
+        if (threadIdx.x == 0) {
           // all rows staged (the peer's buffer xr is free: see XR)
           go = mbar_wait(bar_xs_full, j & 1, abort_flag, 34);
           if (go) {
-            bulk_copy_to_peer(x_peer + xr * C::X_BYTES, smem_u32(xs), C::X_BYTES, bar_x_full_peer0 + 8 * xr);
+            bulk_copy_to_peer(x_peer + xr * C::X_BYTES, smem_u32(xs + xb * (C::X_BYTES / 4)), C::X_BYTES,
+                              bar_x_full_peer0 + 8 * xr);
             bulk_commit_group();
           }
         }
@@ -522,7 +491,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
       return true;
     };
-    float sv[C::BN], s_next[C::BN];
+    float sv[C::HB], s_next[C::HB];
     if (n_tiles > 0 && !load_and_push(0, sv)) ok = false;
     for (int it = 0; ok && it < n_tiles; ++it) {
       const int sb = it % C::NSB;   // S buffer of this tile; its P goes there too
@@ -533,34 +502,41 @@ __global__ void __launch_bounds__(C::NT, 1)
         if (!mbar_wait_warp(bar_x_full(xr), (it / C::XR) & 1, abort_flag, 28)) { ok = false; break; }
         const float* xrow = xbuf + xr * (C::X_BYTES / 4) + h * C::BN;
 #pragma unroll
-        for (int c = 0; c < C::BN / 4; ++c) {
-          const int slot = (c + h) & (C::BN / 4 - 1);
+        for (int k = 0; k < C::HB / 4; ++k) {
+          const int slot = (4 * c + k + h) & (C::BN / 4 - 1);
           const float4 v = *reinterpret_cast<const float4*>(xrow + slot * 4);
-          sv[4 * c] += v.x;
-          sv[4 * c + 1] += v.y;
-          sv[4 * c + 2] += v.z;
-          sv[4 * c + 3] += v.w;
+          sv[4 * k] += v.x;
+          sv[4 * k + 1] += v.y;
+          sv[4 * k + 2] += v.z;
+          sv[4 * k + 3] += v.w;
         }
       }
       // validity of the tile's entries (written by the producer before it armed c_full)
       if (!mbar_wait_warp(bar_c_full(it % C::NS), (it / C::NS) & 1, abort_flag, 29)) { ok = false; break; }
-      const uint32_t vmask = mask_s[it % C::NS];
+      const uint32_t vmask = mask_s[it % C::NS] >> (c * C::HB);
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int j = 0; j < C::BN; ++j) {
+      for (int j = 0; j < C::HB; ++j) {
         sv[j] = ((vmask >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
         mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
       }
-      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      // the row's max over the whole tile: this half's, then the partner's
+      // (bounded waits: a partner that gave up never arrives, and this warp
+      // then gives up too instead of waiting for good)
+      float* mxp = mx_s + (it & 1) * 256;
+      mxp[c * 128 + h] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      mbar_arrive_warp(bar_pair_mx(q4, it & 1));
+      if (!mbar_wait_warp(bar_pair_mx(q4, it & 1), (it >> 1) & 1, abort_flag, 38)) { ok = false; break; }
+      const float mt = fmaxf(mxp[h], mxp[128 + h]);
       float corr = 1.f;
       if (mt > m_used + C::kRescaleThreshold) {
         corr = exp2f(m_used - mt);   // 0 on the first tile with a valid entry
         m_used = mt;
       }
-      uint32_t pk[C::BN / 2];
+      uint32_t pk[C::HB / 2];
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < C::BN; j += 2) {
+      for (int j = 0; j < C::HB; j += 2) {
         const float e0 = sv[j] == -INFINITY ? 0.f : ex2_approx(sv[j] - m_used);
         const float e1 = sv[j + 1] == -INFINITY ? 0.f : ex2_approx(sv[j + 1] - m_used);
         const __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
@@ -569,9 +545,10 @@ __global__ void __launch_bounds__(C::NT, 1)
         pk[j / 2] = *reinterpret_cast<const uint32_t*>(&b2);
       }
       l_run = l_run * corr + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-      // The rescale decision is per head row, but the TMEM accesses below are
-      // warp-collective (.sync.aligned): the warp rescales if any lane needs
-      // it, and lanes that do not multiply by 1.
+      // The rescale decision is per head row (and the same in both threads of
+      // the row), but the TMEM accesses below are warp-collective
+      // (.sync.aligned): the warp rescales if any lane needs it, and lanes
+      // that do not multiply by 1.
       if (__any_sync(0xFFFFFFFFu, corr != 1.f && it > 0)) {
         // O must hold every earlier PV before it is rescaled in place
         if (!mbar_wait_warp(bar_pv_done((it - 1) % C::NSB), ((it - 1) / C::NSB) & 1, abort_flag, 31)) {
@@ -580,7 +557,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int c0 = 0; c0 < C::DVS; c0 += 16) {
+        for (int c0 = c * (C::DVS / 2); c0 < (c + 1) * (C::DVS / 2); c0 += 16) {
           uint32_t o[16];
           tmem_ld16(tmem + lane_base + c0, o);
           tmem_wait_ld();
@@ -590,18 +567,23 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
         tmem_wait_st();
       }
-      // P row h (bf16 pairs) over the scores of this tile (already in registers);
-      // the PV MMA reads it from there
-      tmem_st16(tmem + lane_base + C::TMEM_S + sb * C::BN, pk);
+      // P row h, this thread's columns (bf16 pairs), over the scores of this
+      // tile (already in registers); the PV MMA reads it from there
+      tmem_st8(tmem + lane_base + C::TMEM_S + sb * C::BN + c * (C::HB / 2), pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(bar_p_full(sb));
 #pragma unroll
-      for (int c = 0; c < C::BN; ++c) sv[c] = s_next[c];
+      for (int k = 0; k < C::HB; ++k) sv[k] = s_next[k];
     }
-    if (C::SPLIT == 2 && h == 0) bulk_wait_group<0>();   // outgoing copies have completed
+    if (C::SPLIT == 2 && threadIdx.x == 0) bulk_wait_group<0>();   // outgoing copies have completed
     if (lane == 0) DSA_PROF_SPAN(63, t_role);
     // ------------------------------------------------------------ epilogue
+    // the row sum over both halves
+    l_s[c * 128 + h] = l_run;
+    mbar_arrive_warp(bar_pair_l(q4));
+    if (!mbar_wait_warp(bar_pair_l(q4), 0, abort_flag, 39)) ok = false;
+    l_run = l_s[h] + l_s[128 + h];
     const int t_out = static_cast<int>(t);
     if (ok && n_tiles > 0) {
       const int j = n_tiles - 1;
@@ -614,7 +596,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       __nv_bfloat16* orow = p.out + (static_cast<int64_t>(t_out) * C::H + (store ? h : 0)) * C::DV + rank * C::DVS;
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < C::DVS; c0 += 16) {
+      for (int c0 = c * (C::DVS / 2); c0 < (c + 1) * (C::DVS / 2); c0 += 16) {
         uint32_t o[16];
         if (n_tiles > 0) {
           tmem_ld16(tmem + lane_base + c0, o);
@@ -636,13 +618,13 @@ __global__ void __launch_bounds__(C::NT, 1)
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
-      if (store && rank == 0 && p.lse != nullptr)
+      if (store && c == 0 && rank == 0 && p.lse != nullptr)
         p.lse[static_cast<int64_t>(t_out) * C::H + h] =
             l_run > 0.f ? (m_used + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
-  if (lane == 0 && warp < 4) DSA_PROF_SPAN(60, t_role);
+  if (lane == 0 && warp < C::NSM) DSA_PROF_SPAN(60, t_role);
   tc_fence_before();
   __syncthreads();
   if (C::SPLIT == 2) cluster_sync();   // no remote access into this CTA after this point

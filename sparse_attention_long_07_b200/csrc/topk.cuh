@@ -50,7 +50,7 @@ struct TopkCfg {
   static constexpr int OFF_CIDX = OFF_CKEY + CAP * 4;
   static constexpr int OFF_WTOT = OFF_CIDX + CAP * 4;
   static constexpr int OFF_CNT = OFF_WTOT + 2 * NW * 4;   // select: per-warp digit counts + totals
-  static constexpr int OFF_BAR = OFF_CNT + (128 + NW) * 4;
+  static constexpr int OFF_BAR = OFF_CNT + 128 * 4;   // block reductions: slots and results
   static constexpr int OFF_MISC = OFF_BAR + STAGES * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 64 + 128;   // + alignment slack
   static_assert(PMAX_CAP * 4 + BITMAP_BITS / 8 <= NW * (BINS1 / 2) * 4, "fast-path union fits");
@@ -260,24 +260,66 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     __syncthreads();
   };
 
+  // Block-wide sums and scans.  Each warp reduces with redux/shuffles, warp 0
+  // combines the 16 warp values, and every thread reads back one word, so a
+  // call costs two barriers and a couple of shared loads per thread.
+  // red_sum2(a, b): the CTA totals of a and b (each total < 2^16).
+  uint32_t red_phase = 0;   // alternates the result words between calls
+  auto red_sum2 = [&](uint32_t a, uint32_t b) -> uint2 {
+    const uint32_t w2 = __reduce_add_sync(0xFFFFFFFFu, a | (b << 16));   // per-warp sums stay < 2^16
+    uint32_t* sl = cnt;
+    uint32_t* res = cnt + 32 + (red_phase & 1u) * 2;
+    ++red_phase;
+    if (lane == 0) sl[warp] = w2;
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t v = lane < static_cast<uint32_t>(C::NW) ? sl[lane] : 0u;
+      const uint32_t lo = __reduce_add_sync(0xFFFFFFFFu, v & 0xFFFFu);
+      const uint32_t hi = __reduce_add_sync(0xFFFFFFFFu, v >> 16);
+      if (lane == 0) {
+        res[0] = lo;
+        res[1] = hi;
+      }
+    }
+    __syncthreads();
+    return make_uint2(res[0], res[1]);
+  };
+  // block_scan(v, &total): exclusive prefix of v over the threads in order.
+  auto block_scan = [&](uint32_t v, uint32_t* total) -> uint32_t {
+    uint32_t wt;
+    const uint32_t pre = warp_excl_scan(v, lane, &wt);
+    uint32_t* sl = cnt + 40;
+    uint32_t* wpre = cnt + 40 + 32 + (red_phase & 1u) * (C::NW + 1);
+    ++red_phase;
+    if (lane == 31) sl[warp] = pre + v;
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t x = lane < static_cast<uint32_t>(C::NW) ? sl[lane] : 0u;
+      uint32_t tot;
+      const uint32_t ex = warp_excl_scan(x, lane, &tot);
+      if (lane < static_cast<uint32_t>(C::NW)) wpre[lane] = ex;
+      if (lane == 0) wpre[C::NW] = tot;
+    }
+    __syncthreads();
+    *total = wpre[C::NW];
+    return wpre[warp] + pre;
+  };
   // Radix-4 selection.  select(count, key_of, use, kth, &thr, &rem, steps):
   // the kth largest key among the entries i < count with use(i) (at least kth
   // of them), found 2 bits at a time from the top: each step counts, for the
-  // 3 candidate values of the next digit, the entries at or above them
-  // (compares in registers, warp sums by redux, one shared slot per warp and
-  // value), and keeps the largest digit with at least kth entries at or above
-  // it.  No atomics, so concentrated key distributions cost nothing extra.
-  // Up to SEL_REG entries per thread are read once into registers.  With
-  // steps < 16 only the top 2*steps bits are resolved and the lower bits are
-  // 0: thr is then a lower bound of the kth largest key with at least kth
-  // entries >= thr.  *rem = kth - (entries > thr) (meaningful for steps = 16).
-  // Called by every thread.
-  uint32_t* slots = cnt;   // [16 warps][4]; slots + 64: the 3 totals
+  // 3 candidate values of the next digit, the entries at or above them and
+  // keeps the largest digit with at least kth entries at or above it.  No
+  // atomics, so concentrated key distributions cost nothing extra.  Up to
+  // SEL_REG entries per thread are read once into registers.  With steps <
+  // 16 only the top 2*steps bits are resolved and the lower bits are 0: thr
+  // is then a lower bound of the kth largest key with at least kth entries
+  // >= thr.  *rem = kth - (entries > thr) (meaningful for steps = 16).
+  // Called by every thread; counts stay below 2^16 (count <= 65535).
   auto select = [&](uint32_t count, auto&& key_of, auto&& use, uint32_t kth, uint32_t* out_thr,
                     uint32_t* out_rem, int steps = 16) {
     constexpr int SEL_REG = 12;
     const bool in_regs = count <= static_cast<uint32_t>(SEL_REG * C::NT);
-    uint32_t kr[SEL_REG];   // this thread's keys (entries tid, tid + NT, ...); unused ones are 0 with use = false
+    uint32_t kr[SEL_REG];   // this thread's keys (entries tid, tid + NT, ...)
     uint32_t ur = 0;        // bit e: entry e is used
 #pragma unroll
     for (int e = 0; e < SEL_REG; ++e) {
@@ -311,24 +353,10 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
           c3 += k >= t3 ? 1u : 0u;
         }
       }
-      c1 = __reduce_add_sync(0xFFFFFFFFu, c1);
-      c2 = __reduce_add_sync(0xFFFFFFFFu, c2);
-      c3 = __reduce_add_sync(0xFFFFFFFFu, c3);
-      uint32_t* sl = slots + (st & 1) * 64;   // alternate slot sets: one barrier per step
-      if (lane == 0) {
-        sl[warp * 4 + 0] = c1;
-        sl[warp * 4 + 1] = c2;
-        sl[warp * 4 + 2] = c3;
-      }
-      __syncthreads();
-      uint32_t s1 = 0, s2 = 0, s3 = 0;
-#pragma unroll
-      for (int w = 0; w < C::NW; ++w) {
-        s1 += sl[w * 4 + 0];
-        s2 += sl[w * 4 + 1];
-        s3 += sl[w * 4 + 2];
-      }
-      const uint32_t digit = (s1 >= kth ? 1u : 0u) + (s2 >= kth ? 1u : 0u) + (s3 >= kth ? 1u : 0u);
+      // c1 >= c2 >= c3: the digit is the number of thresholds still reached
+      const uint2 s12 = red_sum2(c1, c2);
+      uint32_t digit = (s12.x >= kth ? 1u : 0u) + (s12.y >= kth ? 1u : 0u);
+      if (digit == 2u) digit += red_sum2(c3, 0u).x >= kth ? 1u : 0u;   // block-uniform branch
       prefix |= digit << shift;
     }
     uint32_t gt = 0;
@@ -340,33 +368,8 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
         for (uint32_t i = tid; i < count; i += C::NT) gt += (use(i) && key_of(i) > prefix) ? 1u : 0u;
       }
     }
-    gt = __reduce_add_sync(0xFFFFFFFFu, gt);
-    uint32_t* sl = slots + 128;
-    if (lane == 0) sl[warp] = gt;
-    __syncthreads();
-    uint32_t total = 0;
-#pragma unroll
-    for (int w = 0; w < C::NW; ++w) total += sl[w];
-    __syncthreads();
     *out_thr = prefix;
-    *out_rem = kth - total;
-  };
-  // Block-wide exclusive prefix of one count per thread (in thread order) and the total.
-  auto block_scan = [&](uint32_t v, uint32_t* total) -> uint32_t {
-    uint32_t wt;
-    const uint32_t pre = warp_excl_scan(v, lane, &wt);
-    if (lane == 31) wtot[warp] = pre + v;
-    __syncthreads();
-    uint32_t base = pre, tot = 0;
-#pragma unroll
-    for (int w = 0; w < C::NW; ++w) {
-      const uint32_t x = wtot[w];
-      base += w < static_cast<int>(warp) ? x : 0u;
-      tot += x;
-    }
-    __syncthreads();
-    *total = tot;
-    return base;
+    *out_rem = kth - red_sum2(gt, 0u).x;
   };
   // Exact selection among candidates ckey/cidx[0, nc) that hold every key
   // >= some bound b with at least topk keys >= b: the topk largest keys, ties
@@ -400,14 +403,9 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     __syncthreads();
     const int per = (nwords + C::NT - 1) / C::NT;
     const int w0 = min(nwords, static_cast<int>(tid) * per), w1 = min(nwords, w0 + per);
-    uint32_t cnt = 0;
-    for (int wdx = w0; wdx < w1; ++wdx) cnt += __popc(bitmap[wdx]);
-    uint32_t wt;
-    const uint32_t pre = warp_excl_scan(cnt, lane, &wt);
-    if (lane == 31) wtot[warp] = pre + cnt;
-    __syncthreads();
-    uint32_t pos_out = pre;
-    for (int w = 0; w < static_cast<int>(warp); ++w) pos_out += wtot[w];
+    uint32_t bits_mine = 0, unused_total;
+    for (int wdx = w0; wdx < w1; ++wdx) bits_mine += __popc(bitmap[wdx]);
+    uint32_t pos_out = block_scan(bits_mine, &unused_total);
     for (int wdx = w0; wdx < w1; ++wdx) {
       uint32_t bits = bitmap[wdx];
       while (bits) {

@@ -115,13 +115,15 @@ def test_topk_and_attention_validation(dsa):
     assert lib.dsa_topk(FAKE, 100, None, 0, v, 0, 4, 2049, FAKE, None) == INV
     assert lib.dsa_topk(FAKE, 96, None, 0, v, 0, 4, 16, FAKE, None) == INV
     assert lib.dsa_topk(0, 100, None, 0, v, 0, 4, 16, FAKE, None) == INV
-    args = dict(topk=64, h=128, dqk=576, dv=512, scale=0.07)
+    args = dict(topk=64, h=128, dqk=576, dv=512, scale=0.07, rope=None, max_pos=0)
 
     def mla(**kw):
         a = dict(args)
         a.update(kw)
         return lib.dsa_sparse_mla_attn(FAKE, FAKE, FAKE, v, 0, 4, a["topk"], a["h"], a["dqk"], a["dv"],
-                                       ctypes.c_float(a["scale"]), FAKE, FAKE, None)
+                                       ctypes.c_float(a["scale"]), a["rope"], a["max_pos"], FAKE, FAKE, None)
+    assert mla(rope=FAKE + 4, max_pos=100) == INV      # RoPE table not 8-byte aligned
+    assert mla(rope=FAKE, max_pos=99) == INV           # positions reach 99: a table of 99 is short
     assert mla(topk=0) == INV
     assert mla(scale=0.0) == INV
     assert mla(scale=float("nan")) == INV
@@ -208,3 +210,36 @@ def test_fp8_quantize_arguments(dsa):
     assert lib.dsa_hadamard_quantize_fp8(FAKE, 0, FAKE, FAKE, None) == dsa.DSA_OK          # nothing to do
     assert lib.dsa_hadamard_quantize_fp8(FAKE + 8, 4, FAKE, FAKE, None) == dsa.DSA_ERR_INVALID_ARG
     assert lib.dsa_hadamard_quantize_fp8(FAKE, 4, FAKE, FAKE + 2, None) == dsa.DSA_ERR_INVALID_ARG
+
+
+@host_only
+def test_paged_layout_validation(dsa):
+    lib = dsa.library()
+
+    def paged(page_size, pages_per_seq, n_pages, table=FAKE):
+        v = varlen([0, 1, 2], [0, 300, 370])
+        v.block_table, v.page_size, v.pages_per_seq, v.n_pages = table, page_size, pages_per_seq, n_pages
+        return lib.dsa_forward_workspace_size(v, 16, 0)
+    assert paged(64, 5, 10) > 0                    # 5 pages of 64 hold the 300 entries
+    assert paged(128, 3, 10) > 0
+    assert paged(64, 4, 10) == 0                   # 4 pages of 64 < 300 entries
+    assert paged(32, 10, 10) == 0                  # pages shorter than 64 rows
+    assert paged(192, 2, 10) == 0                  # not a power of two
+    assert paged(64, 5, 0) == 0                    # empty pool
+    assert paged(1 << 20, 1, 1 << 11) == 0         # pool of 2^31 rows
+    assert paged(64, 5, 10, table=FAKE + 2) == 0   # misaligned table
+    # packed layout: the page fields are ignored
+    assert paged(0, 0, 0, table=None) > 0
+
+
+@host_only
+def test_up_projection_arguments(dsa):
+    lib = dsa.library()
+    INV, UNS = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_mla_up_proj(FAKE, FAKE, 0, 128, 512, 128, FAKE, None) == dsa.DSA_OK       # nothing to do
+    assert lib.dsa_mla_up_proj(FAKE, FAKE, -1, 128, 512, 128, FAKE, None) == INV
+    assert lib.dsa_mla_up_proj(FAKE + 8, FAKE, 4, 128, 512, 128, FAKE, None) == INV
+    assert lib.dsa_mla_up_proj(FAKE, FAKE, 4, 128, 512, 128, None, None) == INV
+    assert lib.dsa_mla_up_proj(FAKE, FAKE, 4, 64, 512, 128, FAKE, None) == UNS
+    assert lib.dsa_mla_up_proj(FAKE, FAKE, 4, 128, 576, 128, FAKE, None) == UNS
+    assert lib.dsa_mla_up_proj(FAKE, FAKE, 128 * 65536, 128, 512, 128, FAKE, None) == UNS
