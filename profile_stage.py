@@ -30,13 +30,22 @@ def main():
     ap.add_argument("--seqs", type=int, default=0, help="first N sequences only (0 = all)")
     ap.add_argument("--stage", default="indexer", choices=["indexer", "topk", "attention", "forward"])
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--fp8-indexer", action="store_true",
+                    help="the FP8 indexer: queries and keys Hadamard-rotated and quantized to e4m3")
     ap.add_argument("--wait-profile", action="store_true",
                     help="print per-wait-site cycles (library built with --profile-waits)")
     args = ap.parse_args()
     spec = di.config(args.workload)
     seqs = list(range(spec.B)) if args.seqs <= 0 else list(range(min(args.seqs, spec.B)))
     dev = torch.device("cuda", 0)
-    d = di.make_inputs(spec, device=dev, seqs=seqs)
+    q_scale = None
+    if args.fp8_indexer:
+        from dataclasses import replace
+        d = di.make_inputs(replace(spec, kfp8=False), device=dev, seqs=seqs)
+        d["q_idx"], q_scale = dsa.dsa_hadamard_quantize_fp8(d["q_idx"])
+        d["k_idx"], d["k_scale"] = dsa.dsa_hadamard_quantize_fp8(d["k_idx"])
+    else:
+        d = di.make_inputs(spec, device=dev, seqs=seqs)
     v = dsa.Varlen(d["cu_q"], d["cu_k"], dev)
     T, k = v.T, spec.topk
     ld = (v.max_kv + 3) // 4 * 4
@@ -47,20 +56,22 @@ def main():
     lse = torch.empty((T, spec.H), dtype=torch.float32, device=dev)
     ws = torch.empty(dsa.dsa_forward_workspace_size(v, k), dtype=torch.uint8, device=dev)
     # inputs of the later stages
-    dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores, part_max=part_max)
+    dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores, part_max=part_max,
+                           q_scale=q_scale)
     dsa.dsa_topk(scores, v, 0, T, k, idx, part_max=part_max)
     torch.cuda.synchronize()
 
     def run():
         if args.stage == "indexer":
-            dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores, part_max=part_max)
+            dsa.dsa_indexer_scores(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], v, 0, T, scores, part_max=part_max,
+                                   q_scale=q_scale)
         elif args.stage == "topk":
             dsa.dsa_topk(scores, v, 0, T, k, idx, part_max=part_max)
         elif args.stage == "attention":
             dsa.dsa_sparse_mla_attn(d["q"], d["latent"], idx, v, 0, T, spec.softmax_scale, out, lse)
         else:
             dsa.dsa_forward(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], d["q"], d["latent"], v, k,
-                            spec.softmax_scale, out, lse, ws)
+                            spec.softmax_scale, out, lse, ws, q_scale=q_scale)
 
     if args.wait_profile:
         dsa.dsa_debug_wait_profile(reset=True)
@@ -75,7 +86,8 @@ def main():
         prof = dsa.dsa_debug_wait_profile(reset=True) or {}
         print(json.dumps({"wait_sites": {str(k): {"cycles_per_wait": round(c / max(n, 1), 1), "waits": n,
                                                   "cycles_total": c} for k, (c, n) in sorted(prof.items())}}))
-    print(json.dumps({"workload": spec.name, "seqs": len(seqs), "stage": args.stage, "query_rows": T,
+    print(json.dumps({"workload": spec.name, "seqs": len(seqs), "stage": args.stage,
+                      "indexer": "fp8" if args.fp8_indexer else "bf16 q", "query_rows": T,
                       "keys": v.S, "mean_ms": a.elapsed_time(b) / args.iters,
                       "device_bytes_allocated": torch.cuda.memory_allocated()}))
 

@@ -19,7 +19,10 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdsa.so")
+# DSA_LIBRARY_VARIANT=checked loads the build with device-side bounds checks
+# (libdsa_checked.so, build.py --checked); the default is the release build.
+LIB_PATH = os.path.join(_HERE, "libdsa_checked.so" if os.environ.get("DSA_LIBRARY_VARIANT") == "checked"
+                        else "libdsa.so")
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA, DSA_ERR_DEVICE_TIMEOUT, DSA_ERR_WORKSPACE = range(6)
 DSA_KIDX_BF16, DSA_KIDX_FP8_E4M3 = 0, 1

@@ -36,6 +36,7 @@ struct AppendParams {
   int B;
   int64_t T;
   PageMap pages;
+  int cache_rows;                    // rows of the caches (checked builds)
   const float2* rope;                // null, or [max_pos, (dqk - dv) / 2] (cos, sin)
   int dqk, dv, di;
   int k_quant;                       // KeyQuant
@@ -54,6 +55,7 @@ __global__ void __launch_bounds__(256) cache_append_kernel(const AppendParams p)
     if (lane == 0) record_device_error(kErrMissingPage | (24 << 8));
     return;
   }
+  if (!in_bounds(r < p.cache_rows, 87)) return;
   if (p.latent_new != nullptr) {
     const uint4* src = reinterpret_cast<const uint4*>(p.latent_new + t * p.dqk);
     uint4* dst = reinterpret_cast<uint4*>(p.latent_cache + static_cast<int64_t>(r) * p.dqk);

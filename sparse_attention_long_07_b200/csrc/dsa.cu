@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <nvtx3/nvToolsExt.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -42,6 +43,15 @@ struct Layout {
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// NVTX range around each stage's launches and each entry point (visible in
+// Nsight timelines; a no-op unless a tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 dsa::PageMap page_map(const dsa_varlen& v) {
   dsa::PageMap m;
@@ -224,6 +234,7 @@ dsa_status launch_indexer(const void* q_idx, const float* q_scale, const float* 
   p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.pages = page_map(v);
+  p.cache_rows = static_cast<int>(L.S);
   p.cu_q = v.cu_q;
   p.cu_k = v.cu_k;
   p.B = v.batch;
@@ -245,7 +256,7 @@ dsa_status launch_indexer(const void* q_idx, const float* q_scale, const float* 
 
 // Decode-like calls: one persistent CTA per SM over the flat (sequence, key tile) list.
 template <class C>
-dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const void* k_idx,
+dsa_status launch_indexer_persistent(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
                                      const float* k_scale, const dsa_varlen& v, const Layout& L,
                                      int64_t q_begin, int64_t q_end, float* scores, int64_t ld,
                                      float* part_max, int64_t ld_pm, cudaStream_t stream) {
@@ -262,8 +273,8 @@ dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const vo
   if (units == 0) return DSA_OK;
   if (sms <= 0) return DSA_ERR_CUDA;
   CUtensorMap tm_q, tm_k;
-  if (!make_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q_idx, C::D_I, static_cast<uint64_t>(L.T) * C::H_I,
-                C::D_I * 2, C::ATOM_ELEMS, C::N, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_map(&tm_q, C::QFP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q_idx, C::D_I,
+                static_cast<uint64_t>(L.T) * C::H_I, C::D_I * C::ELEM, C::ATOM_ELEMS, C::N, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   if (!make_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_idx, C::D_I, static_cast<uint64_t>(L.S), C::D_I, C::D_I,
                 v.block_table ? 64u : static_cast<uint32_t>(C::BK), CU_TENSOR_MAP_SWIZZLE_128B))
@@ -271,9 +282,10 @@ dsa_status launch_indexer_persistent(const void* q_idx, const float* w, const vo
   if (ensure_smem<dsa::indexer_persistent_kernel<C>>(C::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
   dsa::IndexerParams p;
   p.w = w;
-  p.q_scale = nullptr;
+  p.q_scale = q_scale;
   p.k_scale = k_scale;
   p.pages = page_map(v);
+  p.cache_rows = static_cast<int>(L.S);
   p.cu_q = v.cu_q;
   p.cu_k = v.cu_k;
   p.B = v.batch;
@@ -307,6 +319,7 @@ dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, con
   p.cu_q = v.cu_q;
   p.cu_k = v.cu_k;
   p.pages = page_map(v);
+  p.cache_rows = static_cast<int>(L.S);
   p.B = v.batch;
   p.q_begin = q_begin;
   p.topk = topk;
@@ -369,12 +382,18 @@ dsa_status check_mla_args(const void* q, const void* latent, const int32_t* idx,
 // Which indexer kernel a pass uses.  Decode-like passes (at most one query row
 // per sequence) over an e4m3 cache take the persistent kernel; otherwise the
 // query-block grid kernel with 1 or 4 queries per CTA.
-enum class IndexerKind { kTiny, kPersistent, kGridFp8x1, kGridFp8x4, kGridBf16x1, kGridBf16x4, kFp8Fp8x1, kFp8Fp8x4 };
+enum class IndexerKind {
+  kTiny, kPersistent, kGridFp8x1, kGridFp8x4, kGridBf16x1, kGridBf16x4, kFp8Fp8Persistent, kFp8Fp8x1, kFp8Fp8x4
+};
 
 IndexerKind choose_indexer(bool q_fp8, dsa_kidx_dtype kd, int h, int d, const dsa_varlen& v, const Layout& L) {
   if (is_tiny_indexer(h, d)) return IndexerKind::kTiny;
   const bool decode_like = L.max_q_rows <= 2;
-  if (q_fp8) return decode_like ? IndexerKind::kFp8Fp8x1 : IndexerKind::kFp8Fp8x4;
+  if (q_fp8) {
+    if (L.max_q_rows <= 1 && v.batch <= IndexerCfg<64, 128, 1, true, true, true>::MAX_SEQ)
+      return IndexerKind::kFp8Fp8Persistent;
+    return decode_like ? IndexerKind::kFp8Fp8x1 : IndexerKind::kFp8Fp8x4;
+  }
   if (kd == DSA_KIDX_FP8_E4M3) {
     if (L.max_q_rows <= 1 && v.batch <= IndexerCfg<64, 128, 1, true, true>::MAX_SEQ) return IndexerKind::kPersistent;
     return decode_like ? IndexerKind::kGridFp8x1 : IndexerKind::kGridFp8x4;
@@ -386,7 +405,7 @@ IndexerKind choose_indexer(bool q_fp8, dsa_kidx_dtype kd, int h, int d, const ds
 dsa_status indexer_limits(bool q_fp8, dsa_kidx_dtype kd, int h, int d, const dsa_varlen& v, const Layout& L) {
   if (L.max_q_rows == 0) return DSA_OK;
   const IndexerKind k = choose_indexer(q_fp8, kd, h, d, v, L);
-  if (k == IndexerKind::kPersistent) return DSA_OK;
+  if (k == IndexerKind::kPersistent || k == IndexerKind::kFp8Fp8Persistent) return DSA_OK;
   const int nq = (k == IndexerKind::kGridFp8x1 || k == IndexerKind::kGridBf16x1 || k == IndexerKind::kFp8Fp8x1) ? 1 : 4;
   const int64_t qblocks = (L.max_q_rows + nq - 1) / nq;
   if (qblocks > 65535 || v.batch > 65535) return DSA_ERR_UNSUPPORTED;   // gridDim.y / gridDim.z
@@ -398,7 +417,12 @@ dsa_status run_indexer(const void* q_idx, const float* q_scale, const float* w, 
                        int64_t q_begin, int64_t q_end, float* scores, int64_t ld, float* part_max,
                        int64_t ld_pm, cudaStream_t stream) {
   if (q_end == q_begin) return DSA_OK;
+  NvtxRange range("dsa.indexer");
   switch (choose_indexer(q_scale != nullptr, kd, h, d, v, L)) {
+    case IndexerKind::kFp8Fp8Persistent:
+      return launch_indexer_persistent<IndexerCfg<64, 128, 1, true, true, true>>(q_idx, q_scale, w, k_idx, k_scale,
+                                                                                 v, L, q_begin, q_end, scores, ld,
+                                                                                 part_max, ld_pm, stream);
     case IndexerKind::kFp8Fp8x1:
       return launch_indexer<IndexerCfg<64, 128, 1, true, false, true>>(q_idx, q_scale, w, k_idx, k_scale, v, L,
                                                                         q_begin, q_end, scores, ld, part_max, ld_pm,
@@ -411,7 +435,7 @@ dsa_status run_indexer(const void* q_idx, const float* q_scale, const float* w, 
       return launch_indexer<IndexerCfg<4, 32, 4, false>>(q_idx, nullptr, w, k_idx, k_scale, v, L, q_begin, q_end,
                                                           scores, ld, part_max, ld_pm, stream);
     case IndexerKind::kPersistent:
-      return launch_indexer_persistent<IndexerCfg<64, 128, 1, true, true>>(q_idx, w, k_idx, k_scale, v, L,
+      return launch_indexer_persistent<IndexerCfg<64, 128, 1, true, true>>(q_idx, nullptr, w, k_idx, k_scale, v, L,
                                                                            q_begin, q_end, scores, ld, part_max, ld_pm, stream);
     case IndexerKind::kGridFp8x1:
       return launch_indexer<IndexerCfg<64, 128, 1, true>>(q_idx, nullptr, w, k_idx, k_scale, v, L, q_begin, q_end,
@@ -443,6 +467,7 @@ dsa_status run_topk(const float* scores, int64_t ld, const float* part_max, int6
                     const Layout& L, int64_t q_begin, int64_t q_end, int topk, int32_t* idx, cudaStream_t stream) {
   const int64_t rows = q_end - q_begin;
   if (rows == 0) return DSA_OK;
+  NvtxRange range("dsa.topk");
   if (topk_limits(L, rows) != DSA_OK) return DSA_ERR_UNSUPPORTED;
   if (ensure_smem<dsa::topk_kernel>(dsa::TopkCfg::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
   dsa::topk_kernel<<<static_cast<unsigned>(rows), dsa::TopkCfg::NT, dsa::TopkCfg::SMEM_BYTES, stream>>>(
@@ -453,6 +478,7 @@ dsa_status run_topk(const float* scores, int64_t ld, const float* part_max, int6
 dsa_status run_mla(const void* q, const void* latent, const int32_t* idx, const dsa_varlen& v,
                    const Layout& L, int64_t q_begin, int64_t q_end, int topk, int h, int dqk, int dv,
                    float scale, const float* rope, void* out, float* lse, cudaStream_t stream) {
+  NvtxRange range("dsa.sparse_mla");
   if (is_tiny_mla(h, dqk, dv))
     return launch_mla<MlaCfg<4, 80, 64, 1, 32>>(q, latent, idx, v, L, q_begin, q_end, topk, scale, rope, out,
                                                 lse, stream);
@@ -601,6 +627,7 @@ dsa_status dsa_forward(const void* q_idx, const float* q_scale, const float* w, 
   if (need == 0) return DSA_ERR_INVALID_ARG;
   if (workspace_bytes < need) return DSA_ERR_WORKSPACE;
   if ((st = injected_fault()) != DSA_OK) return st;
+  NvtxRange range("dsa.forward");
 
   Layout full;
   check_varlen(v, 0, v.cu_q_host[v.batch], &full);
@@ -727,6 +754,7 @@ dsa_status dsa_cache_append(const void* latent_new, const void* kidx_new, dsa_va
   if ((L.T + 7) / 8 > 0x7FFFFFFF) return DSA_ERR_UNSUPPORTED;
   if (L.T == 0 || (!latent_new && !kidx_new)) return DSA_OK;
   if ((st = injected_fault()) != DSA_OK) return st;
+  NvtxRange range("dsa.cache_append");
   dsa::AppendParams p;
   p.latent_new = static_cast<const __nv_bfloat16*>(latent_new);
   p.kidx_new = static_cast<const __nv_bfloat16*>(kidx_new);
@@ -735,6 +763,7 @@ dsa_status dsa_cache_append(const void* latent_new, const void* kidx_new, dsa_va
   p.B = v.batch;
   p.T = L.T;
   p.pages = page_map(v);
+  p.cache_rows = static_cast<int>(L.S);
   p.rope = reinterpret_cast<const float2*>(rope_cs);
   p.dqk = d_qk;
   p.dv = d_v;
@@ -773,6 +802,7 @@ dsa_status dsa_mla_up_proj(const void* o, const void* w_uv, int64_t n_rows, int3
       return DSA_ERR_CUDA;
   }
   if (ensure_smem<dsa::up_proj_kernel>(C::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
+  NvtxRange range("dsa.up_proj");
   const dim3 grid(C::H, static_cast<unsigned>((n_rows + C::BM - 1) / C::BM));
   dsa::up_proj_kernel<<<grid, C::NT, C::SMEM_BYTES, stream>>>(tm_o, tm_w, static_cast<__nv_bfloat16*>(y), n_rows);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

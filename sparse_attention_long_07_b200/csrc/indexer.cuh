@@ -55,11 +55,13 @@ struct IndexerCfg {
   static constexpr int NATOM = ROWB / SWB;                // swizzle-atom columns per row
   static constexpr int ATOM_ELEMS = SWB / ELEM;
   static constexpr int KSTEPS = ROWB / 32;                // 32 bytes of K per MMA (16 bf16 or 32 e4m3)
-  // Persistent schedule: the widened bf16 key tile is written to tensor memory
-  // and read from there as the A operand (TS-form MMA), so shared memory holds
-  // only the raw e4m3 ring; otherwise the bf16 tile ring is in shared memory.
-  static constexpr bool K_IN_TMEM = PERSIST;
-  static constexpr int STAGES = K_IN_TMEM ? 4 : (CONVERT ? 2 : 4);  // key-tile ring (MMA operand)
+  // Persistent schedule with bf16 queries: the widened bf16 key tile is
+  // written to tensor memory and read from there as the A operand (TS-form
+  // MMA), so shared memory holds only the raw e4m3 ring; otherwise the key
+  // tile ring (bf16, or e4m3 as loaded for the FP8 indexer) is in shared
+  // memory, twelve deep for the persistent FP8 schedule.
+  static constexpr bool K_IN_TMEM = PERSIST && CONVERT;
+  static constexpr int STAGES = K_IN_TMEM ? 4 : (PERSIST ? 12 : (CONVERT ? 2 : 4));  // key-tile ring (MMA operand)
   static constexpr int RSTAGES = CONVERT ? (PERSIST ? 11 : 4) : 0;  // raw e4m3 ring (to widen)
   static constexpr int A_TILE = BK * ROWB;
   static constexpr int B_TILE = N * ROWB;
@@ -95,7 +97,10 @@ struct IndexerCfg {
   static constexpr int OFF_RAW = OFF_K + (K_IN_TMEM ? 0 : STAGES * A_TILE);
   static constexpr int OFF_W = OFF_RAW + RSTAGES * RAW_TILE;
   static constexpr int OFF_BAR = OFF_W + NQ * H_I * 4;
-  static constexpr int NBAR = 2 + 2 * STAGES + 2 * RSTAGES + 2 * NACC + 1;
+  // barriers: grid schedule 2 + 2 STAGES + 2 RSTAGES + 2 NACC; persistent
+  // schedule 7 + STAGES (ready) + 2 RSTAGES + NACC (acc_full) + 2 STAGES
+  // (k_full, k_empty) + NACC (acc_empty), every array reserved in both forms
+  static constexpr int NBAR = 7 + 3 * STAGES + 2 * RSTAGES + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_UPRE = OFF_MISC + 16;          // persistent: unit prefix per sequence
   // persistent: per-warp head weights, read as float4 (16-byte aligned)
@@ -105,11 +110,12 @@ struct IndexerCfg {
   static_assert(B_TILE % 1024 == 0 && A_TILE % 1024 == 0, "atom alignment");
   static_assert(COLS_PER_THREAD % LD_CHUNK == 0, "TMEM load chunking");
   static_assert(!KFP8 || D_I == 128, "e4m3 keys: 128-byte rows");
-  static_assert(!QFP8 || (KFP8 && !PERSIST && D_I == 128), "FP8 indexer: e4m3 keys, query-block grid, 128-byte rows");
+  static_assert(!QFP8 || (KFP8 && D_I == 128), "FP8 indexer: e4m3 keys, 128-byte rows");
   static_assert(TMEM_COLS <= 512, "tensor memory columns");
   static_assert(!K_IN_TMEM || (KFP8 && STAGES % CONV_TEAMS == 0), "converter teams own alternate stages");
   static_assert(NACC % EPI_WG == 0, "each accumulator is drained by one epilogue warpgroup");
-  static_assert(!PERSIST || 7 + STAGES + 2 * RSTAGES + NACC <= NBAR, "persistent barrier layout");
+  static_assert(2 + 2 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "grid barrier layout");
+  static_assert(!PERSIST || 7 + 3 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "persistent barrier layout");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(!K_IN_TMEM || STAGES == NACC, "key stage and accumulator of a tile share one barrier");
   static_assert(!PERSIST || NQ == 1, "persistent schedule: one query per sequence block");
@@ -181,6 +187,7 @@ struct IndexerParams {
   const float* q_scale;      // [T, H_I] (FP8 indexer) or null
   const float* k_scale;      // [cache rows] (e4m3 keys) or null
   PageMap pages;             // where the caches keep each entry
+  int cache_rows;            // rows of the index-key cache (checked builds)
   const int32_t* cu_q;
   const int32_t* cu_k;
   int B;
@@ -307,7 +314,9 @@ __global__ void __launch_bounds__(C::NT, 1)
         int y[C::BK / 64];
 #pragma unroll
         for (int h = 0; h < C::BK / 64; ++h) {
-          const int r = p.pages.row(b, k_base, s0 + 64 * h);
+          // (a box that starts past the sequence is never read: its scores are masked)
+          int r = p.pages.row(b, k_base, s0 + 64 * h);
+          if (r >= 0 && s0 + 64 * h < kv_len && !in_bounds(r < p.cache_rows, 81)) r = -1;
           y[h] = r >= 0 ? r : -64;
         }
         const int nbox = p.pages.paged() ? C::BK / 64 : 1;
@@ -374,8 +383,9 @@ __global__ void __launch_bounds__(C::NT, 1)
       while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < kWaitLimitCycles) {
       }
     }
-  } else if (C::CONVERT && warp >= C::CONVERT_WARP0) {
+  } else if (warp >= C::CONVERT_WARP0) {
     // ------------------------------------------------------------ e4m3 -> bf16
+    // (bf16 queries only: the FP8 schedule has no converter warps)
     if constexpr (C::CONVERT) {
     const int row = threadIdx.x - C::CONVERT_WARP0 * 32;  // key row of the tile
     for (int it = 0; it < n_iter; ++it) {
@@ -427,7 +437,7 @@ __global__ void __launch_bounds__(C::NT, 1)
           kscale = p.k_scale[k_base + s];
         } else {
           const int r = p.pages.row(b, k_base, s);
-          kscale = r >= 0 ? p.k_scale[r] : 0.f;
+          kscale = (r >= 0 && in_bounds(r < p.cache_rows, 85)) ? p.k_scale[r] : 0.f;
         }
       }
 #pragma unroll
@@ -437,7 +447,7 @@ __global__ void __launch_bounds__(C::NT, 1)
           // keys past the query's position (and past the cache) score -inf
           const float val = s <= pos0 + qi ? acc[q] * kscale : -INFINITY;
           const int64_t row = q0 + qi - p.q_begin;
-          if (in_seq) p.scores[row * p.ld + s] = val;
+          if (in_seq && in_bounds(s < p.ld, 83)) p.scores[row * p.ld + s] = val;
           if (p.part_max != nullptr) {
             const float m = part_max8(val);
             if ((lane & (PART - 1)) == 0 && in_seq) p.part_max[row * p.ld_pm + s / PART] = m;
@@ -466,6 +476,9 @@ __global__ void __launch_bounds__(C::NT, 1)
     indexer_persistent_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k, const IndexerParams p) {
   static_assert(C::PERSIST && C::KFP8 && C::NQ == 1, "persistent path: e4m3 keys, one query per block");
+  // bf16 queries: e4m3 key tiles are widened into tensor memory by converter
+  // warps.  FP8 indexer (QFP8): the e4m3 key tiles go from the TMA ring
+  // straight into kind::f8f6f4 MMAs; no converter warps.
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   int* upre = reinterpret_cast<int*>(smem + C::OFF_UPRE);      // upre[b] = first unit of sequence b
@@ -526,6 +539,7 @@ __global__ void __launch_bounds__(C::NT, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t s_q = sbase + C::OFF_Q;
   const uint32_t s_raw = sbase + C::OFF_RAW;
+  const uint32_t s_k = sbase + C::OFF_K;
   const uint32_t bar0 = sbase + C::OFF_BAR;
   const uint32_t bar_drain = bar0;
   // query tile of segment g (the g-th sequence of this CTA) in buffer g & 1:
@@ -539,6 +553,10 @@ __global__ void __launch_bounds__(C::NT, 1)
   auto bar_raw_full = [&](int s) { return bar0 + 56 + 8 * (C::STAGES + s); };
   auto bar_raw_empty = [&](int s) { return bar0 + 56 + 8 * (C::STAGES + C::RSTAGES + s); };
   auto bar_acc_full = [&](int a) { return bar0 + 56 + 8 * (C::STAGES + 2 * C::RSTAGES + a); };
+  // FP8 indexer: key ring full / empty, accumulator drained by the epilogue
+  auto bar_k_full = [&](int s) { return bar0 + 56 + 8 * (C::STAGES + 2 * C::RSTAGES + C::NACC + s); };
+  auto bar_k_empty = [&](int s) { return bar0 + 56 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + C::NACC + s); };
+  auto bar_acc_empty = [&](int a) { return bar0 + 56 + 8 * (3 * C::STAGES + 2 * C::RSTAGES + C::NACC + a); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -548,16 +566,25 @@ __global__ void __launch_bounds__(C::NT, 1)
       mbar_init(bar_q_full(buf), 1);
       for (int t = 0; t < C::MMA_THREADS; ++t) mbar_init(bar_q_empty(t, buf), 1);
     }
-    for (int s = 0; s < C::STAGES; ++s) mbar_init(bar_ready(s), 256);
-    for (int s = 0; s < C::RSTAGES; ++s) {
-      mbar_init(bar_raw_full(s), 1);
-      mbar_init(bar_raw_empty(s), 128);
+    if constexpr (C::CONVERT) {
+      for (int s = 0; s < C::STAGES; ++s) mbar_init(bar_ready(s), 256);
+      for (int s = 0; s < C::RSTAGES; ++s) {
+        mbar_init(bar_raw_full(s), 1);
+        mbar_init(bar_raw_empty(s), 128);
+      }
+    } else {
+      for (int s = 0; s < C::STAGES; ++s) {
+        mbar_init(bar_k_full(s), 1);
+        mbar_init(bar_k_empty(s), 1);
+      }
+      for (int a = 0; a < C::NACC; ++a) mbar_init(bar_acc_empty(a), 128);
     }
     for (int a = 0; a < C::NACC; ++a) mbar_init(bar_acc_full(a), 1);
     *abort_flag = 0;
     fence_mbar_init();
     // every accumulator starts drained: the epilogue's share of the first phase
-    for (int s = 0; s < C::STAGES; ++s) mbar_arrive_count(bar_ready(s), 128);
+    if constexpr (C::CONVERT)
+      for (int s = 0; s < C::STAGES; ++s) mbar_arrive_count(bar_ready(s), 128);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -598,22 +625,29 @@ __global__ void __launch_bounds__(C::NT, 1)
           loaded_q = seg + 1;
         }
         const int tile = u - upre[b];
-        const int r = it % C::RSTAGES;
-        if (!mbar_wait(bar_raw_empty(r), ((it / C::RSTAGES) & 1) ^ 1, abort_flag, 51)) break;
-        mbar_arrive_expect_tx(bar_raw_full(r), C::RAW_TILE);
+        // the raw ring (widened by the converters) or the key ring (FP8 MMA operand)
+        constexpr int ring = C::CONVERT ? C::RSTAGES : C::STAGES;
+        const int r = it % ring;
+        const uint32_t full = C::CONVERT ? bar_raw_full(r) : bar_k_full(r);
+        const uint32_t empty = C::CONVERT ? bar_raw_empty(r) : bar_k_empty(r);
+        const uint32_t dst = C::CONVERT ? s_raw + r * C::RAW_TILE : s_k + r * C::A_TILE;
+        if (!mbar_wait(empty, ((it / ring) & 1) ^ 1, abort_flag, 51)) break;
+        mbar_arrive_expect_tx(full, C::RAW_TILE);
         if (!p.pages.paged()) {
-          tma_load_2d(s_raw + r * C::RAW_TILE, &tm_k, bar_raw_full(r), 0, q.k_base + tile * C::BK);
+          tma_load_2d(dst, &tm_k, full, 0, q.k_base + tile * C::BK);
         } else {
           for (int h = 0; h < C::BK / 64; ++h) {   // 64-row boxes, each inside one page
-            const int y = p.pages.row(q.b, q.k_base, tile * C::BK + 64 * h);
-            tma_load_2d(s_raw + r * C::RAW_TILE + h * 64 * C::RAW_ROWB, &tm_k, bar_raw_full(r), 0, y >= 0 ? y : -64);
+            int y = p.pages.row(q.b, q.k_base, tile * C::BK + 64 * h);
+            if (y >= 0 && tile * C::BK + 64 * h < q.kv_len && !in_bounds(y < p.cache_rows, 82)) y = -1;
+            tma_load_2d(dst + h * 64 * C::RAW_ROWB, &tm_k, full, 0, y >= 0 ? y : -64);
           }
         }
       }
       if (*abort_flag) {
         long long t0 = clock64();
-        for (int j = (it > C::RSTAGES ? it - C::RSTAGES : 0); j < it; ++j)
-          while (!mbar_try_wait(bar_raw_full(j % C::RSTAGES), (j / C::RSTAGES) & 1) &&
+        constexpr int ring = C::CONVERT ? C::RSTAGES : C::STAGES;
+        for (int j = (it > ring ? it - ring : 0); j < it; ++j)
+          while (!mbar_try_wait(C::CONVERT ? bar_raw_full(j % ring) : bar_k_full(j % ring), (j / ring) & 1) &&
                  clock64() - t0 < kWaitLimitCycles) {
           }
         for (int g = (loaded_q > 2 ? loaded_q - 2 : 0); g < loaded_q; ++g)
@@ -659,22 +693,40 @@ __global__ void __launch_bounds__(C::NT, 1)
           have_q = true;
           b_desc = b_desc0 + static_cast<uint64_t>(((seg & 1) * C::B_TILE) >> 4);
         }
-        const int s = it % C::STAGES;
-        const int a = s;
-        if (!mbar_wait(bar_ready(s), (it / C::STAGES) & 1, abort_flag, 53)) { ok = false; break; }
-        tc_fence_after();
-        // A: the key tile in tensor memory, 8 columns (16 bf16) per k-step.
-        // B: the query descriptor's start-address field (16-byte units, low
-        // bits) advances by the k-step offset; it never carries.
-        const uint32_t a_tile = tmem + C::ACC_COLS + s * C::A_COLS;
+        if constexpr (C::CONVERT) {
+          const int s = it % C::STAGES;
+          const int a = s;
+          if (!mbar_wait(bar_ready(s), (it / C::STAGES) & 1, abort_flag, 53)) { ok = false; break; }
+          tc_fence_after();
+          // A: the key tile in tensor memory, 8 columns (16 bf16) per k-step.
+          // B: the query descriptor's start-address field (16-byte units, low
+          // bits) advances by the k-step offset; it never carries.
+          const uint32_t a_tile = tmem + C::ACC_COLS + s * C::A_COLS;
 #pragma unroll
-        for (int kk = 0; kk < C::KSTEPS; ++kk) {
-          const int atom = (kk * 32) / C::SWB;
-          const int off = (kk * 32) % C::SWB;
-          const uint64_t bd = b_desc + static_cast<uint64_t>((atom * C::N * C::SWB + off) >> 4);
-          umma_ts(tmem + a * C::N, a_tile + kk * 8, bd, C::IDESC, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::KSTEPS; ++kk) {
+            const int atom = (kk * 32) / C::SWB;
+            const int off = (kk * 32) % C::SWB;
+            const uint64_t bd = b_desc + static_cast<uint64_t>((atom * C::N * C::SWB + off) >> 4);
+            umma_ts(tmem + a * C::N, a_tile + kk * 8, bd, C::IDESC, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_acc_full(a));   // also frees key stage s (== a)
+        } else {
+          // FP8 indexer: A = the e4m3 key tile as loaded (128 rows of 128
+          // bytes, 128-byte swizzle), B = the e4m3 query tile; 32 bytes of K
+          // per MMA, the start addresses advance inside the swizzle atom.
+          const int s = it % C::STAGES;
+          const int a = it % C::NACC;
+          if (!mbar_wait(bar_k_full(s), (it / C::STAGES) & 1, abort_flag, 53)) { ok = false; break; }
+          if (!mbar_wait(bar_acc_empty(a), ((it / C::NACC) & 1) ^ 1, abort_flag, 54)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t a_desc = smem_desc(s_k + s * C::A_TILE, 16, 8 * C::SWB, C::SWZ);
+#pragma unroll
+          for (int kk = 0; kk < C::KSTEPS; ++kk)
+            umma_ss_e4m3(tmem + a * C::N, a_desc + static_cast<uint64_t>((kk * 32) >> 4),
+                         b_desc + static_cast<uint64_t>((kk * 32) >> 4), C::IDESC, kk > 0 ? 1u : 0u);
+          umma_commit(bar_k_empty(s));
+          umma_commit(bar_acc_full(a));
         }
-        umma_commit(bar_acc_full(a));   // also frees key stage s (== a)
       }
       // release the current segment and every later one of the CTA
       while (ok && !*abort_flag) {
@@ -690,6 +742,8 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
   } else if (warp >= C::CONVERT_WARP0) {
     // ------------------------------------------------------------ e4m3 -> bf16
+    // (bf16 queries only: the FP8 schedule has no converter warps)
+    if constexpr (C::CONVERT) {
     // Each thread widens one key row into its own TMEM lane: a warp reaches
     // lanes 32 (warp % 4) .. +31, so the row is fixed by the warp's position.
     const int team = (warp - C::CONVERT_WARP0) / 4;
@@ -726,6 +780,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       tc_fence_before();
       mbar_arrive_warp(bar_ready(s));
     }
+    }
     if (lane == 0) DSA_PROF_SPAN(63, t_role);
   } else {
     // ------------------------------------------------------------ epilogue
@@ -745,7 +800,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       const int s_key = (u - upre[bp]) * C::BK + key_in_tile;
       if (s_key >= p.cu_k[bp + 1] - kb) return 0.f;
       const int r = p.pages.row(bp, kb, s_key);
-      return r >= 0 ? p.k_scale[r] : 0.f;
+      return (r >= 0 && in_bounds(r < p.cache_rows, 86)) ? p.k_scale[r] : 0.f;
     };
     float ks = fetch_scale(g);
     for (int it = g; it < n_iter; it += C::EPI_WG) {
@@ -758,7 +813,17 @@ __global__ void __launch_bounds__(C::NT, 1)
         q = seq_of(b);
         __syncwarp();
         const float4* w4 = reinterpret_cast<const float4*>(p.w + static_cast<int64_t>(q.q0) * C::H_I);
-        if (lane < C::H_I / 4) reinterpret_cast<float4*>(wsm)[lane] = w4[lane];
+        if (lane < C::H_I / 4) {
+          float4 wv = w4[lane];
+          if constexpr (C::QFP8) {   // fold in each query head's scale and the 2^-7 of the rotation
+            const float* qs = p.q_scale + static_cast<int64_t>(q.q0) * C::H_I + 4 * lane;
+            wv.x *= ldexpf(qs[0], -FP8_HADAMARD_LOG2);
+            wv.y *= ldexpf(qs[1], -FP8_HADAMARD_LOG2);
+            wv.z *= ldexpf(qs[2], -FP8_HADAMARD_LOG2);
+            wv.w *= ldexpf(qs[3], -FP8_HADAMARD_LOG2);
+          }
+          reinterpret_cast<float4*>(wsm)[lane] = wv;
+        }
         __syncwarp();
       }
       if (!mbar_wait_warp(bar_acc_full(a), (it / C::NACC) & 1, abort_flag, 57)) break;
@@ -780,12 +845,13 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive_warp(bar_ready(a));   // accumulator a is free for tile it + NACC
+      if constexpr (C::CONVERT) mbar_arrive_warp(bar_ready(a));   // accumulator a is free for tile it + NACC
+      else mbar_arrive_warp(bar_acc_empty(a));
       const int s_key = (u - upre[b]) * C::BK + key_in_tile;
       // keys past the query's position (and past the cache) score -inf
       const float val = s_key <= q.pos ? (acc0 + acc1) * ks : -INFINITY;
       const int64_t row = static_cast<int64_t>(q.q0) - p.q_begin;
-      if (s_key < q.kv_len) p.scores[row * p.ld + s_key] = val;
+      if (s_key < q.kv_len && in_bounds(s_key < p.ld, 84)) p.scores[row * p.ld + s_key] = val;
       if (p.part_max != nullptr) {
         const float m = part_max8(val);
         if ((lane & (PART - 1)) == 0 && s_key < q.kv_len) p.part_max[row * p.ld_pm + s_key / PART] = m;

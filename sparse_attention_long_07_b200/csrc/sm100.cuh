@@ -18,6 +18,7 @@ __device__ int g_device_error;
 enum DeviceErrorCode : int {
   kErrWaitTimeout = 1,      // an mbarrier wait exceeded its limit; bits 8.. hold the wait site
   kErrMissingPage = 2,      // a paged cache entry that was needed had no valid page; bits 8.. hold the site
+  kErrBounds = 3,           // checked builds: an index or coordinate outside its buffer (access skipped)
 };
 
 #ifdef DSA_PROFILE_WAITS
@@ -66,6 +67,21 @@ constexpr long long kWaitLimitCycles = 4000000000LL;
 
 __device__ __forceinline__ void record_device_error(int code) {
   atomicCAS(&g_device_error, 0, code);
+}
+
+// Checked builds (-DDSA_DEBUG): in_bounds(ok, site) records kErrBounds at the
+// site when ok is false, and the caller skips the access.  Other builds
+// compile the check away (the host validation and the kernels' own index
+// arithmetic keep every access inside its buffer).
+__device__ __forceinline__ bool in_bounds(bool ok, int site) {
+#ifdef DSA_DEBUG
+  if (!ok) record_device_error(kErrBounds | (site << 8));
+  return ok;
+#else
+  (void)ok;
+  (void)site;
+  return true;
+#endif
 }
 
 // ----------------------------------------------------------------------------

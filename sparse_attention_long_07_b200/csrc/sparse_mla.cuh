@@ -130,6 +130,7 @@ struct MlaParams {
   const int32_t* cu_q;
   const int32_t* cu_k;
   PageMap pages;             // where the latent cache keeps each entry
+  int cache_rows;            // rows of the latent cache (checked builds)
   int B;
   int64_t q_begin;
   int topk;
@@ -143,10 +144,11 @@ struct MlaParams {
 // skipped: outside 0 .. pos (the -1 padding included), or (paged caches) on
 // a missing page, which is also recorded in the device error word.  Skipped
 // entries are gathered from row 0 and masked.
-__device__ __forceinline__ int gather_row(const PageMap& pages, const RowInfo& ri, int sel) {
+__device__ __forceinline__ int gather_row(const PageMap& pages, const RowInfo& ri, int sel, int cache_rows) {
   if (sel < 0 || sel > ri.pos) return -1;
   const int r = pages.row(ri.b, ri.k_base, sel);
   if (r < 0) record_device_error(kErrMissingPage | (23 << 8));
+  if (r >= 0 && !in_bounds(r < cache_rows, 80)) return -1;
   return r;
 }
 
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         if (!ok) break;
         const int e = it * C::BN + lane;
         const int sel = e < p.topk ? idx_row[e] : -1;
-        const int grow = gather_row(p.pages, ri, sel);
+        const int grow = gather_row(p.pages, ri, sel, p.cache_rows);
         const bool valid = grow >= 0;
         const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, valid);
         int y[4];
@@ -309,7 +311,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         if (!ok) break;
         const int e = it * C::BN + lane;
         const int sel = e < p.topk ? idx_row[e] : -1;
-        const int grow = gather_row(p.pages, ri, sel);
+        const int grow = gather_row(p.pages, ri, sel, p.cache_rows);
         const bool valid = grow >= 0;
         int y[4];
 #pragma unroll

@@ -260,30 +260,10 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     __syncthreads();
   };
 
-  // Block-wide sums and scans.  Each warp reduces with redux/shuffles, warp 0
-  // combines the 16 warp values, and every thread reads back one word, so a
-  // call costs two barriers and a couple of shared loads per thread.
-  // red_sum2(a, b): the CTA totals of a and b (each total < 2^16).
+  // Block-wide scan.  Each warp scans with shuffles, warp 0 combines the 16
+  // warp totals, and every thread reads back one word, so a call costs two
+  // barriers and a couple of shared loads per thread.
   uint32_t red_phase = 0;   // alternates the result words between calls
-  auto red_sum2 = [&](uint32_t a, uint32_t b) -> uint2 {
-    const uint32_t w2 = __reduce_add_sync(0xFFFFFFFFu, a | (b << 16));   // per-warp sums stay < 2^16
-    uint32_t* sl = cnt;
-    uint32_t* res = cnt + 32 + (red_phase & 1u) * 2;
-    ++red_phase;
-    if (lane == 0) sl[warp] = w2;
-    __syncthreads();
-    if (warp == 0) {
-      const uint32_t v = lane < static_cast<uint32_t>(C::NW) ? sl[lane] : 0u;
-      const uint32_t lo = __reduce_add_sync(0xFFFFFFFFu, v & 0xFFFFu);
-      const uint32_t hi = __reduce_add_sync(0xFFFFFFFFu, v >> 16);
-      if (lane == 0) {
-        res[0] = lo;
-        res[1] = hi;
-      }
-    }
-    __syncthreads();
-    return make_uint2(res[0], res[1]);
-  };
   // block_scan(v, &total): exclusive prefix of v over the threads in order.
   auto block_scan = [&](uint32_t v, uint32_t* total) -> uint32_t {
     uint32_t wt;
@@ -304,78 +284,51 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     *total = wpre[C::NW];
     return wpre[warp] + pre;
   };
-  // Radix-4 selection.  select(count, key_of, use, kth, &thr, &rem, steps):
+  // Radix-256 selection.  select(count, key_of, use, kth, &thr, &rem, steps):
   // the kth largest key among the entries i < count with use(i) (at least kth
-  // of them), found 2 bits at a time from the top: each step counts, for the
-  // 3 candidate values of the next digit, the entries at or above them and
-  // keeps the largest digit with at least kth entries at or above it.  No
-  // atomics, so concentrated key distributions cost nothing extra.  Up to
-  // SEL_REG entries per thread are read once into registers.  With steps <
-  // 16 only the top 2*steps bits are resolved and the lower bits are 0: thr
-  // is then a lower bound of the kth largest key with at least kth entries
-  // >= thr.  *rem = kth - (entries > thr) (meaningful for steps = 16).
-  // Called by every thread; counts stay below 2^16 (count <= 65535).
+  // of them), found 8 bits at a time from the top.  Each pass builds a
+  // 256-bin histogram of the next digit over the entries that share the
+  // digits found so far (warp-aggregated shared atomics), and one CTA scan of
+  // the bins (find_digit_fn) gives the digit holding the kth entry and the
+  // entries above it.  steps counts 2-bit steps: steps = 16 resolves all 32
+  // bits; with steps = 8 only the top 16 bits are resolved and the lower bits
+  // are 0, so thr is then a lower bound of the kth largest key with at least
+  // kth entries >= thr.  *rem = kth - (entries > thr) (meaningful for steps =
+  // 16).  Called by every thread (three barriers per pass).
   auto select = [&](uint32_t count, auto&& key_of, auto&& use, uint32_t kth, uint32_t* out_thr,
                     uint32_t* out_rem, int steps = 16) {
-    constexpr int SEL_REG = 12;
-    const bool in_regs = count <= static_cast<uint32_t>(SEL_REG * C::NT);
-    uint32_t kr[SEL_REG];   // this thread's keys (entries tid, tid + NT, ...)
-    uint32_t ur = 0;        // bit e: entry e is used
-#pragma unroll
-    for (int e = 0; e < SEL_REG; ++e) {
-      const uint32_t i = tid + static_cast<uint32_t>(e) * C::NT;
-      kr[e] = 0u;
-      if (in_regs && i < count && use(i)) {
-        kr[e] = key_of(i);
-        ur |= 1u << e;
+    uint32_t* h = hist;                 // 256 bins (the first words of the pass-1 histogram)
+    uint32_t prefix = 0, need = kth;    // need: rank of the target among the entries matching prefix
+    const int passes = steps / 4;
+    for (int d = 0; d < passes; ++d) {
+      const int shift = 24 - 8 * d;
+      const uint32_t hi_mask = d == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
+      if (tid < 256) h[tid] = 0u;
+      __syncthreads();
+      for (uint32_t base = 0; base < count; base += C::NT) {   // uniform trip count: whole warps call hist_add
+        const uint32_t i = base + tid;
+        bool valid = i < count && use(i);
+        const uint32_t k = valid ? key_of(i) : 0u;
+        valid = valid && (k & hi_mask) == prefix;
+        hist_add(h, (k >> shift) & 0xFFu, valid);
       }
-    }
-    uint32_t prefix = 0;
-    for (int st = 0; st < steps; ++st) {
-      const int shift = 30 - 2 * st;
-      const uint32_t t1 = prefix | (1u << shift), t2 = prefix | (2u << shift), t3 = prefix | (3u << shift);
-      uint32_t c1 = 0, c2 = 0, c3 = 0;
-      if (in_regs) {
-#pragma unroll
-        for (int e = 0; e < SEL_REG; ++e) {
-          const uint32_t k = kr[e];
-          const uint32_t u = (ur >> e) & 1u;
-          c1 += u & (k >= t1 ? 1u : 0u);
-          c2 += u & (k >= t2 ? 1u : 0u);
-          c3 += u & (k >= t3 ? 1u : 0u);
-        }
-      } else {
-        for (uint32_t i = tid; i < count; i += C::NT) {
-          if (!use(i)) continue;
-          const uint32_t k = key_of(i);
-          c1 += k >= t1 ? 1u : 0u;
-          c2 += k >= t2 ? 1u : 0u;
-          c3 += k >= t3 ? 1u : 0u;
-        }
-      }
-      // c1 >= c2 >= c3: the digit is the number of thresholds still reached
-      const uint2 s12 = red_sum2(c1, c2);
-      uint32_t digit = (s12.x >= kth ? 1u : 0u) + (s12.y >= kth ? 1u : 0u);
-      if (digit == 2u) digit += red_sum2(c3, 0u).x >= kth ? 1u : 0u;   // block-uniform branch
-      prefix |= digit << shift;
-    }
-    uint32_t gt = 0;
-    if (steps == 16) {
-      if (in_regs) {
-#pragma unroll
-        for (int e = 0; e < SEL_REG; ++e) gt += ((ur >> e) & 1u) & (kr[e] > prefix ? 1u : 0u);
-      } else {
-        for (uint32_t i = tid; i < count; i += C::NT) gt += (use(i) && key_of(i) > prefix) ? 1u : 0u;
-      }
+      __syncthreads();
+      find_digit_fn(h, 256, need, &misc[4], &misc[5]);
+      prefix |= misc[4] << shift;
+      need -= misc[5];
+      __syncthreads();   // every thread has read misc[4..5] before the next pass writes them
     }
     *out_thr = prefix;
-    *out_rem = kth - red_sum2(gt, 0u).x;
+    *out_rem = need;
   };
   // Exact selection among candidates ckey/cidx[0, nc) that hold every key
   // >= some bound b with at least topk keys >= b: the topk largest keys, ties
-  // to the lowest index, written in increasing index order through a bitmap
-  // of the row (n <= BITMAP_BITS).  Called by every thread.
-  auto finish_candidates = [&](uint32_t nc) {
+  // to the lowest index.  ordered: the candidates sit in an order that does
+  // not depend on timing, and the chosen ones are written in that order;
+  // otherwise (candidates placed by atomics) they are written in increasing
+  // index order through a bitmap of the row (n <= BITMAP_BITS), so repeated
+  // runs agree either way.  Called by every thread.
+  auto finish_candidates = [&](uint32_t nc, bool ordered) {
     uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + C::OFF_BITMAP);
     uint32_t thr, need_eq;
     select(nc, [&](uint32_t i) { return ckey[i]; }, [&](uint32_t) { return true; },
@@ -390,16 +343,28 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
       select(nc, [&](uint32_t i) { return ~static_cast<uint32_t>(cidx[i]); },
              [&](uint32_t i) { return ckey[i] == thr; }, need_eq, &inv_idx_thr, &rem2);
     }
+    auto chosen = [&](uint32_t i) {
+      const uint32_t key = ckey[i];
+      return key > thr || (key == thr && ~static_cast<uint32_t>(cidx[i]) >= inv_idx_thr);
+    };
+    if (ordered) {
+      // candidates in a deterministic order: compact the chosen ones in that order
+      uint32_t mine = 0, unused_total;
+      for (uint32_t i = tid; i < nc; i += C::NT) mine += chosen(i) ? 1u : 0u;
+      uint32_t pos_out = block_scan(mine, &unused_total);
+      for (uint32_t i = tid; i < nc; i += C::NT)
+        if (chosen(i)) {
+          if (in_bounds(pos_out < static_cast<uint32_t>(topk), 88)) out[pos_out] = cidx[i];
+          ++pos_out;
+        }
+      return;
+    }
     // ---- selection -> bitmap -> indices in increasing order
     const int nwords = (n + 31) / 32;
     for (int i = tid; i < nwords; i += C::NT) bitmap[i] = 0u;
     __syncthreads();
-    for (uint32_t i = tid; i < nc; i += C::NT) {
-      const uint32_t key = ckey[i];
-      const int id = cidx[i];
-      if (key > thr || (key == thr && ~static_cast<uint32_t>(id) >= inv_idx_thr))
-        atomicOr(&bitmap[id >> 5], 1u << (id & 31));
-    }
+    for (uint32_t i = tid; i < nc; i += C::NT)
+      if (chosen(i)) atomicOr(&bitmap[cidx[i] >> 5], 1u << (cidx[i] & 31));
     __syncthreads();
     const int per = (nwords + C::NT - 1) / C::NT;
     const int w0 = min(nwords, static_cast<int>(tid) * per), w1 = min(nwords, w0 + per);
@@ -411,7 +376,8 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
       while (bits) {
         const int bpos = __ffs(bits) - 1;
         bits &= bits - 1;
-        out[pos_out++] = wdx * 32 + bpos;
+        if (in_bounds(pos_out < static_cast<uint32_t>(topk), 90)) out[pos_out] = wdx * 32 + bpos;
+        ++pos_out;
       }
     }
   };
@@ -429,8 +395,8 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
   // the bitmap, or candidate overflows (massive ties) take the paths below.
   if (part_max != nullptr && n <= C::BITMAP_BITS) {
     const int P = (n + PART - 1) / PART;
-    // Groups of G2 parts: about 2 k to 4 k groups keep the selection cheap
-    // (its cost grows with the groups) while the candidates stay near k.
+    // Groups of G2 parts (a power of two): about 2 k to 4 k groups keep the
+    // selection over the group maxima short while the candidates stay near k.
     int G2 = 1;
     while ((P + 2 * G2 - 1) / (2 * G2) >= 2 * topk || (P + G2 - 1) / G2 > C::PM_CAP) G2 <<= 1;
     const int Pg = (P + G2 - 1) / G2;
@@ -560,7 +526,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
           }
           __syncthreads();
           phase(49);
-          finish_candidates(nc);
+          finish_candidates(nc, true);
           phase(45);
           DSA_PROF_END();
           return;
@@ -694,7 +660,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
       if (!ok) { DSA_PROF_END(); return; }
       const uint32_t nc = *cand_n;
       if (nc <= static_cast<uint32_t>(C::CAP)) {
-        finish_candidates(nc);
+        finish_candidates(nc, false);
         phase(45);
         DSA_PROF_END();
         return;
@@ -747,7 +713,9 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
           gt = b > bin_b;
           eq = b == bin_b;
         },
-        [&](uint32_t rank, int gi, uint32_t) { out[rank] = gi; },
+        [&](uint32_t rank, int gi, uint32_t) {
+          if (in_bounds(rank < static_cast<uint32_t>(topk), 89)) out[rank] = gi;
+        },
         [&](uint32_t rank, int gi, uint32_t key) {
           if (rank < static_cast<uint32_t>(C::CAP)) {
             ckey[rank] = key;

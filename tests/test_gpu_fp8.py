@@ -67,9 +67,11 @@ def test_hadamard_quantize_matches_the_oracle(dsa, oracle_lib):
 
 
 @pytest.mark.parametrize("q_lens,kv_lens", [
-    ((1, 1, 1, 1, 1), (1, 129, 1000, 4097, 20000)),     # decode-like: one query per block
+    ((1, 1, 1, 1, 1), (1, 129, 1000, 4097, 20000)),     # decode: the persistent schedule
+    ((1,) * 8, (20000, 130, 65536, 1, 7000, 128, 129, 30000)),   # decode: sequences split across CTAs
+    ((2, 1), (3000, 500)),                              # decode-like blocks of one query (grid)
     ((37, 3, 130), (600, 128, 2200)),                   # prefill blocks of four queries, ragged tails
-], ids=["decode", "prefill"])
+], ids=["decode", "decode-long", "decode-grid", "prefill"])
 def test_fp8_indexer_scores_match_the_oracle(dsa, oracle_lib, q_lens, kv_lens):
     spec = di.Spec("fp8", tuple(q_lens), tuple(kv_lens), seed=31, **RELEASED)
     d = di.make_inputs(spec, tensors=("q_idx", "w", "k_idx"))

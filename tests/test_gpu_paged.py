@@ -164,6 +164,7 @@ CASES = [
     ("prefill-e4m3", (40, 3), (700, 2600), True, False),             # grid indexer, 4 queries per CTA
     ("prefill-bf16", (1, 30), (3000, 900), False, False),            # bf16 keys
     ("fp8-indexer", (1, 9), (2500, 1300), True, True),               # e4m3 queries and keys
+    ("fp8-decode", (1, 1, 1), (300, 5000, 2049), True, True),        # persistent FP8 indexer
 ]
 
 

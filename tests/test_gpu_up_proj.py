@@ -2,7 +2,8 @@
 transformers doc, DSA: MLA with latents shared by all heads; released config
 kv_lora_rank 512, v_head_dim 128, n_heads 128) against the oracle.
 
-Bound per element: the bf16 rounding of y (half an ulp, 2^-9 relative) plus the
+Bound per element: the bf16 rounding of y (half an ulp: bf16 carries 8
+significant bits, so at most 2^-8 relative) plus the
 accumulation of 512 exact products in fp32 by the tensor core, which adds
 products in groups aligned to the largest exponent and truncates: at most two
 fp32 ulps (2^-22) of the running magnitude per addition, 512 * 2^-22 * sum_c
@@ -37,7 +38,7 @@ def test_up_proj_matches_the_oracle(dsa, oracle_lib, n):
     got = y_full[:n].float().cpu().numpy().astype(np.float64)
     ref = oracle_lib.up_proj(o, w)
     mag = np.einsum("rhc,hce->rhe", np.abs(o.double().numpy()), np.abs(w.double().numpy()))
-    bound = 2.0 ** -9 * np.abs(ref) + 2.0 ** -13 * mag + 1e-30
+    bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -13 * mag + 1e-30
     err = np.abs(got - ref)
     P._margin("up-projection", float((err / bound).max()))
     assert np.all(err <= bound), f"worst {float((err / bound).max()):.3f} of the bound"
