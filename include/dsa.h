@@ -144,7 +144,7 @@ dsa_status dsa_indexer_scores(const void* q_idx, const float* q_scale, const flo
  *           dsa_indexer_scores (only columns 0..pos(t) are read)
  * part_max  NULL, or the part maxima dsa_indexer_scores wrote beside these
  *           scores (same rows, layout as described there).  With them, a row
- *           with at least topk parts and at most 262,144 keys is selected
+ *           with at least 1.25 topk parts and at most 262,144 keys is selected
  *           from the maxima and the parts whose maximum reaches the topk-th
  *           largest maximum; the result is the same set.  Maxima that do not
  *           belong to the scores give a wrong selection (never an access
