@@ -293,6 +293,10 @@ def gpu_arm(args, rank, world):
     # ---------------------------------------------------------------- e2e (public API, host buffers)
     e2e = e2e_measure(dsa, spec, d, v, q_chunk, args, world)
     peaks, peaks_src = load_peaks()
+    # the rows beyond the three stages (FP8 indexer, paged caches, RoPE, W_UV, append), 1 GPU only
+    ext = None
+    if world == 1 and not args.no_extensions and args.workload == "decode128k":
+        ext = extensions_measure(dsa, spec, d, v, out, idx, peaks)
     # the indexer on a long causal prefill (its dense tensor-core regime), 1 GPU only
     idx_prefill = None
     if world == 1 and not args.no_indexer_prefill and args.workload == "decode128k":
@@ -327,8 +331,148 @@ def gpu_arm(args, rank, world):
         "value": value, "ms_per_step": ms_per_step, "stage_ms": {n: round(t, 4) for n, t in stage_ms.items()},
         "roofline": roof, "step_roofline_frac": round(t_roof * 1e3 / ms_per_step, 4), "e2e": e2e,
         "gpu_launches": 3 * launches * args.steps, "clocks": clocks, "config": describe(spec, idx_fp8),
-        "q_chunk": q_chunk, "inputs": d, "indexer_prefill": idx_prefill,
+        "q_chunk": q_chunk, "inputs": d, "indexer_prefill": idx_prefill, "extensions": ext,
     }
+
+
+def _time_ms(fn, n, stream):
+    """Mean milliseconds of fn() over n launches (CUDA events on `stream`, after 3 warm-up calls)."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
+def extensions_measure(dsa, spec, d, v, out, idx, peaks, n=50):
+    """Decode128k with the scope rows that extend the three stages, each timed
+    with CUDA events over n launches (inputs resident in HBM):
+      fp8_indexer  the whole step with the FP8 indexer: the step's index queries
+                   rotated and quantized to e4m3 (dsa_hadamard_quantize_fp8,
+                   inside the step), keys prepared once the same way from the
+                   bf16 keys of the workload (before their own e4m3 form);
+      paged        the whole step on caches moved into a shuffled pool of
+                   64-row pages (one block table for both caches);
+      rope         the attention with RoPE applied to the queries' rope
+                   columns while they load, against the same call without;
+      up_proj      the per-head W_UV up-projection of the step's output;
+      append       dsa_cache_append of the step's 64 new tokens (latent with
+                   RoPE, index key quantized to e4m3 with an amax/448 scale)."""
+    from dataclasses import replace
+    stream = torch.cuda.current_stream()
+    dev = out.device
+    T, k = spec.T, spec.topk
+    ld = (max(spec.kv_lens) + 3) // 4 * 4
+    scores = torch.empty((T, ld), dtype=torch.float32, device=dev)
+    pm = torch.empty((T, dsa.part_max_ld(ld)), dtype=torch.float32, device=dev)
+    idx2 = torch.empty_like(idx)
+    out2 = torch.empty_like(out)
+    lse2 = torch.empty((T, spec.H), dtype=torch.float32, device=dev)
+    hbm = peaks["hbm_gbs"] * 1e9
+    res = {}
+
+    # ---- FP8 indexer
+    kb = di.make_inputs(replace(spec, kfp8=False), device=dev, tensors=("k_idx",))["k_idx"]
+    kq, ks = dsa.dsa_hadamard_quantize_fp8(kb)
+    del kb
+    qb = d["q_idx"]
+    qq = torch.empty(qb.shape, dtype=torch.float8_e4m3fn, device=dev)
+    qs = torch.empty(qb.shape[:-1], dtype=torch.float32, device=dev)
+
+    def fp8_indexer():
+        dsa.dsa_hadamard_quantize_fp8(qb, qq, qs, stream=stream)
+        dsa.dsa_indexer_scores(qq, d["w"], kq, ks, v, 0, T, scores, stream, part_max=pm, q_scale=qs)
+
+    def fp8_step():
+        fp8_indexer()
+        dsa.dsa_topk(scores, v, 0, T, k, idx2, stream, part_max=pm)
+        dsa.dsa_sparse_mla_attn(d["q"], d["latent"], idx2, v, 0, T, spec.softmax_scale, out2, lse2, stream=stream)
+
+    ms_step = _time_ms(fp8_step, n, stream)
+    ms_idx = _time_ms(fp8_indexer, n, stream)
+    idx_bytes = work_model(spec, True)["indexer"]["bytes"]
+    res["fp8_indexer"] = {
+        "value": round(T / (ms_step / 1e3), 1), "unit": "query tokens/s", "ms_per_step": round(ms_step, 4),
+        "indexer_ms": round(ms_idx, 4), "indexer_achieved_gbs": round(idx_bytes / (ms_idx / 1e3) / 1e9, 1),
+        "indexer_hbm_frac": round(idx_bytes / (ms_idx / 1e3) / hbm, 4),
+        "kernels": "hadamard_quantize_kernel + indexer_persistent_kernel (e4m3 x e4m3, kind::f8f6f4)"}
+    del kq, ks, qq, qs
+    torch.cuda.empty_cache()
+
+    # ---- paged caches (64-row pages, shuffled)
+    P = 64
+    kv = list(spec.kv_lens)
+    pps = max((x + P - 1) // P for x in kv)
+    n_pages = sum((x + P - 1) // P for x in kv) + 8
+    g = torch.Generator().manual_seed(7)
+    perm = torch.randperm(n_pages, generator=g)
+    bt = torch.full((len(kv), pps), -1, dtype=torch.int32)
+    at = 0
+    for b, x in enumerate(kv):
+        np_b = (x + P - 1) // P
+        bt[b, :np_b] = perm[at:at + np_b].to(torch.int32)
+        at += np_b
+    rows = torch.cat([(bt[b, torch.arange(x) // P].to(torch.int64) * P + torch.arange(x) % P)
+                      for b, x in enumerate(kv)]).to(dev)
+    lat_p = torch.zeros((n_pages * P, spec.d_qk), dtype=torch.bfloat16, device=dev)
+    lat_p[rows] = d["latent"]
+    k_p = torch.zeros((n_pages * P, spec.d_I), dtype=torch.uint8, device=dev)
+    k_p[rows] = d["k_idx"].view(torch.uint8)
+    ks_p = torch.zeros(n_pages * P, dtype=torch.float32, device=dev)
+    ks_p[rows] = d["k_scale"]
+    del rows
+    vp = dsa.Varlen(d["cu_q"], d["cu_k"], dev, block_table=bt.to(dev), page_size=P, n_pages=n_pages)
+    k_pv = k_p.view(torch.float8_e4m3fn)
+
+    def paged_step():
+        dsa.dsa_indexer_scores(d["q_idx"], d["w"], k_pv, ks_p, vp, 0, T, scores, stream, part_max=pm)
+        dsa.dsa_topk(scores, vp, 0, T, k, idx2, stream, part_max=pm)
+        dsa.dsa_sparse_mla_attn(d["q"], lat_p, idx2, vp, 0, T, spec.softmax_scale, out2, lse2, stream=stream)
+
+    ms_paged = _time_ms(paged_step, n, stream)
+    res["paged"] = {"value": round(T / (ms_paged / 1e3), 1), "unit": "query tokens/s",
+                    "ms_per_step": round(ms_paged, 4), "page_size": P, "pages": n_pages}
+    del lat_p, k_p, ks_p, k_pv
+    torch.cuda.empty_cache()
+
+    # ---- RoPE of the queries inside the attention
+    i = torch.arange(32, dtype=torch.float64)
+    ang = torch.arange(max(kv), dtype=torch.float64)[:, None] * (10000.0 ** (-2.0 * i / 64))[None, :]
+    rope = torch.stack([torch.cos(ang), torch.sin(ang)], dim=-1).to(torch.float32).to(dev)
+    ms_rope = _time_ms(lambda: dsa.dsa_sparse_mla_attn(d["q"], d["latent"], idx, v, 0, T, spec.softmax_scale,
+                                                       out2, lse2, stream=stream, rope=rope), n, stream)
+    ms_norope = _time_ms(lambda: dsa.dsa_sparse_mla_attn(d["q"], d["latent"], idx, v, 0, T, spec.softmax_scale,
+                                                         out2, lse2, stream=stream), n, stream)
+    res["rope"] = {"attention_ms_with_rope": round(ms_rope, 4), "attention_ms_without": round(ms_norope, 4)}
+
+    # ---- W_UV up-projection of the step's output
+    w_uv = di.make_w_uv(11, device=dev)
+    y = torch.empty((T, spec.H, 128), dtype=torch.bfloat16, device=dev)
+    ms_up = _time_ms(lambda: dsa.dsa_mla_up_proj(out, w_uv, y, stream=stream), n, stream)
+    up_bytes = w_uv.numel() * 2 + out.numel() * 2 + y.numel() * 2
+    res["up_proj"] = {"ms": round(ms_up, 4), "bytes": up_bytes,
+                      "achieved_gbs": round(up_bytes / (ms_up / 1e3) / 1e9, 1),
+                      "hbm_frac": round(up_bytes / (ms_up / 1e3) / hbm, 4),
+                      "flops": 2 * T * spec.H * spec.d_v * 128, "kernel": "up_proj_kernel (tcgen05, M=128 rows)"}
+
+    # ---- append of the step's new tokens (one per sequence) into the caches
+    gg = torch.Generator().manual_seed(12)
+    lat_new = torch.randn(T, spec.d_qk, generator=gg).to(torch.bfloat16).to(dev)
+    k_new = torch.randn(T, spec.d_I, generator=gg).to(torch.bfloat16).to(dev)
+    ms_app = _time_ms(lambda: dsa.dsa_cache_append(v, lat_new, d["latent"], k_new, d["k_idx"], d["k_scale"],
+                                                   k_quant=dsa.DSA_KQ_E4M3_AMAX, rope=rope, stream=stream),
+                      n, stream)
+    res["append"] = {"ms": round(ms_app, 4), "tokens": T, "bytes_per_token": (spec.d_qk + spec.d_I) * 2 +
+                     spec.d_qk * 2 + spec.d_I + 4}
+    assert dsa.dsa_device_error() == 0
+    del scores, pm, idx2, out2, lse2, rope, w_uv, y
+    torch.cuda.empty_cache()
+    return res
 
 
 def load_traffic(stage, workload, alg_bytes_per_launch):
@@ -614,6 +758,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-indexer-prefill", action="store_true",
                     help="skip the secondary indexer measurement on the 32K prefill")
+    ap.add_argument("--no-extensions", action="store_true",
+                    help="skip the FP8-indexer, paged, RoPE, up-projection and append measurements")
     args = ap.parse_args()
     if args.impl == "reference":
         args.steps = 1 if args.steps is None else args.steps
@@ -643,6 +789,8 @@ def main():
         }
         if r.get("indexer_prefill"):
             line["indexer_prefill"] = r["indexer_prefill"]
+        if r.get("extensions"):
+            line["extensions"] = r["extensions"]
         if world == 1 and not args.no_cpu_baseline:
             spec = di.config(args.workload)
             import oracle
