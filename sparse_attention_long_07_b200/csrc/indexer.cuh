@@ -68,8 +68,11 @@ struct IndexerCfg {
   static constexpr int RAW_ROWB = D_I;                    // bytes of one e4m3 key row
   static constexpr int RAW_TILE = BK * RAW_ROWB;
   // epilogue warpgroups: two split the queries of a wide tile, or (persistent
-  // schedule) take alternate tiles, each owning one TMEM accumulator
-  static constexpr int EPI_WG = (PERSIST || N >= 256) ? 2 : 1;
+  // schedule) four take every fourth tile, each owning one TMEM accumulator:
+  // the epilogue's per-tile chain (tensor-memory loads, 64 ReLU-FMAs, the score
+  // and part-maximum stores) is then spread over four tile periods (measured:
+  // 0.154 -> 0.131 ms with bf16 queries, 0.119 -> 0.102 ms FP8, decode128k)
+  static constexpr int EPI_WG = PERSIST ? 4 : (N >= 256 ? 2 : 1);
   static constexpr int QW = PERSIST ? NQ : NQ / EPI_WG;   // queries per epilogue warpgroup
   static constexpr int COLS_PER_THREAD = QW * H_I;
   static constexpr int LD_CHUNK = COLS_PER_THREAD >= 32 ? 32 : 16;
