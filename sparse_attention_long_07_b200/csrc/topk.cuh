@@ -284,41 +284,88 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     *total = wpre[C::NW];
     return wpre[warp] + pre;
   };
-  // Radix-256 selection.  select(count, key_of, use, kth, &thr, &rem, steps):
-  // the kth largest key among the entries i < count with use(i) (at least kth
-  // of them), found 8 bits at a time from the top.  Each pass builds a
-  // 256-bin histogram of the next digit over the entries that share the
-  // digits found so far (warp-aggregated shared atomics), and one CTA scan of
-  // the bins (find_digit_fn) gives the digit holding the kth entry and the
-  // entries above it.  steps counts 2-bit steps: steps = 16 resolves all 32
-  // bits; with steps = 8 only the top 16 bits are resolved and the lower bits
-  // are 0, so thr is then a lower bound of the kth largest key with at least
-  // kth entries >= thr.  *rem = kth - (entries > thr) (meaningful for steps =
-  // 16).  Called by every thread (three barriers per pass).
-  auto select = [&](uint32_t count, auto&& key_of, auto&& use, uint32_t kth, uint32_t* out_thr,
-                    uint32_t* out_rem, int steps = 16) {
-    uint32_t* h = hist;                 // 256 bins (the first words of the pass-1 histogram)
-    uint32_t prefix = 0, need = kth;    // need: rank of the target among the entries matching prefix
-    const int passes = steps / 4;
-    for (int d = 0; d < passes; ++d) {
-      const int shift = 24 - 8 * d;
-      const uint32_t hi_mask = d == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-      if (tid < 256) h[tid] = 0u;
+  // Range-histogram selection.  select(hb, count, key_of, use, kth, &thr,
+  // &rem, exact): the kth largest key among the entries i < count with use(i)
+  // (at least kth of them).  The keys' range [lo, hi] (a CTA min/max) is cut
+  // into 4096 bins of 2^s keys, s chosen so that the range fits; one pass of
+  // shared atomics fills the histogram hb[4096] and a CTA scan finds the bin
+  // holding the kth entry; the window shrinks to that bin.  exact: repeat until
+  // a bin is one key value (two passes for a range of up to 2^24 keys): thr is
+  // then the kth largest key and *rem = kth - (entries > thr).  Otherwise one
+  // pass: thr is the start of the bin, a lower bound of the kth largest key
+  // with at least kth entries >= thr.  Bins follow the data, so a narrow
+  // distribution does not pile into a few bins.  Called by every thread.
+  auto select = [&](uint32_t* hb, uint32_t count, auto&& key_of, auto&& use, uint32_t kth, uint32_t* out_thr,
+                    uint32_t* out_rem, bool exact) {
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+    for (uint32_t i = tid; i < count; i += C::NT)
+      if (use(i)) {
+        const uint32_t k = key_of(i);
+        mn = min(mn, k);
+        mx = max(mx, k);
+      }
+    mn = __reduce_min_sync(0xFFFFFFFFu, mn);
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if (lane == 0) {
+      wtot[warp] = mn;
+      wtot[C::NW + warp] = mx;
+    }
+    __syncthreads();
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+    for (int w = 0; w < C::NW; ++w) {
+      lo = min(lo, wtot[w]);
+      hi = max(hi, wtot[C::NW + w]);
+    }
+    __syncthreads();   // wtot is reused below
+    uint32_t need = kth;
+    constexpr int HB_BITS = 12, HB_BINS = 1 << HB_BITS, PER_T = HB_BINS / C::NT;
+    static_assert(HB_BINS % C::NT == 0, "bins per thread");
+    for (;;) {
+      const uint32_t span = hi - lo;
+      const int bits = span == 0u ? 0 : 32 - __clz(span);
+      const int sh = bits > HB_BITS ? bits - HB_BITS : 0;
+      for (int i = tid; i < HB_BINS; i += C::NT) hb[i] = 0u;
       __syncthreads();
-      for (uint32_t base = 0; base < count; base += C::NT) {   // uniform trip count: whole warps call hist_add
-        const uint32_t i = base + tid;
-        bool valid = i < count && use(i);
-        const uint32_t k = valid ? key_of(i) : 0u;
-        valid = valid && (k & hi_mask) == prefix;
-        hist_add(h, (k >> shift) & 0xFFu, valid);
+      for (uint32_t i = tid; i < count; i += C::NT)
+        if (use(i)) {
+          const uint32_t k = key_of(i);
+          if (k >= lo && k <= hi) atomicAdd(&hb[(k - lo) >> sh], 1u);
+        }
+      __syncthreads();
+      // thread t owns bins HB_BINS-1-PER_T t .. down (descending); a CTA scan
+      // gives the entries above them
+      const int top = HB_BINS - 1 - PER_T * static_cast<int>(tid);
+      uint32_t c8[PER_T], sum = 0;
+#pragma unroll
+      for (int j = 0; j < PER_T; ++j) {
+        c8[j] = hb[top - j];
+        sum += c8[j];
+      }
+      uint32_t unused_total;
+      const uint32_t excl = block_scan(sum, &unused_total);
+      if (excl < need && need <= excl + sum) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int j = 0; j < PER_T; ++j) {
+          if (acc + c8[j] >= need) {
+            misc[4] = static_cast<uint32_t>(top - j);
+            misc[5] = acc;
+            break;
+          }
+          acc += c8[j];
+        }
       }
       __syncthreads();
-      find_digit_fn(h, 256, need, &misc[4], &misc[5]);
-      prefix |= misc[4] << shift;
+      const uint32_t bin = misc[4];
       need -= misc[5];
-      __syncthreads();   // every thread has read misc[4..5] before the next pass writes them
+      __syncthreads();   // every thread has read misc[4..5]
+      lo += bin << sh;
+      if (sh > 0) hi = min(hi, lo + ((1u << sh) - 1u));
+      else hi = lo;
+      if (sh == 0 || !exact) break;
     }
-    *out_thr = prefix;
+    *out_thr = lo;
     *out_rem = need;
   };
   // Exact selection among candidates ckey/cidx[0, nc) that hold every key
@@ -331,8 +378,9 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
   auto finish_candidates = [&](uint32_t nc, bool ordered) {
     uint32_t* bitmap = reinterpret_cast<uint32_t*>(smem + C::OFF_BITMAP);
     uint32_t thr, need_eq;
-    select(nc, [&](uint32_t i) { return ckey[i]; }, [&](uint32_t) { return true; },
-           static_cast<uint32_t>(topk), &thr, &need_eq);
+    uint32_t* hb = reinterpret_cast<uint32_t*>(smem + C::OFF_WHIST);   // free once the candidates exist
+    select(hb, nc, [&](uint32_t i) { return ckey[i]; }, [&](uint32_t) { return true; },
+           static_cast<uint32_t>(topk), &thr, &need_eq, true);
     // ties at the threshold: the need_eq lowest indices (largest ~index)
     uint32_t ties_mine = 0, n_ties;
     for (uint32_t i = tid; i < nc; i += C::NT) ties_mine += ckey[i] == thr ? 1u : 0u;
@@ -340,8 +388,8 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
     uint32_t inv_idx_thr = 0u;   // select every tie
     if (n_ties > need_eq) {
       uint32_t rem2;
-      select(nc, [&](uint32_t i) { return ~static_cast<uint32_t>(cidx[i]); },
-             [&](uint32_t i) { return ckey[i] == thr; }, need_eq, &inv_idx_thr, &rem2);
+      select(hb, nc, [&](uint32_t i) { return ~static_cast<uint32_t>(cidx[i]); },
+             [&](uint32_t i) { return ckey[i] == thr; }, need_eq, &inv_idx_thr, &rem2, true);
     }
     auto chosen = [&](uint32_t i) {
       const uint32_t key = ckey[i];
@@ -451,8 +499,9 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
       // A lower bound of the k-th largest group maximum (its top 16 bits):
       // at least k groups, hence k scores, are >= b.
       uint32_t b, unused_rem;
-      select(static_cast<uint32_t>(Pg), [&](uint32_t i) { return pk[i]; }, [&](uint32_t) { return true; },
-             static_cast<uint32_t>(topk), &b, &unused_rem, 8);
+      select(reinterpret_cast<uint32_t*>(smem + C::OFF_WHIST), static_cast<uint32_t>(Pg),
+             [&](uint32_t i) { return pk[i]; }, [&](uint32_t) { return true; }, static_cast<uint32_t>(topk), &b,
+             &unused_rem, false);
       phase(50);
       // the groups whose maximum is >= b, in order (contiguous ranges per thread, one block scan)
       const int per = (Pg + C::NT - 1) / C::NT;
@@ -613,8 +662,10 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
       if (!ok) { DSA_PROF_END(); return; }
       // ---- lower bound b of the k-th largest part maximum (its top 16 bits)
       uint32_t b_lo, unused_rem;
-      select(static_cast<uint32_t>(P), [&](uint32_t i) { return pmax[i]; }, [&](uint32_t) { return true; },
-             static_cast<uint32_t>(topk), &b_lo, &unused_rem, 8);
+      // (the histogram goes into the ring, free between the two streaming passes)
+      select(reinterpret_cast<uint32_t*>(smem + C::OFF_RING), static_cast<uint32_t>(P),
+             [&](uint32_t i) { return pmax[i]; }, [&](uint32_t) { return true; }, static_cast<uint32_t>(topk), &b_lo,
+             &unused_rem, false);
       if (tid == 0) misc[4] = 0u;   // candidate count
       __syncthreads();
       phase(42);
