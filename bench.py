@@ -586,21 +586,23 @@ E2E_MIN_CALLS = 100
 
 def e2e_measure(dsa, spec, d, v, q_chunk, args, world):
     """dsa_forward through the public API, each step's inputs copied from
-    pinned host memory and its outputs copied back.  Two batches are kept in
-    flight, as a server would: lane 0 serves the benchmark's batch and lane 1
-    another batch of the same shape (other seed), each on its own stream with
-    its own buffers, and the steps alternate between them, so that one lane's
-    host transfers overlap the other lane's kernels.  Every step still copies
-    its whole input in and its whole output out."""
+    pinned host memory and its outputs copied back.  Several batches are kept
+    in flight, as a server would: lane 0 serves the benchmark's batch and the
+    other lanes other batches of the same shape (other seeds), each on its own
+    stream with its own buffers, and the steps go round the lanes, so that one
+    lane's host transfers overlap the other lanes' kernels.  Every step still
+    copies its whole input in and its whole output out."""
     import dataclasses
     dev = d["q"].device
     decode = all(q == 1 for q in spec.q_lens)
-    spec2 = dataclasses.replace(spec, seed=spec.seed + 500)
-    d2 = di.make_inputs(spec2, device=dev)
-    v2 = type(v)(d2["cu_q"], d2["cu_k"], dev)
-    lanes = [_E2ELane(dsa, spec, d, v, q_chunk, decode), _E2ELane(dsa, spec2, d2, v2, q_chunk, decode)]
-    for i in range(4):
-        lanes[i % 2].step(dsa)
+    n_lanes = max(1, args.e2e_lanes)
+    lanes = [_E2ELane(dsa, spec, d, v, q_chunk, decode)]
+    for j in range(1, n_lanes):
+        spec_j = dataclasses.replace(spec, seed=spec.seed + 500 + j)
+        d_j = di.make_inputs(spec_j, device=dev)
+        lanes.append(_E2ELane(dsa, spec_j, d_j, type(v)(d_j["cu_q"], d_j["cu_k"], dev), q_chunk, decode))
+    for i in range(2 * n_lanes):
+        lanes[i % n_lanes].step(dsa)
     torch.cuda.synchronize()
     n = max(E2E_MIN_CALLS, min(args.steps, 1000))
     start = torch.cuda.Event(enable_timing=True)
@@ -608,20 +610,21 @@ def e2e_measure(dsa, spec, d, v, q_chunk, args, world):
     barrier(world)
     torch.cuda.synchronize()
     start.record(lanes[0].stream)
-    lanes[1].stream.wait_event(start)
+    for ln in lanes[1:]:
+        ln.stream.wait_event(start)
     for i in range(n):
-        lanes[i % 2].step(dsa)
+        lanes[i % n_lanes].step(dsa)
     for e, ln in zip(ends, lanes):
         e.record(ln.stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(max(start.elapsed_time(e) for e in ends), world) / n
     assert dsa.dsa_device_error() == 0
     h2d, d2h = lanes[0].h2d, lanes[0].d2h
-    del lanes, d2
+    del lanes
     torch.cuda.empty_cache()
     return {"value": world * spec.T / (ms / 1e3), "unit": "query tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4), "steps": n, "api": "dsa_forward",
-            "batches_in_flight": 2}
+            "batches_in_flight": n_lanes}
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -758,6 +761,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-indexer-prefill", action="store_true",
                     help="skip the secondary indexer measurement on the 32K prefill")
+    ap.add_argument("--e2e-lanes", type=int, default=3,
+                    help="batches in flight in the end-to-end measurement (one stream each)")
     ap.add_argument("--no-extensions", action="store_true",
                     help="skip the FP8-indexer, paged, RoPE, up-projection and append measurements")
     args = ap.parse_args()
