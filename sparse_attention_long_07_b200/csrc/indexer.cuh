@@ -67,12 +67,14 @@ struct IndexerCfg {
   static constexpr int B_TILE = N * ROWB;
   static constexpr int RAW_ROWB = D_I;                    // bytes of one e4m3 key row
   static constexpr int RAW_TILE = BK * RAW_ROWB;
-  // epilogue warpgroups: two split the queries of a wide tile, or (persistent
-  // schedule) four take every fourth tile, each owning one TMEM accumulator:
-  // the epilogue's per-tile chain (tensor-memory loads, 64 ReLU-FMAs, the score
-  // and part-maximum stores) is then spread over four tile periods (measured:
-  // 0.154 -> 0.131 ms with bf16 queries, 0.119 -> 0.102 ms FP8, decode128k)
-  static constexpr int EPI_WG = PERSIST ? 4 : (N >= 256 ? 2 : 1);
+  // epilogue warpgroups: four split the four queries of a wide tile (one
+  // each), or (persistent schedule) four take every fourth tile, each owning
+  // one TMEM accumulator.  The epilogue's per-tile chain (tensor-memory
+  // loads, 64 ReLU-FMAs, the score and part-maximum stores) bounded both
+  // schedules; measured with four warpgroups instead of two: decode128k
+  // 0.154 -> 0.131 ms (bf16 queries), 0.119 -> 0.102 ms (FP8); prefill32k
+  // 8.7 -> 8.0 ms.
+  static constexpr int EPI_WG = (PERSIST || N >= 256) ? 4 : 1;
   static constexpr int QW = PERSIST ? NQ : NQ / EPI_WG;   // queries per epilogue warpgroup
   static constexpr int COLS_PER_THREAD = QW * H_I;
   static constexpr int LD_CHUNK = COLS_PER_THREAD >= 32 ? 32 : 16;
@@ -116,7 +118,7 @@ struct IndexerCfg {
   static_assert(!QFP8 || (KFP8 && D_I == 128), "FP8 indexer: e4m3 keys, 128-byte rows");
   static_assert(TMEM_COLS <= 512, "tensor memory columns");
   static_assert(!K_IN_TMEM || (KFP8 && STAGES % CONV_TEAMS == 0), "converter teams own alternate stages");
-  static_assert(NACC % EPI_WG == 0, "each accumulator is drained by one epilogue warpgroup");
+  static_assert(!PERSIST || NACC % EPI_WG == 0, "each accumulator is drained by one epilogue warpgroup");
   static_assert(2 + 2 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "grid barrier layout");
   static_assert(!PERSIST || 7 + 3 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "persistent barrier layout");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
