@@ -61,6 +61,11 @@ struct IndexerCfg {
   // tile ring (bf16, or e4m3 as loaded for the FP8 indexer) is in shared
   // memory, twelve deep for the persistent FP8 schedule.
   static constexpr bool K_IN_TMEM = PERSIST && CONVERT;
+  // ... and there the MMAs take f16 operands: e4m3 keys widen to f16 in one
+  // conversion instruction per pair, and each sequence's bf16 query tile is
+  // rewritten in place as f16, scaled by a power of two 2^sq that puts its
+  // largest magnitude in [2^14, 2^15); the epilogue multiplies by 2^-sq.
+  static constexpr bool QF16 = K_IN_TMEM;
   static constexpr int STAGES = K_IN_TMEM ? 4 : (PERSIST ? 12 : (CONVERT ? 2 : 4));  // key-tile ring (MMA operand)
   static constexpr int RSTAGES = CONVERT ? (PERSIST ? 11 : 4) : 0;  // raw e4m3 ring (to widen)
   static constexpr int A_TILE = BK * ROWB;
@@ -94,7 +99,8 @@ struct IndexerCfg {
   static constexpr int CONV_TEAMS = PERSIST ? 2 : 1;      // e4m3 converter teams (alternate tiles)
   static constexpr int NWARPS = MMA_WARP + MMA_THREADS + (CONVERT ? 4 * CONV_TEAMS : 0);
   static constexpr int NT = NWARPS * 32;
-  static constexpr uint32_t IDESC = QFP8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N, false, false);
+  static constexpr uint32_t IDESC =
+      QFP8 ? idesc_e4m3_f32(128, N) : (QF16 ? idesc_f16_f32(128, N) : idesc_bf16_f32(128, N, false, false));
   // shared memory layout (offsets from a 1024-byte aligned base)
   static constexpr int QBUF = PERSIST ? 2 : 1;            // query tiles (double buffer when persistent)
   static constexpr int OFF_Q = 0;
@@ -104,10 +110,14 @@ struct IndexerCfg {
   static constexpr int OFF_BAR = OFF_W + NQ * H_I * 4;
   // barriers: grid schedule 2 + 2 STAGES + 2 RSTAGES + 2 NACC; persistent
   // schedule 7 + STAGES (ready) + 2 RSTAGES + NACC (acc_full) + 2 STAGES
-  // (k_full, k_empty) + NACC (acc_empty), every array reserved in both forms
-  static constexpr int NBAR = 7 + 3 * STAGES + 2 * RSTAGES + 2 * NACC;
+  // (k_full, k_empty) + NACC (acc_empty) + 2 (q_conv), every array reserved
+  // in both forms
+  static constexpr int NBAR = 9 + 3 * STAGES + 2 * RSTAGES + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int OFF_UPRE = OFF_MISC + 16;          // persistent: unit prefix per sequence
+  // f16 queries: descale 2^-sq per query buffer and per accumulator, and the
+  // converter teams' partial maxima (team, buffer, warp)
+  static constexpr int OFF_QCONV = OFF_MISC + 16;
+  static constexpr int OFF_UPRE = OFF_QCONV + 128;        // persistent: unit prefix per sequence
   // persistent: per-warp head weights, read as float4 (16-byte aligned)
   static constexpr int OFF_WEPI = (OFF_UPRE + (PERSIST ? (MAX_SEQ + 1) * 4 : 0) + 15) / 16 * 16;
   static constexpr int SMEM_BYTES = OFF_WEPI + (PERSIST ? 4 * EPI_WG * H_I * 4 : 0) + 1024;  // + alignment slack
@@ -120,7 +130,9 @@ struct IndexerCfg {
   static_assert(!K_IN_TMEM || (KFP8 && STAGES % CONV_TEAMS == 0), "converter teams own alternate stages");
   static_assert(!PERSIST || NACC % EPI_WG == 0, "each accumulator is drained by one epilogue warpgroup");
   static_assert(2 + 2 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "grid barrier layout");
-  static_assert(!PERSIST || 7 + 3 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "persistent barrier layout");
+  static_assert(!PERSIST || 9 + 3 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "persistent barrier layout");
+  static_assert(4 * (2 + NACC) + 4 * 2 * CONV_TEAMS * 4 <= 128, "query-conversion scratch");
+  static_assert(!QF16 || (B_TILE / 16) % 128 == 0, "query tile in 16-byte pieces per converter thread");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
   static_assert(!K_IN_TMEM || STAGES == NACC, "key stage and accumulator of a tile share one barrier");
   static_assert(!PERSIST || NQ == 1, "persistent schedule: one query per sequence block");
@@ -185,6 +197,15 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t src, uint32_t& lo, uin
   b = (b << 4) & 0x87F087F0u;
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0x7B807B80u));   // 0x7B80 = bf16 2^120
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0x7B807B80u));
+}
+
+// Four e4m3 bytes -> four f16 values (two f16x2 words, lower element in the
+// low half), exact: one hardware conversion per pair.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t src, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(src));
 }
 
 struct IndexerParams {
@@ -562,8 +583,14 @@ __global__ void __launch_bounds__(C::NT, 1)
   auto bar_k_full = [&](int s) { return bar0 + 56 + 8 * (C::STAGES + 2 * C::RSTAGES + C::NACC + s); };
   auto bar_k_empty = [&](int s) { return bar0 + 56 + 8 * (2 * C::STAGES + 2 * C::RSTAGES + C::NACC + s); };
   auto bar_acc_empty = [&](int a) { return bar0 + 56 + 8 * (3 * C::STAGES + 2 * C::RSTAGES + C::NACC + a); };
+  // f16 queries: q_conv(buf) once the converter team of the segment's first
+  // tile has rewritten the query tile as f16 (128 arrivals)
+  auto bar_q_conv = [&](int buf) { return bar0 + 56 + 8 * (3 * C::STAGES + 2 * C::RSTAGES + 2 * C::NACC + buf); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* qfac_buf = reinterpret_cast<float*>(smem + C::OFF_QCONV);        // [2]: 2^-sq of each query buffer
+  float* qfac_acc = qfac_buf + 2;                                         // [NACC]: 2^-sq of each accumulator
+  uint32_t* qmax_part = reinterpret_cast<uint32_t*>(qfac_acc + C::NACC);  // [team][buf][warp]
 
   if (threadIdx.x == 0) {
     mbar_init(bar_drain, C::MMA_THREADS);
@@ -577,6 +604,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         mbar_init(bar_raw_full(s), 1);
         mbar_init(bar_raw_empty(s), 128);
       }
+      for (int buf = 0; buf < 2; ++buf) mbar_init(bar_q_conv(buf), 128);
     } else {
       for (int s = 0; s < C::STAGES; ++s) {
         mbar_init(bar_k_full(s), 1);
@@ -584,7 +612,9 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
       for (int a = 0; a < C::NACC; ++a) mbar_init(bar_acc_empty(a), 128);
     }
-    for (int a = 0; a < C::NACC; ++a) mbar_init(bar_acc_full(a), 1);
+    // f16 queries: the MMA thread's arrival (after it stored the descale of
+    // the accumulator) joins the commit's
+    for (int a = 0; a < C::NACC; ++a) mbar_init(bar_acc_full(a), C::QF16 ? 2 : 1);
     *abort_flag = 0;
     fence_mbar_init();
     // every accumulator starts drained: the epilogue's share of the first phase
@@ -680,8 +710,11 @@ __global__ void __launch_bounds__(C::NT, 1)
         } while (upre[b + 1] == upre[b]);   // sequences without units in the call
         seq_end = upre[b + 1];
       };
+      // the query tile as the MMAs read it: loaded, and (f16 queries) rewritten
+      auto q_ready = [&](int sg) { return C::QF16 ? bar_q_conv(sg & 1) : bar_q_full(sg & 1); };
+      float qfac = 1.f;
       auto release_segment = [&]() -> bool {   // done with segment seg
-        if (!have_q && !mbar_wait(bar_q_full(seg & 1), (seg >> 1) & 1, abort_flag, 52)) return false;
+        if (!have_q && !mbar_wait(q_ready(seg), (seg >> 1) & 1, abort_flag, 52)) return false;
         umma_commit(bar_q_empty(mt, seg & 1));
         have_q = false;
         return true;
@@ -694,9 +727,10 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
         if (!ok) break;
         if (!have_q) {
-          if (!mbar_wait(bar_q_full(seg & 1), (seg >> 1) & 1, abort_flag, 52)) { ok = false; break; }
+          if (!mbar_wait(q_ready(seg), (seg >> 1) & 1, abort_flag, 52)) { ok = false; break; }
           have_q = true;
           b_desc = b_desc0 + static_cast<uint64_t>(((seg & 1) * C::B_TILE) >> 4);
+          if constexpr (C::QF16) qfac = qfac_buf[seg & 1];
         }
         if constexpr (C::CONVERT) {
           const int s = it % C::STAGES;
@@ -715,6 +749,10 @@ __global__ void __launch_bounds__(C::NT, 1)
             umma_ts(tmem + a * C::N, a_tile + kk * 8, bd, C::IDESC, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar_acc_full(a));   // also frees key stage s (== a)
+          // the epilogue of tile it reads this after acc_full(a); it was last
+          // read by the epilogue of tile it - NACC, before its ready(a) arrival
+          qfac_acc[a] = qfac;
+          mbar_arrive(bar_acc_full(a));
         } else {
           // FP8 indexer: A = the e4m3 key tile as loaded (128 rows of 128
           // bytes, 128-byte swizzle), B = the e4m3 query tile; 32 bytes of K
@@ -754,9 +792,62 @@ __global__ void __launch_bounds__(C::NT, 1)
     const int team = (warp - C::CONVERT_WARP0) / 4;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + C::ACC_COLS;
+    // The query tile of segment sg (buffer sg & 1), bf16 as loaded, rewritten
+    // in place as f16 x 2^sq (same 16-bit element positions, so the swizzled
+    // layout holds).  sq = 14 - E for the largest magnitude 2^E (1 + f): that
+    // value becomes < 2^15, every element of magnitude >= 2^(E-31) stays
+    // exact (f16 keeps 11 significant bits down to 2^-14 and whole multiples
+    // of 2^-24 below), and smaller ones move by at most 2^(E-39).  A zero or
+    // non-finite maximum keeps sq = 0; sq <= 126 keeps 2^-sq a normal float.
+    auto widen_query = [&](int sg) -> bool {
+      const int buf = sg & 1;
+      if (!mbar_wait(bar_q_full(buf), (sg >> 1) & 1, abort_flag, 58)) return false;
+      uint4* qv = reinterpret_cast<uint4*>(smem + C::OFF_Q + buf * C::B_TILE);
+      constexpr int PER = C::B_TILE / 16 / 128;
+      const int tt = row;   // 0..127 across the team
+      uint4 x[PER];
+      uint32_t m2 = 0;      // the largest magnitude (bf16 bit patterns order as magnitudes)
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        x[i] = qv[tt + 128 * i];
+        m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(x[i].x & 0x7FFF7FFFu, x[i].y & 0x7FFF7FFFu),
+                                   __vmaxu2(x[i].z & 0x7FFF7FFFu, x[i].w & 0x7FFF7FFFu)));
+      }
+      uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
+      uint32_t* part = qmax_part + (team * 2 + buf) * 4;
+      if (lane == 0) part[warp & 3] = m;
+      named_bar_sync(1 + team, 128);
+      m = max(max(part[0], part[1]), max(part[2], part[3]));
+      const int ef = static_cast<int>(m >> 7);   // biased exponent of the maximum
+      int sq = 0;
+      if (m != 0 && ef < 255) sq = min(141 - ef, 126);
+      const float up = __int_as_float((127 + sq) << 23);
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float lo = __uint_as_float(w[e] << 16) * up;
+          const float hi = __uint_as_float(w[e] & 0xFFFF0000u) * up;
+          asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w[e]) : "f"(hi), "f"(lo));
+        }
+        qv[tt + 128 * i] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();   // the MMAs read the tile through the async proxy
+      if (tt == 0) qfac_buf[buf] = __int_as_float((127 - sq) << 23);
+      mbar_arrive(bar_q_conv(buf));
+      return true;
+    };
+    int b = b_first, seg = 0;
     for (int it = team; it < n_iter; it += C::CONV_TEAMS) {
       const int r = it % C::RSTAGES;
       const int s = it % C::STAGES;
+      const int u = u0 + it;
+      while (u >= upre[b + 1]) {
+        ++b;
+        if (upre[b + 1] > upre[b]) ++seg;   // sequences with units in the call
+      }
+      if (u == max(upre[b], u0) && !widen_query(seg)) break;   // the segment's first tile
       if (!mbar_wait(bar_raw_full(r), (it / C::RSTAGES) & 1, abort_flag, 55)) break;
       const uint8_t* raw_row = smem + C::OFF_RAW + r * C::RAW_TILE + row * 128;
       uint4 chunk[8];
@@ -775,10 +866,10 @@ __global__ void __launch_bounds__(C::NT, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint4 c = chunk[4 * h + j];
-          e4m3x4_to_bf16x4(c.x, cols[8 * j + 0], cols[8 * j + 1]);
-          e4m3x4_to_bf16x4(c.y, cols[8 * j + 2], cols[8 * j + 3]);
-          e4m3x4_to_bf16x4(c.z, cols[8 * j + 4], cols[8 * j + 5]);
-          e4m3x4_to_bf16x4(c.w, cols[8 * j + 6], cols[8 * j + 7]);
+          e4m3x4_to_f16x4(c.x, cols[8 * j + 0], cols[8 * j + 1]);
+          e4m3x4_to_f16x4(c.y, cols[8 * j + 2], cols[8 * j + 3]);
+          e4m3x4_to_f16x4(c.z, cols[8 * j + 4], cols[8 * j + 5]);
+          e4m3x4_to_f16x4(c.w, cols[8 * j + 6], cols[8 * j + 7]);
         }
         tmem_st32(t_lane + s * C::A_COLS + 32 * h, cols);
       }
@@ -834,6 +925,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
       if (!mbar_wait_warp(bar_acc_full(a), (it / C::NACC) & 1, abort_flag, 57)) break;
       tc_fence_after();
+      const float qfac = C::QF16 ? qfac_acc[a] : 1.f;
       const uint32_t t_row = tmem + (static_cast<uint32_t>(sub * 32) << 16) + a * C::N;
       float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
@@ -856,7 +948,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       else mbar_arrive_warp(bar_acc_empty(a));
       const int s_key = (u - upre[b]) * C::BK + key_in_tile;
       // keys past the query's position (and past the cache) score -inf
-      const float val = s_key <= q.pos ? (acc0 + acc1) * ks : -INFINITY;
+      const float val = s_key <= q.pos ? (acc0 + acc1) * qfac * ks : -INFINITY;
       const int64_t row = static_cast<int64_t>(q.q0) - p.q_begin;
       if (s_key < q.kv_len && in_bounds(s_key < p.ld, 84)) p.scores[row * p.ld + s_key] = val;
       if (p.part_max != nullptr) {

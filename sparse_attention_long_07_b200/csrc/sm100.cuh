@@ -228,6 +228,11 @@ __device__ __forceinline__ bool device_error_pending() {
   return *reinterpret_cast<volatile int*>(&g_device_error) != 0;
 }
 
+// Named barrier `id` (1..15; 0 is __syncthreads) over `n` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // ----------------------------------------------------------------------------
 // Proxy fences
 // ----------------------------------------------------------------------------
@@ -349,6 +354,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | (1u << 10)                                // B format: bf16
          | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16 with f16 A and B (both
+// K-major) and an fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4)                                   // D format: f32
+         | (0u << 7)                                 // A format: f16
+         | (0u << 10)                                // B format: f16
+         | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor of tcgen05.mma kind::f8f6f4 with e4m3 A and B (both

@@ -224,6 +224,44 @@ def test_indexer_widens_every_e4m3_code_exactly(dsa, oracle_lib, q_lens, kv_lens
     P.assert_scores_close(got, ref, pos, exact=True)
 
 
+# Query tiles of very different magnitudes, one per sequence: the decode
+# schedule rewrites each sequence's bf16 query tile as f16 times a power of
+# two chosen from the tile's largest magnitude, so the scores must follow the
+# oracle whatever that magnitude is (the tolerance is relative to the row).
+# Sequence 0 holds an all-zero query (exact zeros); the last spreads its heads
+# over 2^0 .. 2^-126, so most of its elements fall below f16's normal range
+# once the tile is scaled and only the largest heads decide the scores.
+QUERY_EXPONENTS = (None, -100, -60, -24, -10, 0, 8, 20, 60, 100, "spread")
+
+
+@pytest.mark.parametrize("q_lens", [(1,) * len(QUERY_EXPONENTS), (2,) * len(QUERY_EXPONENTS)],
+                         ids=["decode", "prefill"])
+def test_indexer_query_magnitudes(dsa, oracle_lib, q_lens):
+    kv_lens = tuple(300 + 97 * b for b in range(len(QUERY_EXPONENTS)))
+    spec = released("idx", q_lens, kv_lens, seed=11, kfp8=True)
+    d = di.make_inputs(spec)
+    q = d["q_idx"].float()
+    cu_q = d["cu_q"]
+    for b, e in enumerate(QUERY_EXPONENTS):
+        rows = slice(int(cu_q[b]), int(cu_q[b + 1]))
+        if e is None:
+            q[rows] = 0.0
+        elif e == "spread":
+            q[rows] = q[rows] * torch.exp2(-2.0 * torch.arange(64, dtype=torch.float32))[None, :, None]
+        else:
+            q[rows] = q[rows] * 2.0 ** e
+    d["q_idx"] = q.to(torch.bfloat16)    # powers of two: the bf16 values scale exactly
+    dd = P.to_device(d)
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], "cuda")
+    ld = ld_for(spec)
+    got = gpu_scores(dsa, dd, v, 0, spec.T, ld).cpu().numpy()
+    ref = oracle_lib.indexer_scores(d["cu_q"], d["cu_k"], d["q_idx"], d["w"], d["k_idx"], d["k_scale"], ld=ld)
+    pos = P.row_positions(d["cu_q"], d["cu_k"])
+    P.assert_scores_close(got, ref, pos)
+    for r in range(int(cu_q[1])):          # the all-zero query
+        assert np.all(got[r, : pos[r] + 1] == 0.0)
+
+
 # ------------------------------------------------------------------ sparse MLA
 
 def _attention_case(dsa, oracle_lib, spec, idx=None):
