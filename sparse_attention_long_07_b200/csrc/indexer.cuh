@@ -110,9 +110,9 @@ struct IndexerCfg {
   static constexpr int OFF_BAR = OFF_W + NQ * H_I * 4;
   // barriers: grid schedule 2 + 2 STAGES + 2 RSTAGES + 2 NACC; persistent
   // schedule 7 + STAGES (ready) + 2 RSTAGES + NACC (acc_full) + 2 STAGES
-  // (k_full, k_empty) + NACC (acc_empty) + 2 (q_conv), every array reserved
-  // in both forms
-  static constexpr int NBAR = 9 + 3 * STAGES + 2 * RSTAGES + 2 * NACC;
+  // (k_full, k_empty) + NACC (acc_empty) + 2 (q_conv) + 2 (q_max), every
+  // array reserved in both forms
+  static constexpr int NBAR = 11 + 3 * STAGES + 2 * RSTAGES + 2 * NACC;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   // f16 queries: descale 2^-sq per query buffer and per accumulator, and the
   // converter teams' partial maxima (team, buffer, warp)
@@ -130,7 +130,8 @@ struct IndexerCfg {
   static_assert(!K_IN_TMEM || (KFP8 && STAGES % CONV_TEAMS == 0), "converter teams own alternate stages");
   static_assert(!PERSIST || NACC % EPI_WG == 0, "each accumulator is drained by one epilogue warpgroup");
   static_assert(2 + 2 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "grid barrier layout");
-  static_assert(!PERSIST || 9 + 3 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "persistent barrier layout");
+  static_assert(!PERSIST || 11 + 3 * STAGES + 2 * RSTAGES + 2 * NACC <= NBAR, "persistent barrier layout");
+  static_assert(!PERSIST || CONV_TEAMS <= 2, "query-maximum barriers");
   static_assert(4 * (2 + NACC) + 4 * 2 * CONV_TEAMS * 4 <= 128, "query-conversion scratch");
   static_assert(!QF16 || (B_TILE / 16) % 128 == 0, "query tile in 16-byte pieces per converter thread");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -586,11 +587,16 @@ __global__ void __launch_bounds__(C::NT, 1)
   // f16 queries: q_conv(buf) once the converter team of the segment's first
   // tile has rewritten the query tile as f16 (128 arrivals)
   auto bar_q_conv = [&](int buf) { return bar0 + 56 + 8 * (3 * C::STAGES + 2 * C::RSTAGES + 2 * C::NACC + buf); };
+  // q_max(team): the team's four partial maxima of a query tile are stored
+  // (128 arrivals; one phase per query tile the team rewrites)
+  auto bar_q_max = [&](int team) {
+    return bar0 + 56 + 8 * (3 * C::STAGES + 2 * C::RSTAGES + 2 * C::NACC + 2 + team);
+  };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* qfac_buf = reinterpret_cast<float*>(smem + C::OFF_QCONV);        // [2]: 2^-sq of each query buffer
   float* qfac_acc = qfac_buf + 2;                                         // [NACC]: 2^-sq of each accumulator
-  uint32_t* qmax_part = reinterpret_cast<uint32_t*>(qfac_acc + C::NACC);  // [team][buf][warp]
+  uint32_t* qmax_part = reinterpret_cast<uint32_t*>(qfac_acc + C::NACC);  // [team][parity][warp]
 
   if (threadIdx.x == 0) {
     mbar_init(bar_drain, C::MMA_THREADS);
@@ -605,6 +611,7 @@ __global__ void __launch_bounds__(C::NT, 1)
         mbar_init(bar_raw_empty(s), 128);
       }
       for (int buf = 0; buf < 2; ++buf) mbar_init(bar_q_conv(buf), 128);
+      for (int team = 0; team < C::CONV_TEAMS; ++team) mbar_init(bar_q_max(team), 128);
     } else {
       for (int s = 0; s < C::STAGES; ++s) {
         mbar_init(bar_k_full(s), 1);
@@ -799,32 +806,38 @@ __global__ void __launch_bounds__(C::NT, 1)
     // exact (f16 keeps 11 significant bits down to 2^-14 and whole multiples
     // of 2^-24 below), and smaller ones move by at most 2^(E-39).  A zero or
     // non-finite maximum keeps sq = 0; sq <= 126 keeps 2^-sq a normal float.
+    int n_widened = 0;   // query tiles this team has rewritten
     auto widen_query = [&](int sg) -> bool {
       const int buf = sg & 1;
       if (!mbar_wait(bar_q_full(buf), (sg >> 1) & 1, abort_flag, 58)) return false;
       uint4* qv = reinterpret_cast<uint4*>(smem + C::OFF_Q + buf * C::B_TILE);
       constexpr int PER = C::B_TILE / 16 / 128;
       const int tt = row;   // 0..127 across the team
-      uint4 x[PER];
       uint32_t m2 = 0;      // the largest magnitude (bf16 bit patterns order as magnitudes)
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
-        x[i] = qv[tt + 128 * i];
-        m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(x[i].x & 0x7FFF7FFFu, x[i].y & 0x7FFF7FFFu),
-                                   __vmaxu2(x[i].z & 0x7FFF7FFFu, x[i].w & 0x7FFF7FFFu)));
+        const uint4 x = qv[tt + 128 * i];
+        m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(x.x & 0x7FFF7FFFu, x.y & 0x7FFF7FFFu),
+                                   __vmaxu2(x.z & 0x7FFF7FFFu, x.w & 0x7FFF7FFFu)));
       }
       uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(m2 & 0xFFFFu, m2 >> 16));
-      uint32_t* part = qmax_part + (team * 2 + buf) * 4;
+      // the team's four warps meet: slot n_widened & 1 is rewritten only after
+      // every warp has passed this phase of q_max and read it
+      const int par = n_widened & 1;
+      ++n_widened;
+      uint32_t* part = qmax_part + (team * 2 + par) * 4;
       if (lane == 0) part[warp & 3] = m;
-      named_bar_sync(1 + team, 128);
+      mbar_arrive_warp(bar_q_max(team));
+      if (!mbar_wait_warp(bar_q_max(team), par, abort_flag, 59)) return false;
       m = max(max(part[0], part[1]), max(part[2], part[3]));
       const int ef = static_cast<int>(m >> 7);   // biased exponent of the maximum
       int sq = 0;
       if (m != 0 && ef < 255) sq = min(141 - ef, 126);
       const float up = __int_as_float((127 + sq) << 23);
 #pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+      for (int i = 0; i < PER; ++i) {   // read again: the same thread's own 16-byte pieces
+        const uint4 x = qv[tt + 128 * i];
+        uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float lo = __uint_as_float(w[e] << 16) * up;

@@ -228,11 +228,6 @@ __device__ __forceinline__ bool device_error_pending() {
   return *reinterpret_cast<volatile int*>(&g_device_error) != 0;
 }
 
-// Named barrier `id` (1..15; 0 is __syncthreads) over `n` threads (a multiple of 32).
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 // ----------------------------------------------------------------------------
 // Proxy fences
 // ----------------------------------------------------------------------------
@@ -501,7 +496,7 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 // Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into
 // another CTA's shared memory in the cluster; completes the bytes on that
-// CTA's mbarrier.  A plain (non-multicast) copy.
+// CTA's mbarrier.  One destination CTA per copy.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
                                                   uint32_t bar_cluster) {
   asm volatile(

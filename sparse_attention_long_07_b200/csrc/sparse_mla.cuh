@@ -23,10 +23,10 @@
 // selected row and no MMA is duplicated.  Random-row gathers are bound by
 // the rate at which an SM can have rows requested and in flight, so eight
 // warps issue them (warp w the four rows 4w .. 4w+3 of a tile, one gather4
-// per atom) into a seven-deep ring.  The two partial score tiles are
+// per atom) into a six-deep ring.  The two partial score tiles are
 // exchanged through distributed shared memory (each CTA stages its part in its
-// own shared memory and one bulk copy moves it into the peer's buffer,
-// completing on the peer's mbarrier); both CTAs add them in the same
+// own shared memory and bulk copies, one per softmax warp, move it into the
+// peer's buffer, completing on the peer's mbarrier); both CTAs add them in the same
 // commutative way, so both hold bit-identical scores and take the same
 // softmax decisions.  Tensor memory holds O, three score buffers (a tile's P,
 // in bf16, overwrites its scores once they are in registers) and this CTA's
@@ -36,9 +36,10 @@
 // max grows by more than 2^8, which is exact arithmetic with the same final
 // normalisation.
 //
-// Roles per CTA: warps 0-7 query load, softmax and epilogue (a head row and
-// half of a tile's columns per thread), warp 8 MMA issuer (and TMEM owner),
-// warps 9.. gather (eight with two CTAs, one with one CTA).
+// Roles per CTA: warps 0-7 query load, softmax and epilogue (two teams of
+// four warps taking alternate tiles, a head row and all of a tile's columns
+// per thread), warp 8 MMA issuer (and TMEM owner), warps 9.. gather (eight
+// with two CTAs, one with one CTA).
 #pragma once
 
 #include "common.cuh"
@@ -72,23 +73,22 @@ struct MlaCfg {
   // only after it had consumed tile j - 4, the buffer's previous content.
   static constexpr int XR = 4;
   static constexpr int OFF_X = OFF_C + NS * C_STAGE;
-  static constexpr int XS = 2;                             // outgoing tiles staged (double buffer)
+  static constexpr int XS = 2;                             // outgoing tiles staged (one per softmax team)
   static constexpr int OFF_XS = OFF_X + XR * X_BYTES;
-  // softmax warps: two per TMEM lane quarter, each thread one head row and
-  // half of a tile's columns; the pair exchanges row maxima (by tile parity)
-  // and, at the end, row sums through shared memory
+  // softmax warps: two teams of four (one warp per TMEM lane quarter) taking
+  // alternate tiles, each thread one head row and all of a tile's columns;
+  // the teams pass the softmax reference max along through shared memory and
+  // add their row sums at the end
   static constexpr int NSM = 8;
-  static constexpr int HB = BN / 2;                        // columns of a tile per softmax thread
-  static constexpr int OFF_MX = OFF_XS + XS * X_BYTES;     // [2 parities][2 halves][128] fp32
-  static constexpr int OFF_LS = OFF_MX + 2 * 2 * 128 * 4;  // [2 halves][128] fp32
+  static constexpr int OFF_MX = OFF_XS + XS * X_BYTES;     // [2 teams][128] published, [2 teams][128] final
+  static constexpr int OFF_LS = OFF_MX + 2 * 2 * 128 * 4;  // [2 teams][128] fp32
   static constexpr int OFF_MASK = OFF_LS + 2 * 128 * 4;
   static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
   static constexpr int NSB = 3;                            // S buffers (each later holds its P)
   static constexpr int LOOKAHEAD = 2;                      // QK tiles issued ahead of PV
   // q_ready, c_full/c_empty per stage, 3 per S buffer, x_full per receive
-  // buffer, drain, xs_full, xs_free per staging buffer, and per lane quarter
-  // the pair's max exchange (two tile parities) and row-sum exchange
-  static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + XR + 3 + XS + 4 * 3;
+  // buffer, drain, m_pub per team, and per lane quarter the row-sum exchange
+  static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + XR + 1 + 2 + 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   // tensor memory columns: O [0, DVS); S[NSB] (fp32, BN each; P of the same
@@ -119,7 +119,7 @@ struct MlaCfg {
   static_assert(TMEM_USED <= 512, "tensor memory");
   static_assert(OFF_C % 1024 == 0 && C_STAGE % 1024 == 0 && C_ATOM_BYTES % 1024 == 0, "swizzle atoms");
   static_assert(SPLIT == 1 || NA_MAX <= 32, "one lane per atom");
-  static_assert(HB % 16 == 0 && (DVS / 2) % 16 == 0 && QCOLS % 8 == 0, "column halves of the softmax threads");
+  static_assert(BN == 32 && (DVS / 2) % 16 == 0 && QCOLS % 8 == 0, "softmax rows (32 columns) and column halves");
   static_assert(OFF_XS % 16 == 0 && OFF_MX % 16 == 0, "bulk-copy / vector alignment");
   static_assert(OFF_X % 16 == 0 && OFF_XS % 16 == 0 && OFF_BAR % 8 == 0, "vector / bulk-copy / barrier alignment");
 };
@@ -186,15 +186,12 @@ __global__ void __launch_bounds__(C::NT, 1)
   constexpr int XB0 = SB0 + 3 * C::NSB;
   auto bar_x_full = [&](int b) { return bar0 + 8 * (XB0 + b); };          // b < XR
   const uint32_t bar_drain = bar0 + 8 * (XB0 + C::XR);
-  // outgoing staging: every row written (one arrival per softmax thread) /
-  // staging buffer b read by its last copy (thread 0)
-  const uint32_t bar_xs_full = bar0 + 8 * (XB0 + C::XR + 1);
-  auto bar_xs_free = [&](int b) { return bar0 + 8 * (XB0 + C::XR + 2 + b); };
-  // the two softmax warps of lane quarter q meet here (64 arrivals): row
-  // maxima of tiles of parity par, and the row sums at the end
-  constexpr int PB0 = XB0 + C::XR + 2 + C::XS;
-  auto bar_pair_mx = [&](int q, int par) { return bar0 + 8 * (PB0 + 2 * q + par); };
-  auto bar_pair_l = [&](int q) { return bar0 + 8 * (PB0 + 8 + q); };
+  // m_pub(c): softmax team c published the reference max of its latest tile
+  // (128 arrivals, one phase per tile of the team but its last)
+  auto bar_m_pub = [&](int team) { return bar0 + 8 * (XB0 + C::XR + 1 + team); };
+  // the two softmax warps of lane quarter q (one per team) meet here (64
+  // arrivals) with their row sums at the end
+  auto bar_pair_l = [&](int q) { return bar0 + 8 * (XB0 + C::XR + 3 + q); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   int* ntiles_s = reinterpret_cast<int*>(smem + C::OFF_MISC + 8);
@@ -212,17 +209,12 @@ __global__ void __launch_bounds__(C::NT, 1)
     for (int a = 0; a < C::NSB; ++a) {
       mbar_init(bar_s_full(a), 1);
       mbar_init(bar_pv_done(a), 1);
-      mbar_init(bar_p_full(a), C::NSM * 32);
+      mbar_init(bar_p_full(a), C::NSM * 16);   // the four warps of the tile's team
     }
     for (int b = 0; b < C::XR; ++b) mbar_init(bar_x_full(b), 1);   // armed locally; filled by the peer's copy
     mbar_init(bar_drain, 1);
-    mbar_init(bar_xs_full, C::NSM * 32);
-    for (int b = 0; b < C::XS; ++b) mbar_init(bar_xs_free(b), 1);
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(bar_pair_mx(q, 0), 64);
-      mbar_init(bar_pair_mx(q, 1), 64);
-      mbar_init(bar_pair_l(q), 64);
-    }
+    for (int team = 0; team < 2; ++team) mbar_init(bar_m_pub(team), C::NSM * 16);
+    for (int q = 0; q < 4; ++q) mbar_init(bar_pair_l(q), 64);
     *abort_flag = 0;
     *ntiles_s = 0;
     // an error recorded earlier by any CTA of this library: skip the work
@@ -395,17 +387,17 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    // Thread (head row h, column half c): warps q4 and q4 + 4 share the TMEM
-    // lanes 32 q4 .. 32 q4 + 31; warp q4 + 4c takes columns [c HB, c HB + HB)
-    // of every score tile, columns [c DVS/2, ...) of O, and the 8-column
+    // Thread (head row h, team c): warps q4 and q4 + 4 share the TMEM lanes
+    // 32 q4 .. 32 q4 + 31; warp q4 + 4c takes the tiles of team c (all their
+    // columns), columns [c DVS/2, ...) of O in the epilogue, and the 8-column
     // chunks c, c + 2, ... of the query slice.
     const int q4 = warp & 3, c = warp >> 2;
     const int h = q4 * 32 + lane;                          // head row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t x_peer = C::SPLIT == 2 ? mapa_shared(smem_u32(xbuf), peer) : 0u;
     const uint32_t bar_x_full_peer0 = C::SPLIT == 2 ? mapa_shared(bar_x_full(0), peer) : 0u;
-    float m_used = -INFINITY;    // running max (log2 units) the exponentials are taken against
-    float l_run = 0.f;           // this thread's columns only; the pair adds at the end
+    float m_used = -INFINITY;    // reference max (log2 units) of this team's latest tile
+    float l_run = 0.f;           // this team's tiles, against m_used; the teams add at the end
     bool ok = true;
     // Query slice of head row h (the gathered columns) into TMEM lane h: the A
     // operand of every QK MMA.  Rows h >= H hold zeros.
@@ -440,72 +432,64 @@ __global__ void __launch_bounds__(C::NT, 1)
       tc_fence_before();
       mbar_arrive_warp(bar_q_ready);
     }
-    // Load this thread's half of tile j's partial scores S[j % 3] and (2-CTA
-    // split) start sending them to the peer.  Tile it+1 is started before
-    // tile it is finished, so the exchange of a tile has a whole softmax
-    // iteration to complete.  Staging row h holds 8 16-byte chunks, chunk k
-    // at slot (k + h) & 7 (no bank conflicts); this thread writes chunks 4c ..
-    auto load_and_push = [&](int j, float* dst) -> bool {
-      const int sb = j % C::NSB;
-      if (!mbar_wait_warp(bar_s_full(sb), (j / C::NSB) & 1, abort_flag, 26)) return false;
+    // Team c takes tiles j = c, c + 2, ...; a thread owns head row h of its
+    // team's tiles, all BN columns, so a tile's row maximum needs no partner.
+    // The reference max the exponentials are taken against is one sequence
+    // over the tiles (O accumulates every tile's P against it): team c reads
+    // the decision of tile j - 1 (the other team's) from m_pub and publishes
+    // its own for tile j + 1.  Each team sums its own tiles' probabilities
+    // against the reference it last used; the epilogue brings both sums to the
+    // final reference.
+    //
+    // 2-CTA split: a tile's partial scores go to the peer as four bulk copies,
+    // one per warp (its 32 rows of the team's staging buffer), completing on
+    // the peer's x_full(j % XR); team c's first warp arms that phase with the
+    // bytes to expect.  A tile is sent when its team starts on it, after the
+    // team took tile j - 2 from the peer, which the peer sent only once it had
+    // finished tile j - 4 -- the previous content of receive buffer j % XR.
+    // Staging row h holds BN / 4 16-byte chunks, chunk k at slot (k + h) mod
+    // (BN / 4) (no bank conflicts); the receiver reads with the same rotation.
+    float* m_pub = mx_s;                                   // [2 teams][128]: reference after the team's last tile
+    float sv[C::BN];
+    for (int j = c; ok && j < n_tiles; j += 2) {
+      const int sb = j % C::NSB;   // S buffer of this tile; its P goes there too
+      if (!mbar_wait_warp(bar_s_full(sb), (j / C::NSB) & 1, abort_flag, 26)) { ok = false; break; }
       tc_fence_after();
-      uint32_t raw[C::HB];
-      tmem_ld16(tmem + lane_base + C::TMEM_S + sb * C::BN + c * C::HB, raw);
-      tmem_wait_ld();
+      {
+        uint32_t raw[C::BN];
+        tmem_ld32(tmem + lane_base + C::TMEM_S + sb * C::BN, raw);
+        tmem_wait_ld();
 #pragma unroll
-      for (int k = 0; k < C::HB; ++k) dst[k] = __uint_as_float(raw[k]);
+        for (int k = 0; k < C::BN; ++k) sv[k] = __uint_as_float(raw[k]);
+      }
       if (C::SPLIT == 2) {
-        // The tile goes to the peer in one bulk copy: every thread stages its
-        // half row, then thread 0 copies the 128 rows.  Staging buffer j & 1
-        // was last read by the copy of tile j - 2.
-        const int xr = j % C::XR;    // receive buffer of tile j, on both CTAs
-        const int xb = j & 1;
-        if (threadIdx.x == 0) {
-          // receive side: arm tile j's phase with the bytes the peer will send
-          mbar_arrive_expect_tx(bar_x_full(xr), C::X_BYTES);
-          if (j >= 2) {
-            bulk_wait_group_read<1>();   // every copy but the last one (tile j - 1) has read its source
-            mbar_arrive(bar_xs_free(xb));
-          }
-        }
-        if (j >= 2 && !mbar_wait_warp(bar_xs_free(xb), ((j >> 1) - 1) & 1, abort_flag, 33)) return false;
-        float* row = xs + xb * (C::X_BYTES / 4) + h * C::BN;
+        const int xr = j % C::XR;
+        if (q4 == 0 && lane == 0) mbar_arrive_expect_tx(bar_x_full(xr), C::X_BYTES);
+        // this warp's rows of the staging buffer were last read by its copy of tile j - 2
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        float* row = xs + c * (C::X_BYTES / 4) + h * C::BN;
 #pragma unroll
-        for (int k = 0; k < C::HB / 4; ++k) {
-          const int slot = (4 * c + k + h) & (C::BN / 4 - 1);
-          *reinterpret_cast<float4*>(row + slot * 4) = make_float4(dst[4 * k], dst[4 * k + 1], dst[4 * k + 2],
-                                                                   dst[4 * k + 3]);
+        for (int k = 0; k < C::BN / 4; ++k) {
+          const int slot = (k + h) & (C::BN / 4 - 1);
+          *reinterpret_cast<float4*>(row + slot * 4) = make_float4(sv[4 * k], sv[4 * k + 1], sv[4 * k + 2],
+                                                                   sv[4 * k + 3]);
         }
         fence_proxy_async_smem();
-        mbar_arrive_warp(bar_xs_full);
-        int go = 1;
-        if (threadIdx.x == 0) {
-          // all rows staged (the peer's buffer xr is free: see XR)
-          go = mbar_wait(bar_xs_full, j & 1, abort_flag, 34);
-          if (go) {
-            bulk_copy_to_peer(x_peer + xr * C::X_BYTES, smem_u32(xs + xb * (C::X_BYTES / 4)), C::X_BYTES,
-                              bar_x_full_peer0 + 8 * xr);
-            bulk_commit_group();
-          }
+        __syncwarp();
+        if (lane == 0) {
+          constexpr uint32_t kWarpBytes = 32 * C::BN * 4;
+          bulk_copy_to_peer(x_peer + xr * C::X_BYTES + q4 * kWarpBytes,
+                            smem_u32(xs + c * (C::X_BYTES / 4)) + q4 * kWarpBytes, kWarpBytes,
+                            bar_x_full_peer0 + 8 * xr);
+          bulk_commit_group();
         }
-        // warp 0 leaves together if thread 0 gave up; other warps see the abort flag
-        if (__shfl_sync(0xFFFFFFFFu, go, 0) == 0) return false;
-      }
-      return true;
-    };
-    float sv[C::HB], s_next[C::HB];
-    if (n_tiles > 0 && !load_and_push(0, sv)) ok = false;
-    for (int it = 0; ok && it < n_tiles; ++it) {
-      const int sb = it % C::NSB;   // S buffer of this tile; its P goes there too
-      if (it + 1 < n_tiles && !load_and_push(it + 1, s_next)) { ok = false; break; }
-      if (C::SPLIT == 2) {
         // the copy completes on this CTA's own barrier: CTA-scope acquire, as for a TMA load
-        const int xr = it % C::XR;
-        if (!mbar_wait_warp(bar_x_full(xr), (it / C::XR) & 1, abort_flag, 28)) { ok = false; break; }
+        if (!mbar_wait_warp(bar_x_full(xr), (j / C::XR) & 1, abort_flag, 28)) { ok = false; break; }
         const float* xrow = xbuf + xr * (C::X_BYTES / 4) + h * C::BN;
 #pragma unroll
-        for (int k = 0; k < C::HB / 4; ++k) {
-          const int slot = (4 * c + k + h) & (C::BN / 4 - 1);
+        for (int k = 0; k < C::BN / 4; ++k) {
+          const int slot = (k + h) & (C::BN / 4 - 1);
           const float4 v = *reinterpret_cast<const float4*>(xrow + slot * 4);
           sv[4 * k] += v.x;
           sv[4 * k + 1] += v.y;
@@ -514,78 +498,84 @@ __global__ void __launch_bounds__(C::NT, 1)
         }
       }
       // validity of the tile's entries (written by the producer before it armed c_full)
-      if (!mbar_wait_warp(bar_c_full(it % C::NS), (it / C::NS) & 1, abort_flag, 29)) { ok = false; break; }
-      const uint32_t vmask = mask_s[it % C::NS] >> (c * C::HB);
+      if (!mbar_wait_warp(bar_c_full(j % C::NS), (j / C::NS) & 1, abort_flag, 29)) { ok = false; break; }
+      const uint32_t vmask = mask_s[j % C::NS];
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int j = 0; j < C::HB; ++j) {
-        sv[j] = ((vmask >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
-        mx[j & 3] = fmaxf(mx[j & 3], sv[j]);
+      for (int k = 0; k < C::BN; ++k) {
+        sv[k] = ((vmask >> k) & 1u) ? sv[k] * p.scale_log2 : -INFINITY;
+        mx[k & 3] = fmaxf(mx[k & 3], sv[k]);
       }
-      // the row's max over the whole tile: this half's, then the partner's
-      // (bounded waits: a partner that gave up never arrives, and this warp
-      // then gives up too instead of waiting for good)
-      float* mxp = mx_s + (it & 1) * 256;
-      mxp[c * 128 + h] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      mbar_arrive_warp(bar_pair_mx(q4, it & 1));
-      if (!mbar_wait_warp(bar_pair_mx(q4, it & 1), (it >> 1) & 1, abort_flag, 38)) { ok = false; break; }
-      const float mt = fmaxf(mxp[h], mxp[128 + h]);
-      float corr = 1.f;
-      if (mt > m_used + C::kRescaleThreshold) {
-        corr = exp2f(m_used - mt);   // 0 on the first tile with a valid entry
-        m_used = mt;
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      // the reference after tile j - 1 (the other team's decision)
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        if (!mbar_wait_warp(bar_m_pub(c ^ 1), ((j - 1) >> 1) & 1, abort_flag, 38)) { ok = false; break; }
+        m_prev = m_pub[(c ^ 1) * 128 + h];
       }
-      uint32_t pk[C::HB / 2];
+      const float m_new = mt > m_prev + C::kRescaleThreshold ? mt : m_prev;
+      if (j + 1 < n_tiles) {
+        m_pub[c * 128 + h] = m_new;
+        mbar_arrive_warp(bar_m_pub(c));
+      }
+      const float corr_o = m_new > m_prev ? exp2f(m_prev - m_new) : 1.f;   // 0 on the first valid tile
+      const float corr_l = m_new > m_used ? exp2f(m_used - m_new) : 1.f;
+      m_used = m_new;
+      uint32_t pk[C::BN / 2];
       float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int j = 0; j < C::HB; j += 2) {
-        const float e0 = sv[j] == -INFINITY ? 0.f : ex2_approx(sv[j] - m_used);
-        const float e1 = sv[j + 1] == -INFINITY ? 0.f : ex2_approx(sv[j + 1] - m_used);
+      for (int k = 0; k < C::BN; k += 2) {
+        const float e0 = sv[k] == -INFINITY ? 0.f : ex2_approx(sv[k] - m_used);
+        const float e1 = sv[k + 1] == -INFINITY ? 0.f : ex2_approx(sv[k + 1] - m_used);
         const __nv_bfloat162 b2 = __floats2bfloat162_rn(e0, e1);
         const float2 back = __bfloat1622float2(b2);
-        ps[(j >> 1) & 3] += back.x + back.y;
-        pk[j / 2] = *reinterpret_cast<const uint32_t*>(&b2);
+        ps[(k >> 1) & 3] += back.x + back.y;
+        pk[k / 2] = *reinterpret_cast<const uint32_t*>(&b2);
       }
-      l_run = l_run * corr + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-      // The rescale decision is per head row (and the same in both threads of
-      // the row), but the TMEM accesses below are warp-collective
+      l_run = l_run * corr_l + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+      // O holds the PVs of tiles < j against m_prev.  The rescale decision is
+      // per head row, but the TMEM accesses below are warp-collective
       // (.sync.aligned): the warp rescales if any lane needs it, and lanes
       // that do not multiply by 1.
-      if (__any_sync(0xFFFFFFFFu, corr != 1.f && it > 0)) {
+      if (__any_sync(0xFFFFFFFFu, corr_o != 1.f && j > 0)) {
         // O must hold every earlier PV before it is rescaled in place
-        if (!mbar_wait_warp(bar_pv_done((it - 1) % C::NSB), ((it - 1) / C::NSB) & 1, abort_flag, 31)) {
+        if (!mbar_wait_warp(bar_pv_done((j - 1) % C::NSB), ((j - 1) / C::NSB) & 1, abort_flag, 31)) {
           ok = false;
           break;
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int c0 = c * (C::DVS / 2); c0 < (c + 1) * (C::DVS / 2); c0 += 16) {
+        for (int c0 = 0; c0 < C::DVS; c0 += 16) {
           uint32_t o[16];
           tmem_ld16(tmem + lane_base + c0, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * corr);
+          for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * corr_o);
           tmem_st16(tmem + lane_base + c0, o);
         }
         tmem_wait_st();
       }
-      // P row h, this thread's columns (bf16 pairs), over the scores of this
-      // tile (already in registers); the PV MMA reads it from there
-      tmem_st8(tmem + lane_base + C::TMEM_S + sb * C::BN + c * (C::HB / 2), pk);
+      // P row h (bf16 pairs) over the first BN / 2 columns of the S buffer; the PV MMA reads it from there
+      tmem_st16(tmem + lane_base + C::TMEM_S + sb * C::BN, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(bar_p_full(sb));
-#pragma unroll
-      for (int k = 0; k < C::HB; ++k) sv[k] = s_next[k];
     }
-    if (C::SPLIT == 2 && threadIdx.x == 0) bulk_wait_group<0>();   // outgoing copies have completed
+    if (C::SPLIT == 2 && lane == 0) bulk_wait_group<0>();   // this warp's outgoing copies have completed
     if (lane == 0) DSA_PROF_SPAN(63, t_role);
     // ------------------------------------------------------------ epilogue
-    // the row sum over both halves
+    // the row sum over both teams, against the final reference (the larger
+    // of the two teams' last ones: the reference never decreases)
     l_s[c * 128 + h] = l_run;
+    m_pub[256 + c * 128 + h] = m_used;
     mbar_arrive_warp(bar_pair_l(q4));
     if (!mbar_wait_warp(bar_pair_l(q4), 0, abort_flag, 39)) ok = false;
-    l_run = l_s[h] + l_s[128 + h];
+    {
+      const float m0 = m_pub[256 + h], m1 = m_pub[256 + 128 + h];
+      const float l0 = l_s[h], l1 = l_s[128 + h];
+      m_used = fmaxf(m0, m1);
+      l_run = (l0 > 0.f ? l0 * exp2f(m0 - m_used) : 0.f) + (l1 > 0.f ? l1 * exp2f(m1 - m_used) : 0.f);
+    }
     const int t_out = static_cast<int>(t);
     if (ok && n_tiles > 0) {
       const int j = n_tiles - 1;
