@@ -38,8 +38,8 @@
 //
 // Roles per CTA: warps 0-7 query load, softmax and epilogue (two teams of
 // four warps taking alternate tiles, a head row and all of a tile's columns
-// per thread), warp 8 MMA issuer (and TMEM owner), warps 9.. gather (eight
-// with two CTAs, one with one CTA).
+// per thread), warps 8 and 9 MMA issuers (QK and PV; warp 8 owns the TMEM),
+// warps 10.. gather (eight with two CTAs, one with one CTA).
 #pragma once
 
 #include "common.cuh"
@@ -85,7 +85,6 @@ struct MlaCfg {
   static constexpr int OFF_MASK = OFF_LS + 2 * 128 * 4;
   static constexpr int OFF_BAR = (OFF_MASK + NS * 4 + 7) / 8 * 8;
   static constexpr int NSB = 3;                            // S buffers (each later holds its P)
-  static constexpr int LOOKAHEAD = 2;                      // QK tiles issued ahead of PV
   // q_ready, c_full/c_empty per stage, 3 per S buffer, x_full per receive
   // buffer, drain, m_pub per team, and per lane quarter the row-sum exchange
   static constexpr int NBAR = 1 + 2 * NS + 3 * NSB + XR + 1 + 2 + 4;
@@ -99,12 +98,12 @@ struct MlaCfg {
   static constexpr int QCOLS = NA_MAX * ATOM / 2;
   static constexpr int TMEM_USED = TMEM_Q + QCOLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
-  // roles: warps 0-3 softmax and epilogue, MMA_WARP the MMA issuer (and TMEM
-  // owner), then NPROD gather warps: more warps issuing TMA gathers raise the
-  // rate at which one SM requests rows
+  // roles: warps 0 .. NSM-1 softmax and epilogue, MMA_WARP the QK issuer (and
+  // TMEM owner), MMA_WARP + 1 the PV issuer, then NPROD gather warps: more
+  // warps issuing TMA gathers raise the rate at which one SM requests rows
   static constexpr int MMA_WARP = NSM;
   static constexpr int NPROD = SPLIT == 2 ? BN / 4 : 1;   // one per four-row group of a tile
-  static constexpr int PROD_WARP0 = NSM + 1;
+  static constexpr int PROD_WARP0 = NSM + 2;
   static constexpr int NT = (PROD_WARP0 + NPROD) * 32;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, BN, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, DVS, false, true);
@@ -114,7 +113,7 @@ struct MlaCfg {
   static_assert(DVS % ATOM == 0 && DVS <= 256 && DVS % 16 == 0, "PV N");
   static_assert(SPLIT == 1 || NV <= NA1, "rank 1 must gather its value columns");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
-  static_assert(LOOKAHEAD < NSB && LOOKAHEAD + 2 <= NS, "S buffers and gather stages in flight");
+  static_assert(NSB <= NS, "the rows of every score tile in flight stay resident");
   static_assert(QCOLS % 8 == 0, "query columns are stored eight at a time");
   static_assert(TMEM_USED <= 512, "tensor memory");
   static_assert(OFF_C % 1024 == 0 && C_STAGE % 1024 == 0 && C_ATOM_BYTES % 1024 == 0, "swizzle atoms");
@@ -212,7 +211,7 @@ __global__ void __launch_bounds__(C::NT, 1)
       mbar_init(bar_p_full(a), C::NSM * 16);   // the four warps of the tile's team
     }
     for (int b = 0; b < C::XR; ++b) mbar_init(bar_x_full(b), 1);   // armed locally; filled by the peer's copy
-    mbar_init(bar_drain, 1);
+    mbar_init(bar_drain, 2);   // both MMA threads
     for (int team = 0; team < 2; ++team) mbar_init(bar_m_pub(team), C::NSM * 16);
     for (int q = 0; q < 4; ++q) mbar_init(bar_pair_l(q), 64);
     *abort_flag = 0;
@@ -327,59 +326,59 @@ __global__ void __launch_bounds__(C::NT, 1)
       }
     }
     if (lane == 0 && w == 0) DSA_PROF_SPAN(61, t_role);
-  } else if (warp == C::MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == C::MMA_WARP || warp == C::MMA_WARP + 1) {
+    // ------------------------------------------------------------ MMA issuers
+    // Lane 0 of MMA_WARP issues every QK, lane 0 of MMA_WARP + 1 every PV, so
+    // that a PV goes out as soon as its P is stored instead of waiting behind
+    // the (much longer) issue of a QK.  Each thread's commits track its own
+    // MMAs.  QK(j) waits for the gathered rows of tile j and for PV(j - NSB),
+    // the last reader of S buffer j % NSB; PV(j) waits for P(j), which the
+    // softmax stores only after QK(j) completed, so its commit of c_empty also
+    // covers QK(j)'s reads of the stage.
+    const bool qk_thread = warp == C::MMA_WARP;
     if (lane == 0 && n_tiles > 0) {
-      auto issue_pv = [&](int j) -> bool {
-        const int sb = j % C::NSB;
-        if (!mbar_wait(bar_p_full(sb), (j / C::NSB) & 1, abort_flag, 22)) return false;
+      bool ok = true;
+      if (qk_thread) {
+        const int ksteps = na * C::KPA;
+        ok = mbar_wait(bar_q_ready, 0, abort_flag, 23);
         tc_fence_after();
-        const uint32_t v_base = s_c + (j % C::NS) * C::C_STAGE;
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int s = j % C::NS;
+          const int sb = j % C::NSB;
+          if (!mbar_wait(bar_c_full(s), (j / C::NS) & 1, abort_flag, 24)) break;
+          // S buffer sb last held P(j - NSB): its PV must have read it
+          if (!mbar_wait(bar_pv_done(sb), ((j / C::NSB) & 1) ^ 1, abort_flag, 25)) break;
+          tc_fence_after();
+          const uint32_t c_base = s_c + s * C::C_STAGE;
+          for (int kk = 0; kk < ksteps; ++kk) {
+            // A = the query slice in tensor memory (8 columns per 16-wide k-step)
+            const int atom = kk / C::KPA;
+            const int off = (kk % C::KPA) * 32;
+            const uint64_t bd = smem_desc(c_base + atom * C::C_ATOM_BYTES + off, 16, 8 * C::SWB, C::SWZ);
+            umma_ts(tmem + C::TMEM_S + sb * C::BN, tmem + C::TMEM_Q + kk * 8, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar_s_full(sb));
+        }
+      } else {
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int sb = j % C::NSB;
+          if (!mbar_wait(bar_p_full(sb), (j / C::NSB) & 1, abort_flag, 22)) break;
+          tc_fence_after();
+          const uint32_t v_base = s_c + (j % C::NS) * C::C_STAGE;
 #pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          // A = P (bf16 pairs in S buffer sb): 16 k-elements = 8 columns per step
-          const uint32_t a_tmem = tmem + C::TMEM_S + sb * C::BN + kk * 8;
-          const uint64_t bd = smem_desc(v_base + kk * 16 * C::SWB, C::C_ATOM_BYTES, 8 * C::SWB, C::SWZ);
-          umma_ts(tmem, a_tmem, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            // A = P (bf16 pairs in S buffer sb): 16 k-elements = 8 columns per step
+            const uint32_t a_tmem = tmem + C::TMEM_S + sb * C::BN + kk * 8;
+            const uint64_t bd = smem_desc(v_base + kk * 16 * C::SWB, C::C_ATOM_BYTES, 8 * C::SWB, C::SWZ);
+            umma_ts(tmem, a_tmem, bd, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(bar_c_empty(j % C::NS));
+          umma_commit(bar_pv_done(sb));
         }
-        umma_commit(bar_c_empty(j % C::NS));
-        umma_commit(bar_pv_done(sb));
-        return true;
-      };
-      const int ksteps = na * C::KPA;
-      // QK(j) -> S[j % NSB]; issued LOOKAHEAD tiles ahead of the PV that trails it
-      auto issue_qk = [&](int j) -> bool {
-        const int s = j % C::NS;
-        const int sb = j % C::NSB;
-        if (!mbar_wait(bar_c_full(s), (j / C::NS) & 1, abort_flag, 24)) return false;
-        // S buffer sb last held P(j - NSB): its PV must have read it
-        if (!mbar_wait(bar_pv_done(sb), ((j / C::NSB) & 1) ^ 1, abort_flag, 25)) return false;
-        tc_fence_after();
-        const uint32_t c_base = s_c + s * C::C_STAGE;
-        for (int kk = 0; kk < ksteps; ++kk) {
-          // A = the query slice in tensor memory (8 columns per 16-wide k-step)
-          const int atom = kk / C::KPA;
-          const int off = (kk % C::KPA) * 32;
-          const uint64_t bd = smem_desc(c_base + atom * C::C_ATOM_BYTES + off, 16, 8 * C::SWB, C::SWZ);
-          umma_ts(tmem + C::TMEM_S + sb * C::BN, tmem + C::TMEM_Q + kk * 8, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_s_full(sb));
-        return true;
-      };
-      // QK runs LOOKAHEAD tiles ahead of PV, and QK(j + LOOKAHEAD) is issued
-      // before PV(j): it needs only S buffer (j + LOOKAHEAD) % NSB, which the
-      // softmax frees when it starts on tile j - 1, so the tensor core works on
-      // the next scores while the softmax finishes tile j.
-      bool ok = mbar_wait(bar_q_ready, 0, abort_flag, 23);
-      tc_fence_after();
-      for (int j = 0; ok && j < C::LOOKAHEAD && j < n_tiles; ++j) ok = issue_qk(j);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + C::LOOKAHEAD < n_tiles && !issue_qk(j + C::LOOKAHEAD)) break;
-        if (!issue_pv(j)) break;
       }
     }
     if (lane == 0) {
-      DSA_PROF_SPAN(62, t_role);
+      DSA_PROF_SPAN(qk_thread ? 62 : 20, t_role);
       umma_commit(bar_drain);
       long long t0 = clock64();
       while (!mbar_try_wait(bar_drain, 0) && clock64() - t0 < kWaitLimitCycles) {
