@@ -18,9 +18,11 @@
 // output accumulator O[128 x 512] alone fills all 512 columns of an SM's
 // tensor memory, so the released shape runs on a cluster of two CTAs (two
 // SMs): CTA r owns output columns [256 r, 256 r + 256).  QK is split along K
-// the same way -- CTA 0 multiplies latent columns [0, 256), CTA 1 columns
-// [256, 576) -- so each CTA needs only its own 256 or 320 columns of every
-// selected row and no MMA is duplicated.  Random-row gathers are bound by
+// in halves -- CTA 0 multiplies columns [0, 288), CTA 1 columns [288, 576),
+// 18 k-steps each, since a CTA's tile time is its QK issue -- so each CTA
+// gathers 320 columns of every selected row (CTA 0 [0, 320), CTA 1
+// [256, 576): its values and its QK half, one 64-column atom shared) and no
+// MMA is duplicated.  Random-row gathers are bound by
 // the rate at which an SM can have rows requested and in flight, so eight
 // warps issue them (warp w the four rows 4w .. 4w+3 of a tile, one gather4
 // per atom) into a six-deep ring.  The two partial score tiles are
@@ -58,10 +60,17 @@ struct MlaCfg {
   static constexpr int NATOM_ALL = DQK / ATOM;
   static constexpr int DVS = DV / SPLIT;                  // output columns per CTA
   static constexpr int NV = DVS / ATOM;                   // value atoms per CTA
-  static constexpr int SPLIT_ATOM = SPLIT == 1 ? NATOM_ALL : DVS / ATOM;
-  static constexpr int NA0 = SPLIT_ATOM;                  // atoms gathered by rank 0
-  static constexpr int NA1 = NATOM_ALL - SPLIT_ATOM;      // atoms gathered by rank 1
+  // QK reduction: CTA r multiplies query / latent elements [r QKH, r QKH + QKH)
+  static constexpr int QKH = DQK / SPLIT;
+  static constexpr int KSTEPS = QKH / 16;                 // QK k-steps per tile and CTA
+  // atoms gathered: rank 0 from atom 0, rank 1 from atom A0_R1 (its first
+  // value column), each through the last atom its values or QK elements reach
+  static constexpr int A0_R1 = SPLIT == 1 ? 0 : DVS / ATOM;
+  static constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
+  static constexpr int NA0 = SPLIT == 1 ? NATOM_ALL : (NV > cdiv(QKH, ATOM) ? NV : cdiv(QKH, ATOM));
+  static constexpr int NA1 = SPLIT == 1 ? 0 : NATOM_ALL - A0_R1;
   static constexpr int NA_MAX = NA0 > NA1 ? NA0 : NA1;
+  static constexpr int KF1 = SPLIT == 1 ? 0 : (QKH - A0_R1 * ATOM) / 16;   // rank 1's first local k-step
   static constexpr int NS = SPLIT == 1 ? 4 : 6;           // gather ring depth
   static constexpr int C_ATOM_BYTES = BN * SWB;
   static constexpr int C_STAGE = NA_MAX * C_ATOM_BYTES;
@@ -95,7 +104,7 @@ struct MlaCfg {
   // query slice this CTA multiplies, bf16 pairs (the A operand of QK)
   static constexpr int TMEM_S = DVS;
   static constexpr int TMEM_Q = DVS + NSB * BN;
-  static constexpr int QCOLS = NA_MAX * ATOM / 2;
+  static constexpr int QCOLS = QKH / 2;
   static constexpr int TMEM_USED = TMEM_Q + QCOLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : (TMEM_USED <= 256 ? 256 : 512);
   // roles: warps 0 .. NSM-1 softmax and epilogue, MMA_WARP the QK issuer (and
@@ -112,6 +121,9 @@ struct MlaCfg {
   static_assert(DQK % ATOM == 0, "every TMA box stays inside the row: no partial atoms");
   static_assert(DVS % ATOM == 0 && DVS <= 256 && DVS % 16 == 0, "PV N");
   static_assert(SPLIT == 1 || NV <= NA1, "rank 1 must gather its value columns");
+  static_assert(QKH % 16 == 0 && (SPLIT == 1 || (A0_R1 * ATOM <= QKH && 2 * DVS <= DQK)),
+                "QK halves in whole k-steps, rank 1's half inside its atoms");
+  static_assert(SPLIT == 1 || (QKH * 2) % 16 == 0, "16-byte query loads from the half's first element");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(NSB <= NS, "the rows of every score tile in flight stay resident");
   static_assert(QCOLS % 8 == 0, "query columns are stored eight at a time");
@@ -160,8 +172,10 @@ __global__ void __launch_bounds__(C::NT, 1)
   const int64_t t = p.q_begin + r_local;
   const RowInfo ri = locate_row(p.cu_q, p.cu_k, p.B, t);
   const int32_t* __restrict__ idx_row = p.idx + r_local * p.topk;
-  const int a0 = rank == 0 ? 0 : C::SPLIT_ATOM;           // first atom of this CTA's columns (global)
+  const int a0 = rank == 0 ? 0 : C::A0_R1;                // first atom of this CTA's columns (global)
   const int na = rank == 0 ? C::NA0 : C::NA1;             // atoms of this CTA's columns
+  const int kf = rank == 0 ? 0 : C::KF1;                  // first QK k-step (local to the gathered atoms)
+  const int qk_lo = static_cast<int>(rank) * C::QKH;      // first query / latent element of this CTA's QK
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -339,7 +353,6 @@ __global__ void __launch_bounds__(C::NT, 1)
     if (lane == 0 && n_tiles > 0) {
       bool ok = true;
       if (qk_thread) {
-        const int ksteps = na * C::KPA;
         ok = mbar_wait(bar_q_ready, 0, abort_flag, 23);
         tc_fence_after();
         for (int j = 0; ok && j < n_tiles; ++j) {
@@ -350,12 +363,14 @@ __global__ void __launch_bounds__(C::NT, 1)
           if (!mbar_wait(bar_pv_done(sb), ((j / C::NSB) & 1) ^ 1, abort_flag, 25)) break;
           tc_fence_after();
           const uint32_t c_base = s_c + s * C::C_STAGE;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            // A = the query slice in tensor memory (8 columns per 16-wide k-step)
+          for (int ks = 0; ks < C::KSTEPS; ++ks) {
+            // A = the query slice in tensor memory (8 columns per 16-wide k-step);
+            // B = k-step kf + ks of the gathered atoms
+            const int kk = kf + ks;
             const int atom = kk / C::KPA;
             const int off = (kk % C::KPA) * 32;
             const uint64_t bd = smem_desc(c_base + atom * C::C_ATOM_BYTES + off, 16, 8 * C::SWB, C::SWZ);
-            umma_ts(tmem + C::TMEM_S + sb * C::BN, tmem + C::TMEM_Q + kk * 8, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+            umma_ts(tmem + C::TMEM_S + sb * C::BN, tmem + C::TMEM_Q + ks * 8, bd, C::IDESC_QK, ks > 0 ? 1u : 0u);
           }
           umma_commit(bar_s_full(sb));
         }
@@ -398,21 +413,21 @@ __global__ void __launch_bounds__(C::NT, 1)
     float m_used = -INFINITY;    // reference max (log2 units) of this team's latest tile
     float l_run = 0.f;           // this team's tiles, against m_used; the teams add at the end
     bool ok = true;
-    // Query slice of head row h (the gathered columns) into TMEM lane h: the A
+    // Query elements [qk_lo, qk_lo + QKH) of head row h into TMEM lane h: the A
     // operand of every QK MMA.  Rows h >= H hold zeros.
     if (n_tiles > 0) {
       const bool row_ok = h < C::H;
       const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * C::H + (row_ok ? h : 0)) * C::DQK +
-                                                         a0 * C::ATOM);
+                                                         qk_lo);
 #pragma unroll 1
-      for (int c0 = 8 * c; c0 < na * C::ATOM / 2; c0 += 16) {   // 8 columns = 16 bf16 = two 16-byte loads
+      for (int c0 = 8 * c; c0 < C::QCOLS; c0 += 16) {   // 8 columns = 16 bf16 = two 16-byte loads
         uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
         if (row_ok) {
           v0 = __ldg(qrow + c0 / 4);
           v1 = __ldg(qrow + c0 / 4 + 1);
         }
         uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        const int g0 = a0 * C::ATOM + 2 * c0;   // first query element of this chunk
+        const int g0 = qk_lo + 2 * c0;   // first query element of this chunk
         if (p.rope != nullptr && g0 >= C::DV) {
           // RoPE of the rope columns at this row's position: element pair
           // (2i, 2i + 1) of the rope part times (cos, sin) of pair i.
