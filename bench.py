@@ -475,18 +475,77 @@ def extensions_measure(dsa, spec, d, v, out, idx, peaks, n=50):
     return res
 
 
+# The kernel of each stage (a substring of its name in an ncu launch list) and
+# the sources it is compiled from: a recorded DRAM figure counts only while the
+# digest of those sources is the one it was recorded with.
+STAGE_KERNELS = {"indexer": "indexer", "topk": "topk_kernel", "attention": "sparse_mla"}
+STAGE_SOURCES = {"indexer": ("indexer.cuh", "fp8.cuh"), "topk": ("topk.cuh",), "attention": ("sparse_mla.cuh",)}
+COMMON_SOURCES = ("common.cuh", "sm100.cuh", "dsa.cu")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def sources_digest(stage):
+    """sha256 over the stage kernel's own source files and the shared ones."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_attention_long_07_b200", "csrc")
+    for name in STAGE_SOURCES[stage] + COMMON_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
 def load_traffic(stage, workload, alg_bytes_per_launch):
-    """DRAM bytes per launch of the kernel from the committed ncu summary, if it matches."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
+    """DRAM bytes per launch of the kernel from the committed ncu figures, or
+    None when there is none for this stage and workload or the kernel's
+    sources changed since it was taken."""
+    if not os.path.exists(TRAFFIC_PATH):
         return None
     try:
-        with open(path) as f:
+        with open(TRAFFIC_PATH) as f:
             t = json.load(f)
         e = t.get(f"{workload}/{stage}")
-        return None if e is None else e.get("dram_bytes_per_launch")
+        if e is None or e.get("sources_sha256") != sources_digest(stage):
+            return None
+        return e.get("dram_bytes_per_launch")
     except (OSError, ValueError):
         return None
+
+
+def record_traffic(csv_path, workload):
+    """Average DRAM bytes per launch of each stage's kernel from an ncu CSV
+    (--metrics dram__bytes_read.sum,dram__bytes_write.sum ... --csv) into
+    profiles/traffic.json, stamped with the current source digests."""
+    import csv
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "KB": 1e3, "MB": 1e6, "GB": 1e9}
+    launches = {}
+    with open(csv_path) as f:
+        rows = [ln for ln in f if ln.startswith('"')]
+    for r in csv.DictReader(rows):
+        m = r["Metric Name"]
+        if m not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        v = float(r["Metric Value"].replace(",", "")) * scale[r["Metric Unit"]]
+        launches.setdefault((r["ID"], r["Kernel Name"]), {})[m] = v
+    t = {}
+    if os.path.exists(TRAFFIC_PATH):
+        with open(TRAFFIC_PATH) as f:
+            t = json.load(f)
+    t["_note"] = ("DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from ncu on the "
+                  "full-size workload; an entry counts only while sources_sha256 matches the kernel's sources")
+    for stage, pat in STAGE_KERNELS.items():
+        got = [(name, v) for (_, name), v in launches.items() if pat in name and len(v) == 2]
+        if not got:
+            continue
+        rd = sum(v["dram__bytes_read.sum"] for _, v in got) / len(got)
+        wr = sum(v["dram__bytes_write.sum"] for _, v in got) / len(got)
+        t[f"{workload}/{stage}"] = {"kernel": got[0][0].split("(")[0].replace("void ", ""), "launches": len(got),
+                                    "dram_bytes_per_launch": int(round(rd + wr)), "read": int(round(rd)),
+                                    "write": int(round(wr)), "sources_sha256": sources_digest(stage)}
+    with open(TRAFFIC_PATH, "w") as f:
+        json.dump(t, f, indent=1)
+        f.write("\n")
+    return t
 
 
 INDEXER_PREFILL_WORKLOAD = "prefill32k"
@@ -765,7 +824,12 @@ def main():
                     help="batches in flight in the end-to-end measurement (one stream each)")
     ap.add_argument("--no-extensions", action="store_true",
                     help="skip the FP8-indexer, paged, RoPE, up-projection and append measurements")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV", default=None,
+                    help="write profiles/traffic.json from an ncu DRAM-bytes CSV of --workload and exit")
     args = ap.parse_args()
+    if args.record_traffic:
+        print(json.dumps(record_traffic(args.record_traffic, args.workload), indent=1))
+        return
     if args.impl == "reference":
         args.steps = 1 if args.steps is None else args.steps
         args.warmup = 0 if args.warmup is None else args.warmup

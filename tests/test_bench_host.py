@@ -95,3 +95,31 @@ def test_bench_line_carries_every_contract_key(monkeypatch, capsys):
     for key in ("value", "unit", "cores", "kind", "sample"):
         assert key in line["cpu_baseline"], key
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_traffic_counts_only_for_the_sources_it_was_recorded_with(tmp_path, monkeypatch):
+    """profiles/traffic.json figures come from an ncu DRAM-bytes CSV; bench
+    reports one only while the kernel's sources are unchanged."""
+    hdr = ('"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size",'
+           '"Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"\n')
+    rows = []
+    for i, (name, rd, wr) in enumerate([("void indexer_persistent_kernel<X>(A)", "583909888", "19066112"),
+                                        ("void indexer_persistent_kernel<X>(A)", "583909890", "19066110"),
+                                        ("void topk_kernel(B)", "14.9", "0")]):
+        unit = "Mbyte" if "topk" in name else "byte"
+        for m, v in (("dram__bytes_read.sum", rd), ("dram__bytes_write.sum", wr)):
+            rows.append(f'"{i}","1","python","h","{name}","1","7","(1, 1, 1)","(1, 1, 1)","0","10.0",'
+                        f'"Command line profiler metrics","{m}","{unit}","{v}"\n')
+    csv_path = tmp_path / "dram.csv"
+    csv_path.write_text("==PROF== Connected\n" + hdr + "".join(rows))
+    monkeypatch.setattr(bench, "TRAFFIC_PATH", str(tmp_path / "traffic.json"))
+    t = bench.record_traffic(str(csv_path), "decode128k")
+    assert t["decode128k/indexer"]["launches"] == 2
+    assert t["decode128k/indexer"]["dram_bytes_per_launch"] == 583909889 + 19066111
+    assert t["decode128k/topk"]["read"] == 14_900_000 and t["decode128k/topk"]["write"] == 0
+    assert "decode128k/attention" not in t
+    assert bench.load_traffic("indexer", "decode128k", 0) == 583909889 + 19066111
+    assert bench.load_traffic("attention", "decode128k", 0) is None
+    # a different source digest (a changed kernel) withdraws the figure
+    monkeypatch.setattr(bench, "sources_digest", lambda stage: "0" * 64)
+    assert bench.load_traffic("indexer", "decode128k", 0) is None
