@@ -591,14 +591,12 @@ def indexer_prefill_measure(dsa, args, peaks):
 
 
 class _E2ELane:
-    """One batch in flight for the end-to-end measurement: its own stream,
-    device inputs, pinned host copies of the step's inputs, outputs and
-    workspace."""
+    """One batch in flight for the end-to-end measurement: its device inputs,
+    pinned host copies of the step's inputs, outputs and workspace."""
 
     def __init__(self, dsa, spec, d, v, q_chunk, decode):
         dev = d["q"].device
         self.spec, self.d, self.v, self.q_chunk, self.decode = spec, d, v, q_chunk, decode
-        self.stream = torch.cuda.Stream(device=dev)
         cu_k = [int(x) for x in d["cu_k"]]
         # decode: the step's new inputs are the query tensors and the new
         # token's cache rows (the caches are resident device state); prefill:
@@ -621,23 +619,41 @@ class _E2ELane:
         self.ws = torch.empty(dsa.dsa_forward_workspace_size(v, spec.topk, q_chunk), dtype=torch.uint8, device=dev)
         self.h2d = sum(t.numel() * t.element_size() for t in self.host.values())
         self.d2h = self.out_h.numel() * self.out_h.element_size() + self.lse_h.numel() * self.lse_h.element_size()
+        self.ev_in = torch.cuda.Event()        # inputs on the device
+        self.ev_used = torch.cuda.Event()      # the forward that read them (and wrote out / lse) is done
+        self.ev_out = torch.cuda.Event()       # out / lse copied back
+        self.ev_used.record(torch.cuda.current_stream(dev))
+        self.ev_out.record(torch.cuda.current_stream(dev))
 
-    def step(self, dsa):
+    def step(self, dsa, s_in, s_comp, s_out):
+        """One step: inputs in on s_in, the forward on s_comp (every lane's
+        forward on the same stream, so the kernels run one after another as in
+        the device-timed step), outputs back on s_out."""
         d, spec = self.d, self.spec
-        with torch.cuda.stream(self.stream):
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(self.ev_used)     # the previous forward of this lane has read its inputs
             for n in self.names:
                 d[n].copy_(self.host[n], non_blocking=True)
             if self.decode:
                 for n, rd in self.rows_dev.items():
                     rd.copy_(self.host[n], non_blocking=True)
+            self.ev_in.record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(self.ev_in)
+            s_comp.wait_event(self.ev_out)    # out / lse of this lane's previous step are back on the host
+            if self.decode:
                 self.k_bytes.index_copy_(0, self.new_rows, self.rows_dev["k_rows"])
                 d["latent"].index_copy_(0, self.new_rows, self.rows_dev["lat_rows"])
                 if spec.kfp8:
                     d["k_scale"].index_copy_(0, self.new_rows, self.rows_dev["ks_rows"])
             dsa.dsa_forward(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], d["q"], d["latent"], self.v, spec.topk,
-                            spec.softmax_scale, self.out, self.lse, self.ws, q_chunk=self.q_chunk, stream=self.stream)
+                            spec.softmax_scale, self.out, self.lse, self.ws, q_chunk=self.q_chunk, stream=s_comp)
+            self.ev_used.record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(self.ev_used)
             self.out_h.copy_(self.out, non_blocking=True)
             self.lse_h.copy_(self.lse, non_blocking=True)
+            self.ev_out.record(s_out)
 
 
 E2E_MIN_CALLS = 100
@@ -647,9 +663,11 @@ def e2e_measure(dsa, spec, d, v, q_chunk, args, world):
     """dsa_forward through the public API, each step's inputs copied from
     pinned host memory and its outputs copied back.  Several batches are kept
     in flight, as a server would: lane 0 serves the benchmark's batch and the
-    other lanes other batches of the same shape (other seeds), each on its own
-    stream with its own buffers, and the steps go round the lanes, so that one
-    lane's host transfers overlap the other lanes' kernels.  Every step still
+    other lanes other batches of the same shape (other seeds), each with its
+    own buffers, and the steps go round the lanes.  Host-to-device copies run
+    on one stream, the forwards on a second (one after another, as in the
+    device-timed step) and device-to-host copies on a third, so that the
+    transfers of one step overlap the kernels of another.  Every step still
     copies its whole input in and its whole output out."""
     import dataclasses
     dev = d["q"].device
@@ -660,30 +678,29 @@ def e2e_measure(dsa, spec, d, v, q_chunk, args, world):
         spec_j = dataclasses.replace(spec, seed=spec.seed + 500 + j)
         d_j = di.make_inputs(spec_j, device=dev)
         lanes.append(_E2ELane(dsa, spec_j, d_j, type(v)(d_j["cu_q"], d_j["cu_k"], dev), q_chunk, decode))
+    s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
     for i in range(2 * n_lanes):
-        lanes[i % n_lanes].step(dsa)
+        lanes[i % n_lanes].step(dsa, s_in, s_comp, s_out)
     torch.cuda.synchronize()
     n = max(E2E_MIN_CALLS, min(args.steps, 1000))
-    start = torch.cuda.Event(enable_timing=True)
-    ends = [torch.cuda.Event(enable_timing=True) for _ in lanes]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    start.record(lanes[0].stream)
-    for ln in lanes[1:]:
-        ln.stream.wait_event(start)
+    start.record(s_in)
+    s_comp.wait_event(start)
+    s_out.wait_event(start)
     for i in range(n):
-        lanes[i % n_lanes].step(dsa)
-    for e, ln in zip(ends, lanes):
-        e.record(ln.stream)
+        lanes[i % n_lanes].step(dsa, s_in, s_comp, s_out)
+    end.record(s_out)
     torch.cuda.synchronize()
-    ms = max_over_ranks(max(start.elapsed_time(e) for e in ends), world) / n
+    ms = max_over_ranks(start.elapsed_time(end), world) / n
     assert dsa.dsa_device_error() == 0
     h2d, d2h = lanes[0].h2d, lanes[0].d2h
     del lanes
     torch.cuda.empty_cache()
     return {"value": world * spec.T / (ms / 1e3), "unit": "query tokens/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4), "steps": n, "api": "dsa_forward",
-            "batches_in_flight": n_lanes}
+            "batches_in_flight": n_lanes, "streams": "host-to-device, forward, device-to-host"}
 
 
 # --------------------------------------------------------------------------- CPU oracle
