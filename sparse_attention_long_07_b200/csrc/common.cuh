@@ -63,6 +63,27 @@ __device__ __forceinline__ RowInfo locate_row(const int32_t* __restrict__ cu_q,
   return r;
 }
 
+// locate_row with the whole CTA at once (every thread of the block must call
+// it: it synchronises the block): b is the number of sequences b' >= 1 with
+// cu_q[b'] <= t (cu_q is non-decreasing, so they form a prefix), counted with
+// one load per thread per blockDim.x sequences instead of a chain of
+// dependent loads.
+__device__ __forceinline__ RowInfo locate_row_block(const int32_t* __restrict__ cu_q,
+                                                    const int32_t* __restrict__ cu_k, int B, int64_t t) {
+  int b = 0;
+  for (int base = 1; base < B; base += static_cast<int>(blockDim.x)) {
+    const int i = base + static_cast<int>(threadIdx.x);
+    b += __syncthreads_count(i < B && cu_q[i] <= t);
+  }
+  RowInfo r;
+  r.b = b;
+  const int q0 = cu_q[b], q1 = cu_q[b + 1];
+  r.k_base = cu_k[b];
+  r.kv_len = cu_k[b + 1] - r.k_base;
+  r.pos = r.kv_len - (q1 - q0) + static_cast<int>(t - q0);
+  return r;
+}
+
 // Order-preserving map of a non-NaN float to uint32 (larger float -> larger
 // key); -0.0 is first folded onto +0.0 so that the two tie.
 __device__ __forceinline__ uint32_t order_key(float x) {

@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(C::NT, 1)
   const uint32_t peer = rank ^ 1u;
   const int64_t r_local = blockIdx.x / C::SPLIT;          // chunk-relative query row
   const int64_t t = p.q_begin + r_local;
-  const RowInfo ri = locate_row(p.cu_q, p.cu_k, p.B, t);
+  const RowInfo ri = locate_row_block(p.cu_q, p.cu_k, p.B, t);
   const int32_t* __restrict__ idx_row = p.idx + r_local * p.topk;
   const int a0 = rank == 0 ? 0 : C::A0_R1;                // first atom of this CTA's columns (global)
   const int na = rank == 0 ? C::NA0 : C::NA1;             // atoms of this CTA's columns

@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
   using C = TopkCfg;
   const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t r = blockIdx.x;
-  const RowInfo ri = locate_row(cu_q, cu_k, B, q_begin + r);
+  const RowInfo ri = locate_row_block(cu_q, cu_k, B, q_begin + r);
   const int n = ri.pos + 1;
   const float* __restrict__ row = scores + r * ld;
   int32_t* __restrict__ out = idx + r * topk;
