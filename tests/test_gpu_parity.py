@@ -348,6 +348,24 @@ def test_forward_chunking_does_not_change_results(dsa):
         assert torch.equal(x, y)
 
 
+def test_forward_many_sequences(dsa, oracle_lib):
+    """700 decode sequences: more than the threads of a top-k (512) or an
+    attention CTA (576), so the kernels' parallel count over cu_q that finds a
+    row's sequence takes several rounds; rows sampled around those counts.
+    Most caches are shorter than k (every key selected); three are longer."""
+    g = np.random.default_rng(21)
+    kv = [int(x) for x in g.integers(1, 401, size=700)]
+    for b in (300, 520, 600):
+        kv[b] = 5000
+    spec = released("many", (1,) * 700, tuple(kv), seed=21, kfp8=True)
+    d = di.make_inputs(spec)
+    dd = P.to_device(d)
+    v = dsa.Varlen(d["cu_q"], d["cu_k"], "cuda")
+    out, lse, idx = _forward(dsa, dd, spec, v)
+    rows = [0, 1, 255, 256, 300, 511, 512, 513, 520, 575, 576, 577, 600, 698, 699]
+    _check_sampled(dsa, oracle_lib, spec, dd, d["cu_q"], d["cu_k"], out, lse, idx, rows)
+
+
 def _check_sampled(dsa, oracle_lib, spec, dd, cu_q, cu_k, out, lse, idx, rows):
     """Oracle on sampled rows of a (possibly huge) GPU-resident workload."""
     cu_q_l, cu_k_l = list(map(int, cu_q)), list(map(int, cu_k))
