@@ -240,19 +240,66 @@ __global__ void __launch_bounds__(C::NT, 1)
   }
   if (warp >= C::PROD_WARP0 && lane == 0) tma_prefetch_desc(&tm_lat);
   DSA_PROF_BEGIN();
-  __syncthreads();
-  // Tiles up to the last one holding a valid entry (trailing -1 padding is skipped).
-  {
+  tc_fence_before();
+  __syncthreads();   // barriers initialised, tensor memory allocated
+  if (warp < C::NSM) {
+    // The softmax warps load the query slice (the A operand of every QK MMA)
+    // into tensor memory while the other warps scan the selection and start
+    // gathering: it is on every cluster's critical path.  This CTA's barriers
+    // are initialised, so its arrival at the cluster barrier goes first; the
+    // wait (for the peer's) comes before any access to the peer.
+    if (C::SPLIT == 2) cluster_arrive();
+    tc_fence_after();
+    const uint32_t tmem_q = *tmem_holder;
+    const int c = warp >> 2;
+    const int h = (warp & 3) * 32 + lane;                // head row = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    // Query elements [qk_lo, qk_lo + QKH) of head row h into TMEM lane h; rows
+    // h >= H hold zeros.  (Loaded whatever the selection holds.)
+    {
+      const bool row_ok = h < C::H;
+      const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * C::H + (row_ok ? h : 0)) * C::DQK +
+                                                         qk_lo);
+#pragma unroll 1
+      for (int c0 = 8 * c; c0 < C::QCOLS; c0 += 16) {   // 8 columns = 16 bf16 = two 16-byte loads
+        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+        if (row_ok) {
+          v0 = __ldg(qrow + c0 / 4);
+          v1 = __ldg(qrow + c0 / 4 + 1);
+        }
+        uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const int g0 = qk_lo + 2 * c0;   // first query element of this chunk
+        if (p.rope != nullptr && g0 >= C::DV) {
+          // RoPE of the rope columns at this row's position: element pair
+          // (2i, 2i + 1) of the rope part times (cos, sin) of pair i.
+          const float2* cs = p.rope + static_cast<int64_t>(ri.pos) * ((C::DQK - C::DV) / 2) + (g0 - C::DV) / 2;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float re = __uint_as_float(w8[j] << 16), im = __uint_as_float(w8[j] & 0xFFFF0000u);
+            const float2 r = __ldg(cs + j);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(re, r.x, -im * r.y), fmaf(re, r.y, im * r.x));
+            w8[j] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+        }
+        tmem_st8(tmem_q + lane_base + C::TMEM_Q + c0, w8);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_warp(bar_q_ready);
+    }
+    if (C::SPLIT == 2) cluster_wait(); else __syncthreads();
+  } else {
+    // Tiles up to the last one holding a valid entry (trailing -1 padding is skipped).
     int last = -1;
-    for (int e = threadIdx.x; e < p.topk; e += C::NT) {
+    for (int e = static_cast<int>(threadIdx.x) - C::NSM * 32; e < p.topk; e += C::NT - C::NSM * 32) {
       const int s = idx_row[e];
       if (s >= 0 && s <= ri.pos) last = e;
     }
     for (int off = 16; off > 0; off >>= 1) last = max(last, __shfl_xor_sync(0xFFFFFFFFu, last, off));
     if (lane == 0 && last >= 0) atomicMax(ntiles_s, last / C::BN + 1);
+    tc_fence_before();
+    if (C::SPLIT == 2) cluster_sync(); else __syncthreads();   // peer barriers initialised
   }
-  tc_fence_before();
-  if (C::SPLIT == 2) cluster_sync(); else __syncthreads();   // peer barriers initialised
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   // Both CTAs of a cluster take the same skip decision (own flag OR the peer's),
@@ -413,39 +460,6 @@ __global__ void __launch_bounds__(C::NT, 1)
     float m_used = -INFINITY;    // reference max (log2 units) of this team's latest tile
     float l_run = 0.f;           // this team's tiles, against m_used; the teams add at the end
     bool ok = true;
-    // Query elements [qk_lo, qk_lo + QKH) of head row h into TMEM lane h: the A
-    // operand of every QK MMA.  Rows h >= H hold zeros.
-    if (n_tiles > 0) {
-      const bool row_ok = h < C::H;
-      const uint4* qrow = reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * C::H + (row_ok ? h : 0)) * C::DQK +
-                                                         qk_lo);
-#pragma unroll 1
-      for (int c0 = 8 * c; c0 < C::QCOLS; c0 += 16) {   // 8 columns = 16 bf16 = two 16-byte loads
-        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
-        if (row_ok) {
-          v0 = __ldg(qrow + c0 / 4);
-          v1 = __ldg(qrow + c0 / 4 + 1);
-        }
-        uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        const int g0 = qk_lo + 2 * c0;   // first query element of this chunk
-        if (p.rope != nullptr && g0 >= C::DV) {
-          // RoPE of the rope columns at this row's position: element pair
-          // (2i, 2i + 1) of the rope part times (cos, sin) of pair i.
-          const float2* cs = p.rope + static_cast<int64_t>(ri.pos) * ((C::DQK - C::DV) / 2) + (g0 - C::DV) / 2;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float re = __uint_as_float(w8[j] << 16), im = __uint_as_float(w8[j] & 0xFFFF0000u);
-            const float2 r = __ldg(cs + j);
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(re, r.x, -im * r.y), fmaf(re, r.y, im * r.x));
-            w8[j] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-        }
-        tmem_st8(tmem + lane_base + C::TMEM_Q + c0, w8);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive_warp(bar_q_ready);
-    }
     // Team c takes tiles j = c, c + 2, ...; a thread owns head row h of its
     // team's tiles, all BN columns, so a tile's row maximum needs no partner.
     // The reference max the exponentials are taken against is one sequence
