@@ -334,13 +334,18 @@ dsa_status launch_mla(const void* q, const void* latent, const int32_t* idx, con
   cfg.blockDim = dim3(C::NT, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C::SPLIT;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // a dependent of the previous kernel in the stream: it may start while that
+  // kernel finishes (the top-k frees most SMs early) and waits for it before
+  // it reads the selection
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, dsa::sparse_mla_kernel<C>, tm_lat, p);
   return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
@@ -470,9 +475,21 @@ dsa_status run_topk(const float* scores, int64_t ld, const float* part_max, int6
   NvtxRange range("dsa.topk");
   if (topk_limits(L, rows) != DSA_OK) return DSA_ERR_UNSUPPORTED;
   if (ensure_smem<dsa::topk_kernel>(dsa::TopkCfg::SMEM_BYTES) != cudaSuccess) return DSA_ERR_CUDA;
-  dsa::topk_kernel<<<static_cast<unsigned>(rows), dsa::TopkCfg::NT, dsa::TopkCfg::SMEM_BYTES, stream>>>(
-      scores, ld, part_max, ld_pm, v.cu_q, v.cu_k, v.batch, q_begin, topk, idx);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  // a dependent of the previous kernel in the stream (see run_mla): its
+  // launch overlaps that kernel's end; it waits for it before reading scores
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows), 1, 1);
+  cfg.blockDim = dim3(dsa::TopkCfg::NT, 1, 1);
+  cfg.dynamicSmemBytes = dsa::TopkCfg::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, dsa::topk_kernel, scores, ld, part_max, ld_pm, v.cu_q, v.cu_k,
+                                           v.batch, q_begin, topk, idx);
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status run_mla(const void* q, const void* latent, const int32_t* idx, const dsa_varlen& v,

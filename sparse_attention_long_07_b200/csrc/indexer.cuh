@@ -254,6 +254,7 @@ __global__ void __launch_bounds__(C::NT, 1)
   const int ntiles = (pos0 + nq - 1) / C::BK + 1;
   const int t_begin = blockIdx.x * p.chunk_tiles;
   const int t_end = min(ntiles, t_begin + p.chunk_tiles);
+  grid_launch_dependents();   // the top-k may be scheduled as SMs free up (it waits for this grid)
   if (t_begin >= t_end || device_error_pending()) return;
   const int n_iter = t_end - t_begin;
 
@@ -511,6 +512,7 @@ __global__ void __launch_bounds__(C::NT, 1)
   int* upre = reinterpret_cast<int*>(smem + C::OFF_UPRE);      // upre[b] = first unit of sequence b
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  grid_launch_dependents();   // the top-k may be scheduled as SMs free up (it waits for this grid)
   if (device_error_pending()) return;
 
   // ---------------------------------------------------------------- unit list

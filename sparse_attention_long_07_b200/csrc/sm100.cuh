@@ -540,6 +540,18 @@ __device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
   return v;
 }
 
+// Programmatic dependent launch.  grid_launch_dependents: this CTA no longer
+// holds back the launch of the next kernel in the stream (launched with
+// programmatic stream serialisation); that kernel may then start on free SMs.
+// grid_dependency_wait: wait until the kernel(s) this one depends on have
+// completed and their memory is visible (a no-op when launched normally).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // The two halves of cluster_sync, for threads that have work to do between
 // announcing their CTA ready and needing the other CTAs to be.
 __device__ __forceinline__ void cluster_arrive() {

@@ -289,6 +289,10 @@ __global__ void __launch_bounds__(C::NT, 1)
     }
     if (C::SPLIT == 2) cluster_wait(); else __syncthreads();
   } else {
+    // The selection comes from the previous kernel (the top-k): when this
+    // kernel is launched as its dependent it may start early, so wait for it
+    // here (the query slice above is an input of the call, not its output).
+    grid_dependency_wait();
     // Tiles up to the last one holding a valid entry (trailing -1 padding is skipped).
     int last = -1;
     for (int e = static_cast<int>(threadIdx.x) - C::NSM * 32; e < p.topk; e += C::NT - C::NSM * 32) {

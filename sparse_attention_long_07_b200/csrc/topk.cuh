@@ -77,6 +77,11 @@ __global__ void __launch_bounds__(TopkCfg::NT, 1)
   using C = TopkCfg;
   const uint32_t tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t r = blockIdx.x;
+  // every CTA of this grid is resident once it gets here: the next kernel (the
+  // attention, when launched as a dependent) may start on the free SMs; the
+  // scores come from the previous kernel (the indexer), so wait for it
+  grid_launch_dependents();
+  grid_dependency_wait();
   const RowInfo ri = locate_row_block(cu_q, cu_k, B, q_begin + r);
   const int n = ri.pos + 1;
   const float* __restrict__ row = scores + r * ld;
