@@ -69,6 +69,7 @@ def test_bench_line_carries_every_contract_key(monkeypatch, capsys):
 
     def fake_gpu_arm(args, rank, world):
         return {"value": 1.0e5, "ms_per_step": 0.64, "stage_ms": {"indexer": 0.2, "topk": 0.1, "attention": 0.3},
+                "stage_ms_steps": 5,
                 "roofline": fake_roof, "step_roofline_frac": 0.3,
                 "e2e": {"value": 5.0e4, "unit": "query tokens/s", "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 2},
                 "gpu_launches": 3 * args.steps, "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
