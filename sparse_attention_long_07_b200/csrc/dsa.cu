@@ -297,7 +297,18 @@ dsa_status launch_indexer_persistent(const void* q_idx, const float* q_scale, co
   p.ld_pm = ld_pm;
   p.chunk_tiles = 0;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(units, sms));
-  dsa::indexer_persistent_kernel<C><<<grid, C::NT, C::SMEM_BYTES, stream>>>(tm_q, tm_k, p);
+  // a dependent of the previous kernel in the stream (see run_mla)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(C::NT, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dsa::indexer_persistent_kernel<C>, tm_q, tm_k, p) != cudaSuccess) return DSA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

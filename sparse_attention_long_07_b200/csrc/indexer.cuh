@@ -642,6 +642,11 @@ __global__ void __launch_bounds__(C::NT, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // Launched as a dependent of the previous kernel in the stream (the previous
+  // step's attention): the set-up above overlaps its end; the scores and part
+  // maxima this kernel writes may still be read by that step's kernels until
+  // it completes, so wait for it here.
+  grid_dependency_wait();
   const long long t_role = clock64();
 
   if (warp == C::PRODUCER_WARP) {

@@ -166,6 +166,7 @@ __device__ __forceinline__ int gather_row(const PageMap& pages, const RowInfo& r
 template <class C>
 __global__ void __launch_bounds__(C::NT, 1)
     sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_lat, const MlaParams p) {
+  grid_launch_dependents();   // the next step's indexer may be scheduled as SMs free up (it waits for this grid)
   const uint32_t rank = C::SPLIT == 2 ? cluster_ctarank() : 0u;
   const uint32_t peer = rank ^ 1u;
   const int64_t r_local = blockIdx.x / C::SPLIT;          // chunk-relative query row
