@@ -13,6 +13,13 @@
  *    never allocates, frees or keeps a pointer after the call returns.
  *  - Calls are asynchronous on `stream`.  Argument errors are detected on the
  *    host and returned before anything is launched; nothing is written then.
+ *  - The decode indexer (at most one query row per sequence), the top-k and
+ *    the sparse attention are launched with programmatic stream serialisation:
+ *    they may start while the kernel before them on `stream` finishes, and
+ *    wait for it to complete before they read or write any memory it may use,
+ *    so the results are those of plain stream order.  (Only this library's
+ *    kernels release their successor early; after any other kernel the
+ *    launch waits for it as usual.)
  *  - Sequences are packed ("varlen"): sequence b owns query rows
  *    [cu_q[b], cu_q[b+1]) and key/cache rows [cu_k[b], cu_k[b+1]).  The new
  *    queries are the last q_len_b tokens of the sequence, so local query i sits
