@@ -142,44 +142,6 @@ struct IndexerCfg {
   static_assert(OFF_BAR % 8 == 0 && OFF_UPRE % 4 == 0, "barrier / prefix alignment");
 };
 
-// One key row of a raw e4m3 tile (128 bytes, 128-byte TMA swizzle) -> the
-// same row of the bf16 UMMA tile (two 128-byte swizzle atoms).  Exact: every
-// e4m3 value is a bf16 value (e4m3 -> f16x2 -> f32 -> bf16x2, all exact).
-template <int BK>
-__device__ __forceinline__ void e4m3_row_to_bf16(const uint8_t* raw_row, uint8_t* dst_tile, int row) {
-  uint4 chunk[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j)  // 128-byte swizzle: logical chunk j sits at j ^ (row & 7)
-    chunk[j] = *reinterpret_cast<const uint4*>(raw_row + ((j ^ (row & 7)) << 4));
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t src[4] = {chunk[j].x, chunk[j].y, chunk[j].z, chunk[j].w};
-    uint32_t outw[8];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      uint32_t h01, h23;
-      asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-          "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
-          : "=r"(h01), "=r"(h23)
-          : "r"(src[e]));
-      const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
-      const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
-      uint32_t b01, b23;
-      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b01) : "f"(f01.y), "f"(f01.x));
-      asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b23) : "f"(f23.y), "f"(f23.x));
-      outw[2 * e] = b01;
-      outw[2 * e + 1] = b23;
-    }
-    // 16 bf16 = logical chunks 2j, 2j+1 of the row; 64 elements per atom
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int lc = 2 * j + h;
-      uint8_t* dst = dst_tile + (lc >> 3) * (BK * 128) + row * 128 + (((lc & 7) ^ (row & 7)) << 4);
-      *reinterpret_cast<uint4*>(dst) = make_uint4(outw[4 * h], outw[4 * h + 1], outw[4 * h + 2], outw[4 * h + 3]);
-    }
-  }
-}
-
 // Four e4m3 bytes -> four bf16 values (two bf16x2 words, lower element in the
 // low half), with integer and bf16 arithmetic only.  PRMT puts each byte in
 // the low byte of a 16-bit half and fills the high byte with copies of its
@@ -198,6 +160,31 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t src, uint32_t& lo, uin
   b = (b << 4) & 0x87F087F0u;
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0x7B807B80u));   // 0x7B80 = bf16 2^120
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0x7B807B80u));
+}
+
+// One key row of a raw e4m3 tile (128 bytes, 128-byte TMA swizzle) -> the
+// same row of the bf16 UMMA tile (two 128-byte swizzle atoms).  Exact: every
+// e4m3 value is a bf16 value (e4m3x4_to_bf16x4).
+template <int BK>
+__device__ __forceinline__ void e4m3_row_to_bf16(const uint8_t* raw_row, uint8_t* dst_tile, int row) {
+  uint4 chunk[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)  // 128-byte swizzle: logical chunk j sits at j ^ (row & 7)
+    chunk[j] = *reinterpret_cast<const uint4*>(raw_row + ((j ^ (row & 7)) << 4));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t src[4] = {chunk[j].x, chunk[j].y, chunk[j].z, chunk[j].w};
+    uint32_t outw[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) e4m3x4_to_bf16x4(src[e], outw[2 * e], outw[2 * e + 1]);
+    // 16 bf16 = logical chunks 2j, 2j+1 of the row; 64 elements per atom
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int lc = 2 * j + h;
+      uint8_t* dst = dst_tile + (lc >> 3) * (BK * 128) + row * 128 + (((lc & 7) ^ (row & 7)) << 4);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(outw[4 * h], outw[4 * h + 1], outw[4 * h + 2], outw[4 * h + 3]);
+    }
+  }
 }
 
 // Four e4m3 bytes -> four f16 values (two f16x2 words, lower element in the
