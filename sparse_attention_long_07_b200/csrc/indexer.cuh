@@ -15,12 +15,14 @@
 //
 // Roles (query-block grid): one TMA warp streams key tiles through a
 // shared-memory ring; one thread issues the MMAs into two TMEM accumulators;
-// one or two epilogue warpgroups drain them.  For an e4m3 index-key cache, four
-// more warps widen each raw tile to bf16 in the shared-memory UMMA layout
-// (exact: every e4m3 value is a bf16 value), and the per-key fp32 scale
-// multiplies the head-reduced score (a positive scale commutes with ReLU).
-// The persistent decode schedule (below) widens keys into tensor memory
-// instead, and issues MMAs from two threads.
+// one epilogue warpgroup (four, one per query, for four-query blocks) drains
+// them.  For an e4m3 index-key cache, four more warps widen each raw tile to
+// bf16 in the shared-memory UMMA layout (exact: every e4m3 value is a bf16
+// value), and the per-key fp32 scale multiplies the head-reduced score (a
+// positive scale commutes with ReLU).  The persistent decode schedule (below)
+// widens keys to f16 into tensor memory instead, multiplies f16 operands,
+// issues MMAs from two threads and drains four accumulators with four
+// epilogue warpgroups.
 #pragma once
 
 #include "common.cuh"
