@@ -348,6 +348,44 @@ def test_forward_chunking_does_not_change_results(dsa):
         assert torch.equal(x, y)
 
 
+def test_back_to_back_forwards_match_separate_calls(dsa):
+    """The decode indexer, the top-k and the attention start while the kernel
+    before them finishes (programmatic dependent launch) and wait for it
+    before touching its data.  Forwards of two batches issued back to back
+    through one workspace, with nothing between them, must give exactly what
+    the same calls give with the device synchronised after each."""
+    specs = [released("b2b", (1,) * 12, tuple(3000 + 700 * b for b in range(12)), seed=s, kfp8=True)
+             for s in (31, 32)]
+    ds = [P.to_device(di.make_inputs(sp)) for sp in specs]
+    vs = [dsa.Varlen(sp_d["cu_q"], sp_d["cu_k"], "cuda") for sp_d in ds]
+    sp = specs[0]
+    ws = torch.empty(dsa.dsa_forward_workspace_size(vs[0], sp.topk), dtype=torch.uint8, device="cuda")
+
+    def fwd(i, out, lse, idx):
+        dsa.dsa_forward(ds[i]["q_idx"], ds[i]["w"], ds[i]["k_idx"], ds[i]["k_scale"], ds[i]["q"], ds[i]["latent"],
+                        vs[i], sp.topk, sp.softmax_scale, out, lse, ws, idx_out=idx)
+
+    def bufs():
+        return (torch.empty((sp.T, sp.H, sp.d_v), dtype=torch.bfloat16, device="cuda"),
+                torch.empty((sp.T, sp.H), dtype=torch.float32, device="cuda"),
+                torch.empty((sp.T, sp.topk), dtype=torch.int32, device="cuda"))
+
+    ref = [bufs(), bufs()]
+    for i in (0, 1):
+        fwd(i, *ref[i])
+        torch.cuda.synchronize()
+    got = [[bufs(), bufs()] for _ in range(3)]
+    for r in range(3):
+        for i in (0, 1):
+            fwd(i, *got[r][i])
+    torch.cuda.synchronize()
+    assert dsa.dsa_device_error() == 0
+    for r in range(3):
+        for i in (0, 1):
+            for a, b in zip(got[r][i], ref[i]):
+                assert torch.equal(a, b), f"round {r}, batch {i}"
+
+
 def test_forward_many_sequences(dsa, oracle_lib):
     """700 decode sequences: more than the threads of a top-k (512) or an
     attention CTA (576), so the kernels' parallel count over cu_q that finds a
