@@ -602,34 +602,54 @@ def indexer_prefill_measure(dsa, args, peaks):
 
 
 class _E2ELane:
-    """One batch in flight for the end-to-end measurement: its device inputs,
-    pinned host copies of the step's inputs, outputs and workspace."""
+    """One batch in flight for the end-to-end measurement.  Everything a step
+    copies in sits in one device buffer with a pinned host twin (one copy per
+    step), and so do its outputs (one copy back): decode steps bring the query
+    tensors and the new token of every sequence (its index key and latent
+    row, bf16), which dsa_cache_append writes into the resident caches;
+    prefill steps bring every input tensor."""
+
+    @staticmethod
+    def _packed(tensors, dev):
+        """One device buffer and one pinned host buffer holding the tensors at
+        256-byte boundaries; returns (device views, host views, both buffers)."""
+        offs, total = [], 0
+        for _, t in tensors:
+            offs.append(total)
+            total += (t.numel() * t.element_size() + 255) // 256 * 256
+        dbuf = torch.empty(max(total, 256), dtype=torch.uint8, device=dev)
+        hbuf = torch.empty(max(total, 256), dtype=torch.uint8).pin_memory()
+        dv, hv = {}, {}
+        for (n, t), o in zip(tensors, offs):
+            nb = t.numel() * t.element_size()
+            dv[n] = dbuf[o:o + nb].view(t.dtype).view(t.shape)
+            hv[n] = hbuf[o:o + nb].view(t.dtype).view(t.shape)
+            dv[n].copy_(t)
+            hv[n].copy_(t.cpu())
+        return dv, hv, dbuf, hbuf
 
     def __init__(self, dsa, spec, d, v, q_chunk, decode):
         dev = d["q"].device
         self.spec, self.d, self.v, self.q_chunk, self.decode = spec, d, v, q_chunk, decode
-        cu_k = [int(x) for x in d["cu_k"]]
-        # decode: the step's new inputs are the query tensors and the new
-        # token's cache rows (the caches are resident device state); prefill:
-        # every input tensor is the step's input
-        self.names = ["q_idx", "w", "q"] + ([] if decode else ["k_idx", "latent"] + (["k_scale"] if spec.kfp8 else []))
-        self.host = {n: d[n].cpu().pin_memory() for n in self.names}
-        self.k_bytes = d["k_idx"].view(torch.uint8) if spec.kfp8 else d["k_idx"]
+        names = ["q_idx", "w", "q"] + ([] if decode else ["k_idx", "latent"] + (["k_scale"] if spec.kfp8 else []))
+        staged = [(n, d[n]) for n in names]
         if decode:
-            self.new_rows = torch.tensor([c - 1 for c in cu_k[1:]], dtype=torch.long, device=dev)
-            self.host["k_rows"] = self.k_bytes[self.new_rows].cpu().pin_memory()
-            self.host["lat_rows"] = d["latent"][self.new_rows].cpu().pin_memory()
-            if spec.kfp8:
-                self.host["ks_rows"] = d["k_scale"][self.new_rows].cpu().pin_memory()
-            self.rows_dev = {n: torch.empty(self.host[n].shape, dtype=self.host[n].dtype, device=dev)
-                             for n in ("k_rows", "lat_rows", "ks_rows") if n in self.host}
-        self.out = torch.empty((spec.T, spec.H, spec.d_v), dtype=torch.bfloat16, device=dev)
-        self.lse = torch.empty((spec.T, spec.H), dtype=torch.float32, device=dev)
-        self.out_h = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
-        self.lse_h = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
+            new_rows = torch.tensor([int(c) - 1 for c in d["cu_k"][1:]], dtype=torch.long, device=dev)
+            k_new = d["k_idx"][new_rows]
+            if spec.kfp8:   # the new tokens' index keys in bf16 (dsa_cache_append quantizes them)
+                k_new = (k_new.float() * d["k_scale"][new_rows][:, None]).to(torch.bfloat16)
+            staged += [("k_new", k_new.contiguous()), ("lat_new", d["latent"][new_rows].contiguous())]
+        self.din, _, self.din_buf, self.hin_buf = self._packed(staged, dev)
+        for n in names:
+            d[n] = self.din[n]   # the forward reads the copied-in tensors
+        outs = [("out", torch.empty((spec.T, spec.H, spec.d_v), dtype=torch.bfloat16, device=dev)),
+                ("lse", torch.empty((spec.T, spec.H), dtype=torch.float32, device=dev))]
+        dout, _, self.dout_buf, self.hout_buf = self._packed(outs, dev)
+        self.out, self.lse = dout["out"], dout["lse"]
         self.ws = torch.empty(dsa.dsa_forward_workspace_size(v, spec.topk, q_chunk), dtype=torch.uint8, device=dev)
-        self.h2d = sum(t.numel() * t.element_size() for t in self.host.values())
-        self.d2h = self.out_h.numel() * self.out_h.element_size() + self.lse_h.numel() * self.lse_h.element_size()
+        self.h2d = self.hin_buf.numel()
+        self.d2h = self.hout_buf.numel()
+        self.k_quant = dsa.DSA_KQ_E4M3_AMAX if spec.kfp8 else dsa.DSA_KQ_BF16
         self.ev_in = torch.cuda.Event()        # inputs on the device
         self.ev_used = torch.cuda.Event()      # the forward that read them (and wrote out / lse) is done
         self.ev_out = torch.cuda.Event()       # out / lse copied back
@@ -637,33 +657,27 @@ class _E2ELane:
         self.ev_out.record(torch.cuda.current_stream(dev))
 
     def step(self, dsa, s_in, s_comp, s_out):
-        """One step: inputs in on s_in, the forward on s_comp (every lane's
-        forward on the same stream, so the kernels run one after another as in
-        the device-timed step), outputs back on s_out."""
+        """One step: inputs in on s_in, the append and the forward on s_comp
+        (every lane's on the same stream, so the kernels run one after another
+        as in the device-timed step), outputs back on s_out."""
         d, spec = self.d, self.spec
         with torch.cuda.stream(s_in):
             s_in.wait_event(self.ev_used)     # the previous forward of this lane has read its inputs
-            for n in self.names:
-                d[n].copy_(self.host[n], non_blocking=True)
-            if self.decode:
-                for n, rd in self.rows_dev.items():
-                    rd.copy_(self.host[n], non_blocking=True)
+            self.din_buf.copy_(self.hin_buf, non_blocking=True)
             self.ev_in.record(s_in)
         with torch.cuda.stream(s_comp):
             s_comp.wait_event(self.ev_in)
             s_comp.wait_event(self.ev_out)    # out / lse of this lane's previous step are back on the host
             if self.decode:
-                self.k_bytes.index_copy_(0, self.new_rows, self.rows_dev["k_rows"])
-                d["latent"].index_copy_(0, self.new_rows, self.rows_dev["lat_rows"])
-                if spec.kfp8:
-                    d["k_scale"].index_copy_(0, self.new_rows, self.rows_dev["ks_rows"])
+                dsa.dsa_cache_append(self.v, latent_new=self.din["lat_new"], latent_cache=d["latent"],
+                                     kidx_new=self.din["k_new"], k_cache=d["k_idx"], k_scale=d["k_scale"],
+                                     k_quant=self.k_quant, d_v=spec.d_v, stream=s_comp)
             dsa.dsa_forward(d["q_idx"], d["w"], d["k_idx"], d["k_scale"], d["q"], d["latent"], self.v, spec.topk,
                             spec.softmax_scale, self.out, self.lse, self.ws, q_chunk=self.q_chunk, stream=s_comp)
             self.ev_used.record(s_comp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(self.ev_used)
-            self.out_h.copy_(self.out, non_blocking=True)
-            self.lse_h.copy_(self.lse, non_blocking=True)
+            self.hout_buf.copy_(self.dout_buf, non_blocking=True)
             self.ev_out.record(s_out)
 
 
@@ -672,8 +686,8 @@ STAGE_STEPS = 500   # steps of the stage-breakdown region (events between the st
 
 
 def e2e_measure(dsa, spec, d, v, q_chunk, args, world):
-    """dsa_forward through the public API, each step's inputs copied from
-    pinned host memory and its outputs copied back.  Several batches are kept
+    """dsa_cache_append + dsa_forward through the public API, each step's
+    inputs copied from pinned host memory and its outputs copied back.  Several batches are kept
     in flight, as a server would: lane 0 serves the benchmark's batch and the
     other lanes other batches of the same shape (other seeds), each with its
     own buffers, and the steps go round the lanes.  Host-to-device copies run
@@ -711,7 +725,8 @@ def e2e_measure(dsa, spec, d, v, q_chunk, args, world):
     del lanes
     torch.cuda.empty_cache()
     return {"value": world * spec.T / (ms / 1e3), "unit": "query tokens/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4), "steps": n, "api": "dsa_forward",
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4), "steps": n,
+            "api": "dsa_cache_append + dsa_forward" if decode else "dsa_forward",
             "batches_in_flight": n_lanes, "streams": "host-to-device, forward, device-to-host"}
 
 
