@@ -41,7 +41,10 @@
 // Roles per CTA: warps 0-7 query load, softmax and epilogue (two teams of
 // four warps taking alternate tiles, a head row and all of a tile's columns
 // per thread), warps 8 and 9 MMA issuers (QK and PV; warp 8 owns the TMEM),
-// warps 10.. gather (eight with two CTAs, one with one CTA).
+// warps 10.. gather (eight with two CTAs, one with one CTA).  The query slice
+// is loaded while the other warps scan the selection; the kernel may start
+// while the top-k before it finishes (a programmatic dependent launch), and
+// only the warps that read the selection wait for it.
 #pragma once
 
 #include "common.cuh"

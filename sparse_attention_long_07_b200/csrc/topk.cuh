@@ -4,10 +4,19 @@
 // item 2: every query keeps the index_topk highest-scoring earlier tokens.
 // Order: higher score first, ties to the lower index; -0.0 ties +0.0.
 //
-// One CTA per query row.  The row (fp32 scores, usually still in L2 after the
-// indexer wrote it) streams through a 3-stage shared-memory ring of 32 KB bulk
-// async copies issued by one thread, so each SM keeps ~96 KB in flight.
-// Scores become order-preserving 32-bit keys.
+// One CTA per query row (launched as a programmatic dependent of the indexer:
+// it waits for it before reading anything).  Three paths, the first that
+// applies:
+//   part maxima  (the indexer wrote the maximum of every 8 scores; rows of at
+//                least 1.25 k parts) -- a lower bound of the k-th score from
+//                the group maxima, one pass over the groups that can hold a
+//                selection, the exact selection among those candidates;
+//   fast         the same with part maxima taken from the streamed row;
+//   exact        the passes below over the whole row.
+// The row (fp32 scores, usually still in L2 after the indexer wrote it)
+// streams through a 3-stage shared-memory ring of 32 KB bulk async copies
+// issued by one thread, so each SM keeps ~96 KB in flight.  Scores become
+// order-preserving 32-bit keys.
 //   pass 1  histogram of the top 11 key bits (2048 bins; every warp counts into
 //           its own copy, so the hot bins of a score distribution never see
 //           atomics from two warps)  ->  the bin B that holds the k-th largest
