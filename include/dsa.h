@@ -134,6 +134,12 @@ typedef struct {
  *           parts of the row that can hold a selected key.
  * Accumulation is fp32 (bf16 x bf16 products are exact); for e4m3 keys the
  * per-key scale multiplies the head-reduced score (scale > 0 commutes with ReLU).
+ * With e4m3 keys and at most one query row per sequence (the decode kernel),
+ * the tensor cores multiply f16 operands: the keys widen exactly, and each
+ * query tile (all heads of the row) is multiplied by the power of two 2^sq
+ * that puts its largest magnitude 2^E(1+f) below 2^15 and rounded to f16 --
+ * exact for every element of magnitude >= 2^(E-31), smaller ones move by at
+ * most 2^(E-39) -- and the score by 2^-sq.
  * Alignment: all tensors 16-byte aligned; ld_scores a multiple of 4.
  */
 dsa_status dsa_indexer_scores(const void* q_idx, const float* q_scale, const float* w, const void* k_idx,
