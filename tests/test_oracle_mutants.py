@@ -49,15 +49,48 @@ MUTANTS = [
     ("rotation sign", "y[v * d + 2 * i] = re * c - im * s;", "y[v * d + 2 * i] = re * c + im * s;"),
     ("pair halves swapped", "const double re = x[v * d + 2 * i], im = x[v * d + 2 * i + 1];",
      "const double re = x[v * d + 2 * i + 1], im = x[v * d + 2 * i];"),
-    # up-projection
     # paged layout and append quantization
     ("row inside the page taken from the wrong end", "r = (page >= 0 && page < n_pages) ? page * page_size + s % page_size : -1;",
      "r = (page >= 0 && page < n_pages) ? page * page_size + (page_size - 1 - s % page_size) : -1;"),
     ("page table row stride dropped", "block_table[(int64_t)b * pages_per_seq + j]", "block_table[j]"),
     ("pages beyond the pool accepted", "r = (page >= 0 && page < n_pages) ?", "r = (page >= 0) ?"),
     ("amax scale of the wrong format maximum", "(float)(amax / 448.0)", "(float)(amax / 240.0)"),
+    # up-projection
     ("up-projection matrix transposed", "load_elem(w_kind, w, ((int64_t)h * d_c + c) * d_v + e, NULL, 0);",
      "load_elem(w_kind, w, ((int64_t)h * d_v + e) * d_c + c, NULL, 0);"),
+    ("up-projection reads head 0 of the output", "acc += o[(r * H + h) * (int64_t)d_c + c]",
+     "acc += o[(r * H) * (int64_t)d_c + c]"),
+    # more slips of the three steps (every mutated index stays inside its array)
+    ("query position counted from the start of the cache", "*pos_out = kv_len - q_len + (t - cu_q[b]);",
+     "*pos_out = t - cu_q[b];"),
+    ("key scale taken by the sequence-local index", "load_elem(k_kind, k_idx, key_row * d_I + d, k_scale, key_row);",
+     "load_elem(k_kind, k_idx, key_row * d_I + d, k_scale, s);"),
+    ("top-k padded with index 0", "idx[r * topk + i] = i < keep ? c[i].index : -1;",
+     "idx[r * topk + i] = i < keep ? c[i].index : 0;"),
+    ("QK reduced over the value columns only",
+     "for (int d = 0; d < d_qk; ++d)\n          dot += load_elem(q_kind, q, (t * H + h) * (int64_t)d_qk + d, NULL, 0) *\n"
+     "                 load_elem(c_kind, latent, row * d_qk + d, NULL, 0);\n        z[i]",
+     "for (int d = 0; d < d_v; ++d)\n          dot += load_elem(q_kind, q, (t * H + h) * (int64_t)d_qk + d, NULL, 0) *\n"
+     "                 load_elem(c_kind, latent, row * d_qk + d, NULL, 0);\n        z[i]"),
+    ("softmax numerator without the max", "double p = exp(z[i] - zmax) / denom;", "double p = exp(z[i]) / denom;"),
+    ("e4m3 mantissa read as four bits", "v = ldexp(1.0 + m / 8.0, e - 7);", "v = ldexp(1.0 + m / 16.0, e - 7);"),
+    ("Hadamard normalised by 1/d", "1.0 / sqrt((double)d)", "1.0 / (double)d"),
+    ("RoPE table pairs in reverse order",
+     "const double c = freqs[((int64_t)pos[v] * (d / 2) + i) * 2 + 0];\n"
+     "      const double s = freqs[((int64_t)pos[v] * (d / 2) + i) * 2 + 1];",
+     "const double c = freqs[((int64_t)pos[v] * (d / 2) + (d / 2 - 1 - i)) * 2 + 0];\n"
+     "      const double s = freqs[((int64_t)pos[v] * (d / 2) + (d / 2 - 1 - i)) * 2 + 1];"),
+    ("RoPE cos and sin swapped",
+     "const double c = freqs[((int64_t)pos[v] * (d / 2) + i) * 2 + 0];\n"
+     "      const double s = freqs[((int64_t)pos[v] * (d / 2) + i) * 2 + 1];",
+     "const double c = freqs[((int64_t)pos[v] * (d / 2) + i) * 2 + 1];\n"
+     "      const double s = freqs[((int64_t)pos[v] * (d / 2) + i) * 2 + 0];"),
+    ("power-of-two scale from the signed maximum",
+     "amax = fmax(amax, fabs(x[v * d + i]));\n    const double s",
+     "amax = fmax(amax, x[v * d + i]);\n    const double s"),
+    ("amax scale from the signed maximum",
+     "amax = fmax(amax, fabs(x[v * d + i]));\n    const float s",
+     "amax = fmax(amax, x[v * d + i]);\n    const float s"),
 ]
 
 from tests import test_oracle_pins_cache as pins_cache
