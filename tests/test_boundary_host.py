@@ -243,3 +243,38 @@ def test_up_projection_arguments(dsa):
     assert lib.dsa_mla_up_proj(FAKE, FAKE, 4, 64, 512, 128, FAKE, None) == UNS
     assert lib.dsa_mla_up_proj(FAKE, FAKE, 4, 128, 576, 128, FAKE, None) == UNS
     assert lib.dsa_mla_up_proj(FAKE, FAKE, 128 * 65536, 128, 512, 128, FAKE, None) == UNS
+
+
+@host_only
+def test_cache_append_arguments(dsa):
+    """dsa_cache_append's host checks: paired buffers, alignment, supported
+    shapes, the RoPE table and the index-key forms; a call with nothing to
+    write returns DSA_OK without a launch."""
+    lib = dsa.library()
+    INV, UNS, OK = dsa.DSA_ERR_INVALID_ARG, dsa.DSA_ERR_UNSUPPORTED, dsa.DSA_OK
+    BF16, AMAX, HAD = dsa.DSA_KQ_BF16, dsa.DSA_KQ_E4M3_AMAX, dsa.DSA_KQ_E4M3_HADAMARD
+    v = varlen([0, 1, 2], [0, 300, 370])   # caches of 300 and 70 entries, one new token each
+
+    def call(lat=None, kid=None, d_qk=576, d_v=512, idx_dim=128, rope=None, max_pos=0, kq=BF16,
+             lat_c=None, k_c=None, k_s=None, layout=v):
+        return lib.dsa_cache_append(lat, kid, layout, d_qk, d_v, idx_dim, rope, max_pos, kq, lat_c, k_c, k_s, None)
+
+    assert call() == OK                                                  # nothing to write
+    assert call(lat=FAKE, lat_c=FAKE, layout=varlen([0, 0], [0, 5])) == OK   # no new tokens
+    assert call(lat=FAKE) == INV                                         # new latents without a cache
+    assert call(lat_c=FAKE) == INV
+    assert call(kid=FAKE) == INV                                         # new keys without a cache
+    assert call(lat=FAKE + 8, lat_c=FAKE) == INV                         # misaligned rows
+    assert call(kid=FAKE, k_c=FAKE + 8) == INV
+    assert call(lat=FAKE, lat_c=FAKE, d_qk=512, d_v=512) == UNS          # not a supported MLA shape
+    assert call(lat=FAKE, lat_c=FAKE, rope=FAKE + 4, max_pos=370) == INV  # table not 8-byte aligned
+    assert call(rope=FAKE, max_pos=370) == INV                           # a table with no latents to rotate
+    assert call(lat=FAKE, lat_c=FAKE, rope=FAKE, max_pos=299) == INV     # table shorter than the longest cache (300)
+    assert call(kid=FAKE, k_c=FAKE, kq=7) == INV                         # unknown key form
+    assert call(kid=FAKE, k_c=FAKE, idx_dim=64) == UNS                   # bf16 keys of an unsupported width
+    for kq in (AMAX, HAD):
+        assert call(kid=FAKE, k_c=FAKE, kq=kq) == INV                    # e4m3 keys need their scales
+        assert call(kid=FAKE, k_c=FAKE, k_s=FAKE + 2, kq=kq) == INV      # scales not 4-byte aligned
+        assert call(kid=FAKE, k_c=FAKE, k_s=FAKE, kq=kq, idx_dim=32) == UNS
+    bad = varlen([0, 2], [0, 1])                                          # more new tokens than cache entries
+    assert call(lat=FAKE, lat_c=FAKE, layout=bad) == INV
