@@ -278,3 +278,14 @@ def test_cache_append_arguments(dsa):
         assert call(kid=FAKE, k_c=FAKE, k_s=FAKE, kq=kq, idx_dim=32) == UNS
     bad = varlen([0, 2], [0, 1])                                          # more new tokens than cache entries
     assert call(lat=FAKE, lat_c=FAKE, layout=bad) == INV
+
+
+def test_wait_profile_is_a_profiling_build_feature(dsa):
+    """The regular library has no wait counters: the diagnostic call answers
+    DSA_ERR_UNSUPPORTED and touches neither array (no device access, so this
+    also holds where a GPU is present)."""
+    lib = dsa.library()
+    cyc = (ctypes.c_uint64 * 4)(*([7] * 4))
+    cnt = (ctypes.c_uint64 * 4)(*([9] * 4))
+    assert lib.dsa_debug_wait_profile(cyc, cnt, 4, 1) == dsa.DSA_ERR_UNSUPPORTED
+    assert list(cyc) == [7] * 4 and list(cnt) == [9] * 4
