@@ -10,7 +10,9 @@
  *
  * Conventions shared by every entry point
  *  - Every tensor pointer is DEVICE memory owned by the caller; the library
- *    never allocates, frees or keeps a pointer after the call returns.
+ *    never allocates, frees or keeps a pointer after the call returns (its
+ *    one device array, the scratch of dsa_forward_static_scratch, is static
+ *    and comes with the library's device code).
  *  - Calls are asynchronous on `stream`.  Argument errors are detected on the
  *    host and returned before anything is launched; nothing is written then.
  *  - The decode indexer (at most one query row per sequence), the top-k and
