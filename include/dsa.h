@@ -106,8 +106,8 @@ typedef struct {
 /*
  * Step 1: lightning-indexer scores.
  * Source: "DeepSeek-V3.2" (transformers model doc), section "DeepSeek Sparse
- * Attention (DSA)", item 1 -- a light, low-head-count module scores each query
- * against every preceding key; the released config has index_n_heads 64 and
+ * Attention (DSA)", item 1 -- a cheap module with few heads scores every key
+ * at or before each query's position; the released config has index_n_heads 64 and
  * index_head_dim 128 ("DeepSeek-V3.2-Exp" token-ids page).  Score:
  *     I[t,s] = sum_j w[t,j] * max(0, q_idx[t,j,:] . k[s,:]),   0 <= s <= pos(t)
  * q_idx     bf16 [T, n_idx_heads, idx_dim], row-major, global rows; or, for
@@ -153,8 +153,9 @@ dsa_status dsa_indexer_scores(const void* q_idx, const float* q_scale, const flo
 /*
  * Step 2: fine-grained token selection.
  * Source: "DeepSeek-V3.2" (transformers model doc), section "DeepSeek Sparse
- * Attention (DSA)", item 2 -- each query keeps the top index_topk (2048 by
- * default) tokens.  Ties are broken toward the lower key index; -0.0 ties +0.0.
+ * Attention (DSA)", item 2 -- every query retains the index_topk (default
+ * 2048) keys with the highest scores.  Ties are broken toward the lower key
+ * index; -0.0 ties +0.0.
  * scores    fp32 [q_end - q_begin, ld_scores] chunk-relative, as written by
  *           dsa_indexer_scores (only columns 0..pos(t) are read)
  * part_max  NULL, or the part maxima dsa_indexer_scores wrote beside these
@@ -217,8 +218,8 @@ dsa_status dsa_sparse_mla_attn(const void* q, const void* latent, const int32_t*
 /*
  * Inputs of the FP8 indexer.
  * Source: "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse
- * Attention (DSA)", item 1 -- the reference indexer runs in FP8 with a
- * Hadamard (rotate_activation) transform; "DeepSeek-V3.2-Exp" token-ids page,
+ * Attention (DSA)", item 1 -- DeepSeek's own indexer scores in e4m3 after a
+ * Hadamard rotation of both operands (rotate_activation); "DeepSeek-V3.2-Exp" token-ids page,
  * released config: scale_fmt ue8m0 (power-of-two scales).
  * Each of the n vectors of 128 values is rotated by the Sylvester-Hadamard
  * matrix H (entries +-1, H[i][j] = (-1)^popcount(i & j), not normalised) and

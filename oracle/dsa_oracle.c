@@ -9,14 +9,15 @@
  *
  * Sources (page title, section):
  *  - "DeepSeek-V3.2" (transformers model doc), section "DeepSeek Sparse
- *    Attention (DSA)", item 1 "Lightning indexer": an index score between each
- *    query and every preceding key, computed by a low-head-count module; item
- *    2 "Fine-grained token selection": keep the top-index_topk tokens, main MLA
- *    attention over those tokens only via an additive mask.
+ *    Attention (DSA)", item 1 "Lightning indexer": a module with few heads
+ *    scores every pair of a query and a key at or before its position; item
+ *    2 "Fine-grained token selection": every query retains its index_topk
+ *    highest-scoring tokens and the main MLA attention sees only those (the
+ *    transformers port expresses the restriction as an additive mask).
  *  - "DeepSeek-V3.2 / Exp" (visual-learn explainer), "Different questions
  *    select different tokens": cached entries are MLA's compressed vectors.
  *  - "DeepSeek-V3.2 - Experimental Exp Version" (altools), "Technical
- *    Principles": a small number of index heads; MLA with MQA so that key
+ *    Principles": the indexer has few heads; MLA with MQA so that key
  *    entries are shared by all query heads.
  *  - "DeepSeek-V3.2-Exp" (token-ids page), released config excerpt
  *    (index_n_heads 64, index_head_dim 128, index_topk 2048, kv_lora_rank 512,
@@ -185,7 +186,7 @@ static int candidate_cmp(const void* a, const void* b) {
 }
 
 /*
- * Step 2, fine-grained token selection.  For each requested row: sort the
+ * Step 2, fine-grained token selection.  Every requested row: sort the
  * candidates s = 0..pos(t) by (score desc, index asc) and keep the first
  * min(topk, pos(t)+1); idx[r, :] holds them in that order, then -1 padding.
  * scores rows follow the layout written by oracle_indexer_scores.
@@ -364,9 +365,9 @@ int oracle_dense_mla_masked(int B, const int32_t* cu_q, const int32_t* cu_k, int
 
 /* ===========================================================================
  * The FP8 indexer ("DeepSeek-V3.2", transformers model doc, section "DeepSeek
- * Sparse Attention (DSA)", item 1: the reference indexer runs in FP8 with a
- * Hadamard (rotate_activation) transform; "DeepSeek-V3.2-Exp" token-ids page,
- * released config: scale_fmt "ue8m0").  Readings where the pages are silent:
+ * Sparse Attention (DSA)", item 1: DeepSeek's own indexer scores in e4m3
+ * after a Hadamard rotation of both operands (rotate_activation);
+ * "DeepSeek-V3.2-Exp" token-ids page, released config: scale_fmt "ue8m0").  Readings where the pages are silent:
  *  - the rotation is the Sylvester-Hadamard matrix of order d (d a power of
  *    two), H[i][j] = (-1)^popcount(i & j), orthonormal as H / sqrt(d); the
  *    FP8 path rotates both operands by H itself, so (Hq).(Hk) = d (q.k) and

@@ -1,10 +1,10 @@
 // fp8.cuh -- inputs of the FP8 lightning indexer: Hadamard rotation and e4m3
 // quantization with power-of-two scales.
 //
-// "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse Attention
-// (DSA)", item 1: the reference indexer runs in FP8 with a Hadamard
-// (rotate_activation) transform; "DeepSeek-V3.2-Exp" token-ids page, released
-// config: scale_fmt "ue8m0" (power-of-two scales).
+// "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse Attention (DSA)",
+// item 1: DeepSeek's own indexer scores in e4m3 after a Hadamard rotation of
+// queries and keys (rotate_activation); "DeepSeek-V3.2-Exp" token-ids page,
+// released config: scale_fmt "ue8m0" (power-of-two scales).
 //
 // Every vector of 128 values (one index-head query, or one index key) is
 // rotated by the Sylvester-Hadamard matrix H (entries +-1, H[i][j] =
