@@ -495,14 +495,43 @@ COMMON_SOURCES = ("common.cuh", "sm100.cuh", "dsa.cu")
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.json")
 
 
+def code_text(src):
+    """C/C++/CUDA source with its comments removed and every run of white
+    space made one blank: what the compiler turns into code.  String and
+    character literals are kept as they are (a comment marker inside one is
+    not a comment)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == "/" and src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif c == "/" and src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def sources_digest(stage):
-    """sha256 over the stage kernel's own source files and the shared ones."""
+    """sha256 over the code (comments and layout ignored, code_text) of the
+    stage kernel's own source files and the shared ones."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_attention_long_07_b200", "csrc")
     for name in STAGE_SOURCES[stage] + COMMON_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + code_text(f.read()).encode())
     return h.hexdigest()
 
 
@@ -543,7 +572,8 @@ def record_traffic(csv_path, workload):
         with open(TRAFFIC_PATH) as f:
             t = json.load(f)
     t["_note"] = ("DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch from ncu on the "
-                  "full-size workload; an entry counts only while sources_sha256 matches the kernel's sources")
+                  "full-size workload; an entry counts only while sources_sha256 matches the code (comments and "
+                  "layout ignored) of the kernel's sources")
     for stage, pat in STAGE_KERNELS.items():
         got = [(name, v) for (_, name), v in launches.items() if pat in name and len(v) == 2]
         if not got:

@@ -124,3 +124,16 @@ def test_traffic_counts_only_for_the_sources_it_was_recorded_with(tmp_path, monk
     # a different source digest (a changed kernel) withdraws the figure
     monkeypatch.setattr(bench, "sources_digest", lambda stage: "0" * 64)
     assert bench.load_traffic("indexer", "decode128k", 0) is None
+
+
+def test_traffic_digest_follows_the_code_not_its_comments():
+    """A reworded comment or a reflowed line leaves the digest of a kernel's
+    sources as it was; a changed token does not."""
+    base = 'int f(int x) { // doubles x\n  return 2 * x; /* "twice" */ }\nconst char* s = "a // b";\n'
+    reworded = '/* a new header\n   comment */\nint f(int x) {   // twice x\n  return 2 * x;  }\nconst char* s = "a // b";'
+    changed = 'int f(int x) { // doubles x\n  return 3 * x; }\nconst char* s = "a // b";\n'
+    in_string = 'int f(int x) { // doubles x\n  return 2 * x; }\nconst char* s = "a /* b";\n'
+    assert bench.code_text(base) == bench.code_text(reworded)
+    assert bench.code_text(base) != bench.code_text(changed)
+    assert bench.code_text(base) != bench.code_text(in_string)
+    assert '"a // b"' in bench.code_text(base)
