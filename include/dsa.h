@@ -30,9 +30,9 @@
  *    the diagonal -- "DeepSeek-V3.2-Exp" token-ids page, "Position IDs").
  *    Key indices in scores and idx are sequence-local (0 = first key of the
  *    sequence).  The caller appends the new tokens to the index-key cache and to
- *    the latent cache before the call ("DeepSeek-V3.2", transformers doc: the
- *    indexer keeps its own per-token key cache beside the main cache and it is
- *    updated before scoring).
+ *    the latent cache before the call ("DeepSeek-V3.2", transformers doc: besides
+ *    the main cache, the indexer stores one single-head key per token in a
+ *    cache of its own, refreshed before scoring).
  *  - A query range [q_begin, q_end) of global query rows selects the rows a
  *    call processes.  Tensors indexed by query row (q_idx, w, q, out, lse) are
  *    addressed by GLOBAL row; the scores and idx buffers of the stage calls are
@@ -246,9 +246,9 @@ typedef enum {
 /*
  * Appends a step's new tokens to the caches (the update before scoring).
  * Source: "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse
- * Attention (DSA)": the indexer keeps its own per-token key cache beside the
- * main cache and updates it every step (update_indexer), in a growing or a
- * preallocated cache layer; "DeepSeek-V3.2-Exp" token-ids page, released
+ * Attention (DSA)": besides the main cache, the indexer stores one
+ * single-head key per token in a cache of its own, refreshed each step
+ * (update_indexer), in a growing or a preallocated cache layer; "DeepSeek-V3.2-Exp" token-ids page, released
  * config: kv_lora_rank 512, qk_rope_head_dim 64, index_head_dim 128.
  * The new tokens are the step's query rows: global row t is entry pos(t) of
  * its sequence (v's kv lengths already count the new tokens), stored at that

@@ -504,10 +504,10 @@ int oracle_up_proj(int64_t n_rows, int H, int d_c, int d_v, const double* o, int
 }
 
 /* ===========================================================================
- * Cache rows of a paged layout ("DeepSeek-V3.2" transformers doc, DSA: the
- * indexer keeps its own per-token key cache beside the main cache, in a
- * growing (DynamicIndexedLayer) or a preallocated (StaticIndexedLayer) cache
- * layer).  Reading: a preallocated pool of n_pages pages of page_size rows
+ * Cache rows of a paged layout ("DeepSeek-V3.2" transformers doc, DSA:
+ * besides the main cache, the indexer stores one key per token in a cache of
+ * its own, held in a growing (DynamicIndexedLayer) or a preallocated
+ * (StaticIndexedLayer) cache layer).  Reading: a preallocated pool of n_pages pages of page_size rows
  * each, shared by the index-key cache and the latent cache; entry s of
  * sequence b sits in page block_table[b * pages_per_seq + s / page_size], at
  * row s % page_size of that page.  With no block table the caches are packed:

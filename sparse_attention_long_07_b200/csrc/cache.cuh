@@ -1,8 +1,8 @@
 // cache.cuh -- appending a step's new tokens to the index-key and latent caches.
 //
 // "DeepSeek-V3.2" (transformers model doc), "DeepSeek Sparse Attention
-// (DSA)": the indexer keeps its own per-token key cache of index_head_dim
-// beside the main cache and it is updated every step (update_indexer), in a
+// (DSA)": besides the main cache, the indexer stores one index_head_dim key
+// per token in a cache of its own, refreshed each step (update_indexer), in a
 // growing or a preallocated cache layer; MLA caches one compressed latent per
 // token, whose RoPE part carries the token's position ("DeepSeek-V3.2-Exp"
 // token-ids page, released config: kv_lora_rank 512, qk_rope_head_dim 64,
